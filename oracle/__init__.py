@@ -1,0 +1,272 @@
+"""CPU oracle for the Hadamard-rotated ("ConvRot") INT8 linear layer.
+
+TEST INFRASTRUCTURE. Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline
+leg of ``bench.py`` may import this package. The product path (the CUDA library and its
+Python binding) never imports, links or runs anything here, and this package imports
+nothing from the product.
+
+The arithmetic lives in ``oracle.c`` (plain C, fp contraction off); this module only
+builds it with gcc, loads it with ctypes and marshals numpy arrays. bf16 values travel as
+their raw 16-bit patterns in ``numpy.uint16`` arrays.
+
+Every function follows the readings stated in ``oracle.c``'s header, with the pages cited
+there ("ConvRot / Hadamard SDNQ", "SDNQ: SD.Next Quantization Engine",
+"Hybrid-Sensitivity-Weighted-Quantization").
+
+Parity status: every function here is pinned by tests in ``tests/test_oracle_pins.py``
+except the summation order of the LoRA terms, which is pinned only to within the
+fp64-sum bound (see ``lora_down`` / ``lora_up``).
+"""
+from __future__ import annotations
+
+import contextlib
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_CFLAGS = ["-std=c11", "-O2", "-ffp-contract=off", "-fno-fast-math", "-fopenmp",
+           "-shared", "-fPIC"]
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile ``oracle.c`` into ``liboracle.so`` (gcc) unless it is up to date."""
+    with _lock:
+        stale = (not os.path.exists(_LIB)
+                 or os.path.getmtime(_LIB) < os.path.getmtime(_SRC))
+        if force or stale:
+            tmp = _LIB + f".tmp{os.getpid()}"
+            subprocess.run(["gcc", *_CFLAGS, _SRC, "-o", tmp, "-lm"], check=True)
+            os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _open(path: str):
+    lib = ctypes.CDLL(path)
+    P = ctypes.c_void_p
+    I64 = ctypes.c_int64
+    INT = ctypes.c_int
+    F = ctypes.c_float
+    sig = {
+        "oracle_bf16_to_f32": [P, I64, P],
+        "oracle_f32_to_bf16": [P, I64, P],
+        "oracle_f64_to_bf16": [P, I64, P],
+        "oracle_fwht_f32": [P, I64, I64],
+        "oracle_fwht_f64": [P, I64, I64],
+        "oracle_rotate_quantize": [P, I64, I64, I64, I64, P, P, INT],
+        "oracle_gemm_s8": [P, P, I64, I64, I64, P, INT],
+        "oracle_dequant_epilogue": [P, P, P, P, P, F, I64, I64, P, INT],
+        "oracle_lora_down": [P, I64, I64, I64, P, I64, P, INT],
+        "oracle_lora_up": [P, P, I64, I64, I64, P, INT],
+        "oracle_gelu_bf16": [P, I64, P, INT],
+    }
+    for name, args in sig.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = None if name in ("oracle_bf16_to_f32", "oracle_f32_to_bf16",
+                                      "oracle_f64_to_bf16") else ctypes.c_int
+    return lib
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        _lib = _open(_LIB)
+    return _lib
+
+
+@contextlib.contextmanager
+def built_from(source_text: str, workdir: str):
+    """Test hook: run this wrapper against a build of another version of ``oracle.c``
+    (used to plant a mistake in the oracle and check that the pins catch it)."""
+    global _lib
+    src = os.path.join(workdir, "oracle_variant.c")
+    so = os.path.join(workdir, "liboracle_variant.so")
+    with open(src, "w") as f:
+        f.write(source_text)
+    subprocess.run(["gcc", *_CFLAGS, src, "-o", so, "-lm"], check=True)
+    saved = _lib
+    _lib = _open(so)
+    try:
+        yield
+    finally:
+        _lib = saved
+
+
+def source_text() -> str:
+    with open(_SRC) as f:
+        return f.read()
+
+
+def _ptr(a: np.ndarray):
+    return ctypes.c_void_p(a.ctypes.data)
+
+
+def _c(a, dtype):
+    a = np.ascontiguousarray(a)
+    if a.dtype != dtype:
+        raise TypeError(f"expected {np.dtype(dtype)}, got {a.dtype}")
+    return a
+
+
+def _check(rc, name):
+    if rc != 0:
+        raise ValueError(f"{name}: oracle returned error {rc}")
+
+
+def default_threads() -> int:
+    return os.cpu_count() or 1
+
+
+# ---- number formats ---------------------------------------------------------------
+
+def bf16_to_f32(bits: np.ndarray) -> np.ndarray:
+    bits = _c(bits, np.uint16)
+    out = np.empty(bits.shape, np.float32)
+    _load().oracle_bf16_to_f32(_ptr(bits), bits.size, _ptr(out))
+    return out
+
+
+def f32_to_bf16(x: np.ndarray) -> np.ndarray:
+    x = _c(x, np.float32)
+    out = np.empty(x.shape, np.uint16)
+    _load().oracle_f32_to_bf16(_ptr(x), x.size, _ptr(out))
+    return out
+
+
+def f64_to_bf16(x: np.ndarray) -> np.ndarray:
+    x = _c(x, np.float64)
+    out = np.empty(x.shape, np.uint16)
+    _load().oracle_f64_to_bf16(_ptr(x), x.size, _ptr(out))
+    return out
+
+
+# ---- the method ---------------------------------------------------------------------
+
+def fwht_f32(v: np.ndarray, g: int) -> np.ndarray:
+    """Unnormalised block-diagonal Walsh-Hadamard butterfly (fp32, ascending stages)
+    along the last axis, in groups of ``g``. Returns a new array."""
+    out = np.array(v, dtype=np.float32, copy=True, order="C")
+    _check(_load().oracle_fwht_f32(_ptr(out), out.size, g), "fwht_f32")
+    return out
+
+
+def fwht_f64(v: np.ndarray, g: int) -> np.ndarray:
+    """The same butterfly in fp64 (quality reports and pins only)."""
+    out = np.array(v, dtype=np.float64, copy=True, order="C")
+    _check(_load().oracle_fwht_f64(_ptr(out), out.size, g), "fwht_f64")
+    return out
+
+
+def rotate_quantize(x_bits: np.ndarray, g: int, nthreads: int | None = None):
+    """Rotate each row by the block-diagonal H_g and quantize it to int8 with one fp32
+    scale per row. ``x_bits``: bf16 patterns [rows, K]. Returns (codes int8 [rows, K],
+    scales fp32 [rows])."""
+    x_bits = _c(x_bits, np.uint16)
+    rows, K = x_bits.shape
+    q = np.empty((rows, K), np.int8)
+    s = np.empty((rows,), np.float32)
+    rc = _load().oracle_rotate_quantize(_ptr(x_bits), rows, K, K, g, _ptr(q), _ptr(s),
+                                        nthreads or default_threads())
+    _check(rc, "rotate_quantize")
+    return q, s
+
+
+def gemm_s8(a: np.ndarray, b: np.ndarray, nthreads: int | None = None) -> np.ndarray:
+    """acc[m, n] = sum_k a[m, k] * b[n, k] in int32."""
+    a = _c(a, np.int8)
+    b = _c(b, np.int8)
+    M, K = a.shape
+    N, K2 = b.shape
+    if K != K2:
+        raise ValueError("K mismatch")
+    acc = np.empty((M, N), np.int32)
+    _check(_load().oracle_gemm_s8(_ptr(a), _ptr(b), M, N, K, _ptr(acc),
+                                  nthreads or default_threads()), "gemm_s8")
+    return acc
+
+
+def dequant_epilogue(acc, sx, sw, bias_bits=None, L=None, lora_scale=1.0,
+                     nthreads: int | None = None) -> np.ndarray:
+    """fp32 de-quant epilogue; returns bf16 patterns [M, N]."""
+    acc = _c(acc, np.int32)
+    sx = _c(sx, np.float32)
+    sw = _c(sw, np.float32)
+    M, N = acc.shape
+    out = np.empty((M, N), np.uint16)
+    bias_p = None
+    L_p = None
+    if bias_bits is not None:
+        bias_bits = _c(bias_bits, np.uint16)
+        bias_p = _ptr(bias_bits)
+    if L is not None:
+        L = _c(L, np.float32)
+        L_p = _ptr(L)
+    rc = _load().oracle_dequant_epilogue(_ptr(acc), _ptr(sx), _ptr(sw), bias_p, L_p,
+                                         float(lora_scale), M, N, _ptr(out),
+                                         nthreads or default_threads())
+    _check(rc, "dequant_epilogue")
+    return out
+
+
+def lora_down(x_bits, A_bits, nthreads: int | None = None) -> np.ndarray:
+    """u = bf16(x @ A), fp64 sums. x [M, K], A [K, r] bf16 patterns -> u [M, r]."""
+    x_bits = _c(x_bits, np.uint16)
+    A_bits = _c(A_bits, np.uint16)
+    M, K = x_bits.shape
+    K2, r = A_bits.shape
+    if K != K2:
+        raise ValueError("K mismatch")
+    u = np.empty((M, r), np.uint16)
+    _check(_load().oracle_lora_down(_ptr(x_bits), M, K, K, _ptr(A_bits), r, _ptr(u),
+                                    nthreads or default_threads()), "lora_down")
+    return u
+
+
+def lora_up(u_bits, B_bits, nthreads: int | None = None) -> np.ndarray:
+    """L = fp32(u @ B), fp64 sums. u [M, r], B [r, N] bf16 patterns -> fp32 [M, N]."""
+    u_bits = _c(u_bits, np.uint16)
+    B_bits = _c(B_bits, np.uint16)
+    M, r = u_bits.shape
+    r2, N = B_bits.shape
+    if r != r2:
+        raise ValueError("rank mismatch")
+    L = np.empty((M, N), np.float32)
+    _check(_load().oracle_lora_up(_ptr(u_bits), _ptr(B_bits), M, N, r, _ptr(L),
+                                  nthreads or default_threads()), "lora_up")
+    return L
+
+
+def gelu_bf16(x_bits, nthreads: int | None = None) -> np.ndarray:
+    """Exact-erf GELU in fp64, rounded once to bf16."""
+    x_bits = _c(x_bits, np.uint16)
+    out = np.empty(x_bits.shape, np.uint16)
+    _check(_load().oracle_gelu_bf16(_ptr(x_bits), x_bits.size, _ptr(out),
+                                    nthreads or default_threads()), "gelu_bf16")
+    return out
+
+
+def linear(x_bits, qw, sw, g, bias_bits=None, A_bits=None, B_bits=None, lora_scale=1.0,
+           nthreads: int | None = None):
+    """Whole quantized linear for the rows given: rotate+quantize x, int8 GEMM against the
+    (already rotated and quantized) weight codes, fp32 epilogue, optional LoRA.
+    Returns a dict with every intermediate."""
+    qx, sx = rotate_quantize(x_bits, g, nthreads)
+    acc = gemm_s8(qx, qw, nthreads)
+    res = {"qx": qx, "sx": sx, "acc": acc}
+    L = None
+    if A_bits is not None:
+        u = lora_down(x_bits, A_bits, nthreads)
+        L = lora_up(u, B_bits, nthreads)
+        res["u"] = u
+        res["L"] = L
+    res["out"] = dequant_epilogue(acc, sx, sw, bias_bits, L, lora_scale, nthreads)
+    return res

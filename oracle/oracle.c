@@ -1,0 +1,317 @@
+/*
+ * CPU oracle for the Hadamard-rotated ("ConvRot") INT8 linear layer.
+ *
+ * TEST INFRASTRUCTURE. This file is the slow, plain reference that the CUDA
+ * library is checked against. Only the test suite, the smoke check and the
+ * benchmark's CPU-baseline leg may load it; the product path never does.
+ * It shares no code, header, table or helper with the CUDA library.
+ *
+ * Build: gcc -std=c11 -O2 -ffp-contract=off -fno-fast-math -fopenmp -shared -fPIC
+ * (contraction off: every fp32 operation below is one IEEE-754 round-to-nearest-even
+ * step, in the order written). OpenMP is used only across independent rows, so the
+ * results do not depend on the thread count.
+ *
+ * Sources (web pages on the method; cited by page title and section):
+ *  [CR]   "ConvRot / Hadamard SDNQ" (SimpleTuner docs): Quick Setup, What The Options Do,
+ *         PEFT Behavior.
+ *  [SD]   "SDNQ: SD.Next Quantization Engine" (README): feature list (Hadamard on both
+ *         quantized weights and quantized matmul; INT8 quantized matmul), SDNQConfig example
+ *         (group_size -1 = row-wise; hadamard_group_size; dequantize_fp32 = FP32 scales and
+ *         FP32 de-quant steps).
+ *  [HS]   "Hybrid-Sensitivity-Weighted-Quantization" README: Rigorous grid / pack simulation
+ *         (ConvRot = Hadamard rotate, then channelwise absmax onto the symmetric INT8 grid).
+ *
+ * Readings taken where the pages are silent (each one is listed in the design notes):
+ *  - H_g is the Sylvester Hadamard matrix in natural order, H[i][j] = (-1)^popcount(i&j),
+ *    applied block-diagonally along K in groups of g columns, normalised by 1/sqrt(g).
+ *  - The butterfly runs in fp32 with stages h = 1, 2, 4, ..., g/2 in that order; each
+ *    stage replaces (a, b) = (v[j], v[j+h]) for (j & h) == 0 by (a + b, a - b).
+ *  - Codes come from the unnormalised rotation z; the 1/sqrt(g) factor is folded into the
+ *    stored scale: s = fp32(amax / 127) * fp32(1/sqrt(g)).
+ *  - Scale granularity: one scale per row of the operand (full row for weights, per token
+ *    for activations), absmax over all K/g groups of the row.
+ *  - Rounding to integer is half-to-even on the IEEE fp32 quotient z / s_z; codes are
+ *    clamped to the symmetric range [-127, 127]. An all-zero row gives s = 0 and codes 0.
+ *  - Epilogue, fp32: t = s_x*s_w; v = float(acc)*t; v = v + bias; v = v + lora_scale*L;
+ *    out = bf16_rne(v).
+ *  - LoRA: u = bf16_rne(sum_k x*A) summed in fp64; L = fp32(sum_r u*B) summed in fp64;
+ *    x is the unrotated bf16 input (the adapter sits beside the frozen base, [CR] PEFT
+ *    Behavior).
+ *  - GELU (MLP glue between the up and down projections): exact erf form
+ *    x * Phi(x) = 0.5 * x * erfc(-x / sqrt(2)) in fp64, rounded once to bf16.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORACLE_OK 0
+#define ORACLE_ERR_ARG 1
+#define ORACLE_ERR_NOMEM 2
+
+/* ---- bf16 <-> binary32 / binary64, written out from the IEEE-754 formats ---- */
+
+static float bf16_bits_to_f32(uint16_t b)
+{
+    uint32_t u = (uint32_t)b << 16; /* bf16 is the top half of a binary32 */
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+/* binary32 -> bf16, round to nearest, ties to even. */
+static uint16_t f32_to_bf16_rne(float f)
+{
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    if ((u & 0x7fffffffu) > 0x7f800000u) /* NaN: keep it a quiet NaN */
+        return (uint16_t)((u >> 16) | 0x0040u);
+    uint32_t lsb = (u >> 16) & 1u;
+    u += 0x7fffu + lsb;
+    return (uint16_t)(u >> 16);
+}
+
+/* binary64 -> bf16 with a single rounding (nearest, ties to even). */
+static uint16_t f64_to_bf16_rne(double d)
+{
+    if (isnan(d))
+        return 0x7fc0u;
+    uint16_t sign = signbit(d) ? 0x8000u : 0u;
+    if (isinf(d))
+        return (uint16_t)(sign | 0x7f80u);
+    double a = fabs(d);
+    double r;
+    if (a < 0x1p-126) {
+        /* bf16 subnormal range: the grid step is 2^-133 */
+        r = nearbyint(a * 0x1p133) * 0x1p-133;
+    } else {
+        /* keep 1 + 7 significand bits: drop the low 45 of binary64's 52 */
+        uint64_t u;
+        memcpy(&u, &a, sizeof u);
+        uint64_t lsb = (u >> 45) & 1u;
+        u += (((uint64_t)1) << 44) - 1u + lsb;
+        u &= ~((((uint64_t)1) << 45) - 1u);
+        memcpy(&r, &u, sizeof r);
+    }
+    float f = (float)r; /* exact (8 significant bits), or +inf past the bf16 range */
+    uint32_t fu;
+    memcpy(&fu, &f, sizeof fu);
+    return (uint16_t)(sign | (uint16_t)(fu >> 16));
+}
+
+void oracle_bf16_to_f32(const uint16_t *in, int64_t n, float *out)
+{
+    for (int64_t i = 0; i < n; i++)
+        out[i] = bf16_bits_to_f32(in[i]);
+}
+
+void oracle_f32_to_bf16(const float *in, int64_t n, uint16_t *out)
+{
+    for (int64_t i = 0; i < n; i++)
+        out[i] = f32_to_bf16_rne(in[i]);
+}
+
+void oracle_f64_to_bf16(const double *in, int64_t n, uint16_t *out)
+{
+    for (int64_t i = 0; i < n; i++)
+        out[i] = f64_to_bf16_rne(in[i]);
+}
+
+static int is_pow2(int64_t g) { return g >= 1 && (g & (g - 1)) == 0; }
+
+/* ---- Walsh-Hadamard butterfly ([SD] feature list; [CR] What The Options Do) ----
+ * Unnormalised transform of one group of g values, fp32, ascending stages. */
+static void fwht_group_f32(float *v, int64_t g)
+{
+    for (int64_t h = 1; h < g; h <<= 1) {
+        for (int64_t j = 0; j < g; j++) {
+            if ((j & h) == 0) {
+                float a = v[j];
+                float b = v[j + h];
+                v[j] = a + b;
+                v[j + h] = a - b;
+            }
+        }
+    }
+}
+
+/* Block-diagonal butterfly over n values (n a multiple of g), in place. */
+int oracle_fwht_f32(float *v, int64_t n, int64_t g)
+{
+    if (!v || !is_pow2(g) || n < 0 || n % g != 0)
+        return ORACLE_ERR_ARG;
+    for (int64_t k0 = 0; k0 < n; k0 += g)
+        fwht_group_f32(v + k0, g);
+    return ORACLE_OK;
+}
+
+/* The same butterfly in binary64: used only for quality reports and pins. */
+int oracle_fwht_f64(double *v, int64_t n, int64_t g)
+{
+    if (!v || !is_pow2(g) || n < 0 || n % g != 0)
+        return ORACLE_ERR_ARG;
+    for (int64_t k0 = 0; k0 < n; k0 += g) {
+        double *w = v + k0;
+        for (int64_t h = 1; h < g; h <<= 1)
+            for (int64_t j = 0; j < g; j++)
+                if ((j & h) == 0) {
+                    double a = w[j], b = w[j + h];
+                    w[j] = a + b;
+                    w[j + h] = a - b;
+                }
+    }
+    return ORACLE_OK;
+}
+
+/* ---- Rotate + quantize one row per scale ([SD] SDNQConfig; [CR] What The Options Do;
+ * [HS] Rigorous grid / pack simulation) ----
+ * x:  bf16 bits [rows, K], row stride ldx elements.
+ * q:  int8 codes [rows, K], dense.  s: fp32 scale per row (scale of the normalised
+ * rotation, so that x_rot[r][k] ~= s[r] * q[r][k]).  Works for weights (one scale per
+ * output row, static) and activations (one scale per token, dynamic) alike. */
+int oracle_rotate_quantize(const uint16_t *x, int64_t rows, int64_t K, int64_t ldx,
+                           int64_t g, int8_t *q, float *s, int nthreads)
+{
+    if (!x || !q || !s || rows < 0 || K <= 0 || ldx < K || !is_pow2(g) || K % g != 0)
+        return ORACLE_ERR_ARG;
+    const float c_g = (float)(1.0 / sqrt((double)g));
+    int err = 0;
+#pragma omp parallel for num_threads(nthreads > 0 ? nthreads : 1) schedule(static)
+    for (int64_t r = 0; r < rows; r++) {
+        float *z = (float *)malloc((size_t)K * sizeof(float));
+        if (!z) {
+#pragma omp atomic write
+            err = 1;
+            continue;
+        }
+        const uint16_t *xr = x + r * ldx;
+        for (int64_t k = 0; k < K; k++)
+            z[k] = bf16_bits_to_f32(xr[k]);
+        for (int64_t k0 = 0; k0 < K; k0 += g)
+            fwht_group_f32(z + k0, g);
+        float amax = 0.0f;
+        for (int64_t k = 0; k < K; k++) {
+            float a = fabsf(z[k]);
+            if (a > amax)
+                amax = a;
+        }
+        const float s_z = amax / 127.0f;
+        int8_t *qr = q + r * K;
+        for (int64_t k = 0; k < K; k++) {
+            int code = 0;
+            if (amax != 0.0f) {
+                float t = z[k] / s_z;      /* IEEE fp32 quotient */
+                float n = nearbyintf(t);   /* half-to-even */
+                if (n > 127.0f)
+                    n = 127.0f;
+                if (n < -127.0f)
+                    n = -127.0f;
+                code = (n == n) ? (int)n : 0;
+            }
+            qr[k] = (int8_t)code;
+        }
+        s[r] = s_z * c_g;
+        free(z);
+    }
+    return err ? ORACLE_ERR_NOMEM : ORACLE_OK;
+}
+
+/* ---- INT8 x INT8 -> INT32 matmul ([SD] feature list: INT8 quantized matmul) ----
+ * acc[m][n] = sum_k a[m][k] * b[n][k]; both operands K-contiguous, dense. */
+int oracle_gemm_s8(const int8_t *a, const int8_t *b, int64_t M, int64_t N, int64_t K,
+                   int32_t *acc, int nthreads)
+{
+    if (!a || !b || !acc || M < 0 || N < 0 || K <= 0)
+        return ORACLE_ERR_ARG;
+#pragma omp parallel for num_threads(nthreads > 0 ? nthreads : 1) schedule(static)
+    for (int64_t m = 0; m < M; m++) {
+        const int8_t *am = a + m * K;
+        for (int64_t n = 0; n < N; n++) {
+            const int8_t *bn = b + n * K;
+            int32_t sum = 0;
+            for (int64_t k = 0; k < K; k++)
+                sum += (int32_t)am[k] * (int32_t)bn[k];
+            acc[m * N + n] = sum;
+        }
+    }
+    return ORACLE_OK;
+}
+
+/* ---- FP32 de-quant epilogue ([SD] SDNQConfig dequantize_fp32) ----
+ * out[m][n] = bf16( ((float)acc * (s_x[m]*s_w[n])) + bias[n] + lora_scale*L[m][n] ).
+ * bias (bf16 bits [N]) and L (fp32 [M,N]) may be NULL. */
+int oracle_dequant_epilogue(const int32_t *acc, const float *sx, const float *sw,
+                            const uint16_t *bias, const float *L, float lora_scale,
+                            int64_t M, int64_t N, uint16_t *out, int nthreads)
+{
+    if (!acc || !sx || !sw || !out || M < 0 || N < 0)
+        return ORACLE_ERR_ARG;
+#pragma omp parallel for num_threads(nthreads > 0 ? nthreads : 1) schedule(static)
+    for (int64_t m = 0; m < M; m++) {
+        for (int64_t n = 0; n < N; n++) {
+            float t = sx[m] * sw[n];
+            float v = (float)acc[m * N + n] * t;
+            if (bias)
+                v = v + bf16_bits_to_f32(bias[n]);
+            if (L) {
+                float l = lora_scale * L[m * N + n];
+                v = v + l;
+            }
+            out[m * N + n] = f32_to_bf16_rne(v);
+        }
+    }
+    return ORACLE_OK;
+}
+
+/* ---- LoRA side path on the frozen base ([CR] PEFT Behavior: adapters stay bf16) ----
+ * u[m][j] = bf16( sum_k x[m][k] * A[k][j] ), summed in fp64. x row stride ldx. */
+int oracle_lora_down(const uint16_t *x, int64_t M, int64_t K, int64_t ldx,
+                     const uint16_t *A, int64_t rank, uint16_t *u, int nthreads)
+{
+    if (!x || !A || !u || M < 0 || K <= 0 || ldx < K || rank <= 0)
+        return ORACLE_ERR_ARG;
+#pragma omp parallel for num_threads(nthreads > 0 ? nthreads : 1) schedule(static)
+    for (int64_t m = 0; m < M; m++) {
+        for (int64_t j = 0; j < rank; j++) {
+            double sum = 0.0;
+            for (int64_t k = 0; k < K; k++)
+                sum += (double)bf16_bits_to_f32(x[m * ldx + k]) *
+                       (double)bf16_bits_to_f32(A[k * rank + j]);
+            u[m * rank + j] = f64_to_bf16_rne(sum);
+        }
+    }
+    return ORACLE_OK;
+}
+
+/* L[m][n] = fp32( sum_j u[m][j] * B[j][n] ), summed in fp64. */
+int oracle_lora_up(const uint16_t *u, const uint16_t *B, int64_t M, int64_t N, int64_t rank,
+                   float *L, int nthreads)
+{
+    if (!u || !B || !L || M < 0 || N < 0 || rank <= 0)
+        return ORACLE_ERR_ARG;
+#pragma omp parallel for num_threads(nthreads > 0 ? nthreads : 1) schedule(static)
+    for (int64_t m = 0; m < M; m++) {
+        for (int64_t n = 0; n < N; n++) {
+            double sum = 0.0;
+            for (int64_t j = 0; j < rank; j++)
+                sum += (double)bf16_bits_to_f32(u[m * rank + j]) *
+                       (double)bf16_bits_to_f32(B[j * N + n]);
+            L[m * N + n] = (float)sum;
+        }
+    }
+    return ORACLE_OK;
+}
+
+/* ---- GELU between the MLP projections (exact erf form), bf16 -> bf16 ---- */
+int oracle_gelu_bf16(const uint16_t *in, int64_t n, uint16_t *out, int nthreads)
+{
+    if (!in || !out || n < 0)
+        return ORACLE_ERR_ARG;
+#pragma omp parallel for num_threads(nthreads > 0 ? nthreads : 1) schedule(static)
+    for (int64_t i = 0; i < n; i++) {
+        double x = (double)bf16_bits_to_f32(in[i]);
+        double y = 0.5 * x * erfc(-x / sqrt(2.0));
+        out[i] = f64_to_bf16_rne(y);
+    }
+    return ORACLE_OK;
+}

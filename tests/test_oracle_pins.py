@@ -1,0 +1,420 @@
+"""Pins for the CPU oracle: each test checks the oracle against something other than
+itself (closed forms, library routines, brute force, hand-derived worked examples), so
+that a plausible slip in the oracle (a dropped term, a wrong sign or index, a transposed
+operand, a wrong rounding rule) fails at least one test. No GPU is needed."""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from hadamard_rotated_int8_b200 import synthetic
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+GROUPS = [1, 2, 4, 8, 16, 32, 64, 128, 256]
+
+
+def sylvester(g: int) -> np.ndarray:
+    """Closed form H[i][j] = (-1)^popcount(i & j), as int64."""
+    i = np.arange(g)[:, None]
+    j = np.arange(g)[None, :]
+    pc = np.vectorize(lambda v: bin(int(v)).count("1"))(i & j)
+    return np.where(pc % 2 == 0, 1, -1).astype(np.int64)
+
+
+def bf16_bits_from_f32(x: np.ndarray) -> np.ndarray:
+    """Library routine: torch's fp32 -> bf16 cast (round to nearest even)."""
+    return synthetic.bits(torch.from_numpy(np.asarray(x, np.float32)).to(torch.bfloat16))
+
+
+def bf16_value(bits: np.ndarray) -> np.ndarray:
+    return (np.asarray(bits, np.uint32) << 16).view(np.float32)
+
+
+# ---------------------------------------------------------------- number formats
+
+def test_f32_to_bf16_matches_torch_cast():
+    rng = np.random.default_rng(0)
+    x = rng.standard_normal(200_000).astype(np.float32) * np.float32(1e3)
+    # exact ties: low 16 bits 0x8000 with even and odd upper halves
+    ties = (rng.integers(0, 2**31, 4096, dtype=np.uint32) & 0xffff0000) | 0x8000
+    ties = ties.view(np.float32)
+    ties = ties[np.isfinite(ties)]
+    special = np.array([0.0, -0.0, 1.0, -1.0, 3.0e38, -3.0e38, 3.3895e38, 1e-40, -1e-40,
+                        np.inf, -np.inf], np.float32)
+    for arr in (x, ties, special):
+        assert np.array_equal(oracle.f32_to_bf16(arr), bf16_bits_from_f32(arr))
+
+
+def _nearest_bf16_brute(d: float) -> int:
+    """Brute force: try the candidate bf16 patterns around d and keep the nearest, ties to
+    the even pattern."""
+    f = np.float32(d)
+    base = int(np.array([f], np.float32).view(np.uint32)[0] >> 16)
+    cands = []
+    for b in range(base - 2, base + 3):
+        b &= 0xffff
+        v = float(bf16_value(np.array([b]))[0])
+        if math.isnan(v):
+            continue
+        cands.append((abs(v - d), b & 1, b, v))
+    # the infinity is the right answer only past the overflow threshold
+    cands.sort()
+    return cands[0][2]
+
+
+def test_f64_to_bf16_is_single_correct_rounding():
+    rng = np.random.default_rng(1)
+    vals = list(rng.standard_normal(3000) * 10.0 ** rng.integers(-40, 38, 3000))
+    # double-rounding traps: just above a bf16 midpoint, within fp32 rounding distance
+    for _ in range(500):
+        b = int(rng.integers(0x0100, 0x7f00))
+        lo = float(bf16_value(np.array([b]))[0])
+        hi = float(bf16_value(np.array([b + 1]))[0])
+        mid = (lo + hi) / 2
+        vals += [mid, mid + (hi - lo) * 2.0 ** -20, mid - (hi - lo) * 2.0 ** -20]
+    # bf16 subnormals (grid 2^-133)
+    vals += list(rng.uniform(-2.0 ** -126, 2.0 ** -126, 500))
+    vals += [0.0, -0.0, 2.0 ** -133, 2.0 ** -134, 3 * 2.0 ** -135]
+    d = np.array(vals, np.float64)
+    got = oracle.f64_to_bf16(d)
+    for di, gi in zip(d, got):
+        if di == 0.0:
+            assert gi == (0x8000 if math.copysign(1, di) < 0 else 0)
+            continue
+        assert gi == _nearest_bf16_brute(float(di)), (di, hex(gi))
+
+
+def test_f64_to_bf16_overflow_and_sign():
+    big = np.array([3.4e38, -3.4e38, 1e300, -1e300, np.inf, -np.inf], np.float64)
+    got = oracle.f64_to_bf16(big)
+    assert list(got) == [0x7f80, 0xff80, 0x7f80, 0xff80, 0x7f80, 0xff80]
+
+
+# ---------------------------------------------------------------- Walsh-Hadamard butterfly
+
+@pytest.mark.parametrize("g", GROUPS)
+def test_butterfly_matrix_is_sylvester_and_orthogonal(g):
+    """Applying the oracle butterfly to the unit vectors reproduces the closed form
+    H[i][j] = (-1)^popcount(i&j), and H H^T = g I."""
+    eye = np.eye(g, dtype=np.float32)
+    cols = oracle.fwht_f32(eye, g)  # row i = FWHT(e_i) = column i of H
+    H = cols.T.astype(np.int64)
+    assert np.array_equal(H, sylvester(g))
+    assert np.array_equal(H @ H.T, g * np.eye(g, dtype=np.int64))
+
+
+@pytest.mark.parametrize("g", GROUPS)
+def test_butterfly_equals_dense_product_on_integers(g):
+    """For integer inputs with |v| < 2^24/g every fp32 step is exact, so the butterfly must
+    equal the dense integer product bit for bit (numpy int64 matmul)."""
+    rng = np.random.default_rng(g)
+    bound = (1 << 24) // g - 1
+    rows, K = 7, 4 * g
+    v = rng.integers(-bound, bound + 1, size=(rows, K))
+    got = oracle.fwht_f32(v.astype(np.float32), g)
+    H = sylvester(g)
+    want = (v.reshape(rows, K // g, g) @ H.T).reshape(rows, K)
+    assert np.array_equal(got.astype(np.int64), want)
+
+
+@pytest.mark.parametrize("g", [8, 64, 256])
+def test_butterfly_is_an_involution_up_to_g(g):
+    rng = np.random.default_rng(100 + g)
+    v = rng.integers(-1000, 1001, size=(3, 2 * g)).astype(np.float32)
+    twice = oracle.fwht_f32(oracle.fwht_f32(v, g), g)
+    assert np.array_equal(twice, g * v)
+
+
+@pytest.mark.parametrize("g", [64, 128, 256])
+def test_butterfly_fp32_error_within_textbook_bound(g):
+    """Real-valued input: fp32 butterfly vs the exact (fp64 dense) product, within the
+    standard bound log2(g) * u * sum|v| per output (u = 2^-24) + a small slack."""
+    rng = np.random.default_rng(7 + g)
+    v = rng.standard_normal((16, g)).astype(np.float32)
+    got = oracle.fwht_f32(v, g).astype(np.float64)
+    exact = v.astype(np.float64) @ sylvester(g).T.astype(np.float64)
+    bound = (math.log2(g) * 2.0 ** -24 * 1.01) * np.abs(v).astype(np.float64).sum(1,
+                                                                                 keepdims=True)
+    assert np.all(np.abs(got - exact) <= bound)
+
+
+@pytest.mark.parametrize("g", [64, 128, 256])
+def test_rotation_cancels_in_the_product(g):
+    """(x H)(W H)^T = g * x W^T: in exact integer arithmetic through the oracle's own
+    fp32 butterfly, and in fp64 to ~1e-12 through its fp64 butterfly (normalised)."""
+    rng = np.random.default_rng(11 + g)
+    K = 2 * g
+    x = rng.integers(-50, 51, size=(5, K))
+    W = rng.integers(-50, 51, size=(6, K))
+    zx = oracle.fwht_f32(x.astype(np.float32), g).astype(np.int64)
+    zw = oracle.fwht_f32(W.astype(np.float32), g).astype(np.int64)
+    assert np.array_equal(zx @ zw.T, g * (x @ W.T))
+    xf = rng.standard_normal((5, K))
+    Wf = rng.standard_normal((6, K))
+    rx = oracle.fwht_f64(xf, g) / math.sqrt(g)
+    rw = oracle.fwht_f64(Wf, g) / math.sqrt(g)
+    ref = xf @ Wf.T
+    assert np.max(np.abs(rx @ rw.T - ref)) <= 1e-12 * np.max(np.abs(ref)) * K
+
+
+# ---------------------------------------------------------------- rotate + quantize
+
+def _ties_even_nearest(t: np.float32) -> int:
+    """Brute force over the whole grid [-127, 127]: nearest point, ties to the even one."""
+    best = None
+    for q in range(-127, 128):
+        d = abs(float(t) - q)
+        key = (d, q & 1)
+        if best is None or key < best[0]:
+            best = (key, q)
+    return best[1]
+
+
+@pytest.mark.parametrize("K", [8, 16, 32])
+def test_codes_brute_force_g8(K):
+    """g = 8, K <= 32, integer inputs (so the rotation z is exact): every code is the
+    nearest grid point to the IEEE fp32 quotient z / fp32(amax/127), ties to even, and the
+    scale is fp32(amax/127) * fp32(1/sqrt(8))."""
+    rng = np.random.default_rng(K)
+    rows = 40
+    x = rng.integers(-200, 201, size=(rows, K)).astype(np.float32)
+    x[3] = 0.0                       # zero row
+    x[4, :] = 0.0
+    x[4, 0] = 5.0                    # single spike -> flat rotation
+    xb = bf16_bits_from_f32(x)
+    assert np.array_equal(bf16_value(xb), x)  # integers < 256 are exact in bf16
+    q, s = oracle.rotate_quantize(xb, 8)
+    H = sylvester(8)
+    z = (x.astype(np.int64).reshape(rows, K // 8, 8) @ H.T).reshape(rows, K)
+    c8 = np.float32(1.0 / math.sqrt(8.0))
+    for r in range(rows):
+        amax = np.float32(np.abs(z[r]).max())
+        sz = np.float32(amax / np.float32(127.0))
+        if amax == 0:
+            assert np.all(q[r] == 0) and s[r] == 0
+            continue
+        assert s[r] == np.float32(sz * c8)
+        for k in range(K):
+            t = np.float32(np.float32(z[r, k]) / sz)
+            assert q[r, k] == _ties_even_nearest(t), (r, k, t)
+
+
+def test_g1_is_textbook_per_row_absmax_int8():
+    """g = 1 (no rotation) must be plain per-row absmax INT8: s = amax/127,
+    q = round_half_even(x / s)."""
+    rng = np.random.default_rng(5)
+    x = (rng.standard_normal((64, 96)) * 3).astype(np.float32)
+    xb = bf16_bits_from_f32(x)
+    xv = bf16_value(xb)
+    q, s = oracle.rotate_quantize(xb, 1)
+    amax = np.abs(xv).max(1)
+    s_ref = (amax / np.float32(127)).astype(np.float32)
+    q_ref = np.clip(np.round(xv / s_ref[:, None]), -127, 127).astype(np.int8)
+    assert np.array_equal(s, s_ref)
+    assert np.array_equal(q, q_ref)
+
+
+@pytest.mark.parametrize("g", [8, 16, 32, 64, 128, 256])
+def test_quantization_invariants(g):
+    case = synthetic.make_case(M=33, N=8, K=1024, g=g, seed=g, outlier_count=10,
+                               outlier_factor=25.0)
+    xb = synthetic.bits(case.x)
+    q, s = oracle.rotate_quantize(xb, g)
+    z = oracle.fwht_f32(bf16_value(xb), g)
+    c = np.float32(1.0 / math.sqrt(g))
+    assert q.min() >= -127 and q.max() <= 127
+    for r in range(q.shape[0]):
+        amax = np.abs(z[r]).max()
+        sz = np.float32(amax / np.float32(127))
+        # the element(s) attaining the row absmax land on the top of the grid
+        top = np.abs(z[r]) == amax
+        assert np.all(np.abs(q[r][top]) == 127)
+        # half-step bound (plus the fp32 rounding of the quotient)
+        err = np.abs(z[r].astype(np.float64) - q[r].astype(np.float64) * float(sz))
+        assert np.all(err <= float(sz) * (0.5 + 2.0 ** -16))
+        assert s[r] == np.float32(sz * c)
+
+
+@pytest.mark.parametrize("g", [64, 256])
+def test_power_of_four_groups_equal_quantizing_the_normalised_rotation(g):
+    """For g = 4^k the normaliser 1/sqrt(g) is a power of two, so folding it into the scale
+    is the same as quantizing the normalised rotation z/sqrt(g) directly (the HSWQ page
+    sizes its ConvRot groups in powers of 4)."""
+    case = synthetic.make_case(M=20, N=8, K=2 * g, g=g, seed=3, outlier_count=3,
+                               outlier_factor=30.0)
+    xb = synthetic.bits(case.x)
+    q, s = oracle.rotate_quantize(xb, g)
+    zn32 = oracle.fwht_f32(bf16_value(xb), g) * np.float32(1 / math.sqrt(g))
+    s_direct = (np.abs(zn32).max(1) / np.float32(127)).astype(np.float32)
+    q_direct = np.clip(np.round(zn32 / s_direct[:, None]), -127, 127).astype(np.int8)
+    assert np.array_equal(s, s_direct)
+    assert np.array_equal(q, q_direct)
+
+
+def test_golden_worked_rotquant():
+    d = json.load(open(os.path.join(GOLDEN, "rotquant_g8_worked.json")))
+    g = d["g"]
+    for case in d["cases"]:
+        x = np.array([case["x"]], np.float32)
+        z = oracle.fwht_f32(x, g)
+        assert np.array_equal(z[0], np.array(case["z"], np.float32))
+        q, s = oracle.rotate_quantize(bf16_bits_from_f32(x), g)
+        assert list(q[0]) == case["codes"]
+        want_s = np.float32(np.float32(case["amax"]) / np.float32(127)) * np.float32(
+            1 / math.sqrt(g))
+        assert s[0] == np.float32(want_s)
+
+
+def test_rows_are_independent_and_strided_input():
+    case = synthetic.make_case(M=50, N=8, K=512, g=256, seed=9)
+    xb = synthetic.bits(case.x)
+    q_all, s_all = oracle.rotate_quantize(xb, 256)
+    for r in (0, 17, 49):
+        q1, s1 = oracle.rotate_quantize(xb[r:r + 1], 256, nthreads=1)
+        assert np.array_equal(q1[0], q_all[r]) and s1[0] == s_all[r]
+
+
+def test_reconstruction_quality_and_rotation_helps_outliers():
+    """Quality report (not parity): dequantised rotated product vs fp64 x W^T. With outlier
+    channels the Hadamard rotation lowers the max-token error against no rotation."""
+    case = synthetic.make_case(M=64, N=96, K=1024, g=256, seed=21, outlier_frac=0.01,
+                               outlier_factor=30.0)
+    xb, wb = synthetic.bits(case.x), synthetic.bits(case.W)
+    ref = bf16_value(xb).astype(np.float64) @ bf16_value(wb).astype(np.float64).T
+    errs = {}
+    for g in (1, 256):
+        qx, sx = oracle.rotate_quantize(xb, g)
+        qw, sw = oracle.rotate_quantize(wb, g)
+        acc = oracle.gemm_s8(qx, qw).astype(np.float64)
+        y = acc * sx[:, None].astype(np.float64) * sw[None, :].astype(np.float64)
+        tok_err = np.abs(y - ref).max(1) / np.abs(ref).max(1)
+        errs[g] = tok_err.max()
+    assert errs[256] < 0.05
+    assert errs[256] < errs[1]
+
+
+# ---------------------------------------------------------------- GEMM and epilogue
+
+@pytest.mark.parametrize("shape", [(1, 1, 16), (17, 33, 48), (64, 40, 1024)])
+def test_gemm_matches_numpy_int64(shape):
+    M, N, K = shape
+    rng = np.random.default_rng(M * N)
+    a = rng.integers(-127, 128, size=(M, K), dtype=np.int8)
+    b = rng.integers(-127, 128, size=(N, K), dtype=np.int8)
+    acc = oracle.gemm_s8(a, b)
+    assert np.array_equal(acc.astype(np.int64), a.astype(np.int64) @ b.astype(np.int64).T)
+
+
+def test_gemm_extreme_accumulator():
+    K = 131072
+    a = np.full((1, K), -127, np.int8)
+    b = np.full((2, K), -127, np.int8)
+    b[1] = 127
+    acc = oracle.gemm_s8(a, b)
+    assert acc[0, 0] == 127 * 127 * K and acc[0, 1] == -127 * 127 * K
+
+
+def test_golden_worked_epilogue():
+    d = json.load(open(os.path.join(GOLDEN, "linear_int8_worked.json")))
+    qx = np.array(d["qx"], np.int8)
+    qw = np.array(d["qw"], np.int8)
+    acc = oracle.gemm_s8(qx, qw)
+    assert acc.tolist() == d["acc"]
+    out = oracle.dequant_epilogue(acc, np.array(d["sx"], np.float32),
+                                  np.array(d["sw"], np.float32),
+                                  bf16_bits_from_f32(np.array(d["bias"], np.float32)))
+    assert bf16_value(out).tolist() == d["out"]
+
+
+def test_epilogue_within_one_ulp_of_fp64_and_op_order():
+    """Against an fp64 recompute from the same codes and scales: every output within one
+    bf16 ulp; the fp32 op order (s_x*s_w first, no fused multiply-add) is checked by a
+    float32 numpy recompute that must match bit for bit."""
+    rng = np.random.default_rng(3)
+    # large enough that an fp32 op-order change shows up after the bf16 rounding
+    M, N, K = 1024, 2048, 512
+    acc = rng.integers(-2_000_000, 2_000_001, size=(M, N)).astype(np.int32)
+    sx = (rng.random(M) * 0.05).astype(np.float32)
+    sw = (rng.random(N) * 1e-4).astype(np.float32)
+    bias = bf16_bits_from_f32(rng.standard_normal(N).astype(np.float32) * 0.01)
+    L = (rng.standard_normal((M, N)) * 0.1).astype(np.float32)
+    for use_bias, use_L in ((False, False), (True, False), (True, True)):
+        out = oracle.dequant_epilogue(acc, sx, sw, bias if use_bias else None,
+                                      L if use_L else None, 0.75)
+        exact = acc.astype(np.float64) * sx[:, None].astype(np.float64) * sw[None, :]
+        if use_bias:
+            exact = exact + bf16_value(bias)[None, :].astype(np.float64)
+        if use_L:
+            exact = exact + 0.75 * L.astype(np.float64)
+        got = bf16_value(out).astype(np.float64)
+        # one bf16 ulp of the result, plus the fp32 rounding of the terms (which only
+        # matters where bias and product nearly cancel)
+        terms = np.abs(acc.astype(np.float64) * sx[:, None] * sw[None, :])
+        if use_bias:
+            terms = terms + np.abs(bf16_value(bias))[None, :]
+        if use_L:
+            terms = terms + 0.75 * np.abs(L)
+        bound = np.abs(exact) * 2.0 ** -7 + terms * 2.0 ** -21
+        assert np.all(np.abs(got - exact) <= bound)
+        v = acc.astype(np.float32) * (sx[:, None] * sw[None, :])
+        if use_bias:
+            v = v + bf16_value(bias)[None, :]
+        if use_L:
+            v = v + np.float32(0.75) * L
+        assert np.array_equal(out, bf16_bits_from_f32(v))
+
+
+def test_zero_row_gives_bias_only():
+    M, N, K = 3, 16, 256
+    x = np.zeros((M, K), np.float32)
+    x[1] = np.linspace(-1, 1, K, dtype=np.float32)
+    rng = np.random.default_rng(0)
+    W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    bias = bf16_bits_from_f32(rng.standard_normal(N).astype(np.float32) * 0.01)
+    qw, sw = oracle.rotate_quantize(bf16_bits_from_f32(W), 256)
+    res = oracle.linear(bf16_bits_from_f32(x), qw, sw, 256, bias_bits=bias)
+    assert res["sx"][0] == 0 and res["sx"][2] == 0
+    assert np.array_equal(res["out"][0], bias) and np.array_equal(res["out"][2], bias)
+
+
+# ---------------------------------------------------------------- LoRA and GELU
+
+def test_lora_down_and_up_against_fp64_products():
+    case = synthetic.make_case(M=37, N=70, K=320, g=64, seed=4, lora_rank=16,
+                               outlier_count=3, outlier_factor=30.0)
+    xb, Ab, Bb = (synthetic.bits(t) for t in (case.x, case.A, case.B))
+    u = oracle.lora_down(xb, Ab)
+    exact_u = bf16_value(xb).astype(np.float64) @ bf16_value(Ab).astype(np.float64)
+    got_u = bf16_value(u).astype(np.float64)
+    assert np.all(np.abs(got_u - exact_u) <= np.abs(exact_u) * 2.0 ** -8 + 1e-30)
+    # u is the single rounding of the fp64 sum: equal to torch's rounding of it except at
+    # double-rounding traps, which are rare
+    via_torch = bf16_bits_from_f32(exact_u.astype(np.float32))
+    assert (u == via_torch).mean() > 0.999
+    L = oracle.lora_up(u, Bb)
+    exact_L = got_u @ bf16_value(Bb).astype(np.float64)
+    assert np.all(np.abs(L.astype(np.float64) - exact_L) <=
+                  np.abs(exact_L) * 2.0 ** -23 + 1e-30)
+
+
+def test_gelu_against_scipy_normal_cdf_and_special_values():
+    """GELU(x) = x * Phi(x), with Phi from scipy's normal CDF (accurate in relative terms
+    in the lower tail, where 1 + erf cancels)."""
+    from scipy.special import ndtr
+    rng = np.random.default_rng(8)
+    x = np.concatenate([rng.standard_normal(20000) * 3, np.linspace(-12, 12, 2001),
+                        [0.0, -0.0, 1e-30, -1e-30, 50.0, -50.0, 3e38, -3e38]])
+    xb = bf16_bits_from_f32(x.astype(np.float32))
+    xv = bf16_value(xb).astype(np.float64)
+    got = bf16_value(oracle.gelu_bf16(xb)).astype(np.float64)
+    ref = xv * ndtr(xv)
+    ok = np.abs(got - ref) <= np.abs(ref) * 2.0 ** -8 + 1e-37
+    assert ok.all()
+    g = oracle.gelu_bf16(bf16_bits_from_f32(np.array([0.0, 50.0, -50.0, 2.0], np.float32)))
+    assert g[0] == 0 and bf16_value(g[1:2])[0] == 50.0
+    assert g[2] == 0x8000  # -50 * Phi(-50) underflows to -0
+    assert bf16_value(g[3:4])[0] == np.float32(1.953125)  # 2*Phi(2)=1.9545 -> bf16 1.953125
