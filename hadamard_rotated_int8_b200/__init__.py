@@ -1,5 +1,32 @@
 """Hadamard-rotated ("ConvRot") INT8 linear layer for NVIDIA B200 (sm_100a).
 
-The compute lives in ``libsdnq.so`` (hand-written CUDA behind a C ABI, see
-``include/sdnq.h``); this package is the thin Python binding over it.
+The compute lives in ``libsdnq.so`` (hand-written CUDA behind the C ABI of
+``include/sdnq.h``); this package is the thin Python binding over it, with the same names:
+
+* ``sdnq_rotate_quant_weight``  weight rotate + row-wise int8 quantize (offline)
+* ``sdnq_rotquant_act``         online activation rotate + per-token int8 quantize
+* ``sdnq_int8_linear``          int8 x int8 -> int32 tensor-core matmul + fp32 de-quant epilogue
+* ``sdnq_int8_linear_lora``     the same plus the bf16 LoRA side term
+* ``sdnq_gelu_bf16``            exact-erf GELU (MLP glue)
+
+``linear`` composes the online path (rotate + quantize, then the int8 linear).
 """
+from ._native import (SdnqError, lib, sdnq_device_status, sdnq_gelu_bf16, sdnq_int8_linear,
+                      sdnq_int8_linear_lora, sdnq_rotate_quant_weight, sdnq_rotquant_act,
+                      sdnq_selftest_wait_timeout, status_string, version)
+
+__all__ = [
+    "SdnqError", "lib", "linear", "sdnq_device_status", "sdnq_gelu_bf16", "sdnq_int8_linear",
+    "sdnq_int8_linear_lora", "sdnq_rotate_quant_weight", "sdnq_rotquant_act",
+    "sdnq_selftest_wait_timeout", "status_string", "version",
+]
+
+
+def linear(x, qW, sW, group=256, bias=None, lora=None, out=None, stream=None):
+    """y = rotated-int8 linear of x [M, K] bf16 against pre-quantized weights (qW, sW).
+    ``lora`` = (A, B, lora_scale) adds the bf16 adapter term."""
+    qx, sx = sdnq_rotquant_act(x, group, stream=stream)
+    if lora is None:
+        return sdnq_int8_linear(qx, sx, qW, sW, bias, out=out, stream=stream)
+    A, B, scale = lora
+    return sdnq_int8_linear_lora(qx, sx, qW, sW, bias, x, A, B, scale, out=out, stream=stream)

@@ -1,0 +1,210 @@
+"""ctypes binding of ``libsdnq.so`` (C ABI in ``include/sdnq.h``).
+
+Argument marshalling only: every step of the layer runs in the library's CUDA kernels.
+Tensors are torch CUDA tensors; bf16 tensors are passed by pointer and read as raw 16-bit
+patterns. Calls are asynchronous on torch's current CUDA stream. There is no fallback: if
+the library is missing or the device is not a B200 (sm_100), calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+from . import _build
+
+_lib = None
+_lock = threading.Lock()
+
+SDNQ_OK = 0
+SDNQ_ERR_NULL = 1
+SDNQ_ERR_SHAPE = 2
+SDNQ_ERR_ALIGN = 3
+SDNQ_ERR_UNSUPPORTED = 4
+SDNQ_ERR_CUDA = 5
+SDNQ_ERR_TIMEOUT = 6
+
+MAX_K = 131072
+MIN_GROUP = 8
+MAX_GROUP = 256
+MAX_RANK = 256
+
+_P = ctypes.c_void_p
+_I64 = ctypes.c_int64
+_I32 = ctypes.c_int32
+_F = ctypes.c_float
+
+SIGNATURES = {
+    "sdnq_rotate_quant_weight": [_P, _I64, _I64, _I64, _I32, _P, _P, _P],
+    "sdnq_rotquant_act": [_P, _I64, _I64, _I64, _I32, _P, _P, _P],
+    "sdnq_int8_linear": [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _I64, _P, _P],
+    "sdnq_int8_linear_lora": [_P, _P, _P, _P, _P, _P, _I64, _P, _P, _I32, _F, _P, _I64, _I64,
+                              _I64, _P, _I64, _P, _P],
+    "sdnq_gelu_bf16": [_P, _I64, _I64, _I64, _P, _I64, _P],
+    "sdnq_device_status": [_P],
+    "sdnq_selftest_wait_timeout": [_I64, _P],
+    "sdnq_status_string": [ctypes.c_int],
+    "sdnq_version": [],
+}
+
+
+class SdnqError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)}")
+
+
+def lib_path() -> str:
+    return _build.LIB
+
+
+def lib():
+    """The loaded ``libsdnq.so`` (ctypes.CDLL with argument types set). Raises if the
+    library has not been built (``python -m hadamard_rotated_int8_b200._build``)."""
+    global _lib
+    if _lib is None:
+        with _lock:
+            if _lib is None:
+                path = lib_path()
+                if not os.path.exists(path):
+                    raise RuntimeError(
+                        f"libsdnq.so not found at {path}: build it with "
+                        "`python -m hadamard_rotated_int8_b200._build` (needs nvcc); "
+                        "there is no non-CUDA fallback")
+                cdll = ctypes.CDLL(path)
+                for name, args in SIGNATURES.items():
+                    fn = getattr(cdll, name)
+                    fn.argtypes = args
+                    fn.restype = ctypes.c_char_p if name in ("sdnq_status_string",
+                                                             "sdnq_version") else ctypes.c_int
+                _lib = cdll
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().sdnq_status_string(int(status)).decode()
+
+
+def version() -> str:
+    return lib().sdnq_version().decode()
+
+
+def _check(status: int, where: str):
+    if status != SDNQ_OK:
+        raise SdnqError(status, where)
+
+
+def _stream(stream):
+    if stream is None:
+        return _P(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, torch.cuda.Stream):
+        return _P(stream.cuda_stream)
+    return _P(int(stream))
+
+
+def _ptr(t: torch.Tensor | None):
+    return _P(t.data_ptr()) if t is not None else _P(0)
+
+
+def _req(t: torch.Tensor, dtype, name: str, ndim: int):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name}: expected a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name}: must be a CUDA tensor (no CPU path)")
+    if t.dim() != ndim:
+        raise ValueError(f"{name}: expected {ndim} dims, got {t.dim()}")
+    if t.stride(-1) != 1:
+        raise ValueError(f"{name}: last dimension must be contiguous")
+
+
+def _dense(t: torch.Tensor, name: str):
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+
+
+# ---------------------------------------------------------------- the C ABI, by name
+
+def sdnq_rotate_quant_weight(W: torch.Tensor, group: int = 256, qW=None, sW=None, stream=None):
+    """W [N, K] bf16 -> (qW [N, K] int8, sW [N] fp32)."""
+    _req(W, torch.bfloat16, "W", 2)
+    N, K = W.shape
+    qW = torch.empty((N, K), dtype=torch.int8, device=W.device) if qW is None else qW
+    sW = torch.empty((N,), dtype=torch.float32, device=W.device) if sW is None else sW
+    _check(lib().sdnq_rotate_quant_weight(_ptr(W), N, K, W.stride(0), group, _ptr(qW), _ptr(sW),
+                                          _stream(stream)), "sdnq_rotate_quant_weight")
+    return qW, sW
+
+
+def sdnq_rotquant_act(x: torch.Tensor, group: int = 256, qx=None, sx=None, stream=None):
+    """x [M, K] bf16 -> (qx [M, K] int8, sx [M] fp32)."""
+    _req(x, torch.bfloat16, "x", 2)
+    M, K = x.shape
+    qx = torch.empty((M, K), dtype=torch.int8, device=x.device) if qx is None else qx
+    sx = torch.empty((M,), dtype=torch.float32, device=x.device) if sx is None else sx
+    _check(lib().sdnq_rotquant_act(_ptr(x), M, K, x.stride(0), group, _ptr(qx), _ptr(sx),
+                                   _stream(stream)), "sdnq_rotquant_act")
+    return qx, sx
+
+
+def sdnq_int8_linear(qx, sx, qW, sW, bias=None, out=None, acc_out=None, stream=None):
+    """out [M, N] bf16 = bf16(float(qx qW^T) * (sx sW^T) + bias)."""
+    _req(qx, torch.int8, "qx", 2)
+    _req(qW, torch.int8, "qW", 2)
+    _dense(qx, "qx")
+    _dense(qW, "qW")
+    M, K = qx.shape
+    N = qW.shape[0]
+    if qW.shape[1] != K:
+        raise ValueError("qx and qW disagree on K")
+    out = torch.empty((M, N), dtype=torch.bfloat16, device=qx.device) if out is None else out
+    _check(lib().sdnq_int8_linear(_ptr(qx), _ptr(sx), _ptr(qW), _ptr(sW), _ptr(bias), M, N, K,
+                                  _ptr(out), out.stride(0), _ptr(acc_out), _stream(stream)),
+           "sdnq_int8_linear")
+    return out
+
+
+def sdnq_int8_linear_lora(qx, sx, qW, sW, bias, x, A, B, lora_scale: float = 1.0, u_ws=None,
+                          out=None, acc_out=None, stream=None):
+    """As sdnq_int8_linear plus lora_scale * bf16(x A) B; u_ws [M, rank] receives bf16(x A)."""
+    _req(qx, torch.int8, "qx", 2)
+    _req(qW, torch.int8, "qW", 2)
+    _req(x, torch.bfloat16, "x", 2)
+    _dense(A, "A")
+    _dense(B, "B")
+    M, K = qx.shape
+    N = qW.shape[0]
+    rank = A.shape[1]
+    if A.shape[0] != K or B.shape != (rank, N) or x.shape != (M, K):
+        raise ValueError("LoRA shapes disagree")
+    u_ws = torch.empty((M, rank), dtype=torch.bfloat16, device=qx.device) if u_ws is None else u_ws
+    out = torch.empty((M, N), dtype=torch.bfloat16, device=qx.device) if out is None else out
+    _check(lib().sdnq_int8_linear_lora(_ptr(qx), _ptr(sx), _ptr(qW), _ptr(sW), _ptr(bias),
+                                       _ptr(x), x.stride(0), _ptr(A), _ptr(B), rank,
+                                       float(lora_scale), _ptr(u_ws), M, N, K, _ptr(out),
+                                       out.stride(0), _ptr(acc_out), _stream(stream)),
+           "sdnq_int8_linear_lora")
+    return out
+
+
+def sdnq_gelu_bf16(x: torch.Tensor, out=None, stream=None):
+    """Exact-erf GELU, bf16 -> bf16 (the MLP glue between up and down projections)."""
+    _req(x, torch.bfloat16, "x", 2)
+    M, N = x.shape
+    out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device) if out is None else out
+    _check(lib().sdnq_gelu_bf16(_ptr(x), M, N, x.stride(0), _ptr(out), out.stride(0),
+                                _stream(stream)), "sdnq_gelu_bf16")
+    return out
+
+
+def sdnq_device_status(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device error word status."""
+    return lib().sdnq_device_status(_stream(stream))
+
+
+def sdnq_selftest_wait_timeout(limit_ns: int, stream=None):
+    _check(lib().sdnq_selftest_wait_timeout(int(limit_ns), _stream(stream)),
+           "sdnq_selftest_wait_timeout")

@@ -1,0 +1,96 @@
+// GELU between the up and down projections of a DiT MLP, bf16 -> bf16, exact-erf form
+// GELU(x) = x * Phi(x) = 0.5 * x * erfc(-x / sqrt(2)), rounded once to bf16.
+//
+// Fast path in fp32 with CUDA's erfcf. Its relative error against the exact value is at
+// most about (x^2 + 6.5) * 2^-23 (argument rounding of x/sqrt(2), amplified by the
+// logarithmic slope of erfc, which is at most 2a^2 + 2 for a = -x/sqrt(2); erfcf's own
+// 4 ulp; one final product). The kernel widens that to a margin of (x^2 + 16) * 2^-22 and
+// keeps the fp32 result only when the whole interval value +- margin rounds to one bf16
+// value: then that value is the correctly rounded bf16 of the exact GELU. Otherwise (a value
+// near a bf16 rounding boundary, or |x| > 10 where fp32 underflows) it recomputes in fp64
+// and rounds the fp64 value to bf16 directly, with a single rounding.
+#pragma once
+
+#include <cuda_bf16.h>
+
+#include "device.cuh"
+
+namespace sdnq {
+
+// binary64 -> bf16, round to nearest even, one rounding (bf16 keeps 1 + 7 significand bits).
+__device__ __forceinline__ uint32_t f64_to_bf16_bits(double d)
+{
+    if (isnan(d))
+        return 0x7fc0u;
+    const uint32_t sign = signbit(d) ? 0x8000u : 0u;
+    const double a = fabs(d);
+    if (isinf(a))
+        return sign | 0x7f80u;
+    double r;
+    if (a < 0x1p-126) {
+        r = rint(a * 0x1p133) * 0x1p-133;  // bf16 subnormal grid 2^-133
+    } else {
+        unsigned long long u = static_cast<unsigned long long>(__double_as_longlong(a));
+        u += (1ull << 44) - 1ull + ((u >> 45) & 1ull);
+        u &= ~((1ull << 45) - 1ull);
+        r = __longlong_as_double(static_cast<long long>(u));
+    }
+    const float f = __double2float_rn(r);  // exact, or +inf past the range
+    return sign | (__float_as_uint(f) >> 16);
+}
+
+__device__ __forceinline__ uint32_t f32_to_bf16_bits_rn(float f)
+{
+    return static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(f)));
+}
+
+__device__ __forceinline__ uint32_t gelu_bf16_bits(uint32_t xb)
+{
+    const float x = __uint_as_float(xb << 16);
+    if (fabsf(x) <= 10.0f) {
+        const float a = __fmul_rn(x, -0.70710678118654752440f);
+        const float e = erfcf(a);
+        const float v = __fmul_rn(__fmul_rn(0.5f, x), e);
+        const float margin = __fmul_rn(fabsf(v), __fmul_rn(__fadd_rn(__fmul_rn(x, x), 16.0f), 0x1p-22f));
+        const uint32_t lo = f32_to_bf16_bits_rn(__fsub_rn(v, margin));
+        const uint32_t hi = f32_to_bf16_bits_rn(__fadd_rn(v, margin));
+        if (lo == hi)
+            return lo;
+    }
+    const double xd = static_cast<double>(x);
+    const double y = 0.5 * xd * erfc(-xd * 0.70710678118654752440);
+    return f64_to_bf16_bits(y);
+}
+
+struct GeluParams {
+    const uint16_t *in;
+    uint16_t *out;
+    int64_t M, N, ld_in, ld_out;
+    int64_t vecs_per_row;  // ceil(N / 8)
+};
+
+__global__ void __launch_bounds__(256) gelu_kernel(const GeluParams p)
+{
+    const int64_t total = p.M * p.vecs_per_row;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t row = i / p.vecs_per_row;
+        const int64_t col = (i - row * p.vecs_per_row) * 8;
+        const uint16_t *src = p.in + row * p.ld_in + col;
+        uint16_t *dst = p.out + row * p.ld_out + col;
+        if (col + 8 <= p.N) {
+            const uint4 r = *reinterpret_cast<const uint4 *>(src);
+            const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+            uint32_t o[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                o[j] = gelu_bf16_bits(w[j] & 0xffffu) | (gelu_bf16_bits(w[j] >> 16) << 16);
+            st_v4(dst, o[0], o[1], o[2], o[3]);
+        } else {
+            for (int64_t j = 0; col + j < p.N; ++j)
+                dst[j] = static_cast<uint16_t>(gelu_bf16_bits(src[j]));
+        }
+    }
+}
+
+} // namespace sdnq

@@ -1,0 +1,330 @@
+// INT8 x INT8 -> INT32 matmul on the 5th-generation tensor cores (tcgen05.mma kind::i8,
+// accumulators in tensor memory), fed by TMA through a shared-memory ring, with the fp32
+// de-quant epilogue fused: out = bf16(float(acc) * (sx[m] * sw[n]) + bias[n]
+// [+ lora_scale * L[m][n]]), where L = u B is a second, bf16 x bf16 -> fp32 tensor-core
+// accumulator (the PEFT adapter beside the frozen int8 base).
+//
+// Sources: "SDNQ: SD.Next Quantization Engine" README, feature list (INT8 quantized matmul)
+// and SDNQConfig (dequantize_fp32: FP32 scales and FP32 de-quant steps); "ConvRot / Hadamard
+// SDNQ", PEFT Behavior (int8 frozen base, bf16 adapters).
+//
+// Shape of the kernel (one CTA per SM, persistent over output tiles):
+//   warp 0      TMA producer (one lane): A tile [128 x 128 B], B tile [BN x 128 B] per stage
+//   warp 1      TMEM allocator and MMA issuer (one lane): 4 MMAs of K = 32 per stage
+//   warps 2..5  epilogue: TMEM -> registers -> scales, bias, LoRA -> bf16 -> global
+// Two accumulator buffers in TMEM let the epilogue of tile i overlap the MMAs of tile i+1.
+// Operand tiles use the 128-byte swizzle written by TMA and read by the MMA descriptors.
+//
+// Every wait is bounded (mbar_wait_bounded): on timeout the CTA raises its abort flag and
+// the device error word, each role leaves its loop, in-flight copies and MMAs are drained
+// with bounded waits, and TMEM is freed before the CTA exits.
+#pragma once
+
+#include <cuda_bf16.h>
+
+#include "device.cuh"
+
+namespace sdnq {
+
+struct GemmParams {
+    const float *sx;          // [M]
+    const float *sw;          // [N]
+    const uint16_t *bias;     // [N] bf16 or nullptr
+    uint16_t *out;            // [M, ldo] bf16
+    int64_t ldo;
+    int32_t *acc_out;         // [M, N] int32 or nullptr
+    int32_t M, N, K;
+    int32_t num_kb;           // ceil(K / 128)
+    int32_t num_m_blocks;     // ceil(M / 128)
+    int32_t num_tiles;
+    int32_t lora_chunks;      // ceil(rank / 64); 0 without LoRA
+    float lora_scale;
+    uint64_t timeout_ns;
+};
+
+template <int BN, bool LORA>
+struct GemmConfig {
+    static constexpr int BM = 128;
+    static constexpr int BK = 128;                     // bytes of K per stage (int8)
+    static constexpr int A_BYTES = BM * BK;            // 16 KB
+    static constexpr int B_BYTES = BN * BK;            // 16 or 32 KB
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    static constexpr int STAGES = (BN == 256) ? 4 : 6;
+    static constexpr int ACC_COLS = LORA ? 2 * BN : BN;   // TMEM columns per buffer
+    static constexpr int TMEM_COLS = 2 * ACC_COLS;        // two buffers
+    static constexpr int THREADS = 192;
+    // barriers: full[S], empty[S], tfull[2], tempty[2], drain; then tmem base + abort flag
+    static constexpr int BAR_BYTES = (2 * STAGES + 5) * 8;
+    static constexpr int SMEM_BYTES = 1024 /*align slack*/ + STAGES * STAGE_BYTES + BAR_BYTES + 16;
+    static_assert(TMEM_COLS <= 512, "tensor memory holds 512 columns");
+    static_assert(BN % 32 == 0 && BN >= 64 && BN <= 256, "tile width");
+};
+
+__device__ __forceinline__ float bf16_bits_to_float(uint32_t b) { return __uint_as_float(b << 16); }
+
+__device__ __forceinline__ uint32_t float_to_bf16_bits(float f)
+{
+    return static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(f)));
+}
+
+template <int BN, bool LORA>
+__global__ void __launch_bounds__(192, 1)
+    gemm_s8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CUtensorMap tmL,
+                   const GemmParams p)
+{
+    using C = GemmConfig<BN, LORA>;
+    extern __shared__ uint8_t smem_raw[];
+    // 1024-byte alignment for the 128-byte swizzle atoms
+    const uint32_t raw_addr = smem_u32(smem_raw);
+    const uint32_t base = (raw_addr + 1023u) & ~1023u;
+    uint8_t *smem = smem_raw + (base - raw_addr);
+    const uint32_t bar0 = base + C::STAGES * C::STAGE_BYTES;
+    auto full_bar = [&](int s) { return bar0 + 8u * s; };
+    auto empty_bar = [&](int s) { return bar0 + 8u * (C::STAGES + s); };
+    auto tfull_bar = [&](int b) { return bar0 + 8u * (2 * C::STAGES + b); };
+    auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * C::STAGES + 2 + b); };
+    const uint32_t drain_bar = bar0 + 8u * (2 * C::STAGES + 4);
+    uint32_t *tmem_holder =
+        reinterpret_cast<uint32_t *>(smem + C::STAGES * C::STAGE_BYTES + C::BAR_BYTES);
+    volatile int *abort = reinterpret_cast<volatile int *>(tmem_holder + 1);
+
+    const uint32_t warp = threadIdx.x >> 5;
+    const uint32_t lane = lane_id();
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::STAGES; ++s) {
+            mbar_init(full_bar(s), 1);
+            mbar_init(empty_bar(s), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(tfull_bar(b), 1);
+            mbar_init(tempty_bar(b), 128);
+        }
+        mbar_init(drain_bar, 1);
+        *abort = 0;
+        fence_mbar_init();
+        prefetch_tensormap(&tmA);
+        prefetch_tensormap(&tmB);
+        if (LORA) {
+            prefetch_tensormap(&tmU);
+            prefetch_tensormap(&tmL);
+        }
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_holder), C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem_base = *tmem_holder;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int issued = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
+                const int m0 = (tile % p.num_m_blocks) * C::BM;
+                const int n0 = (tile / p.num_m_blocks) * BN;
+                const int steps = p.num_kb + (LORA ? p.lora_chunks : 0);
+                for (int kb = 0; kb < steps; ++kb) {
+                    if (!mbar_wait_bounded(empty_bar(stage), phase ^ 1u, abort, p.timeout_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t sa = base + stage * C::STAGE_BYTES;
+                    const uint32_t sb = sa + C::A_BYTES;
+                    if (!LORA || kb < p.num_kb) {
+                        mbar_arrive_expect_tx(full_bar(stage), C::STAGE_BYTES);
+                        tma_load_2d(sa, &tmA, full_bar(stage), kb * C::BK, m0);
+                        tma_load_2d(sb, &tmB, full_bar(stage), kb * C::BK, n0);
+                    } else {
+                        // LoRA chunk c: U [128 x 64] bf16 (K-major) into the A slot and
+                        // B [64 x BN] bf16 (N-major) as BN/64 boxes into the B slot
+                        const int c = kb - p.num_kb;
+                        mbar_arrive_expect_tx(full_bar(stage), 128 * 128 + BN * 128);
+                        tma_load_2d(sa, &tmU, full_bar(stage), c * 64, m0);
+#pragma unroll
+                        for (int j = 0; j < BN / 64; ++j)
+                            tma_load_2d(sb + j * 8192, &tmL, full_bar(stage), n0 + 64 * j, c * 64);
+                    }
+                    ++issued;
+                    if (++stage == C::STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (!ok) {
+                // drain: wait (bounded) for the copies of the last stages issued
+                const int n = issued < C::STAGES ? issued : C::STAGES;
+                int s = stage;
+                uint32_t ph = phase;
+                for (int i = 0; i < n; ++i) {
+                    if (--s < 0) {
+                        s = C::STAGES - 1;
+                        ph ^= 1u;
+                    }
+                    volatile int no_abort = 0;
+                    mbar_wait_bounded(full_bar(s), ph, &no_abort, p.timeout_ns);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t IDESC_I8 = idesc_s8_s32(128, BN);
+            constexpr uint32_t IDESC_BF = idesc_bf16_f32(128, BN, true);
+            int stage = 0;
+            uint32_t phase = 0;
+            int local = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x, ++local) {
+                const int buf = local & 1;
+                const uint32_t use = static_cast<uint32_t>(local >> 1);
+                if (!mbar_wait_bounded(tempty_bar(buf), (use & 1u) ^ 1u, abort, p.timeout_ns)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after_sync();
+                const uint32_t d_acc = tmem_base + buf * C::ACC_COLS;
+                for (int kb = 0; kb < p.num_kb; ++kb) {
+                    if (!mbar_wait_bounded(full_bar(stage), phase, abort, p.timeout_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after_sync();
+                    const uint32_t sa = base + stage * C::STAGE_BYTES;
+                    const uint32_t sb = sa + C::A_BYTES;
+#pragma unroll
+                    for (int k = 0; k < C::BK / 32; ++k)
+                        mma_s8(d_acc, kmajor_desc(sa + 32 * k), kmajor_desc(sb + 32 * k), IDESC_I8,
+                               (kb | k) != 0 ? 1u : 0u);
+                    tc_commit(empty_bar(stage));
+                    if (++stage == C::STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (LORA) {
+                    const uint32_t d_lora = d_acc + BN;
+                    for (int c = 0; ok && c < p.lora_chunks; ++c) {
+                        if (!mbar_wait_bounded(full_bar(stage), phase, abort, p.timeout_ns)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after_sync();
+                        const uint32_t sa = base + stage * C::STAGE_BYTES;
+                        const uint32_t sb = sa + C::A_BYTES;
+                        // 4 MMAs of K = 16 rows of rank each: A advances 32 bytes along its
+                        // swizzled K-major rows, B advances 16 K-rows = 2048 bytes
+#pragma unroll
+                        for (int k = 0; k < 4; ++k)
+                            mma_f16(d_lora, kmajor_desc(sa + 32 * k), mnmajor_desc(sb + 2048 * k, 8192),
+                                    IDESC_BF, (c | k) != 0 ? 1u : 0u);
+                        tc_commit(empty_bar(stage));
+                        if (++stage == C::STAGES) {
+                            stage = 0;
+                            phase ^= 1u;
+                        }
+                    }
+                }
+                if (!ok)
+                    break;
+                tc_commit(tfull_bar(buf));
+            }
+            // drain: every MMA this thread issued has completed before TMEM is freed
+            tc_commit(drain_bar);
+            volatile int no_abort = 0;
+            mbar_wait_bounded(drain_bar, 0u, &no_abort, p.timeout_ns);
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue (warps 2..5)
+        const uint32_t quad = warp & 3u;  // TMEM lanes this warp may access: 32*quad ..
+        const int row_in_tile = static_cast<int>(quad * 32u + lane);
+        int local = 0;
+        for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++local) {
+            const int buf = local & 1;
+            const uint32_t use = static_cast<uint32_t>(local >> 1);
+            // warp-uniform decision: tcgen05.ld below needs the whole warp converged
+            const bool ready = mbar_wait_bounded(tfull_bar(buf), use & 1u, abort, p.timeout_ns);
+            if (!__all_sync(0xffffffffu, ready))
+                break;
+            tc_fence_after_sync();
+            const int m0 = (tile % p.num_m_blocks) * C::BM;
+            const int n0 = (tile / p.num_m_blocks) * BN;
+            const int m = m0 + row_in_tile;
+            const bool row_ok = m < p.M;
+            const float sxm = row_ok ? p.sx[m] : 0.0f;
+            const uint32_t t_row = tmem_base + ((quad * 32u) << 16) + buf * C::ACC_COLS;
+            uint16_t *orow = p.out + static_cast<int64_t>(row_ok ? m : 0) * p.ldo;
+#pragma unroll 1
+            for (int c = 0; c < BN / 32; ++c) {
+                const int nc = n0 + c * 32;
+                if (nc >= p.N)
+                    break;  // warp-uniform
+                uint32_t acc[32];
+                tmem_ld_32x32b_x32(t_row + c * 32, acc);
+                uint32_t lacc[LORA ? 32 : 1];
+                if constexpr (LORA)
+                    tmem_ld_32x32b_x32(t_row + BN + c * 32, lacc);
+                tmem_ld_wait();
+                if (!row_ok)
+                    continue;
+                const bool full = nc + 32 <= p.N;
+                uint32_t ob[16];
+#pragma unroll
+                for (int j2 = 0; j2 < 16; ++j2) {
+                    uint32_t h[2];
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const int j = 2 * j2 + e;
+                        const int n = nc + j;
+                        const bool nok = full || n < p.N;
+                        const float swn = nok ? __ldg(p.sw + n) : 0.0f;
+                        const float t = __fmul_rn(sxm, swn);
+                        float v = __fmul_rn(__int2float_rn(static_cast<int>(acc[j])), t);
+                        if (p.bias != nullptr)
+                            v = __fadd_rn(v, nok ? bf16_bits_to_float(__ldg(p.bias + n)) : 0.0f);
+                        if constexpr (LORA)
+                            v = __fadd_rn(v, __fmul_rn(p.lora_scale, __uint_as_float(lacc[j])));
+                        h[e] = float_to_bf16_bits(v);
+                    }
+                    ob[j2] = h[0] | (h[1] << 16);
+                }
+                if (full) {
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        st_v4(orow + nc + 8 * q, ob[4 * q], ob[4 * q + 1], ob[4 * q + 2], ob[4 * q + 3]);
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        if (nc + j < p.N)
+                            orow[nc + j] = static_cast<uint16_t>(ob[j >> 1] >> (16 * (j & 1)));
+                }
+                if (p.acc_out != nullptr) {
+                    int32_t *arow = p.acc_out + static_cast<int64_t>(m) * p.N;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        if (nc + j < p.N)
+                            arow[nc + j] = static_cast<int32_t>(acc[j]);
+                }
+            }
+            tc_fence_before_sync();
+            mbar_arrive(tempty_bar(buf));
+        }
+    }
+
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after_sync();
+        tmem_dealloc(tmem_base, C::TMEM_COLS);
+    }
+}
+
+} // namespace sdnq

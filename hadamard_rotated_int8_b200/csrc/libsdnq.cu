@@ -1,0 +1,447 @@
+// libsdnq.so: the C ABI declared in include/sdnq.h. Host side: argument validation, TMA
+// tensor-map encoding, launch configuration and the device error word. All arithmetic of the
+// layer runs in the kernels included below.
+#include <cmath>
+#include <cstdint>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "sdnq.h"
+
+#include "device.cuh"
+#include "gelu.cuh"
+#include "gemm.cuh"
+#include "lora_down.cuh"
+#include "rotquant.cuh"
+
+#define SDNQ_API extern "C" __attribute__((visibility("default")))
+
+namespace sdnq {
+namespace {
+
+constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;  // 2 s for any single wait
+
+// ---------------------------------------------------------------- device checks
+
+struct DeviceInfo {
+    int checked = 0;
+    int supported = 0;
+    int sm_count = 0;
+};
+DeviceInfo g_dev[64];
+std::mutex g_dev_mutex;
+
+sdnq_status current_device(DeviceInfo *out)
+{
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+        cudaGetLastError();
+        return SDNQ_ERR_UNSUPPORTED;  // no usable CUDA device: no sm_100 to run on
+    }
+    std::lock_guard<std::mutex> lock(g_dev_mutex);
+    DeviceInfo &d = g_dev[dev];
+    if (!d.checked) {
+        int major = 0, minor = 0, sms = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+            cudaGetLastError();
+            return SDNQ_ERR_CUDA;
+        }
+        d.supported = (major == 10 && minor == 0) ? 1 : 0;
+        d.sm_count = sms;
+        d.checked = 1;
+    }
+    *out = d;
+    return d.supported ? SDNQ_OK : SDNQ_ERR_UNSUPPORTED;
+}
+
+// ---------------------------------------------------------------- tensor maps
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+        cudaGetLastError();
+    });
+    return fn;
+}
+
+// 2-D row-major tensor [outer, inner] with a row stride in bytes, 128-byte swizzled boxes.
+bool make_tmap_2d(CUtensorMap *map, CUtensorMapDataType dtype, const void *ptr, uint64_t inner,
+                  uint64_t outer, uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn)
+        return false;
+    const cuuint64_t dims[2] = {inner, outer};
+    const cuuint64_t strides[1] = {row_stride_bytes};
+    const cuuint32_t box[2] = {box_inner, box_outer};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = fn(map, dtype, 2, const_cast<void *>(ptr), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// ---------------------------------------------------------------- validation helpers
+
+inline bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+inline bool is_pow2(int64_t v) { return v > 0 && (v & (v - 1)) == 0; }
+
+sdnq_status launch_status()
+{
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? SDNQ_OK : SDNQ_ERR_CUDA;
+}
+
+template <typename Kernel>
+bool set_smem(Kernel k, int bytes)
+{
+    return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess;
+}
+
+// ---------------------------------------------------------------- rotate + quantize
+
+sdnq_status validate_rotquant(const void *x, int64_t rows, int64_t K, int64_t ld, int32_t group,
+                              const void *q, const void *s)
+{
+    if (!x || !q || !s)
+        return SDNQ_ERR_NULL;
+    if (rows < 0 || rows > INT32_MAX || K <= 0 || K > SDNQ_MAX_K || K % 16 != 0 || ld < K)
+        return SDNQ_ERR_SHAPE;
+    if (!is_pow2(group) || group < SDNQ_MIN_GROUP || group > SDNQ_MAX_GROUP)
+        return SDNQ_ERR_UNSUPPORTED;
+    if (K % group != 0)
+        return SDNQ_ERR_SHAPE;
+    if (ld % 8 != 0 || !aligned(x, 16) || !aligned(q, 16) || !aligned(s, 4))
+        return SDNQ_ERR_ALIGN;
+    return SDNQ_OK;
+}
+
+template <int G>
+void launch_rotquant_g(const RotquantParams &p, dim3 grid, dim3 block, cudaStream_t st)
+{
+    rotquant_kernel<G><<<grid, block, 0, st>>>(p);
+}
+
+sdnq_status run_rotquant(const uint16_t *x, int64_t rows, int64_t K, int64_t ld, int32_t group,
+                         int8_t *q, float *s, void *stream)
+{
+    sdnq_status st = validate_rotquant(x, rows, K, ld, group, q, s);
+    if (st != SDNQ_OK)
+        return st;
+    DeviceInfo dev;
+    if ((st = current_device(&dev)) != SDNQ_OK)
+        return st;
+    if (rows == 0)
+        return SDNQ_OK;
+    RotquantParams p;
+    p.x = x;
+    p.ldx = ld;
+    p.q = q;
+    p.s = s;
+    p.M = rows;
+    p.K = static_cast<int32_t>(K);
+    p.nchunks = static_cast<int32_t>((K + 1023) / 1024);
+    p.wpr = p.nchunks < 16 ? p.nchunks : 16;  // <= 512 threads per CTA
+    p.rpc = p.wpr <= 8 ? 8 / p.wpr : 1;
+    p.c_g = static_cast<float>(1.0 / std::sqrt(static_cast<double>(group)));
+    const dim3 block(32 * p.wpr * p.rpc);
+    const dim3 grid(static_cast<unsigned>((rows + p.rpc - 1) / p.rpc));
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    cudaGetLastError();
+    switch (group) {
+    case 8: launch_rotquant_g<8>(p, grid, block, cs); break;
+    case 16: launch_rotquant_g<16>(p, grid, block, cs); break;
+    case 32: launch_rotquant_g<32>(p, grid, block, cs); break;
+    case 64: launch_rotquant_g<64>(p, grid, block, cs); break;
+    case 128: launch_rotquant_g<128>(p, grid, block, cs); break;
+    default: launch_rotquant_g<256>(p, grid, block, cs); break;
+    }
+    return launch_status();
+}
+
+// ---------------------------------------------------------------- int8 linear (+ LoRA)
+
+sdnq_status validate_linear(const void *qx, const void *sx, const void *qW, const void *sW,
+                            const void *bias, int64_t M, int64_t N, int64_t K, const void *out,
+                            int64_t ldo, const void *acc_out)
+{
+    if (!qx || !sx || !qW || !sW || !out)
+        return SDNQ_ERR_NULL;
+    if (M < 0 || M > INT32_MAX || N <= 0 || N > INT32_MAX || K < 16 || K > SDNQ_MAX_K ||
+        K % 16 != 0 || ldo < N)
+        return SDNQ_ERR_SHAPE;
+    if (ldo % 8 != 0 || !aligned(qx, 16) || !aligned(qW, 16) || !aligned(out, 16) ||
+        !aligned(sx, 4) || !aligned(sW, 4) || (bias && !aligned(bias, 2)) ||
+        (acc_out && !aligned(acc_out, 16)))
+        return SDNQ_ERR_ALIGN;
+    return SDNQ_OK;
+}
+
+template <int BN, bool LORA>
+sdnq_status launch_gemm(const DeviceInfo &dev, const int8_t *qx, const int8_t *qW,
+                        const uint16_t *u, const uint16_t *B, int32_t rank, GemmParams p,
+                        cudaStream_t cs)
+{
+    using C = GemmConfig<BN, LORA>;
+    CUtensorMap tmA, tmB, tmU, tmL;
+    if (!make_tmap_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, qx, p.K, p.M, p.K, 128, 128) ||
+        !make_tmap_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, qW, p.K, p.N, p.K, 128, BN))
+        return SDNQ_ERR_CUDA;
+    if (LORA) {
+        if (!make_tmap_2d(&tmU, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, u, rank, p.M, 2ull * rank, 64, 128) ||
+            !make_tmap_2d(&tmL, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, B, p.N, rank, 2ull * p.N, 64, 64))
+            return SDNQ_ERR_CUDA;
+    } else {
+        tmU = tmA;
+        tmL = tmA;
+    }
+    static std::once_flag once;
+    static bool smem_ok = false;
+    std::call_once(once, [] { smem_ok = set_smem(gemm_s8_kernel<BN, LORA>, C::SMEM_BYTES); });
+    if (!smem_ok)
+        return SDNQ_ERR_CUDA;
+    p.num_kb = (p.K + C::BK - 1) / C::BK;
+    p.num_m_blocks = (p.M + C::BM - 1) / C::BM;
+    p.num_tiles = p.num_m_blocks * ((p.N + BN - 1) / BN);
+    const int grid = p.num_tiles < dev.sm_count ? p.num_tiles : dev.sm_count;
+    cudaGetLastError();
+    gemm_s8_kernel<BN, LORA><<<grid, C::THREADS, C::SMEM_BYTES, cs>>>(tmA, tmB, tmU, tmL, p);
+    return launch_status();
+}
+
+template <int RANK_PAD>
+sdnq_status launch_lora_down(const uint16_t *x, int64_t ldx, const uint16_t *A, int32_t rank,
+                             uint16_t *u, int32_t M, int32_t K, cudaStream_t cs)
+{
+    using C = LoraDownConfig<RANK_PAD>;
+    CUtensorMap tmX, tmA;
+    if (!make_tmap_2d(&tmX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, K, M, 2ull * ldx, 64, 128) ||
+        !make_tmap_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, A, rank, K, 2ull * rank, 64, 64))
+        return SDNQ_ERR_CUDA;
+    static std::once_flag once;
+    static bool smem_ok = false;
+    std::call_once(once, [] { smem_ok = set_smem(lora_down_kernel<RANK_PAD>, C::SMEM_BYTES); });
+    if (!smem_ok)
+        return SDNQ_ERR_CUDA;
+    LoraDownParams p;
+    p.u = u;
+    p.M = M;
+    p.K = K;
+    p.rank = rank;
+    p.num_kb = (K + 63) / 64;
+    p.timeout_ns = kDefaultTimeoutNs;
+    cudaGetLastError();
+    lora_down_kernel<RANK_PAD><<<(M + 127) / 128, 192, C::SMEM_BYTES, cs>>>(tmX, tmA, p);
+    return launch_status();
+}
+
+sdnq_status run_linear(const int8_t *qx, const float *sx, const int8_t *qW, const float *sW,
+                       const uint16_t *bias, const uint16_t *x, int64_t ldx, const uint16_t *A,
+                       const uint16_t *B, int32_t rank, float lora_scale, uint16_t *u_ws,
+                       int64_t M, int64_t N, int64_t K, uint16_t *out, int64_t ldo,
+                       int32_t *acc_out, void *stream, bool lora)
+{
+    sdnq_status st = validate_linear(qx, sx, qW, sW, bias, M, N, K, out, ldo, acc_out);
+    if (st != SDNQ_OK)
+        return st;
+    if (lora) {
+        if (!x || !A || !B || !u_ws)
+            return SDNQ_ERR_NULL;
+        if (ldx < K)
+            return SDNQ_ERR_SHAPE;
+        if (rank < 16 || rank > SDNQ_MAX_RANK || rank % 16 != 0)
+            return SDNQ_ERR_UNSUPPORTED;
+        if (N % 8 != 0)
+            return SDNQ_ERR_SHAPE;
+        if (ldx % 8 != 0 || !aligned(x, 16) || !aligned(A, 16) || !aligned(B, 16) ||
+            !aligned(u_ws, 16))
+            return SDNQ_ERR_ALIGN;
+    }
+    DeviceInfo dev;
+    if ((st = current_device(&dev)) != SDNQ_OK)
+        return st;
+    if (M == 0)
+        return SDNQ_OK;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    GemmParams p;
+    p.sx = sx;
+    p.sw = sW;
+    p.bias = bias;
+    p.out = out;
+    p.ldo = ldo;
+    p.acc_out = acc_out;
+    p.M = static_cast<int32_t>(M);
+    p.N = static_cast<int32_t>(N);
+    p.K = static_cast<int32_t>(K);
+    p.lora_chunks = 0;
+    p.lora_scale = lora_scale;
+    p.timeout_ns = kDefaultTimeoutNs;
+    if (!lora)
+        return launch_gemm<256, false>(dev, qx, qW, nullptr, nullptr, 0, p, cs);
+    const int32_t Mi = static_cast<int32_t>(M), Ki = static_cast<int32_t>(K);
+    if (rank <= 64)
+        st = launch_lora_down<64>(x, ldx, A, rank, u_ws, Mi, Ki, cs);
+    else if (rank <= 128)
+        st = launch_lora_down<128>(x, ldx, A, rank, u_ws, Mi, Ki, cs);
+    else
+        st = launch_lora_down<256>(x, ldx, A, rank, u_ws, Mi, Ki, cs);
+    if (st != SDNQ_OK)
+        return st;
+    p.lora_chunks = (rank + 63) / 64;
+    return launch_gemm<128, true>(dev, qx, qW, u_ws, B, rank, p, cs);
+}
+
+// ---------------------------------------------------------------- self-test kernel
+
+__global__ void wait_timeout_selftest_kernel(uint64_t limit_ns)
+{
+    __shared__ alignas(8) uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        abort_flag = 0;
+        mbar_init(smem_u32(&bar), 1);
+        fence_mbar_init();
+        // nothing ever arrives: phase 0 never completes, the bounded wait gives up
+        mbar_wait_bounded(smem_u32(&bar), 0u, &abort_flag, limit_ns);
+        mbar_arrive(smem_u32(&bar));  // leave the barrier consistent
+    }
+}
+
+} // namespace
+} // namespace sdnq
+
+using namespace sdnq;
+
+SDNQ_API sdnq_status sdnq_rotate_quant_weight(const uint16_t *W, int64_t N, int64_t K, int64_t ldw,
+                                              int32_t group, int8_t *qW, float *sW, void *stream)
+{
+    return run_rotquant(W, N, K, ldw, group, qW, sW, stream);
+}
+
+SDNQ_API sdnq_status sdnq_rotquant_act(const uint16_t *x, int64_t M, int64_t K, int64_t ldx,
+                                       int32_t group, int8_t *qx, float *sx, void *stream)
+{
+    return run_rotquant(x, M, K, ldx, group, qx, sx, stream);
+}
+
+SDNQ_API sdnq_status sdnq_int8_linear(const int8_t *qx, const float *sx, const int8_t *qW,
+                                      const float *sW, const uint16_t *bias, int64_t M, int64_t N,
+                                      int64_t K, uint16_t *out, int64_t ldo, int32_t *acc_out,
+                                      void *stream)
+{
+    return run_linear(qx, sx, qW, sW, bias, nullptr, 0, nullptr, nullptr, 0, 0.0f, nullptr, M, N, K,
+                      out, ldo, acc_out, stream, false);
+}
+
+SDNQ_API sdnq_status sdnq_int8_linear_lora(const int8_t *qx, const float *sx, const int8_t *qW,
+                                           const float *sW, const uint16_t *bias, const uint16_t *x,
+                                           int64_t ldx, const uint16_t *A, const uint16_t *B,
+                                           int32_t rank, float lora_scale, uint16_t *u_ws,
+                                           int64_t M, int64_t N, int64_t K, uint16_t *out,
+                                           int64_t ldo, int32_t *acc_out, void *stream)
+{
+    return run_linear(qx, sx, qW, sW, bias, x, ldx, A, B, rank, lora_scale, u_ws, M, N, K, out, ldo,
+                      acc_out, stream, true);
+}
+
+SDNQ_API sdnq_status sdnq_gelu_bf16(const uint16_t *in, int64_t M, int64_t N, int64_t ld_in,
+                                    uint16_t *out, int64_t ld_out, void *stream)
+{
+    if (!in || !out)
+        return SDNQ_ERR_NULL;
+    if (M < 0 || N <= 0 || ld_in < N || ld_out < N)
+        return SDNQ_ERR_SHAPE;
+    if (ld_in % 8 != 0 || ld_out % 8 != 0 || !aligned(in, 16) || !aligned(out, 16))
+        return SDNQ_ERR_ALIGN;
+    if (in == out && ld_in != ld_out)
+        return SDNQ_ERR_SHAPE;
+    DeviceInfo dev;
+    sdnq_status st = current_device(&dev);
+    if (st != SDNQ_OK)
+        return st;
+    if (M == 0)
+        return SDNQ_OK;
+    GeluParams p;
+    p.in = in;
+    p.out = out;
+    p.M = M;
+    p.N = N;
+    p.ld_in = ld_in;
+    p.ld_out = ld_out;
+    p.vecs_per_row = (N + 7) / 8;
+    const int64_t total = M * p.vecs_per_row;
+    int64_t blocks = (total + 255) / 256;
+    const int64_t cap = static_cast<int64_t>(dev.sm_count) * 16;
+    if (blocks > cap)
+        blocks = cap;
+    cudaGetLastError();
+    gelu_kernel<<<static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
+    return launch_status();
+}
+
+SDNQ_API sdnq_status sdnq_device_status(void *stream)
+{
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+        cudaGetLastError();
+        return SDNQ_ERR_CUDA;
+    }
+    unsigned int word = 0;
+    if (cudaMemcpyFromSymbol(&word, g_device_error, sizeof(word)) != cudaSuccess)
+        return SDNQ_ERR_CUDA;
+    if (word != kDevOk) {
+        const unsigned int zero = 0;
+        if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero)) != cudaSuccess)
+            return SDNQ_ERR_CUDA;
+        return SDNQ_ERR_TIMEOUT;
+    }
+    return SDNQ_OK;
+}
+
+SDNQ_API sdnq_status sdnq_selftest_wait_timeout(int64_t limit_ns, void *stream)
+{
+    if (limit_ns < 1000 || limit_ns > 10000000000ll)
+        return SDNQ_ERR_SHAPE;
+    DeviceInfo dev;
+    sdnq_status st = current_device(&dev);
+    if (st != SDNQ_OK)
+        return st;
+    cudaGetLastError();
+    wait_timeout_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<uint64_t>(limit_ns));
+    return launch_status();
+}
+
+SDNQ_API const char *sdnq_status_string(sdnq_status s)
+{
+    switch (s) {
+    case SDNQ_OK: return "SDNQ_OK";
+    case SDNQ_ERR_NULL: return "SDNQ_ERR_NULL: a required pointer is NULL";
+    case SDNQ_ERR_SHAPE: return "SDNQ_ERR_SHAPE: a size is out of range or sizes are inconsistent";
+    case SDNQ_ERR_ALIGN: return "SDNQ_ERR_ALIGN: a pointer or leading dimension breaks the 16-byte rule";
+    case SDNQ_ERR_UNSUPPORTED: return "SDNQ_ERR_UNSUPPORTED: unsupported group/rank or device is not sm_100";
+    case SDNQ_ERR_CUDA: return "SDNQ_ERR_CUDA: a CUDA runtime call or kernel launch failed";
+    case SDNQ_ERR_TIMEOUT: return "SDNQ_ERR_TIMEOUT: a bounded wait inside a kernel gave up";
+    }
+    return "SDNQ_ERR_UNKNOWN";
+}
+
+SDNQ_API const char *sdnq_version(void) { return "sdnq-b200 0.1.0 sm_100a"; }

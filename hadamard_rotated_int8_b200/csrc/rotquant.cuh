@@ -1,0 +1,247 @@
+// Fused online rotate + quantize: per row (token or weight row), a block-diagonal
+// Walsh-Hadamard butterfly over groups of G columns, the full-row absmax, the fp32 scale and
+// round-half-to-even int8 codes, in one pass over HBM.
+//
+// Sources: "SDNQ: SD.Next Quantization Engine" README (Hadamard rotations on both the
+// quantized weights and the quantized matmul; row-wise scales, FP32 de-quant); "ConvRot /
+// Hadamard SDNQ" (group 256 = ConvRot, smaller = QuaRot-style); "Hybrid-Sensitivity-
+// Weighted-Quantization" README, Rigorous grid / pack simulation (rotate, then absmax onto
+// the symmetric int8 grid).
+//
+// Work mapping. A row is cut into chunks of 1024 elements; one warp owns one chunk at a
+// time. Lane l = (hi2, lo3) with lo3 = l & 7 and hi2 = l >> 3; the lane holds four 16-byte
+// vectors v = 0..3, each of 8 consecutive bf16. Element index inside the chunk:
+//     e = hi2*256 + v*64 + lo3*8 + i          (i = 0..7 inside the vector)
+// so for a fixed v the warp's 32 loads cover four fully used 128-byte lines. For a
+// 256-group the butterfly bits map as: b0..b2 = i (in registers), b3..b5 = lo3 (lane
+// shuffles), b6..b7 = v (in registers): three of the eight stages need a shuffle.
+// Smaller groups use a prefix of the same bit order.
+//
+// Exactness. The butterfly runs its stages in ascending order h = 1, 2, ..., G/2, each
+// element one IEEE fp32 add or subtract. A shuffle stage computes fma(self, +-1, partner),
+// which is the single rounding of partner +- self. The quotient z / s_z is formed as
+// z * (1/s_z) and accepted only when it lies farther than 2^-14 from a half-integer (the
+// product is within 2.3e-5 of the IEEE quotient for |z/s_z| <= 127.5), so its
+// round-half-even integer equals that of the IEEE quotient; otherwise the IEEE division is
+// taken.
+#pragma once
+
+#include "device.cuh"
+
+namespace sdnq {
+
+struct RotquantParams {
+    const uint16_t *x;   // [M, K] bf16 patterns, row stride ldx
+    int64_t ldx;
+    int8_t *q;           // [M, K] dense
+    float *s;            // [M]
+    int64_t M;
+    int32_t K;
+    int32_t nchunks;     // ceil(K / 1024)
+    int32_t wpr;         // warps per row
+    int32_t rpc;         // rows per CTA
+    float c_g;           // fp32(1/sqrt(G))
+};
+
+__device__ __forceinline__ void bf16x8_to_f32(const uint4 r, float (&f)[8])
+{
+    f[0] = __uint_as_float(r.x << 16);
+    f[1] = __uint_as_float(r.x & 0xffff0000u);
+    f[2] = __uint_as_float(r.y << 16);
+    f[3] = __uint_as_float(r.y & 0xffff0000u);
+    f[4] = __uint_as_float(r.z << 16);
+    f[5] = __uint_as_float(r.z & 0xffff0000u);
+    f[6] = __uint_as_float(r.w << 16);
+    f[7] = __uint_as_float(r.w & 0xffff0000u);
+}
+
+// Unnormalised butterfly of the G-groups held by one warp (one chunk, 32 values per lane).
+template <int G>
+__device__ __forceinline__ void chunk_butterfly(float (&v)[4][8], uint32_t lane)
+{
+    // stages h = 1, 2, 4: inside each 8-element vector
+#pragma unroll
+    for (int h = 1; h <= 4; h <<= 1) {
+        if (G > h) {
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    if ((i & h) == 0) {
+                        const float a = v[t][i];
+                        const float b = v[t][i + h];
+                        v[t][i] = __fadd_rn(a, b);
+                        v[t][i + h] = __fsub_rn(a, b);
+                    }
+                }
+            }
+        }
+    }
+    // stages h = 8, 16, 32: across lanes lo3 ^ 1, ^ 2, ^ 4
+#pragma unroll
+    for (int sb = 0; sb < 3; ++sb) {
+        if (G > (8 << sb)) {
+            const float sgn = ((lane >> sb) & 1u) ? -1.0f : 1.0f;
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const float partner = __shfl_xor_sync(0xffffffffu, v[t][i], 1 << sb);
+                    v[t][i] = __fmaf_rn(v[t][i], sgn, partner);
+                }
+            }
+        }
+    }
+    // stages h = 64, 128: across the lane's vectors (v ^ 1, v ^ 2)
+#pragma unroll
+    for (int vb = 1; vb <= 2; vb <<= 1) {
+        if (G > (32 << vb)) {
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+                if ((t & vb) == 0) {
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const float a = v[t][i];
+                        const float b = v[t + vb][i];
+                        v[t][i] = __fadd_rn(a, b);
+                        v[t + vb][i] = __fsub_rn(a, b);
+                    }
+                }
+            }
+        }
+    }
+}
+
+__device__ __forceinline__ void load_chunk(const uint16_t *xr, int32_t K, int32_t c, bool ok,
+                                           uint32_t lane, float (&v)[4][8])
+{
+    const int32_t base = c * 1024 + static_cast<int32_t>(lane >> 3) * 256 +
+                         static_cast<int32_t>(lane & 7u) * 8;
+    uint4 raw[4];
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+        const int32_t e = base + t * 64;
+        raw[t] = make_uint4(0u, 0u, 0u, 0u);
+        if (ok && e < K)
+            raw[t] = ld_nc_v4(xr + e);
+    }
+#pragma unroll
+    for (int t = 0; t < 4; ++t)
+        bf16x8_to_f32(raw[t], v[t]);
+}
+
+__device__ __forceinline__ float chunk_absmax(const float (&v)[4][8])
+{
+    float m = 0.0f;
+#pragma unroll
+    for (int t = 0; t < 4; ++t)
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            m = fmaxf(m, fabsf(v[t][i]));
+    return m;
+}
+
+// Code of one value: round_half_even(z / s_z), as described in the file header.
+__device__ __forceinline__ uint32_t quant_code(float z, float s_z, float rcp, bool fast)
+{
+    const float p = __fmul_rn(z, rcp);
+    const float f = __fadd_rn(p, 12582912.0f);  // 1.5 * 2^23: rounds p to an integer
+    const float n = __fsub_rn(f, 12582912.0f);
+    const float e = fabsf(__fsub_rn(p, n));      // exact distance to that integer
+    if (fast && e < 0.5f - 0x1p-14f)
+        return __float_as_uint(f);               // low byte = the code (two's complement)
+    const float t = __fdiv_rn(z, s_z);
+    float r = rintf(t);
+    r = fminf(fmaxf(r, -127.0f), 127.0f);
+    return (t == t) ? static_cast<uint32_t>(__float2int_rn(r)) : 0u;
+}
+
+__device__ __forceinline__ uint32_t pack4(uint32_t a, uint32_t b, uint32_t c, uint32_t d)
+{
+    return __byte_perm(__byte_perm(a, b, 0x0040u), __byte_perm(c, d, 0x0040u), 0x5410u);
+}
+
+__device__ __forceinline__ void quant_store_chunk(const float (&v)[4][8], int8_t *qr, int32_t K,
+                                                  int32_t c, bool ok, uint32_t lane, float s_z,
+                                                  bool zero)
+{
+    const bool fast = s_z >= 0x1p-126f;
+    const float rcp = __frcp_rn(s_z);
+    const int32_t base = c * 1024 + static_cast<int32_t>(lane >> 3) * 256 +
+                         static_cast<int32_t>(lane & 7u) * 8;
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+        const int32_t e = base + t * 64;
+        uint32_t w0 = 0u, w1 = 0u;
+        if (!zero) {
+            uint32_t cd[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                cd[i] = quant_code(v[t][i], s_z, rcp, fast);
+            w0 = pack4(cd[0], cd[1], cd[2], cd[3]);
+            w1 = pack4(cd[4], cd[5], cd[6], cd[7]);
+        }
+        if (ok && e < K)
+            st_v2(qr + e, w0, w1);
+    }
+}
+
+template <int G>
+__global__ void __launch_bounds__(512) rotquant_kernel(const RotquantParams p)
+{
+    __shared__ float s_amax[32];
+    const uint32_t lane = lane_id();
+    const int32_t warp = static_cast<int32_t>(threadIdx.x >> 5);
+    const int32_t r_local = warp / p.wpr;
+    const int32_t wr = warp - r_local * p.wpr;
+    const int64_t row = static_cast<int64_t>(blockIdx.x) * p.rpc + r_local;
+    const bool row_ok = row < p.M;
+    const uint16_t *xr = p.x + (row_ok ? row : 0) * p.ldx;
+    int8_t *qr = p.q + (row_ok ? row : 0) * static_cast<int64_t>(p.K);
+
+    // chunks of this warp: wr, wr + wpr, ...
+    const int32_t my_chunks = (wr < p.nchunks) ? (p.nchunks - 1 - wr) / p.wpr + 1 : 0;
+    const bool single = my_chunks <= 1;
+
+    float v[4][8];
+    float amax = 0.0f;
+    if (single) {
+        load_chunk(xr, p.K, wr, row_ok && my_chunks == 1, lane, v);
+        chunk_butterfly<G>(v, lane);
+        amax = chunk_absmax(v);
+    } else {
+        // long rows: first pass for the absmax only; the second pass recomputes the
+        // rotation (the row is then read from L2)
+        for (int32_t j = 0; j < my_chunks; ++j) {
+            load_chunk(xr, p.K, wr + j * p.wpr, row_ok, lane, v);
+            chunk_butterfly<G>(v, lane);
+            amax = fmaxf(amax, chunk_absmax(v));
+        }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1)
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+    if (lane == 0)
+        s_amax[warp] = amax;
+    __syncthreads();
+    amax = 0.0f;
+    for (int32_t w = 0; w < p.wpr; ++w)
+        amax = fmaxf(amax, s_amax[r_local * p.wpr + w]);
+
+    const float s_z = __fdiv_rn(amax, 127.0f);
+    const bool zero = !(amax > 0.0f);
+    if (row_ok && wr == 0 && lane == 0)
+        p.s[row] = zero ? 0.0f : __fmul_rn(s_z, p.c_g);
+
+    if (single) {
+        quant_store_chunk(v, qr, p.K, wr, row_ok && my_chunks == 1, lane, s_z, zero);
+    } else {
+        for (int32_t j = 0; j < my_chunks; ++j) {
+            load_chunk(xr, p.K, wr + j * p.wpr, row_ok, lane, v);
+            chunk_butterfly<G>(v, lane);
+            quant_store_chunk(v, qr, p.K, wr + j * p.wpr, row_ok, lane, s_z, zero);
+        }
+    }
+}
+
+} // namespace sdnq

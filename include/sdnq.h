@@ -1,0 +1,163 @@
+/*
+ * sdnq.h -- C ABI of libsdnq.so: the Hadamard-rotated ("ConvRot") INT8 linear layer
+ * on NVIDIA B200 (sm_100a).
+ *
+ * What it computes (sources are web pages on the method, cited by title and section):
+ *  - "SDNQ: SD.Next Quantization Engine" README, feature list: Hadamard rotations apply on
+ *    both the quantized weights and the quantized matmul; INT8 quantized matmul.
+ *  - same README, SDNQConfig example: group_size = -1 is row-wise (one scale per output
+ *    row); hadamard_group_size; dequantize_fp32 keeps the scales in FP32 and runs the
+ *    de-quant steps in FP32.
+ *  - "ConvRot / Hadamard SDNQ" (SimpleTuner), What The Options Do: group 256 is ConvRot,
+ *    smaller groups are QuaRot-style; static full-row weight scales; the INT8 matmul path
+ *    stays active. PEFT Behavior: the frozen base runs in int8 while LoRA adapters stay bf16.
+ *  - "Hybrid-Sensitivity-Weighted-Quantization" README, Rigorous grid / pack simulation:
+ *    ConvRot = Hadamard rotate, then channelwise absmax onto the symmetric INT8 grid.
+ *
+ * Exact definition (the readings where the pages are silent are stated here too):
+ *  rotation   H_g = Sylvester Hadamard matrix in natural order, H[i][j] = (-1)^popcount(i&j),
+ *             applied block-diagonally along K in groups of g, normalised by 1/sqrt(g).
+ *             z = unnormalised butterfly of each group in fp32 with stages h = 1,2,..,g/2
+ *             in ascending order, (a,b) -> (a+b, a-b), every step IEEE round-to-nearest-even.
+ *  quantize   per row r: amax = max_k |z[r][k]| over the whole row; s_z = fp32(amax / 127);
+ *             q[r][k] = clamp(round_half_even(fp32(z[r][k] / s_z)), -127, 127);
+ *             stored scale s[r] = fp32(s_z * fp32(1/sqrt(g))). An all-zero row gives s = 0 and
+ *             codes 0. So x_rot ~= s * q, with x_rot = x H_g / sqrt(g).
+ *  matmul     acc[m][n] = sum_k qx[m][k] * qW[n][k] in int32 (exact for K <= 131072).
+ *  epilogue   fp32: t = sx[m]*sW[n]; v = float(acc)*t; v = v + bias[n];
+ *             (LoRA) v = v + lora_scale * L[m][n]; out = bf16_rne(v).
+ *  LoRA       u = bf16_rne(x A) (fp32 accumulation), L = u B (fp32 accumulation), where x is
+ *             the UNROTATED bf16 input: the adapter sits beside the frozen base layer.
+ *
+ * Conventions for every call:
+ *  - Pointers are DEVICE pointers owned by the caller; the library allocates no device
+ *    memory and keeps no per-call state. bf16 tensors are passed as their raw 16-bit
+ *    patterns (uint16_t). Matrices are row-major; "ld" arguments are row strides in
+ *    elements.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy default stream).
+ *    The return value reports only argument validation and launch errors; nothing is
+ *    launched when it is not SDNQ_OK, and outputs are then unspecified. Faults inside a
+ *    kernel surface at the caller's next synchronisation.
+ *  - Every bounded wait inside a kernel that gives up (default limit about 2 s) sets a
+ *    device error word; sdnq_device_status() reads and clears it (SDNQ_ERR_TIMEOUT).
+ *  - Only sm_100 devices are supported (SDNQ_ERR_UNSUPPORTED otherwise). There is no CPU
+ *    and no other-architecture path.
+ */
+#ifndef SDNQ_H
+#define SDNQ_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SDNQ_OK = 0,
+    SDNQ_ERR_NULL = 1,        /* a required pointer is NULL                               */
+    SDNQ_ERR_SHAPE = 2,       /* a size is out of range or sizes are inconsistent          */
+    SDNQ_ERR_ALIGN = 3,       /* a pointer or leading dimension breaks the 16-byte rule    */
+    SDNQ_ERR_UNSUPPORTED = 4, /* group size or rank not supported, or device is not sm_100 */
+    SDNQ_ERR_CUDA = 5,        /* a CUDA runtime call or a kernel launch failed             */
+    SDNQ_ERR_TIMEOUT = 6      /* a bounded wait inside a kernel gave up                    */
+} sdnq_status;
+
+/* Largest K accepted by every call (int32 accumulators stay exact: 127*127*K < 2^31). */
+#define SDNQ_MAX_K 131072
+/* Supported Hadamard group sizes: powers of two in [SDNQ_MIN_GROUP, SDNQ_MAX_GROUP]. */
+#define SDNQ_MIN_GROUP 8
+#define SDNQ_MAX_GROUP 256
+/* Supported LoRA ranks: multiples of 16 up to SDNQ_MAX_RANK. */
+#define SDNQ_MAX_RANK 256
+
+/*
+ * Weight rotate + quantize (offline, once per weight): "ConvRot / Hadamard SDNQ", Quick
+ * Setup and What The Options Do (sdnq_use_hadamard, sdnq_hadamard_group_size,
+ * sdnq_group_size = -1 static full-row scales); "SDNQ: SD.Next Quantization Engine",
+ * post-load quantization.
+ *   W   [N, K] bf16, row stride ldw (>= K, multiple of 8), 16-byte aligned.
+ *   qW  [N, K] int8 out, dense (row stride K), 16-byte aligned.
+ *   sW  [N]    fp32 out, scale of row n of the normalised rotation.
+ *   group: power of two, SDNQ_MIN_GROUP..SDNQ_MAX_GROUP; K % group == 0, K % 16 == 0,
+ *   K <= SDNQ_MAX_K. N == 0 is a no-op.
+ */
+sdnq_status sdnq_rotate_quant_weight(const uint16_t *W, int64_t N, int64_t K, int64_t ldw,
+                                     int32_t group, int8_t *qW, float *sW, void *stream);
+
+/*
+ * Online activation rotate + quantize, one dynamic scale per token: "SDNQ: SD.Next
+ * Quantization Engine", feature list (Hadamard on the quantized matmul; INT8 matmul).
+ * Same math as sdnq_rotate_quant_weight, applied to the rows (tokens) of x.
+ *   x   [M, K] bf16, row stride ldx (>= K, multiple of 8), 16-byte aligned.
+ *   qx  [M, K] int8 out, dense.   sx [M] fp32 out.   M == 0 is a no-op.
+ */
+sdnq_status sdnq_rotquant_act(const uint16_t *x, int64_t M, int64_t K, int64_t ldx,
+                              int32_t group, int8_t *qx, float *sx, void *stream);
+
+/*
+ * INT8 x INT8 -> INT32 matmul with the FP32 de-quant epilogue: "SDNQ: SD.Next Quantization
+ * Engine", feature list (INT8 quantized matmul) and SDNQConfig (dequantize_fp32).
+ *   qx [M, K] int8 dense, sx [M] fp32 (from sdnq_rotquant_act);
+ *   qW [N, K] int8 dense, sW [N] fp32 (from sdnq_rotate_quant_weight), same group size.
+ *   bias [N] bf16 or NULL.
+ *   out [M, N] bf16, row stride ldo (>= N, multiple of 8), 16-byte aligned.
+ *   acc_out: NULL, or [M, N] int32 dense that also receives the raw accumulators (for
+ *   parity checks; slower).
+ *   K % 16 == 0, K <= SDNQ_MAX_K, N >= 1. M == 0 is a no-op.
+ */
+sdnq_status sdnq_int8_linear(const int8_t *qx, const float *sx, const int8_t *qW,
+                             const float *sW, const uint16_t *bias, int64_t M, int64_t N,
+                             int64_t K, uint16_t *out, int64_t ldo, int32_t *acc_out,
+                             void *stream);
+
+/*
+ * As sdnq_int8_linear, plus the bf16 LoRA side term of PEFT training on a frozen int8
+ * base ("ConvRot / Hadamard SDNQ", PEFT Behavior): out = bf16(v + lora_scale * (u B)),
+ * u = bf16(x A).
+ *   x  [M, K] bf16, the UNROTATED layer input, row stride ldx (multiple of 8).
+ *   A  [K, rank] bf16 dense.   B [rank, N] bf16 dense (N % 8 == 0).
+ *   rank: multiple of 16, 16..SDNQ_MAX_RANK.
+ *   u_ws [M, rank] bf16: caller-provided workspace; holds u = bf16(x A) afterwards.
+ */
+sdnq_status sdnq_int8_linear_lora(const int8_t *qx, const float *sx, const int8_t *qW,
+                                  const float *sW, const uint16_t *bias, const uint16_t *x,
+                                  int64_t ldx, const uint16_t *A, const uint16_t *B,
+                                  int32_t rank, float lora_scale, uint16_t *u_ws, int64_t M,
+                                  int64_t N, int64_t K, uint16_t *out, int64_t ldo,
+                                  int32_t *acc_out, void *stream);
+
+/*
+ * GELU between the up and down projections of a DiT MLP (exact erf form,
+ * x * Phi(x), rounded once to bf16). Not on the pages; the MLP workload needs it.
+ *   in [M, N] bf16 row stride ld_in; out [M, N] bf16 row stride ld_out (may alias in when
+ *   ld_out == ld_in). Strides multiples of 8, pointers 16-byte aligned.
+ */
+sdnq_status sdnq_gelu_bf16(const uint16_t *in, int64_t M, int64_t N, int64_t ld_in,
+                           uint16_t *out, int64_t ld_out, void *stream);
+
+/*
+ * Synchronises `stream`, then reads and clears the device error word that bounded waits
+ * inside the kernels set when they give up. Returns SDNQ_OK, SDNQ_ERR_TIMEOUT, or
+ * SDNQ_ERR_CUDA if the synchronisation itself failed.
+ */
+sdnq_status sdnq_device_status(void *stream);
+
+/*
+ * Self-test of the bounded-wait machinery: launches one small kernel whose wait can never
+ * be satisfied (an mbarrier that nothing arrives on), with a limit of `limit_ns`
+ * nanoseconds (1e3..1e10). The kernel gives up, records SDNQ_ERR_TIMEOUT in the device
+ * error word and returns; no fault, trap or hang is involved.
+ */
+sdnq_status sdnq_selftest_wait_timeout(int64_t limit_ns, void *stream);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *sdnq_status_string(sdnq_status s);
+
+/* Library version string, e.g. "sdnq-b200 0.1.0 sm_100a". */
+const char *sdnq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SDNQ_H */

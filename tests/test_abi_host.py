@@ -1,0 +1,148 @@
+"""Host-only checks of the C ABI: the library loads, exports every entry point that
+include/sdnq.h declares, and rejects bad arguments before touching a GPU. Nothing here
+launches a kernel: every call either fails validation or (on a machine without a B200)
+fails the device check."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+import torch
+
+from hadamard_rotated_int8_b200 import _build, _native
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sdnq.h")
+
+A16 = 0x10000      # 16-byte aligned fake address: never dereferenced (validation fails first)
+MIS = 0x10001      # misaligned fake address
+S = 0              # stream: NULL
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"\b(sdnq_[a-z0-9_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    _build.build()
+    return _native.lib()
+
+
+def test_header_declares_the_four_layer_calls():
+    syms = declared_symbols()
+    for name in ("sdnq_rotate_quant_weight", "sdnq_rotquant_act", "sdnq_int8_linear",
+                 "sdnq_int8_linear_lora", "sdnq_status_string"):
+        assert name in syms
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+    out = subprocess.run(["nm", "-D", "--defined-only", _build.LIB], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (sdnq_\w+)", out))
+    assert set(declared_symbols()) <= exported
+    # nothing but the ABI is exported under the sdnq_ prefix
+    assert exported == set(declared_symbols())
+
+
+def test_binding_names_match_the_abi(lib):
+    import hadamard_rotated_int8_b200 as pkg
+    for name in ("sdnq_rotate_quant_weight", "sdnq_rotquant_act", "sdnq_int8_linear",
+                 "sdnq_int8_linear_lora", "sdnq_gelu_bf16"):
+        assert callable(getattr(pkg, name))
+    assert set(_native.SIGNATURES) == set(declared_symbols())
+
+
+def test_status_strings(lib):
+    for code in range(7):
+        s = _native.status_string(code)
+        assert s.startswith("SDNQ_")
+    assert _native.status_string(99) == "SDNQ_ERR_UNKNOWN"
+    assert "sm_100a" in _native.version()
+
+
+def rq(lib, x=A16, M=4, K=256, ld=256, g=256, q=A16, s=A16):
+    return lib.sdnq_rotquant_act(x, M, K, ld, g, q, s, S)
+
+
+def test_rotquant_validation(lib):
+    assert rq(lib, x=0) == _native.SDNQ_ERR_NULL
+    assert rq(lib, q=0) == _native.SDNQ_ERR_NULL
+    assert rq(lib, s=0) == _native.SDNQ_ERR_NULL
+    assert rq(lib, M=-1) == _native.SDNQ_ERR_SHAPE
+    assert rq(lib, K=0) == _native.SDNQ_ERR_SHAPE
+    assert rq(lib, K=264, ld=264) == _native.SDNQ_ERR_SHAPE        # K % 16
+    assert rq(lib, K=256, ld=128) == _native.SDNQ_ERR_SHAPE        # ld < K
+    assert rq(lib, K=262144, ld=262144) == _native.SDNQ_ERR_SHAPE  # K > max
+    assert rq(lib, g=4) == _native.SDNQ_ERR_UNSUPPORTED
+    assert rq(lib, g=512) == _native.SDNQ_ERR_UNSUPPORTED
+    assert rq(lib, g=96) == _native.SDNQ_ERR_UNSUPPORTED           # not a power of two
+    assert rq(lib, K=384, ld=384, g=256) == _native.SDNQ_ERR_SHAPE  # K % g
+    assert rq(lib, ld=260) == _native.SDNQ_ERR_ALIGN
+    assert rq(lib, x=MIS) == _native.SDNQ_ERR_ALIGN
+    assert rq(lib, q=A16 + 8) == _native.SDNQ_ERR_ALIGN
+    assert lib.sdnq_rotate_quant_weight(A16, 4, 256, 256, 256, 0, A16, S) == _native.SDNQ_ERR_NULL
+
+
+def lin(lib, qx=A16, sx=A16, qw=A16, sw=A16, bias=0, M=128, N=256, K=256, out=A16, ldo=256,
+        acc=0):
+    return lib.sdnq_int8_linear(qx, sx, qw, sw, bias, M, N, K, out, ldo, acc, S)
+
+
+def test_linear_validation(lib):
+    assert lin(lib, qx=0) == _native.SDNQ_ERR_NULL
+    assert lin(lib, sw=0) == _native.SDNQ_ERR_NULL
+    assert lin(lib, out=0) == _native.SDNQ_ERR_NULL
+    assert lin(lib, M=-3) == _native.SDNQ_ERR_SHAPE
+    assert lin(lib, N=0) == _native.SDNQ_ERR_SHAPE
+    assert lin(lib, K=8) == _native.SDNQ_ERR_SHAPE
+    assert lin(lib, K=200) == _native.SDNQ_ERR_SHAPE
+    assert lin(lib, ldo=128) == _native.SDNQ_ERR_SHAPE
+    assert lin(lib, ldo=260) == _native.SDNQ_ERR_ALIGN
+    assert lin(lib, qx=MIS) == _native.SDNQ_ERR_ALIGN
+    assert lin(lib, sx=A16 + 2) == _native.SDNQ_ERR_ALIGN
+    assert lin(lib, acc=A16 + 4) == _native.SDNQ_ERR_ALIGN
+
+
+def lora(lib, x=A16, A=A16, B=A16, rank=64, u=A16, N=256, ldx=256):
+    return lib.sdnq_int8_linear_lora(A16, A16, A16, A16, 0, x, ldx, A, B, rank, 1.0, u, 128, N,
+                                     256, A16, 256, 0, S)
+
+
+def test_lora_validation(lib):
+    assert lora(lib, x=0) == _native.SDNQ_ERR_NULL
+    assert lora(lib, u=0) == _native.SDNQ_ERR_NULL
+    assert lora(lib, rank=8) == _native.SDNQ_ERR_UNSUPPORTED
+    assert lora(lib, rank=24) == _native.SDNQ_ERR_UNSUPPORTED
+    assert lora(lib, rank=512) == _native.SDNQ_ERR_UNSUPPORTED
+    assert lora(lib, ldx=128) == _native.SDNQ_ERR_SHAPE
+    assert lora(lib, N=252) == _native.SDNQ_ERR_SHAPE  # B rows must be 16-byte strided
+    assert lora(lib, A=MIS) == _native.SDNQ_ERR_ALIGN
+
+
+def test_gelu_and_selftest_validation(lib):
+    assert lib.sdnq_gelu_bf16(0, 4, 8, 8, A16, 8, S) == _native.SDNQ_ERR_NULL
+    assert lib.sdnq_gelu_bf16(A16, 4, 0, 8, A16, 8, S) == _native.SDNQ_ERR_SHAPE
+    assert lib.sdnq_gelu_bf16(A16, 4, 8, 12, A16, 16, S) == _native.SDNQ_ERR_ALIGN
+    assert lib.sdnq_gelu_bf16(A16, 4, 8, 8, A16, 16, S) == _native.SDNQ_ERR_SHAPE  # alias, ld differ
+    assert lib.sdnq_selftest_wait_timeout(10, S) == _native.SDNQ_ERR_SHAPE
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU path only")
+def test_valid_arguments_without_a_b200_are_refused(lib):
+    # no silent CPU path: a well-formed call on a machine without an sm_100 GPU is refused
+    assert rq(lib) == _native.SDNQ_ERR_UNSUPPORTED
+    assert rq(lib, M=0) == _native.SDNQ_ERR_UNSUPPORTED
+    assert lin(lib) == _native.SDNQ_ERR_UNSUPPORTED
+    assert lora(lib) == _native.SDNQ_ERR_UNSUPPORTED
+    assert lib.sdnq_gelu_bf16(A16, 4, 8, 8, A16, 8, S) == _native.SDNQ_ERR_UNSUPPORTED
+
+
+def test_binding_refuses_cpu_tensors(lib):
+    import hadamard_rotated_int8_b200 as pkg
+    with pytest.raises(ValueError):
+        pkg.sdnq_rotquant_act(torch.zeros(4, 256, dtype=torch.bfloat16))

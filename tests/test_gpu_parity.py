@@ -1,0 +1,244 @@
+"""GPU parity: the CUDA library against the CPU oracle, element by element, on the same
+seeded bf16 inputs. Bit-exact on int8 codes, fp32 scales and int32 accumulators; bit-exact
+on bf16 outputs without LoRA (same fp32 op order), within one bf16 ulp with LoRA (the
+adapter's fp32 accumulation order differs). Every input comes from the seeded generator;
+every expected value from the oracle."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import hadamard_rotated_int8_b200 as sd
+from hadamard_rotated_int8_b200 import _build, synthetic
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    _build.build()
+    oracle.build()
+    torch.cuda.init()
+    yield
+    assert sd.sdnq_device_status() == 0
+
+
+def bits_of(t: torch.Tensor) -> np.ndarray:
+    return synthetic.bits(t.detach().cpu().contiguous())
+
+
+def bf16_val(b: np.ndarray) -> np.ndarray:
+    return (np.asarray(b, np.uint32) << 16).view(np.float32)
+
+
+def ulp_diff(a_bits: np.ndarray, b_bits: np.ndarray) -> np.ndarray:
+    """Distance in bf16 ulps (monotone integer mapping of the bit patterns)."""
+    def key(b):
+        b = b.astype(np.int32)
+        return np.where(b & 0x8000, 0x8000 - (b & 0x7fff), 0x8000 + b)
+    return np.abs(key(a_bits) - key(b_bits))
+
+
+def assert_equal(got, want, what):
+    got = np.asarray(got)
+    want = np.asarray(want)
+    assert got.shape == want.shape, (what, got.shape, want.shape)
+    bad = got != want
+    if bad.any():
+        idx = np.argwhere(bad)[:5]
+        raise AssertionError(f"{what}: {bad.sum()} of {bad.size} differ; first at {idx.tolist()}: "
+                             f"got {[got[tuple(i)] for i in idx]} want {[want[tuple(i)] for i in idx]}")
+
+
+def gpu_rotquant(x_cpu: torch.Tensor, g: int, weight=False):
+    x = x_cpu.cuda()
+    fn = sd.sdnq_rotate_quant_weight if weight else sd.sdnq_rotquant_act
+    q, s = fn(x, g)
+    torch.cuda.synchronize()
+    return q.cpu().numpy(), s.cpu().numpy()
+
+
+# ------------------------------------------------------------------ rotate + quantize
+
+ROTQUANT_CASES = [
+    (1, 256, 256), (37, 768, 256), (300, 3072, 256), (5, 16, 8), (64, 1040, 16),
+    (33, 4096, 64), (33, 4096, 128), (19, 3840, 256), (7, 10240, 256), (9, 2048, 32),
+    (3, 20480, 256), (2, 131072, 256), (1000, 256, 64),
+]
+
+
+@pytest.mark.parametrize("M,K,g", ROTQUANT_CASES)
+def test_rotquant_bit_exact(M, K, g):
+    case = synthetic.make_case(M=M, N=8, K=K, g=g, seed=M + K + g, outlier_count=min(K // 100, 40),
+                               outlier_factor=30.0)
+    x = case.x.clone()
+    if M > 4:
+        x[1] = 0                      # all-zero row
+        x[2, : min(K, 64)] = 1e-38    # tiny row: scale in the subnormal range
+        x[2, min(K, 64):] = 0
+        x[3] = x[3] * 1e30            # huge row, no overflow in the rotation
+    q, s = gpu_rotquant(x, g)
+    q_ref, s_ref = oracle.rotate_quantize(synthetic.bits(x), g)
+    assert_equal(q, q_ref, f"codes M={M} K={K} g={g}")
+    assert_equal(s.view(np.uint32), s_ref.view(np.uint32), f"scales M={M} K={K} g={g}")
+
+
+def test_rotquant_strided_input_and_weights_entry():
+    case = synthetic.make_case(M=70, N=96, K=1536, g=256, seed=5, outlier_count=12,
+                               outlier_factor=20.0)
+    wide = torch.zeros(70, 1536 + 64, dtype=torch.bfloat16)
+    wide[:, :1536] = case.x
+    xg = wide.cuda()[:, :1536]
+    assert xg.stride(0) == 1600
+    q, s = sd.sdnq_rotquant_act(xg, 256)
+    q_ref, s_ref = oracle.rotate_quantize(synthetic.bits(case.x), 256)
+    assert_equal(q.cpu().numpy(), q_ref, "strided codes")
+    assert_equal(s.cpu().numpy().view(np.uint32), s_ref.view(np.uint32), "strided scales")
+    qw, sw = gpu_rotquant(case.W, 256, weight=True)
+    qw_ref, sw_ref = oracle.rotate_quantize(synthetic.bits(case.W), 256)
+    assert_equal(qw, qw_ref, "weight codes")
+    assert_equal(sw.view(np.uint32), sw_ref.view(np.uint32), "weight scales")
+
+
+def test_rotquant_empty_batch_is_a_noop():
+    x = torch.zeros(0, 256, dtype=torch.bfloat16, device="cuda")
+    q, s = sd.sdnq_rotquant_act(x, 256)
+    assert q.shape == (0, 256) and s.shape == (0,)
+
+
+# ------------------------------------------------------------------ int8 linear
+
+def run_linear_case(case, with_acc=True, lora=False):
+    xg = case.x.cuda()
+    Wg = case.W.cuda()
+    qW, sW = sd.sdnq_rotate_quant_weight(Wg, case.g)
+    qx, sx = sd.sdnq_rotquant_act(xg, case.g)
+    bias = case.bias.cuda() if case.bias is not None else None
+    acc = torch.empty((case.M, case.N), dtype=torch.int32, device="cuda") if with_acc else None
+    if lora:
+        u = torch.empty((case.M, case.A.shape[1]), dtype=torch.bfloat16, device="cuda")
+        out = sd.sdnq_int8_linear_lora(qx, sx, qW, sW, bias, xg, case.A.cuda(), case.B.cuda(),
+                                       case.lora_scale, u_ws=u, acc_out=acc)
+    else:
+        u = None
+        out = sd.sdnq_int8_linear(qx, sx, qW, sW, bias, acc_out=acc)
+    torch.cuda.synchronize()
+    res = {"qx": qx.cpu().numpy(), "sx": sx.cpu().numpy(), "qW": qW.cpu().numpy(),
+           "sW": sW.cpu().numpy(), "out": bits_of(out)}
+    if acc is not None:
+        res["acc"] = acc.cpu().numpy()
+    if u is not None:
+        res["u"] = bits_of(u)
+    return res
+
+
+LINEAR_CASES = [
+    (128, 256, 128, 256), (1, 1, 256, 256), (300, 520, 768, 256), (257, 8, 256, 64),
+    (130, 300, 1040, 16), (129, 257, 4096, 128), (64, 1000, 512, 8), (512, 768, 3072, 256),
+]
+
+
+@pytest.mark.parametrize("M,N,K,g", LINEAR_CASES)
+@pytest.mark.parametrize("bias", [False, True])
+def test_linear_bit_exact_small(M, N, K, g, bias):
+    case = synthetic.make_case(M=M, N=N, K=K, g=g, seed=M * 7 + N, outlier_count=K // 64,
+                               outlier_factor=30.0, bias_std=0.01 if bias else None)
+    got = run_linear_case(case)
+    ref = oracle.linear(synthetic.bits(case.x),
+                        *oracle.rotate_quantize(synthetic.bits(case.W), g), g,
+                        bias_bits=synthetic.bits(case.bias) if bias else None)
+    assert_equal(got["qx"], ref["qx"], "qx")
+    assert_equal(got["sx"].view(np.uint32), ref["sx"].view(np.uint32), "sx")
+    assert_equal(got["acc"], ref["acc"], "int32 accumulators")
+    assert_equal(got["out"], ref["out"], "bf16 outputs")
+
+
+def test_linear_empty_batch_is_a_noop():
+    qx = torch.zeros(0, 256, dtype=torch.int8, device="cuda")
+    sx = torch.zeros(0, dtype=torch.float32, device="cuda")
+    qW = torch.zeros(64, 256, dtype=torch.int8, device="cuda")
+    sW = torch.zeros(64, dtype=torch.float32, device="cuda")
+    out = sd.sdnq_int8_linear(qx, sx, qW, sW)
+    assert out.shape == (0, 64)
+
+
+def test_linear_extreme_codes_max_accumulator():
+    """Every code +-127 at K = 131072 (the largest accepted K): |acc| = 127^2 K < 2^31."""
+    M, N, K = 3, 40, 131072
+    qx = torch.full((M, K), -127, dtype=torch.int8, device="cuda")
+    qx[1] = 127
+    qx[2, ::2] = 127
+    qW = torch.full((N, K), -127, dtype=torch.int8, device="cuda")
+    qW[5] = 127
+    sx = torch.ones(M, dtype=torch.float32, device="cuda")
+    sW = torch.ones(N, dtype=torch.float32, device="cuda")
+    acc = torch.empty((M, N), dtype=torch.int32, device="cuda")
+    out = sd.sdnq_int8_linear(qx, sx, qW, sW, acc_out=acc)
+    ref = oracle.gemm_s8(qx.cpu().numpy(), qW.cpu().numpy())
+    assert_equal(acc.cpu().numpy(), ref, "extreme accumulators")
+    ref_out = oracle.dequant_epilogue(ref, np.ones(M, np.float32), np.ones(N, np.float32))
+    assert_equal(bits_of(out), ref_out, "extreme outputs")
+
+
+# ------------------------------------------------------------------ LoRA
+
+@pytest.mark.parametrize("M,N,K,rank", [(128, 128, 256, 64), (300, 264, 512, 16),
+                                        (200, 520, 1024, 80), (129, 136, 768, 256)])
+def test_lora_within_one_ulp(M, N, K, rank):
+    case = synthetic.make_case(M=M, N=N, K=K, g=256, seed=rank + M, outlier_count=K // 100,
+                               outlier_factor=30.0, bias_std=0.01, lora_rank=rank,
+                               lora_scale=0.75)
+    got = run_linear_case(case, lora=True)
+    ref = oracle.linear(synthetic.bits(case.x), *oracle.rotate_quantize(synthetic.bits(case.W), 256),
+                        256, bias_bits=synthetic.bits(case.bias), A_bits=synthetic.bits(case.A),
+                        B_bits=synthetic.bits(case.B), lora_scale=0.75)
+    assert_equal(got["acc"], ref["acc"], "int32 accumulators (LoRA kernel)")
+    du = ulp_diff(got["u"], ref["u"])
+    assert du.max() <= 1, f"u: max {du.max()} ulp"
+    d = ulp_diff(got["out"], ref["out"])
+    assert d.max() <= 1, f"out: max {d.max()} ulp, {np.count_nonzero(d)} of {d.size} differ"
+
+
+# ------------------------------------------------------------------ GELU
+
+def test_gelu_bit_exact():
+    rng = np.random.default_rng(0)
+    vals = np.concatenate([rng.standard_normal(300_000) * 3, np.linspace(-14, 14, 40_001),
+                           [0.0, -0.0, 1e-30, -1e-30, 50, -50, 3e38, -3e38, 1e-40, -1e-40]])
+    n = (len(vals) // 8) * 8
+    x = torch.from_numpy(vals[:n].astype(np.float32)).to(torch.bfloat16).view(-1, 8)
+    out = sd.sdnq_gelu_bf16(x.cuda())
+    torch.cuda.synchronize()
+    assert_equal(bits_of(out), oracle.gelu_bf16(synthetic.bits(x)), "gelu")
+
+
+def test_gelu_ragged_and_strided():
+    x = (torch.randn(37, 133 + 11, generator=torch.Generator().manual_seed(3)) * 4).to(torch.bfloat16)
+    wide = x.cuda()
+    src = wide[:, :133]  # row stride 144, 133 columns: ragged tail
+    out = sd.sdnq_gelu_bf16(src.contiguous())
+    assert_equal(bits_of(out), oracle.gelu_bf16(synthetic.bits(x[:, :133].contiguous())), "gelu ragged")
+
+
+# ------------------------------------------------------------------ failure detection
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    assert sd.sdnq_device_status() == 0
+    sd.sdnq_selftest_wait_timeout(2_000_000)  # 2 ms limit on a wait nothing can satisfy
+    assert sd.sdnq_device_status() == sd._native.SDNQ_ERR_TIMEOUT
+    assert sd.sdnq_device_status() == 0       # cleared
+    x = torch.ones(2, 256, dtype=torch.bfloat16, device="cuda")
+    q, s = sd.sdnq_rotquant_act(x, 256)       # the context is still usable
+    assert int(q[0, 0]) == 127
+
+
+def test_calls_follow_the_current_stream():
+    case = synthetic.make_case(M=256, N=256, K=512, g=256, seed=11)
+    side = torch.cuda.Stream()
+    x = case.x.cuda()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(side):
+        q, s = sd.sdnq_rotquant_act(x, 256)
+    side.synchronize()
+    q_ref, _ = oracle.rotate_quantize(synthetic.bits(case.x), 256)
+    assert_equal(q.cpu().numpy(), q_ref, "side-stream codes")
