@@ -1,0 +1,477 @@
+"""Benchmark of the Hadamard-rotated INT8 linear layer on B200.
+
+One step = one pass of the online hot path over one batch of synthetic input: rotate +
+quantize the activations (per-token scales) and run the tensor-core int8 matmul with the
+fused fp32 de-quant epilogue (plus the LoRA term, or the MLP chain, for those workloads).
+Weights are rotated and quantized once before timing (offline, as on the pages).
+
+Default workload: the DiT attention projection, x [4096, 3072] bf16 with 1% outlier
+channels x30, W [3072, 3072], bias, Hadamard group 256.
+
+Output: one JSON line on rank 0. ``value`` is int8 TOPS of the whole step (2*M*N*K per
+GEMM over the device time of every kernel of the step), summed over ranks (replicas:
+each rank runs its own copy of the workload, no data-path collective).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--group G]
+  python bench.py --impl reference   # the CPU oracle on a bounded sample, same metric
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "int8 rotated-linear TOPS and % of dense INT8 peak; rotate+quant HBM GB/s"
+INT8_SPEC_TOPS = 4500.0        # B200 dense INT8, NVIDIA public spec
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+NOMINAL_INT8_OVER_BF16 = 2.0   # 4.5 / 2.25 PFLOP/s dense
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "hadamard_rotated_int8_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary for this workload,
+    if it was taken on the current kernel sources; else None."""
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    fields = {}
+    for line in text.splitlines():
+        if line.startswith("- ") and ":" in line:
+            k, v = line[2:].split(":", 1)
+            fields[k.strip()] = v.strip().strip("`")
+    if fields.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    try:
+        return float(fields["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+# ---------------------------------------------------------------------- workloads
+
+def workload_ops(case, name):
+    """int8 GEMM ops (2*M*N*K summed over the step's GEMMs) and extra bf16 LoRA flops."""
+    if name.startswith("dit_mlp"):
+        return 2 * 2 * case.M * case.N * case.K, 0
+    lora = 0
+    if case.A is not None:
+        r = case.A.shape[1]
+        lora = 2 * case.M * case.K * r + 2 * case.M * r * case.N
+    return 2 * case.M * case.N * case.K, lora
+
+
+def rotquant_bytes(M, K):
+    return M * K * 2 + M * K + M * 4   # read bf16, write int8 codes, write fp32 scale
+
+
+class Step:
+    """Device buffers and the stages of one step of a workload."""
+
+    def __init__(self, name, case, sd, torch):
+        self.name, self.case, self.sd, self.torch = name, case, sd, torch
+        dev = "cuda"
+        g = case.g
+        self.x = case.x.to(dev)
+        self.qx = torch.empty((case.M, case.K), dtype=torch.int8, device=dev)
+        self.sx = torch.empty((case.M,), dtype=torch.float32, device=dev)
+        self.bias = case.bias.to(dev) if case.bias is not None else None
+        self.qW, self.sW = sd.sdnq_rotate_quant_weight(case.W.to(dev), g)
+        self.out = torch.empty((case.M, case.N), dtype=torch.bfloat16, device=dev)
+        self.gemm_stages = []
+        if name.startswith("dit_mlp"):
+            Wd = case.extra["W_down"].to(dev)
+            self.qWd, self.sWd = sd.sdnq_rotate_quant_weight(Wd, g)
+            self.h = torch.empty((case.M, case.N), dtype=torch.bfloat16, device=dev)
+            self.qh = torch.empty((case.M, case.N), dtype=torch.int8, device=dev)
+            self.sh = torch.empty((case.M,), dtype=torch.float32, device=dev)
+            self.down = torch.empty((case.M, case.K), dtype=torch.bfloat16, device=dev)
+            self.stages = [
+                ("rotquant", lambda: sd.sdnq_rotquant_act(self.x, g, self.qx, self.sx)),
+                ("gemm_up", lambda: sd.sdnq_int8_linear(self.qx, self.sx, self.qW, self.sW,
+                                                        None, out=self.out)),
+                ("gelu", lambda: sd.sdnq_gelu_bf16(self.out, out=self.h)),
+                ("rotquant_h", lambda: sd.sdnq_rotquant_act(self.h, g, self.qh, self.sh)),
+                ("gemm_down", lambda: sd.sdnq_int8_linear(self.qh, self.sh, self.qWd, self.sWd,
+                                                          None, out=self.down)),
+            ]
+            self.gemm_stages = ["gemm_up", "gemm_down"]
+            self.launches = 5
+        elif case.A is not None:
+            self.A, self.B = case.A.to(dev), case.B.to(dev)
+            self.u = torch.empty((case.M, case.A.shape[1]), dtype=torch.bfloat16, device=dev)
+            self.stages = [
+                ("rotquant", lambda: sd.sdnq_rotquant_act(self.x, g, self.qx, self.sx)),
+                ("gemm_lora", lambda: sd.sdnq_int8_linear_lora(
+                    self.qx, self.sx, self.qW, self.sW, self.bias, self.x, self.A, self.B,
+                    case.lora_scale, u_ws=self.u, out=self.out)),
+            ]
+            self.gemm_stages = ["gemm_lora"]
+            self.launches = 3  # rotquant, LoRA down-projection, fused GEMM
+        else:
+            self.stages = [
+                ("rotquant", lambda: sd.sdnq_rotquant_act(self.x, g, self.qx, self.sx)),
+                ("gemm", lambda: sd.sdnq_int8_linear(self.qx, self.sx, self.qW, self.sW,
+                                                     self.bias, out=self.out)),
+            ]
+            self.gemm_stages = ["gemm"]
+            self.launches = 2
+
+    def run(self):
+        for _, fn in self.stages:
+            fn()
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons with NVML while the timed region runs."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+        0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+    }
+
+    def __init__(self, device_index: int, period_s: float = 0.01):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.period = period_s
+        self._stop = threading.Event()
+        self._t = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # pragma: no cover - NVML missing
+            log(f"clock sampling unavailable: {e}")
+            self.nvml = None
+
+    def _loop(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nvml.nvmlDeviceGetClockInfo(self.h, self.nvml.NVML_CLOCK_SM))
+                mask = self.nvml.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if mask & bit and bit != 0x1:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nvml is not None:
+            self._t = threading.Thread(target=self._loop, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._t is not None:
+            self._t.join()
+
+    def summary(self):
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------- CPU oracle timing
+
+def oracle_step(case, rows, nthreads):
+    """The oracle's pass over `rows` tokens of the workload (weights already quantized)."""
+    import oracle
+    from hadamard_rotated_int8_b200 import synthetic
+    xb = synthetic.bits(case.x)[:rows]
+    qx, sx = oracle.rotate_quantize(xb, case.g, nthreads)
+    acc = oracle.gemm_s8(qx, case._oracle_qW, nthreads)
+    L = None
+    if case.A is not None:
+        u = oracle.lora_down(xb, synthetic.bits(case.A), nthreads)
+        L = oracle.lora_up(u, synthetic.bits(case.B), nthreads)
+    bias = synthetic.bits(case.bias) if case.bias is not None else None
+    out = oracle.dequant_epilogue(acc, sx, case._oracle_sW, bias, L, case.lora_scale, nthreads)
+    if case._oracle_down is not None:
+        h = oracle.gelu_bf16(out, nthreads)
+        qh, sh = oracle.rotate_quantize(h, case.g, nthreads)
+        acc2 = oracle.gemm_s8(qh, case._oracle_down[0], nthreads)
+        oracle.dequant_epilogue(acc2, sh, case._oracle_down[1], None, None, 1.0, nthreads)
+
+
+def oracle_prepare(case, name, nthreads):
+    import oracle
+    from hadamard_rotated_int8_b200 import synthetic
+    case._oracle_qW, case._oracle_sW = oracle.rotate_quantize(synthetic.bits(case.W), case.g,
+                                                              nthreads)
+    case._oracle_down = None
+    if name.startswith("dit_mlp"):
+        case._oracle_down = oracle.rotate_quantize(synthetic.bits(case.extra["W_down"]), case.g,
+                                                   nthreads)
+
+
+def oracle_rows_for(case, name, nthreads, seconds):
+    """Rows (tokens) of the workload the oracle processes in about `seconds`."""
+    ops_full, _ = workload_ops(case, name)
+    probe = max(1, min(case.M, 16))
+    t0 = time.perf_counter()
+    oracle_step(case, probe, nthreads)
+    dt = max(time.perf_counter() - t0, 1e-4)
+    per_row = dt / probe
+    return int(max(1, min(case.M, seconds / per_row))), ops_full / case.M
+
+
+def cpu_baseline(case, name, budget_s=12.0):
+    nthreads = os.cpu_count() or 1
+    oracle_prepare(case, name, nthreads)
+    rows, ops_per_row = oracle_rows_for(case, name, nthreads, budget_s / 2)
+    reps, total, t_start = 0, 0.0, time.perf_counter()
+    while reps < 1 or (time.perf_counter() - t_start < budget_s and reps < 5):
+        t0 = time.perf_counter()
+        oracle_step(case, rows, nthreads)
+        total += time.perf_counter() - t0
+        reps += 1
+    tops = ops_per_row * rows * reps / total / 1e12
+    return {"value": tops, "unit": "TOPS", "cores": nthreads, "kind": "oracle",
+            "sample": f"{rows} of {case.M} tokens of {name} x{reps} (rotate+quantize, int8 GEMM "
+                      f"against all {case.N} weight rows, fp32 epilogue), {total:.2f} s"}
+
+
+def run_reference(args):
+    """The reference arm: the CPU oracle as it stands, on the machine's host cores, timed on a
+    bounded sample of the same workload per step."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from hadamard_rotated_int8_b200 import synthetic
+    case = synthetic.workload(args.workload, g=args.group)
+    nthreads = os.cpu_count() or 1
+    oracle_prepare(case, args.workload, nthreads)
+    per_step_budget = max(0.05, 150.0 / max(1, args.steps + args.warmup))
+    rows, ops_per_row = oracle_rows_for(case, args.workload, nthreads, per_step_budget)
+    for _ in range(args.warmup):
+        oracle_step(case, rows, nthreads)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_step(case, rows, nthreads)
+    dt = time.perf_counter() - t0
+    tops = ops_per_row * rows * args.steps / dt / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": tops, "unit": "TOPS",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+        "config": config_of(case, args),
+        "cpu_baseline": {"value": tops, "unit": "TOPS", "cores": nthreads, "kind": "oracle",
+                         "sample": f"{rows} of {case.M} tokens per step"},
+        "e2e": {"value": tops, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_of(case, args):
+    c = {"workload": args.workload, "M": case.M, "N": case.N, "K": case.K,
+         "hadamard_group": case.g, "bias": case.bias is not None,
+         "lora_rank": case.A.shape[1] if case.A is not None else 0,
+         "parallelism": f"replicas x{args.gpus}",
+         "l2": "flushed before every timed step (write of 2x the L2 size)"}
+    if args.workload.startswith("dit_mlp"):
+        c["chain"] = "rotquant -> up GEMM -> GELU -> rotquant -> down GEMM"
+    return c
+
+
+# ---------------------------------------------------------------------- GPU arm
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="sdnq", choices=["sdnq", "reference"])
+    ap.add_argument("--workload", default="dit_attn_4096x3072x3072")
+    ap.add_argument("--group", type=int, default=None)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        log("warmup raised to 3 (timing rules)")
+        args.warmup = 3
+
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+    import hadamard_rotated_int8_b200 as sd
+    from hadamard_rotated_int8_b200 import _build, synthetic
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    if rank == 0:
+        _build.build()
+    if world > 1:
+        dist.barrier()
+    sd.lib()
+
+    case = synthetic.workload(args.workload, g=args.group)
+    step = Step(args.workload, case, sd, torch)
+    l2 = torch.cuda.get_device_properties(local).L2_cache_size
+    flush = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device="cuda")
+    names = [n for n, _ in step.stages]
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step.run()
+    torch.cuda.synchronize()
+    assert sd.sdnq_device_status() == 0
+
+    # timed region: K steps, L2 flushed before each, per-stage CUDA events on the stream
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]
+           for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        for i in range(args.steps):
+            flush.zero_()
+            e = evs[i]
+            e[0].record()
+            for j, (_, fn) in enumerate(step.stages):
+                fn()
+                e[j + 1].record()
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    stage_ms = {n: 0.0 for n in names}
+    for e in evs:
+        for j, n in enumerate(names):
+            stage_ms[n] += e[j].elapsed_time(e[j + 1])
+    step_ms_total = sum(stage_ms.values())
+    t = torch.tensor([step_ms_total] + [stage_ms[n] for n in names], dtype=torch.float64,
+                     device="cuda")
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    step_ms_total = float(t[0])
+    stage_ms = {n: float(t[1 + j]) for j, n in enumerate(names)}
+    assert sd.sdnq_device_status() == 0
+
+    ops, lora_flops = workload_ops(case, args.workload)
+    ms_per_step = step_ms_total / args.steps
+    value = world * ops / (ms_per_step * 1e-3) / 1e12
+
+    # end to end through the public API: pinned host input -> device -> step -> host output
+    e2e = None
+    if not args.no_e2e:
+        n_e2e = max(3, min(args.steps, 50))
+        x_host = case.x.pin_memory()
+        out_host = torch.empty(step.out.shape if not args.workload.startswith("dit_mlp")
+                               else step.down.shape, dtype=torch.bfloat16).pin_memory()
+        res = step.down if args.workload.startswith("dit_mlp") else step.out
+        for _ in range(2):
+            step.x.copy_(x_host, non_blocking=True)
+            step.run()
+            out_host.copy_(res, non_blocking=True)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(n_e2e):
+            step.x.copy_(x_host, non_blocking=True)
+            step.run()
+            out_host.copy_(res, non_blocking=True)
+        e1.record()
+        torch.cuda.synchronize()
+        te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device="cuda")
+        if world > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        e2e = {"value": world * ops * n_e2e / (float(te[0]) * 1e-3) / 1e12, "unit": "TOPS",
+               "h2d_bytes_per_step": x_host.numel() * 2,
+               "d2h_bytes_per_step": out_host.numel() * 2, "steps": n_e2e}
+
+    peaks, peak_src = measured_peaks()
+    int8_peak = peaks["bf16_tflops"] * NOMINAL_INT8_OVER_BF16
+    gemm_ms = sum(stage_ms[n] for n in step.gemm_stages) / args.steps
+    gemm_launch_ms = gemm_ms / len(step.gemm_stages)
+    gemm_tops = ops / (gemm_ms * 1e-3) / 1e12
+    rq_ms = stage_ms["rotquant"] / args.steps
+    rq_gbs = rotquant_bytes(case.M, case.K) / (rq_ms * 1e-3) / 1e9
+    gemm_kernel = "gemm_s8_kernel" if case.A is None else "gemm_s8_kernel_lora"
+    line = {
+        "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
+        "data": "synthetic (seeded DiT-shaped bf16 activations with outlier channels, "
+                "random-init weights)",
+        "config": config_of(case, args),
+        "roofline": {
+            "kernel": gemm_kernel, "bound": "tensor", "achieved": gemm_tops,
+            "peak": int8_peak, "unit": "TFLOP/s", "frac": gemm_tops / int8_peak,
+            "traffic": profiled_traffic("gemm_s8", args.workload),
+            "ops_per_launch": ops / len(step.gemm_stages), "ms_per_launch": gemm_launch_ms,
+            "peak_source": f"{peak_src} bf16 burst x {NOMINAL_INT8_OVER_BF16} (int8/bf16 nominal)",
+            "frac_of_int8_spec": gemm_tops / INT8_SPEC_TOPS,
+        },
+        "roofline_rotquant": {
+            "kernel": "rotquant_kernel", "bound": "hbm", "achieved": rq_gbs,
+            "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": rq_gbs / peaks["hbm_gbs"],
+            "traffic": profiled_traffic("rotquant", args.workload),
+            "bytes_per_launch": rotquant_bytes(case.M, case.K), "ms_per_launch": rq_ms,
+            "peak_source": f"{peak_src} copy bandwidth",
+        },
+        "stage_ms_per_step": {n: stage_ms[n] / args.steps for n in names},
+        "clocks": clocks.summary(),
+        "gpu_launches": step.launches * args.steps,
+        "e2e": e2e,
+    }
+    if lora_flops:
+        line["tops_with_lora_flops"] = world * (ops + lora_flops) / (ms_per_step * 1e-3) / 1e12
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(case, args.workload)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

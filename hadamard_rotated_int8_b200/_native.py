@@ -126,6 +126,14 @@ def _dense(t: torch.Tensor, name: str):
         raise ValueError(f"{name}: must be contiguous")
 
 
+def _rows_out(M: int, N: int, dtype, device) -> torch.Tensor:
+    """[M, N] output whose row stride is padded to a multiple of 8 elements (the library
+    wants 16-byte aligned rows); returned as a view of the first N columns."""
+    ld = (N + 7) // 8 * 8
+    buf = torch.empty((M, ld), dtype=dtype, device=device)
+    return buf[:, :N] if ld != N else buf
+
+
 # ---------------------------------------------------------------- the C ABI, by name
 
 def sdnq_rotate_quant_weight(W: torch.Tensor, group: int = 256, qW=None, sW=None, stream=None):
@@ -160,7 +168,7 @@ def sdnq_int8_linear(qx, sx, qW, sW, bias=None, out=None, acc_out=None, stream=N
     N = qW.shape[0]
     if qW.shape[1] != K:
         raise ValueError("qx and qW disagree on K")
-    out = torch.empty((M, N), dtype=torch.bfloat16, device=qx.device) if out is None else out
+    out = _rows_out(M, N, torch.bfloat16, qx.device) if out is None else out
     _check(lib().sdnq_int8_linear(_ptr(qx), _ptr(sx), _ptr(qW), _ptr(sW), _ptr(bias), M, N, K,
                                   _ptr(out), out.stride(0), _ptr(acc_out), _stream(stream)),
            "sdnq_int8_linear")
@@ -181,7 +189,7 @@ def sdnq_int8_linear_lora(qx, sx, qW, sW, bias, x, A, B, lora_scale: float = 1.0
     if A.shape[0] != K or B.shape != (rank, N) or x.shape != (M, K):
         raise ValueError("LoRA shapes disagree")
     u_ws = torch.empty((M, rank), dtype=torch.bfloat16, device=qx.device) if u_ws is None else u_ws
-    out = torch.empty((M, N), dtype=torch.bfloat16, device=qx.device) if out is None else out
+    out = _rows_out(M, N, torch.bfloat16, qx.device) if out is None else out
     _check(lib().sdnq_int8_linear_lora(_ptr(qx), _ptr(sx), _ptr(qW), _ptr(sW), _ptr(bias),
                                        _ptr(x), x.stride(0), _ptr(A), _ptr(B), rank,
                                        float(lora_scale), _ptr(u_ws), M, N, K, _ptr(out),
@@ -194,7 +202,7 @@ def sdnq_gelu_bf16(x: torch.Tensor, out=None, stream=None):
     """Exact-erf GELU, bf16 -> bf16 (the MLP glue between up and down projections)."""
     _req(x, torch.bfloat16, "x", 2)
     M, N = x.shape
-    out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device) if out is None else out
+    out = _rows_out(M, N, torch.bfloat16, x.device) if out is None else out
     _check(lib().sdnq_gelu_bf16(_ptr(x), M, N, x.stride(0), _ptr(out), out.stride(0),
                                 _stream(stream)), "sdnq_gelu_bf16")
     return out

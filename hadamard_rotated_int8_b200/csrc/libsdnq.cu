@@ -122,7 +122,7 @@ bool set_smem(Kernel k, int bytes)
 sdnq_status validate_rotquant(const void *x, int64_t rows, int64_t K, int64_t ld, int32_t group,
                               const void *q, const void *s)
 {
-    if (!x || !q || !s)
+    if (rows != 0 && (!x || !q || !s))  // an empty batch may come with NULL buffers
         return SDNQ_ERR_NULL;
     if (rows < 0 || rows > INT32_MAX || K <= 0 || K > SDNQ_MAX_K || K % 16 != 0 || ld < K)
         return SDNQ_ERR_SHAPE;
@@ -184,7 +184,7 @@ sdnq_status validate_linear(const void *qx, const void *sx, const void *qW, cons
                             const void *bias, int64_t M, int64_t N, int64_t K, const void *out,
                             int64_t ldo, const void *acc_out)
 {
-    if (!qx || !sx || !qW || !sW || !out)
+    if (!qW || !sW || (M != 0 && (!qx || !sx || !out)))  // empty batch: NULL row buffers ok
         return SDNQ_ERR_NULL;
     if (M < 0 || M > INT32_MAX || N <= 0 || N > INT32_MAX || K < 16 || K > SDNQ_MAX_K ||
         K % 16 != 0 || ldo < N)
@@ -264,7 +264,7 @@ sdnq_status run_linear(const int8_t *qx, const float *sx, const int8_t *qW, cons
     if (st != SDNQ_OK)
         return st;
     if (lora) {
-        if (!x || !A || !B || !u_ws)
+        if (!A || !B || (M != 0 && (!x || !u_ws)))
             return SDNQ_ERR_NULL;
         if (ldx < K)
             return SDNQ_ERR_SHAPE;
@@ -366,7 +366,7 @@ SDNQ_API sdnq_status sdnq_int8_linear_lora(const int8_t *qx, const float *sx, co
 SDNQ_API sdnq_status sdnq_gelu_bf16(const uint16_t *in, int64_t M, int64_t N, int64_t ld_in,
                                     uint16_t *out, int64_t ld_out, void *stream)
 {
-    if (!in || !out)
+    if (M != 0 && (!in || !out))
         return SDNQ_ERR_NULL;
     if (M < 0 || N <= 0 || ld_in < N || ld_out < N)
         return SDNQ_ERR_SHAPE;

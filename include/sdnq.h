@@ -33,7 +33,8 @@
  *  - Pointers are DEVICE pointers owned by the caller; the library allocates no device
  *    memory and keeps no per-call state. bf16 tensors are passed as their raw 16-bit
  *    patterns (uint16_t). Matrices are row-major; "ld" arguments are row strides in
- *    elements.
+ *    elements. When the row count of a call (M, or N for the weight call) is 0 the call
+ *    is a no-op and the buffers that hold those rows may be NULL.
  *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy default stream).
  *    The return value reports only argument validation and launch errors; nothing is
  *    launched when it is not SDNQ_OK, and outputs are then unspecified. Faults inside a

