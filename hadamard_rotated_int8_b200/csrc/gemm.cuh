@@ -11,7 +11,9 @@
 // Shape of the kernel (one CTA per SM, persistent over output tiles):
 //   warp 0      TMA producer (one lane): A tile [128 x 128 B], B tile [BN x 128 B] per stage
 //   warp 1      TMEM allocator and MMA issuer (one lane): 4 MMAs of K = 32 per stage
-//   warps 2..5  epilogue: TMEM -> registers -> scales, bias, LoRA -> bf16 -> global
+//   warps 2..9  epilogue: TMEM -> registers -> scales, bias, LoRA -> bf16 -> global. A warp
+//               may only read the TMEM lanes 32*(warp % 4) .. +31, so two warps share each
+//               lane quarter and split the tile's columns in halves.
 // Two accumulator buffers in TMEM let the epilogue of tile i overlap the MMAs of tile i+1.
 // Operand tiles use the 128-byte swizzle written by TMA and read by the MMA descriptors.
 //
@@ -52,7 +54,8 @@ struct GemmConfig {
     static constexpr int STAGES = (BN == 256) ? 4 : 6;
     static constexpr int ACC_COLS = LORA ? 2 * BN : BN;   // TMEM columns per buffer
     static constexpr int TMEM_COLS = 2 * ACC_COLS;        // two buffers
-    static constexpr int THREADS = 192;
+    static constexpr int THREADS = 320;               // 2 + 8 warps
+    static constexpr int EPI_WARPS = 8;
     // barriers: full[S], empty[S], tfull[2], tempty[2], drain; then tmem base + abort flag
     static constexpr int BAR_BYTES = (2 * STAGES + 5) * 8;
     static constexpr int SMEM_BYTES = 1024 /*align slack*/ + STAGES * STAGE_BYTES + BAR_BYTES + 16;
@@ -68,7 +71,7 @@ __device__ __forceinline__ uint32_t float_to_bf16_bits(float f)
 }
 
 template <int BN, bool LORA>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     gemm_s8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CUtensorMap tmL,
                    const GemmParams p)
@@ -99,7 +102,7 @@ __global__ void __launch_bounds__(192, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(tfull_bar(b), 1);
-            mbar_init(tempty_bar(b), 128);
+            mbar_init(tempty_bar(b), C::EPI_WARPS);
         }
         mbar_init(drain_bar, 1);
         *abort = 0;
@@ -243,8 +246,9 @@ __global__ void __launch_bounds__(192, 1)
             mbar_wait_bounded(drain_bar, 0u, &no_abort, p.timeout_ns);
         }
     } else {
-        // ------------------------------------------------------------ epilogue (warps 2..5)
+        // ------------------------------------------------------------ epilogue (warps 2..9)
         const uint32_t quad = warp & 3u;  // TMEM lanes this warp may access: 32*quad ..
+        const int col_base = static_cast<int>((warp - 2u) >> 2) * (BN / 2);
         const int row_in_tile = static_cast<int>(quad * 32u + lane);
         int local = 0;
         for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++local) {
@@ -263,38 +267,63 @@ __global__ void __launch_bounds__(192, 1)
             const uint32_t t_row = tmem_base + ((quad * 32u) << 16) + buf * C::ACC_COLS;
             uint16_t *orow = p.out + static_cast<int64_t>(row_ok ? m : 0) * p.ldo;
 #pragma unroll 1
-            for (int c = 0; c < BN / 32; ++c) {
-                const int nc = n0 + c * 32;
+            for (int c = 0; c < BN / 2; c += 32) {
+                const int cc = col_base + c;   // column inside the tile
+                const int nc = n0 + cc;
                 if (nc >= p.N)
                     break;  // warp-uniform
+                const bool full = nc + 32 <= p.N;
+                // scales and bias of the 32 columns: the same addresses in every lane
+                float swv[32];
+                uint32_t bw[16];
+                if (full) {
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        const float4 f = __ldg(reinterpret_cast<const float4 *>(p.sw + nc) + q);
+                        swv[4 * q] = f.x; swv[4 * q + 1] = f.y; swv[4 * q + 2] = f.z; swv[4 * q + 3] = f.w;
+                    }
+                    if (p.bias != nullptr) {
+#pragma unroll
+                        for (int q = 0; q < 16; ++q)
+                            bw[q] = __ldg(reinterpret_cast<const uint32_t *>(p.bias + nc) + q);
+                    }
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        swv[j] = (nc + j < p.N) ? __ldg(p.sw + nc + j) : 0.0f;
+                    if (p.bias != nullptr) {
+#pragma unroll
+                        for (int q = 0; q < 16; ++q) {
+                            const uint32_t lo = (nc + 2 * q < p.N) ? __ldg(p.bias + nc + 2 * q) : 0u;
+                            const uint32_t hi = (nc + 2 * q + 1 < p.N) ? __ldg(p.bias + nc + 2 * q + 1) : 0u;
+                            bw[q] = lo | (hi << 16);
+                        }
+                    }
+                }
                 uint32_t acc[32];
-                tmem_ld_32x32b_x32(t_row + c * 32, acc);
+                tmem_ld_32x32b_x32(t_row + cc, acc);
                 uint32_t lacc[LORA ? 32 : 1];
                 if constexpr (LORA)
-                    tmem_ld_32x32b_x32(t_row + BN + c * 32, lacc);
+                    tmem_ld_32x32b_x32(t_row + BN + cc, lacc);
                 tmem_ld_wait();
                 if (!row_ok)
                     continue;
-                const bool full = nc + 32 <= p.N;
                 uint32_t ob[16];
 #pragma unroll
                 for (int j2 = 0; j2 < 16; ++j2) {
-                    uint32_t h[2];
+                    float v[2];
 #pragma unroll
                     for (int e = 0; e < 2; ++e) {
                         const int j = 2 * j2 + e;
-                        const int n = nc + j;
-                        const bool nok = full || n < p.N;
-                        const float swn = nok ? __ldg(p.sw + n) : 0.0f;
-                        const float t = __fmul_rn(sxm, swn);
-                        float v = __fmul_rn(__int2float_rn(static_cast<int>(acc[j])), t);
+                        const float t = __fmul_rn(sxm, swv[j]);
+                        v[e] = __fmul_rn(__int2float_rn(static_cast<int>(acc[j])), t);
                         if (p.bias != nullptr)
-                            v = __fadd_rn(v, nok ? bf16_bits_to_float(__ldg(p.bias + n)) : 0.0f);
+                            v[e] = __fadd_rn(v[e], __uint_as_float(e ? (bw[j2] & 0xffff0000u) : (bw[j2] << 16)));
                         if constexpr (LORA)
-                            v = __fadd_rn(v, __fmul_rn(p.lora_scale, __uint_as_float(lacc[j])));
-                        h[e] = float_to_bf16_bits(v);
+                            v[e] = __fadd_rn(v[e], __fmul_rn(p.lora_scale, __uint_as_float(lacc[j])));
                     }
-                    ob[j2] = h[0] | (h[1] << 16);
+                    const __nv_bfloat162 h2 = __floats2bfloat162_rn(v[0], v[1]);
+                    ob[j2] = *reinterpret_cast<const uint32_t *>(&h2);
                 }
                 if (full) {
 #pragma unroll
@@ -315,7 +344,9 @@ __global__ void __launch_bounds__(192, 1)
                 }
             }
             tc_fence_before_sync();
-            mbar_arrive(tempty_bar(buf));
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(tempty_bar(buf));
         }
     }
 

@@ -190,7 +190,7 @@ sdnq_status validate_linear(const void *qx, const void *sx, const void *qW, cons
         K % 16 != 0 || ldo < N)
         return SDNQ_ERR_SHAPE;
     if (ldo % 8 != 0 || !aligned(qx, 16) || !aligned(qW, 16) || !aligned(out, 16) ||
-        !aligned(sx, 4) || !aligned(sW, 4) || (bias && !aligned(bias, 2)) ||
+        !aligned(sx, 4) || !aligned(sW, 16) || (bias && !aligned(bias, 16)) ||
         (acc_out && !aligned(acc_out, 16)))
         return SDNQ_ERR_ALIGN;
     return SDNQ_OK;

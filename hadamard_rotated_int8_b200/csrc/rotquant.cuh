@@ -18,12 +18,13 @@
 // Smaller groups use a prefix of the same bit order.
 //
 // Exactness. The butterfly runs its stages in ascending order h = 1, 2, ..., G/2, each
-// element one IEEE fp32 add or subtract. A shuffle stage computes fma(self, +-1, partner),
-// which is the single rounding of partner +- self. The quotient z / s_z is formed as
-// z * (1/s_z) and accepted only when it lies farther than 2^-14 from a half-integer (the
-// product is within 2.3e-5 of the IEEE quotient for |z/s_z| <= 127.5), so its
-// round-half-even integer equals that of the IEEE quotient; otherwise the IEEE division is
-// taken.
+// element one IEEE fp32 add or subtract (packed two at a time with the f32x2 instructions,
+// which round each lane like the scalar ones). A shuffle stage computes fma(self, +-1,
+// partner), the single rounding of partner +- self. The quotient z / s_z is formed as
+// z * (1/s_z), which lies within 2.3e-5 of the IEEE quotient for |z/s_z| <= 127.5; when
+// every value of a vector lies farther than 2^-14 from a half-integer, its round-half-even
+// integer is therefore that of the IEEE quotient. Otherwise (about 3% of vectors) the whole
+// warp takes the IEEE division for that vector, so no per-element branch is needed.
 #pragma once
 
 #include "device.cuh"
@@ -55,29 +56,69 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4 r, float (&f)[8])
     f[7] = __uint_as_float(r.w & 0xffff0000u);
 }
 
+// Packed fp32 pairs (sm_100 f32x2 instructions): each op is two independent IEEE fp32
+// operations with round-to-nearest-even, the same results as the scalar ones.
+__device__ __forceinline__ void add2(float &d0, float &d1, float a0, float a1, float b0, float b1)
+{
+    asm("{\n\t.reg .b64 a, b, d;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+        "add.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
+        : "=f"(d0), "=f"(d1) : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+__device__ __forceinline__ void sub2(float &d0, float &d1, float a0, float a1, float b0, float b1)
+{
+    asm("{\n\t.reg .b64 a, b, d;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+        "sub.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
+        : "=f"(d0), "=f"(d1) : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+__device__ __forceinline__ void mul2(float &d0, float &d1, float a0, float a1, float b0, float b1)
+{
+    asm("{\n\t.reg .b64 a, b, d;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+        "mul.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
+        : "=f"(d0), "=f"(d1) : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+// d = a * b + c with one rounding per lane
+__device__ __forceinline__ void fma2(float &d0, float &d1, float a0, float a1, float b0, float b1,
+                                     float c0, float c1)
+{
+    asm("{\n\t.reg .b64 a, b, c, d;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+        "mov.b64 c, {%6, %7};\n\tfma.rn.f32x2 d, a, b, c;\n\tmov.b64 {%0, %1}, d;\n\t}"
+        : "=f"(d0), "=f"(d1) : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+
+// Butterfly pair (a, b) -> (a + b, a - b) on two adjacent pairs at once.
+__device__ __forceinline__ void bfly2(float &a0, float &a1, float &b0, float &b1)
+{
+    float s0, s1, d0, d1;
+    add2(s0, s1, a0, a1, b0, b1);
+    sub2(d0, d1, a0, a1, b0, b1);
+    a0 = s0; a1 = s1; b0 = d0; b1 = d1;
+}
+
 // Unnormalised butterfly of the G-groups held by one warp (one chunk, 32 values per lane).
 template <int G>
 __device__ __forceinline__ void chunk_butterfly(float (&v)[4][8], uint32_t lane)
 {
-    // stages h = 1, 2, 4: inside each 8-element vector
 #pragma unroll
-    for (int h = 1; h <= 4; h <<= 1) {
-        if (G > h) {
+    for (int t = 0; t < 4; ++t) {
+        // stage h = 1: the two halves of each loaded 32-bit word
 #pragma unroll
-            for (int t = 0; t < 4; ++t) {
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    if ((i & h) == 0) {
-                        const float a = v[t][i];
-                        const float b = v[t][i + h];
-                        v[t][i] = __fadd_rn(a, b);
-                        v[t][i + h] = __fsub_rn(a, b);
-                    }
-                }
-            }
+        for (int i = 0; i < 8; i += 2) {
+            const float a = v[t][i], b = v[t][i + 1];
+            v[t][i] = __fadd_rn(a, b);
+            v[t][i + 1] = __fsub_rn(a, b);
+        }
+        // stage h = 2: (0,1)+-(2,3), (4,5)+-(6,7)
+        if (G > 2) {
+            bfly2(v[t][0], v[t][1], v[t][2], v[t][3]);
+            bfly2(v[t][4], v[t][5], v[t][6], v[t][7]);
+        }
+        // stage h = 4: (0,1)+-(4,5), (2,3)+-(6,7)
+        if (G > 4) {
+            bfly2(v[t][0], v[t][1], v[t][4], v[t][5]);
+            bfly2(v[t][2], v[t][3], v[t][6], v[t][7]);
         }
     }
-    // stages h = 8, 16, 32: across lanes lo3 ^ 1, ^ 2, ^ 4
+    // stages h = 8, 16, 32: across lanes lo3 ^ 1, ^ 2, ^ 4; fma(self, +-1, partner)
 #pragma unroll
     for (int sb = 0; sb < 3; ++sb) {
         if (G > (8 << sb)) {
@@ -85,9 +126,10 @@ __device__ __forceinline__ void chunk_butterfly(float (&v)[4][8], uint32_t lane)
 #pragma unroll
             for (int t = 0; t < 4; ++t) {
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const float partner = __shfl_xor_sync(0xffffffffu, v[t][i], 1 << sb);
-                    v[t][i] = __fmaf_rn(v[t][i], sgn, partner);
+                for (int i = 0; i < 8; i += 2) {
+                    const float p0 = __shfl_xor_sync(0xffffffffu, v[t][i], 1 << sb);
+                    const float p1 = __shfl_xor_sync(0xffffffffu, v[t][i + 1], 1 << sb);
+                    fma2(v[t][i], v[t][i + 1], v[t][i], v[t][i + 1], sgn, sgn, p0, p1);
                 }
             }
         }
@@ -100,12 +142,8 @@ __device__ __forceinline__ void chunk_butterfly(float (&v)[4][8], uint32_t lane)
             for (int t = 0; t < 4; ++t) {
                 if ((t & vb) == 0) {
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const float a = v[t][i];
-                        const float b = v[t + vb][i];
-                        v[t][i] = __fadd_rn(a, b);
-                        v[t + vb][i] = __fsub_rn(a, b);
-                    }
+                    for (int i = 0; i < 8; i += 2)
+                        bfly2(v[t][i], v[t][i + 1], v[t + vb][i], v[t + vb][i + 1]);
                 }
             }
         }
@@ -141,24 +179,51 @@ __device__ __forceinline__ float chunk_absmax(const float (&v)[4][8])
     return m;
 }
 
-// Code of one value: round_half_even(z / s_z), as described in the file header.
-__device__ __forceinline__ uint32_t quant_code(float z, float s_z, float rcp, bool fast)
-{
-    const float p = __fmul_rn(z, rcp);
-    const float f = __fadd_rn(p, 12582912.0f);  // 1.5 * 2^23: rounds p to an integer
-    const float n = __fsub_rn(f, 12582912.0f);
-    const float e = fabsf(__fsub_rn(p, n));      // exact distance to that integer
-    if (fast && e < 0.5f - 0x1p-14f)
-        return __float_as_uint(f);               // low byte = the code (two's complement)
-    const float t = __fdiv_rn(z, s_z);
-    float r = rintf(t);
-    r = fminf(fmaxf(r, -127.0f), 127.0f);
-    return (t == t) ? static_cast<uint32_t>(__float2int_rn(r)) : 0u;
-}
-
 __device__ __forceinline__ uint32_t pack4(uint32_t a, uint32_t b, uint32_t c, uint32_t d)
 {
     return __byte_perm(__byte_perm(a, b, 0x0040u), __byte_perm(c, d, 0x0040u), 0x5410u);
+}
+
+// The exact path for one vector of 8 values: IEEE fp32 quotient, half-to-even, clamp.
+__device__ __noinline__ uint2 quant8_exact(float z0, float z1, float z2, float z3, float z4,
+                                           float z5, float z6, float z7, float s_z)
+{
+    const float z[8] = {z0, z1, z2, z3, z4, z5, z6, z7};
+    uint32_t c[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const float t = __fdiv_rn(z[i], s_z);
+        const float r = fminf(fmaxf(rintf(t), -127.0f), 127.0f);
+        c[i] = (t == t) ? static_cast<uint32_t>(__float2int_rn(r)) : 0u;
+    }
+    return make_uint2(pack4(c[0], c[1], c[2], c[3]), pack4(c[4], c[5], c[6], c[7]));
+}
+
+// Codes of one vector of 8 values: z * (1/s_z) rounded with the 1.5*2^23 trick; the exact
+// path runs (warp-uniformly) when any value of the warp's vector lies within 2^-14 of a
+// half-integer, or when s_z is subnormal.
+__device__ __forceinline__ uint2 quant8(const float (&z)[8], float s_z, float rcp, bool fast)
+{
+    constexpr float MAGIC = 12582912.0f;  // 1.5 * 2^23
+    float f[8];
+    float emax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; i += 2) {
+        float p0, p1, n0, n1, e0, e1;
+        mul2(p0, p1, z[i], z[i + 1], rcp, rcp);
+        add2(f[i], f[i + 1], p0, p1, MAGIC, MAGIC);
+        sub2(n0, n1, f[i], f[i + 1], MAGIC, MAGIC);
+        sub2(e0, e1, p0, p1, n0, n1);  // exact: |p - n| <= 1/2
+        emax = fmaxf(emax, fmaxf(fabsf(e0), fabsf(e1)));
+    }
+    const bool slow = !fast || !(emax < 0.5f - 0x1p-14f);
+    if (__any_sync(0xffffffffu, slow))
+        return quant8_exact(z[0], z[1], z[2], z[3], z[4], z[5], z[6], z[7], s_z);
+    // the low byte of f is the code in two's complement
+    return make_uint2(pack4(__float_as_uint(f[0]), __float_as_uint(f[1]), __float_as_uint(f[2]),
+                            __float_as_uint(f[3])),
+                      pack4(__float_as_uint(f[4]), __float_as_uint(f[5]), __float_as_uint(f[6]),
+                            __float_as_uint(f[7])));
 }
 
 __device__ __forceinline__ void quant_store_chunk(const float (&v)[4][8], int8_t *qr, int32_t K,
@@ -172,17 +237,11 @@ __device__ __forceinline__ void quant_store_chunk(const float (&v)[4][8], int8_t
 #pragma unroll
     for (int t = 0; t < 4; ++t) {
         const int32_t e = base + t * 64;
-        uint32_t w0 = 0u, w1 = 0u;
-        if (!zero) {
-            uint32_t cd[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-                cd[i] = quant_code(v[t][i], s_z, rcp, fast);
-            w0 = pack4(cd[0], cd[1], cd[2], cd[3]);
-            w1 = pack4(cd[4], cd[5], cd[6], cd[7]);
-        }
+        uint2 w = make_uint2(0u, 0u);
+        if (!zero)  // warp-uniform: the whole warp works on one row
+            w = quant8(v[t], s_z, rcp, fast);
         if (ok && e < K)
-            st_v2(qr + e, w0, w1);
+            st_v2(qr + e, w.x, w.y);
     }
 }
 

@@ -100,7 +100,7 @@ sdnq_status sdnq_rotquant_act(const uint16_t *x, int64_t M, int64_t K, int64_t l
  * Engine", feature list (INT8 quantized matmul) and SDNQConfig (dequantize_fp32).
  *   qx [M, K] int8 dense, sx [M] fp32 (from sdnq_rotquant_act);
  *   qW [N, K] int8 dense, sW [N] fp32 (from sdnq_rotate_quant_weight), same group size.
- *   bias [N] bf16 or NULL.
+ *   bias [N] bf16 or NULL. qx, qW, sW, bias and out are 16-byte aligned; sx 4-byte.
  *   out [M, N] bf16, row stride ldo (>= N, multiple of 8), 16-byte aligned.
  *   acc_out: NULL, or [M, N] int32 dense that also receives the raw accumulators (for
  *   parity checks; slower).

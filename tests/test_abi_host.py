@@ -105,6 +105,8 @@ def test_linear_validation(lib):
     assert lin(lib, ldo=260) == _native.SDNQ_ERR_ALIGN
     assert lin(lib, qx=MIS) == _native.SDNQ_ERR_ALIGN
     assert lin(lib, sx=A16 + 2) == _native.SDNQ_ERR_ALIGN
+    assert lin(lib, sw=A16 + 4) == _native.SDNQ_ERR_ALIGN
+    assert lin(lib, bias=A16 + 8) == _native.SDNQ_ERR_ALIGN
     assert lin(lib, acc=A16 + 4) == _native.SDNQ_ERR_ALIGN
 
 

@@ -207,9 +207,9 @@ def lora_tolerances(x_bits, A_bits, B_bits, u_ref_bits, out_ref_bits, scale, row
     Bv = np.abs(bf16_val(B_bits).astype(np.float64))
     K, r = Av.shape
     u_ref = bf16_val(u_ref_bits).astype(np.float64)
-    tol_u = np.abs(u_ref) * 2.0 ** -8 + 2 * K * 2.0 ** -24 * (np.abs(xv) @ Av) + 1e-30
+    tol_u = np.abs(u_ref) * 2.0 ** -7 + 2 * K * 2.0 ** -24 * (np.abs(xv) @ Av) + 1e-30
     out_ref = bf16_val(out_ref_bits).astype(np.float64)
-    tol_out = (np.abs(out_ref) * 2.0 ** -8
+    tol_out = (np.abs(out_ref) * 2.0 ** -7
                + abs(scale) * ((2 * tol_u) @ Bv + 2 * r * 2.0 ** -24 * (np.abs(u_ref) @ Bv))
                + 1e-30)
     return tol_u, tol_out
