@@ -56,9 +56,18 @@ struct GemmConfig {
     static constexpr int TMEM_COLS = 2 * ACC_COLS;        // two buffers
     static constexpr int THREADS = 320;               // 2 + 8 warps
     static constexpr int EPI_WARPS = 8;
+    static constexpr int EPI_COLS = BN / 2;           // columns per epilogue warp
+    // per epilogue warp: an output staging block [32 rows x 32 bf16] written with the
+    // 64-byte swizzle for the TMA store, and its columns' scales and bias as fp32
+    static constexpr int STAGE_OUT_BYTES = 32 * 64;
+    static constexpr int OUT_OFF = STAGES * STAGE_BYTES;
+    static constexpr int SCALE_OFF = OUT_OFF + EPI_WARPS * STAGE_OUT_BYTES;
+    static constexpr int SCALE_BYTES = EPI_COLS * 8;  // sw[EPI_COLS], bias[EPI_COLS]
+    static constexpr int BAR_OFF = SCALE_OFF + EPI_WARPS * SCALE_BYTES;
     // barriers: full[S], empty[S], tfull[2], tempty[2], drain; then tmem base + abort flag
     static constexpr int BAR_BYTES = (2 * STAGES + 5) * 8;
-    static constexpr int SMEM_BYTES = 1024 /*align slack*/ + STAGES * STAGE_BYTES + BAR_BYTES + 16;
+    static constexpr int SMEM_BYTES = 1024 /*align slack*/ + BAR_OFF + BAR_BYTES + 16;
+    static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
     static_assert(TMEM_COLS <= 512, "tensor memory holds 512 columns");
     static_assert(BN % 32 == 0 && BN >= 64 && BN <= 256, "tile width");
 };
@@ -74,7 +83,7 @@ template <int BN, bool LORA>
 __global__ void __launch_bounds__(320, 1)
     gemm_s8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CUtensorMap tmL,
-                   const GemmParams p)
+                   const __grid_constant__ CUtensorMap tmO, const GemmParams p)
 {
     using C = GemmConfig<BN, LORA>;
     extern __shared__ uint8_t smem_raw[];
@@ -82,14 +91,13 @@ __global__ void __launch_bounds__(320, 1)
     const uint32_t raw_addr = smem_u32(smem_raw);
     const uint32_t base = (raw_addr + 1023u) & ~1023u;
     uint8_t *smem = smem_raw + (base - raw_addr);
-    const uint32_t bar0 = base + C::STAGES * C::STAGE_BYTES;
+    const uint32_t bar0 = base + C::BAR_OFF;
     auto full_bar = [&](int s) { return bar0 + 8u * s; };
     auto empty_bar = [&](int s) { return bar0 + 8u * (C::STAGES + s); };
     auto tfull_bar = [&](int b) { return bar0 + 8u * (2 * C::STAGES + b); };
     auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * C::STAGES + 2 + b); };
     const uint32_t drain_bar = bar0 + 8u * (2 * C::STAGES + 4);
-    uint32_t *tmem_holder =
-        reinterpret_cast<uint32_t *>(smem + C::STAGES * C::STAGE_BYTES + C::BAR_BYTES);
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C::BAR_OFF + C::BAR_BYTES);
     volatile int *abort = reinterpret_cast<volatile int *>(tmem_holder + 1);
 
     const uint32_t warp = threadIdx.x >> 5;
@@ -109,6 +117,7 @@ __global__ void __launch_bounds__(320, 1)
         fence_mbar_init();
         prefetch_tensormap(&tmA);
         prefetch_tensormap(&tmB);
+        prefetch_tensormap(&tmO);
         if (LORA) {
             prefetch_tensormap(&tmU);
             prefetch_tensormap(&tmL);
@@ -248,94 +257,116 @@ __global__ void __launch_bounds__(320, 1)
     } else {
         // ------------------------------------------------------------ epilogue (warps 2..9)
         const uint32_t quad = warp & 3u;  // TMEM lanes this warp may access: 32*quad ..
-        const int col_base = static_cast<int>((warp - 2u) >> 2) * (BN / 2);
+        const uint32_t ew = warp - 2u;    // epilogue warp index 0..7
+        const int col_base = static_cast<int>(ew >> 2) * C::EPI_COLS;
         const int row_in_tile = static_cast<int>(quad * 32u + lane);
+        const uint32_t s_out = base + C::OUT_OFF + ew * C::STAGE_OUT_BYTES;
+        const uint32_t s_sw = base + C::SCALE_OFF + ew * C::SCALE_BYTES;
+        const uint32_t s_bias = s_sw + C::EPI_COLS * 4;
+        const bool has_bias = p.bias != nullptr;
         int local = 0;
         for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++local) {
             const int buf = local & 1;
             const uint32_t use = static_cast<uint32_t>(local >> 1);
+            const int m0 = (tile % p.num_m_blocks) * C::BM;
+            const int n0 = (tile / p.num_m_blocks) * BN;
+            const int nw = n0 + col_base;     // first column of this warp
+            // this warp's column scales and bias -> shared memory (fp32), before the wait
+            // on the accumulator so that their latency overlaps the MMAs
+#pragma unroll
+            for (int j = static_cast<int>(lane) * 4; j < C::EPI_COLS; j += 128) {
+                float w4[4], b4[4];
+                if (nw + j + 4 <= p.N) {
+                    const float4 f = __ldg(reinterpret_cast<const float4 *>(p.sw + nw + j));
+                    w4[0] = f.x; w4[1] = f.y; w4[2] = f.z; w4[3] = f.w;
+                    if (has_bias) {
+                        const uint2 bb = __ldg(reinterpret_cast<const uint2 *>(p.bias + nw + j));
+                        b4[0] = bf16_bits_to_float(bb.x & 0xffffu);
+                        b4[1] = bf16_bits_to_float(bb.x >> 16);
+                        b4[2] = bf16_bits_to_float(bb.y & 0xffffu);
+                        b4[3] = bf16_bits_to_float(bb.y >> 16);
+                    }
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const bool ok = nw + j + e < p.N;
+                        w4[e] = ok ? __ldg(p.sw + nw + j + e) : 0.0f;
+                        b4[e] = (ok && has_bias) ? bf16_bits_to_float(__ldg(p.bias + nw + j + e)) : 0.0f;
+                    }
+                }
+                if (!has_bias)
+                    b4[0] = b4[1] = b4[2] = b4[3] = 0.0f;
+                sts_v4(s_sw + 4 * j, __float_as_uint(w4[0]), __float_as_uint(w4[1]),
+                       __float_as_uint(w4[2]), __float_as_uint(w4[3]));
+                sts_v4(s_bias + 4 * j, __float_as_uint(b4[0]), __float_as_uint(b4[1]),
+                       __float_as_uint(b4[2]), __float_as_uint(b4[3]));
+            }
+            __syncwarp();
             // warp-uniform decision: tcgen05.ld below needs the whole warp converged
             const bool ready = mbar_wait_bounded(tfull_bar(buf), use & 1u, abort, p.timeout_ns);
             if (!__all_sync(0xffffffffu, ready))
                 break;
             tc_fence_after_sync();
-            const int m0 = (tile % p.num_m_blocks) * C::BM;
-            const int n0 = (tile / p.num_m_blocks) * BN;
             const int m = m0 + row_in_tile;
             const bool row_ok = m < p.M;
             const float sxm = row_ok ? p.sx[m] : 0.0f;
             const uint32_t t_row = tmem_base + ((quad * 32u) << 16) + buf * C::ACC_COLS;
-            uint16_t *orow = p.out + static_cast<int64_t>(row_ok ? m : 0) * p.ldo;
 #pragma unroll 1
-            for (int c = 0; c < BN / 2; c += 32) {
+            for (int c = 0; c < C::EPI_COLS; c += 32) {
                 const int cc = col_base + c;   // column inside the tile
                 const int nc = n0 + cc;
                 if (nc >= p.N)
                     break;  // warp-uniform
-                const bool full = nc + 32 <= p.N;
-                // scales and bias of the 32 columns: the same addresses in every lane
-                float swv[32];
-                uint32_t bw[16];
-                if (full) {
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        const float4 f = __ldg(reinterpret_cast<const float4 *>(p.sw + nc) + q);
-                        swv[4 * q] = f.x; swv[4 * q + 1] = f.y; swv[4 * q + 2] = f.z; swv[4 * q + 3] = f.w;
-                    }
-                    if (p.bias != nullptr) {
-#pragma unroll
-                        for (int q = 0; q < 16; ++q)
-                            bw[q] = __ldg(reinterpret_cast<const uint32_t *>(p.bias + nc) + q);
-                    }
-                } else {
-#pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        swv[j] = (nc + j < p.N) ? __ldg(p.sw + nc + j) : 0.0f;
-                    if (p.bias != nullptr) {
-#pragma unroll
-                        for (int q = 0; q < 16; ++q) {
-                            const uint32_t lo = (nc + 2 * q < p.N) ? __ldg(p.bias + nc + 2 * q) : 0u;
-                            const uint32_t hi = (nc + 2 * q + 1 < p.N) ? __ldg(p.bias + nc + 2 * q + 1) : 0u;
-                            bw[q] = lo | (hi << 16);
-                        }
-                    }
-                }
                 uint32_t acc[32];
                 tmem_ld_32x32b_x32(t_row + cc, acc);
                 uint32_t lacc[LORA ? 32 : 1];
                 if constexpr (LORA)
                     tmem_ld_32x32b_x32(t_row + BN + cc, lacc);
                 tmem_ld_wait();
-                if (!row_ok)
-                    continue;
+                // v = float(acc) * (sx * sw) [+ bias] [+ lora_scale * L], fp32 pairs
                 uint32_t ob[16];
 #pragma unroll
-                for (int j2 = 0; j2 < 16; ++j2) {
-                    float v[2];
+                for (int q = 0; q < 8; ++q) {
+                    const float4 w = lds_v4(s_sw + 4 * (c + 4 * q));
+                    const float4 b = lds_v4(s_bias + 4 * (c + 4 * q));
+                    const float wv[4] = {w.x, w.y, w.z, w.w};
+                    const float bv[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        const int j = 2 * j2 + e;
-                        const float t = __fmul_rn(sxm, swv[j]);
-                        v[e] = __fmul_rn(__int2float_rn(static_cast<int>(acc[j])), t);
-                        if (p.bias != nullptr)
-                            v[e] = __fadd_rn(v[e], __uint_as_float(e ? (bw[j2] & 0xffff0000u) : (bw[j2] << 16)));
-                        if constexpr (LORA)
-                            v[e] = __fadd_rn(v[e], __fmul_rn(p.lora_scale, __uint_as_float(lacc[j])));
+                    for (int h = 0; h < 2; ++h) {
+                        const int j = 4 * q + 2 * h;
+                        float t0, t1, v0, v1;
+                        mul2(t0, t1, sxm, sxm, wv[2 * h], wv[2 * h + 1]);
+                        mul2(v0, v1, __int2float_rn(static_cast<int>(acc[j])),
+                             __int2float_rn(static_cast<int>(acc[j + 1])), t0, t1);
+                        if (has_bias)
+                            add2(v0, v1, v0, v1, bv[2 * h], bv[2 * h + 1]);
+                        if constexpr (LORA) {
+                            float l0, l1;
+                            mul2(l0, l1, p.lora_scale, p.lora_scale, __uint_as_float(lacc[j]),
+                                 __uint_as_float(lacc[j + 1]));
+                            add2(v0, v1, v0, v1, l0, l1);
+                        }
+                        const __nv_bfloat162 h2 = __floats2bfloat162_rn(v0, v1);
+                        ob[j >> 1] = *reinterpret_cast<const uint32_t *>(&h2);
                     }
-                    const __nv_bfloat162 h2 = __floats2bfloat162_rn(v[0], v[1]);
-                    ob[j2] = *reinterpret_cast<const uint32_t *>(&h2);
                 }
-                if (full) {
+                // stage the 32 x 32 block (64-byte swizzle) and hand it to the TMA engine;
+                // rows >= M and columns >= N fall outside the tensor and are not written
+                if (lane == 0)
+                    bulk_wait_read_all();  // the previous block has left the staging buffer
+                __syncwarp();
+                const uint32_t row_addr = s_out + lane * 64u;
 #pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        st_v4(orow + nc + 8 * q, ob[4 * q], ob[4 * q + 1], ob[4 * q + 2], ob[4 * q + 3]);
-                } else {
-#pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        if (nc + j < p.N)
-                            orow[nc + j] = static_cast<uint16_t>(ob[j >> 1] >> (16 * (j & 1)));
+                for (int q = 0; q < 4; ++q)
+                    sts_v4(row_addr + ((static_cast<uint32_t>(q) ^ ((lane >> 1) & 3u)) << 4), ob[4 * q],
+                           ob[4 * q + 1], ob[4 * q + 2], ob[4 * q + 3]);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_2d(&tmO, s_out, nc, m0 + static_cast<int>(quad * 32u));
+                    bulk_commit_group();
                 }
-                if (p.acc_out != nullptr) {
+                if (p.acc_out != nullptr && row_ok) {
                     int32_t *arow = p.acc_out + static_cast<int64_t>(m) * p.N;
 #pragma unroll
                     for (int j = 0; j < 32; ++j)
@@ -348,6 +379,8 @@ __global__ void __launch_bounds__(320, 1)
             if (lane == 0)
                 mbar_arrive(tempty_bar(buf));
         }
+        if (lane == 0)
+            bulk_wait_all();  // every output block is in global memory before the CTA exits
     }
 
     tc_fence_before_sync();

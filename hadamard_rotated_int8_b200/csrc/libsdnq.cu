@@ -83,9 +83,10 @@ EncodeTiledFn encode_fn()
     return fn;
 }
 
-// 2-D row-major tensor [outer, inner] with a row stride in bytes, 128-byte swizzled boxes.
+// 2-D row-major tensor [outer, inner] with a row stride in bytes and swizzled boxes.
 bool make_tmap_2d(CUtensorMap *map, CUtensorMapDataType dtype, const void *ptr, uint64_t inner,
-                  uint64_t outer, uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer)
+                  uint64_t outer, uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer,
+                  CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B)
 {
     EncodeTiledFn fn = encode_fn();
     if (!fn)
@@ -95,7 +96,7 @@ bool make_tmap_2d(CUtensorMap *map, CUtensorMapDataType dtype, const void *ptr, 
     const cuuint32_t box[2] = {box_inner, box_outer};
     const cuuint32_t estr[2] = {1, 1};
     const CUresult r = fn(map, dtype, 2, const_cast<void *>(ptr), dims, strides, box, estr,
-                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
@@ -135,10 +136,29 @@ sdnq_status validate_rotquant(const void *x, int64_t rows, int64_t K, int64_t ld
     return SDNQ_OK;
 }
 
+// Rows of at most 16 chunks go to the persistent, prefetching kernel (grid = resident
+// CTAs); longer rows to the two-pass kernel with one CTA per row.
 template <int G>
-void launch_rotquant_g(const RotquantParams &p, dim3 grid, dim3 block, cudaStream_t st)
+void launch_rotquant_g(const RotquantParams &p, dim3 grid, dim3 block, int sm_count,
+                       cudaStream_t st)
 {
-    rotquant_kernel<G><<<grid, block, 0, st>>>(p);
+    if (p.nchunks <= 16) {
+        static int per_sm[33] = {0};  // resident CTAs per SM, by warps per CTA
+        const int warps = static_cast<int>(block.x / 32);
+        if (per_sm[warps] == 0) {
+            int n = 0;
+            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, rotquant_persistent_kernel<G>,
+                                                              block.x, 0) != cudaSuccess || n < 1)
+                n = 1;
+            per_sm[warps] = n;
+        }
+        const int64_t groups = grid.x;
+        const int64_t resident = static_cast<int64_t>(per_sm[warps]) * sm_count;
+        const dim3 pgrid(static_cast<unsigned>(groups < resident ? groups : resident));
+        rotquant_persistent_kernel<G><<<pgrid, block, 0, st>>>(p);
+    } else {
+        rotquant_kernel<G><<<grid, block, 0, st>>>(p);
+    }
 }
 
 sdnq_status run_rotquant(const uint16_t *x, int64_t rows, int64_t K, int64_t ld, int32_t group,
@@ -168,12 +188,12 @@ sdnq_status run_rotquant(const uint16_t *x, int64_t rows, int64_t K, int64_t ld,
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     cudaGetLastError();
     switch (group) {
-    case 8: launch_rotquant_g<8>(p, grid, block, cs); break;
-    case 16: launch_rotquant_g<16>(p, grid, block, cs); break;
-    case 32: launch_rotquant_g<32>(p, grid, block, cs); break;
-    case 64: launch_rotquant_g<64>(p, grid, block, cs); break;
-    case 128: launch_rotquant_g<128>(p, grid, block, cs); break;
-    default: launch_rotquant_g<256>(p, grid, block, cs); break;
+    case 8: launch_rotquant_g<8>(p, grid, block, dev.sm_count, cs); break;
+    case 16: launch_rotquant_g<16>(p, grid, block, dev.sm_count, cs); break;
+    case 32: launch_rotquant_g<32>(p, grid, block, dev.sm_count, cs); break;
+    case 64: launch_rotquant_g<64>(p, grid, block, dev.sm_count, cs); break;
+    case 128: launch_rotquant_g<128>(p, grid, block, dev.sm_count, cs); break;
+    default: launch_rotquant_g<256>(p, grid, block, dev.sm_count, cs); break;
     }
     return launch_status();
 }
@@ -202,9 +222,11 @@ sdnq_status launch_gemm(const DeviceInfo &dev, const int8_t *qx, const int8_t *q
                         cudaStream_t cs)
 {
     using C = GemmConfig<BN, LORA>;
-    CUtensorMap tmA, tmB, tmU, tmL;
+    CUtensorMap tmA, tmB, tmU, tmL, tmO;
     if (!make_tmap_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, qx, p.K, p.M, p.K, 128, 128) ||
-        !make_tmap_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, qW, p.K, p.N, p.K, 128, BN))
+        !make_tmap_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, qW, p.K, p.N, p.K, 128, BN) ||
+        !make_tmap_2d(&tmO, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.out, p.N, p.M, 2ull * p.ldo, 32, 32,
+                      CU_TENSOR_MAP_SWIZZLE_64B))
         return SDNQ_ERR_CUDA;
     if (LORA) {
         if (!make_tmap_2d(&tmU, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, u, rank, p.M, 2ull * rank, 64, 128) ||
@@ -224,7 +246,7 @@ sdnq_status launch_gemm(const DeviceInfo &dev, const int8_t *qx, const int8_t *q
     p.num_tiles = p.num_m_blocks * ((p.N + BN - 1) / BN);
     const int grid = p.num_tiles < dev.sm_count ? p.num_tiles : dev.sm_count;
     cudaGetLastError();
-    gemm_s8_kernel<BN, LORA><<<grid, C::THREADS, C::SMEM_BYTES, cs>>>(tmA, tmB, tmU, tmL, p);
+    gemm_s8_kernel<BN, LORA><<<grid, C::THREADS, C::SMEM_BYTES, cs>>>(tmA, tmB, tmU, tmL, tmO, p);
     return launch_status();
 }
 

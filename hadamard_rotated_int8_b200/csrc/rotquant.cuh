@@ -31,7 +31,7 @@
 
 namespace sdnq {
 
-struct RotquantParams {
+struct RotquantParams {  // shared by both rotate+quantize kernels
     const uint16_t *x;   // [M, K] bf16 patterns, row stride ldx
     int64_t ldx;
     int8_t *q;           // [M, K] dense
@@ -54,35 +54,6 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4 r, float (&f)[8])
     f[5] = __uint_as_float(r.z & 0xffff0000u);
     f[6] = __uint_as_float(r.w << 16);
     f[7] = __uint_as_float(r.w & 0xffff0000u);
-}
-
-// Packed fp32 pairs (sm_100 f32x2 instructions): each op is two independent IEEE fp32
-// operations with round-to-nearest-even, the same results as the scalar ones.
-__device__ __forceinline__ void add2(float &d0, float &d1, float a0, float a1, float b0, float b1)
-{
-    asm("{\n\t.reg .b64 a, b, d;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
-        "add.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
-        : "=f"(d0), "=f"(d1) : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
-}
-__device__ __forceinline__ void sub2(float &d0, float &d1, float a0, float a1, float b0, float b1)
-{
-    asm("{\n\t.reg .b64 a, b, d;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
-        "sub.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
-        : "=f"(d0), "=f"(d1) : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
-}
-__device__ __forceinline__ void mul2(float &d0, float &d1, float a0, float a1, float b0, float b1)
-{
-    asm("{\n\t.reg .b64 a, b, d;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
-        "mul.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
-        : "=f"(d0), "=f"(d1) : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
-}
-// d = a * b + c with one rounding per lane
-__device__ __forceinline__ void fma2(float &d0, float &d1, float a0, float a1, float b0, float b1,
-                                     float c0, float c1)
-{
-    asm("{\n\t.reg .b64 a, b, c, d;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
-        "mov.b64 c, {%6, %7};\n\tfma.rn.f32x2 d, a, b, c;\n\tmov.b64 {%0, %1}, d;\n\t}"
-        : "=f"(d0), "=f"(d1) : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
 }
 
 // Butterfly pair (a, b) -> (a + b, a - b) on two adjacent pairs at once.
@@ -242,6 +213,74 @@ __device__ __forceinline__ void quant_store_chunk(const float (&v)[4][8], int8_t
             w = quant8(v[t], s_z, rcp, fast);
         if (ok && e < K)
             st_v2(qr + e, w.x, w.y);
+    }
+}
+
+__device__ __forceinline__ void load_raw(const uint16_t *xr, int32_t K, int32_t c, bool ok,
+                                         uint32_t lane, uint4 (&raw)[4])
+{
+    const int32_t base = c * 1024 + static_cast<int32_t>(lane >> 3) * 256 +
+                         static_cast<int32_t>(lane & 7u) * 8;
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+        const int32_t e = base + t * 64;
+        raw[t] = make_uint4(0u, 0u, 0u, 0u);
+        if (ok && e < K)
+            raw[t] = ld_nc_v4(xr + e);
+    }
+}
+
+// Rows of at most 16 chunks (K <= 16384): each warp owns one chunk of a row, a CTA owns
+// `rpc` rows at a time and walks row groups persistently, loading the next row group into
+// registers while it rotates and quantizes the current one.
+template <int G>
+__global__ void __launch_bounds__(512) rotquant_persistent_kernel(const RotquantParams p)
+{
+    __shared__ float s_amax[2][32];
+    const uint32_t lane = lane_id();
+    const int32_t warp = static_cast<int32_t>(threadIdx.x >> 5);
+    const int32_t r_local = warp / p.wpr;
+    const int32_t wr = warp - r_local * p.wpr;   // this warp's chunk of the row
+    const bool has_chunk = wr < p.nchunks;
+    const int64_t n_groups = (p.M + p.rpc - 1) / p.rpc;
+
+    int64_t rg = blockIdx.x;
+    uint4 raw[4];
+    {
+        const int64_t row = rg * p.rpc + r_local;
+        const bool ok = rg < n_groups && row < p.M && has_chunk;
+        load_raw(p.x + (ok ? row : 0) * p.ldx, p.K, wr, ok, lane, raw);
+    }
+    for (int parity = 0; rg < n_groups; rg += gridDim.x, parity ^= 1) {
+        const int64_t row = rg * p.rpc + r_local;
+        const bool row_ok = row < p.M;
+        float v[4][8];
+#pragma unroll
+        for (int t = 0; t < 4; ++t)
+            bf16x8_to_f32(raw[t], v[t]);
+        {   // prefetch the next row group while this one is computed
+            const int64_t nrg = rg + gridDim.x;
+            const int64_t nrow = nrg * p.rpc + r_local;
+            const bool ok = nrg < n_groups && nrow < p.M && has_chunk;
+            load_raw(p.x + (ok ? nrow : 0) * p.ldx, p.K, wr, ok, lane, raw);
+        }
+        chunk_butterfly<G>(v, lane);
+        float amax = chunk_absmax(v);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1)
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+        if (lane == 0)
+            s_amax[parity][warp] = amax;
+        __syncthreads();  // one barrier per row group: s_amax is double-buffered
+        amax = 0.0f;
+        for (int32_t w = 0; w < p.wpr; ++w)
+            amax = fmaxf(amax, s_amax[parity][r_local * p.wpr + w]);
+        const float s_z = __fdiv_rn(amax, 127.0f);
+        const bool zero = !(amax > 0.0f);
+        if (row_ok && wr == 0 && lane == 0)
+            p.s[row] = zero ? 0.0f : __fmul_rn(s_z, p.c_g);
+        int8_t *qr = p.q + (row_ok ? row : 0) * static_cast<int64_t>(p.K);
+        quant_store_chunk(v, qr, p.K, wr, row_ok && has_chunk, lane, s_z, zero);
     }
 }
 
