@@ -300,6 +300,20 @@ def run_reference(args):
     return 0
 
 
+def reduce_max_over_ranks(values, dist=None, world=1, device="cuda"):
+    """Element-wise max of a list of floats over all ranks (the slowest rank's times)."""
+    import torch
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t]
+
+
+def whole_job_tops(ops_per_rank, world, ms_per_step):
+    """Aggregate throughput of N replicas: every rank's work over the slowest rank's time."""
+    return world * ops_per_rank / (ms_per_step * 1e-3) / 1e12
+
+
 def config_of(case, args):
     c = {"workload": args.workload, "M": case.M, "N": case.N, "K": case.K,
          "hadamard_group": case.g, "bias": case.bias is not None,
@@ -384,17 +398,14 @@ def main():
         for j, n in enumerate(names):
             stage_ms[n] += e[j].elapsed_time(e[j + 1])
     step_ms_total = sum(stage_ms.values())
-    t = torch.tensor([step_ms_total] + [stage_ms[n] for n in names], dtype=torch.float64,
-                     device="cuda")
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    step_ms_total = float(t[0])
-    stage_ms = {n: float(t[1 + j]) for j, n in enumerate(names)}
+    t = reduce_max_over_ranks([step_ms_total] + [stage_ms[n] for n in names], dist, world)
+    step_ms_total = t[0]
+    stage_ms = {n: t[1 + j] for j, n in enumerate(names)}
     assert sd.sdnq_device_status() == 0
 
     ops, lora_flops = workload_ops(case, args.workload)
     ms_per_step = step_ms_total / args.steps
-    value = world * ops / (ms_per_step * 1e-3) / 1e12
+    value = whole_job_tops(ops, world, ms_per_step)
 
     # end to end through the public API: pinned host input -> device -> step -> host output
     e2e = None
@@ -419,10 +430,8 @@ def main():
             out_host.copy_(res, non_blocking=True)
         e1.record()
         torch.cuda.synchronize()
-        te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device="cuda")
-        if world > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
-        e2e = {"value": world * ops * n_e2e / (float(te[0]) * 1e-3) / 1e12, "unit": "TOPS",
+        te = reduce_max_over_ranks([e0.elapsed_time(e1)], dist, world)
+        e2e = {"value": whole_job_tops(ops, world, te[0] / n_e2e), "unit": "TOPS",
                "h2d_bytes_per_step": x_host.numel() * 2,
                "d2h_bytes_per_step": out_host.numel() * 2, "steps": n_e2e}
 
@@ -462,7 +471,7 @@ def main():
         "e2e": e2e,
     }
     if lora_flops:
-        line["tops_with_lora_flops"] = world * (ops + lora_flops) / (ms_per_step * 1e-3) / 1e12
+        line["tops_with_lora_flops"] = whole_job_tops(ops + lora_flops, world, ms_per_step)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(case, args.workload)
     if rank == 0:
