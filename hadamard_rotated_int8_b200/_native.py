@@ -42,6 +42,8 @@ SIGNATURES = {
     "sdnq_int8_linear": [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _I64, _P, _P],
     "sdnq_int8_linear_lora": [_P, _P, _P, _P, _P, _P, _I64, _P, _P, _I32, _F, _P, _I64, _I64,
                               _I64, _P, _I64, _P, _P],
+    "sdnq_int8_linear_lora_noalloc": [_P, _P, _P, _P, _P, _P, _I64, _P, _P, _I32, _F, _I64,
+                                      _I64, _I64, _P, _I64, _P, _P],
     "sdnq_gelu_bf16": [_P, _I64, _I64, _I64, _P, _I64, _P],
     "sdnq_device_status": [_P],
     "sdnq_selftest_wait_timeout": [_I64, _P],
@@ -195,6 +197,37 @@ def sdnq_int8_linear_lora(qx, sx, qW, sW, bias, x, A, B, lora_scale: float = 1.0
                                        float(lora_scale), _ptr(u_ws), M, N, K, _ptr(out),
                                        out.stride(0), _ptr(acc_out), _stream(stream)),
            "sdnq_int8_linear_lora")
+    return out
+
+
+NOALLOC_MAX_U_ELEMS = 1 << 22
+
+
+def sdnq_int8_linear_lora_noalloc(qx, sx, qW, sW, bias, x, A, B, lora_scale: float = 1.0,
+                                  out=None, acc_out=None, stream=None):
+    """sdnq_int8_linear_lora for callers that cannot provide device memory for the u
+    workspace: u lives in a fixed 8 MiB array inside the library (M * rank must not exceed
+    NOALLOC_MAX_U_ELEMS). Calls that overlap on the GPU share that array and race."""
+    _req(qx, torch.int8, "qx", 2)
+    _req(qW, torch.int8, "qW", 2)
+    _req(x, torch.bfloat16, "x", 2)
+    _dense(A, "A")
+    _dense(B, "B")
+    M, K = qx.shape
+    N = qW.shape[0]
+    rank = A.shape[1]
+    if A.shape[0] != K or B.shape != (rank, N) or x.shape != (M, K):
+        raise ValueError("LoRA shapes disagree")
+    if M * rank > NOALLOC_MAX_U_ELEMS:
+        raise ValueError(f"M * rank = {M * rank} exceeds the library's fixed scratch of "
+                         f"{NOALLOC_MAX_U_ELEMS} values; use sdnq_int8_linear_lora with u_ws")
+    out = _rows_out(M, N, torch.bfloat16, qx.device) if out is None else out
+    _check(lib().sdnq_int8_linear_lora_noalloc(_ptr(qx), _ptr(sx), _ptr(qW), _ptr(sW),
+                                               _ptr(bias), _ptr(x), x.stride(0), _ptr(A),
+                                               _ptr(B), rank, float(lora_scale), M, N, K,
+                                               _ptr(out), out.stride(0), _ptr(acc_out),
+                                               _stream(stream)),
+           "sdnq_int8_linear_lora_noalloc")
     return out
 
 

@@ -467,3 +467,6 @@ SDNQ_API const char *sdnq_status_string(sdnq_status s)
 }
 
 SDNQ_API const char *sdnq_version(void) { return "sdnq-b200 0.1.0 sm_100a"; }
+
+// The no-allocation LoRA variant (its own file; shares this translation unit).
+#include "lora_noalloc.cu"

@@ -128,6 +128,31 @@ sdnq_status sdnq_int8_linear_lora(const int8_t *qx, const float *sx, const int8_
                                   int32_t *acc_out, void *stream);
 
 /*
+ * sdnq_int8_linear_lora without the caller-provided workspace. The pages have no
+ * counterpart: this entry point is for callers that cannot allocate device memory for u_ws,
+ * because their host framework owns all device memory (a caching allocator or a fixed
+ * memory plan) and forbids allocations from outside it, or because a cudaMalloc, which may
+ * synchronise the device and has unpredictable latency, is not acceptable where they run.
+ * It allocates nothing: u = bf16(x A) lives in a fixed array inside the library, of
+ * SDNQ_NOALLOC_MAX_U_ELEMS bf16 values (8 MiB), held on every GPU that loads the library
+ * until the process exits. Arguments and results are those of sdnq_int8_linear_lora minus
+ * u_ws; u itself is not returned.
+ *   Limit: M * rank <= SDNQ_NOALLOC_MAX_U_ELEMS, else SDNQ_ERR_SHAPE and nothing is launched.
+ *   The first call on each device looks up the array's device address (with that device
+ *   current); make that first call before any stream capture.
+ *   Every call uses the same array, which keeps the last call's u: calls whose kernels
+ *   overlap on the GPU (different streams, or different host threads) race on it and must
+ *   be serialised by the caller. Nothing in it needs clearing between calls.
+ */
+#define SDNQ_NOALLOC_MAX_U_ELEMS (1 << 22)
+sdnq_status sdnq_int8_linear_lora_noalloc(const int8_t *qx, const float *sx, const int8_t *qW,
+                                          const float *sW, const uint16_t *bias,
+                                          const uint16_t *x, int64_t ldx, const uint16_t *A,
+                                          const uint16_t *B, int32_t rank, float lora_scale,
+                                          int64_t M, int64_t N, int64_t K, uint16_t *out,
+                                          int64_t ldo, int32_t *acc_out, void *stream);
+
+/*
  * GELU between the up and down projections of a DiT MLP (exact erf form,
  * x * Phi(x), rounded once to bf16). Not on the pages; the MLP workload needs it.
  *   in [M, N] bf16 row stride ld_in; out [M, N] bf16 row stride ld_out (may alias in when
