@@ -20,11 +20,8 @@
 // Exactness. The butterfly runs its stages in ascending order h = 1, 2, ..., G/2, each
 // element one IEEE fp32 add or subtract (packed two at a time with the f32x2 instructions,
 // which round each lane like the scalar ones). A shuffle stage computes fma(self, +-1,
-// partner), the single rounding of partner +- self. The quotient z / s_z is formed as
-// z * (1/s_z), which lies within 2.3e-5 of the IEEE quotient for |z/s_z| <= 127.5; when
-// every value of a vector lies farther than 2^-14 from a half-integer, its round-half-even
-// integer is therefore that of the IEEE quotient. Otherwise (about 3% of vectors) the whole
-// warp takes the IEEE division for that vector, so no per-element branch is needed.
+// partner), the single rounding of partner +- self. The codes use the exact IEEE quotient
+// z / s_z (see quant8), so they are those of round_half_even(fp32(z / s_z)).
 #pragma once
 
 #include "device.cuh"
@@ -170,26 +167,28 @@ __device__ __noinline__ uint2 quant8_exact(float z0, float z1, float z2, float z
     return make_uint2(pack4(c[0], c[1], c[2], c[3]), pack4(c[4], c[5], c[6], c[7]));
 }
 
-// Codes of one vector of 8 values: z * (1/s_z) rounded with the 1.5*2^23 trick; the exact
-// path runs (warp-uniformly) when any value of the warp's vector lies within 2^-14 of a
-// half-integer, or when s_z is subnormal.
+// Codes of one vector of 8 values. The IEEE quotient Q = RN(z / s_z) is obtained without a
+// division by Markstein's correction (P. Markstein, "Computation of elementary functions on
+// the IBM RISC System/6000 processor", IBM J. Res. Dev. 34(1), 1990): with y = RN(1/s_z) and
+// q0 = RN(z * y), the residual r = z - q0 * s_z is exact in one fused multiply-add and
+// RN(q0 + r * y) = RN(z / s_z). Q is then rounded half-to-even to an integer by adding
+// 1.5 * 2^23 (|Q| <= 127.5, so the integer lands in the low mantissa bits). Needs s_z normal;
+// otherwise (a row whose scale is subnormal) the IEEE division is used.
 __device__ __forceinline__ uint2 quant8(const float (&z)[8], float s_z, float rcp, bool fast)
 {
+    if (!fast)  // warp-uniform: s_z is the row's scale
+        return quant8_exact(z[0], z[1], z[2], z[3], z[4], z[5], z[6], z[7], s_z);
     constexpr float MAGIC = 12582912.0f;  // 1.5 * 2^23
+    const float neg_s = -s_z;
     float f[8];
-    float emax = 0.0f;
 #pragma unroll
     for (int i = 0; i < 8; i += 2) {
-        float p0, p1, n0, n1, e0, e1;
-        mul2(p0, p1, z[i], z[i + 1], rcp, rcp);
-        add2(f[i], f[i + 1], p0, p1, MAGIC, MAGIC);
-        sub2(n0, n1, f[i], f[i + 1], MAGIC, MAGIC);
-        sub2(e0, e1, p0, p1, n0, n1);  // exact: |p - n| <= 1/2
-        emax = fmaxf(emax, fmaxf(fabsf(e0), fabsf(e1)));
+        float q0, q1, r0, r1, c0, c1;
+        mul2(q0, q1, z[i], z[i + 1], rcp, rcp);             // q = RN(z * y)
+        fma2(r0, r1, q0, q1, neg_s, neg_s, z[i], z[i + 1]);  // r = z - q * s_z, exact
+        fma2(c0, c1, r0, r1, rcp, rcp, q0, q1);              // Q = RN(q + r * y)
+        add2(f[i], f[i + 1], c0, c1, MAGIC, MAGIC);          // M + rne(Q)
     }
-    const bool slow = !fast || !(emax < 0.5f - 0x1p-14f);
-    if (__any_sync(0xffffffffu, slow))
-        return quant8_exact(z[0], z[1], z[2], z[3], z[4], z[5], z[6], z[7], s_z);
     // the low byte of f is the code in two's complement
     return make_uint2(pack4(__float_as_uint(f[0]), __float_as_uint(f[1]), __float_as_uint(f[2]),
                             __float_as_uint(f[3])),

@@ -85,6 +85,37 @@ def test_rotquant_bit_exact(M, K, g):
     assert_equal(s.view(np.uint32), s_ref.view(np.uint32), f"scales M={M} K={K} g={g}")
 
 
+@pytest.mark.parametrize("g", [8, 64, 256])
+def test_rotquant_exact_ties_round_half_even(g):
+    """Integer rows whose rotated absmax is 127 * 2^k make s_z a power of two, so many
+    quotients z / s_z are exact half-integers: the codes must round those ties to even."""
+    rng = np.random.default_rng(g)
+    M, K = 96, 4 * max(g, 256)
+    x = rng.integers(-1, 2, size=(M, K)).astype(np.float32)
+    for r in range(M):
+        k = r % 3                       # amax = 127 * 2^(k+1) in the first group
+        target = 127 * 2 ** (k + 1)
+        x[r, :g] = 0
+        base, rem = divmod(target, g)
+        x[r, :g] = base
+        x[r, :rem] += 1
+        # a few opposite pairs keep the group sum (z_0 = target) and vary the other z
+        idx = rng.choice(g, size=min(8, g) // 2 * 2, replace=False)
+        x[r, idx[0::2]] += 1
+        x[r, idx[1::2]] -= 1
+    xb = torch.from_numpy(x).to(torch.bfloat16)
+    assert torch.equal(xb.float(), torch.from_numpy(x))  # small integers are exact in bf16
+    q, s = gpu_rotquant(xb, g)
+    q_ref, s_ref = oracle.rotate_quantize(synthetic.bits(xb), g)
+    z = oracle.fwht_f32(x, g)
+    sz = (np.abs(z).max(1) / np.float32(127)).astype(np.float32)
+    t = z / sz[:, None]
+    ties = np.count_nonzero(t - np.floor(t) == 0.5)
+    assert ties > 100, ties
+    assert_equal(q, q_ref, f"codes with exact ties g={g}")
+    assert_equal(s.view(np.uint32), s_ref.view(np.uint32), f"scales with exact ties g={g}")
+
+
 def test_rotquant_strided_input_and_weights_entry():
     case = synthetic.make_case(M=70, N=96, K=1536, g=256, seed=5, outlier_count=12,
                                outlier_factor=20.0)
