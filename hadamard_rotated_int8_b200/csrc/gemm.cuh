@@ -14,7 +14,8 @@
 //   warps 2..9  epilogue: TMEM -> registers -> scales, bias, LoRA -> bf16 -> global. A warp
 //               may only read the TMEM lanes 32*(warp % 4) .. +31, so two warps share each
 //               lane quarter and split the tile's columns in halves.
-// Two accumulator buffers in TMEM let the epilogue of tile i overlap the MMAs of tile i+1.
+// Two accumulator buffers in TMEM let the epilogue of tile i overlap the MMAs of tile i+1
+// (one buffer when a tile's accumulators fill all 512 columns, as with LoRA at N = 256).
 // Operand tiles use the 128-byte swizzle written by TMA and read by the MMA descriptors.
 //
 // Every wait is bounded (mbar_wait_bounded): on timeout the CTA raises its abort flag and
@@ -53,7 +54,8 @@ struct GemmConfig {
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
     static constexpr int STAGES = (BN == 256) ? 4 : 6;
     static constexpr int ACC_COLS = LORA ? 2 * BN : BN;   // TMEM columns per buffer
-    static constexpr int TMEM_COLS = 2 * ACC_COLS;        // two buffers
+    static constexpr int NBUF = 512 / ACC_COLS >= 2 ? 2 : 1;  // accumulator buffers
+    static constexpr int TMEM_COLS = NBUF * ACC_COLS;
     static constexpr int THREADS = 320;               // 2 + 8 warps
     static constexpr int EPI_WARPS = 8;
     static constexpr int EPI_COLS = BN / 2;           // columns per epilogue warp
@@ -108,7 +110,7 @@ __global__ void __launch_bounds__(320, 1)
             mbar_init(full_bar(s), 1);
             mbar_init(empty_bar(s), 1);
         }
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < C::NBUF; ++b) {
             mbar_init(tfull_bar(b), 1);
             mbar_init(tempty_bar(b), C::EPI_WARPS);
         }
@@ -196,8 +198,8 @@ __global__ void __launch_bounds__(320, 1)
             int local = 0;
             bool ok = true;
             for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x, ++local) {
-                const int buf = local & 1;
-                const uint32_t use = static_cast<uint32_t>(local >> 1);
+                const int buf = local % C::NBUF;
+                const uint32_t use = static_cast<uint32_t>(local / C::NBUF);
                 if (!mbar_wait_bounded(tempty_bar(buf), (use & 1u) ^ 1u, abort, p.timeout_ns)) {
                     ok = false;
                     break;
@@ -266,8 +268,8 @@ __global__ void __launch_bounds__(320, 1)
         const bool has_bias = p.bias != nullptr;
         int local = 0;
         for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++local) {
-            const int buf = local & 1;
-            const uint32_t use = static_cast<uint32_t>(local >> 1);
+            const int buf = local % C::NBUF;
+            const uint32_t use = static_cast<uint32_t>(local / C::NBUF);
             const int m0 = (tile % p.num_m_blocks) * C::BM;
             const int n0 = (tile / p.num_m_blocks) * BN;
             const int nw = n0 + col_base;     // first column of this warp

@@ -25,6 +25,12 @@ namespace {
 
 constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;  // 2 s for any single wait
 
+// Tile width of the LoRA GEMM: 128 keeps two TMEM accumulator buffers (int32 + fp32 per
+// tile), 256 uses one.
+#ifndef SDNQ_LORA_BN
+#define SDNQ_LORA_BN 256
+#endif
+
 // ---------------------------------------------------------------- device checks
 
 struct DeviceInfo {
@@ -329,7 +335,7 @@ sdnq_status run_linear(const int8_t *qx, const float *sx, const int8_t *qW, cons
     if (st != SDNQ_OK)
         return st;
     p.lora_chunks = (rank + 63) / 64;
-    return launch_gemm<128, true>(dev, qx, qW, u_ws, B, rank, p, cs);
+    return launch_gemm<SDNQ_LORA_BN, true>(dev, qx, qW, u_ws, B, rank, p, cs);
 }
 
 // ---------------------------------------------------------------- self-test kernel

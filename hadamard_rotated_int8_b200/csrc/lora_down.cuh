@@ -27,7 +27,9 @@ struct LoraDownConfig {
     static constexpr int X_BYTES = 128 * 128;             // 128 rows x 64 bf16
     static constexpr int A_BYTES = (RANK_PAD / 64) * 8192;  // boxes of 64 x 64 bf16
     static constexpr int STAGE_BYTES = X_BYTES + A_BYTES;
-    static constexpr int STAGES = 4;
+    // as many stages as fit 192 KB (8 at rank 64): the kernel streams x and has one CTA per
+    // 128 rows, so the bytes each CTA keeps in flight set its bandwidth
+    static constexpr int STAGES = (196608 / STAGE_BYTES) < 8 ? (196608 / STAGE_BYTES) : 8;
     static constexpr int TMEM_COLS = RANK_PAD < 32 ? 32 : RANK_PAD;  // power of two >= 32
     static constexpr int BAR_BYTES = (2 * STAGES + 2) * 8;
     static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES + 16;
