@@ -128,15 +128,15 @@ class Step:
             self.down = torch.empty((case.M, case.K), dtype=torch.bfloat16, device=dev)
             self.stages = [
                 ("rotquant", lambda: sd.sdnq_rotquant_act(self.x, g, self.qx, self.sx)),
-                ("gemm_up", lambda: sd.sdnq_int8_linear(self.qx, self.sx, self.qW, self.sW,
-                                                        None, out=self.out)),
-                ("gelu", lambda: sd.sdnq_gelu_bf16(self.out, out=self.h)),
+                # up-projection with GELU in its epilogue: h = bf16(GELU(bf16(up)))
+                ("gemm_up", lambda: sd.sdnq_int8_linear_gelu(self.qx, self.sx, self.qW, self.sW,
+                                                             None, out=self.h)),
                 ("rotquant_h", lambda: sd.sdnq_rotquant_act(self.h, g, self.qh, self.sh)),
                 ("gemm_down", lambda: sd.sdnq_int8_linear(self.qh, self.sh, self.qWd, self.sWd,
                                                           None, out=self.down)),
             ]
             self.gemm_stages = ["gemm_up", "gemm_down"]
-            self.launches = 5
+            self.launches = 4
         elif case.A is not None:
             self.A, self.B = case.A.to(dev), case.B.to(dev)
             self.u = torch.empty((case.M, case.A.shape[1]), dtype=torch.bfloat16, device=dev)

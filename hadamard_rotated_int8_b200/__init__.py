@@ -6,26 +6,34 @@ The compute lives in ``libsdnq.so`` (hand-written CUDA behind the C ABI of
 * ``sdnq_rotate_quant_weight``  weight rotate + row-wise int8 quantize (offline)
 * ``sdnq_rotquant_act``         online activation rotate + per-token int8 quantize
 * ``sdnq_int8_linear``          int8 x int8 -> int32 tensor-core matmul + fp32 de-quant epilogue
+* ``sdnq_int8_linear_gelu``     the same with GELU fused into the epilogue (MLP up-projection)
 * ``sdnq_int8_linear_lora``     the same plus the bf16 LoRA side term
 * ``sdnq_gelu_bf16``            exact-erf GELU (MLP glue)
 
 ``linear`` composes the online path (rotate + quantize, then the int8 linear).
 """
 from ._native import (SdnqError, lib, sdnq_device_status, sdnq_gelu_bf16, sdnq_int8_linear,
-                      sdnq_int8_linear_lora, sdnq_rotate_quant_weight, sdnq_rotquant_act,
-                      sdnq_selftest_wait_timeout, status_string, version)
+                      sdnq_int8_linear_gelu, sdnq_int8_linear_lora,
+                      sdnq_int8_linear_lora_noalloc, sdnq_rotate_quant_weight,
+                      sdnq_rotquant_act, sdnq_selftest_wait_timeout, status_string, version)
 
 __all__ = [
     "SdnqError", "lib", "linear", "sdnq_device_status", "sdnq_gelu_bf16", "sdnq_int8_linear",
-    "sdnq_int8_linear_lora", "sdnq_rotate_quant_weight", "sdnq_rotquant_act",
-    "sdnq_selftest_wait_timeout", "status_string", "version",
+    "sdnq_int8_linear_gelu", "sdnq_int8_linear_lora", "sdnq_int8_linear_lora_noalloc",
+    "sdnq_rotate_quant_weight", "sdnq_rotquant_act", "sdnq_selftest_wait_timeout",
+    "status_string", "version",
 ]
 
 
-def linear(x, qW, sW, group=256, bias=None, lora=None, out=None, stream=None):
+def linear(x, qW, sW, group=256, bias=None, lora=None, gelu=False, out=None, stream=None):
     """y = rotated-int8 linear of x [M, K] bf16 against pre-quantized weights (qW, sW).
-    ``lora`` = (A, B, lora_scale) adds the bf16 adapter term."""
+    ``lora`` = (A, B, lora_scale) adds the bf16 adapter term; ``gelu`` applies GELU to the
+    output inside the GEMM epilogue (not combined with ``lora``)."""
+    if gelu and lora is not None:
+        raise ValueError("gelu with lora is not provided")
     qx, sx = sdnq_rotquant_act(x, group, stream=stream)
+    if gelu:
+        return sdnq_int8_linear_gelu(qx, sx, qW, sW, bias, out=out, stream=stream)
     if lora is None:
         return sdnq_int8_linear(qx, sx, qW, sW, bias, out=out, stream=stream)
     A, B, scale = lora

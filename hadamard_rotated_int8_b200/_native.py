@@ -40,6 +40,7 @@ SIGNATURES = {
     "sdnq_rotate_quant_weight": [_P, _I64, _I64, _I64, _I32, _P, _P, _P],
     "sdnq_rotquant_act": [_P, _I64, _I64, _I64, _I32, _P, _P, _P],
     "sdnq_int8_linear": [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _I64, _P, _P],
+    "sdnq_int8_linear_gelu": [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _I64, _P, _P],
     "sdnq_int8_linear_lora": [_P, _P, _P, _P, _P, _P, _I64, _P, _P, _I32, _F, _P, _I64, _I64,
                               _I64, _P, _I64, _P, _P],
     "sdnq_int8_linear_lora_noalloc": [_P, _P, _P, _P, _P, _P, _I64, _P, _P, _I32, _F, _I64,
@@ -160,8 +161,7 @@ def sdnq_rotquant_act(x: torch.Tensor, group: int = 256, qx=None, sx=None, strea
     return qx, sx
 
 
-def sdnq_int8_linear(qx, sx, qW, sW, bias=None, out=None, acc_out=None, stream=None):
-    """out [M, N] bf16 = bf16(float(qx qW^T) * (sx sW^T) + bias)."""
+def _linear_call(name, qx, sx, qW, sW, bias, out, acc_out, stream):
     _req(qx, torch.int8, "qx", 2)
     _req(qW, torch.int8, "qW", 2)
     _dense(qx, "qx")
@@ -171,10 +171,19 @@ def sdnq_int8_linear(qx, sx, qW, sW, bias=None, out=None, acc_out=None, stream=N
     if qW.shape[1] != K:
         raise ValueError("qx and qW disagree on K")
     out = _rows_out(M, N, torch.bfloat16, qx.device) if out is None else out
-    _check(lib().sdnq_int8_linear(_ptr(qx), _ptr(sx), _ptr(qW), _ptr(sW), _ptr(bias), M, N, K,
-                                  _ptr(out), out.stride(0), _ptr(acc_out), _stream(stream)),
-           "sdnq_int8_linear")
+    _check(getattr(lib(), name)(_ptr(qx), _ptr(sx), _ptr(qW), _ptr(sW), _ptr(bias), M, N, K,
+                                _ptr(out), out.stride(0), _ptr(acc_out), _stream(stream)), name)
     return out
+
+
+def sdnq_int8_linear(qx, sx, qW, sW, bias=None, out=None, acc_out=None, stream=None):
+    """out [M, N] bf16 = bf16(float(qx qW^T) * (sx sW^T) + bias)."""
+    return _linear_call("sdnq_int8_linear", qx, sx, qW, sW, bias, out, acc_out, stream)
+
+
+def sdnq_int8_linear_gelu(qx, sx, qW, sW, bias=None, out=None, acc_out=None, stream=None):
+    """out [M, N] bf16 = GELU of sdnq_int8_linear's output, rounded once more to bf16."""
+    return _linear_call("sdnq_int8_linear_gelu", qx, sx, qW, sW, bias, out, acc_out, stream)
 
 
 def sdnq_int8_linear_lora(qx, sx, qW, sW, bias, x, A, B, lora_scale: float = 1.0, u_ws=None,

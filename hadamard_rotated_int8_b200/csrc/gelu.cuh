@@ -44,6 +44,14 @@ __device__ __forceinline__ uint32_t f32_to_bf16_bits_rn(float f)
     return static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(f)));
 }
 
+// fp64 evaluation, rounded once to bf16: the rare inputs the fp32 path cannot decide
+__device__ __noinline__ uint32_t gelu_bf16_bits_fp64(uint32_t xb)
+{
+    const double xd = static_cast<double>(__uint_as_float(xb << 16));
+    const double y = 0.5 * xd * erfc(-xd * 0.70710678118654752440);
+    return f64_to_bf16_bits(y);
+}
+
 __device__ __forceinline__ uint32_t gelu_bf16_bits(uint32_t xb)
 {
     const float x = __uint_as_float(xb << 16);
@@ -57,9 +65,69 @@ __device__ __forceinline__ uint32_t gelu_bf16_bits(uint32_t xb)
         if (lo == hi)
             return lo;
     }
-    const double xd = static_cast<double>(x);
-    const double y = 0.5 * xd * erfc(-xd * 0.70710678118654752440);
-    return f64_to_bf16_bits(y);
+    return gelu_bf16_bits_fp64(xb);
+}
+
+// ---- table form, for bf16 inputs produced inside another kernel (the GEMM epilogue) ----
+// A bf16 -> bf16 function has only 65536 inputs, and outside |x| in [2^-10, 16) the correctly
+// rounded GELU has a closed form:
+//   * |x| < 2^-10 (normal): GELU(x) = x/2 + x^2/sqrt(2 pi) + O(x^4) differs from x/2 (a bf16
+//     value) by a relative 0.8|x| < 2^-10.3, less than half a bf16 ulp (>= 2^-9 relative,
+//     also just below a binade boundary), so the result is x/2, exactly;
+//   * x >= 16: 1 - Phi(16) ~ 6e-58, the result is x; x <= -16: |GELU(x)| < 1e-56, far
+//     below half the smallest bf16 subnormal, the result is -0;
+//   * +-0: +-0.
+// The 3584 inputs in between (both signs, biased exponents 117..130, all 128 mantissas) go
+// through a table built with gelu_bf16_bits; subnormal, NaN and Inf inputs take
+// gelu_bf16_bits directly.
+constexpr int kGeluLutExpLo = 117;                    // 2^-10
+constexpr int kGeluLutExpHi = 130;                    // [8, 16)
+constexpr int kGeluLutHalf = (kGeluLutExpHi - kGeluLutExpLo + 1) * 128;
+constexpr int kGeluLutEntries = 2 * kGeluLutHalf;     // 3584
+constexpr int kGeluLutBytes = 2 * kGeluLutEntries;    // 7168
+
+// bf16 input pattern of table entry i
+__device__ __forceinline__ uint32_t gelu_lut_input(int i)
+{
+    const uint32_t sign = i >= kGeluLutHalf ? 1u : 0u;
+    const uint32_t r = static_cast<uint32_t>(i) - sign * kGeluLutHalf;
+    return (sign << 15) | ((kGeluLutExpLo + (r >> 7)) << 7) | (r & 127u);
+}
+
+__device__ __noinline__ uint32_t gelu_bf16_bits_rare(uint32_t b) { return gelu_bf16_bits(b); }
+
+// Table-form GELU of the 16 bf16 patterns packed in w[8] (two per word), in place; `lut`
+// is the table in shared memory. Branch-free apart from the rare inputs (subnormal, NaN,
+// Inf), so that the table loads are independent and in flight together.
+__device__ __forceinline__ void gelu_bf16x16_lut(uint32_t *w, const uint16_t *lut)
+{
+    uint32_t r[16];
+    bool rare = false;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+        const uint32_t b = (k & 1) ? (w[k >> 1] >> 16) : (w[k >> 1] & 0xffffu);
+        const uint32_t e = (b >> 7) & 0xffu;
+        const uint32_t sign = b >> 15;
+        const bool in_tab = e - kGeluLutExpLo <= static_cast<uint32_t>(kGeluLutExpHi - kGeluLutExpLo);
+        const uint32_t i = in_tab ? sign * kGeluLutHalf + ((e - kGeluLutExpLo) << 7) + (b & 127u) : 0u;
+        // outside the table: x >= 16 -> x, x <= -16 -> -0, tiny normal -> x/2, +-0 -> +-0
+        const uint32_t alt = e > kGeluLutExpHi ? (sign ? 0x8000u : b) : (e >= 2u ? b - 0x80u : b);
+        const uint32_t t = lut[i];
+        r[k] = in_tab ? t : alt;
+        rare |= e == 255u || (e < 2u && (b & 0x7fffu) != 0u);
+    }
+    if (rare) {
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            const uint32_t b = (k & 1) ? (w[k >> 1] >> 16) : (w[k >> 1] & 0xffffu);
+            const uint32_t e = (b >> 7) & 0xffu;
+            if (e == 255u || (e < 2u && (b & 0x7fffu) != 0u))
+                r[k] = gelu_bf16_bits_rare(b);
+        }
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+        w[k] = r[2 * k] | (r[2 * k + 1] << 16);
 }
 
 struct GeluParams {

@@ -2,7 +2,9 @@
 // accumulators in tensor memory), fed by TMA through a shared-memory ring, with the fp32
 // de-quant epilogue fused: out = bf16(float(acc) * (sx[m] * sw[n]) + bias[n]
 // [+ lora_scale * L[m][n]]), where L = u B is a second, bf16 x bf16 -> fp32 tensor-core
-// accumulator (the PEFT adapter beside the frozen int8 base).
+// accumulator (the PEFT adapter beside the frozen int8 base). With GELU the epilogue
+// then applies the exact-erf GELU to that bf16 value and rounds once more to bf16, which is
+// bit for bit the separate GELU pass of a DiT MLP's up-projection output.
 //
 // Sources: "SDNQ: SD.Next Quantization Engine" README, feature list (INT8 quantized matmul)
 // and SDNQConfig (dequantize_fp32: FP32 scales and FP32 de-quant steps); "ConvRot / Hadamard
@@ -26,6 +28,7 @@
 #include <cuda_bf16.h>
 
 #include "device.cuh"
+#include "gelu.cuh"
 
 namespace sdnq {
 
@@ -45,7 +48,7 @@ struct GemmParams {
     uint64_t timeout_ns;
 };
 
-template <int BN, bool LORA>
+template <int BN, bool LORA, bool GELU = false>
 struct GemmConfig {
     static constexpr int BM = 128;
     static constexpr int BK = 128;                     // bytes of K per stage (int8)
@@ -65,7 +68,9 @@ struct GemmConfig {
     static constexpr int OUT_OFF = STAGES * STAGE_BYTES;
     static constexpr int SCALE_OFF = OUT_OFF + EPI_WARPS * STAGE_OUT_BYTES;
     static constexpr int SCALE_BYTES = EPI_COLS * 8;  // sw[EPI_COLS], bias[EPI_COLS]
-    static constexpr int BAR_OFF = SCALE_OFF + EPI_WARPS * SCALE_BYTES;
+    static constexpr int LUT_OFF = SCALE_OFF + EPI_WARPS * SCALE_BYTES;  // GELU table
+    static constexpr int LUT_BYTES = GELU ? kGeluLutBytes : 0;
+    static constexpr int BAR_OFF = LUT_OFF + LUT_BYTES;
     // barriers: full[S], empty[S], tfull[2], tempty[2], drain; then tmem base + abort flag
     static constexpr int BAR_BYTES = (2 * STAGES + 5) * 8;
     static constexpr int SMEM_BYTES = 1024 /*align slack*/ + BAR_OFF + BAR_BYTES + 16;
@@ -81,13 +86,13 @@ __device__ __forceinline__ uint32_t float_to_bf16_bits(float f)
     return static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(f)));
 }
 
-template <int BN, bool LORA>
+template <int BN, bool LORA, bool GELU>
 __global__ void __launch_bounds__(320, 1)
     gemm_s8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CUtensorMap tmL,
                    const __grid_constant__ CUtensorMap tmO, const GemmParams p)
 {
-    using C = GemmConfig<BN, LORA>;
+    using C = GemmConfig<BN, LORA, GELU>;
     extern __shared__ uint8_t smem_raw[];
     // 1024-byte alignment for the 128-byte swizzle atoms
     const uint32_t raw_addr = smem_u32(smem_raw);
@@ -266,6 +271,13 @@ __global__ void __launch_bounds__(320, 1)
         const uint32_t s_sw = base + C::SCALE_OFF + ew * C::SCALE_BYTES;
         const uint32_t s_bias = s_sw + C::EPI_COLS * 4;
         const bool has_bias = p.bias != nullptr;
+        uint16_t *lut = reinterpret_cast<uint16_t *>(smem + C::LUT_OFF);
+        if constexpr (GELU) {
+            // the GELU table, while the first tile's operands load and multiply
+            for (int i = static_cast<int>(ew * 32u + lane); i < kGeluLutEntries; i += 32 * C::EPI_WARPS)
+                lut[i] = static_cast<uint16_t>(gelu_bf16_bits(gelu_lut_input(i)));
+            bar_sync_or(1, 32 * C::EPI_WARPS, false);  // epilogue warps only
+        }
         int local = 0;
         for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++local) {
             const int buf = local % C::NBUF;
@@ -325,7 +337,7 @@ __global__ void __launch_bounds__(320, 1)
                 if constexpr (LORA)
                     tmem_ld_32x32b_x32(t_row + BN + cc, lacc);
                 tmem_ld_wait();
-                // v = float(acc) * (sx * sw) [+ bias] [+ lora_scale * L], fp32 pairs
+                // v = float(acc) * (sx * sw) [+ bias] [+ lora_scale * L], each op one fp32 rounding
                 uint32_t ob[16];
 #pragma unroll
                 for (int q = 0; q < 8; ++q) {
@@ -336,21 +348,29 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
                         const int j = 4 * q + 2 * h;
-                        float t0, t1, v0, v1;
+                        // t in f32x2; the products that feed an add are scalar __fmul_rn /
+                        // __fadd_rn, never merged into a multiply-add (a mul.rn.f32x2
+                        // followed by an add.rn.f32x2 was observed to execute as one fused
+                        // multiply-add, which differs from two roundings on ties)
+                        float t0, t1;
                         mul2(t0, t1, sxm, sxm, wv[2 * h], wv[2 * h + 1]);
-                        mul2(v0, v1, __int2float_rn(static_cast<int>(acc[j])),
-                             __int2float_rn(static_cast<int>(acc[j + 1])), t0, t1);
-                        if (has_bias)
-                            add2(v0, v1, v0, v1, bv[2 * h], bv[2 * h + 1]);
+                        float v0 = __fmul_rn(__int2float_rn(static_cast<int>(acc[j])), t0);
+                        float v1 = __fmul_rn(__int2float_rn(static_cast<int>(acc[j + 1])), t1);
+                        if (has_bias) {
+                            v0 = __fadd_rn(v0, bv[2 * h]);
+                            v1 = __fadd_rn(v1, bv[2 * h + 1]);
+                        }
                         if constexpr (LORA) {
-                            float l0, l1;
-                            mul2(l0, l1, p.lora_scale, p.lora_scale, __uint_as_float(lacc[j]),
-                                 __uint_as_float(lacc[j + 1]));
-                            add2(v0, v1, v0, v1, l0, l1);
+                            v0 = __fadd_rn(v0, __fmul_rn(p.lora_scale, __uint_as_float(lacc[j])));
+                            v1 = __fadd_rn(v1, __fmul_rn(p.lora_scale, __uint_as_float(lacc[j + 1])));
                         }
                         const __nv_bfloat162 h2 = __floats2bfloat162_rn(v0, v1);
                         ob[j >> 1] = *reinterpret_cast<const uint32_t *>(&h2);
                     }
+                }
+                if constexpr (GELU) {
+                    gelu_bf16x16_lut(ob, lut);
+                    gelu_bf16x16_lut(ob + 8, lut);
                 }
                 // stage the 32 x 32 block (64-byte swizzle) and hand it to the TMA engine;
                 // rows >= M and columns >= N fall outside the tensor and are not written

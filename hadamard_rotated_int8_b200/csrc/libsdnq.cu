@@ -222,12 +222,12 @@ sdnq_status validate_linear(const void *qx, const void *sx, const void *qW, cons
     return SDNQ_OK;
 }
 
-template <int BN, bool LORA>
+template <int BN, bool LORA, bool GELU = false>
 sdnq_status launch_gemm(const DeviceInfo &dev, const int8_t *qx, const int8_t *qW,
                         const uint16_t *u, const uint16_t *B, int32_t rank, GemmParams p,
                         cudaStream_t cs)
 {
-    using C = GemmConfig<BN, LORA>;
+    using C = GemmConfig<BN, LORA, GELU>;
     CUtensorMap tmA, tmB, tmU, tmL, tmO;
     if (!make_tmap_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, qx, p.K, p.M, p.K, 128, 128) ||
         !make_tmap_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, qW, p.K, p.N, p.K, 128, BN) ||
@@ -244,7 +244,7 @@ sdnq_status launch_gemm(const DeviceInfo &dev, const int8_t *qx, const int8_t *q
     }
     static std::once_flag once;
     static bool smem_ok = false;
-    std::call_once(once, [] { smem_ok = set_smem(gemm_s8_kernel<BN, LORA>, C::SMEM_BYTES); });
+    std::call_once(once, [] { smem_ok = set_smem(gemm_s8_kernel<BN, LORA, GELU>, C::SMEM_BYTES); });
     if (!smem_ok)
         return SDNQ_ERR_CUDA;
     p.num_kb = (p.K + C::BK - 1) / C::BK;
@@ -252,7 +252,7 @@ sdnq_status launch_gemm(const DeviceInfo &dev, const int8_t *qx, const int8_t *q
     p.num_tiles = p.num_m_blocks * ((p.N + BN - 1) / BN);
     const int grid = p.num_tiles < dev.sm_count ? p.num_tiles : dev.sm_count;
     cudaGetLastError();
-    gemm_s8_kernel<BN, LORA><<<grid, C::THREADS, C::SMEM_BYTES, cs>>>(tmA, tmB, tmU, tmL, tmO, p);
+    gemm_s8_kernel<BN, LORA, GELU><<<grid, C::THREADS, C::SMEM_BYTES, cs>>>(tmA, tmB, tmU, tmL, tmO, p);
     return launch_status();
 }
 
@@ -286,7 +286,7 @@ sdnq_status run_linear(const int8_t *qx, const float *sx, const int8_t *qW, cons
                        const uint16_t *bias, const uint16_t *x, int64_t ldx, const uint16_t *A,
                        const uint16_t *B, int32_t rank, float lora_scale, uint16_t *u_ws,
                        int64_t M, int64_t N, int64_t K, uint16_t *out, int64_t ldo,
-                       int32_t *acc_out, void *stream, bool lora)
+                       int32_t *acc_out, void *stream, bool lora, bool gelu = false)
 {
     sdnq_status st = validate_linear(qx, sx, qW, sW, bias, M, N, K, out, ldo, acc_out);
     if (st != SDNQ_OK)
@@ -324,7 +324,8 @@ sdnq_status run_linear(const int8_t *qx, const float *sx, const int8_t *qW, cons
     p.lora_scale = lora_scale;
     p.timeout_ns = kDefaultTimeoutNs;
     if (!lora)
-        return launch_gemm<256, false>(dev, qx, qW, nullptr, nullptr, 0, p, cs);
+        return gelu ? launch_gemm<256, false, true>(dev, qx, qW, nullptr, nullptr, 0, p, cs)
+                    : launch_gemm<256, false>(dev, qx, qW, nullptr, nullptr, 0, p, cs);
     const int32_t Mi = static_cast<int32_t>(M), Ki = static_cast<int32_t>(K);
     if (rank <= 64)
         st = launch_lora_down<64>(x, ldx, A, rank, u_ws, Mi, Ki, cs);
@@ -378,6 +379,15 @@ SDNQ_API sdnq_status sdnq_int8_linear(const int8_t *qx, const float *sx, const i
 {
     return run_linear(qx, sx, qW, sW, bias, nullptr, 0, nullptr, nullptr, 0, 0.0f, nullptr, M, N, K,
                       out, ldo, acc_out, stream, false);
+}
+
+SDNQ_API sdnq_status sdnq_int8_linear_gelu(const int8_t *qx, const float *sx, const int8_t *qW,
+                                           const float *sW, const uint16_t *bias, int64_t M,
+                                           int64_t N, int64_t K, uint16_t *out, int64_t ldo,
+                                           int32_t *acc_out, void *stream)
+{
+    return run_linear(qx, sx, qW, sW, bias, nullptr, 0, nullptr, nullptr, 0, 0.0f, nullptr, M, N, K,
+                      out, ldo, acc_out, stream, false, true);
 }
 
 SDNQ_API sdnq_status sdnq_int8_linear_lora(const int8_t *qx, const float *sx, const int8_t *qW,

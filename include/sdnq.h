@@ -112,6 +112,20 @@ sdnq_status sdnq_int8_linear(const int8_t *qx, const float *sx, const int8_t *qW
                              void *stream);
 
 /*
+ * sdnq_int8_linear with GELU fused into its epilogue, for the up-projection of a DiT MLP
+ * whose output feeds the down-projection's rotate + quantize:
+ *   out = gelu(bf16(float(acc) * (sx * sw) [+ bias])), GELU(y) = y * Phi(y) in the exact
+ *   erf form, rounded once to bf16,
+ * i.e. bit for bit sdnq_int8_linear followed by sdnq_gelu_bf16 on its output, without the
+ * second pass over [M, N] in HBM. Arguments, layouts, alignment and errors are those of
+ * sdnq_int8_linear; acc_out (if set) receives the raw accumulators.
+ */
+sdnq_status sdnq_int8_linear_gelu(const int8_t *qx, const float *sx, const int8_t *qW,
+                                  const float *sW, const uint16_t *bias, int64_t M, int64_t N,
+                                  int64_t K, uint16_t *out, int64_t ldo, int32_t *acc_out,
+                                  void *stream);
+
+/*
  * As sdnq_int8_linear, plus the bf16 LoRA side term of PEFT training on a frozen int8
  * base ("ConvRot / Hadamard SDNQ", PEFT Behavior): out = bf16(v + lora_scale * (u B)),
  * u = bf16(x A).

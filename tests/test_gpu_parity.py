@@ -12,6 +12,7 @@ import torch
 import oracle
 import hadamard_rotated_int8_b200 as sd
 from hadamard_rotated_int8_b200 import _build, synthetic
+from tests.epilogue_ties import fma_sensitive_epilogue_inputs
 
 pytestmark = pytest.mark.gpu
 
@@ -271,6 +272,37 @@ def test_gelu_bit_exact():
     assert_equal(bits_of(out), oracle.gelu_bf16(synthetic.bits(x)), "gelu")
 
 
+def _finite_bf16_patterns():
+    b = np.arange(65536, dtype=np.uint32)
+    return b[((b >> 7) & 0xFF) != 0xFF].astype(np.uint16)  # all but NaN and Inf
+
+
+def test_gelu_exhaustive_over_finite_bf16():
+    pats = _finite_bf16_patterns()
+    x = torch.from_numpy(pats.view(np.int16)).view(torch.bfloat16).reshape(-1, 8).cuda()
+    out = sd.sdnq_gelu_bf16(x)
+    torch.cuda.synchronize()
+    assert_equal(bits_of(out).reshape(-1), oracle.gelu_bf16(pats), "gelu, every finite bf16 input")
+
+
+def test_linear_gelu_epilogue_exhaustive_over_finite_bf16():
+    """Zero codes make the pre-GELU value exactly the bias, so a bias holding every finite
+    bf16 pattern drives the epilogue's GELU (its table and its closed-form ranges) through
+    all of them."""
+    pats = _finite_bf16_patterns()
+    N, K = len(pats), 16
+    qx = torch.zeros((3, K), dtype=torch.int8, device="cuda")
+    qW = torch.zeros((N, K), dtype=torch.int8, device="cuda")
+    sx = torch.ones(3, dtype=torch.float32, device="cuda")
+    sW = torch.ones(N, dtype=torch.float32, device="cuda")
+    bias = torch.from_numpy(pats.view(np.int16)).view(torch.bfloat16).cuda()
+    out = sd.sdnq_int8_linear_gelu(qx, sx, qW, sW, bias)
+    torch.cuda.synchronize()
+    want = oracle.gelu_bf16(oracle.dequant_epilogue(np.zeros((3, N), np.int32), np.ones(3, np.float32),
+                                                    np.ones(N, np.float32), bias_bits=pats))
+    assert_equal(bits_of(out), want, "fused GELU, every finite bf16 pre-activation")
+
+
 def test_gelu_ragged_and_strided():
     x = (torch.randn(37, 133 + 11, generator=torch.Generator().manual_seed(3)) * 4).to(torch.bfloat16)
     wide = x.cuda()
@@ -278,6 +310,52 @@ def test_gelu_ragged_and_strided():
     assert src.stride(0) == 144
     out = sd.sdnq_gelu_bf16(src)
     assert_equal(bits_of(out), oracle.gelu_bf16(synthetic.bits(x[:, :133].contiguous())), "gelu ragged")
+
+
+@pytest.mark.parametrize("gelu", [False, True])
+def test_epilogue_rounds_twice_on_fma_sensitive_ties(gelu):
+    """The de-quant epilogue rounds (float(acc) * t) and (v + bias) separately, as the oracle
+    does; an accidental multiply-add contraction shows up on these inputs (diagonal)."""
+    a1, a2, sx, sw, bias = fma_sensitive_epilogue_inputs()
+    H, K = len(a1), 16
+    qx = np.zeros((H, K), np.int8)
+    qW = np.zeros((H, K), np.int8)
+    qx[:, 0] = a1
+    qW[:, 0] = a2
+    acc = oracle.gemm_s8(qx, qW)
+    want = oracle.dequant_epilogue(acc, sx, sw, bias_bits=bias)
+    if gelu:
+        want = oracle.gelu_bf16(want)
+    fn = sd.sdnq_int8_linear_gelu if gelu else sd.sdnq_int8_linear
+    out = fn(torch.from_numpy(qx).cuda(), torch.from_numpy(sx).cuda(), torch.from_numpy(qW).cuda(),
+             torch.from_numpy(sw).cuda(), torch.from_numpy(bias.view(np.int16)).cuda().view(torch.bfloat16))
+    torch.cuda.synchronize()
+    got = bits_of(out)
+    assert_equal(np.diagonal(got), np.diagonal(want), "tie-sensitive diagonal")
+    assert_equal(got, want, "all outputs")
+
+
+@pytest.mark.parametrize("M,N,K,g,w_std", [(128, 256, 256, 256, 0.02), (300, 520, 768, 256, 0.2),
+                                            (257, 136, 1024, 128, 1.0), (513, 1000, 3840, 256, 0.015)])
+def test_linear_gelu_epilogue_bit_exact(M, N, K, g, w_std):
+    """GELU fused into the GEMM epilogue equals the oracle's linear followed by its GELU, and
+    the library's own two-pass chain, bit for bit. The larger weight scales push outputs past
+    |y| = 10 and near bf16 rounding boundaries, where the fp64 path decides."""
+    case = synthetic.make_case(M=M, N=N, K=K, g=g, seed=M + N + K, dist="student_t",
+                               w_std=w_std, bias_std=0.05)
+    xg = case.x.cuda()
+    qW, sW = sd.sdnq_rotate_quant_weight(case.W.cuda(), g)
+    qx, sx = sd.sdnq_rotquant_act(xg, g)
+    bias = case.bias.cuda()
+    acc = torch.empty((M, N), dtype=torch.int32, device="cuda")
+    fused = sd.sdnq_int8_linear_gelu(qx, sx, qW, sW, bias, acc_out=acc)
+    two_pass = sd.sdnq_gelu_bf16(sd.sdnq_int8_linear(qx, sx, qW, sW, bias))
+    torch.cuda.synchronize()
+    ref = oracle.linear(synthetic.bits(case.x), *oracle.rotate_quantize(synthetic.bits(case.W), g),
+                        g, bias_bits=synthetic.bits(case.bias))
+    assert_equal(acc.cpu().numpy(), ref["acc"], "int32 accumulators (GELU kernel)")
+    assert_equal(bits_of(fused), oracle.gelu_bf16(ref["out"]), "fused GELU outputs")
+    assert_equal(bits_of(fused), bits_of(two_pass), "fused against two-pass GELU")
 
 
 # ------------------------------------------------------------------ failure detection

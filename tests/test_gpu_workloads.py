@@ -102,7 +102,8 @@ def test_workload_parity(name, g):
 
 def test_dit_mlp_chain_parity():
     """Up projection -> GELU -> per-token requantisation -> down projection, on the MLP
-    workload; the oracle runs the same chain from x for sampled tokens."""
+    workload; the oracle runs the same chain from x for sampled tokens, and the fused
+    up-projection + GELU equals the two-pass chain on every element."""
     case = synthetic.workload("dit_mlp_4608x3840x10240")
     g = case.g
     W_down = case.extra["W_down"]
@@ -112,6 +113,7 @@ def test_dit_mlp_chain_parity():
     qx, sx = sd.sdnq_rotquant_act(xg, g)
     up = sd.sdnq_int8_linear(qx, sx, qWu, sWu)
     h = sd.sdnq_gelu_bf16(up)
+    h_fused = sd.sdnq_int8_linear_gelu(qx, sx, qWu, sWu)  # the step's fused up-projection
     qh, sh = sd.sdnq_rotquant_act(h, g)
     down = sd.sdnq_int8_linear(qh, sh, qWd, sWd)
     torch.cuda.synchronize()
@@ -127,6 +129,7 @@ def test_dit_mlp_chain_parity():
     down_r = oracle.dequant_epilogue(oracle.gemm_s8(qh_r, qWd_r), sh_r, sWd_r)
     assert_equal(bits_of(up)[rows], up_r, "up projection")
     assert_equal(bits_of(h)[rows], h_r, "gelu")
+    assert_equal(bits_of(h_fused), bits_of(h), "GELU fused into the up-projection epilogue")
     assert_equal(qh.cpu().numpy()[rows], qh_r, "requantised codes")
     assert_equal(sh.cpu().numpy()[rows].view(np.uint32), sh_r.view(np.uint32), "requantised scales")
     assert_equal(bits_of(down)[rows], down_r, "down projection")

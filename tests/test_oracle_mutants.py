@@ -33,6 +33,10 @@ MUTANTS = {
         "float t = sx[m] * sw[n];\n            float v = (float)acc[m * N + n] * t;",
         "float v = ((float)acc[m * N + n] * sx[m]) * sw[n];",
         [lambda: pins.test_epilogue_within_one_ulp_of_fp64_and_op_order()]),
+    "epilogue bias add fused into a multiply-add": (
+        "v = v + bf16_bits_to_f32(bias[n]);",
+        "v = fmaf((float)acc[m * N + n], t, bf16_bits_to_f32(bias[n]));",
+        [lambda: pins.test_epilogue_rounds_twice_not_fused()]),
     "bias dropped": (
         "v = v + bf16_bits_to_f32(bias[n]);", "v = v;",
         [lambda: pins.test_golden_worked_epilogue()]),

@@ -330,6 +330,30 @@ def test_golden_worked_epilogue():
     assert bf16_value(out).tolist() == d["out"]
 
 
+def test_epilogue_rounds_twice_not_fused():
+    """The pages ask for the de-quant steps in fp32; the reading is one IEEE rounding per
+    operation (no fused multiply-add). On inputs where that is visible after the bf16
+    rounding, the oracle's outputs are those of the two roundings and not of the fma."""
+    from tests.epilogue_ties import fma_sensitive_epilogue_inputs
+    a1, a2, sx, sw, bias = fma_sensitive_epilogue_inputs(count=64)
+    acc = (a1 * a2).astype(np.int32).reshape(8, 8)
+    sx2 = np.ascontiguousarray(sx.reshape(8, 8))
+    sw2 = np.ascontiguousarray(sw.reshape(8, 8))
+    b2 = np.ascontiguousarray(bias.reshape(8, 8))
+    for r in range(8):  # one output row per call: element (r, n) pairs sx2[r, n] with sw2[r, n]
+        for n in range(8):
+            out = oracle.dequant_epilogue(acc[r:r + 1, n:n + 1], sx2[r, n:n + 1], sw2[r, n:n + 1],
+                                          b2[r, n:n + 1])
+            t = np.float32(sx2[r, n]) * np.float32(sw2[r, n])
+            v = np.float32(acc[r, n]) * t
+            two = v + bf16_value(b2[r, n:n + 1])[0]
+            fused = np.float32(np.float64(acc[r, n]) * np.float64(t) +
+                               np.float64(bf16_value(b2[r, n:n + 1])[0]))
+            assert bf16_bits_from_f32(np.array([two], np.float32))[0] != \
+                bf16_bits_from_f32(np.array([fused], np.float32))[0]
+            assert out[0, 0] == bf16_bits_from_f32(np.array([two], np.float32))[0]
+
+
 def test_epilogue_within_one_ulp_of_fp64_and_op_order():
     """Against an fp64 recompute from the same codes and scales: every output within one
     bf16 ulp; the fp32 op order (s_x*s_w first, no fused multiply-add) is checked by a
