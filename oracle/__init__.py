@@ -66,6 +66,9 @@ def _open(path: str):
         "oracle_lora_down": [P, I64, I64, I64, P, I64, P, INT],
         "oracle_lora_up": [P, P, I64, I64, I64, P, INT],
         "oracle_gelu_bf16": [P, I64, P, INT],
+        "oracle_colscale_quantize": [P, I64, I64, I64, P, P, P, INT],
+        "oracle_gemm_s8_nn": [P, P, I64, I64, I64, P, INT],
+        "oracle_grad_input_epilogue": [P, P, I64, I64, I64, P, INT],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -270,3 +273,55 @@ def linear(x_bits, qw, sw, g, bias_bits=None, A_bits=None, B_bits=None, lora_sca
         res["L"] = L
     res["out"] = dequant_epilogue(acc, sx, sw, bias_bits, L, lora_scale, nthreads)
     return res
+
+
+# ---- input gradient through the frozen rotated base ----------------------------------
+
+def colscale_quantize(dy_bits, sw, nthreads: int | None = None):
+    """Per-row int8 quantization of dy * sw (sw [N] multiplies column n). Returns (codes
+    int8 [rows, N], scales fp32 [rows])."""
+    dy_bits = _c(dy_bits, np.uint16)
+    sw = _c(sw, np.float32)
+    rows, N = dy_bits.shape
+    if sw.shape != (N,):
+        raise ValueError("sw must have one scale per column")
+    q = np.empty((rows, N), np.int8)
+    s = np.empty((rows,), np.float32)
+    _check(_load().oracle_colscale_quantize(_ptr(dy_bits), rows, N, N, _ptr(sw), _ptr(q),
+                                            _ptr(s), nthreads or default_threads()),
+           "colscale_quantize")
+    return q, s
+
+
+def gemm_s8_nn(a, b, nthreads: int | None = None) -> np.ndarray:
+    """acc[m, k] = sum_n a[m, n] * b[n, k] in int32."""
+    a = _c(a, np.int8)
+    b = _c(b, np.int8)
+    M, N = a.shape
+    N2, K = b.shape
+    if N != N2:
+        raise ValueError("N mismatch")
+    acc = np.empty((M, K), np.int32)
+    _check(_load().oracle_gemm_s8_nn(_ptr(a), _ptr(b), M, N, K, _ptr(acc),
+                                     nthreads or default_threads()), "gemm_s8_nn")
+    return acc
+
+
+def grad_input_epilogue(acc, s, g, nthreads: int | None = None) -> np.ndarray:
+    """bf16 patterns of fp32(acc * s[m]), rotated back by the butterfly, times 1/sqrt(g)."""
+    acc = _c(acc, np.int32)
+    s = _c(s, np.float32)
+    M, K = acc.shape
+    dx = np.empty((M, K), np.uint16)
+    _check(_load().oracle_grad_input_epilogue(_ptr(acc), _ptr(s), M, K, g, _ptr(dx),
+                                              nthreads or default_threads()),
+           "grad_input_epilogue")
+    return dx
+
+
+def grad_input(dy_bits, qw, sw, g, nthreads: int | None = None):
+    """dx of the frozen rotated int8 layer for output gradients dy [M, N] (bf16 patterns),
+    given its stored codes qw [N, K] and row scales sw [N]. Returns every intermediate."""
+    qg, sg = colscale_quantize(dy_bits, sw, nthreads)
+    acc = gemm_s8_nn(qg, qw, nthreads)
+    return {"qg": qg, "sg": sg, "acc": acc, "dx": grad_input_epilogue(acc, sg, g, nthreads)}

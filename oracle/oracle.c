@@ -39,6 +39,9 @@
  *    Behavior).
  *  - GELU (MLP glue between the up and down projections): exact erf form
  *    x * Phi(x) = 0.5 * x * erfc(-x / sqrt(2)) in fp64, rounded once to bf16.
+ *  - Input gradient of the frozen base: dy * sW quantized per token (no rotation on that
+ *    operand), int8 matmul against the stored codes, then v = fp32(acc) * s, the fp32
+ *    butterfly, times fp32(1/sqrt(g)), bf16_rne.
  */
 #include <math.h>
 #include <stdint.h>
@@ -314,4 +317,104 @@ int oracle_gelu_bf16(const uint16_t *in, int64_t n, uint16_t *out, int nthreads)
         out[i] = f64_to_bf16_rne(y);
     }
     return ORACLE_OK;
+}
+
+/* ---- Input gradient through the frozen rotated int8 base ----
+ * [SD] quantized training example (the quantized matmul runs on the forward and on the
+ * backward pass); [CR] PEFT Behavior (the base is frozen under bf16 adapters, so the only
+ * gradient it passes on is the one with respect to its input).
+ * The weight the layer holds is W_hat = W_rot H with W_rot[n][k] = sW[n] * qW[n][k] (the
+ * rotated, normalised rows) and H the normalised block-diagonal Hadamard matrix, which is
+ * symmetric and its own inverse. So dx = dy W_hat = ((dy * sW) qW) H, computed in three
+ * steps: a per-token int8 quantization of dy * sW (sW varies along the contraction, so it is
+ * folded into dy before the integer matmul), the int8 matmul against the stored codes qW
+ * read as [N][K], and an epilogue that applies the row scale, the butterfly and 1/sqrt(g). */
+
+/* Step 1: c[m][n] = fp32(dy[m][n]) * sw[n]; amax over the row; s = amax / 127;
+ * codes rne(c / s) clamped to [-127, 127]; stored scale s. dy row stride ld. */
+int oracle_colscale_quantize(const uint16_t *dy, int64_t rows, int64_t N, int64_t ld,
+                             const float *sw, int8_t *q, float *s, int nthreads)
+{
+    if (!dy || !sw || !q || !s || rows < 0 || N <= 0 || ld < N)
+        return ORACLE_ERR_ARG;
+    int err = 0;
+#pragma omp parallel for num_threads(nthreads > 0 ? nthreads : 1) schedule(static)
+    for (int64_t r = 0; r < rows; r++) {
+        float *c = (float *)malloc((size_t)N * sizeof(float));
+        if (!c) {
+#pragma omp atomic write
+            err = 1;
+            continue;
+        }
+        float amax = 0.0f;
+        for (int64_t n = 0; n < N; n++) {
+            c[n] = bf16_bits_to_f32(dy[r * ld + n]) * sw[n];
+            float a = fabsf(c[n]);
+            if (a > amax)
+                amax = a;
+        }
+        const float s_c = amax / 127.0f;
+        for (int64_t n = 0; n < N; n++) {
+            int code = 0;
+            if (amax != 0.0f) {
+                float n_ = nearbyintf(c[n] / s_c);
+                if (n_ > 127.0f)
+                    n_ = 127.0f;
+                if (n_ < -127.0f)
+                    n_ = -127.0f;
+                code = (n_ == n_) ? (int)n_ : 0;
+            }
+            q[r * N + n] = (int8_t)code;
+        }
+        s[r] = s_c;
+        free(c);
+    }
+    return err ? ORACLE_ERR_NOMEM : ORACLE_OK;
+}
+
+/* Step 2: acc[m][k] = sum_n a[m][n] * b[n][k] in int32; a [M][N] and b [N][K] dense. */
+int oracle_gemm_s8_nn(const int8_t *a, const int8_t *b, int64_t M, int64_t N, int64_t K,
+                      int32_t *acc, int nthreads)
+{
+    if (!a || !b || !acc || M < 0 || N <= 0 || K < 0)
+        return ORACLE_ERR_ARG;
+#pragma omp parallel for num_threads(nthreads > 0 ? nthreads : 1) schedule(static)
+    for (int64_t m = 0; m < M; m++) {
+        for (int64_t k = 0; k < K; k++) {
+            int32_t sum = 0;
+            for (int64_t n = 0; n < N; n++)
+                sum += (int32_t)a[m * N + n] * (int32_t)b[n * K + k];
+            acc[m * K + k] = sum;
+        }
+    }
+    return ORACLE_OK;
+}
+
+/* Step 3: v[m][k] = fp32(acc[m][k]) * s[m]; the fp32 butterfly of each group of g columns
+ * (ascending stages, as in the forward rotation); dx[m][k] = bf16_rne(z[k] * c_g) with
+ * c_g = fp32(1/sqrt(g)). */
+int oracle_grad_input_epilogue(const int32_t *acc, const float *s, int64_t M, int64_t K,
+                               int64_t g, uint16_t *dx, int nthreads)
+{
+    if (!acc || !s || !dx || M < 0 || K <= 0 || !is_pow2(g) || K % g != 0)
+        return ORACLE_ERR_ARG;
+    const float c_g = (float)(1.0 / sqrt((double)g));
+    int err = 0;
+#pragma omp parallel for num_threads(nthreads > 0 ? nthreads : 1) schedule(static)
+    for (int64_t m = 0; m < M; m++) {
+        float *z = (float *)malloc((size_t)K * sizeof(float));
+        if (!z) {
+#pragma omp atomic write
+            err = 1;
+            continue;
+        }
+        for (int64_t k = 0; k < K; k++)
+            z[k] = (float)acc[m * K + k] * s[m];
+        for (int64_t k0 = 0; k0 < K; k0 += g)
+            fwht_group_f32(z + k0, g);
+        for (int64_t k = 0; k < K; k++)
+            dx[m * K + k] = f32_to_bf16_rne(z[k] * c_g);
+        free(z);
+    }
+    return err ? ORACLE_ERR_NOMEM : ORACLE_OK;
 }

@@ -53,6 +53,20 @@ MUTANTS = {
     "lora B transposed": (
         "(double)bf16_bits_to_f32(B[j * N + n]);", "(double)bf16_bits_to_f32(B[n * rank + j]);",
         [lambda: pins.test_lora_down_and_up_against_fp64_products()]),
+    "backward: column scale not folded into dy": (
+        "c[n] = bf16_bits_to_f32(dy[r * ld + n]) * sw[n];", "c[n] = bf16_bits_to_f32(dy[r * ld + n]);",
+        [lambda: pins.test_grad_input_exact_case_against_explicit_hadamard(64)]),
+    "backward: weight codes read transposed": (
+        "sum += (int32_t)a[m * N + n] * (int32_t)b[n * K + k];",
+        "sum += (int32_t)a[m * N + n] * (int32_t)b[k * N + n];",
+        [lambda: pins.test_gemm_nn_matches_numpy_int64()]),
+    "backward: rotation not undone": (
+        "            fwht_group_f32(z + k0, g);\n        for (int64_t k = 0; k < K; k++)\n            dx[",
+        "            (void)k0;\n        for (int64_t k = 0; k < K; k++)\n            dx[",
+        [lambda: pins.test_grad_input_exact_case_against_explicit_hadamard(256)]),
+    "backward: 1/sqrt(g) dropped": (
+        "dx[m * K + k] = f32_to_bf16_rne(z[k] * c_g);", "dx[m * K + k] = f32_to_bf16_rne(z[k]);",
+        [lambda: pins.test_grad_input_exact_case_against_explicit_hadamard(256)]),
 }
 
 

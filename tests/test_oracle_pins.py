@@ -442,3 +442,118 @@ def test_gelu_against_scipy_normal_cdf_and_special_values():
     assert g[0] == 0 and bf16_value(g[1:2])[0] == 50.0
     assert g[2] == 0x8000  # -50 * Phi(-50) underflows to -0
     assert bf16_value(g[3:4])[0] == np.float32(1.953125)  # 2*Phi(2)=1.9545 -> bf16 1.953125
+
+
+# ---------------------------------------------------------------- input gradient (backward)
+
+def _exact_grad_case(g, M=6, N=48, groups=2, seed=0):
+    """Inputs on which every step of the input-gradient path is exact: codes Q with +-127 in
+    every row, power-of-two row scales S and column scales sw, dy = Q S / sw (exact in bf16:
+    |Q| < 128 has at most 7 significant bits), weight codes in [-7, 7] so that the butterfly
+    of the accumulators stays below 2^24."""
+    rng = np.random.default_rng(seed)
+    K = g * groups
+    Q = rng.integers(-127, 128, size=(M, N))
+    Q[np.arange(M), rng.integers(0, N, M)] = 127 * rng.choice([-1, 1], M)
+    e_row = rng.integers(3, 9, M)                       # S = 2^-e_row
+    e_col = rng.integers(2, 7, N)                       # sw = 2^-e_col
+    sw = np.ldexp(1.0, -e_col).astype(np.float32)
+    dy = np.ldexp(Q.astype(np.float64), (e_col[None, :] - e_row[:, None]))
+    dyb = bf16_bits_from_f32(dy.astype(np.float32))
+    assert np.array_equal(bf16_value(dyb).astype(np.float64), dy)
+    qw = rng.integers(-7, 8, size=(N, K)).astype(np.int8)
+    return Q, e_row, sw, dyb, qw
+
+
+@pytest.mark.parametrize("g", [8, 64, 128, 256])
+def test_grad_input_exact_case_against_explicit_hadamard(g):
+    """dx = ((dy * sw) qw) H_g / sqrt(g) with the explicit Sylvester matrix, in exact integer
+    arithmetic, rounded once to bf16; the oracle's codes and scales are the constructed ones."""
+    Q, e_row, sw, dyb, qw = _exact_grad_case(g, seed=g)
+    res = oracle.grad_input(dyb, qw, sw, g)
+    assert np.array_equal(res["qg"], Q.astype(np.int8))
+    assert np.array_equal(res["sg"], np.ldexp(1.0, -e_row).astype(np.float32))
+    M, K = Q.shape[0], qw.shape[1]
+    acc = Q.astype(np.int64) @ qw.astype(np.int64)
+    H = sylvester(g)
+    rot = (acc.reshape(M, K // g, g) @ H).reshape(M, K)       # H symmetric
+    assert np.abs(rot).max() < 2 ** 24
+    if g in (64, 256):
+        exact = np.ldexp(rot.astype(np.float64), -e_row[:, None]) / math.sqrt(g)
+        assert np.array_equal(res["dx"], oracle.f64_to_bf16(exact))
+    else:
+        # 1/sqrt(g) is not a power of two: the oracle rounds z * fp32(1/sqrt(g)) in fp32
+        c_g = np.float32(1.0 / math.sqrt(g))
+        z = np.ldexp(rot.astype(np.float64), -e_row[:, None]).astype(np.float32)
+        assert np.array_equal(res["dx"], bf16_bits_from_f32(z * c_g))
+
+
+def test_colscale_quantize_with_unit_scales_is_textbook_per_row_int8():
+    """sw = 1 reduces the backward quantizer to plain per-row absmax int8 (the g = 1 case of
+    the forward quantizer, itself pinned against the textbook formula)."""
+    rng = np.random.default_rng(11)
+    dyb = bf16_bits_from_f32((rng.standard_normal((37, 200)) * 0.01).astype(np.float32))
+    q, s = oracle.colscale_quantize(dyb, np.ones(200, np.float32))
+    q1, s1 = oracle.rotate_quantize(dyb, 1)
+    assert np.array_equal(q, q1) and np.array_equal(s, s1)
+
+
+def test_colscale_quantize_brute_force_codes():
+    """Every code is the nearest grid point to fp32(fp32(dy * sw) / fp32(amax / 127)), ties to
+    even, over rows that include a zero row."""
+    rng = np.random.default_rng(12)
+    dy = (rng.standard_normal((12, 24)) * 0.3).astype(np.float32)
+    dy[5] = 0.0
+    dyb = bf16_bits_from_f32(dy)
+    sw = (rng.random(24) * 0.01 + 1e-4).astype(np.float32)
+    q, s = oracle.colscale_quantize(dyb, sw)
+    c = (bf16_value(dyb) * sw[None, :]).astype(np.float32)
+    for r in range(12):
+        amax = np.float32(np.abs(c[r]).max())
+        if amax == 0:
+            assert s[r] == 0 and np.all(q[r] == 0)
+            continue
+        sz = np.float32(amax / np.float32(127.0))
+        assert s[r] == sz
+        for n in range(24):
+            assert q[r, n] == _ties_even_nearest(np.float32(c[r, n] / sz))
+
+
+def test_gemm_nn_matches_numpy_int64():
+    rng = np.random.default_rng(13)
+    a = rng.integers(-127, 128, size=(9, 70), dtype=np.int8)
+    b = rng.integers(-127, 128, size=(70, 33), dtype=np.int8)
+    assert np.array_equal(oracle.gemm_s8_nn(a, b).astype(np.int64),
+                          a.astype(np.int64) @ b.astype(np.int64))
+
+
+@pytest.mark.parametrize("g", [64, 256])
+def test_grad_input_is_the_chain_rule_of_the_dequantized_layer(g):
+    """Against fp64 dy W_hat, with W_hat = diag(sw) qw H_g / sqrt(g) the weight the layer
+    holds: the error is bounded by the int8 quantization of dy * sw (half a step per
+    element, carried through |qw H|/sqrt(g)), plus one bf16 ulp and fp32 rounding."""
+    rng = np.random.default_rng(g)
+    M, N, K = 16, 96, 2 * g
+    case = synthetic.make_case(M=N, N=1, K=K, g=g, seed=g)
+    qw, sw = oracle.rotate_quantize(synthetic.bits(case.x), g)   # a weight's codes
+    dyb = bf16_bits_from_f32((rng.standard_normal((M, N)) * 0.05).astype(np.float32))
+    res = oracle.grad_input(dyb, qw, sw, g)
+    H = sylvester(g).astype(np.float64) / math.sqrt(g)
+    Hb = np.kron(np.eye(K // g), H)
+    w_hat = (sw.astype(np.float64)[:, None] * qw.astype(np.float64)) @ Hb
+    ref = bf16_value(dyb).astype(np.float64) @ w_hat
+    got = bf16_value(res["dx"]).astype(np.float64)
+    qstep = res["sg"].astype(np.float64)[:, None] / 2.0
+    spread = np.abs(qw.astype(np.float64) @ Hb).sum(0)[None, :]
+    bound = qstep * spread + np.abs(ref) * 2.0 ** -7 + 2.0 ** -20 * np.abs(got) * g + 1e-30
+    assert np.all(np.abs(got - ref) <= bound)
+
+
+def test_grad_input_zero_gradient_row():
+    rng = np.random.default_rng(14)
+    dy = (rng.standard_normal((4, 32)) * 0.1).astype(np.float32)
+    dy[2] = 0.0
+    qw = rng.integers(-127, 128, size=(32, 256), dtype=np.int8)
+    res = oracle.grad_input(bf16_bits_from_f32(dy), qw, np.full(32, 0.01, np.float32), 256)
+    assert res["sg"][2] == 0 and np.all(res["qg"][2] == 0)
+    assert np.all(bf16_value(res["dx"][2]) == 0)
