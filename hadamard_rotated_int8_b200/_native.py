@@ -41,6 +41,8 @@ SIGNATURES = {
     "sdnq_rotquant_act": [_P, _I64, _I64, _I64, _I32, _P, _P, _P],
     "sdnq_int8_linear": [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _I64, _P, _P],
     "sdnq_int8_linear_gelu": [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _I64, _P, _P],
+    "sdnq_int8_linear_grad_input": [_P, _I64, _P, _P, _I64, _I64, _I64, _I32, _P, _P, _P, _I64,
+                                    _P, _P],
     "sdnq_int8_linear_lora": [_P, _P, _P, _P, _P, _P, _I64, _P, _P, _I32, _F, _P, _I64, _I64,
                               _I64, _P, _I64, _P, _P],
     "sdnq_int8_linear_lora_noalloc": [_P, _P, _P, _P, _P, _P, _I64, _P, _P, _I32, _F, _I64,
@@ -184,6 +186,28 @@ def sdnq_int8_linear(qx, sx, qW, sW, bias=None, out=None, acc_out=None, stream=N
 def sdnq_int8_linear_gelu(qx, sx, qW, sW, bias=None, out=None, acc_out=None, stream=None):
     """out [M, N] bf16 = GELU of sdnq_int8_linear's output, rounded once more to bf16."""
     return _linear_call("sdnq_int8_linear_gelu", qx, sx, qW, sW, bias, out, acc_out, stream)
+
+
+def sdnq_int8_linear_grad_input(dy, qW, sW, group: int, qg_ws=None, sg_ws=None, out=None,
+                                acc_out=None, stream=None):
+    """dx [M, K] bf16 of the frozen rotated int8 layer (qW [N, K], sW [N]) for output
+    gradients dy [M, N] bf16. qg_ws [M, N] int8 / sg_ws [M] fp32 receive the quantized dy * sW."""
+    _req(dy, torch.bfloat16, "dy", 2)
+    _req(qW, torch.int8, "qW", 2)
+    _dense(qW, "qW")
+    M, N = dy.shape
+    if qW.shape[0] != N:
+        raise ValueError("dy and qW disagree on N")
+    K = qW.shape[1]
+    dev = dy.device
+    qg_ws = torch.empty((M, N), dtype=torch.int8, device=dev) if qg_ws is None else qg_ws
+    sg_ws = torch.empty((M,), dtype=torch.float32, device=dev) if sg_ws is None else sg_ws
+    out = _rows_out(M, K, torch.bfloat16, dev) if out is None else out
+    _check(lib().sdnq_int8_linear_grad_input(_ptr(dy), dy.stride(0), _ptr(qW), _ptr(sW), M, N, K,
+                                             group, _ptr(qg_ws), _ptr(sg_ws), _ptr(out),
+                                             out.stride(0), _ptr(acc_out), _stream(stream)),
+           "sdnq_int8_linear_grad_input")
+    return out
 
 
 def sdnq_int8_linear_lora(qx, sx, qW, sW, bias, x, A, B, lora_scale: float = 1.0, u_ws=None,

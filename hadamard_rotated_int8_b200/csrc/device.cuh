@@ -310,9 +310,46 @@ __device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)
                  : "r"(taddr));
 }
 
+// Same, 4 columns.
+__device__ __forceinline__ void tmem_ld_32x32b_x4(uint32_t taddr, uint32_t (&r)[4])
+{
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(taddr));
+}
+
 __device__ __forceinline__ void tmem_ld_wait()
 {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Each thread of the warp writes 32 consecutive 32-bit columns of its own TMEM lane.
+__device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const uint32_t (&r)[32])
+{
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x32.b32 [%0],"
+                 " {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16,"
+                 " %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};"
+                 ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]),
+                   "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]),
+                   "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]),
+                   "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]),
+                   "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]),
+                   "r"(r[30]), "r"(r[31])
+                 : "memory");
+}
+
+// Same, 4 columns.
+__device__ __forceinline__ void tmem_st_32x32b_x4(uint32_t taddr, const uint32_t (&r)[4])
+{
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};"
+                 ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3])
+                 : "memory");
+}
+
+// This thread's tcgen05.st writes have completed.
+__device__ __forceinline__ void tmem_st_wait()
+{
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
 // ---------------------------------------------------------------------------------------
@@ -339,8 +376,8 @@ __device__ __forceinline__ uint64_t kmajor_desc(uint32_t saddr)
     return smem_desc_sw128(saddr, 16u, 1024u);
 }
 
-// MN-major 16-bit operand: atoms of 64 MN-elements (128 bytes) x 8 K-rows; K-row groups of
-// 8 are 1024 bytes apart, MN atoms are `mn_atom_stride` bytes apart.
+// MN-major operand: atoms of 128 bytes of MN (64 16-bit or 128 8-bit elements) x 8 K-rows;
+// K-row groups of 8 are 1024 bytes apart, MN atoms are `mn_atom_stride` bytes apart.
 __device__ __forceinline__ uint64_t mnmajor_desc(uint32_t saddr, uint32_t mn_atom_stride)
 {
     return smem_desc_sw128(saddr, mn_atom_stride, 1024u);
@@ -350,10 +387,10 @@ __device__ __forceinline__ uint64_t mnmajor_desc(uint32_t saddr, uint32_t mn_ato
 //   bits 4-5 accumulator format (1 = f32, 2 = s32); bits 7-9 / 10-12 A / B format
 //   (kind::i8: 1 = signed; kind::f16: 1 = bf16); bit 15 / 16 A / B major (0 = K, 1 = MN);
 //   bits 17-22 N >> 3; bits 24-28 M >> 4.
-__host__ __device__ constexpr uint32_t idesc_s8_s32(int M, int N)
+__host__ __device__ constexpr uint32_t idesc_s8_s32(int M, int N, bool b_mn_major = false)
 {
-    return (2u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
-           (static_cast<uint32_t>(M >> 4) << 24);
+    return (2u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) |
+           (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn_major)

@@ -45,6 +45,7 @@ struct GemmParams {
     int32_t num_tiles;
     int32_t lora_chunks;      // ceil(rank / 64); 0 without LoRA
     float lora_scale;
+    float c_g;                // input-gradient mode: fp32(1/sqrt(g))
     uint64_t timeout_ns;
 };
 
@@ -86,13 +87,190 @@ __device__ __forceinline__ uint32_t float_to_bf16_bits(float f)
     return static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(f)));
 }
 
-template <int BN, bool LORA, bool GELU>
+// One output block: 16 packed bf16 pairs (32 columns) of this thread's row go through the
+// warp's 64-byte-swizzled staging buffer to a TMA store of the warp's 32 x 32 block at
+// (column nc, row mrow0); rows >= M and columns >= N fall outside the tensor and are dropped.
+__device__ __forceinline__ void store_block(const uint32_t (&ob)[16], uint32_t s_out, uint32_t lane,
+                                            const CUtensorMap *tmO, int nc, int mrow0)
+{
+    if (lane == 0)
+        bulk_wait_read_all();  // the previous block has left the staging buffer
+    __syncwarp();
+    const uint32_t row_addr = s_out + lane * 64u;
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+        sts_v4(row_addr + ((static_cast<uint32_t>(q) ^ ((lane >> 1) & 3u)) << 4), ob[4 * q],
+               ob[4 * q + 1], ob[4 * q + 2], ob[4 * q + 3]);
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+        tma_store_2d(tmO, s_out, nc, mrow0);
+        bulk_commit_group();
+    }
+}
+
+// ---- input-gradient epilogue: dx = bf16(FWHT_G(fp32(acc) * s_g) * fp32(1/sqrt(G))) ----
+
+// Butterfly stages h = 1 .. GA/2 over 32 consecutive columns held in registers. Stage 1 adds
+// products, so it uses scalar adds (an f32x2 add fed by a product may be merged with it
+// into a multiply-add); the later stages add sums and use f32x2 pairs.
+template <int GA>
+__device__ __forceinline__ void butterfly32(float (&v)[32])
+{
+    if (GA > 1) {
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+            const float a = v[i], b = v[i + 1];
+            v[i] = __fadd_rn(a, b);
+            v[i + 1] = __fsub_rn(a, b);
+        }
+    }
+#pragma unroll
+    for (int h = 2; h < GA; h <<= 1) {
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+            if ((i & h) == 0) {
+                float s0, s1, d0, d1;
+                add2(s0, s1, v[i], v[i + 1], v[i + h], v[i + h + 1]);
+                sub2(d0, d1, v[i], v[i + 1], v[i + h], v[i + h + 1]);
+                v[i] = s0; v[i + 1] = s1; v[i + h] = d0; v[i + h + 1] = d1;
+            }
+        }
+    }
+}
+
+__device__ __forceinline__ void pack_scaled_bf16(const float (&z)[32], float c_g, uint32_t (&ob)[16])
+{
+#pragma unroll
+    for (int i = 0; i < 32; i += 2) {
+        float a, b;
+        mul2(a, b, z[i], z[i + 1], c_g, c_g);  // feeds no add
+        const __nv_bfloat162 h2 = __floats2bfloat162_rn(a, b);
+        ob[i >> 1] = *reinterpret_cast<const uint32_t *>(&h2);
+    }
+}
+
+// One 128 x 256 accumulator tile; this warp owns TMEM lanes 32*quad.. (one row per thread)
+// and, in passes 1 and 3, the columns [128*half, 128*half + 128). Groups of G columns never
+// straddle tiles (G divides 256) and never straddle N (N % G == 0).
+//   pass 1: v = fp32(acc) * s_g and the stages h < 32 inside each 32-column load (for
+//           G <= 32 that is the whole transform and the block goes straight out);
+//   pass 2: stages h = 32 .. G/2 across the 32-column blocks, 4 columns of every block at a
+//           time, the warp pair splitting the columns; results go back to TMEM;
+//   pass 3: times 1/sqrt(G), bf16, TMA store.
+// Passes exchange columns with the partner warp through TMEM: each ends with wait::st and a
+// barrier of the pair (named barrier `pair_bar`, 64 threads).
+template <int G>
+__device__ __forceinline__ void grad_epilogue_tile(uint32_t t_row, int half, int n0, int N,
+                                                   int mrow0, float sg, float c_g, uint32_t lane,
+                                                   uint32_t pair_bar, uint32_t s_out,
+                                                   const CUtensorMap *tmO, int32_t *acc_row)
+{
+    constexpr int GA = G < 32 ? G : 32;
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+        const int cc = half * 128 + c * 32;
+        if (n0 + cc >= N)
+            break;  // warp-uniform
+        uint32_t a[32];
+        tmem_ld_32x32b_x32(t_row + cc, a);
+        tmem_ld_wait();
+        if (acc_row != nullptr) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+                if (n0 + cc + j < N)
+                    acc_row[n0 + cc + j] = static_cast<int32_t>(a[j]);
+        }
+        float v[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+            v[i] = __fmul_rn(__int2float_rn(static_cast<int>(a[i])), sg);
+        butterfly32<GA>(v);
+        if constexpr (G <= 32) {
+            uint32_t ob[16];
+            pack_scaled_bf16(v, c_g, ob);
+            store_block(ob, s_out, lane, tmO, n0 + cc, mrow0);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+                a[i] = __float_as_uint(v[i]);
+            tmem_st_32x32b_x32(t_row + cc, a);
+        }
+    }
+    if constexpr (G > 32) {
+        tmem_st_wait();
+        tc_fence_before_sync();
+        bar_sync_or(pair_bar, 64, false);
+        tc_fence_after_sync();
+#pragma unroll 1
+        for (int jb = 0; jb < 4; ++jb) {
+            const int j0 = half * 16 + jb * 4;
+            uint32_t r[8][4];
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+                tmem_ld_32x32b_x4(t_row + c * 32 + j0, r[c]);
+            tmem_ld_wait();
+            float w[8][4];
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    w[c][j] = __uint_as_float(r[c][j]);
+#pragma unroll
+            for (int d = 1; 32 * d < G; d <<= 1) {
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    if ((c & d) == 0) {
+#pragma unroll
+                        for (int j = 0; j < 4; j += 2) {
+                            float s0, s1, d0, d1;
+                            add2(s0, s1, w[c][j], w[c][j + 1], w[c + d][j], w[c + d][j + 1]);
+                            sub2(d0, d1, w[c][j], w[c][j + 1], w[c + d][j], w[c + d][j + 1]);
+                            w[c][j] = s0; w[c][j + 1] = s1; w[c + d][j] = d0; w[c + d][j + 1] = d1;
+                        }
+                    }
+                }
+            }
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    r[c][j] = __float_as_uint(w[c][j]);
+                tmem_st_32x32b_x4(t_row + c * 32 + j0, r[c]);
+            }
+        }
+        tmem_st_wait();
+        tc_fence_before_sync();
+        bar_sync_or(pair_bar, 64, false);
+        tc_fence_after_sync();
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+            const int cc = half * 128 + c * 32;
+            if (n0 + cc >= N)
+                break;
+            uint32_t a[32];
+            tmem_ld_32x32b_x32(t_row + cc, a);
+            tmem_ld_wait();
+            float z[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+                z[i] = __uint_as_float(a[i]);
+            uint32_t ob[16];
+            pack_scaled_bf16(z, c_g, ob);
+            store_block(ob, s_out, lane, tmO, n0 + cc, mrow0);
+        }
+    }
+}
+
+template <int BN, bool LORA, bool GELU, int GRAD_G>
 __global__ void __launch_bounds__(320, 1)
     gemm_s8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CUtensorMap tmL,
                    const __grid_constant__ CUtensorMap tmO, const GemmParams p)
 {
     using C = GemmConfig<BN, LORA, GELU>;
+    static_assert(GRAD_G == 0 || (BN == 256 && !LORA && !GELU && 256 % GRAD_G == 0),
+                  "input-gradient mode: plain tiles of 256 columns, G divides 256");
     extern __shared__ uint8_t smem_raw[];
     // 1024-byte alignment for the 128-byte swizzle atoms
     const uint32_t raw_addr = smem_u32(smem_raw);
@@ -160,7 +338,14 @@ __global__ void __launch_bounds__(320, 1)
                     if (!LORA || kb < p.num_kb) {
                         mbar_arrive_expect_tx(full_bar(stage), C::STAGE_BYTES);
                         tma_load_2d(sa, &tmA, full_bar(stage), kb * C::BK, m0);
-                        tma_load_2d(sb, &tmB, full_bar(stage), kb * C::BK, n0);
+                        if constexpr (GRAD_G > 0) {
+                            // B = qW rows kb*128.. (the contraction) x columns n0.. (N-major),
+                            // as two 128-column boxes
+                            tma_load_2d(sb, &tmB, full_bar(stage), n0, kb * C::BK);
+                            tma_load_2d(sb + 16384, &tmB, full_bar(stage), n0 + 128, kb * C::BK);
+                        } else {
+                            tma_load_2d(sb, &tmB, full_bar(stage), kb * C::BK, n0);
+                        }
                     } else {
                         // LoRA chunk c: U [128 x 64] bf16 (K-major) into the A slot and
                         // B [64 x BN] bf16 (N-major) as BN/64 boxes into the B slot
@@ -196,7 +381,7 @@ __global__ void __launch_bounds__(320, 1)
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            constexpr uint32_t IDESC_I8 = idesc_s8_s32(128, BN);
+            constexpr uint32_t IDESC_I8 = idesc_s8_s32(128, BN, GRAD_G > 0);
             constexpr uint32_t IDESC_BF = idesc_bf16_f32(128, BN, true);
             int stage = 0;
             uint32_t phase = 0;
@@ -220,9 +405,14 @@ __global__ void __launch_bounds__(320, 1)
                     const uint32_t sa = base + stage * C::STAGE_BYTES;
                     const uint32_t sb = sa + C::A_BYTES;
 #pragma unroll
-                    for (int k = 0; k < C::BK / 32; ++k)
-                        mma_s8(d_acc, kmajor_desc(sa + 32 * k), kmajor_desc(sb + 32 * k), IDESC_I8,
+                    for (int k = 0; k < C::BK / 32; ++k) {
+                        // K = 32 per MMA: 32 bytes along A's swizzled rows; for the N-major B
+                        // of the input gradient, 32 K-rows of 128 bytes = 4096 bytes
+                        const uint64_t bdesc = GRAD_G > 0 ? mnmajor_desc(sb + 4096 * k, 16384)
+                                                          : kmajor_desc(sb + 32 * k);
+                        mma_s8(d_acc, kmajor_desc(sa + 32 * k), bdesc, IDESC_I8,
                                (kb | k) != 0 ? 1u : 0u);
+                    }
                     tc_commit(empty_bar(stage));
                     if (++stage == C::STAGES) {
                         stage = 0;
@@ -288,7 +478,7 @@ __global__ void __launch_bounds__(320, 1)
             // this warp's column scales and bias -> shared memory (fp32), before the wait
             // on the accumulator so that their latency overlaps the MMAs
 #pragma unroll
-            for (int j = static_cast<int>(lane) * 4; j < C::EPI_COLS; j += 128) {
+            for (int j = static_cast<int>(lane) * 4; GRAD_G == 0 && j < C::EPI_COLS; j += 128) {
                 float w4[4], b4[4];
                 if (nw + j + 4 <= p.N) {
                     const float4 f = __ldg(reinterpret_cast<const float4 *>(p.sw + nw + j));
@@ -318,15 +508,28 @@ __global__ void __launch_bounds__(320, 1)
             __syncwarp();
             // warp-uniform decision: tcgen05.ld below needs the whole warp converged
             const bool ready = mbar_wait_bounded(tfull_bar(buf), use & 1u, abort, p.timeout_ns);
-            if (!__all_sync(0xffffffffu, ready))
-                break;
+            if constexpr (GRAD_G > 0) {
+                // the warp pair leaves together: it meets at named barriers inside the tile
+                if (bar_sync_or(2u + quad, 64, !__all_sync(0xffffffffu, ready)))
+                    break;
+            } else {
+                if (!__all_sync(0xffffffffu, ready))
+                    break;
+            }
             tc_fence_after_sync();
             const int m = m0 + row_in_tile;
             const bool row_ok = m < p.M;
             const float sxm = row_ok ? p.sx[m] : 0.0f;
             const uint32_t t_row = tmem_base + ((quad * 32u) << 16) + buf * C::ACC_COLS;
+            if constexpr (GRAD_G > 0) {
+                int32_t *acc_row = (p.acc_out != nullptr && row_ok)
+                                       ? p.acc_out + static_cast<int64_t>(m) * p.N : nullptr;
+                grad_epilogue_tile<GRAD_G>(t_row, static_cast<int>(ew >> 2), n0, p.N,
+                                           m0 + static_cast<int>(quad * 32u), sxm, p.c_g, lane,
+                                           2u + quad, s_out, &tmO, acc_row);
+            }
 #pragma unroll 1
-            for (int c = 0; c < C::EPI_COLS; c += 32) {
+            for (int c = 0; GRAD_G == 0 && c < C::EPI_COLS; c += 32) {
                 const int cc = col_base + c;   // column inside the tile
                 const int nc = n0 + cc;
                 if (nc >= p.N)
@@ -372,22 +575,7 @@ __global__ void __launch_bounds__(320, 1)
                     gelu_bf16x16_lut(ob, lut);
                     gelu_bf16x16_lut(ob + 8, lut);
                 }
-                // stage the 32 x 32 block (64-byte swizzle) and hand it to the TMA engine;
-                // rows >= M and columns >= N fall outside the tensor and are not written
-                if (lane == 0)
-                    bulk_wait_read_all();  // the previous block has left the staging buffer
-                __syncwarp();
-                const uint32_t row_addr = s_out + lane * 64u;
-#pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    sts_v4(row_addr + ((static_cast<uint32_t>(q) ^ ((lane >> 1) & 3u)) << 4), ob[4 * q],
-                           ob[4 * q + 1], ob[4 * q + 2], ob[4 * q + 3]);
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) {
-                    tma_store_2d(&tmO, s_out, nc, m0 + static_cast<int>(quad * 32u));
-                    bulk_commit_group();
-                }
+                store_block(ob, s_out, lane, &tmO, nc, m0 + static_cast<int>(quad * 32u));
                 if (p.acc_out != nullptr && row_ok) {
                     int32_t *arow = p.acc_out + static_cast<int64_t>(m) * p.N;
 #pragma unroll

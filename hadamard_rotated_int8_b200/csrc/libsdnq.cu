@@ -144,7 +144,7 @@ sdnq_status validate_rotquant(const void *x, int64_t rows, int64_t K, int64_t ld
 
 // Rows of at most 16 chunks go to the persistent, prefetching kernel (grid = resident
 // CTAs); longer rows to the two-pass kernel with one CTA per row.
-template <int G>
+template <int G, bool COLSCALE = false>
 void launch_rotquant_g(const RotquantParams &p, dim3 grid, dim3 block, int sm_count,
                        cudaStream_t st)
 {
@@ -153,18 +153,52 @@ void launch_rotquant_g(const RotquantParams &p, dim3 grid, dim3 block, int sm_co
         const int warps = static_cast<int>(block.x / 32);
         if (per_sm[warps] == 0) {
             int n = 0;
-            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, rotquant_persistent_kernel<G>,
-                                                              block.x, 0) != cudaSuccess || n < 1)
+            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+                    &n, rotquant_persistent_kernel<G, COLSCALE>, block.x, 0) != cudaSuccess ||
+                n < 1)
                 n = 1;
             per_sm[warps] = n;
         }
         const int64_t groups = grid.x;
         const int64_t resident = static_cast<int64_t>(per_sm[warps]) * sm_count;
         const dim3 pgrid(static_cast<unsigned>(groups < resident ? groups : resident));
-        rotquant_persistent_kernel<G><<<pgrid, block, 0, st>>>(p);
+        rotquant_persistent_kernel<G, COLSCALE><<<pgrid, block, 0, st>>>(p);
     } else {
-        rotquant_kernel<G><<<grid, block, 0, st>>>(p);
+        rotquant_kernel<G, COLSCALE><<<grid, block, 0, st>>>(p);
     }
+}
+
+// Per-row int8 quantization of rows x [rows, K] (validated by the caller): rotated by the
+// block-diagonal Hadamard of `group` columns, or (group 1) multiplied by colscale[K].
+sdnq_status launch_rowquant(const uint16_t *x, int64_t rows, int64_t K, int64_t ld,
+                            int32_t group, const float *colscale, int8_t *q, float *s,
+                            const DeviceInfo &dev, cudaStream_t cs)
+{
+    RotquantParams p;
+    p.x = x;
+    p.ldx = ld;
+    p.q = q;
+    p.s = s;
+    p.M = rows;
+    p.K = static_cast<int32_t>(K);
+    p.nchunks = static_cast<int32_t>((K + 1023) / 1024);
+    p.wpr = p.nchunks < 16 ? p.nchunks : 16;  // <= 512 threads per CTA
+    p.rpc = p.wpr <= 8 ? 8 / p.wpr : 1;
+    p.c_g = static_cast<float>(1.0 / std::sqrt(static_cast<double>(group)));
+    p.colscale = colscale;
+    const dim3 block(32 * p.wpr * p.rpc);
+    const dim3 grid(static_cast<unsigned>((rows + p.rpc - 1) / p.rpc));
+    cudaGetLastError();
+    switch (group) {
+    case 1: launch_rotquant_g<1, true>(p, grid, block, dev.sm_count, cs); break;
+    case 8: launch_rotquant_g<8>(p, grid, block, dev.sm_count, cs); break;
+    case 16: launch_rotquant_g<16>(p, grid, block, dev.sm_count, cs); break;
+    case 32: launch_rotquant_g<32>(p, grid, block, dev.sm_count, cs); break;
+    case 64: launch_rotquant_g<64>(p, grid, block, dev.sm_count, cs); break;
+    case 128: launch_rotquant_g<128>(p, grid, block, dev.sm_count, cs); break;
+    default: launch_rotquant_g<256>(p, grid, block, dev.sm_count, cs); break;
+    }
+    return launch_status();
 }
 
 sdnq_status run_rotquant(const uint16_t *x, int64_t rows, int64_t K, int64_t ld, int32_t group,
@@ -178,30 +212,8 @@ sdnq_status run_rotquant(const uint16_t *x, int64_t rows, int64_t K, int64_t ld,
         return st;
     if (rows == 0)
         return SDNQ_OK;
-    RotquantParams p;
-    p.x = x;
-    p.ldx = ld;
-    p.q = q;
-    p.s = s;
-    p.M = rows;
-    p.K = static_cast<int32_t>(K);
-    p.nchunks = static_cast<int32_t>((K + 1023) / 1024);
-    p.wpr = p.nchunks < 16 ? p.nchunks : 16;  // <= 512 threads per CTA
-    p.rpc = p.wpr <= 8 ? 8 / p.wpr : 1;
-    p.c_g = static_cast<float>(1.0 / std::sqrt(static_cast<double>(group)));
-    const dim3 block(32 * p.wpr * p.rpc);
-    const dim3 grid(static_cast<unsigned>((rows + p.rpc - 1) / p.rpc));
-    cudaStream_t cs = static_cast<cudaStream_t>(stream);
-    cudaGetLastError();
-    switch (group) {
-    case 8: launch_rotquant_g<8>(p, grid, block, dev.sm_count, cs); break;
-    case 16: launch_rotquant_g<16>(p, grid, block, dev.sm_count, cs); break;
-    case 32: launch_rotquant_g<32>(p, grid, block, dev.sm_count, cs); break;
-    case 64: launch_rotquant_g<64>(p, grid, block, dev.sm_count, cs); break;
-    case 128: launch_rotquant_g<128>(p, grid, block, dev.sm_count, cs); break;
-    default: launch_rotquant_g<256>(p, grid, block, dev.sm_count, cs); break;
-    }
-    return launch_status();
+    return launch_rowquant(x, rows, K, ld, group, nullptr, q, s, dev,
+                           static_cast<cudaStream_t>(stream));
 }
 
 // ---------------------------------------------------------------- int8 linear (+ LoRA)
@@ -222,15 +234,19 @@ sdnq_status validate_linear(const void *qx, const void *sx, const void *qW, cons
     return SDNQ_OK;
 }
 
-template <int BN, bool LORA, bool GELU = false>
+// GRAD_G > 0: the input gradient's NN product, out [M, N] = epilogue(A [M, K] x W [K, N]),
+// with W = the weight codes qW [N_out = K rows, K_in = N columns] read N-major.
+template <int BN, bool LORA, bool GELU = false, int GRAD_G = 0>
 sdnq_status launch_gemm(const DeviceInfo &dev, const int8_t *qx, const int8_t *qW,
                         const uint16_t *u, const uint16_t *B, int32_t rank, GemmParams p,
                         cudaStream_t cs)
 {
     using C = GemmConfig<BN, LORA, GELU>;
     CUtensorMap tmA, tmB, tmU, tmL, tmO;
-    if (!make_tmap_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, qx, p.K, p.M, p.K, 128, 128) ||
-        !make_tmap_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, qW, p.K, p.N, p.K, 128, BN) ||
+    const bool b_ok = GRAD_G > 0
+                          ? make_tmap_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, qW, p.N, p.K, p.N, 128, 128)
+                          : make_tmap_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, qW, p.K, p.N, p.K, 128, BN);
+    if (!make_tmap_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, qx, p.K, p.M, p.K, 128, 128) || !b_ok ||
         !make_tmap_2d(&tmO, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.out, p.N, p.M, 2ull * p.ldo, 32, 32,
                       CU_TENSOR_MAP_SWIZZLE_64B))
         return SDNQ_ERR_CUDA;
@@ -244,7 +260,7 @@ sdnq_status launch_gemm(const DeviceInfo &dev, const int8_t *qx, const int8_t *q
     }
     static std::once_flag once;
     static bool smem_ok = false;
-    std::call_once(once, [] { smem_ok = set_smem(gemm_s8_kernel<BN, LORA, GELU>, C::SMEM_BYTES); });
+    std::call_once(once, [] { smem_ok = set_smem(gemm_s8_kernel<BN, LORA, GELU, GRAD_G>, C::SMEM_BYTES); });
     if (!smem_ok)
         return SDNQ_ERR_CUDA;
     p.num_kb = (p.K + C::BK - 1) / C::BK;
@@ -252,7 +268,7 @@ sdnq_status launch_gemm(const DeviceInfo &dev, const int8_t *qx, const int8_t *q
     p.num_tiles = p.num_m_blocks * ((p.N + BN - 1) / BN);
     const int grid = p.num_tiles < dev.sm_count ? p.num_tiles : dev.sm_count;
     cudaGetLastError();
-    gemm_s8_kernel<BN, LORA, GELU><<<grid, C::THREADS, C::SMEM_BYTES, cs>>>(tmA, tmB, tmU, tmL, tmO, p);
+    gemm_s8_kernel<BN, LORA, GELU, GRAD_G><<<grid, C::THREADS, C::SMEM_BYTES, cs>>>(tmA, tmB, tmU, tmL, tmO, p);
     return launch_status();
 }
 
@@ -322,6 +338,7 @@ sdnq_status run_linear(const int8_t *qx, const float *sx, const int8_t *qW, cons
     p.K = static_cast<int32_t>(K);
     p.lora_chunks = 0;
     p.lora_scale = lora_scale;
+    p.c_g = 1.0f;
     p.timeout_ns = kDefaultTimeoutNs;
     if (!lora)
         return gelu ? launch_gemm<256, false, true>(dev, qx, qW, nullptr, nullptr, 0, p, cs)
@@ -337,6 +354,62 @@ sdnq_status run_linear(const int8_t *qx, const float *sx, const int8_t *qW, cons
         return st;
     p.lora_chunks = (rank + 63) / 64;
     return launch_gemm<SDNQ_LORA_BN, true>(dev, qx, qW, u_ws, B, rank, p, cs);
+}
+
+// ---------------------------------------------------------------- input gradient
+
+// dx = dy W_hat through the frozen rotated base: q_g, s_g = per-token int8 of dy * sW
+// (into the caller's workspace), then the NN int8 product q_g qW with the row scale,
+// inverse rotation and 1/sqrt(g) in the epilogue.
+sdnq_status run_grad_input(const uint16_t *dy, int64_t lddy, const int8_t *qW, const float *sW,
+                           int64_t M, int64_t N, int64_t K, int32_t group, int8_t *qg_ws,
+                           float *sg_ws, uint16_t *dx, int64_t lddx, int32_t *acc_out,
+                           void *stream)
+{
+    if (!qW || !sW || (M != 0 && (!dy || !qg_ws || !sg_ws || !dx)))
+        return SDNQ_ERR_NULL;
+    if (M < 0 || M > INT32_MAX || N < 16 || N > SDNQ_MAX_K || N % 16 != 0 || K < 16 ||
+        K > INT32_MAX || K % 16 != 0 || lddy < N || lddx < K)
+        return SDNQ_ERR_SHAPE;
+    if (!is_pow2(group) || group < SDNQ_MIN_GROUP || group > SDNQ_MAX_GROUP)
+        return SDNQ_ERR_UNSUPPORTED;
+    if (K % group != 0)
+        return SDNQ_ERR_SHAPE;
+    if (lddy % 8 != 0 || lddx % 8 != 0 || !aligned(dy, 16) || !aligned(qW, 16) ||
+        !aligned(sW, 16) || !aligned(qg_ws, 16) || !aligned(sg_ws, 4) || !aligned(dx, 16) ||
+        (acc_out && !aligned(acc_out, 16)))
+        return SDNQ_ERR_ALIGN;
+    DeviceInfo dev;
+    sdnq_status st = current_device(&dev);
+    if (st != SDNQ_OK)
+        return st;
+    if (M == 0)
+        return SDNQ_OK;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    if ((st = launch_rowquant(dy, M, N, lddy, 1, sW, qg_ws, sg_ws, dev, cs)) != SDNQ_OK)
+        return st;
+    GemmParams p;
+    p.sx = sg_ws;
+    p.sw = sW;          // not read in this mode
+    p.bias = nullptr;
+    p.out = dx;
+    p.ldo = lddx;
+    p.acc_out = acc_out;
+    p.M = static_cast<int32_t>(M);
+    p.N = static_cast<int32_t>(K);   // output columns: the layer's input features
+    p.K = static_cast<int32_t>(N);   // contraction: the layer's output features
+    p.lora_chunks = 0;
+    p.lora_scale = 0.0f;
+    p.c_g = static_cast<float>(1.0 / std::sqrt(static_cast<double>(group)));
+    p.timeout_ns = kDefaultTimeoutNs;
+    switch (group) {
+    case 8: return launch_gemm<256, false, false, 8>(dev, qg_ws, qW, nullptr, nullptr, 0, p, cs);
+    case 16: return launch_gemm<256, false, false, 16>(dev, qg_ws, qW, nullptr, nullptr, 0, p, cs);
+    case 32: return launch_gemm<256, false, false, 32>(dev, qg_ws, qW, nullptr, nullptr, 0, p, cs);
+    case 64: return launch_gemm<256, false, false, 64>(dev, qg_ws, qW, nullptr, nullptr, 0, p, cs);
+    case 128: return launch_gemm<256, false, false, 128>(dev, qg_ws, qW, nullptr, nullptr, 0, p, cs);
+    default: return launch_gemm<256, false, false, 256>(dev, qg_ws, qW, nullptr, nullptr, 0, p, cs);
+    }
 }
 
 // ---------------------------------------------------------------- self-test kernel
@@ -388,6 +461,16 @@ SDNQ_API sdnq_status sdnq_int8_linear_gelu(const int8_t *qx, const float *sx, co
 {
     return run_linear(qx, sx, qW, sW, bias, nullptr, 0, nullptr, nullptr, 0, 0.0f, nullptr, M, N, K,
                       out, ldo, acc_out, stream, false, true);
+}
+
+SDNQ_API sdnq_status sdnq_int8_linear_grad_input(const uint16_t *dy, int64_t lddy,
+                                                 const int8_t *qW, const float *sW, int64_t M,
+                                                 int64_t N, int64_t K, int32_t group,
+                                                 int8_t *qg_ws, float *sg_ws, uint16_t *dx,
+                                                 int64_t lddx, int32_t *acc_out, void *stream)
+{
+    return run_grad_input(dy, lddy, qW, sW, M, N, K, group, qg_ws, sg_ws, dx, lddx, acc_out,
+                          stream);
 }
 
 SDNQ_API sdnq_status sdnq_int8_linear_lora(const int8_t *qx, const float *sx, const int8_t *qW,

@@ -1,6 +1,8 @@
 // Fused online rotate + quantize: per row (token or weight row), a block-diagonal
 // Walsh-Hadamard butterfly over groups of G columns, the full-row absmax, the fp32 scale and
-// round-half-to-even int8 codes, in one pass over HBM.
+// round-half-to-even int8 codes, in one pass over HBM. With G = 1 and a column multiplier
+// (COLSCALE) the same kernels quantize dy * sW per token for the input gradient of the frozen
+// base (no rotation on that operand).
 //
 // Sources: "SDNQ: SD.Next Quantization Engine" README (Hadamard rotations on both the
 // quantized weights and the quantized matmul; row-wise scales, FP32 de-quant); "ConvRot /
@@ -38,7 +40,8 @@ struct RotquantParams {  // shared by both rotate+quantize kernels
     int32_t nchunks;     // ceil(K / 1024)
     int32_t wpr;         // warps per row
     int32_t rpc;         // rows per CTA
-    float c_g;           // fp32(1/sqrt(G))
+    float c_g;           // fp32(1/sqrt(G)); 1 without rotation
+    const float *colscale;  // [K] column multipliers, or nullptr
 };
 
 __device__ __forceinline__ void bf16x8_to_f32(const uint4 r, float (&f)[8])
@@ -69,11 +72,13 @@ __device__ __forceinline__ void chunk_butterfly(float (&v)[4][8], uint32_t lane)
 #pragma unroll
     for (int t = 0; t < 4; ++t) {
         // stage h = 1: the two halves of each loaded 32-bit word
+        if (G > 1) {
 #pragma unroll
-        for (int i = 0; i < 8; i += 2) {
-            const float a = v[t][i], b = v[t][i + 1];
-            v[t][i] = __fadd_rn(a, b);
-            v[t][i + 1] = __fsub_rn(a, b);
+            for (int i = 0; i < 8; i += 2) {
+                const float a = v[t][i], b = v[t][i + 1];
+                v[t][i] = __fadd_rn(a, b);
+                v[t][i + 1] = __fsub_rn(a, b);
+            }
         }
         // stage h = 2: (0,1)+-(2,3), (4,5)+-(6,7)
         if (G > 2) {
@@ -134,6 +139,29 @@ __device__ __forceinline__ void load_chunk(const uint16_t *xr, int32_t K, int32_
 #pragma unroll
     for (int t = 0; t < 4; ++t)
         bf16x8_to_f32(raw[t], v[t]);
+}
+
+// v *= colscale[column] for the lane's 32 values of chunk c (one fp32 rounding each; the
+// products feed no addition, so the pairs cannot be merged into a multiply-add).
+__device__ __forceinline__ void apply_colscale(float (&v)[4][8], const float *cs, int32_t K,
+                                               int32_t c, uint32_t lane)
+{
+    const int32_t base = c * 1024 + static_cast<int32_t>(lane >> 3) * 256 +
+                         static_cast<int32_t>(lane & 7u) * 8;
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+        const int32_t e = base + t * 64;
+        uint4 a = make_uint4(0u, 0u, 0u, 0u), b = make_uint4(0u, 0u, 0u, 0u);
+        if (e < K) {
+            a = ld_nc_v4(cs + e);
+            b = ld_nc_v4(cs + e + 4);
+        }
+        const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+        for (int i = 0; i < 8; i += 2)
+            mul2(v[t][i], v[t][i + 1], v[t][i], v[t][i + 1], __uint_as_float(w[i]),
+                 __uint_as_float(w[i + 1]));
+    }
 }
 
 __device__ __forceinline__ float chunk_absmax(const float (&v)[4][8])
@@ -232,7 +260,7 @@ __device__ __forceinline__ void load_raw(const uint16_t *xr, int32_t K, int32_t 
 // Rows of at most 16 chunks (K <= 16384): each warp owns one chunk of a row, a CTA owns
 // `rpc` rows at a time and walks row groups persistently, loading the next row group into
 // registers while it rotates and quantizes the current one.
-template <int G>
+template <int G, bool COLSCALE>
 __global__ void __launch_bounds__(512) rotquant_persistent_kernel(const RotquantParams p)
 {
     __shared__ float s_amax[2][32];
@@ -263,6 +291,8 @@ __global__ void __launch_bounds__(512) rotquant_persistent_kernel(const Rotquant
             const bool ok = nrg < n_groups && nrow < p.M && has_chunk;
             load_raw(p.x + (ok ? nrow : 0) * p.ldx, p.K, wr, ok, lane, raw);
         }
+        if (COLSCALE && has_chunk)
+            apply_colscale(v, p.colscale, p.K, wr, lane);
         chunk_butterfly<G>(v, lane);
         float amax = chunk_absmax(v);
 #pragma unroll
@@ -283,7 +313,7 @@ __global__ void __launch_bounds__(512) rotquant_persistent_kernel(const Rotquant
     }
 }
 
-template <int G>
+template <int G, bool COLSCALE>
 __global__ void __launch_bounds__(512) rotquant_kernel(const RotquantParams p)
 {
     __shared__ float s_amax[32];
@@ -304,6 +334,8 @@ __global__ void __launch_bounds__(512) rotquant_kernel(const RotquantParams p)
     float amax = 0.0f;
     if (single) {
         load_chunk(xr, p.K, wr, row_ok && my_chunks == 1, lane, v);
+        if (COLSCALE && my_chunks == 1)
+            apply_colscale(v, p.colscale, p.K, wr, lane);
         chunk_butterfly<G>(v, lane);
         amax = chunk_absmax(v);
     } else {
@@ -311,6 +343,8 @@ __global__ void __launch_bounds__(512) rotquant_kernel(const RotquantParams p)
         // rotation (the row is then read from L2)
         for (int32_t j = 0; j < my_chunks; ++j) {
             load_chunk(xr, p.K, wr + j * p.wpr, row_ok, lane, v);
+            if (COLSCALE)
+                apply_colscale(v, p.colscale, p.K, wr + j * p.wpr, lane);
             chunk_butterfly<G>(v, lane);
             amax = fmaxf(amax, chunk_absmax(v));
         }
@@ -335,6 +369,8 @@ __global__ void __launch_bounds__(512) rotquant_kernel(const RotquantParams p)
     } else {
         for (int32_t j = 0; j < my_chunks; ++j) {
             load_chunk(xr, p.K, wr + j * p.wpr, row_ok, lane, v);
+            if (COLSCALE)
+                apply_colscale(v, p.colscale, p.K, wr + j * p.wpr, lane);
             chunk_butterfly<G>(v, lane);
             quant_store_chunk(v, qr, p.K, wr + j * p.wpr, row_ok, lane, s_z, zero);
         }

@@ -126,6 +126,33 @@ sdnq_status sdnq_int8_linear_gelu(const int8_t *qx, const float *sx, const int8_
                                   void *stream);
 
 /*
+ * Input gradient through the frozen rotated int8 base, for PEFT training where the base
+ * layer is frozen and only its input needs a gradient ("ConvRot / Hadamard SDNQ", PEFT
+ * Behavior; "SDNQ: SD.Next Quantization Engine", quantized training example: the quantized
+ * matmul also runs on the backward pass). The layer holds W_hat = diag(sW) qW H_g / sqrt(g)
+ * (H_g the block-diagonal Sylvester matrix, symmetric), so dx = dy W_hat is computed as:
+ *   1. qg, sg = per-token int8 of c = fp32(dy) * sW[n] (sW varies along the contraction, so
+ *      it is folded into dy): sg = fp32(amax_n |c| / 127), qg = rne(c / sg) clamped to
+ *      [-127, 127]; an all-zero row gives sg = 0 and codes 0;
+ *   2. acc[m][k] = sum_n qg[m][n] * qW[n][k] in int32 (tensor cores, qW read in place);
+ *   3. dx = bf16( FWHT_g(fp32(acc) * sg[m]) * fp32(1/sqrt(g)) ), the butterfly in fp32
+ *      with ascending stages per group of g columns.
+ *   dy    [M, N] bf16, row stride lddy (>= N, multiple of 8), 16-byte aligned.
+ *   qW    [N, K] int8 and sW [N] fp32 from sdnq_rotate_quant_weight with this `group`
+ *         (16-byte aligned).
+ *   qg_ws [M, N] int8 dense and sg_ws [M] fp32: caller-provided workspace; they hold qg and
+ *         sg afterwards.
+ *   dx    [M, K] bf16 out, row stride lddx (>= K, multiple of 8), 16-byte aligned.
+ *   acc_out: NULL, or [M, K] int32 dense for the raw accumulators (parity checks).
+ *   N % 16 == 0 (16..SDNQ_MAX_K), K % 16 == 0, K % group == 0. M == 0 is a no-op.
+ */
+sdnq_status sdnq_int8_linear_grad_input(const uint16_t *dy, int64_t lddy, const int8_t *qW,
+                                        const float *sW, int64_t M, int64_t N, int64_t K,
+                                        int32_t group, int8_t *qg_ws, float *sg_ws,
+                                        uint16_t *dx, int64_t lddx, int32_t *acc_out,
+                                        void *stream);
+
+/*
  * As sdnq_int8_linear, plus the bf16 LoRA side term of PEFT training on a frozen int8
  * base ("ConvRot / Hadamard SDNQ", PEFT Behavior): out = bf16(v + lora_scale * (u B)),
  * u = bf16(x A).

@@ -126,6 +126,29 @@ def test_lora_validation(lib):
     assert lora(lib, A=MIS) == _native.SDNQ_ERR_ALIGN
 
 
+def grad(lib, dy=A16, lddy=256, qW=A16, sW=A16, M=128, N=256, K=512, g=256, qg=A16, sg=A16,
+         dx=A16, lddx=512, acc=0):
+    return lib.sdnq_int8_linear_grad_input(dy, lddy, qW, sW, M, N, K, g, qg, sg, dx, lddx, acc, S)
+
+
+def test_grad_input_validation(lib):
+    assert grad(lib, dy=0) == _native.SDNQ_ERR_NULL
+    assert grad(lib, qg=0) == _native.SDNQ_ERR_NULL
+    assert grad(lib, sW=0) == _native.SDNQ_ERR_NULL
+    assert grad(lib, M=-1) == _native.SDNQ_ERR_SHAPE
+    assert grad(lib, N=8) == _native.SDNQ_ERR_SHAPE
+    assert grad(lib, N=264, lddy=264) == _native.SDNQ_ERR_SHAPE   # contraction % 16
+    assert grad(lib, K=520, lddx=520) == _native.SDNQ_ERR_SHAPE   # K % group
+    assert grad(lib, lddy=128) == _native.SDNQ_ERR_SHAPE
+    assert grad(lib, lddx=256) == _native.SDNQ_ERR_SHAPE
+    assert grad(lib, g=48) == _native.SDNQ_ERR_UNSUPPORTED
+    assert grad(lib, g=512) == _native.SDNQ_ERR_UNSUPPORTED
+    assert grad(lib, lddy=260) == _native.SDNQ_ERR_ALIGN
+    assert grad(lib, sW=A16 + 4) == _native.SDNQ_ERR_ALIGN
+    assert grad(lib, qg=MIS) == _native.SDNQ_ERR_ALIGN
+    assert grad(lib, acc=A16 + 4) == _native.SDNQ_ERR_ALIGN
+
+
 def test_gelu_and_selftest_validation(lib):
     assert lib.sdnq_gelu_bf16(0, 4, 8, 8, A16, 8, S) == _native.SDNQ_ERR_NULL
     assert lib.sdnq_gelu_bf16(A16, 4, 0, 8, A16, 8, S) == _native.SDNQ_ERR_SHAPE
@@ -142,6 +165,7 @@ def test_valid_arguments_without_a_b200_are_refused(lib):
     assert lin(lib) == _native.SDNQ_ERR_UNSUPPORTED
     assert lora(lib) == _native.SDNQ_ERR_UNSUPPORTED
     assert lib.sdnq_gelu_bf16(A16, 4, 8, 8, A16, 8, S) == _native.SDNQ_ERR_UNSUPPORTED
+    assert grad(lib) == _native.SDNQ_ERR_UNSUPPORTED
 
 
 def test_binding_refuses_cpu_tensors(lib):

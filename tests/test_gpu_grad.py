@@ -1,0 +1,112 @@
+"""GPU parity of the input gradient through the frozen rotated int8 base
+(sdnq_int8_linear_grad_input) against the oracle's three steps: bit-exact int8 codes of
+dy * sW, fp32 scales, int32 accumulators and bf16 dx, on ragged shapes (M, the contraction N
+and the output width K not multiples of the tiles), every group size, strided dy, zero rows,
+and at the full size of the attention and PEFT layers on sampled rows. Every input is seeded;
+every expected value comes from the oracle."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import hadamard_rotated_int8_b200 as sd
+from hadamard_rotated_int8_b200 import _build, synthetic
+from tests.test_gpu_parity import assert_equal, bits_of
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    _build.build()
+    oracle.build()
+    torch.cuda.init()
+    yield
+    assert sd.sdnq_device_status() == 0
+
+
+def grad_case(M, N, K, g, seed, dy_std=0.01, outlier_cols=0, ld_pad=0):
+    """dy [M, N] (optionally inside a wider buffer), the layer's weight W [N, K]."""
+    gen = torch.Generator("cpu").manual_seed(seed)
+    dy = torch.randn(M, N + ld_pad, generator=gen) * dy_std
+    if outlier_cols:
+        cols = torch.randperm(N, generator=gen)[:outlier_cols]
+        dy[:, cols] *= 40.0
+    W = torch.randn(N, K, generator=gen) * 0.02
+    return dy.to(torch.bfloat16), W.to(torch.bfloat16)
+
+
+def run_gpu(dy_full, W, g, N):
+    dyg = dy_full.cuda()[:, :N]
+    qW, sW = sd.sdnq_rotate_quant_weight(W.cuda(), g)
+    M, K = dyg.shape[0], W.shape[1]
+    acc = torch.empty((M, K), dtype=torch.int32, device="cuda")
+    qg = torch.empty((M, N), dtype=torch.int8, device="cuda")
+    sg = torch.empty((M,), dtype=torch.float32, device="cuda")
+    dx = sd.sdnq_int8_linear_grad_input(dyg, qW, sW, g, qg_ws=qg, sg_ws=sg, acc_out=acc)
+    torch.cuda.synchronize()
+    return {"qg": qg.cpu().numpy(), "sg": sg.cpu().numpy(), "acc": acc.cpu().numpy(),
+            "dx": bits_of(dx)}
+
+
+def oracle_ref(dy_full, W, g, N, rows=None):
+    dyb = synthetic.bits(dy_full[:, :N].contiguous())
+    if rows is not None:
+        dyb = dyb[rows]
+    qW, sW = oracle.rotate_quantize(synthetic.bits(W), g)
+    return oracle.grad_input(dyb, qW, sW, g)
+
+
+CASES = [
+    (128, 256, 256, 256), (300, 512, 768, 256), (257, 96, 512, 64), (130, 160, 384, 128),
+    (64, 48, 256, 8), (200, 1040, 1024, 32), (1, 16, 16, 16), (129, 272, 2304, 256),
+    (77, 3072, 512, 128),
+]
+
+
+@pytest.mark.parametrize("M,N,K,g", CASES)
+def test_grad_input_bit_exact(M, N, K, g):
+    dy, W = grad_case(M, N, K, g, seed=M + N + K + g, outlier_cols=max(1, N // 100))
+    got = run_gpu(dy, W, g, N)
+    ref = oracle_ref(dy, W, g, N)
+    assert_equal(got["qg"], ref["qg"], "codes of dy * sW")
+    assert_equal(got["sg"].view(np.uint32), ref["sg"].view(np.uint32), "scales of dy * sW")
+    assert_equal(got["acc"], ref["acc"], "int32 accumulators")
+    assert_equal(got["dx"], ref["dx"], "bf16 dx")
+
+
+def test_grad_input_strided_dy_and_zero_rows():
+    M, N, K, g = 150, 512, 512, 256
+    dy, W = grad_case(M, N, K, g, seed=9, ld_pad=24)
+    dy[3] = 0.0
+    dy[149] = 0.0
+    got = run_gpu(dy, W, g, N)
+    ref = oracle_ref(dy, W, g, N)
+    assert got["sg"][3] == 0 and got["sg"][149] == 0
+    assert_equal(got["qg"], ref["qg"], "codes")
+    assert_equal(got["dx"], ref["dx"], "bf16 dx")
+
+
+def test_grad_input_empty_batch_is_a_noop():
+    W = torch.zeros(64, 256, dtype=torch.bfloat16, device="cuda")
+    qW, sW = sd.sdnq_rotate_quant_weight(W, 256)
+    dx = sd.sdnq_int8_linear_grad_input(torch.zeros(0, 64, dtype=torch.bfloat16, device="cuda"),
+                                        qW, sW, 256)
+    assert dx.shape == (0, 256)
+
+
+@pytest.mark.parametrize("M,N,K", [(4096, 3072, 3072), (8192, 12288, 3072)])
+def test_grad_input_full_size_sampled_rows(M, N, K):
+    """The attention projection and the PEFT feed-forward layer at full size, in the launch
+    configuration of a real call: codes, scales, accumulators and dx on sampled rows (every
+    column)."""
+    g = 256
+    dy, W = grad_case(M, N, K, g, seed=M // 7 + N, outlier_cols=N // 100)
+    got = run_gpu(dy, W, g, N)
+    rng = np.random.default_rng(M + N)
+    rows = np.unique(np.concatenate([[0, M - 1], rng.choice(M, 14, replace=False)]))
+    ref = oracle_ref(dy, W, g, N, rows=rows)
+    assert_equal(got["qg"][rows], ref["qg"], "codes (sampled rows)")
+    assert_equal(got["sg"][rows].view(np.uint32), ref["sg"].view(np.uint32), "scales")
+    assert_equal(got["acc"][rows], ref["acc"], "accumulators (sampled rows)")
+    assert_equal(got["dx"][rows], ref["dx"], "dx (sampled rows)")
