@@ -92,6 +92,8 @@ def profiled_traffic(kernel: str, workload: str):
 
 def workload_ops(case, name):
     """int8 GEMM ops (2*M*N*K summed over the step's GEMMs) and extra bf16 LoRA flops."""
+    if name.startswith("grad_"):
+        return 2 * case.M * case.N * case.K, 0   # dy [M, N] x qW [N, K]
     if name.startswith("dit_mlp"):
         return 2 * 2 * case.M * case.N * case.K, 0
     lora = 0
@@ -119,7 +121,18 @@ class Step:
         self.qW, self.sW = sd.sdnq_rotate_quant_weight(case.W.to(dev), g)
         self.out = torch.empty((case.M, case.N), dtype=torch.bfloat16, device=dev)
         self.gemm_stages = []
-        if name.startswith("dit_mlp"):
+        if name.startswith("grad_"):
+            # backward through the frozen layer: x holds dy [M, N]; W is [N, K]
+            self.out = torch.empty((case.M, case.K), dtype=torch.bfloat16, device=dev)
+            self.qx = torch.empty((case.M, case.N), dtype=torch.int8, device=dev)
+            self.stages = [
+                ("rotquant", lambda: sd.sdnq_quant_grad_output(self.x, self.sW, self.qx, self.sx)),
+                ("gemm_grad", lambda: sd.sdnq_int8_grad_input_gemm(self.qx, self.sx, self.qW,
+                                                                   g, out=self.out)),
+            ]
+            self.gemm_stages = ["gemm_grad"]
+            self.launches = 2
+        elif name.startswith("dit_mlp"):
             Wd = case.extra["W_down"].to(dev)
             self.qWd, self.sWd = sd.sdnq_rotate_quant_weight(Wd, g)
             self.h = torch.empty((case.M, case.N), dtype=torch.bfloat16, device=dev)
@@ -222,6 +235,11 @@ def oracle_step(case, rows, nthreads):
     import oracle
     from hadamard_rotated_int8_b200 import synthetic
     xb = synthetic.bits(case.x)[:rows]
+    if case.extra.get("grad"):
+        qg, sg = oracle.colscale_quantize(xb, case._oracle_sW, nthreads)
+        acc = oracle.gemm_s8_nn(qg, case._oracle_qW, nthreads)
+        oracle.grad_input_epilogue(acc, sg, case.g, nthreads)
+        return
     qx, sx = oracle.rotate_quantize(xb, case.g, nthreads)
     acc = oracle.gemm_s8(qx, case._oracle_qW, nthreads)
     L = None
@@ -271,8 +289,11 @@ def cpu_baseline(case, name, budget_s=12.0):
         reps += 1
     tops = ops_per_row * rows * reps / total / 1e12
     return {"value": tops, "unit": "TOPS", "cores": nthreads, "kind": "oracle",
-            "sample": f"{rows} of {case.M} tokens of {name} x{reps} (rotate+quantize, int8 GEMM "
-                      f"against all {case.N} weight rows, fp32 epilogue), {total:.2f} s"}
+            "sample": (f"{rows} of {case.M} tokens of {name} x{reps} (int8 of dy*sW, NN int8 "
+                       f"GEMM against the {case.N}x{case.K} codes, inverse-rotation epilogue), "
+                       f"{total:.2f} s") if case.extra.get("grad") else
+                      (f"{rows} of {case.M} tokens of {name} x{reps} (rotate+quantize, int8 GEMM "
+                       f"against all {case.N} weight rows, fp32 epilogue), {total:.2f} s")}
 
 
 def run_reference(args):
@@ -329,7 +350,10 @@ def config_of(case, args):
          "parallelism": f"replicas x{args.gpus}",
          "l2": "flushed before every timed step (write of 2x the L2 size)"}
     if args.workload.startswith("dit_mlp"):
-        c["chain"] = "rotquant -> up GEMM -> GELU -> rotquant -> down GEMM"
+        c["chain"] = "rotquant -> up GEMM with GELU epilogue -> rotquant -> down GEMM"
+    if args.workload.startswith("grad_"):
+        c["chain"] = ("input gradient of a frozen [N, K] layer: int8 of dy*sW [M, N] -> "
+                      "NN int8 GEMM with row scale + inverse Hadamard epilogue -> dx [M, K]")
     return c
 
 
@@ -449,8 +473,11 @@ def main():
     gemm_launch_ms = gemm_ms / len(step.gemm_stages)
     gemm_tops = ops / (gemm_ms * 1e-3) / 1e12
     rq_ms = stage_ms["rotquant"] / args.steps
-    rq_gbs = rotquant_bytes(case.M, case.K) / (rq_ms * 1e-3) / 1e9
-    gemm_kernel = "gemm_s8_kernel" if case.A is None else "gemm_s8_kernel_lora"
+    grad = args.workload.startswith("grad_")
+    rq_rows_k = case.N if grad else case.K        # row length of the quantized operand
+    rq_gbs = rotquant_bytes(case.M, rq_rows_k) / (rq_ms * 1e-3) / 1e9
+    gemm_kernel = ("gemm_s8_kernel_grad_input" if grad else
+                   "gemm_s8_kernel" if case.A is None else "gemm_s8_kernel_lora")
     line = {
         "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
@@ -467,11 +494,11 @@ def main():
             "frac_of_int8_spec": gemm_tops / INT8_SPEC_TOPS,
         },
         "roofline_rotquant": {
-            "kernel": ("rotquant_persistent_kernel" if case.K <= 16384 else "rotquant_kernel"),
+            "kernel": ("rotquant_persistent_kernel" if rq_rows_k <= 16384 else "rotquant_kernel"),
             "bound": "hbm", "achieved": rq_gbs,
             "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": rq_gbs / peaks["hbm_gbs"],
             "traffic": profiled_traffic("rotquant", args.workload),
-            "bytes_per_launch": rotquant_bytes(case.M, case.K), "ms_per_launch": rq_ms,
+            "bytes_per_launch": rotquant_bytes(case.M, rq_rows_k), "ms_per_launch": rq_ms,
             "peak_source": f"{peak_src} copy bandwidth",
         },
         "stage_ms_per_step": {n: stage_ms[n] / args.steps for n in names},

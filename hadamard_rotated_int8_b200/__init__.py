@@ -9,18 +9,22 @@ The compute lives in ``libsdnq.so`` (hand-written CUDA behind the C ABI of
 * ``sdnq_int8_linear_gelu``     the same with GELU fused into the epilogue (MLP up-projection)
 * ``sdnq_int8_linear_lora``     the same plus the bf16 LoRA side term
 * ``sdnq_int8_linear_grad_input`` input gradient through the frozen rotated int8 base
+  (= ``sdnq_quant_grad_output`` then ``sdnq_int8_grad_input_gemm``)
 * ``sdnq_gelu_bf16``            exact-erf GELU (MLP glue)
 
 ``linear`` composes the online path (rotate + quantize, then the int8 linear).
 """
 from ._native import (SdnqError, lib, sdnq_device_status, sdnq_gelu_bf16, sdnq_int8_linear,
-                      sdnq_int8_linear_gelu, sdnq_int8_linear_grad_input, sdnq_int8_linear_lora,
+                      sdnq_int8_grad_input_gemm, sdnq_int8_linear_gelu,
+                      sdnq_int8_linear_grad_input, sdnq_int8_linear_lora,
                       sdnq_int8_linear_lora_noalloc, sdnq_rotate_quant_weight,
-                      sdnq_rotquant_act, sdnq_selftest_wait_timeout, status_string, version)
+                      sdnq_quant_grad_output, sdnq_rotquant_act, sdnq_selftest_wait_timeout,
+                      status_string, version)
 
 __all__ = [
     "SdnqError", "lib", "linear", "sdnq_device_status", "sdnq_gelu_bf16", "sdnq_int8_linear",
-    "sdnq_int8_linear_gelu", "sdnq_int8_linear_grad_input", "sdnq_int8_linear_lora",
+    "sdnq_int8_grad_input_gemm", "sdnq_int8_linear_gelu", "sdnq_int8_linear_grad_input",
+    "sdnq_int8_linear_lora", "sdnq_quant_grad_output",
     "sdnq_int8_linear_lora_noalloc",
     "sdnq_rotate_quant_weight", "sdnq_rotquant_act", "sdnq_selftest_wait_timeout",
     "status_string", "version",

@@ -43,6 +43,8 @@ SIGNATURES = {
     "sdnq_int8_linear_gelu": [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _I64, _P, _P],
     "sdnq_int8_linear_grad_input": [_P, _I64, _P, _P, _I64, _I64, _I64, _I32, _P, _P, _P, _I64,
                                     _P, _P],
+    "sdnq_quant_grad_output": [_P, _I64, _P, _I64, _I64, _P, _P, _P],
+    "sdnq_int8_grad_input_gemm": [_P, _P, _P, _I64, _I64, _I64, _I32, _P, _I64, _P, _P],
     "sdnq_int8_linear_lora": [_P, _P, _P, _P, _P, _P, _I64, _P, _P, _I32, _F, _P, _I64, _I64,
                               _I64, _P, _I64, _P, _P],
     "sdnq_int8_linear_lora_noalloc": [_P, _P, _P, _P, _P, _P, _I64, _P, _P, _I32, _F, _I64,
@@ -207,6 +209,34 @@ def sdnq_int8_linear_grad_input(dy, qW, sW, group: int, qg_ws=None, sg_ws=None, 
                                              group, _ptr(qg_ws), _ptr(sg_ws), _ptr(out),
                                              out.stride(0), _ptr(acc_out), _stream(stream)),
            "sdnq_int8_linear_grad_input")
+    return out
+
+
+def sdnq_quant_grad_output(dy, sW, qg=None, sg=None, stream=None):
+    """(qg [M, N] int8, sg [M] fp32): per-token int8 of fp32(dy) * sW."""
+    _req(dy, torch.bfloat16, "dy", 2)
+    M, N = dy.shape
+    qg = torch.empty((M, N), dtype=torch.int8, device=dy.device) if qg is None else qg
+    sg = torch.empty((M,), dtype=torch.float32, device=dy.device) if sg is None else sg
+    _check(lib().sdnq_quant_grad_output(_ptr(dy), dy.stride(0), _ptr(sW), M, N, _ptr(qg),
+                                        _ptr(sg), _stream(stream)), "sdnq_quant_grad_output")
+    return qg, sg
+
+
+def sdnq_int8_grad_input_gemm(qg, sg, qW, group: int, out=None, acc_out=None, stream=None):
+    """dx [M, K] bf16 from the quantized output gradient (qg, sg) and the layer's codes qW."""
+    _req(qg, torch.int8, "qg", 2)
+    _req(qW, torch.int8, "qW", 2)
+    _dense(qg, "qg")
+    _dense(qW, "qW")
+    M, N = qg.shape
+    if qW.shape[0] != N:
+        raise ValueError("qg and qW disagree on N")
+    K = qW.shape[1]
+    out = _rows_out(M, K, torch.bfloat16, qg.device) if out is None else out
+    _check(lib().sdnq_int8_grad_input_gemm(_ptr(qg), _ptr(sg), _ptr(qW), M, N, K, group,
+                                           _ptr(out), out.stride(0), _ptr(acc_out),
+                                           _stream(stream)), "sdnq_int8_grad_input_gemm")
     return out
 
 

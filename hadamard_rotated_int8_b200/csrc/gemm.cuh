@@ -269,7 +269,8 @@ __global__ void __launch_bounds__(320, 1)
                    const __grid_constant__ CUtensorMap tmO, const GemmParams p)
 {
     using C = GemmConfig<BN, LORA, GELU>;
-    static_assert(GRAD_G == 0 || (BN == 256 && !LORA && !GELU && 256 % GRAD_G == 0),
+    static_assert(GRAD_G == 0 || (BN == 256 && !LORA && !GELU && (GRAD_G & (GRAD_G - 1)) == 0 &&
+                                  GRAD_G <= 256),
                   "input-gradient mode: plain tiles of 256 columns, G divides 256");
     extern __shared__ uint8_t smem_raw[];
     // 1024-byte alignment for the 128-byte swizzle atoms

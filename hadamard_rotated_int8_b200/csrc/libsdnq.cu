@@ -358,39 +358,48 @@ sdnq_status run_linear(const int8_t *qx, const float *sx, const int8_t *qW, cons
 
 // ---------------------------------------------------------------- input gradient
 
-// dx = dy W_hat through the frozen rotated base: q_g, s_g = per-token int8 of dy * sW
-// (into the caller's workspace), then the NN int8 product q_g qW with the row scale,
-// inverse rotation and 1/sqrt(g) in the epilogue.
-sdnq_status run_grad_input(const uint16_t *dy, int64_t lddy, const int8_t *qW, const float *sW,
-                           int64_t M, int64_t N, int64_t K, int32_t group, int8_t *qg_ws,
-                           float *sg_ws, uint16_t *dx, int64_t lddx, int32_t *acc_out,
-                           void *stream)
+// dx = dy W_hat through the frozen rotated base, in two launches: q_g, s_g = per-token int8
+// of dy * sW, then the NN int8 product q_g qW with the row scale, inverse rotation and
+// 1/sqrt(g) in the epilogue.
+sdnq_status validate_grad_quant(const void *dy, int64_t lddy, const void *sW, int64_t M,
+                                int64_t N, const void *qg, const void *sg)
 {
-    if (!qW || !sW || (M != 0 && (!dy || !qg_ws || !sg_ws || !dx)))
+    if (!sW || (M != 0 && (!dy || !qg || !sg)))
+        return SDNQ_ERR_NULL;
+    if (M < 0 || M > INT32_MAX || N < 16 || N > SDNQ_MAX_K || N % 16 != 0 || lddy < N)
+        return SDNQ_ERR_SHAPE;
+    if (lddy % 8 != 0 || !aligned(dy, 16) || !aligned(sW, 16) || !aligned(qg, 16) ||
+        !aligned(sg, 4))
+        return SDNQ_ERR_ALIGN;
+    return SDNQ_OK;
+}
+
+sdnq_status validate_grad_gemm(const void *qg, const void *sg, const void *qW, int64_t M,
+                               int64_t N, int64_t K, int32_t group, const void *dx,
+                               int64_t lddx, const void *acc_out)
+{
+    if (!qW || (M != 0 && (!qg || !sg || !dx)))
         return SDNQ_ERR_NULL;
     if (M < 0 || M > INT32_MAX || N < 16 || N > SDNQ_MAX_K || N % 16 != 0 || K < 16 ||
-        K > INT32_MAX || K % 16 != 0 || lddy < N || lddx < K)
+        K > INT32_MAX || K % 16 != 0 || lddx < K)
         return SDNQ_ERR_SHAPE;
     if (!is_pow2(group) || group < SDNQ_MIN_GROUP || group > SDNQ_MAX_GROUP)
         return SDNQ_ERR_UNSUPPORTED;
     if (K % group != 0)
         return SDNQ_ERR_SHAPE;
-    if (lddy % 8 != 0 || lddx % 8 != 0 || !aligned(dy, 16) || !aligned(qW, 16) ||
-        !aligned(sW, 16) || !aligned(qg_ws, 16) || !aligned(sg_ws, 4) || !aligned(dx, 16) ||
-        (acc_out && !aligned(acc_out, 16)))
+    if (lddx % 8 != 0 || !aligned(qg, 16) || !aligned(sg, 4) || !aligned(qW, 16) ||
+        !aligned(dx, 16) || (acc_out && !aligned(acc_out, 16)))
         return SDNQ_ERR_ALIGN;
-    DeviceInfo dev;
-    sdnq_status st = current_device(&dev);
-    if (st != SDNQ_OK)
-        return st;
-    if (M == 0)
-        return SDNQ_OK;
-    cudaStream_t cs = static_cast<cudaStream_t>(stream);
-    if ((st = launch_rowquant(dy, M, N, lddy, 1, sW, qg_ws, sg_ws, dev, cs)) != SDNQ_OK)
-        return st;
+    return SDNQ_OK;
+}
+
+sdnq_status launch_grad_gemm(const DeviceInfo &dev, const int8_t *qg, const float *sg,
+                             const int8_t *qW, int64_t M, int64_t N, int64_t K, int32_t group,
+                             uint16_t *dx, int64_t lddx, int32_t *acc_out, cudaStream_t cs)
+{
     GemmParams p;
-    p.sx = sg_ws;
-    p.sw = sW;          // not read in this mode
+    p.sx = sg;
+    p.sw = nullptr;    // not read in this mode
     p.bias = nullptr;
     p.out = dx;
     p.ldo = lddx;
@@ -403,13 +412,64 @@ sdnq_status run_grad_input(const uint16_t *dy, int64_t lddy, const int8_t *qW, c
     p.c_g = static_cast<float>(1.0 / std::sqrt(static_cast<double>(group)));
     p.timeout_ns = kDefaultTimeoutNs;
     switch (group) {
-    case 8: return launch_gemm<256, false, false, 8>(dev, qg_ws, qW, nullptr, nullptr, 0, p, cs);
-    case 16: return launch_gemm<256, false, false, 16>(dev, qg_ws, qW, nullptr, nullptr, 0, p, cs);
-    case 32: return launch_gemm<256, false, false, 32>(dev, qg_ws, qW, nullptr, nullptr, 0, p, cs);
-    case 64: return launch_gemm<256, false, false, 64>(dev, qg_ws, qW, nullptr, nullptr, 0, p, cs);
-    case 128: return launch_gemm<256, false, false, 128>(dev, qg_ws, qW, nullptr, nullptr, 0, p, cs);
-    default: return launch_gemm<256, false, false, 256>(dev, qg_ws, qW, nullptr, nullptr, 0, p, cs);
+    case 8: return launch_gemm<256, false, false, 8>(dev, qg, qW, nullptr, nullptr, 0, p, cs);
+    case 16: return launch_gemm<256, false, false, 16>(dev, qg, qW, nullptr, nullptr, 0, p, cs);
+    case 32: return launch_gemm<256, false, false, 32>(dev, qg, qW, nullptr, nullptr, 0, p, cs);
+    case 64: return launch_gemm<256, false, false, 64>(dev, qg, qW, nullptr, nullptr, 0, p, cs);
+    case 128: return launch_gemm<256, false, false, 128>(dev, qg, qW, nullptr, nullptr, 0, p, cs);
+    default: return launch_gemm<256, false, false, 256>(dev, qg, qW, nullptr, nullptr, 0, p, cs);
     }
+}
+
+sdnq_status run_grad_quant(const uint16_t *dy, int64_t lddy, const float *sW, int64_t M,
+                           int64_t N, int8_t *qg, float *sg, void *stream)
+{
+    sdnq_status st = validate_grad_quant(dy, lddy, sW, M, N, qg, sg);
+    if (st != SDNQ_OK)
+        return st;
+    DeviceInfo dev;
+    if ((st = current_device(&dev)) != SDNQ_OK)
+        return st;
+    if (M == 0)
+        return SDNQ_OK;
+    return launch_rowquant(dy, M, N, lddy, 1, sW, qg, sg, dev, static_cast<cudaStream_t>(stream));
+}
+
+sdnq_status run_grad_gemm(const int8_t *qg, const float *sg, const int8_t *qW, int64_t M,
+                          int64_t N, int64_t K, int32_t group, uint16_t *dx, int64_t lddx,
+                          int32_t *acc_out, void *stream)
+{
+    sdnq_status st = validate_grad_gemm(qg, sg, qW, M, N, K, group, dx, lddx, acc_out);
+    if (st != SDNQ_OK)
+        return st;
+    DeviceInfo dev;
+    if ((st = current_device(&dev)) != SDNQ_OK)
+        return st;
+    if (M == 0)
+        return SDNQ_OK;
+    return launch_grad_gemm(dev, qg, sg, qW, M, N, K, group, dx, lddx, acc_out,
+                            static_cast<cudaStream_t>(stream));
+}
+
+sdnq_status run_grad_input(const uint16_t *dy, int64_t lddy, const int8_t *qW, const float *sW,
+                           int64_t M, int64_t N, int64_t K, int32_t group, int8_t *qg_ws,
+                           float *sg_ws, uint16_t *dx, int64_t lddx, int32_t *acc_out,
+                           void *stream)
+{
+    sdnq_status st = validate_grad_quant(dy, lddy, sW, M, N, qg_ws, sg_ws);
+    if (st == SDNQ_OK)
+        st = validate_grad_gemm(qg_ws, sg_ws, qW, M, N, K, group, dx, lddx, acc_out);
+    if (st != SDNQ_OK)
+        return st;
+    DeviceInfo dev;
+    if ((st = current_device(&dev)) != SDNQ_OK)
+        return st;
+    if (M == 0)
+        return SDNQ_OK;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    if ((st = launch_rowquant(dy, M, N, lddy, 1, sW, qg_ws, sg_ws, dev, cs)) != SDNQ_OK)
+        return st;
+    return launch_grad_gemm(dev, qg_ws, sg_ws, qW, M, N, K, group, dx, lddx, acc_out, cs);
 }
 
 // ---------------------------------------------------------------- self-test kernel
@@ -471,6 +531,21 @@ SDNQ_API sdnq_status sdnq_int8_linear_grad_input(const uint16_t *dy, int64_t ldd
 {
     return run_grad_input(dy, lddy, qW, sW, M, N, K, group, qg_ws, sg_ws, dx, lddx, acc_out,
                           stream);
+}
+
+SDNQ_API sdnq_status sdnq_quant_grad_output(const uint16_t *dy, int64_t lddy, const float *sW,
+                                            int64_t M, int64_t N, int8_t *qg, float *sg,
+                                            void *stream)
+{
+    return run_grad_quant(dy, lddy, sW, M, N, qg, sg, stream);
+}
+
+SDNQ_API sdnq_status sdnq_int8_grad_input_gemm(const int8_t *qg, const float *sg, const int8_t *qW,
+                                               int64_t M, int64_t N, int64_t K, int32_t group,
+                                               uint16_t *dx, int64_t lddx, int32_t *acc_out,
+                                               void *stream)
+{
+    return run_grad_gemm(qg, sg, qW, M, N, K, group, dx, lddx, acc_out, stream);
 }
 
 SDNQ_API sdnq_status sdnq_int8_linear_lora(const int8_t *qx, const float *sx, const int8_t *qW,

@@ -141,8 +141,39 @@ __device__ __forceinline__ void load_chunk(const uint16_t *xr, int32_t K, int32_
         bf16x8_to_f32(raw[t], v[t]);
 }
 
-// v *= colscale[column] for the lane's 32 values of chunk c (one fp32 rounding each; the
-// products feed no addition, so the pairs cannot be merged into a multiply-add).
+// The column multipliers of the lane's 32 values of chunk c (0 past the row end).
+__device__ __forceinline__ void load_colscale(float (&m)[4][8], const float *cs, int32_t K,
+                                              int32_t c, uint32_t lane)
+{
+    const int32_t base = c * 1024 + static_cast<int32_t>(lane >> 3) * 256 +
+                         static_cast<int32_t>(lane & 7u) * 8;
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+        const int32_t e = base + t * 64;
+        uint4 a = make_uint4(0u, 0u, 0u, 0u), b = make_uint4(0u, 0u, 0u, 0u);
+        if (e < K) {
+            a = ld_nc_v4(cs + e);
+            b = ld_nc_v4(cs + e + 4);
+        }
+        const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            m[t][i] = __uint_as_float(w[i]);
+    }
+}
+
+// v *= m elementwise (one fp32 rounding each; the products feed no addition, so the pairs
+// cannot be merged into a multiply-add).
+__device__ __forceinline__ void mul_colscale(float (&v)[4][8], const float (&m)[4][8])
+{
+#pragma unroll
+    for (int t = 0; t < 4; ++t)
+#pragma unroll
+        for (int i = 0; i < 8; i += 2)
+            mul2(v[t][i], v[t][i + 1], v[t][i], v[t][i + 1], m[t][i], m[t][i + 1]);
+}
+
+// v *= colscale[column] for the lane's 32 values of chunk c.
 __device__ __forceinline__ void apply_colscale(float (&v)[4][8], const float *cs, int32_t K,
                                                int32_t c, uint32_t lane)
 {
@@ -271,6 +302,10 @@ __global__ void __launch_bounds__(512) rotquant_persistent_kernel(const Rotquant
     const bool has_chunk = wr < p.nchunks;
     const int64_t n_groups = (p.M + p.rpc - 1) / p.rpc;
 
+    // a warp keeps one chunk of every row it visits: its column multipliers stay in registers
+    float cmul[COLSCALE ? 4 : 1][8];
+    if constexpr (COLSCALE)
+        load_colscale(cmul, p.colscale, p.K, has_chunk ? wr : p.nchunks, lane);  // zeros if none
     int64_t rg = blockIdx.x;
     uint4 raw[4];
     {
@@ -291,8 +326,8 @@ __global__ void __launch_bounds__(512) rotquant_persistent_kernel(const Rotquant
             const bool ok = nrg < n_groups && nrow < p.M && has_chunk;
             load_raw(p.x + (ok ? nrow : 0) * p.ldx, p.K, wr, ok, lane, raw);
         }
-        if (COLSCALE && has_chunk)
-            apply_colscale(v, p.colscale, p.K, wr, lane);
+        if constexpr (COLSCALE)
+            mul_colscale(v, cmul);
         chunk_butterfly<G>(v, lane);
         float amax = chunk_absmax(v);
 #pragma unroll

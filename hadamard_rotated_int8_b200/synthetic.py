@@ -12,7 +12,9 @@ attention linears 3072x3072, feed-forward 12288x3072, 4608 joint tokens):
   generator, multiplied by the stated factor before rounding;
 * Student-t(nu) is drawn as ``z / sqrt(chi2_nu / nu)`` with ``chi2_nu`` a sum of ``nu`` squared
   standard normals (nu integer), which is the textbook construction;
-* draw order within a case: x, outlier columns, W (or W_up, W_down), bias, A, B.
+* draw order within a case: x, outlier columns, W (or W_up, W_down), bias, A, B;
+* input-gradient cases (the backward pass through a frozen layer of N outputs and K inputs):
+  dy [M, N] ~ N(0, dy_std^2) with outlier columns, then W [N, K]; dy is kept in ``x``.
 """
 from __future__ import annotations
 
@@ -113,14 +115,42 @@ WORKLOADS = {
 }
 
 
+def make_grad_case(M, N, K, g=256, seed=0, dy_std=0.01, outlier_frac=0.0, outlier_count=None,
+                   outlier_factor=1.0, w_std=0.02, ld_pad=0, name="grad") -> Case:
+    """Output gradient dy [M, N] (in ``x``; ``ld_pad`` extra columns make it a strided view's
+    parent) and the frozen layer's weight W [N, K]."""
+    gen = torch.Generator("cpu").manual_seed(seed)
+    dy = _normal(gen, (M, N + ld_pad), dy_std)
+    count = outlier_count if outlier_count is not None else int(round(outlier_frac * N))
+    cols = torch.randperm(N, generator=gen)[:count]
+    if count:
+        dy[:, cols] *= outlier_factor
+    W = _normal(gen, (N, K), w_std).to(torch.bfloat16)
+    return Case(name, M, N, K, g, dy.to(torch.bfloat16), W,
+                extra={"outlier_cols": cols, "seed": seed, "grad": True, "ld_pad": ld_pad})
+
+
+# Input-gradient workloads: the attention projection and the PEFT feed-forward layer run
+# backwards (dy has the layer's N output features, dx its K input features).
+GRAD_WORKLOADS = {
+    "grad_dit_attn_4096x3072x3072": dict(M=4096, N=3072, K=3072, g=256, seed=5,
+                                         outlier_frac=0.01, outlier_factor=30.0),
+    "grad_peft_8192x12288x3072": dict(M=8192, N=12288, K=3072, g=256, seed=6,
+                                      outlier_frac=0.01, outlier_factor=30.0),
+}
+
+
 def workload(name: str, g: int | None = None, M: int | None = None) -> Case:
     """Build one of the named workloads. ``g`` overrides the Hadamard group (the QuaRot
     sweep runs 64, 128, 256); ``M`` overrides the token count (smaller samples)."""
-    kw = dict(WORKLOADS[name])
+    grad = name in GRAD_WORKLOADS
+    kw = dict(GRAD_WORKLOADS[name] if grad else WORKLOADS[name])
     if g is not None:
         kw["g"] = g
     if M is not None:
         kw["M"] = M
+    if grad:
+        return make_grad_case(name=name, **kw)
     case = make_case(name=name, **kw)
     if name.startswith("dit_mlp"):
         # the down projection: W_down [K_up, N_up] drawn after the up projection's tensors

@@ -153,6 +153,22 @@ sdnq_status sdnq_int8_linear_grad_input(const uint16_t *dy, int64_t lddy, const 
                                         void *stream);
 
 /*
+ * Step 1 of sdnq_int8_linear_grad_input on its own: qg [M, N] int8 dense and sg [M] fp32,
+ * the per-token int8 of fp32(dy) * sW. Arguments and rules as there.
+ */
+sdnq_status sdnq_quant_grad_output(const uint16_t *dy, int64_t lddy, const float *sW, int64_t M,
+                                   int64_t N, int8_t *qg, float *sg, void *stream);
+
+/*
+ * Steps 2 and 3 of sdnq_int8_linear_grad_input on their own: dx [M, K] from qg, sg (step 1)
+ * and the layer's codes qW [N, K] of this `group`. Arguments and rules as there.
+ */
+sdnq_status sdnq_int8_grad_input_gemm(const int8_t *qg, const float *sg, const int8_t *qW,
+                                      int64_t M, int64_t N, int64_t K, int32_t group,
+                                      uint16_t *dx, int64_t lddx, int32_t *acc_out,
+                                      void *stream);
+
+/*
  * As sdnq_int8_linear, plus the bf16 LoRA side term of PEFT training on a frozen int8
  * base ("ConvRot / Hadamard SDNQ", PEFT Behavior): out = bf16(v + lora_scale * (u B)),
  * u = bf16(x A).

@@ -25,15 +25,11 @@ def built():
     assert sd.sdnq_device_status() == 0
 
 
-def grad_case(M, N, K, g, seed, dy_std=0.01, outlier_cols=0, ld_pad=0):
+def grad_case(M, N, K, g, seed, outlier_cols=0, ld_pad=0):
     """dy [M, N] (optionally inside a wider buffer), the layer's weight W [N, K]."""
-    gen = torch.Generator("cpu").manual_seed(seed)
-    dy = torch.randn(M, N + ld_pad, generator=gen) * dy_std
-    if outlier_cols:
-        cols = torch.randperm(N, generator=gen)[:outlier_cols]
-        dy[:, cols] *= 40.0
-    W = torch.randn(N, K, generator=gen) * 0.02
-    return dy.to(torch.bfloat16), W.to(torch.bfloat16)
+    c = synthetic.make_grad_case(M, N, K, g, seed=seed, outlier_count=outlier_cols,
+                                 outlier_factor=40.0, ld_pad=ld_pad)
+    return c.x, c.W
 
 
 def run_gpu(dy_full, W, g, N):
@@ -95,13 +91,14 @@ def test_grad_input_empty_batch_is_a_noop():
     assert dx.shape == (0, 256)
 
 
-@pytest.mark.parametrize("M,N,K", [(4096, 3072, 3072), (8192, 12288, 3072)])
-def test_grad_input_full_size_sampled_rows(M, N, K):
+@pytest.mark.parametrize("name", sorted(synthetic.GRAD_WORKLOADS))
+def test_grad_input_full_size_sampled_rows(name):
     """The attention projection and the PEFT feed-forward layer at full size, in the launch
     configuration of a real call: codes, scales, accumulators and dx on sampled rows (every
     column)."""
-    g = 256
-    dy, W = grad_case(M, N, K, g, seed=M // 7 + N, outlier_cols=N // 100)
+    case = synthetic.workload(name)
+    M, N, g = case.M, case.N, case.g
+    dy, W = case.x, case.W
     got = run_gpu(dy, W, g, N)
     rng = np.random.default_rng(M + N)
     rows = np.unique(np.concatenate([[0, M - 1], rng.choice(M, 14, replace=False)]))
@@ -110,3 +107,18 @@ def test_grad_input_full_size_sampled_rows(M, N, K):
     assert_equal(got["sg"][rows].view(np.uint32), ref["sg"].view(np.uint32), "scales")
     assert_equal(got["acc"][rows], ref["acc"], "accumulators (sampled rows)")
     assert_equal(got["dx"][rows], ref["dx"], "dx (sampled rows)")
+
+
+def test_split_calls_equal_the_composed_call():
+    M, N, K, g = 200, 512, 768, 128
+    dy, W = grad_case(M, N, K, g, seed=21, outlier_cols=5)
+    dyg = dy.cuda()
+    qW, sW = sd.sdnq_rotate_quant_weight(W.cuda(), g)
+    qg, sg = sd.sdnq_quant_grad_output(dyg, sW)
+    dx_split = sd.sdnq_int8_grad_input_gemm(qg, sg, qW, g)
+    qg2 = torch.empty_like(qg)
+    sg2 = torch.empty_like(sg)
+    dx = sd.sdnq_int8_linear_grad_input(dyg, qW, sW, g, qg_ws=qg2, sg_ws=sg2)
+    torch.cuda.synchronize()
+    assert_equal(qg.cpu().numpy(), qg2.cpu().numpy(), "codes")
+    assert_equal(bits_of(dx_split), bits_of(dx), "dx")
