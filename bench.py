@@ -107,6 +107,14 @@ def rotquant_bytes(M, K):
     return M * K * 2 + M * K + M * 4   # read bf16, write int8 codes, write fp32 scale
 
 
+def fused_one_launch(case, torch):
+    """The library's automatic choice for sdnq_int8_linear_fused: one launch when the GEMM has
+    at least three waves of 128 x 256 tiles and the rows fit the in-kernel quantizer."""
+    sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    tiles = ((case.M + 127) // 128) * ((case.N + 255) // 256)
+    return (case.K + 1023) // 1024 <= 8 and tiles >= 3 * sms
+
+
 class Step:
     """Device buffers and the stages of one step of a workload."""
 
@@ -161,6 +169,17 @@ class Step:
             ]
             self.gemm_stages = ["gemm_lora"]
             self.launches = 3  # rotquant, LoRA down-projection, fused GEMM
+        elif fused_one_launch(case, torch):
+            # one launch: the activation quantizer runs inside the GEMM kernel
+            self.sync = torch.zeros(4 * ((case.M + 127) // 128) + 64, dtype=torch.int32,
+                                    device=dev)
+            self.stages = [
+                ("fused", lambda: sd.sdnq_int8_linear_fused(
+                    self.x, g, self.qW, self.sW, self.bias, qx_ws=self.qx, sx_ws=self.sx,
+                    sync_ws=self.sync, out=self.out)),
+            ]
+            self.gemm_stages = ["fused"]
+            self.launches = 1
         else:
             self.stages = [
                 ("rotquant", lambda: sd.sdnq_rotquant_act(self.x, g, self.qx, self.sx)),
@@ -329,6 +348,20 @@ def run_reference(args):
     return 0
 
 
+def standalone_rotquant_ms(step, flush, torch, sd, reps):
+    times = []
+    for i in range(reps + 3):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        sd.sdnq_rotquant_act(step.x, step.case.g, step.qx, step.sx)
+        e1.record()
+        torch.cuda.synchronize()
+        if i >= 3:
+            times.append(e0.elapsed_time(e1))
+    return sum(times) / len(times)
+
+
 def reduce_max_over_ranks(values, dist=None, world=1, device="cuda"):
     """Element-wise max of a list of floats over all ranks (the slowest rank's times)."""
     import torch
@@ -472,11 +505,19 @@ def main():
     gemm_ms = sum(stage_ms[n] for n in step.gemm_stages) / args.steps
     gemm_launch_ms = gemm_ms / len(step.gemm_stages)
     gemm_tops = ops / (gemm_ms * 1e-3) / 1e12
-    rq_ms = stage_ms["rotquant"] / args.steps
+    if "rotquant" in stage_ms:
+        rq_ms = stage_ms["rotquant"] / args.steps
+        rq_note = "the rotate+quantize stage of the timed step"
+    else:
+        # the step's quantizer runs inside the fused kernel: time the standalone kernel on
+        # the same input (L2 flushed before each launch) for its own roofline
+        rq_ms = standalone_rotquant_ms(step, flush, torch, sd, max(args.steps // 4, 10))
+        rq_note = "standalone rotquant kernel on the step's input (the step itself runs it fused)"
     grad = args.workload.startswith("grad_")
     rq_rows_k = case.N if grad else case.K        # row length of the quantized operand
     rq_gbs = rotquant_bytes(case.M, rq_rows_k) / (rq_ms * 1e-3) / 1e9
     gemm_kernel = ("gemm_s8_kernel_grad_input" if grad else
+                   "gemm_s8_kernel_fused_quantizer" if "fused" in stage_ms else
                    "gemm_s8_kernel" if case.A is None else "gemm_s8_kernel_lora")
     line = {
         "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world,
@@ -499,13 +540,14 @@ def main():
             "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": rq_gbs / peaks["hbm_gbs"],
             "traffic": profiled_traffic("rotquant", args.workload),
             "bytes_per_launch": rotquant_bytes(case.M, rq_rows_k), "ms_per_launch": rq_ms,
-            "peak_source": f"{peak_src} copy bandwidth",
+            "peak_source": f"{peak_src} copy bandwidth", "timing": rq_note,
         },
         "stage_ms_per_step": {n: stage_ms[n] / args.steps for n in names},
         "clocks": clocks.summary(),
         "gpu_launches": step.launches * args.steps,
         "e2e": e2e,
     }
+    line["config"]["stages"] = names
     if lora_flops:
         line["tops_with_lora_flops"] = whole_job_tops(ops + lora_flops, world, ms_per_step)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -6,6 +6,7 @@ The compute lives in ``libsdnq.so`` (hand-written CUDA behind the C ABI of
 * ``sdnq_rotate_quant_weight``  weight rotate + row-wise int8 quantize (offline)
 * ``sdnq_rotquant_act``         online activation rotate + per-token int8 quantize
 * ``sdnq_int8_linear``          int8 x int8 -> int32 tensor-core matmul + fp32 de-quant epilogue
+* ``sdnq_int8_linear_fused``    rotate + quantize and the int8 linear in one launch
 * ``sdnq_int8_linear_gelu``     the same with GELU fused into the epilogue (MLP up-projection)
 * ``sdnq_int8_linear_lora``     the same plus the bf16 LoRA side term
 * ``sdnq_int8_linear_grad_input`` input gradient through the frozen rotated int8 base
@@ -15,7 +16,7 @@ The compute lives in ``libsdnq.so`` (hand-written CUDA behind the C ABI of
 ``linear`` composes the online path (rotate + quantize, then the int8 linear).
 """
 from ._native import (SdnqError, lib, sdnq_device_status, sdnq_gelu_bf16, sdnq_int8_linear,
-                      sdnq_int8_grad_input_gemm, sdnq_int8_linear_gelu,
+                      sdnq_int8_grad_input_gemm, sdnq_int8_linear_fused, sdnq_int8_linear_gelu,
                       sdnq_int8_linear_grad_input, sdnq_int8_linear_lora,
                       sdnq_int8_linear_lora_noalloc, sdnq_rotate_quant_weight,
                       sdnq_quant_grad_output, sdnq_rotquant_act, sdnq_selftest_wait_timeout,
@@ -23,7 +24,8 @@ from ._native import (SdnqError, lib, sdnq_device_status, sdnq_gelu_bf16, sdnq_i
 
 __all__ = [
     "SdnqError", "lib", "linear", "sdnq_device_status", "sdnq_gelu_bf16", "sdnq_int8_linear",
-    "sdnq_int8_grad_input_gemm", "sdnq_int8_linear_gelu", "sdnq_int8_linear_grad_input",
+    "sdnq_int8_grad_input_gemm", "sdnq_int8_linear_fused", "sdnq_int8_linear_gelu",
+    "sdnq_int8_linear_grad_input",
     "sdnq_int8_linear_lora", "sdnq_quant_grad_output",
     "sdnq_int8_linear_lora_noalloc",
     "sdnq_rotate_quant_weight", "sdnq_rotquant_act", "sdnq_selftest_wait_timeout",
@@ -37,10 +39,10 @@ def linear(x, qW, sW, group=256, bias=None, lora=None, gelu=False, out=None, str
     output inside the GEMM epilogue (not combined with ``lora``)."""
     if gelu and lora is not None:
         raise ValueError("gelu with lora is not provided")
+    if not gelu and lora is None:
+        return sdnq_int8_linear_fused(x, group, qW, sW, bias, out=out, stream=stream)
     qx, sx = sdnq_rotquant_act(x, group, stream=stream)
     if gelu:
         return sdnq_int8_linear_gelu(qx, sx, qW, sW, bias, out=out, stream=stream)
-    if lora is None:
-        return sdnq_int8_linear(qx, sx, qW, sW, bias, out=out, stream=stream)
     A, B, scale = lora
     return sdnq_int8_linear_lora(qx, sx, qW, sW, bias, x, A, B, scale, out=out, stream=stream)

@@ -41,6 +41,8 @@ SIGNATURES = {
     "sdnq_rotquant_act": [_P, _I64, _I64, _I64, _I32, _P, _P, _P],
     "sdnq_int8_linear": [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _I64, _P, _P],
     "sdnq_int8_linear_gelu": [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _I64, _P, _P],
+    "sdnq_int8_linear_fused": [_P, _I64, _I32, _P, _P, _P, _I64, _I64, _I64, _P, _P, _P, _P, _I64,
+                               _P, _I32, _P],
     "sdnq_int8_linear_grad_input": [_P, _I64, _P, _P, _I64, _I64, _I64, _I32, _P, _P, _P, _I64,
                                     _P, _P],
     "sdnq_quant_grad_output": [_P, _I64, _P, _I64, _I64, _P, _P, _P],
@@ -183,6 +185,55 @@ def _linear_call(name, qx, sx, qW, sW, bias, out, acc_out, stream):
 def sdnq_int8_linear(qx, sx, qW, sW, bias=None, out=None, acc_out=None, stream=None):
     """out [M, N] bf16 = bf16(float(qx qW^T) * (sx sW^T) + bias)."""
     return _linear_call("sdnq_int8_linear", qx, sx, qW, sW, bias, out, acc_out, stream)
+
+
+def fused_sync_words(M: int) -> int:
+    return 2 * ((M + 127) // 128)
+
+
+_SYNC_CACHE = {}
+
+
+def _sync_buffer(device, stream_handle: int, M: int):
+    """A zeroed counter buffer for sdnq_int8_linear_fused, one per (device, stream); the
+    kernel leaves it zero after every successful call, so it is reused as it is."""
+    key = (device.index, stream_handle)
+    need = fused_sync_words(M)
+    buf = _SYNC_CACHE.get(key)
+    if buf is None or buf.numel() < need:
+        buf = torch.zeros(max(need, 256), dtype=torch.int32, device=device)
+        _SYNC_CACHE[key] = buf
+    return buf
+
+
+FUSE_AUTO, FUSE_ALWAYS, FUSE_NEVER = 0, 1, 2
+
+
+def sdnq_int8_linear_fused(x, group: int, qW, sW, bias=None, qx_ws=None, sx_ws=None,
+                           sync_ws=None, out=None, acc_out=None, policy: int = FUSE_AUTO,
+                           stream=None):
+    """out [M, N] bf16 = the rotated int8 linear of x [M, K] bf16, in one launch (activation
+    quantizer inside the GEMM kernel) when ``policy`` and the shape call for it, else in two.
+    qx_ws / sx_ws receive the activation codes and scales."""
+    _req(x, torch.bfloat16, "x", 2)
+    _req(qW, torch.int8, "qW", 2)
+    _dense(qW, "qW")
+    M, K = x.shape
+    N = qW.shape[0]
+    if qW.shape[1] != K:
+        raise ValueError("x and qW disagree on K")
+    dev = x.device
+    qx_ws = torch.empty((M, K), dtype=torch.int8, device=dev) if qx_ws is None else qx_ws
+    sx_ws = torch.empty((M,), dtype=torch.float32, device=dev) if sx_ws is None else sx_ws
+    st = _stream(stream)
+    if sync_ws is None:
+        sync_ws = _sync_buffer(dev, st.value or 0, M)
+    out = _rows_out(M, N, torch.bfloat16, dev) if out is None else out
+    _check(lib().sdnq_int8_linear_fused(_ptr(x), x.stride(0), group, _ptr(qW), _ptr(sW),
+                                        _ptr(bias), M, N, K, _ptr(qx_ws), _ptr(sx_ws),
+                                        _ptr(sync_ws), _ptr(out), out.stride(0), _ptr(acc_out),
+                                        int(policy), st), "sdnq_int8_linear_fused")
+    return out
 
 
 def sdnq_int8_linear_gelu(qx, sx, qW, sW, bias=None, out=None, acc_out=None, stream=None):

@@ -92,6 +92,48 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
 }
 
 // ---------------------------------------------------------------------------------------
+// Counters in global memory between the CTAs of one co-resident (cooperative) grid
+
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t *p)
+{
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void red_add_release_gpu(uint32_t *p, uint32_t v)
+{
+    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Orders this thread's generic-proxy global accesses with its later async-proxy (TMA) ones.
+__device__ __forceinline__ void fence_proxy_async_global()
+{
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// Waits until *p >= target (acquire). Gives up like mbar_wait_bounded.
+__device__ __forceinline__ bool wait_count_bounded(const uint32_t *p, uint32_t target,
+                                                   volatile int *abort, uint64_t limit_ns)
+{
+    if (ld_acquire_gpu(p) >= target)
+        return true;
+    const uint64_t t0 = global_timer_ns();
+    for (;;) {
+        __nanosleep(100);
+        if (ld_acquire_gpu(p) >= target)
+            return true;
+        if (*abort)
+            return false;
+        if (global_timer_ns() - t0 > limit_ns) {
+            *abort = 1;
+            atomicOr(&g_device_error, kDevTimeout);
+            return false;
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------------------
 // TMA: 2-D tiled bulk tensor copy global -> shared, completion counted in bytes on an
 // mbarrier. The innermost coordinate times the element size is always a multiple of 16
 // bytes at every call site.

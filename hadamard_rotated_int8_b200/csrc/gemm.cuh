@@ -29,6 +29,11 @@
 
 #include "device.cuh"
 #include "gelu.cuh"
+#include "rotquant.cuh"
+
+#ifndef SDNQ_FUSED_QUANT_WARPS
+#define SDNQ_FUSED_QUANT_WARPS 8
+#endif
 
 namespace sdnq {
 
@@ -47,9 +52,14 @@ struct GemmParams {
     float lora_scale;
     float c_g;                // input-gradient mode: fp32(1/sqrt(g))
     uint64_t timeout_ns;
+    // fused activation quantizer: rq quantizes x into the A operand (rq.q) and its scales
+    // (rq.s, = sx); sync holds 2 * num_m_blocks counters, zero on entry and on exit
+    RotquantParams rq;
+    uint32_t *sync;
+    int32_t num_n_blocks;
 };
 
-template <int BN, bool LORA, bool GELU = false>
+template <int BN, bool LORA, bool GELU = false, bool FUSE = false>
 struct GemmConfig {
     static constexpr int BM = 128;
     static constexpr int BK = 128;                     // bytes of K per stage (int8)
@@ -60,7 +70,8 @@ struct GemmConfig {
     static constexpr int ACC_COLS = LORA ? 2 * BN : BN;   // TMEM columns per buffer
     static constexpr int NBUF = 512 / ACC_COLS >= 2 ? 2 : 1;  // accumulator buffers
     static constexpr int TMEM_COLS = NBUF * ACC_COLS;
-    static constexpr int THREADS = 320;               // 2 + 8 warps
+    static constexpr int QUANT_WARPS = FUSE ? SDNQ_FUSED_QUANT_WARPS : 0;  // fused quantizer
+    static constexpr int THREADS = 320 + 32 * (FUSE ? QUANT_WARPS + 1 : 0);  // 2 + 8 (+ 8 + 1) warps
     static constexpr int EPI_WARPS = 8;
     static constexpr int EPI_COLS = BN / 2;           // columns per epilogue warp
     // per epilogue warp: an output staging block [32 rows x 32 bf16] written with the
@@ -71,9 +82,14 @@ struct GemmConfig {
     static constexpr int SCALE_BYTES = EPI_COLS * 8;  // sw[EPI_COLS], bias[EPI_COLS]
     static constexpr int LUT_OFF = SCALE_OFF + EPI_WARPS * SCALE_BYTES;  // GELU table
     static constexpr int LUT_BYTES = GELU ? kGeluLutBytes : 0;
-    static constexpr int BAR_OFF = LUT_OFF + LUT_BYTES;
-    // barriers: full[S], empty[S], tfull[2], tempty[2], drain; then tmem base + abort flag
-    static constexpr int BAR_BYTES = (2 * STAGES + 5) * 8;
+    static constexpr int SX_OFF = LUT_OFF + LUT_BYTES;    // fused: row scales per buffer
+    static constexpr int SX_BYTES = FUSE ? 2 * 128 * 4 : 0;
+    static constexpr int AMAX_OFF = SX_OFF + SX_BYTES;     // fused: quantizer row maxima
+    static constexpr int AMAX_BYTES = FUSE ? 2 * QUANT_WARPS * 4 : 0;
+    static constexpr int BAR_OFF = AMAX_OFF + AMAX_BYTES;
+    // barriers: full[S], empty[S], tfull[2], tempty[2], drain, sxfull[2]; then tmem base +
+    // abort flag
+    static constexpr int BAR_BYTES = (2 * STAGES + 7) * 8;
     static constexpr int SMEM_BYTES = 1024 /*align slack*/ + BAR_OFF + BAR_BYTES + 16;
     static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
     static_assert(TMEM_COLS <= 512, "tensor memory holds 512 columns");
@@ -262,13 +278,15 @@ __device__ __forceinline__ void grad_epilogue_tile(uint32_t t_row, int half, int
     }
 }
 
-template <int BN, bool LORA, bool GELU, int GRAD_G>
-__global__ void __launch_bounds__(320, 1)
+template <int BN, bool LORA, bool GELU, int GRAD_G, int FUSE_G>
+__global__ void __launch_bounds__(GemmConfig<BN, LORA, GELU, (FUSE_G > 0)>::THREADS, 1)
     gemm_s8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CUtensorMap tmL,
                    const __grid_constant__ CUtensorMap tmO, const GemmParams p)
 {
-    using C = GemmConfig<BN, LORA, GELU>;
+    using C = GemmConfig<BN, LORA, GELU, (FUSE_G > 0)>;
+    static_assert(FUSE_G == 0 || (BN == 256 && !LORA && !GELU && GRAD_G == 0),
+                  "fused activation quantizer: plain forward tiles of 256 columns");
     static_assert(GRAD_G == 0 || (BN == 256 && !LORA && !GELU && (GRAD_G & (GRAD_G - 1)) == 0 &&
                                   GRAD_G <= 256),
                   "input-gradient mode: plain tiles of 256 columns, G divides 256");
@@ -283,6 +301,13 @@ __global__ void __launch_bounds__(320, 1)
     auto tfull_bar = [&](int b) { return bar0 + 8u * (2 * C::STAGES + b); };
     auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * C::STAGES + 2 + b); };
     const uint32_t drain_bar = bar0 + 8u * (2 * C::STAGES + 4);
+    auto sxfull_bar = [&](int b) { return bar0 + 8u * (2 * C::STAGES + 5 + b); };
+    float *sx_smem = reinterpret_cast<float *>(smem + C::SX_OFF);     // [2][128], fused only
+    float *amax_smem = reinterpret_cast<float *>(smem + C::AMAX_OFF); // [2][8], fused only
+    // tile -> (m block, n block): m fastest; n fastest with the fused quantizer, whose row
+    // blocks become ready in order
+    auto tile_mb = [&](int tile) { return FUSE_G > 0 ? tile / p.num_n_blocks : tile % p.num_m_blocks; };
+    auto tile_nb = [&](int tile) { return FUSE_G > 0 ? tile % p.num_n_blocks : tile / p.num_m_blocks; };
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C::BAR_OFF + C::BAR_BYTES);
     volatile int *abort = reinterpret_cast<volatile int *>(tmem_holder + 1);
 
@@ -299,6 +324,9 @@ __global__ void __launch_bounds__(320, 1)
             mbar_init(tempty_bar(b), C::EPI_WARPS);
         }
         mbar_init(drain_bar, 1);
+        if (FUSE_G > 0)
+            for (int b = 0; b < C::NBUF; ++b)
+                mbar_init(sxfull_bar(b), 1);
         *abort = 0;
         fence_mbar_init();
         prefetch_tensormap(&tmA);
@@ -325,9 +353,21 @@ __global__ void __launch_bounds__(320, 1)
             uint32_t phase = 0;
             int issued = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
-                const int m0 = (tile % p.num_m_blocks) * C::BM;
-                const int n0 = (tile / p.num_m_blocks) * BN;
+            int local = 0;
+            for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x, ++local) {
+                const int m0 = tile_mb(tile) * C::BM;
+                const int n0 = tile_nb(tile) * BN;
+                if constexpr (FUSE_G > 0) {
+                    // the scale warp has seen the tile's activation rows published (and copied
+                    // their scales); order that before the TMA engine reads the rows
+                    const int buf = local % C::NBUF;
+                    const uint32_t use = static_cast<uint32_t>(local / C::NBUF);
+                    if (!mbar_wait_bounded(sxfull_bar(buf), use & 1u, abort, p.timeout_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    fence_proxy_async_global();
+                }
                 const int steps = p.num_kb + (LORA ? p.lora_chunks : 0);
                 for (int kb = 0; kb < steps; ++kb) {
                     if (!mbar_wait_bounded(empty_bar(stage), phase ^ 1u, abort, p.timeout_ns)) {
@@ -452,6 +492,51 @@ __global__ void __launch_bounds__(320, 1)
             volatile int no_abort = 0;
             mbar_wait_bounded(drain_bar, 0u, &no_abort, p.timeout_ns);
         }
+    } else if (FUSE_G > 0 && warp == 10 + C::QUANT_WARPS) {
+        // ------------------------------------------------------------ scale warp (fused)
+        // Per tile of this CTA, ahead of the producer: wait (bounded, acquire) until the
+        // tile's 128 activation rows are published, count this CTA as one of the block's
+        // readers (the last one clears the block's counters for the next launch), wait until
+        // the epilogue has released the buffer's scales, copy the rows' scales to shared
+        // memory and arrive on sxfull, which both the producer and the epilogue wait for.
+        if constexpr (FUSE_G > 0) {
+            int local = 0;
+            for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++local) {
+                const int mb = tile_mb(tile);
+                const int m0 = mb * C::BM;
+                const int buf = local % C::NBUF;
+                const uint32_t use = static_cast<uint32_t>(local / C::NBUF);
+                const uint32_t rows = static_cast<uint32_t>(p.M - m0 < 128 ? p.M - m0 : 128);
+                bool good = true;
+                if (lane == 0) {
+                    good = wait_count_bounded(p.sync + mb, rows * static_cast<uint32_t>(p.rq.wpr),
+                                              abort, p.timeout_ns);
+                    if (good) {
+                        const uint32_t seen = atomicAdd(p.sync + p.num_m_blocks + mb, 1u);
+                        if (seen == static_cast<uint32_t>(p.num_n_blocks) - 1u) {
+                            p.sync[mb] = 0u;
+                            p.sync[p.num_m_blocks + mb] = 0u;
+                        }
+                        good = mbar_wait_bounded(tempty_bar(buf), (use & 1u) ^ 1u, abort,
+                                                 p.timeout_ns);
+                    }
+                }
+                if (__shfl_sync(0xffffffffu, good ? 1 : 0, 0) == 0)
+                    break;
+                for (int i = static_cast<int>(lane); i < 128; i += 32)
+                    sx_smem[buf * 128 + i] = m0 + i < p.M ? p.rq.s[m0 + i] : 0.0f;
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(sxfull_bar(buf));
+            }
+        }
+    } else if (FUSE_G > 0 && warp >= 10) {
+        // ------------------------------------------------------------ activation quantizer
+        // (warps 10..17): rows of x -> rotated int8 codes (the A operand) and their scales,
+        // published per 128-row block for the scale warps of every CTA
+        if constexpr (FUSE_G > 0)
+            rotquant_worker_rows<FUSE_G>(p.rq, static_cast<int32_t>(warp) - 10, C::QUANT_WARPS, 6u,
+                                         amax_smem, p.sync);
     } else {
         // ------------------------------------------------------------ epilogue (warps 2..9)
         const uint32_t quad = warp & 3u;  // TMEM lanes this warp may access: 32*quad ..
@@ -473,8 +558,8 @@ __global__ void __launch_bounds__(320, 1)
         for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++local) {
             const int buf = local % C::NBUF;
             const uint32_t use = static_cast<uint32_t>(local / C::NBUF);
-            const int m0 = (tile % p.num_m_blocks) * C::BM;
-            const int n0 = (tile / p.num_m_blocks) * BN;
+            const int m0 = tile_mb(tile) * C::BM;
+            const int n0 = tile_nb(tile) * BN;
             const int nw = n0 + col_base;     // first column of this warp
             // this warp's column scales and bias -> shared memory (fp32), before the wait
             // on the accumulator so that their latency overlaps the MMAs
@@ -520,7 +605,16 @@ __global__ void __launch_bounds__(320, 1)
             tc_fence_after_sync();
             const int m = m0 + row_in_tile;
             const bool row_ok = m < p.M;
-            const float sxm = row_ok ? p.sx[m] : 0.0f;
+            float sxm;
+            if constexpr (FUSE_G > 0) {
+                // the row scales the producer copied once the rows were published
+                const bool got = mbar_wait_bounded(sxfull_bar(buf), use & 1u, abort, p.timeout_ns);
+                if (!__all_sync(0xffffffffu, got))
+                    break;
+                sxm = row_ok ? sx_smem[buf * 128 + row_in_tile] : 0.0f;
+            } else {
+                sxm = row_ok ? p.sx[m] : 0.0f;
+            }
             const uint32_t t_row = tmem_base + ((quad * 32u) << 16) + buf * C::ACC_COLS;
             if constexpr (GRAD_G > 0) {
                 int32_t *acc_row = (p.acc_out != nullptr && row_ok)

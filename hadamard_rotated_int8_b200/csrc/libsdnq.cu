@@ -236,12 +236,16 @@ sdnq_status validate_linear(const void *qx, const void *sx, const void *qW, cons
 
 // GRAD_G > 0: the input gradient's NN product, out [M, N] = epilogue(A [M, K] x W [K, N]),
 // with W = the weight codes qW [N_out = K rows, K_in = N columns] read N-major.
-template <int BN, bool LORA, bool GELU = false, int GRAD_G = 0>
+// FUSE_G > 0: the activation quantizer runs inside the kernel (p.rq, p.sync set by the
+// caller); the grid is launched cooperatively so that every CTA is resident, because the
+// producers of one CTA wait for rows that the quantizer warps of others publish.
+template <int BN, bool LORA, bool GELU = false, int GRAD_G = 0, int FUSE_G = 0>
 sdnq_status launch_gemm(const DeviceInfo &dev, const int8_t *qx, const int8_t *qW,
                         const uint16_t *u, const uint16_t *B, int32_t rank, GemmParams p,
                         cudaStream_t cs)
 {
-    using C = GemmConfig<BN, LORA, GELU>;
+    using C = GemmConfig<BN, LORA, GELU, (FUSE_G > 0)>;
+    constexpr auto kernel = gemm_s8_kernel<BN, LORA, GELU, GRAD_G, FUSE_G>;
     CUtensorMap tmA, tmB, tmU, tmL, tmO;
     const bool b_ok = GRAD_G > 0
                           ? make_tmap_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, qW, p.N, p.K, p.N, 128, 128)
@@ -260,15 +264,33 @@ sdnq_status launch_gemm(const DeviceInfo &dev, const int8_t *qx, const int8_t *q
     }
     static std::once_flag once;
     static bool smem_ok = false;
-    std::call_once(once, [] { smem_ok = set_smem(gemm_s8_kernel<BN, LORA, GELU, GRAD_G>, C::SMEM_BYTES); });
+    std::call_once(once, [] { smem_ok = set_smem(kernel, C::SMEM_BYTES); });
     if (!smem_ok)
         return SDNQ_ERR_CUDA;
     p.num_kb = (p.K + C::BK - 1) / C::BK;
     p.num_m_blocks = (p.M + C::BM - 1) / C::BM;
-    p.num_tiles = p.num_m_blocks * ((p.N + BN - 1) / BN);
+    p.num_n_blocks = (p.N + BN - 1) / BN;
+    p.num_tiles = p.num_m_blocks * p.num_n_blocks;
     const int grid = p.num_tiles < dev.sm_count ? p.num_tiles : dev.sm_count;
     cudaGetLastError();
-    gemm_s8_kernel<BN, LORA, GELU, GRAD_G><<<grid, C::THREADS, C::SMEM_BYTES, cs>>>(tmA, tmB, tmU, tmL, tmO, p);
+    if constexpr (FUSE_G > 0) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>(grid));
+        cfg.blockDim = dim3(C::THREADS);
+        cfg.dynamicSmemBytes = C::SMEM_BYTES;
+        cfg.stream = cs;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeCooperative;
+        attr[0].val.cooperative = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (cudaLaunchKernelEx(&cfg, kernel, tmA, tmB, tmU, tmL, tmO, p) != cudaSuccess) {
+            cudaGetLastError();
+            return SDNQ_ERR_CUDA;
+        }
+    } else {
+        kernel<<<grid, C::THREADS, C::SMEM_BYTES, cs>>>(tmA, tmB, tmU, tmL, tmO, p);
+    }
     return launch_status();
 }
 
@@ -326,7 +348,7 @@ sdnq_status run_linear(const int8_t *qx, const float *sx, const int8_t *qW, cons
     if (M == 0)
         return SDNQ_OK;
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
-    GemmParams p;
+    GemmParams p = {};
     p.sx = sx;
     p.sw = sW;
     p.bias = bias;
@@ -354,6 +376,95 @@ sdnq_status run_linear(const int8_t *qx, const float *sx, const int8_t *qW, cons
         return st;
     p.lora_chunks = (rank + 63) / 64;
     return launch_gemm<SDNQ_LORA_BN, true>(dev, qx, qW, u_ws, B, rank, p, cs);
+}
+
+// ---------------------------------------------------------------- fused activation path
+
+// the quantizer warps hold at most this many 1024-element chunks of a row
+constexpr int kFusedMaxChunks = SDNQ_FUSED_QUANT_WARPS;
+
+template <int G>
+sdnq_status launch_linear_fused_g(const DeviceInfo &dev, GemmParams p, const int8_t *qW,
+                                  cudaStream_t cs)
+{
+    return launch_gemm<256, false, false, 0, G>(dev, p.rq.q, qW, nullptr, nullptr, 0, p, cs);
+}
+
+sdnq_status run_linear_fused(const uint16_t *x, int64_t ldx, int32_t group, const int8_t *qW,
+                             const float *sW, const uint16_t *bias, int64_t M, int64_t N,
+                             int64_t K, int8_t *qx_ws, float *sx_ws, uint32_t *sync_ws,
+                             uint16_t *out, int64_t ldo, int32_t *acc_out, int32_t policy,
+                             void *stream)
+{
+    if (policy < SDNQ_FUSE_AUTO || policy > SDNQ_FUSE_NEVER)
+        return SDNQ_ERR_UNSUPPORTED;
+    sdnq_status st = validate_rotquant(x, M, K, ldx, group, qx_ws, sx_ws);
+    if (st == SDNQ_OK)
+        st = validate_linear(qx_ws, sx_ws, qW, sW, bias, M, N, K, out, ldo, acc_out);
+    if (st != SDNQ_OK)
+        return st;
+    if (M != 0 && !sync_ws)
+        return SDNQ_ERR_NULL;
+    if (!aligned(sync_ws, 4))
+        return SDNQ_ERR_ALIGN;
+    DeviceInfo dev;
+    if ((st = current_device(&dev)) != SDNQ_OK)
+        return st;
+    if (M == 0)
+        return SDNQ_OK;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    const int32_t nchunks = static_cast<int32_t>((K + 1023) / 1024);
+    // The one-launch kernel overlaps the quantizer with the GEMM; it pays off once the GEMM
+    // has at least three waves of tiles (with fewer, its first wave needs most rows before
+    // it can start). Rows longer than the quantizer warps can hold take the two launches.
+    const int64_t tiles = ((M + 127) / 128) * ((N + 255) / 256);
+    const bool fuse = nchunks <= kFusedMaxChunks &&
+                      (policy == SDNQ_FUSE_ALWAYS ||
+                       (policy == SDNQ_FUSE_AUTO && tiles >= 3ll * dev.sm_count));
+    if (!fuse) {
+        // the two launches (same results)
+        if ((st = launch_rowquant(x, M, K, ldx, group, nullptr, qx_ws, sx_ws, dev, cs)) != SDNQ_OK)
+            return st;
+        return run_linear(qx_ws, sx_ws, qW, sW, bias, nullptr, 0, nullptr, nullptr, 0, 0.0f,
+                          nullptr, M, N, K, out, ldo, acc_out, stream, false);
+    }
+    GemmParams p = {};
+    p.sx = sx_ws;
+    p.sw = sW;
+    p.bias = bias;
+    p.out = out;
+    p.ldo = ldo;
+    p.acc_out = acc_out;
+    p.M = static_cast<int32_t>(M);
+    p.N = static_cast<int32_t>(N);
+    p.K = static_cast<int32_t>(K);
+    p.lora_chunks = 0;
+    p.lora_scale = 0.0f;
+    p.c_g = 1.0f;
+    p.timeout_ns = kDefaultTimeoutNs;
+    p.sync = sync_ws;
+    RotquantParams &q = p.rq;
+    q.x = x;
+    q.ldx = ldx;
+    q.q = qx_ws;
+    q.s = sx_ws;
+    q.M = M;
+    q.K = static_cast<int32_t>(K);
+    q.nchunks = nchunks;
+    q.wpr = nchunks;
+    q.rpc = 1;  // rows per group: a power of two (so a group never straddles a 128-row block)
+    while (2 * q.rpc * nchunks <= SDNQ_FUSED_QUANT_WARPS)
+        q.rpc *= 2;
+    q.c_g = static_cast<float>(1.0 / std::sqrt(static_cast<double>(group)));
+    q.colscale = nullptr;
+    switch (group) {
+    case 8: return launch_linear_fused_g<8>(dev, p, qW, cs);
+    case 16: return launch_linear_fused_g<16>(dev, p, qW, cs);
+    case 32: return launch_linear_fused_g<32>(dev, p, qW, cs);
+    case 64: return launch_linear_fused_g<64>(dev, p, qW, cs);
+    case 128: return launch_linear_fused_g<128>(dev, p, qW, cs);
+    default: return launch_linear_fused_g<256>(dev, p, qW, cs);
+    }
 }
 
 // ---------------------------------------------------------------- input gradient
@@ -397,7 +508,7 @@ sdnq_status launch_grad_gemm(const DeviceInfo &dev, const int8_t *qg, const floa
                              const int8_t *qW, int64_t M, int64_t N, int64_t K, int32_t group,
                              uint16_t *dx, int64_t lddx, int32_t *acc_out, cudaStream_t cs)
 {
-    GemmParams p;
+    GemmParams p = {};
     p.sx = sg;
     p.sw = nullptr;    // not read in this mode
     p.bias = nullptr;
@@ -512,6 +623,17 @@ SDNQ_API sdnq_status sdnq_int8_linear(const int8_t *qx, const float *sx, const i
 {
     return run_linear(qx, sx, qW, sW, bias, nullptr, 0, nullptr, nullptr, 0, 0.0f, nullptr, M, N, K,
                       out, ldo, acc_out, stream, false);
+}
+
+SDNQ_API sdnq_status sdnq_int8_linear_fused(const uint16_t *x, int64_t ldx, int32_t group,
+                                            const int8_t *qW, const float *sW,
+                                            const uint16_t *bias, int64_t M, int64_t N, int64_t K,
+                                            int8_t *qx_ws, float *sx_ws, uint32_t *sync_ws,
+                                            uint16_t *out, int64_t ldo, int32_t *acc_out,
+                                            int32_t policy, void *stream)
+{
+    return run_linear_fused(x, ldx, group, qW, sW, bias, M, N, K, qx_ws, sx_ws, sync_ws, out, ldo,
+                            acc_out, policy, stream);
 }
 
 SDNQ_API sdnq_status sdnq_int8_linear_gelu(const int8_t *qx, const float *sx, const int8_t *qW,

@@ -288,6 +288,80 @@ __device__ __forceinline__ void load_raw(const uint16_t *xr, int32_t K, int32_t 
     }
 }
 
+// The persistent loop below run by `nw` warps inside another kernel (the fused activation
+// quantizer of the int8 GEMM): warp w of the group is `warp`, the group synchronises on named
+// barrier `bar_id` (32 * nw threads) and exchanges row maxima through s_amax[2][nw] in shared
+// memory. Warps beyond wpr * rpc only take part in the barriers. Rows are published per
+// 128-row block: ready[b] counts wpr per stored row of block b (a row group never straddles
+// a block, since rpc divides 128). One lane of the group's last warp adds a whole row group
+// with release semantics once the next barrier shows every warp past its stores, so that one
+// thread, not every warp, waits on the release.
+template <int G>
+__device__ __forceinline__ void rotquant_worker_rows(const RotquantParams &p, int32_t warp,
+                                                     int32_t nw, uint32_t bar_id, float *s_amax,
+                                                     uint32_t *ready)
+{
+    const uint32_t lane = lane_id();
+    const int32_t r_local = warp / p.wpr;
+    const int32_t wr = warp - r_local * p.wpr;
+    const bool active = r_local < p.rpc;
+    const bool has_chunk = active && wr < p.nchunks;
+    const int64_t n_groups = (p.M + p.rpc - 1) / p.rpc;
+    const bool signaller = warp == nw - 1 && lane == 0;
+    auto publish = [&](int64_t group) {
+        const int64_t r0 = group * p.rpc;
+        const int64_t rows = p.M - r0 < p.rpc ? p.M - r0 : p.rpc;
+        red_add_release_gpu(ready + (r0 >> 7), static_cast<uint32_t>(rows * p.wpr));
+    };
+
+    int64_t rg = blockIdx.x;
+    int64_t prev = -1;  // row group stored in the previous iteration, not yet published
+    uint4 raw[4];
+    {
+        const int64_t row = rg * p.rpc + r_local;
+        const bool ok = rg < n_groups && row < p.M && has_chunk;
+        load_raw(p.x + (ok ? row : 0) * p.ldx, p.K, wr, ok, lane, raw);
+    }
+    for (int parity = 0; rg < n_groups; rg += gridDim.x, parity ^= 1) {
+        const int64_t row = rg * p.rpc + r_local;
+        const bool row_ok = active && row < p.M;
+        float v[4][8];
+#pragma unroll
+        for (int t = 0; t < 4; ++t)
+            bf16x8_to_f32(raw[t], v[t]);
+        {
+            const int64_t nrg = rg + gridDim.x;
+            const int64_t nrow = nrg * p.rpc + r_local;
+            const bool ok = nrg < n_groups && nrow < p.M && has_chunk;
+            load_raw(p.x + (ok ? nrow : 0) * p.ldx, p.K, wr, ok, lane, raw);
+        }
+        chunk_butterfly<G>(v, lane);
+        float amax = chunk_absmax(v);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1)
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+        if (lane == 0)
+            s_amax[parity * nw + warp] = amax;
+        asm volatile("bar.sync %0, %1;" ::"r"(bar_id), "r"(32 * nw) : "memory");
+        if (signaller && prev >= 0)
+            publish(prev);  // every warp is past the stores of row group `prev`
+        amax = 0.0f;
+        if (active)
+            for (int32_t w = 0; w < p.wpr; ++w)
+                amax = fmaxf(amax, s_amax[parity * nw + r_local * p.wpr + w]);
+        const float s_z = __fdiv_rn(amax, 127.0f);
+        const bool zero = !(amax > 0.0f);
+        if (row_ok && wr == 0 && lane == 0)
+            p.s[row] = zero ? 0.0f : __fmul_rn(s_z, p.c_g);
+        int8_t *qr = p.q + (row_ok ? row : 0) * static_cast<int64_t>(p.K);
+        quant_store_chunk(v, qr, p.K, wr, row_ok && has_chunk, lane, s_z, zero);
+        prev = rg;
+    }
+    asm volatile("bar.sync %0, %1;" ::"r"(bar_id), "r"(32 * nw) : "memory");
+    if (signaller && prev >= 0)
+        publish(prev);
+}
+
 // Rows of at most 16 chunks (K <= 16384): each warp owns one chunk of a row, a CTA owns
 // `rpc` rows at a time and walks row groups persistently, loading the next row group into
 // registers while it rotates and quantizes the current one.

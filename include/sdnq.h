@@ -112,6 +112,35 @@ sdnq_status sdnq_int8_linear(const int8_t *qx, const float *sx, const int8_t *qW
                              void *stream);
 
 /*
+ * The online path in one launch: sdnq_rotquant_act of x followed by sdnq_int8_linear, with
+ * the activation rotate + quantize running inside the GEMM kernel on warps of its own (rows
+ * are published per 128-row block; the tile loads wait for their block). Results are bit
+ * for bit those of the two calls, which is also what the call runs when `policy` asks for it
+ * or when the one launch does not pay off:
+ *   policy SDNQ_FUSE_AUTO: one launch when the GEMM has at least three waves of 128 x 256
+ *          tiles (ceil(M/128) * ceil(N/256) >= 3 * SM count) and K <= 8192, else two;
+ *   policy SDNQ_FUSE_ALWAYS: one launch whenever K <= 8192;  SDNQ_FUSE_NEVER: two launches.
+ *   x [M, K] bf16, row stride ldx; group as in sdnq_rotquant_act.
+ *   qW, sW, bias, out, ldo, acc_out as in sdnq_int8_linear.
+ *   qx_ws [M, K] int8 dense, sx_ws [M] fp32: caller-provided workspace for the activation
+ *   codes and scales (they hold them afterwards).
+ *   sync_ws: SDNQ_FUSED_SYNC_WORDS(M) uint32 counters, 4-byte aligned, which must be zero on
+ *   entry; a call that returns SDNQ_OK with no device error leaves them zero again, so one
+ *   zeroed buffer serves every later call on the same stream. Calls whose kernels overlap on
+ *   the GPU need separate buffers. After a device timeout (sdnq_device_status) re-zero it.
+ *   The two launches leave sync_ws untouched.
+ *   The kernel is a cooperative launch (one CTA per SM, all resident at once); if the device
+ *   cannot run it, the call returns SDNQ_ERR_CUDA.
+ */
+#define SDNQ_FUSED_SYNC_WORDS(M) (2 * (((M) + 127) / 128))
+enum { SDNQ_FUSE_AUTO = 0, SDNQ_FUSE_ALWAYS = 1, SDNQ_FUSE_NEVER = 2 };
+sdnq_status sdnq_int8_linear_fused(const uint16_t *x, int64_t ldx, int32_t group,
+                                   const int8_t *qW, const float *sW, const uint16_t *bias,
+                                   int64_t M, int64_t N, int64_t K, int8_t *qx_ws, float *sx_ws,
+                                   uint32_t *sync_ws, uint16_t *out, int64_t ldo,
+                                   int32_t *acc_out, int32_t policy, void *stream);
+
+/*
  * sdnq_int8_linear with GELU fused into its epilogue, for the up-projection of a DiT MLP
  * whose output feeds the down-projection's rotate + quantize:
  *   out = gelu(bf16(float(acc) * (sx * sw) [+ bias])), GELU(y) = y * Phi(y) in the exact

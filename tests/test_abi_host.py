@@ -149,6 +149,23 @@ def test_grad_input_validation(lib):
     assert grad(lib, acc=A16 + 4) == _native.SDNQ_ERR_ALIGN
 
 
+def fused(lib, x=A16, ldx=256, g=256, sync=A16, qx=A16, sx=A16, out=A16, M=128, K=256, policy=0):
+    return lib.sdnq_int8_linear_fused(x, ldx, g, A16, A16, 0, M, 256, K, qx, sx, sync, out, 256,
+                                      0, policy, S)
+
+
+def test_fused_validation(lib):
+    assert fused(lib, x=0) == _native.SDNQ_ERR_NULL
+    assert fused(lib, sync=0) == _native.SDNQ_ERR_NULL
+    assert fused(lib, qx=0) == _native.SDNQ_ERR_NULL
+    assert fused(lib, sync=A16 + 2) == _native.SDNQ_ERR_ALIGN
+    assert fused(lib, g=48) == _native.SDNQ_ERR_UNSUPPORTED
+    assert fused(lib, ldx=128) == _native.SDNQ_ERR_SHAPE
+    assert fused(lib, K=200, ldx=200) == _native.SDNQ_ERR_SHAPE
+    assert fused(lib, x=MIS) == _native.SDNQ_ERR_ALIGN
+    assert fused(lib, policy=3) == _native.SDNQ_ERR_UNSUPPORTED
+
+
 def test_gelu_and_selftest_validation(lib):
     assert lib.sdnq_gelu_bf16(0, 4, 8, 8, A16, 8, S) == _native.SDNQ_ERR_NULL
     assert lib.sdnq_gelu_bf16(A16, 4, 0, 8, A16, 8, S) == _native.SDNQ_ERR_SHAPE
@@ -166,6 +183,7 @@ def test_valid_arguments_without_a_b200_are_refused(lib):
     assert lora(lib) == _native.SDNQ_ERR_UNSUPPORTED
     assert lib.sdnq_gelu_bf16(A16, 4, 8, 8, A16, 8, S) == _native.SDNQ_ERR_UNSUPPORTED
     assert grad(lib) == _native.SDNQ_ERR_UNSUPPORTED
+    assert fused(lib) == _native.SDNQ_ERR_UNSUPPORTED
 
 
 def test_binding_refuses_cpu_tensors(lib):
