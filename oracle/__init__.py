@@ -67,6 +67,11 @@ def _open(path: str):
         "oracle_lora_up": [P, P, I64, I64, I64, P, INT],
         "oracle_gelu_bf16": [P, I64, P, INT],
         "oracle_colscale_quantize": [P, I64, I64, I64, P, P, P, INT],
+        "oracle_e4m3_encode": [P, I64, P],
+        "oracle_e4m3_decode": [P, I64, P],
+        "oracle_rotate_quantize_fp8": [P, I64, I64, I64, I64, P, P, INT],
+        "oracle_gemm_fp8": [P, P, I64, I64, I64, P, INT],
+        "oracle_dequant_epilogue_f32": [P, P, P, P, I64, I64, P, INT],
         "oracle_gemm_s8_nn": [P, P, I64, I64, I64, P, INT],
         "oracle_grad_input_epilogue": [P, P, I64, I64, I64, P, INT],
     }
@@ -74,7 +79,8 @@ def _open(path: str):
         fn = getattr(lib, name)
         fn.argtypes = args
         fn.restype = None if name in ("oracle_bf16_to_f32", "oracle_f32_to_bf16",
-                                      "oracle_f64_to_bf16") else ctypes.c_int
+                                      "oracle_f64_to_bf16", "oracle_e4m3_encode",
+                                      "oracle_e4m3_decode") else ctypes.c_int
     return lib
 
 
@@ -325,3 +331,71 @@ def grad_input(dy_bits, qw, sw, g, nthreads: int | None = None):
     qg, sg = colscale_quantize(dy_bits, sw, nthreads)
     acc = gemm_s8_nn(qg, qw, nthreads)
     return {"qg": qg, "sg": sg, "acc": acc, "dx": grad_input_epilogue(acc, sg, g, nthreads)}
+
+
+# ---- FP8 (e4m3) variant ----------------------------------------------------------------
+
+def e4m3_encode(x) -> np.ndarray:
+    """fp32 values -> e4m3 codes (round to nearest, ties to even, saturating at +-448)."""
+    x = _c(x, np.float32)
+    out = np.empty(x.shape, np.uint8)
+    _load().oracle_e4m3_encode(_ptr(x), x.size, _ptr(out))
+    return out
+
+
+def e4m3_decode(c) -> np.ndarray:
+    c = _c(c, np.uint8)
+    out = np.empty(c.shape, np.float32)
+    _load().oracle_e4m3_decode(_ptr(c), c.size, _ptr(out))
+    return out
+
+
+def rotate_quantize_fp8(x_bits, g: int, nthreads: int | None = None):
+    """Rotate each row by H_g and quantize it to e4m3 with one fp32 scale per row (absmax
+    onto +-448). Returns (codes uint8 [rows, K], scales fp32 [rows])."""
+    x_bits = _c(x_bits, np.uint16)
+    rows, K = x_bits.shape
+    q = np.empty((rows, K), np.uint8)
+    s = np.empty((rows,), np.float32)
+    _check(_load().oracle_rotate_quantize_fp8(_ptr(x_bits), rows, K, K, g, _ptr(q), _ptr(s),
+                                              nthreads or default_threads()),
+           "rotate_quantize_fp8")
+    return q, s
+
+
+def gemm_fp8(a, b, nthreads: int | None = None) -> np.ndarray:
+    """acc[m, n] = fp32(sum_k dec(a[m, k]) dec(b[n, k])), summed in fp64."""
+    a = _c(a, np.uint8)
+    b = _c(b, np.uint8)
+    M, K = a.shape
+    N, K2 = b.shape
+    if K != K2:
+        raise ValueError("K mismatch")
+    acc = np.empty((M, N), np.float32)
+    _check(_load().oracle_gemm_fp8(_ptr(a), _ptr(b), M, N, K, _ptr(acc),
+                                   nthreads or default_threads()), "gemm_fp8")
+    return acc
+
+
+def dequant_epilogue_f32(acc, sx, sw, bias_bits=None, nthreads: int | None = None):
+    acc = _c(acc, np.float32)
+    sx = _c(sx, np.float32)
+    sw = _c(sw, np.float32)
+    M, N = acc.shape
+    out = np.empty((M, N), np.uint16)
+    bias_p = None
+    if bias_bits is not None:
+        bias_bits = _c(bias_bits, np.uint16)
+        bias_p = _ptr(bias_bits)
+    _check(_load().oracle_dequant_epilogue_f32(_ptr(acc), _ptr(sx), _ptr(sw), bias_p, M, N,
+                                               _ptr(out), nthreads or default_threads()),
+           "dequant_epilogue_f32")
+    return out
+
+
+def linear_fp8(x_bits, qw, sw, g, bias_bits=None, nthreads: int | None = None):
+    """The FP8 variant of ``linear``: every intermediate in a dict."""
+    qx, sx = rotate_quantize_fp8(x_bits, g, nthreads)
+    acc = gemm_fp8(qx, qw, nthreads)
+    return {"qx": qx, "sx": sx, "acc": acc,
+            "out": dequant_epilogue_f32(acc, sx, sw, bias_bits, nthreads)}

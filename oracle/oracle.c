@@ -418,3 +418,149 @@ int oracle_grad_input_epilogue(const int32_t *acc, const float *s, int64_t M, in
     }
     return err ? ORACLE_ERR_NOMEM : ORACLE_OK;
 }
+
+/* ---- FP8 (e4m3) variant of the rotated quantized matmul ----
+ * [SD] feature list and SDNQConfig (FP8 weights and FP8 quantized matmul beside INT8); the
+ * rotation is the same. e4m3 ("fn" flavour, as used for FP8 matmuls): 1 sign bit, 4 exponent
+ * bits with bias 7, 3 mantissa bits; normal values (1 + m/8) 2^(e-7) for e = 1..15 except
+ * e = 15, m = 7 (NaN), so the largest finite value is 448; subnormals (m/8) 2^-6; no
+ * infinities. Encoding rounds to nearest with ties to the even code and saturates finite
+ * values beyond 448 to +-448. */
+
+static uint8_t e4m3_encode(double v)
+{
+    if (v != v)
+        return 0x7f;
+    const uint8_t sign = (v < 0.0 || (v == 0.0 && signbit(v))) ? 0x80 : 0x00;
+    double a = fabs(v);
+    if (a >= 448.0)
+        return sign | 0x7e; /* saturate */
+    int e;
+    frexp(a, &e);               /* a = f 2^e with f in [0.5, 1): a in [2^(e-1), 2^e) */
+    int E = e - 1;              /* a in [2^E, 2^(E+1)) */
+    if (E < -6)
+        E = -6;                 /* subnormal range shares the quantum of binade -6 */
+    const double quantum = ldexp(1.0, E - 3);
+    double q = nearbyint(a / quantum) * quantum; /* exact scaling; ties to even multiple */
+    if (q >= 448.0)
+        q = 448.0;
+    if (q == 0.0)
+        return sign;
+    /* q is representable: split into exponent / mantissa fields */
+    int qe;
+    double qf = frexp(q, &qe);  /* q = qf 2^qe, qf in [0.5, 1) */
+    int biased = qe - 1 + 7;
+    if (biased >= 1) {
+        int m = (int)(qf * 16.0) - 8; /* (1 + m/8) = 2 qf */
+        return sign | (uint8_t)(biased << 3) | (uint8_t)m;
+    }
+    int m = (int)(q / ldexp(1.0, -9));  /* subnormal: q = m 2^-9 */
+    return sign | (uint8_t)m;
+}
+
+static double e4m3_decode(uint8_t c)
+{
+    const int s = c >> 7, e = (c >> 3) & 15, m = c & 7;
+    double v;
+    if (e == 15 && m == 7)
+        v = NAN;
+    else if (e == 0)
+        v = ldexp((double)m, -9);
+    else
+        v = ldexp(1.0 + m / 8.0, e - 7);
+    return s ? -v : v;
+}
+
+void oracle_e4m3_encode(const float *in, int64_t n, uint8_t *out)
+{
+    for (int64_t i = 0; i < n; i++)
+        out[i] = e4m3_encode((double)in[i]);
+}
+
+void oracle_e4m3_decode(const uint8_t *in, int64_t n, float *out)
+{
+    for (int64_t i = 0; i < n; i++)
+        out[i] = (float)e4m3_decode(in[i]);
+}
+
+/* Rotate + quantize to e4m3: the same butterfly and row absmax as the int8 path, then
+ * s_z = fp32(amax / 448), codes e4m3(fp32(z / s_z)), stored scale fp32(s_z * fp32(1/sqrt g)).
+ * An all-zero row gives s = 0 and codes +0. */
+int oracle_rotate_quantize_fp8(const uint16_t *x, int64_t rows, int64_t K, int64_t ldx,
+                               int64_t g, uint8_t *q, float *s, int nthreads)
+{
+    if (!x || !q || !s || rows < 0 || K <= 0 || ldx < K || !is_pow2(g) || K % g != 0)
+        return ORACLE_ERR_ARG;
+    const float c_g = (float)(1.0 / sqrt((double)g));
+    int err = 0;
+#pragma omp parallel for num_threads(nthreads > 0 ? nthreads : 1) schedule(static)
+    for (int64_t r = 0; r < rows; r++) {
+        float *z = (float *)malloc((size_t)K * sizeof(float));
+        if (!z) {
+#pragma omp atomic write
+            err = 1;
+            continue;
+        }
+        for (int64_t k = 0; k < K; k++)
+            z[k] = bf16_bits_to_f32(x[r * ldx + k]);
+        for (int64_t k0 = 0; k0 < K; k0 += g)
+            fwht_group_f32(z + k0, g);
+        float amax = 0.0f;
+        for (int64_t k = 0; k < K; k++) {
+            float a = fabsf(z[k]);
+            if (a > amax)
+                amax = a;
+        }
+        const float s_z = amax / 448.0f;
+        for (int64_t k = 0; k < K; k++) {
+            float t = (amax != 0.0f) ? z[k] / s_z : 0.0f; /* IEEE fp32 quotient */
+            q[r * K + k] = e4m3_encode((double)t);
+        }
+        s[r] = s_z * c_g;
+        free(z);
+    }
+    return err ? ORACLE_ERR_NOMEM : ORACLE_OK;
+}
+
+/* acc[m][n] = fp32( sum_k dec(a[m][k]) * dec(b[n][k]) ): every product is exact, the sum is
+ * taken in binary64 and rounded once. */
+int oracle_gemm_fp8(const uint8_t *a, const uint8_t *b, int64_t M, int64_t N, int64_t K,
+                    float *acc, int nthreads)
+{
+    if (!a || !b || !acc || M < 0 || N < 0 || K <= 0)
+        return ORACLE_ERR_ARG;
+    double lut[256];
+    for (int c = 0; c < 256; c++)
+        lut[c] = e4m3_decode((uint8_t)c);
+#pragma omp parallel for num_threads(nthreads > 0 ? nthreads : 1) schedule(static)
+    for (int64_t m = 0; m < M; m++) {
+        for (int64_t n = 0; n < N; n++) {
+            double sum = 0.0;
+            for (int64_t k = 0; k < K; k++)
+                sum += lut[a[m * K + k]] * lut[b[n * K + k]];
+            acc[m * N + n] = (float)sum;
+        }
+    }
+    return ORACLE_OK;
+}
+
+/* The fp32 de-quant epilogue on fp32 accumulators (same op order as the int8 one):
+ * t = sx*sw; v = acc*t; v = v + bias; out = bf16_rne(v). */
+int oracle_dequant_epilogue_f32(const float *acc, const float *sx, const float *sw,
+                                const uint16_t *bias, int64_t M, int64_t N, uint16_t *out,
+                                int nthreads)
+{
+    if (!acc || !sx || !sw || !out || M < 0 || N < 0)
+        return ORACLE_ERR_ARG;
+#pragma omp parallel for num_threads(nthreads > 0 ? nthreads : 1) schedule(static)
+    for (int64_t m = 0; m < M; m++) {
+        for (int64_t n = 0; n < N; n++) {
+            float t = sx[m] * sw[n];
+            float v = acc[m * N + n] * t;
+            if (bias)
+                v = v + bf16_bits_to_f32(bias[n]);
+            out[m * N + n] = f32_to_bf16_rne(v);
+        }
+    }
+    return ORACLE_OK;
+}

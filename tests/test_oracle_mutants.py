@@ -13,15 +13,16 @@ MUTANTS = {
         "float b = v[j + h];", "float b = v[j ^ (h >> 1)];",
         [lambda: pins.test_butterfly_equals_dense_product_on_integers(16)]),
     "normaliser not folded into the scale": (
-        "s[r] = s_z * c_g;", "s[r] = s_z;",
+        "qr[k] = (int8_t)code;\n        }\n        s[r] = s_z * c_g;",
+        "qr[k] = (int8_t)code;\n        }\n        s[r] = s_z;",
         [lambda: pins.test_codes_brute_force_g8(16)]),
     "round half away from zero": (
         "float n = nearbyintf(t);", "float n = roundf(t);",
         [lambda: pins.test_codes_brute_force_g8(32),
          lambda: pins.test_g1_is_textbook_per_row_absmax_int8()]),
     "absmax per group instead of per row": (
-        "        for (int64_t k0 = 0; k0 < K; k0 += g)\n            fwht_group_f32(z + k0, g);\n        float amax = 0.0f;\n        for (int64_t k = 0; k < K; k++) {",
-        "        for (int64_t k0 = 0; k0 < K; k0 += g)\n            fwht_group_f32(z + k0, g);\n        float amax = 0.0f;\n        for (int64_t k = 0; k < g; k++) {",
+        "z[k] = bf16_bits_to_f32(xr[k]);\n        for (int64_t k0 = 0; k0 < K; k0 += g)\n            fwht_group_f32(z + k0, g);\n        float amax = 0.0f;\n        for (int64_t k = 0; k < K; k++) {",
+        "z[k] = bf16_bits_to_f32(xr[k]);\n        for (int64_t k0 = 0; k0 < K; k0 += g)\n            fwht_group_f32(z + k0, g);\n        float amax = 0.0f;\n        for (int64_t k = 0; k < g; k++) {",
         [lambda: pins.test_golden_worked_rotquant()]),
     "grid 255 levels (range -128..127)": (
         "const float s_z = amax / 127.0f;", "const float s_z = amax / 127.5f;",
@@ -34,11 +35,12 @@ MUTANTS = {
         "float v = ((float)acc[m * N + n] * sx[m]) * sw[n];",
         [lambda: pins.test_epilogue_within_one_ulp_of_fp64_and_op_order()]),
     "epilogue bias add fused into a multiply-add": (
-        "v = v + bf16_bits_to_f32(bias[n]);",
-        "v = fmaf((float)acc[m * N + n], t, bf16_bits_to_f32(bias[n]));",
+        "(float)acc[m * N + n] * t;\n            if (bias)\n                v = v + bf16_bits_to_f32(bias[n]);",
+        "(float)acc[m * N + n] * t;\n            if (bias)\n                v = fmaf((float)acc[m * N + n], t, bf16_bits_to_f32(bias[n]));",
         [lambda: pins.test_epilogue_rounds_twice_not_fused()]),
     "bias dropped": (
-        "v = v + bf16_bits_to_f32(bias[n]);", "v = v;",
+        "(float)acc[m * N + n] * t;\n            if (bias)\n                v = v + bf16_bits_to_f32(bias[n]);",
+        "(float)acc[m * N + n] * t;\n            if (bias)\n                v = v;",
         [lambda: pins.test_golden_worked_epilogue()]),
     "bf16 rounding truncates": (
         "u += 0x7fffu + lsb;", "u += 0u * lsb;",
@@ -67,6 +69,19 @@ MUTANTS = {
     "backward: 1/sqrt(g) dropped": (
         "dx[m * K + k] = f32_to_bf16_rne(z[k] * c_g);", "dx[m * K + k] = f32_to_bf16_rne(z[k]);",
         [lambda: pins.test_grad_input_exact_case_against_explicit_hadamard(256)]),
+    "fp8: e4m3 ties away from zero": (
+        "double q = nearbyint(a / quantum) * quantum;", "double q = round(a / quantum) * quantum;",
+        [lambda: pins.test_e4m3_encode_matches_torch_cast_in_range()]),
+    "fp8: int8 grid used for the e4m3 scale": (
+        "const float s_z = amax / 448.0f;", "const float s_z = amax / 127.0f;",
+        [lambda: pins.test_rotate_quantize_fp8_brute_force(64)]),
+    "fp8: subnormal spacing wrong": (
+        "if (E < -6)\n        E = -6;", "if (E < -7)\n        E = -7;",
+        [lambda: pins.test_e4m3_encode_matches_torch_cast_in_range()]),
+    "fp8: products summed in fp32": (
+        "            double sum = 0.0;\n            for (int64_t k = 0; k < K; k++)\n                sum += lut[a[m * K + k]] * lut[b[n * K + k]];",
+        "            float sum = 0.0f;\n            for (int64_t k = 0; k < K; k++)\n                sum += (float)(lut[a[m * K + k]] * lut[b[n * K + k]]);",
+        [lambda: pins.test_fp8_gemm_matches_numpy_fp64()]),
 }
 
 

@@ -557,3 +557,117 @@ def test_grad_input_zero_gradient_row():
     res = oracle.grad_input(bf16_bits_from_f32(dy), qw, np.full(32, 0.01, np.float32), 256)
     assert res["sg"][2] == 0 and np.all(res["qg"][2] == 0)
     assert np.all(bf16_value(res["dx"][2]) == 0)
+
+
+# ---------------------------------------------------------------- FP8 (e4m3) variant
+
+def _torch_e4m3(x):
+    """Library routine: torch's fp32 -> float8_e4m3fn cast (round to nearest even)."""
+    return torch.from_numpy(np.asarray(x, np.float32)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
+def test_e4m3_encode_matches_torch_cast_in_range():
+    rng = np.random.default_rng(21)
+    x = np.concatenate([rng.standard_normal(100_000) * 30, rng.standard_normal(20_000) * 0.01,
+                        (rng.random(20_000) - 0.5) * 927.0]).astype(np.float32)
+    x = x[np.abs(x) < 464.0]                     # torch gives NaN beyond; we saturate
+    # exact ties: midpoints between neighbouring codes
+    codes = np.arange(0, 126, dtype=np.uint8)
+    lo, hi = oracle.e4m3_decode(codes[:-1]), oracle.e4m3_decode(codes[1:])
+    mids = ((lo.astype(np.float64) + hi) / 2).astype(np.float32)
+    for arr in (x, mids, -mids):
+        assert np.array_equal(oracle.e4m3_encode(arr), _torch_e4m3(arr))
+
+
+def test_e4m3_decode_matches_torch_for_every_code():
+    codes = np.arange(256, dtype=np.uint8)
+    got = oracle.e4m3_decode(codes)
+    want = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float32).numpy()
+    finite = ~np.isnan(want)
+    assert np.array_equal(np.isnan(got), ~finite)
+    assert np.array_equal(got[finite], want[finite])
+    assert got[0x7E] == 448.0 and got[0x01] == 2.0 ** -9
+
+
+def test_e4m3_encode_brute_force_nearest_ties_even_and_saturation():
+    rng = np.random.default_rng(22)
+    table = oracle.e4m3_decode(np.arange(256, dtype=np.uint8)).astype(np.float64)
+    finite = np.array([c for c in range(256) if not np.isnan(table[c])])
+    x = np.concatenate([rng.standard_normal(3000) * 20, rng.standard_normal(1000) * 0.005,
+                        [448.0, 460.0, 463.9, 500.0, 1e30, -1e30, 0.0]]).astype(np.float32)
+    got = oracle.e4m3_encode(x)
+    for v, c in zip(x.astype(np.float64), got):
+        if abs(v) >= 448.0:
+            assert table[c] == np.sign(v) * 448.0
+            continue
+        d = np.abs(table[finite] - v)
+        best = finite[d == d.min()]
+        if len(best) > 1:  # a tie (or +-0): the even code, sign of v
+            best = [b for b in best if b % 2 == 0 and (np.signbit(table[b]) == np.signbit(v)
+                                                        or table[b] != 0)]
+        assert table[c] == table[best[0]], (v, c, best)
+
+
+def test_fp8_gemm_matches_numpy_fp64():
+    rng = np.random.default_rng(23)
+    a = rng.integers(0, 256, size=(17, 96), dtype=np.uint8)
+    b = rng.integers(0, 256, size=(9, 96), dtype=np.uint8)
+    a[(a & 0x7F) == 0x7F] = 0   # no NaN codes
+    b[(b & 0x7F) == 0x7F] = 0
+    got = oracle.gemm_fp8(a, b)
+    da = oracle.e4m3_decode(a).astype(np.float64)
+    db = oracle.e4m3_decode(b).astype(np.float64)
+    assert np.array_equal(got, (da @ db.T).astype(np.float32))
+
+
+def test_fp8_epilogue_equals_int8_epilogue_on_integral_accumulators():
+    rng = np.random.default_rng(24)
+    acc = rng.integers(-2_000_000, 2_000_001, size=(64, 80)).astype(np.int32)
+    sx = (rng.random(64) * 0.05).astype(np.float32)
+    sw = (rng.random(80) * 1e-4).astype(np.float32)
+    bias = bf16_bits_from_f32(rng.standard_normal(80).astype(np.float32) * 0.01)
+    assert np.array_equal(oracle.dequant_epilogue_f32(acc.astype(np.float32), sx, sw, bias),
+                          oracle.dequant_epilogue(acc, sx, sw, bias))
+
+
+@pytest.mark.parametrize("g", [8, 64, 256])
+def test_rotate_quantize_fp8_brute_force(g):
+    """Integer inputs (exact rotation): codes are e4m3 of the IEEE fp32 quotient
+    z / fp32(amax / 448), the scale is fp32(amax/448) * fp32(1/sqrt g), amax maps to +-448,
+    and a zero row gives s = 0 and +0 codes."""
+    rng = np.random.default_rng(g + 5)
+    rows, K = 12, 2 * g
+    x = rng.integers(-200, 201, size=(rows, K)).astype(np.float32)
+    x[3] = 0.0
+    xb = bf16_bits_from_f32(x)
+    q, s = oracle.rotate_quantize_fp8(xb, g)
+    H = sylvester(g)
+    z = (x.astype(np.int64).reshape(rows, K // g, g) @ H.T).reshape(rows, K)
+    cg = np.float32(1.0 / math.sqrt(g))
+    for r in range(rows):
+        amax = np.float32(np.abs(z[r]).max())
+        if amax == 0:
+            assert s[r] == 0 and np.all(q[r] == 0)
+            continue
+        sz = np.float32(amax / np.float32(448.0))
+        assert s[r] == np.float32(sz * cg)
+        t = (z[r].astype(np.float32) / sz).astype(np.float32)
+        assert np.array_equal(q[r], _torch_e4m3(np.clip(t, -448, 448)))
+        assert np.abs(oracle.e4m3_decode(q[r])).max() == 448.0
+
+
+def test_fp8_rotated_linear_tracks_the_exact_product():
+    """Quality (not parity): the FP8 rotated linear stays close to the fp64 product, and the
+    rotation helps on outlier inputs as it does for int8."""
+    case = synthetic.make_case(M=64, N=96, K=1024, g=256, seed=25, outlier_count=10,
+                               outlier_factor=40.0)
+    xv = bf16_value(synthetic.bits(case.x)).astype(np.float64)
+    wv = bf16_value(synthetic.bits(case.W)).astype(np.float64)
+    ref = xv @ wv.T
+    errs = {}
+    for g in (1, 256):
+        qw, sw = oracle.rotate_quantize_fp8(synthetic.bits(case.W), g)
+        res = oracle.linear_fp8(synthetic.bits(case.x), qw, sw, g)
+        errs[g] = np.abs(bf16_value(res["out"]) - ref).max()
+    assert errs[256] < 0.08 * np.abs(ref).max()
+    assert errs[256] < errs[1]
