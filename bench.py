@@ -129,7 +129,18 @@ class Step:
         self.qW, self.sW = sd.sdnq_rotate_quant_weight(case.W.to(dev), g)
         self.out = torch.empty((case.M, case.N), dtype=torch.bfloat16, device=dev)
         self.gemm_stages = []
-        if name.startswith("grad_"):
+        if name.startswith("fp8_"):
+            # the FP8 (e4m3) variant: rotate + quantize to e4m3, then the kind::f8f6f4 GEMM
+            self.qW, self.sW = sd.sdnq_rotquant_fp8(case.W.to(dev), g)
+            self.qx = torch.empty((case.M, case.K), dtype=torch.uint8, device=dev)
+            self.stages = [
+                ("rotquant", lambda: sd.sdnq_rotquant_fp8(self.x, g, self.qx, self.sx)),
+                ("gemm", lambda: sd.sdnq_fp8_linear(self.qx, self.sx, self.qW, self.sW,
+                                                    self.bias, out=self.out)),
+            ]
+            self.gemm_stages = ["gemm"]
+            self.launches = 2
+        elif name.startswith("grad_"):
             # backward through the frozen layer: x holds dy [M, N]; W is [N, K]
             self.out = torch.empty((case.M, case.K), dtype=torch.bfloat16, device=dev)
             self.qx = torch.empty((case.M, case.N), dtype=torch.int8, device=dev)
@@ -254,6 +265,12 @@ def oracle_step(case, rows, nthreads):
     import oracle
     from hadamard_rotated_int8_b200 import synthetic
     xb = synthetic.bits(case.x)[:rows]
+    if case.extra.get("fp8"):
+        qx, sx = oracle.rotate_quantize_fp8(xb, case.g, nthreads)
+        acc = oracle.gemm_fp8(qx, case._oracle_qW, nthreads)
+        bias = synthetic.bits(case.bias) if case.bias is not None else None
+        oracle.dequant_epilogue_f32(acc, sx, case._oracle_sW, bias, nthreads)
+        return
     if case.extra.get("grad"):
         qg, sg = oracle.colscale_quantize(xb, case._oracle_sW, nthreads)
         acc = oracle.gemm_s8_nn(qg, case._oracle_qW, nthreads)
@@ -277,8 +294,8 @@ def oracle_step(case, rows, nthreads):
 def oracle_prepare(case, name, nthreads):
     import oracle
     from hadamard_rotated_int8_b200 import synthetic
-    case._oracle_qW, case._oracle_sW = oracle.rotate_quantize(synthetic.bits(case.W), case.g,
-                                                              nthreads)
+    quant = oracle.rotate_quantize_fp8 if case.extra.get("fp8") else oracle.rotate_quantize
+    case._oracle_qW, case._oracle_sW = quant(synthetic.bits(case.W), case.g, nthreads)
     case._oracle_down = None
     if name.startswith("dit_mlp"):
         case._oracle_down = oracle.rotate_quantize(synthetic.bits(case.extra["W_down"]), case.g,
@@ -338,7 +355,8 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": tops, "unit": "TOPS",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+        "vs_baseline": None, "dtype": "e4m3" if args.workload.startswith("fp8_") else "int8",
+        "data": "synthetic",
         "config": config_of(case, args),
         "cpu_baseline": {"value": tops, "unit": "TOPS", "cores": nthreads, "kind": "oracle",
                          "sample": f"{rows} of {case.M} tokens per step"},
@@ -516,13 +534,15 @@ def main():
     grad = args.workload.startswith("grad_")
     rq_rows_k = case.N if grad else case.K        # row length of the quantized operand
     rq_gbs = rotquant_bytes(case.M, rq_rows_k) / (rq_ms * 1e-3) / 1e9
-    gemm_kernel = ("gemm_s8_kernel_grad_input" if grad else
+    gemm_kernel = ("gemm_s8_kernel_e4m3" if args.workload.startswith("fp8_") else
+                   "gemm_s8_kernel_grad_input" if grad else
                    "gemm_s8_kernel_fused_quantizer" if "fused" in stage_ms else
                    "gemm_s8_kernel" if case.A is None else "gemm_s8_kernel_lora")
     line = {
         "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "e4m3" if args.workload.startswith("fp8_") else "int8",
         "data": "synthetic (seeded DiT-shaped bf16 activations with outlier channels, "
                 "random-init weights)",
         "config": config_of(case, args),

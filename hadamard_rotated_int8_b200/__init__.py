@@ -12,10 +12,12 @@ The compute lives in ``libsdnq.so`` (hand-written CUDA behind the C ABI of
 * ``sdnq_int8_linear_grad_input`` input gradient through the frozen rotated int8 base
   (= ``sdnq_quant_grad_output`` then ``sdnq_int8_grad_input_gemm``)
 * ``sdnq_gelu_bf16``            exact-erf GELU (MLP glue)
+* ``sdnq_rotquant_fp8``, ``sdnq_fp8_linear``  the FP8 (e4m3) variant of the same path
 
 ``linear`` composes the online path (rotate + quantize, then the int8 linear).
 """
-from ._native import (SdnqError, lib, sdnq_device_status, sdnq_gelu_bf16, sdnq_int8_linear,
+from ._native import (SdnqError, lib, sdnq_device_status, sdnq_fp8_linear, sdnq_gelu_bf16,
+                      sdnq_int8_linear, sdnq_rotquant_fp8,
                       sdnq_int8_grad_input_gemm, sdnq_int8_linear_fused, sdnq_int8_linear_gelu,
                       sdnq_int8_linear_grad_input, sdnq_int8_linear_lora,
                       sdnq_int8_linear_lora_noalloc, sdnq_rotate_quant_weight,
@@ -23,7 +25,8 @@ from ._native import (SdnqError, lib, sdnq_device_status, sdnq_gelu_bf16, sdnq_i
                       status_string, version)
 
 __all__ = [
-    "SdnqError", "lib", "linear", "sdnq_device_status", "sdnq_gelu_bf16", "sdnq_int8_linear",
+    "SdnqError", "lib", "linear", "sdnq_device_status", "sdnq_fp8_linear", "sdnq_gelu_bf16",
+    "sdnq_int8_linear", "sdnq_rotquant_fp8",
     "sdnq_int8_grad_input_gemm", "sdnq_int8_linear_fused", "sdnq_int8_linear_gelu",
     "sdnq_int8_linear_grad_input",
     "sdnq_int8_linear_lora", "sdnq_quant_grad_output",

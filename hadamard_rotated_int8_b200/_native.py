@@ -52,6 +52,8 @@ SIGNATURES = {
     "sdnq_int8_linear_lora_noalloc": [_P, _P, _P, _P, _P, _P, _I64, _P, _P, _I32, _F, _I64,
                                       _I64, _I64, _P, _I64, _P, _P],
     "sdnq_gelu_bf16": [_P, _I64, _I64, _I64, _P, _I64, _P],
+    "sdnq_rotquant_fp8": [_P, _I64, _I64, _I64, _I32, _P, _P, _P],
+    "sdnq_fp8_linear": [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _I64, _P, _P],
     "sdnq_device_status": [_P],
     "sdnq_selftest_wait_timeout": [_I64, _P],
     "sdnq_status_string": [ctypes.c_int],
@@ -185,6 +187,34 @@ def _linear_call(name, qx, sx, qW, sW, bias, out, acc_out, stream):
 def sdnq_int8_linear(qx, sx, qW, sW, bias=None, out=None, acc_out=None, stream=None):
     """out [M, N] bf16 = bf16(float(qx qW^T) * (sx sW^T) + bias)."""
     return _linear_call("sdnq_int8_linear", qx, sx, qW, sW, bias, out, acc_out, stream)
+
+
+def sdnq_rotquant_fp8(x, group: int, q=None, s=None, stream=None):
+    """Rows of x [M, K] bf16 -> (e4m3 codes uint8 [M, K], fp32 scales [M]), rotated."""
+    _req(x, torch.bfloat16, "x", 2)
+    M, K = x.shape
+    q = torch.empty((M, K), dtype=torch.uint8, device=x.device) if q is None else q
+    s = torch.empty((M,), dtype=torch.float32, device=x.device) if s is None else s
+    _check(lib().sdnq_rotquant_fp8(_ptr(x), M, K, x.stride(0), group, _ptr(q), _ptr(s),
+                                   _stream(stream)), "sdnq_rotquant_fp8")
+    return q, s
+
+
+def sdnq_fp8_linear(qx, sx, qW, sW, bias=None, out=None, acc_out=None, stream=None):
+    """out [M, N] bf16 from e4m3 codes qx [M, K], qW [N, K] (uint8) and their scales."""
+    _req(qx, torch.uint8, "qx", 2)
+    _req(qW, torch.uint8, "qW", 2)
+    _dense(qx, "qx")
+    _dense(qW, "qW")
+    M, K = qx.shape
+    N = qW.shape[0]
+    if qW.shape[1] != K:
+        raise ValueError("qx and qW disagree on K")
+    out = _rows_out(M, N, torch.bfloat16, qx.device) if out is None else out
+    _check(lib().sdnq_fp8_linear(_ptr(qx), _ptr(sx), _ptr(qW), _ptr(sW), _ptr(bias), M, N, K,
+                                 _ptr(out), out.stride(0), _ptr(acc_out), _stream(stream)),
+           "sdnq_fp8_linear")
+    return out
 
 
 def fused_sync_words(M: int) -> int:

@@ -311,6 +311,19 @@ __device__ __forceinline__ void mma_s8(uint32_t d_tmem, uint64_t adesc, uint64_t
         : "memory");
 }
 
+// D[tmem] (+)= A[smem] * B[smem]^T, 8-bit float operands (e4m3 here), fp32 accumulators.
+__device__ __forceinline__ void mma_f8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                       uint32_t idesc, uint32_t accumulate)
+{
+    const uint32_t z = 0u;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, {%5, %5, %5, %5}, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(z)
+        : "memory");
+}
+
 // D[tmem] (+)= A[smem] * B[smem]^T, 16-bit float operands, fp32 accumulators.
 __device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
                                         uint32_t idesc, uint32_t accumulate)
@@ -427,12 +440,19 @@ __device__ __forceinline__ uint64_t mnmajor_desc(uint32_t saddr, uint32_t mn_ato
 
 // Instruction descriptors (dense, no negation, no saturation).
 //   bits 4-5 accumulator format (1 = f32, 2 = s32); bits 7-9 / 10-12 A / B format
-//   (kind::i8: 1 = signed; kind::f16: 1 = bf16); bit 15 / 16 A / B major (0 = K, 1 = MN);
+//   (kind::i8: 1 = signed; kind::f16: 1 = bf16; kind::f8f6f4: 0 = e4m3); bit 15 / 16 A / B
+//   major (0 = K, 1 = MN);
 //   bits 17-22 N >> 3; bits 24-28 M >> 4.
 __host__ __device__ constexpr uint32_t idesc_s8_s32(int M, int N, bool b_mn_major = false)
 {
     return (2u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) |
            (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// kind::f8f6f4 with both operands e4m3 (format code 0) and fp32 accumulators
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N)
+{
+    return (1u << 4) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn_major)

@@ -278,7 +278,7 @@ __device__ __forceinline__ void grad_epilogue_tile(uint32_t t_row, int half, int
     }
 }
 
-template <int BN, bool LORA, bool GELU, int GRAD_G, int FUSE_G>
+template <int BN, bool LORA, bool GELU, int GRAD_G, int FUSE_G, bool FP8 = false>
 __global__ void __launch_bounds__(GemmConfig<BN, LORA, GELU, (FUSE_G > 0)>::THREADS, 1)
     gemm_s8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CUtensorMap tmL,
@@ -287,6 +287,8 @@ __global__ void __launch_bounds__(GemmConfig<BN, LORA, GELU, (FUSE_G > 0)>::THRE
     using C = GemmConfig<BN, LORA, GELU, (FUSE_G > 0)>;
     static_assert(FUSE_G == 0 || (BN == 256 && !LORA && !GELU && GRAD_G == 0),
                   "fused activation quantizer: plain forward tiles of 256 columns");
+    static_assert(!FP8 || (!LORA && !GELU && GRAD_G == 0 && FUSE_G == 0),
+                  "e4m3 operands: the plain forward kernel");
     static_assert(GRAD_G == 0 || (BN == 256 && !LORA && !GELU && (GRAD_G & (GRAD_G - 1)) == 0 &&
                                   GRAD_G <= 256),
                   "input-gradient mode: plain tiles of 256 columns, G divides 256");
@@ -422,7 +424,7 @@ __global__ void __launch_bounds__(GemmConfig<BN, LORA, GELU, (FUSE_G > 0)>::THRE
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            constexpr uint32_t IDESC_I8 = idesc_s8_s32(128, BN, GRAD_G > 0);
+            constexpr uint32_t IDESC_I8 = FP8 ? idesc_e4m3_f32(128, BN) : idesc_s8_s32(128, BN, GRAD_G > 0);
             constexpr uint32_t IDESC_BF = idesc_bf16_f32(128, BN, true);
             int stage = 0;
             uint32_t phase = 0;
@@ -451,8 +453,12 @@ __global__ void __launch_bounds__(GemmConfig<BN, LORA, GELU, (FUSE_G > 0)>::THRE
                         // of the input gradient, 32 K-rows of 128 bytes = 4096 bytes
                         const uint64_t bdesc = GRAD_G > 0 ? mnmajor_desc(sb + 4096 * k, 16384)
                                                           : kmajor_desc(sb + 32 * k);
-                        mma_s8(d_acc, kmajor_desc(sa + 32 * k), bdesc, IDESC_I8,
-                               (kb | k) != 0 ? 1u : 0u);
+                        if constexpr (FP8)
+                            mma_f8(d_acc, kmajor_desc(sa + 32 * k), bdesc, IDESC_I8,
+                                   (kb | k) != 0 ? 1u : 0u);
+                        else
+                            mma_s8(d_acc, kmajor_desc(sa + 32 * k), bdesc, IDESC_I8,
+                                   (kb | k) != 0 ? 1u : 0u);
                     }
                     tc_commit(empty_bar(stage));
                     if (++stage == C::STAGES) {
@@ -652,8 +658,12 @@ __global__ void __launch_bounds__(GemmConfig<BN, LORA, GELU, (FUSE_G > 0)>::THRE
                         // multiply-add, which differs from two roundings on ties)
                         float t0, t1;
                         mul2(t0, t1, sxm, sxm, wv[2 * h], wv[2 * h + 1]);
-                        float v0 = __fmul_rn(__int2float_rn(static_cast<int>(acc[j])), t0);
-                        float v1 = __fmul_rn(__int2float_rn(static_cast<int>(acc[j + 1])), t1);
+                        // accumulator: int32 (int8 operands) or fp32 bits (e4m3 operands)
+                        const float a0 = FP8 ? __uint_as_float(acc[j]) : __int2float_rn(static_cast<int>(acc[j]));
+                        const float a1 = FP8 ? __uint_as_float(acc[j + 1])
+                                             : __int2float_rn(static_cast<int>(acc[j + 1]));
+                        float v0 = __fmul_rn(a0, t0);
+                        float v1 = __fmul_rn(a1, t1);
                         if (has_bias) {
                             v0 = __fadd_rn(v0, bv[2 * h]);
                             v1 = __fadd_rn(v1, bv[2 * h + 1]);

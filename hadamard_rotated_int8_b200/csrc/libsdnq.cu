@@ -144,7 +144,7 @@ sdnq_status validate_rotquant(const void *x, int64_t rows, int64_t K, int64_t ld
 
 // Rows of at most 16 chunks go to the persistent, prefetching kernel (grid = resident
 // CTAs); longer rows to the two-pass kernel with one CTA per row.
-template <int G, bool COLSCALE = false>
+template <int G, bool COLSCALE = false, bool FP8 = false>
 void launch_rotquant_g(const RotquantParams &p, dim3 grid, dim3 block, int sm_count,
                        cudaStream_t st)
 {
@@ -154,7 +154,7 @@ void launch_rotquant_g(const RotquantParams &p, dim3 grid, dim3 block, int sm_co
         if (per_sm[warps] == 0) {
             int n = 0;
             if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(
-                    &n, rotquant_persistent_kernel<G, COLSCALE>, block.x, 0) != cudaSuccess ||
+                    &n, rotquant_persistent_kernel<G, COLSCALE, FP8>, block.x, 0) != cudaSuccess ||
                 n < 1)
                 n = 1;
             per_sm[warps] = n;
@@ -162,9 +162,9 @@ void launch_rotquant_g(const RotquantParams &p, dim3 grid, dim3 block, int sm_co
         const int64_t groups = grid.x;
         const int64_t resident = static_cast<int64_t>(per_sm[warps]) * sm_count;
         const dim3 pgrid(static_cast<unsigned>(groups < resident ? groups : resident));
-        rotquant_persistent_kernel<G, COLSCALE><<<pgrid, block, 0, st>>>(p);
+        rotquant_persistent_kernel<G, COLSCALE, FP8><<<pgrid, block, 0, st>>>(p);
     } else {
-        rotquant_kernel<G, COLSCALE><<<grid, block, 0, st>>>(p);
+        rotquant_kernel<G, COLSCALE, FP8><<<grid, block, 0, st>>>(p);
     }
 }
 
@@ -172,7 +172,7 @@ void launch_rotquant_g(const RotquantParams &p, dim3 grid, dim3 block, int sm_co
 // block-diagonal Hadamard of `group` columns, or (group 1) multiplied by colscale[K].
 sdnq_status launch_rowquant(const uint16_t *x, int64_t rows, int64_t K, int64_t ld,
                             int32_t group, const float *colscale, int8_t *q, float *s,
-                            const DeviceInfo &dev, cudaStream_t cs)
+                            const DeviceInfo &dev, cudaStream_t cs, bool fp8 = false)
 {
     RotquantParams p;
     p.x = x;
@@ -189,6 +189,17 @@ sdnq_status launch_rowquant(const uint16_t *x, int64_t rows, int64_t K, int64_t 
     const dim3 block(32 * p.wpr * p.rpc);
     const dim3 grid(static_cast<unsigned>((rows + p.rpc - 1) / p.rpc));
     cudaGetLastError();
+    if (fp8) {
+        switch (group) {
+        case 8: launch_rotquant_g<8, false, true>(p, grid, block, dev.sm_count, cs); break;
+        case 16: launch_rotquant_g<16, false, true>(p, grid, block, dev.sm_count, cs); break;
+        case 32: launch_rotquant_g<32, false, true>(p, grid, block, dev.sm_count, cs); break;
+        case 64: launch_rotquant_g<64, false, true>(p, grid, block, dev.sm_count, cs); break;
+        case 128: launch_rotquant_g<128, false, true>(p, grid, block, dev.sm_count, cs); break;
+        default: launch_rotquant_g<256, false, true>(p, grid, block, dev.sm_count, cs); break;
+        }
+        return launch_status();
+    }
     switch (group) {
     case 1: launch_rotquant_g<1, true>(p, grid, block, dev.sm_count, cs); break;
     case 8: launch_rotquant_g<8>(p, grid, block, dev.sm_count, cs); break;
@@ -239,13 +250,13 @@ sdnq_status validate_linear(const void *qx, const void *sx, const void *qW, cons
 // FUSE_G > 0: the activation quantizer runs inside the kernel (p.rq, p.sync set by the
 // caller); the grid is launched cooperatively so that every CTA is resident, because the
 // producers of one CTA wait for rows that the quantizer warps of others publish.
-template <int BN, bool LORA, bool GELU = false, int GRAD_G = 0, int FUSE_G = 0>
+template <int BN, bool LORA, bool GELU = false, int GRAD_G = 0, int FUSE_G = 0, bool FP8 = false>
 sdnq_status launch_gemm(const DeviceInfo &dev, const int8_t *qx, const int8_t *qW,
                         const uint16_t *u, const uint16_t *B, int32_t rank, GemmParams p,
                         cudaStream_t cs)
 {
     using C = GemmConfig<BN, LORA, GELU, (FUSE_G > 0)>;
-    constexpr auto kernel = gemm_s8_kernel<BN, LORA, GELU, GRAD_G, FUSE_G>;
+    constexpr auto kernel = gemm_s8_kernel<BN, LORA, GELU, GRAD_G, FUSE_G, FP8>;
     CUtensorMap tmA, tmB, tmU, tmL, tmO;
     const bool b_ok = GRAD_G > 0
                           ? make_tmap_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, qW, p.N, p.K, p.N, 128, 128)
@@ -583,6 +594,52 @@ sdnq_status run_grad_input(const uint16_t *dy, int64_t lddy, const int8_t *qW, c
     return launch_grad_gemm(dev, qg_ws, sg_ws, qW, M, N, K, group, dx, lddx, acc_out, cs);
 }
 
+// ---------------------------------------------------------------- FP8 (e4m3) variant
+
+sdnq_status run_rotquant_fp8(const uint16_t *x, int64_t rows, int64_t K, int64_t ld,
+                             int32_t group, uint8_t *q, float *s, void *stream)
+{
+    sdnq_status st = validate_rotquant(x, rows, K, ld, group, q, s);
+    if (st != SDNQ_OK)
+        return st;
+    DeviceInfo dev;
+    if ((st = current_device(&dev)) != SDNQ_OK)
+        return st;
+    if (rows == 0)
+        return SDNQ_OK;
+    return launch_rowquant(x, rows, K, ld, group, nullptr, reinterpret_cast<int8_t *>(q), s, dev,
+                           static_cast<cudaStream_t>(stream), true);
+}
+
+sdnq_status run_fp8_linear(const uint8_t *qx, const float *sx, const uint8_t *qW, const float *sW,
+                           const uint16_t *bias, int64_t M, int64_t N, int64_t K, uint16_t *out,
+                           int64_t ldo, float *acc_out, void *stream)
+{
+    sdnq_status st = validate_linear(qx, sx, qW, sW, bias, M, N, K, out, ldo, acc_out);
+    if (st != SDNQ_OK)
+        return st;
+    DeviceInfo dev;
+    if ((st = current_device(&dev)) != SDNQ_OK)
+        return st;
+    if (M == 0)
+        return SDNQ_OK;
+    GemmParams p = {};
+    p.sx = sx;
+    p.sw = sW;
+    p.bias = bias;
+    p.out = out;
+    p.ldo = ldo;
+    p.acc_out = reinterpret_cast<int32_t *>(acc_out);  // fp32 bits
+    p.M = static_cast<int32_t>(M);
+    p.N = static_cast<int32_t>(N);
+    p.K = static_cast<int32_t>(K);
+    p.c_g = 1.0f;
+    p.timeout_ns = kDefaultTimeoutNs;
+    return launch_gemm<256, false, false, 0, 0, true>(
+        dev, reinterpret_cast<const int8_t *>(qx), reinterpret_cast<const int8_t *>(qW), nullptr,
+        nullptr, 0, p, static_cast<cudaStream_t>(stream));
+}
+
 // ---------------------------------------------------------------- self-test kernel
 
 __global__ void wait_timeout_selftest_kernel(uint64_t limit_ns)
@@ -634,6 +691,20 @@ SDNQ_API sdnq_status sdnq_int8_linear_fused(const uint16_t *x, int64_t ldx, int3
 {
     return run_linear_fused(x, ldx, group, qW, sW, bias, M, N, K, qx_ws, sx_ws, sync_ws, out, ldo,
                             acc_out, policy, stream);
+}
+
+SDNQ_API sdnq_status sdnq_rotquant_fp8(const uint16_t *x, int64_t M, int64_t K, int64_t ldx,
+                                       int32_t group, uint8_t *q, float *s, void *stream)
+{
+    return run_rotquant_fp8(x, M, K, ldx, group, q, s, stream);
+}
+
+SDNQ_API sdnq_status sdnq_fp8_linear(const uint8_t *qx, const float *sx, const uint8_t *qW,
+                                     const float *sW, const uint16_t *bias, int64_t M, int64_t N,
+                                     int64_t K, uint16_t *out, int64_t ldo, float *acc_out,
+                                     void *stream)
+{
+    return run_fp8_linear(qx, sx, qW, sW, bias, M, N, K, out, ldo, acc_out, stream);
 }
 
 SDNQ_API sdnq_status sdnq_int8_linear_gelu(const int8_t *qx, const float *sx, const int8_t *qW,

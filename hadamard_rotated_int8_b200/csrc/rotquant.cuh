@@ -255,6 +255,44 @@ __device__ __forceinline__ uint2 quant8(const float (&z)[8], float s_z, float rc
                             __float_as_uint(f[7])));
 }
 
+// e4m3 codes of two fp32 values (round to nearest even, saturating at +-448), low byte = lo
+__device__ __forceinline__ uint32_t e4m3x2(float lo, float hi)
+{
+    uint16_t d;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(d) : "f"(hi), "f"(lo));
+    return d;
+}
+
+__device__ __noinline__ uint2 quant8_e4m3_exact(float z0, float z1, float z2, float z3, float z4,
+                                                float z5, float z6, float z7, float s_z)
+{
+    const float t[8] = {__fdiv_rn(z0, s_z), __fdiv_rn(z1, s_z), __fdiv_rn(z2, s_z),
+                        __fdiv_rn(z3, s_z), __fdiv_rn(z4, s_z), __fdiv_rn(z5, s_z),
+                        __fdiv_rn(z6, s_z), __fdiv_rn(z7, s_z)};
+    return make_uint2(e4m3x2(t[0], t[1]) | (e4m3x2(t[2], t[3]) << 16),
+                      e4m3x2(t[4], t[5]) | (e4m3x2(t[6], t[7]) << 16));
+}
+
+// e4m3 codes of one vector of 8 values: the IEEE quotient RN(z / s_z) by the same Markstein
+// correction as quant8, then one rounding to e4m3.
+__device__ __forceinline__ uint2 quant8_e4m3(const float (&z)[8], float s_z, float rcp, bool fast)
+{
+    if (!fast)
+        return quant8_e4m3_exact(z[0], z[1], z[2], z[3], z[4], z[5], z[6], z[7], s_z);
+    const float neg_s = -s_z;
+    float c[8];
+#pragma unroll
+    for (int i = 0; i < 8; i += 2) {
+        float q0, q1, r0, r1;
+        mul2(q0, q1, z[i], z[i + 1], rcp, rcp);
+        fma2(r0, r1, q0, q1, neg_s, neg_s, z[i], z[i + 1]);
+        fma2(c[i], c[i + 1], r0, r1, rcp, rcp, q0, q1);
+    }
+    return make_uint2(e4m3x2(c[0], c[1]) | (e4m3x2(c[2], c[3]) << 16),
+                      e4m3x2(c[4], c[5]) | (e4m3x2(c[6], c[7]) << 16));
+}
+
+template <bool FP8 = false>
 __device__ __forceinline__ void quant_store_chunk(const float (&v)[4][8], int8_t *qr, int32_t K,
                                                   int32_t c, bool ok, uint32_t lane, float s_z,
                                                   bool zero)
@@ -268,7 +306,7 @@ __device__ __forceinline__ void quant_store_chunk(const float (&v)[4][8], int8_t
         const int32_t e = base + t * 64;
         uint2 w = make_uint2(0u, 0u);
         if (!zero)  // warp-uniform: the whole warp works on one row
-            w = quant8(v[t], s_z, rcp, fast);
+            w = FP8 ? quant8_e4m3(v[t], s_z, rcp, fast) : quant8(v[t], s_z, rcp, fast);
         if (ok && e < K)
             st_v2(qr + e, w.x, w.y);
     }
@@ -365,7 +403,7 @@ __device__ __forceinline__ void rotquant_worker_rows(const RotquantParams &p, in
 // Rows of at most 16 chunks (K <= 16384): each warp owns one chunk of a row, a CTA owns
 // `rpc` rows at a time and walks row groups persistently, loading the next row group into
 // registers while it rotates and quantizes the current one.
-template <int G, bool COLSCALE>
+template <int G, bool COLSCALE, bool FP8 = false>
 __global__ void __launch_bounds__(512) rotquant_persistent_kernel(const RotquantParams p)
 {
     __shared__ float s_amax[2][32];
@@ -413,16 +451,16 @@ __global__ void __launch_bounds__(512) rotquant_persistent_kernel(const Rotquant
         amax = 0.0f;
         for (int32_t w = 0; w < p.wpr; ++w)
             amax = fmaxf(amax, s_amax[parity][r_local * p.wpr + w]);
-        const float s_z = __fdiv_rn(amax, 127.0f);
+        const float s_z = __fdiv_rn(amax, FP8 ? 448.0f : 127.0f);  // grid: +-127 or +-448
         const bool zero = !(amax > 0.0f);
         if (row_ok && wr == 0 && lane == 0)
             p.s[row] = zero ? 0.0f : __fmul_rn(s_z, p.c_g);
         int8_t *qr = p.q + (row_ok ? row : 0) * static_cast<int64_t>(p.K);
-        quant_store_chunk(v, qr, p.K, wr, row_ok && has_chunk, lane, s_z, zero);
+        quant_store_chunk<FP8>(v, qr, p.K, wr, row_ok && has_chunk, lane, s_z, zero);
     }
 }
 
-template <int G, bool COLSCALE>
+template <int G, bool COLSCALE, bool FP8 = false>
 __global__ void __launch_bounds__(512) rotquant_kernel(const RotquantParams p)
 {
     __shared__ float s_amax[32];
@@ -468,20 +506,20 @@ __global__ void __launch_bounds__(512) rotquant_kernel(const RotquantParams p)
     for (int32_t w = 0; w < p.wpr; ++w)
         amax = fmaxf(amax, s_amax[r_local * p.wpr + w]);
 
-    const float s_z = __fdiv_rn(amax, 127.0f);
+    const float s_z = __fdiv_rn(amax, FP8 ? 448.0f : 127.0f);
     const bool zero = !(amax > 0.0f);
     if (row_ok && wr == 0 && lane == 0)
         p.s[row] = zero ? 0.0f : __fmul_rn(s_z, p.c_g);
 
     if (single) {
-        quant_store_chunk(v, qr, p.K, wr, row_ok && my_chunks == 1, lane, s_z, zero);
+        quant_store_chunk<FP8>(v, qr, p.K, wr, row_ok && my_chunks == 1, lane, s_z, zero);
     } else {
         for (int32_t j = 0; j < my_chunks; ++j) {
             load_chunk(xr, p.K, wr + j * p.wpr, row_ok, lane, v);
             if (COLSCALE)
                 apply_colscale(v, p.colscale, p.K, wr + j * p.wpr, lane);
             chunk_butterfly<G>(v, lane);
-            quant_store_chunk(v, qr, p.K, wr + j * p.wpr, row_ok, lane, s_z, zero);
+            quant_store_chunk<FP8>(v, qr, p.K, wr + j * p.wpr, row_ok, lane, s_z, zero);
         }
     }
 }

@@ -143,6 +143,12 @@ GRAD_WORKLOADS = {
 def workload(name: str, g: int | None = None, M: int | None = None) -> Case:
     """Build one of the named workloads. ``g`` overrides the Hadamard group (the QuaRot
     sweep runs 64, 128, 256); ``M`` overrides the token count (smaller samples)."""
+    if name.startswith("fp8_"):
+        # the FP8 (e4m3) variant runs on the same inputs as the int8 workload it names
+        case = workload(name[len("fp8_"):], g=g, M=M)
+        case.name = name
+        case.extra["fp8"] = True
+        return case
     grad = name in GRAD_WORKLOADS
     kw = dict(GRAD_WORKLOADS[name] if grad else WORKLOADS[name])
     if g is not None:

@@ -239,6 +239,31 @@ sdnq_status sdnq_int8_linear_lora_noalloc(const int8_t *qx, const float *sx, con
                                           int64_t ldo, int32_t *acc_out, void *stream);
 
 /*
+ * FP8 (e4m3) variant of the rotated quantized matmul ("SDNQ: SD.Next Quantization Engine",
+ * feature list and SDNQConfig: FP8 weights and FP8 quantized matmul beside INT8), same
+ * rotation. e4m3 here is the "fn" format: bias 7, 3 mantissa bits, largest finite 448, no
+ * infinities.
+ *
+ * sdnq_rotquant_fp8: rows of x (weights or activations) rotated as in sdnq_rotquant_act,
+ * then s_z = fp32(amax / 448), codes = e4m3(fp32(z / s_z)) (round to nearest even,
+ * saturating), stored scale s = fp32(s_z * fp32(1/sqrt(group))); an all-zero row gives s = 0
+ * and +0 codes. Arguments, layouts and rules as sdnq_rotquant_act, codes as uint8.
+ */
+sdnq_status sdnq_rotquant_fp8(const uint16_t *x, int64_t M, int64_t K, int64_t ldx,
+                              int32_t group, uint8_t *q, float *s, void *stream);
+
+/*
+ * sdnq_fp8_linear: out = bf16(acc * (sx * sw) [+ bias]) with acc[m][n] = sum_k qx[m][k] *
+ * qW[n][k] over e4m3 codes, accumulated in fp32 on the tensor cores (tcgen05 kind::f8f6f4;
+ * the summation order is the hardware's, so acc matches an exact sum only to within fp32
+ * accumulation error). Arguments, layouts and rules as sdnq_int8_linear; acc_out, if set, is
+ * [M, N] fp32.
+ */
+sdnq_status sdnq_fp8_linear(const uint8_t *qx, const float *sx, const uint8_t *qW,
+                            const float *sW, const uint16_t *bias, int64_t M, int64_t N,
+                            int64_t K, uint16_t *out, int64_t ldo, float *acc_out, void *stream);
+
+/*
  * GELU between the up and down projections of a DiT MLP (exact erf form,
  * x * Phi(x), rounded once to bf16). Not on the pages; the MLP workload needs it.
  *   in [M, N] bf16 row stride ld_in; out [M, N] bf16 row stride ld_out (may alias in when
