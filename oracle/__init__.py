@@ -68,6 +68,9 @@ def _open(path: str):
         "oracle_gelu_bf16": [P, I64, P, INT],
         "oracle_colscale_quantize": [P, I64, I64, I64, P, P, P, INT],
         "oracle_e4m3_encode": [P, I64, P],
+        "oracle_attn_prep": [P, P, I64, I64, I64, I64, I64, I64, INT, P, P, P, P, P, INT],
+        "oracle_attn_logits": [P, P, P, P, I64, I64, I64, I64, I64, F, P, INT],
+        "oracle_attn_softmax_pv": [P, P, I64, I64, I64, I64, I64, P, INT],
         "oracle_e4m3_decode": [P, I64, P],
         "oracle_rotate_quantize_fp8": [P, I64, I64, I64, I64, P, P, INT],
         "oracle_gemm_fp8": [P, P, I64, I64, I64, P, INT],
@@ -399,3 +402,54 @@ def linear_fp8(x_bits, qw, sw, g, bias_bits=None, nthreads: int | None = None):
     acc = gemm_fp8(qx, qw, nthreads)
     return {"qx": qx, "sx": sx, "acc": acc,
             "out": dequant_epilogue_f32(acc, sx, sw, bias_bits, nthreads)}
+
+
+# ---- Hadamard-rotated int8 QK inside attention ----------------------------------------
+
+def attn_prep(q_bits, k_bits, g: int, smooth_k: bool = True, nthreads: int | None = None):
+    """q [B, Lq, H, D], k [B, Lk, H, D] bf16 patterns -> dict(qq, sq [B, H, Lq], kq, sk
+    [B, H, Lk], mu [B, H, D]): smooth_k means, rotated per-row int8 codes and scales."""
+    q_bits = _c(q_bits, np.uint16)
+    k_bits = _c(k_bits, np.uint16)
+    B, Lq, H, D = q_bits.shape
+    Lk = k_bits.shape[1]
+    out = {"qq": np.empty((B, Lq, H, D), np.int8), "sq": np.empty((B, H, Lq), np.float32),
+           "kq": np.empty((B, Lk, H, D), np.int8), "sk": np.empty((B, H, Lk), np.float32),
+           "mu": np.empty((B, H, D), np.float32)}
+    _check(_load().oracle_attn_prep(_ptr(q_bits), _ptr(k_bits), B, Lq, Lk, H, D, g,
+                                    1 if smooth_k else 0, _ptr(out["qq"]), _ptr(out["sq"]),
+                                    _ptr(out["kq"]), _ptr(out["sk"]), _ptr(out["mu"]),
+                                    nthreads or default_threads()), "attn_prep")
+    return out
+
+
+def attn_logits(prep, scale: float, nthreads: int | None = None) -> np.ndarray:
+    B, Lq, H, D = prep["qq"].shape
+    Lk = prep["kq"].shape[1]
+    logits = np.empty((B, H, Lq, Lk), np.float32)
+    _check(_load().oracle_attn_logits(_ptr(prep["qq"]), _ptr(prep["sq"]), _ptr(prep["kq"]),
+                                      _ptr(prep["sk"]), B, Lq, Lk, H, D, float(scale),
+                                      _ptr(logits), nthreads or default_threads()), "attn_logits")
+    return logits
+
+
+def attn_softmax_pv(logits, v_bits, nthreads: int | None = None) -> np.ndarray:
+    logits = _c(logits, np.float32)
+    v_bits = _c(v_bits, np.uint16)
+    B, H, Lq, Lk = logits.shape
+    D = v_bits.shape[3]
+    o = np.empty((B, Lq, H, D), np.uint16)
+    _check(_load().oracle_attn_softmax_pv(_ptr(logits), _ptr(v_bits), B, Lq, Lk, H, D, _ptr(o),
+                                          nthreads or default_threads()), "attn_softmax_pv")
+    return o
+
+
+def attention(q_bits, k_bits, v_bits, g: int = 256, scale: float | None = None,
+              smooth_k: bool = True, nthreads: int | None = None):
+    """Attention with Hadamard-rotated int8 QK and a bf16 PV; every intermediate in a dict."""
+    D = q_bits.shape[3]
+    scale = float(np.float32(1.0 / np.sqrt(D))) if scale is None else scale
+    res = attn_prep(q_bits, k_bits, g, smooth_k, nthreads)
+    res["logits"] = attn_logits(res, scale, nthreads)
+    res["o"] = attn_softmax_pv(res["logits"], v_bits, nthreads)
+    return res

@@ -564,3 +564,148 @@ int oracle_dequant_epilogue_f32(const float *acc, const float *sx, const float *
     }
     return ORACLE_OK;
 }
+
+/* ---- Hadamard-rotated int8 QK inside attention ----
+ * [SD] SDNQ attention example (an SDPA replacement: int8 QK matmul, smooth_k, use_hadamard,
+ * hadamard_group_size; the PV matmul left unquantized). Per batch b and head h, with Q
+ * [Lq][D], K and V [Lk][D] (bf16, stored [B][L][H][D]):
+ *   mu[d]    = fp32( sum_j K[j][d] / Lk ), the sum in binary64 (smooth_k);
+ *   K'[j][d] = fp32( K[j][d] - mu[d] )   (softmax is unchanged: q.mu is constant per row);
+ *   Q and K' rows rotated by the butterfly over groups of min(g, D) and quantized per row
+ *   exactly as the linear path's activations (codes, stored scale s = fp32(amax/127) * c);
+ *   logit[i][j] = fp32( fp32( fp32(acc) * fp32(s_q[i] * s_k[j]) ) * scale ),
+ *   acc = sum_d qQ[i][d] qK[j][d] in int32 (the rotation cancels in the product);
+ *   O[i] = sum_j softmax_j(logit[i][j]) V[j] in binary64, rounded once to bf16. */
+
+/* K' rows from bf16 K and the per-(b, h) channel means: kq [B][Lk][H][D] int8, sk [B][H][Lk]. */
+static void quantize_rows_f32(float *z, int64_t K, int64_t g, int8_t *q, float *s, float c_g)
+{
+    for (int64_t k0 = 0; k0 < K; k0 += g)
+        fwht_group_f32(z + k0, g);
+    float amax = 0.0f;
+    for (int64_t k = 0; k < K; k++) {
+        float a = fabsf(z[k]);
+        if (a > amax)
+            amax = a;
+    }
+    const float s_z = amax / 127.0f;
+    for (int64_t k = 0; k < K; k++) {
+        int code = 0;
+        if (amax != 0.0f) {
+            float n_ = nearbyintf(z[k] / s_z);
+            if (n_ > 127.0f)
+                n_ = 127.0f;
+            if (n_ < -127.0f)
+                n_ = -127.0f;
+            code = (n_ == n_) ? (int)n_ : 0;
+        }
+        q[k] = (int8_t)code;
+    }
+    *s = s_z * c_g;
+}
+
+int oracle_attn_prep(const uint16_t *q, const uint16_t *k, int64_t B, int64_t Lq, int64_t Lk,
+                     int64_t H, int64_t D, int64_t g, int smooth_k, int8_t *qq, float *sq,
+                     int8_t *kq, float *sk, float *mu, int nthreads)
+{
+    if (!q || !k || !qq || !sq || !kq || !sk || !mu || B <= 0 || Lq <= 0 || Lk <= 0 || H <= 0 ||
+        D <= 0 || !is_pow2(g) || !is_pow2(D))
+        return ORACLE_ERR_ARG;
+    const int64_t ge = g < D ? g : D;
+    const float c_g = (float)(1.0 / sqrt((double)ge));
+    for (int64_t b = 0; b < B; b++)
+        for (int64_t h = 0; h < H; h++)
+            for (int64_t d = 0; d < D; d++) {
+                double sum = 0.0;
+                if (smooth_k)
+                    for (int64_t j = 0; j < Lk; j++)
+                        sum += (double)bf16_bits_to_f32(k[((b * Lk + j) * H + h) * D + d]);
+                mu[(b * H + h) * D + d] = (float)(sum / (double)Lk);
+            }
+    int err = 0;
+#pragma omp parallel for num_threads(nthreads > 0 ? nthreads : 1) schedule(static)
+    for (int64_t r = 0; r < B * Lq * H; r++) {
+        float z[1024];
+        if (D > 1024) {
+#pragma omp atomic write
+            err = 1;
+            continue;
+        }
+        const int64_t b = r / (Lq * H), i = (r / H) % Lq, h = r % H;
+        for (int64_t d = 0; d < D; d++)
+            z[d] = bf16_bits_to_f32(q[r * D + d]);
+        quantize_rows_f32(z, D, ge, qq + r * D, sq + (b * H + h) * Lq + i, c_g);
+    }
+#pragma omp parallel for num_threads(nthreads > 0 ? nthreads : 1) schedule(static)
+    for (int64_t r = 0; r < B * Lk * H; r++) {
+        float z[1024];
+        if (D > 1024)
+            continue;
+        const int64_t b = r / (Lk * H), j = (r / H) % Lk, h = r % H;
+        for (int64_t d = 0; d < D; d++)
+            z[d] = bf16_bits_to_f32(k[r * D + d]) - mu[(b * H + h) * D + d];
+        quantize_rows_f32(z, D, ge, kq + r * D, sk + (b * H + h) * Lk + j, c_g);
+    }
+    return err ? ORACLE_ERR_ARG : ORACLE_OK;
+}
+
+/* logits [B][H][Lq][Lk] (fp32) from the prepared codes and scales. */
+int oracle_attn_logits(const int8_t *qq, const float *sq, const int8_t *kq, const float *sk,
+                       int64_t B, int64_t Lq, int64_t Lk, int64_t H, int64_t D, float scale,
+                       float *logits, int nthreads)
+{
+    if (!qq || !sq || !kq || !sk || !logits || B <= 0 || Lq <= 0 || Lk <= 0 || H <= 0 || D <= 0)
+        return ORACLE_ERR_ARG;
+#pragma omp parallel for num_threads(nthreads > 0 ? nthreads : 1) schedule(static)
+    for (int64_t bhi = 0; bhi < B * H * Lq; bhi++) {
+        const int64_t b = bhi / (H * Lq), h = (bhi / Lq) % H, i = bhi % Lq;
+        const int8_t *qr = qq + ((b * Lq + i) * H + h) * D;
+        for (int64_t j = 0; j < Lk; j++) {
+            const int8_t *kr = kq + ((b * Lk + j) * H + h) * D;
+            int32_t acc = 0;
+            for (int64_t d = 0; d < D; d++)
+                acc += (int32_t)qr[d] * (int32_t)kr[d];
+            float t = sq[(b * H + h) * Lq + i] * sk[(b * H + h) * Lk + j];
+            float v = (float)acc * t;
+            logits[bhi * Lk + j] = v * scale;
+        }
+    }
+    return ORACLE_OK;
+}
+
+/* O [B][Lq][H][D] bf16 = softmax(logits) V, in binary64. */
+int oracle_attn_softmax_pv(const float *logits, const uint16_t *v, int64_t B, int64_t Lq,
+                           int64_t Lk, int64_t H, int64_t D, uint16_t *o, int nthreads)
+{
+    if (!logits || !v || !o || B <= 0 || Lq <= 0 || Lk <= 0 || H <= 0 || D <= 0)
+        return ORACLE_ERR_ARG;
+    int err = 0;
+#pragma omp parallel for num_threads(nthreads > 0 ? nthreads : 1) schedule(static)
+    for (int64_t bhi = 0; bhi < B * H * Lq; bhi++) {
+        const int64_t b = bhi / (H * Lq), h = (bhi / Lq) % H, i = bhi % Lq;
+        const float *lr = logits + bhi * Lk;
+        double m = -INFINITY;
+        for (int64_t j = 0; j < Lk; j++)
+            if ((double)lr[j] > m)
+                m = (double)lr[j];
+        double *acc = (double *)calloc((size_t)D, sizeof(double));
+        if (!acc) {
+#pragma omp atomic write
+            err = 1;
+            continue;
+        }
+        double l = 0.0;
+        for (int64_t j = 0; j < Lk; j++) {
+            const double p = exp((double)lr[j] - m);
+            l += p;
+            const uint16_t *vr = v + ((b * Lk + j) * H + h) * D;
+            for (int64_t d = 0; d < D; d++)
+                acc[d] += p * (double)bf16_bits_to_f32(vr[d]);
+        }
+        uint16_t *orow = o + ((b * Lq + i) * H + h) * D;
+        for (int64_t d = 0; d < D; d++)
+            orow[d] = f64_to_bf16_rne(acc[d] / l);
+        free(acc);
+    }
+    return err ? ORACLE_ERR_NOMEM : ORACLE_OK;
+}

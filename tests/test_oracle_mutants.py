@@ -82,6 +82,17 @@ MUTANTS = {
         "            double sum = 0.0;\n            for (int64_t k = 0; k < K; k++)\n                sum += lut[a[m * K + k]] * lut[b[n * K + k]];",
         "            float sum = 0.0f;\n            for (int64_t k = 0; k < K; k++)\n                sum += (float)(lut[a[m * K + k]] * lut[b[n * K + k]]);",
         [lambda: pins.test_fp8_gemm_matches_numpy_fp64()]),
+    "attention: channel mean not subtracted from K": (
+        "z[d] = bf16_bits_to_f32(k[r * D + d]) - mu[(b * H + h) * D + d];",
+        "z[d] = bf16_bits_to_f32(k[r * D + d]);",
+        [lambda: pins.test_attn_smooth_k_subtracts_the_exact_channel_mean()]),
+    "attention: softmax scale dropped": (
+        "logits[bhi * Lk + j] = v * scale;", "logits[bhi * Lk + j] = v;",
+        [lambda: pins.test_attn_logits_are_dequantized_products()]),
+    "attention: V rows of the wrong head": (
+        "const uint16_t *vr = v + ((b * Lk + j) * H + h) * D;",
+        "const uint16_t *vr = v + ((b * Lk + j) * H) * D;",
+        [lambda: pins.test_attn_softmax_pv_matches_torch_fp64()]),
 }
 
 

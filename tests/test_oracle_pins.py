@@ -671,3 +671,80 @@ def test_fp8_rotated_linear_tracks_the_exact_product():
         errs[g] = np.abs(bf16_value(res["out"]) - ref).max()
     assert errs[256] < 0.08 * np.abs(ref).max()
     assert errs[256] < errs[1]
+
+
+# ---------------------------------------------------------------- int8 QK attention
+
+def _attn_inputs(B, Lq, Lk, H, D, seed, scale_q=1.0):
+    gen = torch.Generator().manual_seed(seed)
+    q = (torch.randn(B, Lq, H, D, generator=gen) * scale_q).to(torch.bfloat16)
+    k = torch.randn(B, Lk, H, D, generator=gen).to(torch.bfloat16)
+    v = torch.randn(B, Lk, H, D, generator=gen).to(torch.bfloat16)
+    return q, k, v
+
+
+def test_attn_prep_without_smoothing_is_the_linear_quantizer():
+    """With smooth_k off, Q and K codes and scales are those of the (pinned) row quantizer of
+    the linear path applied to the token-head rows, with the group capped at D."""
+    q, k, _ = _attn_inputs(2, 40, 56, 3, 64, seed=1)
+    res = oracle.attn_prep(synthetic.bits(q), synthetic.bits(k), 256, smooth_k=False)
+    qc, qs = oracle.rotate_quantize(synthetic.bits(q).reshape(-1, 64), 64)
+    kc, ks = oracle.rotate_quantize(synthetic.bits(k).reshape(-1, 64), 64)
+    assert np.array_equal(res["qq"].reshape(-1, 64), qc)
+    assert np.array_equal(res["kq"].reshape(-1, 64), kc)
+    assert np.array_equal(res["sq"], qs.reshape(2, 40, 3).transpose(0, 2, 1))
+    assert np.array_equal(res["sk"], ks.reshape(2, 56, 3).transpose(0, 2, 1))
+    assert np.all(res["mu"] == 0)
+
+
+def test_attn_smooth_k_subtracts_the_exact_channel_mean():
+    """Integer K built so that every channel mean is an integer: mu is that mean, and the K
+    codes are the row quantizer's codes of the integer rows K - mu."""
+    rng = np.random.default_rng(2)
+    B, Lk, H, D = 1, 64, 2, 128
+    k = rng.integers(-60, 61, size=(B, Lk, H, D)).astype(np.float64)
+    shift = rng.integers(-20, 21, size=(B, 1, H, D))
+    k = k - k.mean(axis=1, keepdims=True).round() + shift   # means are exactly `shift` +- 0
+    k[:, -1] += (Lk * shift[:, 0] - k.sum(axis=1))          # force sum == Lk * shift
+    kb = bf16_bits_from_f32(k.astype(np.float32))
+    assert np.array_equal(bf16_value(kb), k.astype(np.float32))
+    q = np.zeros((B, 8, H, D), np.float32)
+    res = oracle.attn_prep(bf16_bits_from_f32(q), kb, 128, smooth_k=True)
+    assert np.array_equal(res["mu"], shift[:, 0].astype(np.float32))
+    centred = (k - shift).astype(np.float32)
+    kc, ks = oracle.rotate_quantize(bf16_bits_from_f32(centred).reshape(-1, D), 128)
+    assert np.array_equal(res["kq"].reshape(-1, D), kc)
+
+
+def test_attn_logits_are_dequantized_products():
+    q, k, _ = _attn_inputs(1, 33, 70, 2, 128, seed=3)
+    res = oracle.attention(synthetic.bits(q), synthetic.bits(k), synthetic.bits(k), 256)
+    acc = np.einsum("bihd,bjhd->bhij", res["qq"].astype(np.int64), res["kq"].astype(np.int64))
+    scale = np.float32(1.0 / np.sqrt(128.0))
+    ref = (acc * res["sq"][..., None].astype(np.float64) * res["sk"][:, :, None, :] * scale)
+    assert np.all(np.abs(res["logits"] - ref) <= 3 * 2.0 ** -24 * np.abs(ref) + 1e-30)
+
+
+def test_attn_softmax_pv_matches_torch_fp64():
+    """softmax(logits) V against torch's fp64 softmax and matmul: within one bf16 rounding."""
+    rng = np.random.default_rng(4)
+    B, H, Lq, Lk, D = 2, 3, 17, 45, 64
+    logits = (rng.standard_normal((B, H, Lq, Lk)) * 3).astype(np.float32)
+    v = torch.randn(B, Lk, H, D, generator=torch.Generator().manual_seed(5)).to(torch.bfloat16)
+    got = bf16_value(oracle.attn_softmax_pv(logits, synthetic.bits(v))).astype(np.float64)
+    p = torch.softmax(torch.from_numpy(logits).double(), dim=-1)
+    ref = torch.einsum("bhij,bjhd->bihd", p, v.double()).numpy()
+    assert np.all(np.abs(got - ref) <= np.abs(ref) * 2.0 ** -8 + 1e-300)
+
+
+@pytest.mark.parametrize("smooth", [False, True])
+def test_attn_tracks_sdpa(smooth):
+    """Quality: the int8-QK attention stays close to fp64 SDPA, with or without smoothing."""
+    q, k, v = _attn_inputs(1, 64, 128, 2, 128, seed=6)
+    res = oracle.attention(synthetic.bits(q), synthetic.bits(k), synthetic.bits(v), 256,
+                           smooth_k=smooth)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        q.double().transpose(1, 2), k.double().transpose(1, 2), v.double().transpose(1, 2)
+    ).transpose(1, 2).numpy()
+    got = bf16_value(res["o"]).astype(np.float64)
+    assert np.abs(got - ref).max() < 0.03
