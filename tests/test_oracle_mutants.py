@@ -25,7 +25,8 @@ MUTANTS = {
         "z[k] = bf16_bits_to_f32(xr[k]);\n        for (int64_t k0 = 0; k0 < K; k0 += g)\n            fwht_group_f32(z + k0, g);\n        float amax = 0.0f;\n        for (int64_t k = 0; k < g; k++) {",
         [lambda: pins.test_golden_worked_rotquant()]),
     "grid 255 levels (range -128..127)": (
-        "const float s_z = amax / 127.0f;", "const float s_z = amax / 127.5f;",
+        "const float s_z = amax / 127.0f;\n        int8_t *qr = q + r * K;",
+        "const float s_z = amax / 127.5f;\n        int8_t *qr = q + r * K;",
         [lambda: pins.test_codes_brute_force_g8(8)]),
     "gemm operand transposed": (
         "const int8_t *bn = b + n * K;", "const int8_t *bn = b + n;",
