@@ -13,10 +13,12 @@ The compute lives in ``libsdnq.so`` (hand-written CUDA behind the C ABI of
   (= ``sdnq_quant_grad_output`` then ``sdnq_int8_grad_input_gemm``)
 * ``sdnq_gelu_bf16``            exact-erf GELU (MLP glue)
 * ``sdnq_rotquant_fp8``, ``sdnq_fp8_linear``  the FP8 (e4m3) variant of the same path
+* ``sdnq_attention_int8qk``     attention with Hadamard-rotated int8 QK and a bf16 PV
 
 ``linear`` composes the online path (rotate + quantize, then the int8 linear).
 """
-from ._native import (SdnqError, lib, sdnq_device_status, sdnq_fp8_linear, sdnq_gelu_bf16,
+from ._native import (SdnqError, lib, sdnq_attention_int8qk, sdnq_device_status,
+                      sdnq_fp8_linear, sdnq_gelu_bf16,
                       sdnq_int8_linear, sdnq_rotquant_fp8,
                       sdnq_int8_grad_input_gemm, sdnq_int8_linear_fused, sdnq_int8_linear_gelu,
                       sdnq_int8_linear_grad_input, sdnq_int8_linear_lora,
@@ -25,7 +27,8 @@ from ._native import (SdnqError, lib, sdnq_device_status, sdnq_fp8_linear, sdnq_
                       status_string, version)
 
 __all__ = [
-    "SdnqError", "lib", "linear", "sdnq_device_status", "sdnq_fp8_linear", "sdnq_gelu_bf16",
+    "SdnqError", "lib", "linear", "sdnq_attention_int8qk", "sdnq_device_status",
+    "sdnq_fp8_linear", "sdnq_gelu_bf16",
     "sdnq_int8_linear", "sdnq_rotquant_fp8",
     "sdnq_int8_grad_input_gemm", "sdnq_int8_linear_fused", "sdnq_int8_linear_gelu",
     "sdnq_int8_linear_grad_input",

@@ -8,6 +8,7 @@ the library is missing or the device is not a B200 (sm_100), calls raise.
 from __future__ import annotations
 
 import ctypes
+import math
 import os
 import threading
 
@@ -53,6 +54,9 @@ SIGNATURES = {
                                       _I64, _I64, _P, _I64, _P, _P],
     "sdnq_gelu_bf16": [_P, _I64, _I64, _I64, _P, _I64, _P],
     "sdnq_rotquant_fp8": [_P, _I64, _I64, _I64, _I32, _P, _P, _P],
+    "sdnq_attention_workspace": [_I64, _I64, _I64, _I64, _I64, _P],
+    "sdnq_attention_int8qk": [_P, _P, _P, _I64, _I64, _I64, _I64, _I64, _I32, _F, _I32, _P, _I64,
+                              _P, _P],
     "sdnq_fp8_linear": [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _I64, _P, _P],
     "sdnq_device_status": [_P],
     "sdnq_selftest_wait_timeout": [_I64, _P],
@@ -214,6 +218,36 @@ def sdnq_fp8_linear(qx, sx, qW, sW, bias=None, out=None, acc_out=None, stream=No
     _check(lib().sdnq_fp8_linear(_ptr(qx), _ptr(sx), _ptr(qW), _ptr(sW), _ptr(bias), M, N, K,
                                  _ptr(out), out.stride(0), _ptr(acc_out), _stream(stream)),
            "sdnq_fp8_linear")
+    return out
+
+
+def attention_workspace(B: int, Lq: int, Lk: int, H: int, D: int):
+    """(total bytes, offsets of: Q codes, K codes, Q scales, K scales, mu, scratch)."""
+    off = (ctypes.c_int64 * 6)()
+    total = lib().sdnq_attention_workspace(B, Lq, Lk, H, D, ctypes.cast(off, _P))
+    if total < 0:
+        raise ValueError("bad attention shape")
+    return int(total), [int(x) for x in off]
+
+
+def sdnq_attention_int8qk(q, k, v, group: int = 256, scale: float | None = None,
+                          smooth_k: bool = True, ws=None, out=None, stream=None):
+    """o [B, Lq, H, D] bf16: attention with Hadamard-rotated int8 QK^T and a bf16 PV. ``ws``
+    (uint8, attention_workspace bytes) receives the codes, scales and key means."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _req(t, torch.bfloat16, n, 4)
+        _dense(t, n)
+    B, Lq, H, D = q.shape
+    Lk = k.shape[1]
+    if k.shape != (B, Lk, H, D) or v.shape != k.shape:
+        raise ValueError("q, k, v shapes disagree")
+    total, _ = attention_workspace(B, Lq, Lk, H, D)
+    ws = torch.empty(total, dtype=torch.uint8, device=q.device) if ws is None else ws
+    out = torch.empty_like(q) if out is None else out
+    scale = float(1.0 / math.sqrt(D)) if scale is None else float(scale)
+    _check(lib().sdnq_attention_int8qk(_ptr(q), _ptr(k), _ptr(v), B, Lq, Lk, H, D, group, scale,
+                                       1 if smooth_k else 0, _ptr(ws), ws.numel(), _ptr(out),
+                                       _stream(stream)), "sdnq_attention_int8qk")
     return out
 
 

@@ -1,0 +1,477 @@
+// Attention with a Hadamard-rotated int8 QK^T and a bf16 PV, on the 5th-generation tensor
+// cores. Sources: "SDNQ: SD.Next Quantization Engine" README, SDNQ attention (an SDPA
+// replacement with an int8 QK matmul, smooth_k, use_hadamard and hadamard_group_size, the PV
+// matmul left unquantized); "ConvRot / Hadamard SDNQ" (group 256 = ConvRot).
+//
+// Q, K, V are [B][L][H][D] bf16 (D = 128): token-head rows of D contiguous values.
+//   1. attn_ksum_kernel + attn_kmean_kernel: mu[b][h][d] = fp32(sum_j K[b][j][h][d] / Lk),
+//      the sum in fp64 (smooth_k; subtracting mu from every key leaves the softmax unchanged).
+//   2. attn_rowquant_kernel: Q rows, and K rows minus mu, rotated by the butterfly over groups
+//      of min(g, D) and quantized per row to int8 as in the linear path (codes, scale
+//      s = fp32(amax/127) * fp32(1/sqrt(G))); scales stored [B][H][L].
+//   3. attn_kernel: one CTA per (b, h, 128 queries).
+//      - warp 0 loads the Q codes once and a 2-stage ring of (K codes, V, key scales) through TMA;
+//      - warp 1 issues S_j = Q K_j^T (tcgen05 kind::i8, int32 in a double-buffered TMEM tile)
+//        and O += P_j V_j (kind::f16, bf16 P and V, fp32 O in TMEM);
+//      - warps 2..5, one query row per thread, turn S_j into logits with the oracle's fp32 op
+//        order, fp32(fp32(acc * fp32(s_q s_k)) * scale), run an online softmax in base 2
+//        (rescaling O and the row sum only when the row maximum grows by more than 2^8, so
+//        P stays below 256), write P_j as bf16 into a 128-byte-swizzled K-major tile for the
+//        MMA, and finally write O / l as bf16.
+// Every wait is bounded as in the GEMM kernel.
+#pragma once
+
+#include <cuda_bf16.h>
+
+#include "device.cuh"
+#include "rotquant.cuh"
+
+namespace sdnq {
+
+constexpr int kAttnD = 128;
+constexpr int kAttnBlock = 128;        // queries per CTA and keys per step
+constexpr int kAttnSumSplits = 32;     // key splits of the channel sums
+
+// ---------------------------------------------------------------- smooth_k channel means
+
+// partial[(bh * splits + split) * D + d] = sum over this split's keys of K[b][j][h][d] (fp64)
+__global__ void __launch_bounds__(256) attn_ksum_kernel(const uint16_t *k, int32_t Lk, int32_t H,
+                                                        double *partial)
+{
+    const int32_t bh = blockIdx.x, split = blockIdx.y;
+    const int32_t b = bh / H, h = bh % H;
+    const int32_t d8 = (threadIdx.x & 15) * 8;   // 16 threads cover the 128 channels
+    const int32_t lane_row = threadIdx.x >> 4;   // 16 keys per pass
+    const int32_t per = (Lk + kAttnSumSplits - 1) / kAttnSumSplits;
+    const int32_t j0 = split * per, j1 = j0 + per < Lk ? j0 + per : Lk;
+    double acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    for (int32_t j = j0 + lane_row; j < j1; j += 16) {
+        const uint4 r = ld_nc_v4(k + ((static_cast<int64_t>(b) * Lk + j) * H + h) * kAttnD + d8);
+        const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            acc[2 * i] += static_cast<double>(__uint_as_float(w[i] << 16));
+            acc[2 * i + 1] += static_cast<double>(__uint_as_float(w[i] & 0xffff0000u));
+        }
+    }
+    __shared__ double red[16][kAttnD];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+        red[lane_row][d8 + i] = acc[i];
+    __syncthreads();
+    if (threadIdx.x < kAttnD) {
+        double s = 0.0;
+        for (int r = 0; r < 16; ++r)
+            s += red[r][threadIdx.x];
+        partial[(static_cast<int64_t>(bh) * kAttnSumSplits + split) * kAttnD + threadIdx.x] = s;
+    }
+}
+
+// mu[bh][d] = fp32(sum of the splits / Lk). The fp64 sums of bf16 values are exact when a
+// channel spans less than 2^45 in magnitude, so the split order does not matter.
+__global__ void attn_kmean_kernel(const double *partial, int32_t Lk, float *mu)
+{
+    const int32_t bh = blockIdx.x, d = threadIdx.x;
+    double s = 0.0;
+    for (int i = 0; i < kAttnSumSplits; ++i)
+        s += partial[(static_cast<int64_t>(bh) * kAttnSumSplits + i) * kAttnD + d];
+    mu[static_cast<int64_t>(bh) * kAttnD + d] = static_cast<float>(s / static_cast<double>(Lk));
+}
+
+// ---------------------------------------------------------------- Q / K row quantizer
+
+struct AttnQuantParams {
+    const uint16_t *x;     // [B][L][H][D] bf16
+    const float *mu;       // [B][H][D] or nullptr (queries)
+    int8_t *q;             // [B][L][H][D]
+    float *s;              // [B][H][L]
+    int64_t rows;          // B * L * H
+    int32_t L, H;
+    float c_g;
+};
+
+// One warp per 1024-element chunk = 8 consecutive token-head rows of 128; the butterfly over
+// groups of G <= 128 never crosses a row. Lane (hi2, lo3) holds rows 2 hi2 (t = 0, 1) and
+// 2 hi2 + 1 (t = 2, 3) of the chunk; a row's maximum combines its 8 lanes by shuffles.
+template <int G>
+__global__ void __launch_bounds__(256) attn_rowquant_kernel(const AttnQuantParams p)
+{
+    const uint32_t lane = lane_id();
+    const int64_t nchunks = (p.rows + 7) / 8;
+    const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+    for (int64_t c = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+         c < nchunks; c += warps) {
+        const int64_t row0 = c * 8 + 2 * static_cast<int64_t>(lane >> 3);
+        const int64_t base = c * 1024 + static_cast<int64_t>(lane >> 3) * 256 +
+                             static_cast<int64_t>(lane & 7u) * 8;
+        float v[4][8];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            const int64_t row = row0 + (t >> 1);
+            uint4 r = make_uint4(0u, 0u, 0u, 0u);
+            if (row < p.rows)
+                r = ld_nc_v4(p.x + base + t * 64);
+            bf16x8_to_f32(r, v[t]);
+            if (p.mu != nullptr && row < p.rows) {
+                const int64_t b = row / (static_cast<int64_t>(p.L) * p.H);
+                const int64_t h = row % p.H;
+                const int32_t d = (t & 1) * 64 + static_cast<int32_t>(lane & 7u) * 8;
+                const float *m = p.mu + (b * p.H + h) * kAttnD + d;
+                const uint4 a = ld_nc_v4(m), bb = ld_nc_v4(m + 4);
+                const uint32_t w[8] = {a.x, a.y, a.z, a.w, bb.x, bb.y, bb.z, bb.w};
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    v[t][i] = __fsub_rn(v[t][i], __uint_as_float(w[i]));
+            }
+        }
+        chunk_butterfly<G>(v, lane);
+        float m0 = 0.0f, m1 = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            m0 = fmaxf(m0, fmaxf(fabsf(v[0][i]), fabsf(v[1][i])));
+            m1 = fmaxf(m1, fmaxf(fabsf(v[2][i]), fabsf(v[3][i])));
+        }
+#pragma unroll
+        for (int off = 1; off < 8; off <<= 1) {
+            m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, off));
+            m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, off));
+        }
+        const float amax[2] = {m0, m1};
+#pragma unroll
+        for (int rr = 0; rr < 2; ++rr) {
+            const int64_t row = row0 + rr;
+            const float s_z = __fdiv_rn(amax[rr], 127.0f);
+            const bool zero = !(amax[rr] > 0.0f);
+            const bool fast = s_z >= 0x1p-126f;
+            const float rcp = __frcp_rn(s_z);
+#pragma unroll
+            for (int tt = 0; tt < 2; ++tt) {
+                const int t = 2 * rr + tt;
+                uint2 w = make_uint2(0u, 0u);
+                if (!zero)
+                    w = quant8(v[t], s_z, rcp, fast);
+                if (row < p.rows)
+                    st_v2(p.q + base + t * 64, w.x, w.y);
+            }
+            if (row < p.rows && (lane & 7u) == 0u) {
+                const int64_t h = row % p.H;
+                const int64_t l = (row / p.H) % p.L;
+                const int64_t b = row / (static_cast<int64_t>(p.L) * p.H);
+                p.s[(b * p.H + h) * p.L + l] = zero ? 0.0f : __fmul_rn(s_z, p.c_g);
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------- the attention kernel
+
+struct AttnParams {
+    const float *sq;       // [B][H][Lq] query scales
+    const float *sk;       // [B][H][Lk] key scales
+    uint16_t *o;           // [B][Lq][H][D] bf16
+    int32_t B, Lq, Lk, H;
+    int32_t q_blocks;      // ceil(Lq / 128)
+    float scale;           // softmax scale applied to the logits (fp32)
+    uint64_t timeout_ns;
+};
+
+struct AttnConfig {
+    static constexpr int THREADS = 192;                   // 6 warps
+    static constexpr int Q_OFF = 0;                       // int8 [128 x 128]
+    static constexpr int K_OFF = 16384;                   // 2 stages x int8 [128 x 128]
+    static constexpr int V_OFF = K_OFF + 2 * 16384;       // 2 stages x bf16 [128 x 128]
+    static constexpr int P_OFF = V_OFF + 2 * 32768;       // bf16 [128 x 128], K-major
+    static constexpr int SK_OFF = P_OFF + 32768;          // 2 stages x 128 fp32
+    static constexpr int BAR_OFF = SK_OFF + 2 * 512;
+    // barriers: q_full, kv_full[2], kv_empty[2], s_full[2], s_empty[2], p_full, pv_done, drain
+    static constexpr int NBARS = 12;
+    static constexpr int SMEM_BYTES = 1024 + BAR_OFF + NBARS * 8 + 16;
+    static constexpr int TMEM_COLS = 512;                 // S0 [0,128), S1 [128,256), O [256,384)
+};
+
+__global__ void __launch_bounds__(AttnConfig::THREADS, 1)
+    attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                const __grid_constant__ CUtensorMap tmV, const AttnParams p)
+{
+    using C = AttnConfig;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_addr = smem_u32(smem_raw);
+    const uint32_t base = (raw_addr + 1023u) & ~1023u;
+    uint8_t *smem = smem_raw + (base - raw_addr);
+    const uint32_t bar0 = base + C::BAR_OFF;
+    const uint32_t q_full = bar0;
+    auto kv_full = [&](int s) { return bar0 + 8u * (1 + s); };
+    auto kv_empty = [&](int s) { return bar0 + 8u * (3 + s); };
+    auto s_full = [&](int s) { return bar0 + 8u * (5 + s); };
+    auto s_empty = [&](int s) { return bar0 + 8u * (7 + s); };
+    const uint32_t p_full = bar0 + 8u * 9;
+    const uint32_t pv_done = bar0 + 8u * 10;
+    const uint32_t drain_bar = bar0 + 8u * 11;
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C::BAR_OFF + C::NBARS * 8);
+    volatile int *abort = reinterpret_cast<volatile int *>(tmem_holder + 1);
+    float *sk_smem = reinterpret_cast<float *>(smem + C::SK_OFF);
+
+    const uint32_t warp = threadIdx.x >> 5;
+    const uint32_t lane = lane_id();
+    const int32_t qb = static_cast<int32_t>(blockIdx.x) % p.q_blocks;
+    const int32_t bh = static_cast<int32_t>(blockIdx.x) / p.q_blocks;
+    const int32_t b = bh / p.H, h = bh % p.H;
+    const int32_t q0 = qb * kAttnBlock;
+    const int32_t nkv = (p.Lk + kAttnBlock - 1) / kAttnBlock;
+
+    if (threadIdx.x == 0) {
+        mbar_init(q_full, 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(kv_full(s), 1);
+            mbar_init(kv_empty(s), 1);
+            mbar_init(s_full(s), 1);
+            mbar_init(s_empty(s), 4);
+        }
+        mbar_init(p_full, 4);
+        mbar_init(pv_done, 1);
+        mbar_init(drain_bar, 1);
+        *abort = 0;
+        fence_mbar_init();
+        prefetch_tensormap(&tmQ);
+        prefetch_tensormap(&tmK);
+        prefetch_tensormap(&tmV);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_holder), C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem_base = *tmem_holder;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ loads
+        bool ok = true;
+        if (lane == 0) {
+            mbar_arrive_expect_tx(q_full, 16384);
+            tma_load_3d(base + C::Q_OFF, &tmQ, q_full, h * kAttnD, q0, b);
+        }
+        int issued = 0;
+        for (int j = 0; ok && j < nkv; ++j) {
+            const int s = j & 1;
+            const uint32_t use = static_cast<uint32_t>(j >> 1);
+            bool good = true;
+            if (lane == 0)
+                good = mbar_wait_bounded(kv_empty(s), (use & 1u) ^ 1u, abort, p.timeout_ns);
+            if (__shfl_sync(0xffffffffu, good ? 1 : 0, 0) == 0) {
+                ok = false;
+                break;
+            }
+            // the block's key scales (0 past Lk)
+            const int32_t j0 = j * kAttnBlock;
+            for (int i = static_cast<int>(lane); i < kAttnBlock; i += 32)
+                sk_smem[s * kAttnBlock + i] =
+                    j0 + i < p.Lk ? p.sk[static_cast<int64_t>(bh) * p.Lk + j0 + i] : 0.0f;
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive_expect_tx(kv_full(s), 16384 + 32768);
+                tma_load_3d(base + C::K_OFF + s * 16384, &tmK, kv_full(s), h * kAttnD, j0, b);
+                tma_load_3d(base + C::V_OFF + s * 32768, &tmV, kv_full(s), h * kAttnD, j0, b);
+                tma_load_3d(base + C::V_OFF + s * 32768 + 16384, &tmV, kv_full(s), h * kAttnD + 64,
+                            j0, b);
+            }
+            ++issued;
+        }
+        if (lane == 0) {
+            // every copy this warp started has landed before the CTA can exit (the Q tile and
+            // the last two stages; already complete on the normal path)
+            volatile int no_abort = 0;
+            mbar_wait_bounded(q_full, 0u, &no_abort, p.timeout_ns);
+            for (int j = issued - 2 < 0 ? 0 : issued - 2; j < issued; ++j)
+                mbar_wait_bounded(kv_full(j & 1), static_cast<uint32_t>(j >> 1) & 1u, &no_abort,
+                                  p.timeout_ns);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issue
+        if (lane == 0) {
+            constexpr uint32_t IDESC_S = idesc_s8_s32(128, 128);
+            constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, 128, true);
+            const uint32_t t_o = tmem_base + 256;
+            bool ok = mbar_wait_bounded(q_full, 0u, abort, p.timeout_ns);
+            auto issue_pv = [&](int j) {
+                // O (+)= P_j V_j: A = P, K-major bf16 in two 64-column atoms; B = V, N-major
+                if (!mbar_wait_bounded(p_full, static_cast<uint32_t>(j) & 1u, abort, p.timeout_ns))
+                    return false;
+                tc_fence_after_sync();
+                const uint32_t sp = base + C::P_OFF;
+                const uint32_t sv = base + C::V_OFF + (j & 1) * 32768;
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    mma_f16(t_o, kmajor_desc(sp + (k >> 2) * 16384 + (k & 3) * 32),
+                            mnmajor_desc(sv + 2048 * k, 16384), IDESC_PV,
+                            (j | k) != 0 ? 1u : 0u);
+                tc_commit(pv_done);
+                tc_commit(kv_empty(j & 1));
+                return true;
+            };
+            for (int j = 0; ok && j < nkv; ++j) {
+                const int s = j & 1;
+                const uint32_t use = static_cast<uint32_t>(j >> 1);
+                if (!mbar_wait_bounded(kv_full(s), use & 1u, abort, p.timeout_ns) ||
+                    !mbar_wait_bounded(s_empty(s), (use & 1u) ^ 1u, abort, p.timeout_ns)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after_sync();
+                const uint32_t sq_addr = base + C::Q_OFF;
+                const uint32_t sk_addr = base + C::K_OFF + s * 16384;
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    mma_s8(tmem_base + s * 128, kmajor_desc(sq_addr + 32 * k),
+                           kmajor_desc(sk_addr + 32 * k), IDESC_S, k != 0 ? 1u : 0u);
+                tc_commit(s_full(s));
+                if (j >= 1 && !issue_pv(j - 1)) {
+                    ok = false;
+                    break;
+                }
+            }
+            if (ok)
+                issue_pv(nkv - 1);
+            tc_commit(drain_bar);
+            volatile int no_abort = 0;
+            mbar_wait_bounded(drain_bar, 0u, &no_abort, p.timeout_ns);
+        }
+    } else {
+        // ------------------------------------------------------------ softmax (warps 2..5)
+        const uint32_t quad = warp & 3u;
+        const int32_t r = static_cast<int32_t>(quad * 32u + lane);   // query row in the block
+        const bool row_ok = q0 + r < p.Lq;
+        const float sqr = row_ok ? p.sq[static_cast<int64_t>(bh) * p.Lq + q0 + r] : 0.0f;
+        const uint32_t t_lane = tmem_base + ((quad * 32u) << 16);
+        const float kLog2e = 1.4426950408889634f;
+        float m_used = -INFINITY;  // base-2 maximum the exponentials are taken against
+        float l_sum = 0.0f;
+        bool ok = true;
+        for (int j = 0; ok && j < nkv; ++j) {
+            const int s = j & 1;
+            const uint32_t use = static_cast<uint32_t>(j >> 1);
+            bool got = mbar_wait_bounded(s_full(s), use & 1u, abort, p.timeout_ns) &&
+                       mbar_wait_bounded(kv_full(s), use & 1u, abort, p.timeout_ns);
+            if (!__all_sync(0xffffffffu, got)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after_sync();
+            float y[kAttnBlock];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                uint32_t a[32];
+                tmem_ld_32x32b_x32(t_lane + s * 128 + c * 32, a);
+                tmem_ld_wait();
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    y[c * 32 + i] = __int_as_float(static_cast<int>(a[i]));  // raw bits for now
+            }
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(s_empty(s));
+            // logits in the oracle's fp32 order, then base 2; keys past Lk masked
+            const int32_t j0 = j * kAttnBlock;
+            float mb = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < kAttnBlock; ++c) {
+                const float t = __fmul_rn(sqr, sk_smem[s * kAttnBlock + c]);
+                const float v = __fmul_rn(__int2float_rn(__float_as_int(y[c])), t);
+                const float lg = __fmul_rn(v, p.scale);
+                y[c] = j0 + c < p.Lk ? __fmul_rn(lg, kLog2e) : -INFINITY;
+                mb = fmaxf(mb, y[c]);
+            }
+            // P_{j-1} has left the P tile (and O is stable) once PV_{j-1} is done
+            if (j >= 1) {
+                got = mbar_wait_bounded(pv_done, static_cast<uint32_t>(j - 1) & 1u, abort, p.timeout_ns);
+                if (!__all_sync(0xffffffffu, got)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after_sync();
+            }
+            // rescale O and l only when the maximum grows by more than 8 (p stays <= 256)
+            const bool grow = mb > m_used + 8.0f;
+            if (__any_sync(0xffffffffu, grow)) {
+                const float m_new = grow ? mb : m_used;
+                const float alpha = grow && m_used != -INFINITY ? exp2f(m_used - m_new)
+                                                                : (grow ? 0.0f : 1.0f);
+                if (j >= 1) {
+#pragma unroll 1
+                    for (int c = 0; c < 4; ++c) {
+                        uint32_t a[32];
+                        tmem_ld_32x32b_x32(t_lane + 256 + c * 32, a);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i)
+                            a[i] = __float_as_uint(__uint_as_float(a[i]) * alpha);
+                        tmem_st_32x32b_x32(t_lane + 256 + c * 32, a);
+                    }
+                    tmem_st_wait();
+                }
+                l_sum *= alpha;
+                m_used = m_new;
+            }
+            // P = 2^(y - m), bf16, into the swizzled K-major tile: row r, 16-byte chunks
+            const uint32_t prow = base + C::P_OFF + static_cast<uint32_t>(r) * 128u;
+#pragma unroll
+            for (int ch = 0; ch < 16; ++ch) {
+                uint32_t w[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float p0 = exp2f(y[ch * 8 + 2 * e] - m_used);
+                    const float p1 = exp2f(y[ch * 8 + 2 * e + 1] - m_used);
+                    l_sum += p0;
+                    l_sum += p1;
+                    const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+                    w[e] = *reinterpret_cast<const uint32_t *>(&h2);
+                }
+                const uint32_t atom = static_cast<uint32_t>(ch >> 3);
+                const uint32_t c16 = static_cast<uint32_t>(ch & 7) ^ (static_cast<uint32_t>(r) & 7u);
+                sts_v4(prow + atom * 16384u + (c16 << 4), w[0], w[1], w[2], w[3]);
+            }
+            fence_proxy_async_smem();
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(p_full);
+        }
+        // O / l as bf16
+        bool fin = ok && mbar_wait_bounded(pv_done, static_cast<uint32_t>(nkv - 1) & 1u, abort,
+                                           p.timeout_ns);
+        if (__all_sync(0xffffffffu, fin)) {
+            tc_fence_after_sync();
+            const float inv = 1.0f / l_sum;
+            uint16_t *orow = p.o + ((static_cast<int64_t>(b) * p.Lq + q0 + r) * p.H + h) * kAttnD;
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+                uint32_t a[32];
+                tmem_ld_32x32b_x32(t_lane + 256 + c * 32, a);
+                tmem_ld_wait();
+                uint32_t w[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(a[2 * i]) * inv,
+                                                                    __uint_as_float(a[2 * i + 1]) * inv);
+                    w[i] = *reinterpret_cast<const uint32_t *>(&h2);
+                }
+                if (row_ok) {
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        st_v4(orow + c * 32 + q * 8, w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+                }
+            }
+        }
+    }
+
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after_sync();
+        tmem_dealloc(tmem_base, C::TMEM_COLS);
+    }
+}
+
+} // namespace sdnq

@@ -15,6 +15,7 @@
 #include "device.cuh"
 #include "gelu.cuh"
 #include "gemm.cuh"
+#include "attention.cuh"
 #include "lora_down.cuh"
 #include "rotquant.cuh"
 
@@ -640,6 +641,139 @@ sdnq_status run_fp8_linear(const uint8_t *qx, const float *sx, const uint8_t *qW
         nullptr, 0, p, static_cast<cudaStream_t>(stream));
 }
 
+// ---------------------------------------------------------------- int8-QK attention
+
+bool make_tmap_3d(CUtensorMap *map, CUtensorMapDataType dtype, const void *ptr, uint64_t d0,
+                  uint64_t d1, uint64_t d2, uint64_t stride1_bytes, uint64_t stride2_bytes,
+                  uint32_t box0, uint32_t box1)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn)
+        return false;
+    const cuuint64_t dims[3] = {d0, d1, d2};
+    const cuuint64_t strides[2] = {stride1_bytes, stride2_bytes};
+    const cuuint32_t box[3] = {box0, box1, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult r = fn(map, dtype, 3, const_cast<void *>(ptr), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// workspace: qq, kq (int8 codes), sq, sk (fp32 scales), mu (fp32 means), partial (fp64 sums)
+int64_t attn_workspace(int64_t B, int64_t Lq, int64_t Lk, int64_t H, int64_t D, int64_t *off)
+{
+    auto up = [](int64_t v) { return (v + 255) / 256 * 256; };
+    int64_t o[6];
+    o[0] = 0;
+    o[1] = o[0] + up(B * Lq * H * D);
+    o[2] = o[1] + up(B * Lk * H * D);
+    o[3] = o[2] + up(4 * B * H * Lq);
+    o[4] = o[3] + up(4 * B * H * Lk);
+    o[5] = o[4] + up(4 * B * H * D);
+    const int64_t total = o[5] + up(8 * B * H * kAttnSumSplits * D);
+    if (off)
+        for (int i = 0; i < 6; ++i)
+            off[i] = o[i];
+    return total;
+}
+
+template <int G>
+void launch_attn_rowquant(const AttnQuantParams &p, int sm_count, cudaStream_t cs)
+{
+    const int64_t chunks = (p.rows + 7) / 8;
+    int64_t blocks = (chunks + 7) / 8;  // 8 warps per block
+    const int64_t cap = static_cast<int64_t>(sm_count) * 8;
+    if (blocks > cap)
+        blocks = cap;
+    attn_rowquant_kernel<G><<<static_cast<unsigned>(blocks), 256, 0, cs>>>(p);
+}
+
+sdnq_status run_attention(const uint16_t *q, const uint16_t *k, const uint16_t *v, int64_t B,
+                          int64_t Lq, int64_t Lk, int64_t H, int64_t D, int32_t group, float scale,
+                          int32_t smooth_k, void *ws, int64_t ws_bytes, uint16_t *o, void *stream)
+{
+    if (!q || !k || !v || !o || !ws)
+        return SDNQ_ERR_NULL;
+    if (B <= 0 || Lq <= 0 || Lk <= 0 || H <= 0 || B * H > INT32_MAX || Lq > INT32_MAX ||
+        Lk > INT32_MAX || (B * H) * ((Lq + 127) / 128) > INT32_MAX)
+        return SDNQ_ERR_SHAPE;
+    if (D != kAttnD || !is_pow2(group) || group < SDNQ_MIN_GROUP || group > SDNQ_MAX_GROUP)
+        return SDNQ_ERR_UNSUPPORTED;
+    int64_t off[6];
+    if (ws_bytes < attn_workspace(B, Lq, Lk, H, D, off))
+        return SDNQ_ERR_SHAPE;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
+        !aligned(ws, 256))
+        return SDNQ_ERR_ALIGN;
+    DeviceInfo dev;
+    sdnq_status st = current_device(&dev);
+    if (st != SDNQ_OK)
+        return st;
+    uint8_t *w = static_cast<uint8_t *>(ws);
+    int8_t *qq = reinterpret_cast<int8_t *>(w + off[0]);
+    int8_t *kq = reinterpret_cast<int8_t *>(w + off[1]);
+    float *sq = reinterpret_cast<float *>(w + off[2]);
+    float *sk = reinterpret_cast<float *>(w + off[3]);
+    float *mu = reinterpret_cast<float *>(w + off[4]);
+    double *partial = reinterpret_cast<double *>(w + off[5]);
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    cudaGetLastError();
+    const int32_t bh = static_cast<int32_t>(B * H);
+    if (smooth_k) {
+        attn_ksum_kernel<<<dim3(bh, kAttnSumSplits), 256, 0, cs>>>(k, static_cast<int32_t>(Lk),
+                                                                   static_cast<int32_t>(H), partial);
+        attn_kmean_kernel<<<bh, kAttnD, 0, cs>>>(partial, static_cast<int32_t>(Lk), mu);
+    } else {
+        cudaMemsetAsync(mu, 0, 4 * B * H * D, cs);
+    }
+    const int32_t ge = group < kAttnD ? group : kAttnD;
+    AttnQuantParams pq = {};
+    pq.c_g = static_cast<float>(1.0 / std::sqrt(static_cast<double>(ge)));
+    pq.H = static_cast<int32_t>(H);
+    for (int pass = 0; pass < 2; ++pass) {
+        pq.x = pass == 0 ? q : k;
+        pq.mu = pass == 0 ? nullptr : mu;
+        pq.q = pass == 0 ? qq : kq;
+        pq.s = pass == 0 ? sq : sk;
+        pq.L = static_cast<int32_t>(pass == 0 ? Lq : Lk);
+        pq.rows = B * pq.L * H;
+        switch (ge) {
+        case 8: launch_attn_rowquant<8>(pq, dev.sm_count, cs); break;
+        case 16: launch_attn_rowquant<16>(pq, dev.sm_count, cs); break;
+        case 32: launch_attn_rowquant<32>(pq, dev.sm_count, cs); break;
+        case 64: launch_attn_rowquant<64>(pq, dev.sm_count, cs); break;
+        default: launch_attn_rowquant<128>(pq, dev.sm_count, cs); break;
+        }
+    }
+    CUtensorMap tmQ, tmK, tmV;
+    const uint64_t row = static_cast<uint64_t>(H * D);
+    if (!make_tmap_3d(&tmQ, CU_TENSOR_MAP_DATA_TYPE_UINT8, qq, row, Lq, B, row, row * Lq, 128, 128) ||
+        !make_tmap_3d(&tmK, CU_TENSOR_MAP_DATA_TYPE_UINT8, kq, row, Lk, B, row, row * Lk, 128, 128) ||
+        !make_tmap_3d(&tmV, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, v, row, Lk, B, 2 * row, 2 * row * Lk,
+                      64, 128))
+        return SDNQ_ERR_CUDA;
+    static std::once_flag once;
+    static bool smem_ok = false;
+    std::call_once(once, [] { smem_ok = set_smem(attn_kernel, AttnConfig::SMEM_BYTES); });
+    if (!smem_ok)
+        return SDNQ_ERR_CUDA;
+    AttnParams p = {};
+    p.sq = sq;
+    p.sk = sk;
+    p.o = o;
+    p.B = static_cast<int32_t>(B);
+    p.Lq = static_cast<int32_t>(Lq);
+    p.Lk = static_cast<int32_t>(Lk);
+    p.H = static_cast<int32_t>(H);
+    p.q_blocks = static_cast<int32_t>((Lq + 127) / 128);
+    p.scale = scale;
+    p.timeout_ns = kDefaultTimeoutNs;
+    attn_kernel<<<static_cast<unsigned>(bh * p.q_blocks), AttnConfig::THREADS, AttnConfig::SMEM_BYTES,
+                  cs>>>(tmQ, tmK, tmV, p);
+    return launch_status();
+}
+
 // ---------------------------------------------------------------- self-test kernel
 
 __global__ void wait_timeout_selftest_kernel(uint64_t limit_ns)
@@ -705,6 +839,22 @@ SDNQ_API sdnq_status sdnq_fp8_linear(const uint8_t *qx, const float *sx, const u
                                      void *stream)
 {
     return run_fp8_linear(qx, sx, qW, sW, bias, M, N, K, out, ldo, acc_out, stream);
+}
+
+SDNQ_API int64_t sdnq_attention_workspace(int64_t B, int64_t Lq, int64_t Lk, int64_t H,
+                                          int64_t D, int64_t *offsets)
+{
+    if (B <= 0 || Lq <= 0 || Lk <= 0 || H <= 0 || D <= 0)
+        return -1;
+    return attn_workspace(B, Lq, Lk, H, D, offsets);
+}
+
+SDNQ_API sdnq_status sdnq_attention_int8qk(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                                           int64_t B, int64_t Lq, int64_t Lk, int64_t H, int64_t D,
+                                           int32_t group, float scale, int32_t smooth_k, void *ws,
+                                           int64_t ws_bytes, uint16_t *o, void *stream)
+{
+    return run_attention(q, k, v, B, Lq, Lk, H, D, group, scale, smooth_k, ws, ws_bytes, o, stream);
 }
 
 SDNQ_API sdnq_status sdnq_int8_linear_gelu(const int8_t *qx, const float *sx, const int8_t *qW,

@@ -264,6 +264,31 @@ sdnq_status sdnq_fp8_linear(const uint8_t *qx, const float *sx, const uint8_t *q
                             int64_t K, uint16_t *out, int64_t ldo, float *acc_out, void *stream);
 
 /*
+ * Attention with a Hadamard-rotated int8 QK^T and a bf16 PV ("SDNQ: SD.Next Quantization
+ * Engine", SDNQ attention: int8 QK matmul, smooth_k, use_hadamard, hadamard_group_size; PV
+ * matmul unquantized). q [B, Lq, H, D], k and v [B, Lk, H, D], o [B, Lq, H, D], all bf16 and
+ * dense (token-head rows of D contiguous values), 16-byte aligned; D must be 128.
+ *   smooth_k != 0: mu[b][h][d] = fp32(sum_j k / Lk) (sum in fp64) is subtracted from every
+ *   key in fp32 (the softmax is unchanged by it); else mu = 0.
+ *   Q rows and K - mu rows are rotated by the butterfly over groups of min(group, D) and
+ *   quantized per row exactly as sdnq_rotquant_act does; logits are
+ *   fp32(fp32(fp32(acc) * fp32(s_q * s_k)) * scale), acc the int32 dot product of the codes;
+ *   o = softmax(logits) v, with the probabilities rounded to bf16 for the PV product (fp32
+ *   accumulation) and o rounded to bf16. A usual scale is fp32(1/sqrt(D)).
+ *   group: power of two, SDNQ_MIN_GROUP..SDNQ_MAX_GROUP (groups above D act as D).
+ *   ws: caller workspace of sdnq_attention_workspace(...) bytes, 256-byte aligned. Afterwards
+ *   it holds, at the offsets that function reports: [0] Q codes int8 [B, Lq, H, D], [1] K codes,
+ *   [2] Q scales fp32 [B, H, Lq], [3] K scales [B, H, Lk], [4] mu fp32 [B, H, D], [5] scratch.
+ * Launches: (smooth_k) two for mu, two row quantizers, one attention kernel.
+ */
+int64_t sdnq_attention_workspace(int64_t B, int64_t Lq, int64_t Lk, int64_t H, int64_t D,
+                                 int64_t *offsets /* [6] or NULL */);
+sdnq_status sdnq_attention_int8qk(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                                  int64_t B, int64_t Lq, int64_t Lk, int64_t H, int64_t D,
+                                  int32_t group, float scale, int32_t smooth_k, void *ws,
+                                  int64_t ws_bytes, uint16_t *o, void *stream);
+
+/*
  * GELU between the up and down projections of a DiT MLP (exact erf form,
  * x * Phi(x), rounded once to bf16). Not on the pages; the MLP workload needs it.
  *   in [M, N] bf16 row stride ld_in; out [M, N] bf16 row stride ld_out (may alias in when
