@@ -91,7 +91,11 @@ def profiled_traffic(kernel: str, workload: str):
 # ---------------------------------------------------------------------- workloads
 
 def workload_ops(case, name):
-    """int8 GEMM ops (2*M*N*K summed over the step's GEMMs) and extra bf16 LoRA flops."""
+    """int8 GEMM ops (2*M*N*K summed over the step's GEMMs) and extra bf16 LoRA flops; for
+    attention, the int8 QK ops and the bf16 PV flops (2 L^2 D per head each)."""
+    if case.extra.get("attn"):
+        qk = 2 * case.extra["B"] * case.N * case.M * case.M * case.K
+        return 2 * qk, 0
     if name.startswith("grad_"):
         return 2 * case.M * case.N * case.K, 0   # dy [M, N] x qW [N, K]
     if name.startswith("dit_mlp"):
@@ -126,10 +130,24 @@ class Step:
         self.qx = torch.empty((case.M, case.K), dtype=torch.int8, device=dev)
         self.sx = torch.empty((case.M,), dtype=torch.float32, device=dev)
         self.bias = case.bias.to(dev) if case.bias is not None else None
-        self.qW, self.sW = sd.sdnq_rotate_quant_weight(case.W.to(dev), g)
+        if not case.extra.get("attn"):
+            self.qW, self.sW = sd.sdnq_rotate_quant_weight(case.W.to(dev), g)
         self.out = torch.empty((case.M, case.N), dtype=torch.bfloat16, device=dev)
         self.gemm_stages = []
-        if name.startswith("fp8_"):
+        if case.extra.get("attn"):
+            B, L, H, D = case.extra["B"], case.M, case.N, case.K
+            self.k = case.W.to(dev)
+            self.v = case.extra["v"].to(dev)
+            self.out = torch.empty((B, L, H, D), dtype=torch.bfloat16, device=dev)
+            total, _ = sd._native.attention_workspace(B, L, L, H, D)
+            self.ws = torch.empty(total, dtype=torch.uint8, device=dev)
+            self.stages = [
+                ("rotquant", lambda: sd._native.sdnq_attention_prep(self.x, self.k, g, ws=self.ws)),
+                ("attention", lambda: sd._native.sdnq_attention_core(self.v, L, self.ws, out=self.out)),
+            ]
+            self.gemm_stages = ["attention"]
+            self.launches = 5   # two for the key means, two quantizers, the attention kernel
+        elif name.startswith("fp8_"):
             # the FP8 (e4m3) variant: rotate + quantize to e4m3, then the kind::f8f6f4 GEMM
             self.qW, self.sW = sd.sdnq_rotquant_fp8(case.W.to(dev), g)
             self.qx = torch.empty((case.M, case.K), dtype=torch.uint8, device=dev)
@@ -264,6 +282,12 @@ def oracle_step(case, rows, nthreads):
     """The oracle's pass over `rows` tokens of the workload (weights already quantized)."""
     import oracle
     from hadamard_rotated_int8_b200 import synthetic
+    if case.extra.get("attn"):
+        import numpy as np
+        qb = np.ascontiguousarray(synthetic.bits(case.x)[:, :rows])
+        oracle.attention(qb, synthetic.bits(case.W), synthetic.bits(case.extra["v"]), case.g,
+                         nthreads=nthreads)
+        return
     xb = synthetic.bits(case.x)[:rows]
     if case.extra.get("fp8"):
         qx, sx = oracle.rotate_quantize_fp8(xb, case.g, nthreads)
@@ -294,6 +318,9 @@ def oracle_step(case, rows, nthreads):
 def oracle_prepare(case, name, nthreads):
     import oracle
     from hadamard_rotated_int8_b200 import synthetic
+    if case.extra.get("attn"):
+        case._oracle_down = None
+        return
     quant = oracle.rotate_quantize_fp8 if case.extra.get("fp8") else oracle.rotate_quantize
     case._oracle_qW, case._oracle_sW = quant(synthetic.bits(case.W), case.g, nthreads)
     case._oracle_down = None
@@ -325,7 +352,10 @@ def cpu_baseline(case, name, budget_s=12.0):
         reps += 1
     tops = ops_per_row * rows * reps / total / 1e12
     return {"value": tops, "unit": "TOPS", "cores": nthreads, "kind": "oracle",
-            "sample": (f"{rows} of {case.M} tokens of {name} x{reps} (int8 of dy*sW, NN int8 "
+            "sample": (f"{rows} of {case.M} query tokens of {name} x{reps} (smooth_k means, "
+                       f"rotate + int8 of q and k, int32 logits, fp64 softmax and PV over all "
+                       f"{case.M} keys of {case.N} heads), {total:.2f} s") if case.extra.get("attn") else
+                      (f"{rows} of {case.M} tokens of {name} x{reps} (int8 of dy*sW, NN int8 "
                        f"GEMM against the {case.N}x{case.K} codes, inverse-rotation epilogue), "
                        f"{total:.2f} s") if case.extra.get("grad") else
                       (f"{rows} of {case.M} tokens of {name} x{reps} (rotate+quantize, int8 GEMM "
@@ -402,6 +432,10 @@ def config_of(case, args):
          "l2": "flushed before every timed step (write of 2x the L2 size)"}
     if args.workload.startswith("dit_mlp"):
         c["chain"] = "rotquant -> up GEMM with GELU epilogue -> rotquant -> down GEMM"
+    if case.extra.get("attn"):
+        c["attention"] = {"B": case.extra["B"], "L": case.M, "H": case.N, "D": case.K,
+                          "qk": "int8, Hadamard-rotated, smooth_k", "pv": "bf16",
+                          "ops": "int8 QK 2 L^2 D H + bf16 PV 2 L^2 D H"}
     if args.workload.startswith("grad_"):
         c["chain"] = ("input gradient of a frozen [N, K] layer: int8 of dy*sW [M, N] -> "
                       "NN int8 GEMM with row scale + inverse Hadamard epilogue -> dx [M, K]")
@@ -495,11 +529,16 @@ def main():
     if not args.no_e2e:
         n_e2e = max(3, min(args.steps, 50))
         x_host = case.x.pin_memory()
+        extra_in = []
+        if case.extra.get("attn"):
+            extra_in = [(step.k, case.W.pin_memory()), (step.v, case.extra["v"].pin_memory())]
         out_host = torch.empty(step.out.shape if not args.workload.startswith("dit_mlp")
                                else step.down.shape, dtype=torch.bfloat16).pin_memory()
         res = step.down if args.workload.startswith("dit_mlp") else step.out
         for _ in range(2):
             step.x.copy_(x_host, non_blocking=True)
+            for dst, src in extra_in:
+                dst.copy_(src, non_blocking=True)
             step.run()
             out_host.copy_(res, non_blocking=True)
         torch.cuda.synchronize()
@@ -509,17 +548,22 @@ def main():
         e0.record()
         for _ in range(n_e2e):
             step.x.copy_(x_host, non_blocking=True)
+            for dst, src in extra_in:
+                dst.copy_(src, non_blocking=True)
             step.run()
             out_host.copy_(res, non_blocking=True)
         e1.record()
         torch.cuda.synchronize()
         te = reduce_max_over_ranks([e0.elapsed_time(e1)], dist, world)
         e2e = {"value": whole_job_tops(ops, world, te[0] / n_e2e), "unit": "TOPS",
-               "h2d_bytes_per_step": x_host.numel() * 2,
+               "h2d_bytes_per_step": (x_host.numel() + sum(t.numel() for _, t in extra_in)) * 2,
                "d2h_bytes_per_step": out_host.numel() * 2, "steps": n_e2e}
 
     peaks, peak_src = measured_peaks()
     int8_peak = peaks["bf16_tflops"] * NOMINAL_INT8_OVER_BF16
+    if case.extra.get("attn"):
+        # half the ops run int8 (QK), half bf16 (PV): the ceiling of that mix
+        int8_peak = 2.0 / (1.0 / int8_peak + 1.0 / peaks["bf16_tflops"])
     gemm_ms = sum(stage_ms[n] for n in step.gemm_stages) / args.steps
     gemm_launch_ms = gemm_ms / len(step.gemm_stages)
     gemm_tops = ops / (gemm_ms * 1e-3) / 1e12
@@ -533,8 +577,14 @@ def main():
         rq_note = "standalone rotquant kernel on the step's input (the step itself runs it fused)"
     grad = args.workload.startswith("grad_")
     rq_rows_k = case.N if grad else case.K        # row length of the quantized operand
-    rq_gbs = rotquant_bytes(case.M, rq_rows_k) / (rq_ms * 1e-3) / 1e9
-    gemm_kernel = ("gemm_s8_kernel_e4m3" if args.workload.startswith("fp8_") else
+    rq_bytes = rotquant_bytes(case.M, rq_rows_k)
+    if case.extra.get("attn"):
+        # q and k rows of D (read bf16, write int8 + scale) and k read once more for the means
+        n_el = case.extra["B"] * case.M * case.N * case.K
+        rq_bytes = 2 * (3 * n_el + 4 * n_el // case.K) + 2 * n_el
+    rq_gbs = rq_bytes / (rq_ms * 1e-3) / 1e9
+    gemm_kernel = ("attn_kernel" if case.extra.get("attn") else
+                   "gemm_s8_kernel_e4m3" if args.workload.startswith("fp8_") else
                    "gemm_s8_kernel_grad_input" if grad else
                    "gemm_s8_kernel_fused_quantizer" if "fused" in stage_ms else
                    "gemm_s8_kernel" if case.A is None else "gemm_s8_kernel_lora")
@@ -559,7 +609,7 @@ def main():
             "bound": "hbm", "achieved": rq_gbs,
             "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": rq_gbs / peaks["hbm_gbs"],
             "traffic": profiled_traffic("rotquant", args.workload),
-            "bytes_per_launch": rotquant_bytes(case.M, rq_rows_k), "ms_per_launch": rq_ms,
+            "bytes_per_launch": rq_bytes, "ms_per_launch": rq_ms,
             "peak_source": f"{peak_src} copy bandwidth", "timing": rq_note,
         },
         "stage_ms_per_step": {n: stage_ms[n] / args.steps for n in names},

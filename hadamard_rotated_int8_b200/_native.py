@@ -57,6 +57,8 @@ SIGNATURES = {
     "sdnq_attention_workspace": [_I64, _I64, _I64, _I64, _I64, _P],
     "sdnq_attention_int8qk": [_P, _P, _P, _I64, _I64, _I64, _I64, _I64, _I32, _F, _I32, _P, _I64,
                               _P, _P],
+    "sdnq_attention_prep": [_P, _P, _I64, _I64, _I64, _I64, _I64, _I32, _I32, _P, _I64, _P],
+    "sdnq_attention_core": [_P, _I64, _I64, _I64, _I64, _I64, _F, _P, _I64, _P, _P],
     "sdnq_fp8_linear": [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _I64, _P, _P],
     "sdnq_device_status": [_P],
     "sdnq_selftest_wait_timeout": [_I64, _P],
@@ -248,6 +250,33 @@ def sdnq_attention_int8qk(q, k, v, group: int = 256, scale: float | None = None,
     _check(lib().sdnq_attention_int8qk(_ptr(q), _ptr(k), _ptr(v), B, Lq, Lk, H, D, group, scale,
                                        1 if smooth_k else 0, _ptr(ws), ws.numel(), _ptr(out),
                                        _stream(stream)), "sdnq_attention_int8qk")
+    return out
+
+
+def sdnq_attention_prep(q, k, group: int = 256, smooth_k: bool = True, ws=None, stream=None):
+    """The preparation half: smooth_k means and Q / K codes and scales into ``ws``."""
+    for t, n in ((q, "q"), (k, "k")):
+        _req(t, torch.bfloat16, n, 4)
+        _dense(t, n)
+    B, Lq, H, D = q.shape
+    Lk = k.shape[1]
+    total, _ = attention_workspace(B, Lq, Lk, H, D)
+    ws = torch.empty(total, dtype=torch.uint8, device=q.device) if ws is None else ws
+    _check(lib().sdnq_attention_prep(_ptr(q), _ptr(k), B, Lq, Lk, H, D, group,
+                                     1 if smooth_k else 0, _ptr(ws), ws.numel(), _stream(stream)),
+           "sdnq_attention_prep")
+    return ws
+
+
+def sdnq_attention_core(v, Lq: int, ws, scale: float | None = None, out=None, stream=None):
+    """The attention kernel on a prepared ``ws``: o [B, Lq, H, D] bf16."""
+    _req(v, torch.bfloat16, "v", 4)
+    _dense(v, "v")
+    B, Lk, H, D = v.shape
+    out = torch.empty((B, Lq, H, D), dtype=torch.bfloat16, device=v.device) if out is None else out
+    scale = float(1.0 / math.sqrt(D)) if scale is None else float(scale)
+    _check(lib().sdnq_attention_core(_ptr(v), B, Lq, Lk, H, D, scale, _ptr(ws), ws.numel(),
+                                     _ptr(out), _stream(stream)), "sdnq_attention_core")
     return out
 
 

@@ -13,11 +13,12 @@
 //      - warp 0 loads the Q codes once and a 2-stage ring of (K codes, V, key scales) through TMA;
 //      - warp 1 issues S_j = Q K_j^T (tcgen05 kind::i8, int32 in a double-buffered TMEM tile)
 //        and O += P_j V_j (kind::f16, bf16 P and V, fp32 O in TMEM);
-//      - warps 2..5, one query row per thread, turn S_j into logits with the oracle's fp32 op
-//        order, fp32(fp32(acc * fp32(s_q s_k)) * scale), run an online softmax in base 2
-//        (rescaling O and the row sum only when the row maximum grows by more than 2^8, so
-//        P stays below 256), write P_j as bf16 into a 128-byte-swizzled K-major tile for the
-//        MMA, and finally write O / l as bf16.
+//      - warps 2..9, two threads per query row (64 key columns each), turn S_j into base-2
+//        logits acc * (s_q * scale * log2 e) * s_k (a few fp32 roundings away from the
+//        oracle's order; the softmax is approximate anyway), run an online softmax with
+//        ex2.approx (rescaling O and the row sum only when the row maximum grows by more
+//        than 2^8, so P stays below 256), write P_j as bf16 into a 128-byte-swizzled K-major
+//        tile for the MMA, and finally write O / l as bf16.
 // Every wait is bounded as in the GEMM kernel.
 #pragma once
 
@@ -165,6 +166,14 @@ __global__ void __launch_bounds__(256) attn_rowquant_kernel(const AttnQuantParam
 
 // ---------------------------------------------------------------- the attention kernel
 
+// 2^x in one MUFU instruction (relative error about 2^-22; 0 for x = -inf)
+__device__ __forceinline__ float ex2_approx(float x)
+{
+    float r;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+
 struct AttnParams {
     const float *sq;       // [B][H][Lq] query scales
     const float *sk;       // [B][H][Lk] key scales
@@ -176,13 +185,14 @@ struct AttnParams {
 };
 
 struct AttnConfig {
-    static constexpr int THREADS = 192;                   // 6 warps
+    static constexpr int THREADS = 320;                   // loader, MMA, 8 softmax warps
     static constexpr int Q_OFF = 0;                       // int8 [128 x 128]
     static constexpr int K_OFF = 16384;                   // 2 stages x int8 [128 x 128]
     static constexpr int V_OFF = K_OFF + 2 * 16384;       // 2 stages x bf16 [128 x 128]
     static constexpr int P_OFF = V_OFF + 2 * 32768;       // bf16 [128 x 128], K-major
     static constexpr int SK_OFF = P_OFF + 32768;          // 2 stages x 128 fp32
-    static constexpr int BAR_OFF = SK_OFF + 2 * 512;
+    static constexpr int XCH_OFF = SK_OFF + 2 * 512;      // row maxima / sums of the pairs
+    static constexpr int BAR_OFF = XCH_OFF + 3 * 128 * 2 * 4;
     // barriers: q_full, kv_full[2], kv_empty[2], s_full[2], s_empty[2], p_full, pv_done, drain
     static constexpr int NBARS = 12;
     static constexpr int SMEM_BYTES = 1024 + BAR_OFF + NBARS * 8 + 16;
@@ -225,9 +235,9 @@ __global__ void __launch_bounds__(AttnConfig::THREADS, 1)
             mbar_init(kv_full(s), 1);
             mbar_init(kv_empty(s), 1);
             mbar_init(s_full(s), 1);
-            mbar_init(s_empty(s), 4);
+            mbar_init(s_empty(s), 8);
         }
-        mbar_init(p_full, 4);
+        mbar_init(p_full, 8);
         mbar_init(pv_done, 1);
         mbar_init(drain_bar, 1);
         *abort = 0;
@@ -338,15 +348,22 @@ __global__ void __launch_bounds__(AttnConfig::THREADS, 1)
             mbar_wait_bounded(drain_bar, 0u, &no_abort, p.timeout_ns);
         }
     } else {
-        // ------------------------------------------------------------ softmax (warps 2..5)
+        // ------------------------------------------------------------ softmax (warps 2..9)
+        // Two threads per query row: warps w and w + 4 share the TMEM lane quarter and take
+        // key columns (and O columns) [64 half, 64 half + 64). They combine their row maxima
+        // through shared memory and a named barrier of the pair (ids 1..4, 64 threads).
         const uint32_t quad = warp & 3u;
+        const uint32_t half = (warp - 2u) >> 2;
+        const uint32_t pair_bar = 1u + quad;
         const int32_t r = static_cast<int32_t>(quad * 32u + lane);   // query row in the block
         const bool row_ok = q0 + r < p.Lq;
         const float sqr = row_ok ? p.sq[static_cast<int64_t>(bh) * p.Lq + q0 + r] : 0.0f;
+        // logit * log2(e) = acc * (s_q * scale * log2 e) * s_k: the row factor folded once
+        const float row_f = sqr * p.scale * 1.4426950408889634f;
         const uint32_t t_lane = tmem_base + ((quad * 32u) << 16);
-        const float kLog2e = 1.4426950408889634f;
+        float *xch = reinterpret_cast<float *>(smem + C::XCH_OFF);   // [2][128][2]
         float m_used = -INFINITY;  // base-2 maximum the exponentials are taken against
-        float l_sum = 0.0f;
+        float l_sum = 0.0f;        // this thread's share of the row sum
         bool ok = true;
         for (int j = 0; ok && j < nkv; ++j) {
             const int s = j & 1;
@@ -358,31 +375,31 @@ __global__ void __launch_bounds__(AttnConfig::THREADS, 1)
                 break;
             }
             tc_fence_after_sync();
-            float y[kAttnBlock];
+            float y[64];
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
+            for (int c = 0; c < 2; ++c) {
                 uint32_t a[32];
-                tmem_ld_32x32b_x32(t_lane + s * 128 + c * 32, a);
+                tmem_ld_32x32b_x32(t_lane + s * 128 + half * 64 + c * 32, a);
                 tmem_ld_wait();
 #pragma unroll
                 for (int i = 0; i < 32; ++i)
-                    y[c * 32 + i] = __int_as_float(static_cast<int>(a[i]));  // raw bits for now
+                    y[c * 32 + i] = __int2float_rn(static_cast<int>(a[i]));
             }
             tc_fence_before_sync();
             __syncwarp();
             if (lane == 0)
                 mbar_arrive(s_empty(s));
-            // logits in the oracle's fp32 order, then base 2; keys past Lk masked
-            const int32_t j0 = j * kAttnBlock;
+            const int32_t j0 = j * kAttnBlock + static_cast<int32_t>(half) * 64;
+            const float *skb = sk_smem + s * kAttnBlock + half * 64;
             float mb = -INFINITY;
 #pragma unroll
-            for (int c = 0; c < kAttnBlock; ++c) {
-                const float t = __fmul_rn(sqr, sk_smem[s * kAttnBlock + c]);
-                const float v = __fmul_rn(__int2float_rn(__float_as_int(y[c])), t);
-                const float lg = __fmul_rn(v, p.scale);
-                y[c] = j0 + c < p.Lk ? __fmul_rn(lg, kLog2e) : -INFINITY;
+            for (int c = 0; c < 64; ++c) {
+                y[c] = j0 + c < p.Lk ? y[c] * (row_f * skb[c]) : -INFINITY;
                 mb = fmaxf(mb, y[c]);
             }
+            xch[((j & 1) * 128 + r) * 2 + half] = mb;
+            asm volatile("bar.sync %0, %1;" ::"r"(pair_bar), "r"(64) : "memory");
+            mb = fmaxf(mb, xch[((j & 1) * 128 + r) * 2 + (half ^ 1u)]);
             // P_{j-1} has left the P tile (and O is stable) once PV_{j-1} is done
             if (j >= 1) {
                 got = mbar_wait_bounded(pv_done, static_cast<uint32_t>(j - 1) & 1u, abort, p.timeout_ns);
@@ -392,45 +409,46 @@ __global__ void __launch_bounds__(AttnConfig::THREADS, 1)
                 }
                 tc_fence_after_sync();
             }
-            // rescale O and l only when the maximum grows by more than 8 (p stays <= 256)
+            // rescale O and l only when the maximum grows by more than 8 (p stays <= 256);
+            // both threads of a row see the same maximum and decide alike
             const bool grow = mb > m_used + 8.0f;
             if (__any_sync(0xffffffffu, grow)) {
                 const float m_new = grow ? mb : m_used;
-                const float alpha = grow && m_used != -INFINITY ? exp2f(m_used - m_new)
+                const float alpha = grow && m_used != -INFINITY ? ex2_approx(m_used - m_new)
                                                                 : (grow ? 0.0f : 1.0f);
                 if (j >= 1) {
 #pragma unroll 1
-                    for (int c = 0; c < 4; ++c) {
+                    for (int c = 0; c < 2; ++c) {
                         uint32_t a[32];
-                        tmem_ld_32x32b_x32(t_lane + 256 + c * 32, a);
+                        tmem_ld_32x32b_x32(t_lane + 256 + half * 64 + c * 32, a);
                         tmem_ld_wait();
 #pragma unroll
                         for (int i = 0; i < 32; ++i)
                             a[i] = __float_as_uint(__uint_as_float(a[i]) * alpha);
-                        tmem_st_32x32b_x32(t_lane + 256 + c * 32, a);
+                        tmem_st_32x32b_x32(t_lane + 256 + half * 64 + c * 32, a);
                     }
                     tmem_st_wait();
                 }
                 l_sum *= alpha;
                 m_used = m_new;
             }
-            // P = 2^(y - m), bf16, into the swizzled K-major tile: row r, 16-byte chunks
-            const uint32_t prow = base + C::P_OFF + static_cast<uint32_t>(r) * 128u;
+            // P = 2^(y - m), bf16, into this thread's 64-column atom of the swizzled K-major
+            // tile (row r: 8 chunks of 16 bytes, chunk index XOR r mod 8)
+            const uint32_t prow = base + C::P_OFF + half * 16384u + static_cast<uint32_t>(r) * 128u;
 #pragma unroll
-            for (int ch = 0; ch < 16; ++ch) {
+            for (int ch = 0; ch < 8; ++ch) {
                 uint32_t w[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    const float p0 = exp2f(y[ch * 8 + 2 * e] - m_used);
-                    const float p1 = exp2f(y[ch * 8 + 2 * e + 1] - m_used);
+                    const float p0 = ex2_approx(y[ch * 8 + 2 * e] - m_used);
+                    const float p1 = ex2_approx(y[ch * 8 + 2 * e + 1] - m_used);
                     l_sum += p0;
                     l_sum += p1;
                     const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
                     w[e] = *reinterpret_cast<const uint32_t *>(&h2);
                 }
-                const uint32_t atom = static_cast<uint32_t>(ch >> 3);
-                const uint32_t c16 = static_cast<uint32_t>(ch & 7) ^ (static_cast<uint32_t>(r) & 7u);
-                sts_v4(prow + atom * 16384u + (c16 << 4), w[0], w[1], w[2], w[3]);
+                const uint32_t c16 = static_cast<uint32_t>(ch) ^ (static_cast<uint32_t>(r) & 7u);
+                sts_v4(prow + (c16 << 4), w[0], w[1], w[2], w[3]);
             }
             fence_proxy_async_smem();
             tc_fence_before_sync();
@@ -438,17 +456,21 @@ __global__ void __launch_bounds__(AttnConfig::THREADS, 1)
             if (lane == 0)
                 mbar_arrive(p_full);
         }
-        // O / l as bf16
+        // O / l as bf16: the two halves' row sums combined, each thread its 64 O columns
         bool fin = ok && mbar_wait_bounded(pv_done, static_cast<uint32_t>(nkv - 1) & 1u, abort,
                                            p.timeout_ns);
+        xch[(2 * 128 + r) * 2 + half] = l_sum;
+        asm volatile("bar.sync %0, %1;" ::"r"(pair_bar), "r"(64) : "memory");
+        const float l_tot = l_sum + xch[(2 * 128 + r) * 2 + (half ^ 1u)];
         if (__all_sync(0xffffffffu, fin)) {
             tc_fence_after_sync();
-            const float inv = 1.0f / l_sum;
-            uint16_t *orow = p.o + ((static_cast<int64_t>(b) * p.Lq + q0 + r) * p.H + h) * kAttnD;
+            const float inv = 1.0f / l_tot;
+            uint16_t *orow = p.o + ((static_cast<int64_t>(b) * p.Lq + q0 + r) * p.H + h) * kAttnD +
+                             half * 64;
 #pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
+            for (int c = 0; c < 2; ++c) {
                 uint32_t a[32];
-                tmem_ld_32x32b_x32(t_lane + 256 + c * 32, a);
+                tmem_ld_32x32b_x32(t_lane + 256 + half * 64 + c * 32, a);
                 tmem_ld_wait();
                 uint32_t w[16];
 #pragma unroll

@@ -689,9 +689,9 @@ void launch_attn_rowquant(const AttnQuantParams &p, int sm_count, cudaStream_t c
     attn_rowquant_kernel<G><<<static_cast<unsigned>(blocks), 256, 0, cs>>>(p);
 }
 
-sdnq_status run_attention(const uint16_t *q, const uint16_t *k, const uint16_t *v, int64_t B,
-                          int64_t Lq, int64_t Lk, int64_t H, int64_t D, int32_t group, float scale,
-                          int32_t smooth_k, void *ws, int64_t ws_bytes, uint16_t *o, void *stream)
+sdnq_status validate_attention(const void *q, const void *k, const void *v, const void *o,
+                               int64_t B, int64_t Lq, int64_t Lk, int64_t H, int64_t D,
+                               int32_t group, const void *ws, int64_t ws_bytes, int64_t *off)
 {
     if (!q || !k || !v || !o || !ws)
         return SDNQ_ERR_NULL;
@@ -700,24 +700,26 @@ sdnq_status run_attention(const uint16_t *q, const uint16_t *k, const uint16_t *
         return SDNQ_ERR_SHAPE;
     if (D != kAttnD || !is_pow2(group) || group < SDNQ_MIN_GROUP || group > SDNQ_MAX_GROUP)
         return SDNQ_ERR_UNSUPPORTED;
-    int64_t off[6];
     if (ws_bytes < attn_workspace(B, Lq, Lk, H, D, off))
         return SDNQ_ERR_SHAPE;
     if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
         !aligned(ws, 256))
         return SDNQ_ERR_ALIGN;
-    DeviceInfo dev;
-    sdnq_status st = current_device(&dev);
-    if (st != SDNQ_OK)
-        return st;
-    uint8_t *w = static_cast<uint8_t *>(ws);
+    return SDNQ_OK;
+}
+
+// smooth_k means and the Q / K codes into the workspace
+sdnq_status launch_attention_prep(const uint16_t *q, const uint16_t *k, int64_t B, int64_t Lq,
+                                  int64_t Lk, int64_t H, int64_t D, int32_t group, int32_t smooth_k,
+                                  uint8_t *w, const int64_t *off, const DeviceInfo &dev,
+                                  cudaStream_t cs)
+{
     int8_t *qq = reinterpret_cast<int8_t *>(w + off[0]);
     int8_t *kq = reinterpret_cast<int8_t *>(w + off[1]);
     float *sq = reinterpret_cast<float *>(w + off[2]);
     float *sk = reinterpret_cast<float *>(w + off[3]);
     float *mu = reinterpret_cast<float *>(w + off[4]);
     double *partial = reinterpret_cast<double *>(w + off[5]);
-    cudaStream_t cs = static_cast<cudaStream_t>(stream);
     cudaGetLastError();
     const int32_t bh = static_cast<int32_t>(B * H);
     if (smooth_k) {
@@ -746,10 +748,20 @@ sdnq_status run_attention(const uint16_t *q, const uint16_t *k, const uint16_t *
         default: launch_attn_rowquant<128>(pq, dev.sm_count, cs); break;
         }
     }
+    return launch_status();
+}
+
+// the attention kernel on prepared codes
+sdnq_status launch_attention_core(const uint16_t *v, int64_t B, int64_t Lq, int64_t Lk, int64_t H,
+                                  int64_t D, float scale, uint8_t *w, const int64_t *off,
+                                  uint16_t *o, cudaStream_t cs)
+{
     CUtensorMap tmQ, tmK, tmV;
     const uint64_t row = static_cast<uint64_t>(H * D);
-    if (!make_tmap_3d(&tmQ, CU_TENSOR_MAP_DATA_TYPE_UINT8, qq, row, Lq, B, row, row * Lq, 128, 128) ||
-        !make_tmap_3d(&tmK, CU_TENSOR_MAP_DATA_TYPE_UINT8, kq, row, Lk, B, row, row * Lk, 128, 128) ||
+    if (!make_tmap_3d(&tmQ, CU_TENSOR_MAP_DATA_TYPE_UINT8, w + off[0], row, Lq, B, row, row * Lq, 128,
+                      128) ||
+        !make_tmap_3d(&tmK, CU_TENSOR_MAP_DATA_TYPE_UINT8, w + off[1], row, Lk, B, row, row * Lk, 128,
+                      128) ||
         !make_tmap_3d(&tmV, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, v, row, Lk, B, 2 * row, 2 * row * Lk,
                       64, 128))
         return SDNQ_ERR_CUDA;
@@ -759,8 +771,8 @@ sdnq_status run_attention(const uint16_t *q, const uint16_t *k, const uint16_t *
     if (!smem_ok)
         return SDNQ_ERR_CUDA;
     AttnParams p = {};
-    p.sq = sq;
-    p.sk = sk;
+    p.sq = reinterpret_cast<const float *>(w + off[2]);
+    p.sk = reinterpret_cast<const float *>(w + off[3]);
     p.o = o;
     p.B = static_cast<int32_t>(B);
     p.Lq = static_cast<int32_t>(Lq);
@@ -769,9 +781,34 @@ sdnq_status run_attention(const uint16_t *q, const uint16_t *k, const uint16_t *
     p.q_blocks = static_cast<int32_t>((Lq + 127) / 128);
     p.scale = scale;
     p.timeout_ns = kDefaultTimeoutNs;
-    attn_kernel<<<static_cast<unsigned>(bh * p.q_blocks), AttnConfig::THREADS, AttnConfig::SMEM_BYTES,
-                  cs>>>(tmQ, tmK, tmV, p);
+    cudaGetLastError();
+    attn_kernel<<<static_cast<unsigned>(B * H * p.q_blocks), AttnConfig::THREADS,
+                  AttnConfig::SMEM_BYTES, cs>>>(tmQ, tmK, tmV, p);
     return launch_status();
+}
+
+// which: 1 = prep, 2 = core, 3 = both
+sdnq_status run_attention(const uint16_t *q, const uint16_t *k, const uint16_t *v, int64_t B,
+                          int64_t Lq, int64_t Lk, int64_t H, int64_t D, int32_t group, float scale,
+                          int32_t smooth_k, void *ws, int64_t ws_bytes, uint16_t *o, void *stream,
+                          int which)
+{
+    int64_t off[6];
+    // the parts check only the tensors they read (unused ones are passed as ws)
+    sdnq_status st = validate_attention(q, k, v, o, B, Lq, Lk, H, D, group, ws, ws_bytes, off);
+    if (st != SDNQ_OK)
+        return st;
+    DeviceInfo dev;
+    if ((st = current_device(&dev)) != SDNQ_OK)
+        return st;
+    uint8_t *w = static_cast<uint8_t *>(ws);
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    if ((which & 1) &&
+        (st = launch_attention_prep(q, k, B, Lq, Lk, H, D, group, smooth_k, w, off, dev, cs)) != SDNQ_OK)
+        return st;
+    if (which & 2)
+        return launch_attention_core(v, B, Lq, Lk, H, D, scale, w, off, o, cs);
+    return SDNQ_OK;
 }
 
 // ---------------------------------------------------------------- self-test kernel
@@ -854,7 +891,26 @@ SDNQ_API sdnq_status sdnq_attention_int8qk(const uint16_t *q, const uint16_t *k,
                                            int32_t group, float scale, int32_t smooth_k, void *ws,
                                            int64_t ws_bytes, uint16_t *o, void *stream)
 {
-    return run_attention(q, k, v, B, Lq, Lk, H, D, group, scale, smooth_k, ws, ws_bytes, o, stream);
+    return run_attention(q, k, v, B, Lq, Lk, H, D, group, scale, smooth_k, ws, ws_bytes, o, stream, 3);
+}
+
+SDNQ_API sdnq_status sdnq_attention_prep(const uint16_t *q, const uint16_t *k, int64_t B,
+                                         int64_t Lq, int64_t Lk, int64_t H, int64_t D,
+                                         int32_t group, int32_t smooth_k, void *ws,
+                                         int64_t ws_bytes, void *stream)
+{
+    // v and o are not touched by the preparation: the workspace stands in for them
+    return run_attention(q, k, static_cast<const uint16_t *>(ws), B, Lq, Lk, H, D, group, 1.0f,
+                         smooth_k, ws, ws_bytes, static_cast<uint16_t *>(ws), stream, 1);
+}
+
+SDNQ_API sdnq_status sdnq_attention_core(const uint16_t *v, int64_t B, int64_t Lq, int64_t Lk,
+                                         int64_t H, int64_t D, float scale, void *ws,
+                                         int64_t ws_bytes, uint16_t *o, void *stream)
+{
+    // q and k are not read by the attention kernel (their codes are in ws)
+    return run_attention(static_cast<const uint16_t *>(ws), static_cast<const uint16_t *>(ws), v,
+                         B, Lq, Lk, H, D, SDNQ_MAX_GROUP, scale, 0, ws, ws_bytes, o, stream, 2);
 }
 
 SDNQ_API sdnq_status sdnq_int8_linear_gelu(const int8_t *qx, const float *sx, const int8_t *qW,

@@ -140,9 +140,34 @@ GRAD_WORKLOADS = {
 }
 
 
+def make_attn_case(B, L, H, D=128, g=256, seed=0, k_offset=3.0, name="attn") -> Case:
+    """Self-attention inputs q, k, v [B, L, H, D] bf16 (q in ``x``, k in ``W``, v in
+    extra["v"]); the keys carry a per-channel offset (the bias smooth_k removes)."""
+    gen = torch.Generator("cpu").manual_seed(seed)
+    q = _normal(gen, (B, L, H, D))
+    k = _normal(gen, (B, L, H, D)) + k_offset * _normal(gen, (1, 1, H, D))
+    v = _normal(gen, (B, L, H, D))
+    return Case(name, L, H, D, g, q.to(torch.bfloat16), k.to(torch.bfloat16),
+                extra={"v": v.to(torch.bfloat16), "attn": True, "B": B, "seed": seed})
+
+
+# Attention workloads: the DiT joint attention of the linear workloads' model (Flux.1: 24
+# heads of 128 over 4608 joint tokens).
+ATTN_WORKLOADS = {
+    "attn_flux_b1_l4608_h24_d128": dict(B=1, L=4608, H=24, D=128, g=256, seed=7),
+}
+
+
 def workload(name: str, g: int | None = None, M: int | None = None) -> Case:
     """Build one of the named workloads. ``g`` overrides the Hadamard group (the QuaRot
     sweep runs 64, 128, 256); ``M`` overrides the token count (smaller samples)."""
+    if name in ATTN_WORKLOADS:
+        kw = dict(ATTN_WORKLOADS[name])
+        if g is not None:
+            kw["g"] = g
+        if M is not None:
+            kw["L"] = M
+        return make_attn_case(name=name, **kw)
     if name.startswith("fp8_"):
         # the FP8 (e4m3) variant runs on the same inputs as the int8 workload it names
         case = workload(name[len("fp8_"):], g=g, M=M)

@@ -288,6 +288,16 @@ sdnq_status sdnq_attention_int8qk(const uint16_t *q, const uint16_t *k, const ui
                                   int32_t group, float scale, int32_t smooth_k, void *ws,
                                   int64_t ws_bytes, uint16_t *o, void *stream);
 
+/* The two halves of sdnq_attention_int8qk, same arguments and rules: the preparation
+ * (smooth_k means, Q and K codes and scales into ws), and the attention kernel on a prepared
+ * ws (o from the codes, the scales and v). */
+sdnq_status sdnq_attention_prep(const uint16_t *q, const uint16_t *k, int64_t B, int64_t Lq,
+                                int64_t Lk, int64_t H, int64_t D, int32_t group,
+                                int32_t smooth_k, void *ws, int64_t ws_bytes, void *stream);
+sdnq_status sdnq_attention_core(const uint16_t *v, int64_t B, int64_t Lq, int64_t Lk, int64_t H,
+                                int64_t D, float scale, void *ws, int64_t ws_bytes, uint16_t *o,
+                                void *stream);
+
 /*
  * GELU between the up and down projections of a DiT MLP (exact erf form,
  * x * Phi(x), rounded once to bf16). Not on the pages; the MLP workload needs it.
