@@ -85,9 +85,10 @@ struct AttnQuantParams {
     const uint16_t *x;     // [B][L][H][D] bf16
     const float *mu;       // [B][H][D] or nullptr (queries)
     int8_t *q;             // [B][L][H][D]
-    float *s;              // [B][H][L]
+    float *s;              // [B][H][ls]
     int64_t rows;          // B * L * H
     int32_t L, H;
+    int32_t ls;            // scale row stride: L rounded up to a multiple of 128
     float c_g;
 };
 
@@ -158,7 +159,7 @@ __global__ void __launch_bounds__(256) attn_rowquant_kernel(const AttnQuantParam
                 const int64_t h = row % p.H;
                 const int64_t l = (row / p.H) % p.L;
                 const int64_t b = row / (static_cast<int64_t>(p.L) * p.H);
-                p.s[(b * p.H + h) * p.L + l] = zero ? 0.0f : __fmul_rn(s_z, p.c_g);
+                p.s[(b * p.H + h) * p.ls + l] = zero ? 0.0f : __fmul_rn(s_z, p.c_g);
             }
         }
     }
@@ -175,11 +176,12 @@ __device__ __forceinline__ float ex2_approx(float x)
 }
 
 struct AttnParams {
-    const float *sq;       // [B][H][Lq] query scales
-    const float *sk;       // [B][H][Lk] key scales
+    const float *sq;       // [B][H][Lq_pad] query scales (rows padded to 128)
+    const float *sk;       // [B][H][Lk_pad] key scales
     uint16_t *o;           // [B][Lq][H][D] bf16
     int32_t B, Lq, Lk, H;
     int32_t q_blocks;      // ceil(Lq / 128)
+    int32_t lq_pad, lk_pad;  // Lq, Lk rounded up to 128
     float scale;           // softmax scale applied to the logits (fp32)
     uint64_t timeout_ns;
 };
@@ -273,14 +275,12 @@ __global__ void __launch_bounds__(AttnConfig::THREADS, 1)
                 ok = false;
                 break;
             }
-            // the block's key scales (0 past Lk)
             const int32_t j0 = j * kAttnBlock;
-            for (int i = static_cast<int>(lane); i < kAttnBlock; i += 32)
-                sk_smem[s * kAttnBlock + i] =
-                    j0 + i < p.Lk ? p.sk[static_cast<int64_t>(bh) * p.Lk + j0 + i] : 0.0f;
-            __syncwarp();
             if (lane == 0) {
-                mbar_arrive_expect_tx(kv_full(s), 16384 + 32768);
+                mbar_arrive_expect_tx(kv_full(s), 16384 + 32768 + 512);
+                // the block's 128 key scales (the padded rows keep this in bounds and aligned)
+                bulk_load_1d(smem_u32(sk_smem + s * kAttnBlock),
+                             p.sk + static_cast<int64_t>(bh) * p.lk_pad + j0, 512, kv_full(s));
                 tma_load_3d(base + C::K_OFF + s * 16384, &tmK, kv_full(s), h * kAttnD, j0, b);
                 tma_load_3d(base + C::V_OFF + s * 32768, &tmV, kv_full(s), h * kAttnD, j0, b);
                 tma_load_3d(base + C::V_OFF + s * 32768 + 16384, &tmV, kv_full(s), h * kAttnD + 64,
@@ -357,7 +357,7 @@ __global__ void __launch_bounds__(AttnConfig::THREADS, 1)
         const uint32_t pair_bar = 1u + quad;
         const int32_t r = static_cast<int32_t>(quad * 32u + lane);   // query row in the block
         const bool row_ok = q0 + r < p.Lq;
-        const float sqr = row_ok ? p.sq[static_cast<int64_t>(bh) * p.Lq + q0 + r] : 0.0f;
+        const float sqr = row_ok ? p.sq[static_cast<int64_t>(bh) * p.lq_pad + q0 + r] : 0.0f;
         // logit * log2(e) = acc * (s_q * scale * log2 e) * s_k: the row factor folded once
         const float row_f = sqr * p.scale * 1.4426950408889634f;
         const uint32_t t_lane = tmem_base + ((quad * 32u) << 16);
@@ -376,14 +376,16 @@ __global__ void __launch_bounds__(AttnConfig::THREADS, 1)
             }
             tc_fence_after_sync();
             float y[64];
-#pragma unroll
-            for (int c = 0; c < 2; ++c) {
-                uint32_t a[32];
-                tmem_ld_32x32b_x32(t_lane + s * 128 + half * 64 + c * 32, a);
+            {
+                uint32_t a0[32], a1[32];
+                tmem_ld_32x32b_x32(t_lane + s * 128 + half * 64, a0);
+                tmem_ld_32x32b_x32(t_lane + s * 128 + half * 64 + 32, a1);
                 tmem_ld_wait();
 #pragma unroll
-                for (int i = 0; i < 32; ++i)
-                    y[c * 32 + i] = __int2float_rn(static_cast<int>(a[i]));
+                for (int i = 0; i < 32; ++i) {
+                    y[i] = __int2float_rn(static_cast<int>(a0[i]));
+                    y[32 + i] = __int2float_rn(static_cast<int>(a1[i]));
+                }
             }
             tc_fence_before_sync();
             __syncwarp();

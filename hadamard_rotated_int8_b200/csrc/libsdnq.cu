@@ -667,9 +667,10 @@ int64_t attn_workspace(int64_t B, int64_t Lq, int64_t Lk, int64_t H, int64_t D, 
     int64_t o[6];
     o[0] = 0;
     o[1] = o[0] + up(B * Lq * H * D);
+    const int64_t lq_pad = (Lq + 127) / 128 * 128, lk_pad = (Lk + 127) / 128 * 128;
     o[2] = o[1] + up(B * Lk * H * D);
-    o[3] = o[2] + up(4 * B * H * Lq);
-    o[4] = o[3] + up(4 * B * H * Lk);
+    o[3] = o[2] + up(4 * B * H * lq_pad);
+    o[4] = o[3] + up(4 * B * H * lk_pad);
     o[5] = o[4] + up(4 * B * H * D);
     const int64_t total = o[5] + up(8 * B * H * kAttnSumSplits * D);
     if (off)
@@ -739,6 +740,7 @@ sdnq_status launch_attention_prep(const uint16_t *q, const uint16_t *k, int64_t 
         pq.q = pass == 0 ? qq : kq;
         pq.s = pass == 0 ? sq : sk;
         pq.L = static_cast<int32_t>(pass == 0 ? Lq : Lk);
+        pq.ls = (pq.L + 127) / 128 * 128;
         pq.rows = B * pq.L * H;
         switch (ge) {
         case 8: launch_attn_rowquant<8>(pq, dev.sm_count, cs); break;
@@ -779,6 +781,8 @@ sdnq_status launch_attention_core(const uint16_t *v, int64_t B, int64_t Lq, int6
     p.Lk = static_cast<int32_t>(Lk);
     p.H = static_cast<int32_t>(H);
     p.q_blocks = static_cast<int32_t>((Lq + 127) / 128);
+    p.lq_pad = p.q_blocks * 128;
+    p.lk_pad = static_cast<int32_t>((Lk + 127) / 128 * 128);
     p.scale = scale;
     p.timeout_ns = kDefaultTimeoutNs;
     cudaGetLastError();

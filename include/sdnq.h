@@ -278,7 +278,8 @@ sdnq_status sdnq_fp8_linear(const uint8_t *qx, const float *sx, const uint8_t *q
  *   group: power of two, SDNQ_MIN_GROUP..SDNQ_MAX_GROUP (groups above D act as D).
  *   ws: caller workspace of sdnq_attention_workspace(...) bytes, 256-byte aligned. Afterwards
  *   it holds, at the offsets that function reports: [0] Q codes int8 [B, Lq, H, D], [1] K codes,
- *   [2] Q scales fp32 [B, H, Lq], [3] K scales [B, H, Lk], [4] mu fp32 [B, H, D], [5] scratch.
+ *   [2] Q scales fp32 [B, H, Lq_pad], [3] K scales [B, H, Lk_pad] (L_pad = L rounded up to a
+ *   multiple of 128; the padding is not written), [4] mu fp32 [B, H, D], [5] scratch.
  * Launches: (smooth_k) two for mu, two row quantizers, one attention kernel.
  */
 int64_t sdnq_attention_workspace(int64_t B, int64_t Lq, int64_t Lk, int64_t H, int64_t D,

@@ -50,9 +50,12 @@ def run_gpu(q, k, v, g, smooth):
     def view(i, dtype, shape):
         n = int(np.prod(shape)) * np.dtype(dtype).itemsize
         return w[off[i]:off[i] + n].view(dtype).reshape(shape)
+    lqp, lkp = (Lq + 127) // 128 * 128, (Lk + 127) // 128 * 128
     return {"o": bits_of(o), "qq": view(0, np.int8, (B, Lq, H, D)),
-            "kq": view(1, np.int8, (B, Lk, H, D)), "sq": view(2, np.float32, (B, H, Lq)),
-            "sk": view(3, np.float32, (B, H, Lk)), "mu": view(4, np.float32, (B, H, D))}
+            "kq": view(1, np.int8, (B, Lk, H, D)),
+            "sq": np.ascontiguousarray(view(2, np.float32, (B, H, lqp))[:, :, :Lq]),
+            "sk": np.ascontiguousarray(view(3, np.float32, (B, H, lkp))[:, :, :Lk]),
+            "mu": view(4, np.float32, (B, H, D))}
 
 
 def check(q, k, v, g, smooth, rows=None):
