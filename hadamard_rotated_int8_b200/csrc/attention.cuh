@@ -10,7 +10,7 @@
 //      of min(g, D) and quantized per row to int8 as in the linear path (codes, scale
 //      s = fp32(amax/127) * fp32(1/sqrt(G))); scales stored [B][H][L].
 //   3. attn_kernel: one CTA per (b, h, 128 queries).
-//      - warp 0 loads the Q codes once and a 2-stage ring of (K codes, V, key scales) through TMA;
+//      - warp 0 loads the Q codes once and a 3-stage ring of (K codes, V, key scales) through TMA;
 //      - warp 1 issues S_j = Q K_j^T (tcgen05 kind::i8, int32 in a double-buffered TMEM tile)
 //        and O += P_j V_j (kind::f16, bf16 P and V, fp32 O in TMEM);
 //      - warps 2..9, two threads per query row (64 key columns each), turn S_j into base-2
@@ -188,15 +188,16 @@ struct AttnParams {
 
 struct AttnConfig {
     static constexpr int THREADS = 320;                   // loader, MMA, 8 softmax warps
+    static constexpr int STAGES = 3;                      // K / V / key-scale ring
     static constexpr int Q_OFF = 0;                       // int8 [128 x 128]
-    static constexpr int K_OFF = 16384;                   // 2 stages x int8 [128 x 128]
-    static constexpr int V_OFF = K_OFF + 2 * 16384;       // 2 stages x bf16 [128 x 128]
-    static constexpr int P_OFF = V_OFF + 2 * 32768;       // bf16 [128 x 128], K-major
-    static constexpr int SK_OFF = P_OFF + 32768;          // 2 stages x 128 fp32
-    static constexpr int XCH_OFF = SK_OFF + 2 * 512;      // row maxima / sums of the pairs
+    static constexpr int K_OFF = 16384;                   // STAGES x int8 [128 x 128]
+    static constexpr int V_OFF = K_OFF + STAGES * 16384;  // STAGES x bf16 [128 x 128]
+    static constexpr int P_OFF = V_OFF + STAGES * 32768;  // bf16 [128 x 128], K-major
+    static constexpr int SK_OFF = P_OFF + 32768;          // STAGES x 128 fp32
+    static constexpr int XCH_OFF = SK_OFF + STAGES * 512; // row maxima / sums of the pairs
     static constexpr int BAR_OFF = XCH_OFF + 3 * 128 * 2 * 4;
-    // barriers: q_full, kv_full[2], kv_empty[2], s_full[2], s_empty[2], p_full, pv_done, drain
-    static constexpr int NBARS = 12;
+    // barriers: q_full, kv_full[S], kv_empty[S], s_full[2], s_empty[2], p_full, pv_done, drain
+    static constexpr int NBARS = 1 + 2 * STAGES + 4 + 3;
     static constexpr int SMEM_BYTES = 1024 + BAR_OFF + NBARS * 8 + 16;
     static constexpr int TMEM_COLS = 512;                 // S0 [0,128), S1 [128,256), O [256,384)
 };
@@ -211,14 +212,15 @@ __global__ void __launch_bounds__(AttnConfig::THREADS, 1)
     const uint32_t base = (raw_addr + 1023u) & ~1023u;
     uint8_t *smem = smem_raw + (base - raw_addr);
     const uint32_t bar0 = base + C::BAR_OFF;
+    constexpr int NS = C::STAGES;
     const uint32_t q_full = bar0;
     auto kv_full = [&](int s) { return bar0 + 8u * (1 + s); };
-    auto kv_empty = [&](int s) { return bar0 + 8u * (3 + s); };
-    auto s_full = [&](int s) { return bar0 + 8u * (5 + s); };
-    auto s_empty = [&](int s) { return bar0 + 8u * (7 + s); };
-    const uint32_t p_full = bar0 + 8u * 9;
-    const uint32_t pv_done = bar0 + 8u * 10;
-    const uint32_t drain_bar = bar0 + 8u * 11;
+    auto kv_empty = [&](int s) { return bar0 + 8u * (1 + NS + s); };
+    auto s_full = [&](int s) { return bar0 + 8u * (1 + 2 * NS + s); };
+    auto s_empty = [&](int s) { return bar0 + 8u * (3 + 2 * NS + s); };
+    const uint32_t p_full = bar0 + 8u * (5 + 2 * NS);
+    const uint32_t pv_done = bar0 + 8u * (6 + 2 * NS);
+    const uint32_t drain_bar = bar0 + 8u * (7 + 2 * NS);
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C::BAR_OFF + C::NBARS * 8);
     volatile int *abort = reinterpret_cast<volatile int *>(tmem_holder + 1);
     float *sk_smem = reinterpret_cast<float *>(smem + C::SK_OFF);
@@ -233,9 +235,11 @@ __global__ void __launch_bounds__(AttnConfig::THREADS, 1)
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < NS; ++s) {
             mbar_init(kv_full(s), 1);
             mbar_init(kv_empty(s), 1);
+        }
+        for (int s = 0; s < 2; ++s) {
             mbar_init(s_full(s), 1);
             mbar_init(s_empty(s), 8);
         }
@@ -266,8 +270,8 @@ __global__ void __launch_bounds__(AttnConfig::THREADS, 1)
         }
         int issued = 0;
         for (int j = 0; ok && j < nkv; ++j) {
-            const int s = j & 1;
-            const uint32_t use = static_cast<uint32_t>(j >> 1);
+            const int s = j % NS;
+            const uint32_t use = static_cast<uint32_t>(j / NS);
             bool good = true;
             if (lane == 0)
                 good = mbar_wait_bounded(kv_empty(s), (use & 1u) ^ 1u, abort, p.timeout_ns);
@@ -293,8 +297,8 @@ __global__ void __launch_bounds__(AttnConfig::THREADS, 1)
             // the last two stages; already complete on the normal path)
             volatile int no_abort = 0;
             mbar_wait_bounded(q_full, 0u, &no_abort, p.timeout_ns);
-            for (int j = issued - 2 < 0 ? 0 : issued - 2; j < issued; ++j)
-                mbar_wait_bounded(kv_full(j & 1), static_cast<uint32_t>(j >> 1) & 1u, &no_abort,
+            for (int j = issued - NS < 0 ? 0 : issued - NS; j < issued; ++j)
+                mbar_wait_bounded(kv_full(j % NS), static_cast<uint32_t>(j / NS) & 1u, &no_abort,
                                   p.timeout_ns);
         }
     } else if (warp == 1) {
@@ -310,32 +314,34 @@ __global__ void __launch_bounds__(AttnConfig::THREADS, 1)
                     return false;
                 tc_fence_after_sync();
                 const uint32_t sp = base + C::P_OFF;
-                const uint32_t sv = base + C::V_OFF + (j & 1) * 32768;
+                const uint32_t sv = base + C::V_OFF + (j % NS) * 32768;
 #pragma unroll
                 for (int k = 0; k < 8; ++k)
                     mma_f16(t_o, kmajor_desc(sp + (k >> 2) * 16384 + (k & 3) * 32),
                             mnmajor_desc(sv + 2048 * k, 16384), IDESC_PV,
                             (j | k) != 0 ? 1u : 0u);
                 tc_commit(pv_done);
-                tc_commit(kv_empty(j & 1));
+                tc_commit(kv_empty(j % NS));
                 return true;
             };
             for (int j = 0; ok && j < nkv; ++j) {
-                const int s = j & 1;
-                const uint32_t use = static_cast<uint32_t>(j >> 1);
-                if (!mbar_wait_bounded(kv_full(s), use & 1u, abort, p.timeout_ns) ||
-                    !mbar_wait_bounded(s_empty(s), (use & 1u) ^ 1u, abort, p.timeout_ns)) {
+                const int ks = j % NS;       // K/V stage
+                const int sb = j & 1;        // S buffer
+                if (!mbar_wait_bounded(kv_full(ks), static_cast<uint32_t>(j / NS) & 1u, abort,
+                                       p.timeout_ns) ||
+                    !mbar_wait_bounded(s_empty(sb), (static_cast<uint32_t>(j >> 1) & 1u) ^ 1u, abort,
+                                       p.timeout_ns)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after_sync();
                 const uint32_t sq_addr = base + C::Q_OFF;
-                const uint32_t sk_addr = base + C::K_OFF + s * 16384;
+                const uint32_t sk_addr = base + C::K_OFF + ks * 16384;
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
-                    mma_s8(tmem_base + s * 128, kmajor_desc(sq_addr + 32 * k),
+                    mma_s8(tmem_base + sb * 128, kmajor_desc(sq_addr + 32 * k),
                            kmajor_desc(sk_addr + 32 * k), IDESC_S, k != 0 ? 1u : 0u);
-                tc_commit(s_full(s));
+                tc_commit(s_full(sb));
                 if (j >= 1 && !issue_pv(j - 1)) {
                     ok = false;
                     break;
@@ -366,10 +372,12 @@ __global__ void __launch_bounds__(AttnConfig::THREADS, 1)
         float l_sum = 0.0f;        // this thread's share of the row sum
         bool ok = true;
         for (int j = 0; ok && j < nkv; ++j) {
-            const int s = j & 1;
-            const uint32_t use = static_cast<uint32_t>(j >> 1);
-            bool got = mbar_wait_bounded(s_full(s), use & 1u, abort, p.timeout_ns) &&
-                       mbar_wait_bounded(kv_full(s), use & 1u, abort, p.timeout_ns);
+            const int s = j & 1;                 // S buffer
+            const int ks = j % NS;               // K/V stage (its key scales)
+            bool got = mbar_wait_bounded(s_full(s), static_cast<uint32_t>(j >> 1) & 1u, abort,
+                                         p.timeout_ns) &&
+                       mbar_wait_bounded(kv_full(ks), static_cast<uint32_t>(j / NS) & 1u, abort,
+                                         p.timeout_ns);
             if (!__all_sync(0xffffffffu, got)) {
                 ok = false;
                 break;
@@ -392,13 +400,15 @@ __global__ void __launch_bounds__(AttnConfig::THREADS, 1)
             if (lane == 0)
                 mbar_arrive(s_empty(s));
             const int32_t j0 = j * kAttnBlock + static_cast<int32_t>(half) * 64;
-            const float *skb = sk_smem + s * kAttnBlock + half * 64;
-            float mb = -INFINITY;
+            const float *skb = sk_smem + ks * kAttnBlock + half * 64;
+            float mx[8];
 #pragma unroll
             for (int c = 0; c < 64; ++c) {
                 y[c] = j0 + c < p.Lk ? y[c] * (row_f * skb[c]) : -INFINITY;
-                mb = fmaxf(mb, y[c]);
+                mx[c & 7] = (c < 8) ? y[c] : fmaxf(mx[c & 7], y[c]);  // 8 independent chains
             }
+            float mb = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                             fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
             xch[((j & 1) * 128 + r) * 2 + half] = mb;
             asm volatile("bar.sync %0, %1;" ::"r"(pair_bar), "r"(64) : "memory");
             mb = fmaxf(mb, xch[((j & 1) * 128 + r) * 2 + (half ^ 1u)]);
@@ -437,6 +447,7 @@ __global__ void __launch_bounds__(AttnConfig::THREADS, 1)
             // P = 2^(y - m), bf16, into this thread's 64-column atom of the swizzled K-major
             // tile (row r: 8 chunks of 16 bytes, chunk index XOR r mod 8)
             const uint32_t prow = base + C::P_OFF + half * 16384u + static_cast<uint32_t>(r) * 128u;
+            float ls[8] = {0, 0, 0, 0, 0, 0, 0, 0};  // 8 independent partial sums
 #pragma unroll
             for (int ch = 0; ch < 8; ++ch) {
                 uint32_t w[4];
@@ -444,14 +455,15 @@ __global__ void __launch_bounds__(AttnConfig::THREADS, 1)
                 for (int e = 0; e < 4; ++e) {
                     const float p0 = ex2_approx(y[ch * 8 + 2 * e] - m_used);
                     const float p1 = ex2_approx(y[ch * 8 + 2 * e + 1] - m_used);
-                    l_sum += p0;
-                    l_sum += p1;
+                    ls[2 * e] += p0;
+                    ls[2 * e + 1] += p1;
                     const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
                     w[e] = *reinterpret_cast<const uint32_t *>(&h2);
                 }
                 const uint32_t c16 = static_cast<uint32_t>(ch) ^ (static_cast<uint32_t>(r) & 7u);
                 sts_v4(prow + (c16 << 4), w[0], w[1], w[2], w[3]);
             }
+            l_sum += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
             fence_proxy_async_smem();
             tc_fence_before_sync();
             __syncwarp();
