@@ -27,6 +27,10 @@
 #include "device.cuh"
 #include "rotquant.cuh"
 
+#ifndef SDNQ_ATTN_CTAS_PER_SM
+#define SDNQ_ATTN_CTAS_PER_SM 1
+#endif
+
 namespace sdnq {
 
 constexpr int kAttnD = 128;
@@ -175,6 +179,14 @@ __device__ __forceinline__ float ex2_approx(float x)
     return r;
 }
 
+// max(a, b, c) in one instruction (sm_100)
+__device__ __forceinline__ float max3f(float a, float b, float c)
+{
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
 struct AttnParams {
     const float *sq;       // [B][H][Lq_pad] query scales (rows padded to 128)
     const float *sk;       // [B][H][Lk_pad] key scales
@@ -188,21 +200,29 @@ struct AttnParams {
 
 struct AttnConfig {
     static constexpr int THREADS = 320;                   // loader, MMA, 8 softmax warps
-    static constexpr int STAGES = 3;                      // K / V / key-scale ring
+    static constexpr int CTAS_PER_SM = SDNQ_ATTN_CTAS_PER_SM;
+    // K and V rings of their own: K_j is free once S_j is done, V_j once PV_j is done
+    static constexpr int NK = CTAS_PER_SM == 2 ? 1 : 3;    // K code stages
+    static constexpr int NV = CTAS_PER_SM == 2 ? 1 : 3;    // V stages
+    static constexpr int NSK = 2;                          // key-scale stages (freed by softmax)
+    static constexpr int SBUF = CTAS_PER_SM == 2 ? 1 : 2;  // S buffers in TMEM
     static constexpr int Q_OFF = 0;                       // int8 [128 x 128]
-    static constexpr int K_OFF = 16384;                   // STAGES x int8 [128 x 128]
-    static constexpr int V_OFF = K_OFF + STAGES * 16384;  // STAGES x bf16 [128 x 128]
-    static constexpr int P_OFF = V_OFF + STAGES * 32768;  // bf16 [128 x 128], K-major
-    static constexpr int SK_OFF = P_OFF + 32768;          // STAGES x 128 fp32
-    static constexpr int XCH_OFF = SK_OFF + STAGES * 512; // row maxima / sums of the pairs
+    static constexpr int K_OFF = 16384;                   // NK x int8 [128 x 128]
+    static constexpr int V_OFF = K_OFF + NK * 16384;      // NV x bf16 [128 x 128]
+    static constexpr int P_OFF = V_OFF + NV * 32768;      // bf16 [128 x 128], K-major
+    static constexpr int SK_OFF = P_OFF + 32768;          // NSK x 128 fp32
+    static constexpr int XCH_OFF = SK_OFF + NSK * 512;    // row maxima / sums of the pairs
     static constexpr int BAR_OFF = XCH_OFF + 3 * 128 * 2 * 4;
-    // barriers: q_full, kv_full[S], kv_empty[S], s_full[2], s_empty[2], p_full, pv_done, drain
-    static constexpr int NBARS = 1 + 2 * STAGES + 4 + 3;
+    // barriers: q_full, k_full[NK], k_empty[NK], v_full[NV], v_empty[NV], sk_full[NSK],
+    // sk_empty[NSK], s_full[2], s_empty[2], p_full, pv_done, drain
+    static constexpr int NBARS = 1 + 2 * NK + 2 * NV + 2 * NSK + 4 + 3;
     static constexpr int SMEM_BYTES = 1024 + BAR_OFF + NBARS * 8 + 16;
-    static constexpr int TMEM_COLS = 512;                 // S0 [0,128), S1 [128,256), O [256,384)
+    // S buffers [0, 128 SBUF), O [128 SBUF, 128 SBUF + 128)
+    static constexpr int O_COL = 128 * SBUF;
+    static constexpr int TMEM_COLS = SBUF == 2 ? 512 : 256;
 };
 
-__global__ void __launch_bounds__(AttnConfig::THREADS, 1)
+__global__ void __launch_bounds__(AttnConfig::THREADS, AttnConfig::CTAS_PER_SM)
     attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const AttnParams p)
 {
@@ -212,15 +232,20 @@ __global__ void __launch_bounds__(AttnConfig::THREADS, 1)
     const uint32_t base = (raw_addr + 1023u) & ~1023u;
     uint8_t *smem = smem_raw + (base - raw_addr);
     const uint32_t bar0 = base + C::BAR_OFF;
-    constexpr int NS = C::STAGES;
+    constexpr int NK = C::NK, NV = C::NV, NSK = C::NSK;
     const uint32_t q_full = bar0;
-    auto kv_full = [&](int s) { return bar0 + 8u * (1 + s); };
-    auto kv_empty = [&](int s) { return bar0 + 8u * (1 + NS + s); };
-    auto s_full = [&](int s) { return bar0 + 8u * (1 + 2 * NS + s); };
-    auto s_empty = [&](int s) { return bar0 + 8u * (3 + 2 * NS + s); };
-    const uint32_t p_full = bar0 + 8u * (5 + 2 * NS);
-    const uint32_t pv_done = bar0 + 8u * (6 + 2 * NS);
-    const uint32_t drain_bar = bar0 + 8u * (7 + 2 * NS);
+    auto k_full = [&](int s) { return bar0 + 8u * (1 + s); };
+    auto k_empty = [&](int s) { return bar0 + 8u * (1 + NK + s); };
+    auto v_full = [&](int s) { return bar0 + 8u * (1 + 2 * NK + s); };
+    auto v_empty = [&](int s) { return bar0 + 8u * (1 + 2 * NK + NV + s); };
+    auto sk_full = [&](int s) { return bar0 + 8u * (1 + 2 * NK + 2 * NV + s); };
+    auto sk_empty = [&](int s) { return bar0 + 8u * (1 + 2 * NK + 2 * NV + NSK + s); };
+    constexpr int SB0 = 1 + 2 * NK + 2 * NV + 2 * NSK;
+    auto s_full = [&](int s) { return bar0 + 8u * (SB0 + s); };
+    auto s_empty = [&](int s) { return bar0 + 8u * (SB0 + 2 + s); };
+    const uint32_t p_full = bar0 + 8u * (SB0 + 4);
+    const uint32_t pv_done = bar0 + 8u * (SB0 + 5);
+    const uint32_t drain_bar = bar0 + 8u * (SB0 + 6);
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C::BAR_OFF + C::NBARS * 8);
     volatile int *abort = reinterpret_cast<volatile int *>(tmem_holder + 1);
     float *sk_smem = reinterpret_cast<float *>(smem + C::SK_OFF);
@@ -235,9 +260,17 @@ __global__ void __launch_bounds__(AttnConfig::THREADS, 1)
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
-        for (int s = 0; s < NS; ++s) {
-            mbar_init(kv_full(s), 1);
-            mbar_init(kv_empty(s), 1);
+        for (int s = 0; s < NK; ++s) {
+            mbar_init(k_full(s), 1);
+            mbar_init(k_empty(s), 1);
+        }
+        for (int s = 0; s < NV; ++s) {
+            mbar_init(v_full(s), 1);
+            mbar_init(v_empty(s), 1);
+        }
+        for (int s = 0; s < NSK; ++s) {
+            mbar_init(sk_full(s), 1);
+            mbar_init(sk_empty(s), 8);
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(s_full(s), 1);
@@ -263,42 +296,50 @@ __global__ void __launch_bounds__(AttnConfig::THREADS, 1)
 
     if (warp == 0) {
         // ------------------------------------------------------------ loads
-        bool ok = true;
+        // Per key block j, in this order: K_j and its scales, then V_j. V_j waits for PV_{j-1},
+        // which the MMA warp issues after S_j, so K_j is never held behind V_{j-1}'s release.
         if (lane == 0) {
             mbar_arrive_expect_tx(q_full, 16384);
             tma_load_3d(base + C::Q_OFF, &tmQ, q_full, h * kAttnD, q0, b);
-        }
-        int issued = 0;
-        for (int j = 0; ok && j < nkv; ++j) {
-            const int s = j % NS;
-            const uint32_t use = static_cast<uint32_t>(j / NS);
-            bool good = true;
-            if (lane == 0)
-                good = mbar_wait_bounded(kv_empty(s), (use & 1u) ^ 1u, abort, p.timeout_ns);
-            if (__shfl_sync(0xffffffffu, good ? 1 : 0, 0) == 0) {
-                ok = false;
-                break;
-            }
-            const int32_t j0 = j * kAttnBlock;
-            if (lane == 0) {
-                mbar_arrive_expect_tx(kv_full(s), 16384 + 32768 + 512);
+            int nk = 0, nsk = 0, nv = 0;   // copies issued per ring
+            for (int j = 0; j < nkv; ++j) {
+                const int32_t j0 = j * kAttnBlock;
+                const int ks = j % NK, ss = j % NSK, vs = j % NV;
+                if (!mbar_wait_bounded(k_empty(ks), (static_cast<uint32_t>(j / NK) & 1u) ^ 1u, abort,
+                                       p.timeout_ns))
+                    break;
+                mbar_arrive_expect_tx(k_full(ks), 16384);
+                tma_load_3d(base + C::K_OFF + ks * 16384, &tmK, k_full(ks), h * kAttnD, j0, b);
+                ++nk;
+                if (!mbar_wait_bounded(sk_empty(ss), (static_cast<uint32_t>(j / NSK) & 1u) ^ 1u,
+                                       abort, p.timeout_ns))
+                    break;
+                mbar_arrive_expect_tx(sk_full(ss), 512);
                 // the block's 128 key scales (the padded rows keep this in bounds and aligned)
-                bulk_load_1d(smem_u32(sk_smem + s * kAttnBlock),
-                             p.sk + static_cast<int64_t>(bh) * p.lk_pad + j0, 512, kv_full(s));
-                tma_load_3d(base + C::K_OFF + s * 16384, &tmK, kv_full(s), h * kAttnD, j0, b);
-                tma_load_3d(base + C::V_OFF + s * 32768, &tmV, kv_full(s), h * kAttnD, j0, b);
-                tma_load_3d(base + C::V_OFF + s * 32768 + 16384, &tmV, kv_full(s), h * kAttnD + 64,
+                bulk_load_1d(smem_u32(sk_smem + ss * kAttnBlock),
+                             p.sk + static_cast<int64_t>(bh) * p.lk_pad + j0, 512, sk_full(ss));
+                ++nsk;
+                if (!mbar_wait_bounded(v_empty(vs), (static_cast<uint32_t>(j / NV) & 1u) ^ 1u, abort,
+                                       p.timeout_ns))
+                    break;
+                mbar_arrive_expect_tx(v_full(vs), 32768);
+                tma_load_3d(base + C::V_OFF + vs * 32768, &tmV, v_full(vs), h * kAttnD, j0, b);
+                tma_load_3d(base + C::V_OFF + vs * 32768 + 16384, &tmV, v_full(vs), h * kAttnD + 64,
                             j0, b);
+                ++nv;
             }
-            ++issued;
-        }
-        if (lane == 0) {
             // every copy this warp started has landed before the CTA can exit (the Q tile and
-            // the last two stages; already complete on the normal path)
+            // the last uses of each ring; already complete on the normal path)
             volatile int no_abort = 0;
             mbar_wait_bounded(q_full, 0u, &no_abort, p.timeout_ns);
-            for (int j = issued - NS < 0 ? 0 : issued - NS; j < issued; ++j)
-                mbar_wait_bounded(kv_full(j % NS), static_cast<uint32_t>(j / NS) & 1u, &no_abort,
+            for (int j = nk - NK < 0 ? 0 : nk - NK; j < nk; ++j)
+                mbar_wait_bounded(k_full(j % NK), static_cast<uint32_t>(j / NK) & 1u, &no_abort,
+                                  p.timeout_ns);
+            for (int j = nsk - NSK < 0 ? 0 : nsk - NSK; j < nsk; ++j)
+                mbar_wait_bounded(sk_full(j % NSK), static_cast<uint32_t>(j / NSK) & 1u, &no_abort,
+                                  p.timeout_ns);
+            for (int j = nv - NV < 0 ? 0 : nv - NV; j < nv; ++j)
+                mbar_wait_bounded(v_full(j % NV), static_cast<uint32_t>(j / NV) & 1u, &no_abort,
                                   p.timeout_ns);
         }
     } else if (warp == 1) {
@@ -306,31 +347,33 @@ __global__ void __launch_bounds__(AttnConfig::THREADS, 1)
         if (lane == 0) {
             constexpr uint32_t IDESC_S = idesc_s8_s32(128, 128);
             constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, 128, true);
-            const uint32_t t_o = tmem_base + 256;
+            const uint32_t t_o = tmem_base + C::O_COL;
             bool ok = mbar_wait_bounded(q_full, 0u, abort, p.timeout_ns);
             auto issue_pv = [&](int j) {
                 // O (+)= P_j V_j: A = P, K-major bf16 in two 64-column atoms; B = V, N-major
-                if (!mbar_wait_bounded(p_full, static_cast<uint32_t>(j) & 1u, abort, p.timeout_ns))
+                if (!mbar_wait_bounded(v_full(j % NV), static_cast<uint32_t>(j / NV) & 1u, abort,
+                                       p.timeout_ns) ||
+                    !mbar_wait_bounded(p_full, static_cast<uint32_t>(j) & 1u, abort, p.timeout_ns))
                     return false;
                 tc_fence_after_sync();
                 const uint32_t sp = base + C::P_OFF;
-                const uint32_t sv = base + C::V_OFF + (j % NS) * 32768;
+                const uint32_t sv = base + C::V_OFF + (j % NV) * 32768;
 #pragma unroll
                 for (int k = 0; k < 8; ++k)
                     mma_f16(t_o, kmajor_desc(sp + (k >> 2) * 16384 + (k & 3) * 32),
                             mnmajor_desc(sv + 2048 * k, 16384), IDESC_PV,
                             (j | k) != 0 ? 1u : 0u);
                 tc_commit(pv_done);
-                tc_commit(kv_empty(j % NS));
+                tc_commit(v_empty(j % NV));
                 return true;
             };
             for (int j = 0; ok && j < nkv; ++j) {
-                const int ks = j % NS;       // K/V stage
-                const int sb = j & 1;        // S buffer
-                if (!mbar_wait_bounded(kv_full(ks), static_cast<uint32_t>(j / NS) & 1u, abort,
+                const int ks = j % NK;       // K stage
+                const int sb = j % C::SBUF;  // S buffer
+                if (!mbar_wait_bounded(k_full(ks), static_cast<uint32_t>(j / NK) & 1u, abort,
                                        p.timeout_ns) ||
-                    !mbar_wait_bounded(s_empty(sb), (static_cast<uint32_t>(j >> 1) & 1u) ^ 1u, abort,
-                                       p.timeout_ns)) {
+                    !mbar_wait_bounded(s_empty(sb), (static_cast<uint32_t>(j / C::SBUF) & 1u) ^ 1u,
+                                       abort, p.timeout_ns)) {
                     ok = false;
                     break;
                 }
@@ -342,6 +385,7 @@ __global__ void __launch_bounds__(AttnConfig::THREADS, 1)
                     mma_s8(tmem_base + sb * 128, kmajor_desc(sq_addr + 32 * k),
                            kmajor_desc(sk_addr + 32 * k), IDESC_S, k != 0 ? 1u : 0u);
                 tc_commit(s_full(sb));
+                tc_commit(k_empty(ks));
                 if (j >= 1 && !issue_pv(j - 1)) {
                     ok = false;
                     break;
@@ -372,17 +416,20 @@ __global__ void __launch_bounds__(AttnConfig::THREADS, 1)
         float l_sum = 0.0f;        // this thread's share of the row sum
         bool ok = true;
         for (int j = 0; ok && j < nkv; ++j) {
-            const int s = j & 1;                 // S buffer
-            const int ks = j % NS;               // K/V stage (its key scales)
-            bool got = mbar_wait_bounded(s_full(s), static_cast<uint32_t>(j >> 1) & 1u, abort,
+            const int s = j % C::SBUF;           // S buffer
+            const int ss = j % NSK;              // key-scale stage
+            bool got = mbar_wait_bounded(s_full(s), static_cast<uint32_t>(j / C::SBUF) & 1u, abort,
                                          p.timeout_ns) &&
-                       mbar_wait_bounded(kv_full(ks), static_cast<uint32_t>(j / NS) & 1u, abort,
+                       mbar_wait_bounded(sk_full(ss), static_cast<uint32_t>(j / NSK) & 1u, abort,
                                          p.timeout_ns);
             if (!__all_sync(0xffffffffu, got)) {
                 ok = false;
                 break;
             }
             tc_fence_after_sync();
+            // fp32(acc) without the conversion pipe: |acc| <= 127 * 127 * 128 < 2^22, so the
+            // bits of acc + 0x4B400000 are the float 1.5 * 2^23 + acc, and subtracting
+            // 1.5 * 2^23 (below, exact) leaves acc
             float y[64];
             {
                 uint32_t a0[32], a1[32];
@@ -391,8 +438,8 @@ __global__ void __launch_bounds__(AttnConfig::THREADS, 1)
                 tmem_ld_wait();
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
-                    y[i] = __int2float_rn(static_cast<int>(a0[i]));
-                    y[32 + i] = __int2float_rn(static_cast<int>(a1[i]));
+                    y[i] = __uint_as_float(a0[i] + 0x4B400000u);
+                    y[32 + i] = __uint_as_float(a1[i] + 0x4B400000u);
                 }
             }
             tc_fence_before_sync();
@@ -400,15 +447,38 @@ __global__ void __launch_bounds__(AttnConfig::THREADS, 1)
             if (lane == 0)
                 mbar_arrive(s_empty(s));
             const int32_t j0 = j * kAttnBlock + static_cast<int32_t>(half) * 64;
-            const float *skb = sk_smem + ks * kAttnBlock + half * 64;
-            float mx[8];
+            const float4 *skb = reinterpret_cast<const float4 *>(sk_smem + ss * kAttnBlock + half * 64);
 #pragma unroll
-            for (int c = 0; c < 64; ++c) {
-                y[c] = j0 + c < p.Lk ? y[c] * (row_f * skb[c]) : -INFINITY;
-                mx[c & 7] = (c < 8) ? y[c] : fmaxf(mx[c & 7], y[c]);  // 8 independent chains
+            for (int c4 = 0; c4 < 16; ++c4) {
+                const float4 k4 = skb[c4];   // same address across the warp: a broadcast
+                float r0, r1, r2, r3, f0, f1, f2, f3;
+                mul2(r0, r1, row_f, row_f, k4.x, k4.y);
+                mul2(r2, r3, row_f, row_f, k4.z, k4.w);
+                sub2(f0, f1, y[4 * c4], y[4 * c4 + 1], 12582912.0f, 12582912.0f);
+                sub2(f2, f3, y[4 * c4 + 2], y[4 * c4 + 3], 12582912.0f, 12582912.0f);
+                mul2(y[4 * c4], y[4 * c4 + 1], f0, f1, r0, r1);
+                mul2(y[4 * c4 + 2], y[4 * c4 + 3], f2, f3, r2, r3);
             }
-            float mb = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                             fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(sk_empty(ss));   // the stage's key scales are read
+            if (j0 + 64 > p.Lk) {            // the ragged last block (warp-uniform)
+#pragma unroll
+                for (int c = 0; c < 64; ++c)
+                    if (j0 + c >= p.Lk)
+                        y[c] = -INFINITY;
+            }
+            // 4 independent chains, chain i over the columns i + 4k (k = 0..15)
+            float mx[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                mx[i] = max3f(y[i], y[i + 4], y[i + 8]);
+#pragma unroll
+                for (int k = 3; k < 15; k += 2)
+                    mx[i] = max3f(mx[i], y[i + 4 * k], y[i + 4 * k + 4]);
+                mx[i] = fmaxf(mx[i], y[i + 60]);
+            }
+            float mb = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
             xch[((j & 1) * 128 + r) * 2 + half] = mb;
             asm volatile("bar.sync %0, %1;" ::"r"(pair_bar), "r"(64) : "memory");
             mb = fmaxf(mb, xch[((j & 1) * 128 + r) * 2 + (half ^ 1u)]);
@@ -432,12 +502,12 @@ __global__ void __launch_bounds__(AttnConfig::THREADS, 1)
 #pragma unroll 1
                     for (int c = 0; c < 2; ++c) {
                         uint32_t a[32];
-                        tmem_ld_32x32b_x32(t_lane + 256 + half * 64 + c * 32, a);
+                        tmem_ld_32x32b_x32(t_lane + C::O_COL + half * 64 + c * 32, a);
                         tmem_ld_wait();
 #pragma unroll
                         for (int i = 0; i < 32; ++i)
                             a[i] = __float_as_uint(__uint_as_float(a[i]) * alpha);
-                        tmem_st_32x32b_x32(t_lane + 256 + half * 64 + c * 32, a);
+                        tmem_st_32x32b_x32(t_lane + C::O_COL + half * 64 + c * 32, a);
                     }
                     tmem_st_wait();
                 }
@@ -453,10 +523,11 @@ __global__ void __launch_bounds__(AttnConfig::THREADS, 1)
                 uint32_t w[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    const float p0 = ex2_approx(y[ch * 8 + 2 * e] - m_used);
-                    const float p1 = ex2_approx(y[ch * 8 + 2 * e + 1] - m_used);
-                    ls[2 * e] += p0;
-                    ls[2 * e + 1] += p1;
+                    float d0, d1;
+                    sub2(d0, d1, y[ch * 8 + 2 * e], y[ch * 8 + 2 * e + 1], m_used, m_used);
+                    const float p0 = ex2_approx(d0);
+                    const float p1 = ex2_approx(d1);
+                    add2(ls[2 * e], ls[2 * e + 1], ls[2 * e], ls[2 * e + 1], p0, p1);
                     const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
                     w[e] = *reinterpret_cast<const uint32_t *>(&h2);
                 }
@@ -484,7 +555,7 @@ __global__ void __launch_bounds__(AttnConfig::THREADS, 1)
 #pragma unroll 1
             for (int c = 0; c < 2; ++c) {
                 uint32_t a[32];
-                tmem_ld_32x32b_x32(t_lane + 256 + half * 64 + c * 32, a);
+                tmem_ld_32x32b_x32(t_lane + C::O_COL + half * 64 + c * 32, a);
                 tmem_ld_wait();
                 uint32_t w[16];
 #pragma unroll
