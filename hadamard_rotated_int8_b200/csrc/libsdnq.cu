@@ -769,7 +769,10 @@ sdnq_status launch_attention_core(const uint16_t *v, int64_t B, int64_t Lq, int6
         return SDNQ_ERR_CUDA;
     static std::once_flag once;
     static bool smem_ok = false;
-    std::call_once(once, [] { smem_ok = set_smem(attn_kernel, AttnConfig::SMEM_BYTES); });
+    std::call_once(once, [] {
+        smem_ok = kAttnPingPong ? set_smem(attn_pp_kernel, AttnPPConfig::SMEM_BYTES)
+                                : set_smem(attn_kernel, AttnConfig::SMEM_BYTES);
+    });
     if (!smem_ok)
         return SDNQ_ERR_CUDA;
     AttnParams p = {};
@@ -781,13 +784,19 @@ sdnq_status launch_attention_core(const uint16_t *v, int64_t B, int64_t Lq, int6
     p.Lk = static_cast<int32_t>(Lk);
     p.H = static_cast<int32_t>(H);
     p.q_blocks = static_cast<int32_t>((Lq + 127) / 128);
-    p.lq_pad = p.q_blocks * 128;
+    p.lq_pad = p.q_blocks * 128;   // the workspace's query-scale row stride
     p.lk_pad = static_cast<int32_t>((Lk + 127) / 128 * 128);
     p.scale = scale;
     p.timeout_ns = kDefaultTimeoutNs;
     cudaGetLastError();
-    attn_kernel<<<static_cast<unsigned>(B * H * p.q_blocks), AttnConfig::THREADS,
-                  AttnConfig::SMEM_BYTES, cs>>>(tmQ, tmK, tmV, p);
+    if (kAttnPingPong) {
+        p.q_blocks = static_cast<int32_t>((Lq + 255) / 256);   // pairs of query tiles
+        attn_pp_kernel<<<static_cast<unsigned>(B * H * p.q_blocks), AttnPPConfig::THREADS,
+                         AttnPPConfig::SMEM_BYTES, cs>>>(tmQ, tmK, tmV, p);
+    } else {
+        attn_kernel<<<static_cast<unsigned>(B * H * p.q_blocks), AttnConfig::THREADS,
+                      AttnConfig::SMEM_BYTES, cs>>>(tmQ, tmK, tmV, p);
+    }
     return launch_status();
 }
 
