@@ -648,8 +648,8 @@ struct AttnPPConfig {
     static constexpr int SK_OFF = P_OFF + 2 * 32768;      // NSK x 128 fp32
     static constexpr int BAR_OFF = SK_OFF + NSK * 512;
     // barriers: q_full, k_full[NK], k_empty[NK], v_full[NV], v_empty[NV], sk_full[NSK],
-    // sk_empty[NSK], then per tile s_full, s_empty, p_full, pv_done, and drain
-    static constexpr int NBARS = 1 + 2 * NK + 2 * NV + 2 * NSK + 8 + 1;
+    // sk_empty[NSK], then per tile s_full, s_empty, p_full, pv_done, turn, and drain
+    static constexpr int NBARS = 1 + 2 * NK + 2 * NV + 2 * NSK + 10 + 1;
     static constexpr int SMEM_BYTES = 1024 + BAR_OFF + NBARS * 8 + 16;
     static constexpr int TMEM_COLS = 512;
     static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
@@ -679,7 +679,9 @@ __global__ void __launch_bounds__(AttnPPConfig::THREADS, 1)
     auto s_empty = [&](int t) { return bar0 + 8u * (TB + 2 + t); };
     auto p_full = [&](int t) { return bar0 + 8u * (TB + 4 + t); };
     auto pv_done = [&](int t) { return bar0 + 8u * (TB + 6 + t); };
-    const uint32_t drain_bar = bar0 + 8u * (TB + 8);
+    // turn(t): tile t may run its exponentials (the tiles alternate on the MUFU pipe)
+    auto turn = [&](int t) { return bar0 + 8u * (TB + 8 + t); };
+    const uint32_t drain_bar = bar0 + 8u * (TB + 10);
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C::BAR_OFF + C::NBARS * 8);
     volatile int *abort = reinterpret_cast<volatile int *>(tmem_holder + 1);
     float *sk_smem = reinterpret_cast<float *>(smem + C::SK_OFF);
@@ -711,6 +713,7 @@ __global__ void __launch_bounds__(AttnPPConfig::THREADS, 1)
             mbar_init(s_empty(t), 4);
             mbar_init(p_full(t), 4);
             mbar_init(pv_done(t), 1);
+            mbar_init(turn(t), 4);
         }
         mbar_init(drain_bar, 1);
         *abort = 0;
@@ -949,6 +952,14 @@ __global__ void __launch_bounds__(AttnPPConfig::THREADS, 1)
                 l_sum *= alpha;
                 m_used = m_new;
             }
+            // the tiles take turns at the exponentials: tile 0 runs block j after tile 1 ran
+            // block j - 1, tile 1 runs block j after tile 0 ran block j (the first wait of tile 0
+            // passes at once); the other tile's scaling and maximum overlap this tile's
+            got = mbar_wait_bounded(turn(tile), tile == 0 ? ph ^ 1u : ph, abort, p.timeout_ns);
+            if (!__all_sync(0xffffffffu, got)) {
+                ok = false;
+                break;
+            }
             // P = 2^(y - m), bf16, into the tile's swizzled K-major P: two 64-column atoms,
             // row r of an atom = 8 chunks of 16 bytes, chunk index XOR r mod 8
             const uint32_t prow = base + C::P_OFF + tile * 32768u + static_cast<uint32_t>(r) * 128u;
@@ -970,6 +981,9 @@ __global__ void __launch_bounds__(AttnPPConfig::THREADS, 1)
                 sts_v4(prow + static_cast<uint32_t>(ch >> 3) * 16384u + (c16 << 4), w[0], w[1], w[2],
                        w[3]);
             }
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(turn(tile ^ 1u));
             l_sum += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
             if (any_grow && j >= 1) {
 #pragma unroll 1
