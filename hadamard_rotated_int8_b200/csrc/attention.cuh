@@ -9,16 +9,16 @@
 //   2. attn_rowquant_kernel: Q rows, and K rows minus mu, rotated by the butterfly over groups
 //      of min(g, D) and quantized per row to int8 as in the linear path (codes, scale
 //      s = fp32(amax/127) * fp32(1/sqrt(G))); scales stored [B][H][L].
-//   3. attn_kernel: one CTA per (b, h, 128 queries).
-//      - warp 0 loads the Q codes once and a 3-stage ring of (K codes, V, key scales) through TMA;
-//      - warp 1 issues S_j = Q K_j^T (tcgen05 kind::i8, int32 in a double-buffered TMEM tile)
-//        and O += P_j V_j (kind::f16, bf16 P and V, fp32 O in TMEM);
-//      - warps 2..9, two threads per query row (64 key columns each), turn S_j into base-2
-//        logits acc * (s_q * scale * log2 e) * s_k (a few fp32 roundings away from the
-//        oracle's order; the softmax is approximate anyway), run an online softmax with
-//        ex2.approx (rescaling O and the row sum only when the row maximum grows by more
-//        than 2^8, so P stays below 256), write P_j as bf16 into a 128-byte-swizzled K-major
-//        tile for the MMA, and finally write O / l as bf16.
+//   3. attn_kernel: one CTA per (b, h, 256 queries) = two 128-query tiles.
+//      - warp 0 loads both Q tiles once, then rings of K codes, key scales and V through TMA;
+//      - warp 1 issues S_t(j) = Q_t K_j^T (tcgen05 kind::i8, int32 in TMEM) and
+//        O_t += P_t(j) V_j (kind::f16, bf16 P and V, fp32 O in TMEM) for both tiles;
+//      - warps 2..5 (tile 0) and 6..9 (tile 1), one thread per query row, form base-2 logits
+//        (acc * s_k) * (s_q * scale * log2 e) (a few fp32 roundings away from the oracle's
+//        order), run an online softmax with ex2.approx (rescaling O and the row sum only when
+//        the row maximum grows by more than 2^8, so P stays below 256), write P_t(j) as bf16
+//        into a 128-byte-swizzled K-major tile, and finally write O / l as bf16. The two tiles
+//        take turns at the exponentials.
 // Every wait is bounded as in the GEMM kernel.
 #pragma once
 
@@ -27,25 +27,11 @@
 #include "device.cuh"
 #include "rotquant.cuh"
 
-#ifndef SDNQ_ATTN_CTAS_PER_SM
-#define SDNQ_ATTN_CTAS_PER_SM 2
-#endif
-#ifndef SDNQ_ATTN_TPR
-#define SDNQ_ATTN_TPR 2
-#endif
-#ifndef SDNQ_ATTN_PBUF
-#define SDNQ_ATTN_PBUF 1
-#endif
-#ifndef SDNQ_ATTN_PINGPONG
-#define SDNQ_ATTN_PINGPONG 1
-#endif
-
 namespace sdnq {
 
 constexpr int kAttnD = 128;
 constexpr int kAttnBlock = 128;        // queries per CTA and keys per step
 constexpr int kAttnSumSplits = 32;     // key splits of the channel sums
-constexpr bool kAttnPingPong = SDNQ_ATTN_PINGPONG != 0;   // two query tiles per CTA
 
 // ---------------------------------------------------------------- smooth_k channel means
 
@@ -202,434 +188,13 @@ struct AttnParams {
     const float *sk;       // [B][H][Lk_pad] key scales
     uint16_t *o;           // [B][Lq][H][D] bf16
     int32_t B, Lq, Lk, H;
-    int32_t q_blocks;      // ceil(Lq / 128)
+    int32_t q_blocks;      // ceil(Lq / 256): pairs of 128-query tiles
     int32_t lq_pad, lk_pad;  // Lq, Lk rounded up to 128
     float scale;           // softmax scale applied to the logits (fp32)
     uint64_t timeout_ns;
 };
 
-struct AttnConfig {
-    static constexpr int TPR = SDNQ_ATTN_TPR;              // softmax threads per query row
-    static constexpr int THREADS = 64 + 128 * TPR;        // loader, MMA, 4 TPR softmax warps
-    static constexpr int SOFTMAX_WARPS = 4 * TPR;
-    static constexpr int CTAS_PER_SM = SDNQ_ATTN_CTAS_PER_SM;
-    // K and V rings of their own: K_j is free once S_j is done, V_j once PV_j is done
-    static constexpr int NK = CTAS_PER_SM == 2 ? 1 : 3;    // K code stages
-    static constexpr int PBUF = SDNQ_ATTN_PBUF;            // P tiles in shared memory
-    static constexpr int NV = CTAS_PER_SM == 2 ? 1 : (PBUF == 2 ? 2 : 3);   // V stages
-    static constexpr int NSK = 2;                          // key-scale stages (freed by softmax)
-    static constexpr int SBUF = CTAS_PER_SM == 2 ? 1 : 2;  // S buffers in TMEM
-    static constexpr int Q_OFF = 0;                       // int8 [128 x 128]
-    static constexpr int K_OFF = 16384;                   // NK x int8 [128 x 128]
-    static constexpr int V_OFF = K_OFF + NK * 16384;      // NV x bf16 [128 x 128]
-    static constexpr int P_OFF = V_OFF + NV * 32768;      // bf16 [128 x 128], K-major
-    static constexpr int SK_OFF = P_OFF + PBUF * 32768;   // NSK x 128 fp32
-    static constexpr int XCH_OFF = SK_OFF + NSK * 512;    // row maxima / sums of the pairs
-    static constexpr int BAR_OFF = XCH_OFF + 3 * 128 * TPR * 4;
-    // barriers: q_full, k_full[NK], k_empty[NK], v_full[NV], v_empty[NV], sk_full[NSK],
-    // sk_empty[NSK], s_full[2], s_empty[2], p_full[2], pv_done[2], drain
-    static constexpr int NBARS = 1 + 2 * NK + 2 * NV + 2 * NSK + 4 + 5;
-    static constexpr int SMEM_BYTES = 1024 + BAR_OFF + NBARS * 8 + 16;
-    // S buffers [0, 128 SBUF), O [128 SBUF, 128 SBUF + 128)
-    static constexpr int O_COL = 128 * SBUF;
-    static constexpr int TMEM_COLS = SBUF == 2 ? 512 : 256;
-    static_assert(SMEM_BYTES * CTAS_PER_SM + 1024 * CTAS_PER_SM <= 233472,
-                  "shared memory of the resident CTAs exceeds the SM's 228 KB");
-    static_assert(TMEM_COLS * CTAS_PER_SM <= 512, "TMEM columns of the resident CTAs");
-};
-
-__global__ void __launch_bounds__(AttnConfig::THREADS, AttnConfig::CTAS_PER_SM)
-    attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                const __grid_constant__ CUtensorMap tmV, const AttnParams p)
-{
-    using C = AttnConfig;
-    extern __shared__ uint8_t smem_raw[];
-    const uint32_t raw_addr = smem_u32(smem_raw);
-    const uint32_t base = (raw_addr + 1023u) & ~1023u;
-    uint8_t *smem = smem_raw + (base - raw_addr);
-    const uint32_t bar0 = base + C::BAR_OFF;
-    constexpr int NK = C::NK, NV = C::NV, NSK = C::NSK;
-    const uint32_t q_full = bar0;
-    auto k_full = [&](int s) { return bar0 + 8u * (1 + s); };
-    auto k_empty = [&](int s) { return bar0 + 8u * (1 + NK + s); };
-    auto v_full = [&](int s) { return bar0 + 8u * (1 + 2 * NK + s); };
-    auto v_empty = [&](int s) { return bar0 + 8u * (1 + 2 * NK + NV + s); };
-    auto sk_full = [&](int s) { return bar0 + 8u * (1 + 2 * NK + 2 * NV + s); };
-    auto sk_empty = [&](int s) { return bar0 + 8u * (1 + 2 * NK + 2 * NV + NSK + s); };
-    constexpr int SB0 = 1 + 2 * NK + 2 * NV + 2 * NSK;
-    auto s_full = [&](int s) { return bar0 + 8u * (SB0 + s); };
-    auto s_empty = [&](int s) { return bar0 + 8u * (SB0 + 2 + s); };
-    // per P tile b: p_full(b) when the softmax has written P_j (j % PBUF = b), pv_done(b) when
-    // PV_j has read it; one phase per use, so no wait can skip a phase
-    auto p_full = [&](int b) { return bar0 + 8u * (SB0 + 4 + b); };
-    auto pv_done = [&](int b) { return bar0 + 8u * (SB0 + 6 + b); };
-    const uint32_t drain_bar = bar0 + 8u * (SB0 + 8);
-    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C::BAR_OFF + C::NBARS * 8);
-    volatile int *abort = reinterpret_cast<volatile int *>(tmem_holder + 1);
-    float *sk_smem = reinterpret_cast<float *>(smem + C::SK_OFF);
-
-    const uint32_t warp = threadIdx.x >> 5;
-    const uint32_t lane = lane_id();
-    const int32_t qb = static_cast<int32_t>(blockIdx.x) % p.q_blocks;
-    const int32_t bh = static_cast<int32_t>(blockIdx.x) / p.q_blocks;
-    const int32_t b = bh / p.H, h = bh % p.H;
-    const int32_t q0 = qb * kAttnBlock;
-    const int32_t nkv = (p.Lk + kAttnBlock - 1) / kAttnBlock;
-
-    if (threadIdx.x == 0) {
-        mbar_init(q_full, 1);
-        for (int s = 0; s < NK; ++s) {
-            mbar_init(k_full(s), 1);
-            mbar_init(k_empty(s), 1);
-        }
-        for (int s = 0; s < NV; ++s) {
-            mbar_init(v_full(s), 1);
-            mbar_init(v_empty(s), 1);
-        }
-        for (int s = 0; s < NSK; ++s) {
-            mbar_init(sk_full(s), 1);
-            mbar_init(sk_empty(s), C::SOFTMAX_WARPS);
-        }
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(s_full(s), 1);
-            mbar_init(s_empty(s), C::SOFTMAX_WARPS);
-        }
-        mbar_init(p_full(0), C::SOFTMAX_WARPS);
-        mbar_init(p_full(1), C::SOFTMAX_WARPS);
-        mbar_init(pv_done(0), 1);
-        mbar_init(pv_done(1), 1);
-        mbar_init(drain_bar, 1);
-        *abort = 0;
-        fence_mbar_init();
-        prefetch_tensormap(&tmQ);
-        prefetch_tensormap(&tmK);
-        prefetch_tensormap(&tmV);
-    }
-    if (warp == 1) {
-        tmem_alloc(smem_u32(tmem_holder), C::TMEM_COLS);
-        tmem_relinquish();
-    }
-    tc_fence_before_sync();
-    __syncthreads();
-    tc_fence_after_sync();
-    const uint32_t tmem_base = *tmem_holder;
-
-    if (warp == 0) {
-        // ------------------------------------------------------------ loads
-        // Per key block j, in this order: K_j and its scales, then V_j. V_j waits for PV_{j-1},
-        // which the MMA warp issues after S_j, so K_j is never held behind V_{j-1}'s release.
-        if (lane == 0) {
-            mbar_arrive_expect_tx(q_full, 16384);
-            tma_load_3d(base + C::Q_OFF, &tmQ, q_full, h * kAttnD, q0, b);
-            int nk = 0, nsk = 0, nv = 0;   // copies issued per ring
-            for (int j = 0; j < nkv; ++j) {
-                const int32_t j0 = j * kAttnBlock;
-                const int ks = j % NK, ss = j % NSK, vs = j % NV;
-                if (!mbar_wait_bounded(k_empty(ks), (static_cast<uint32_t>(j / NK) & 1u) ^ 1u, abort,
-                                       p.timeout_ns))
-                    break;
-                mbar_arrive_expect_tx(k_full(ks), 16384);
-                tma_load_3d(base + C::K_OFF + ks * 16384, &tmK, k_full(ks), h * kAttnD, j0, b);
-                ++nk;
-                if (!mbar_wait_bounded(sk_empty(ss), (static_cast<uint32_t>(j / NSK) & 1u) ^ 1u,
-                                       abort, p.timeout_ns))
-                    break;
-                mbar_arrive_expect_tx(sk_full(ss), 512);
-                // the block's 128 key scales (the padded rows keep this in bounds and aligned)
-                bulk_load_1d(smem_u32(sk_smem + ss * kAttnBlock),
-                             p.sk + static_cast<int64_t>(bh) * p.lk_pad + j0, 512, sk_full(ss));
-                ++nsk;
-                if (!mbar_wait_bounded(v_empty(vs), (static_cast<uint32_t>(j / NV) & 1u) ^ 1u, abort,
-                                       p.timeout_ns))
-                    break;
-                mbar_arrive_expect_tx(v_full(vs), 32768);
-                tma_load_3d(base + C::V_OFF + vs * 32768, &tmV, v_full(vs), h * kAttnD, j0, b);
-                tma_load_3d(base + C::V_OFF + vs * 32768 + 16384, &tmV, v_full(vs), h * kAttnD + 64,
-                            j0, b);
-                ++nv;
-            }
-            // every copy this warp started has landed before the CTA can exit (the Q tile and
-            // the last uses of each ring; already complete on the normal path)
-            volatile int no_abort = 0;
-            mbar_wait_bounded(q_full, 0u, &no_abort, p.timeout_ns);
-            for (int j = nk - NK < 0 ? 0 : nk - NK; j < nk; ++j)
-                mbar_wait_bounded(k_full(j % NK), static_cast<uint32_t>(j / NK) & 1u, &no_abort,
-                                  p.timeout_ns);
-            for (int j = nsk - NSK < 0 ? 0 : nsk - NSK; j < nsk; ++j)
-                mbar_wait_bounded(sk_full(j % NSK), static_cast<uint32_t>(j / NSK) & 1u, &no_abort,
-                                  p.timeout_ns);
-            for (int j = nv - NV < 0 ? 0 : nv - NV; j < nv; ++j)
-                mbar_wait_bounded(v_full(j % NV), static_cast<uint32_t>(j / NV) & 1u, &no_abort,
-                                  p.timeout_ns);
-        }
-    } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issue
-        if (lane == 0) {
-            constexpr uint32_t IDESC_S = idesc_s8_s32(128, 128);
-            constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, 128, true);
-            const uint32_t t_o = tmem_base + C::O_COL;
-            bool ok = mbar_wait_bounded(q_full, 0u, abort, p.timeout_ns);
-            auto issue_pv = [&](int j) {
-                // O (+)= P_j V_j: A = P, K-major bf16 in two 64-column atoms; B = V, N-major
-                if (!mbar_wait_bounded(v_full(j % NV), static_cast<uint32_t>(j / NV) & 1u, abort,
-                                       p.timeout_ns) ||
-                    !mbar_wait_bounded(p_full(j % C::PBUF), static_cast<uint32_t>(j / C::PBUF) & 1u,
-                                       abort, p.timeout_ns))
-                    return false;
-                tc_fence_after_sync();
-                const uint32_t sp = base + C::P_OFF + (j % C::PBUF) * 32768;
-                const uint32_t sv = base + C::V_OFF + (j % NV) * 32768;
-#pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    mma_f16(t_o, kmajor_desc(sp + (k >> 2) * 16384 + (k & 3) * 32),
-                            mnmajor_desc(sv + 2048 * k, 16384), IDESC_PV,
-                            (j | k) != 0 ? 1u : 0u);
-                tc_commit(pv_done(j % C::PBUF));
-                tc_commit(v_empty(j % NV));
-                return true;
-            };
-            for (int j = 0; ok && j < nkv; ++j) {
-                const int ks = j % NK;       // K stage
-                const int sb = j % C::SBUF;  // S buffer
-                if (!mbar_wait_bounded(k_full(ks), static_cast<uint32_t>(j / NK) & 1u, abort,
-                                       p.timeout_ns) ||
-                    !mbar_wait_bounded(s_empty(sb), (static_cast<uint32_t>(j / C::SBUF) & 1u) ^ 1u,
-                                       abort, p.timeout_ns)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after_sync();
-                const uint32_t sq_addr = base + C::Q_OFF;
-                const uint32_t sk_addr = base + C::K_OFF + ks * 16384;
-#pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    mma_s8(tmem_base + sb * 128, kmajor_desc(sq_addr + 32 * k),
-                           kmajor_desc(sk_addr + 32 * k), IDESC_S, k != 0 ? 1u : 0u);
-                tc_commit(s_full(sb));
-                tc_commit(k_empty(ks));
-                if (j >= 1 && !issue_pv(j - 1)) {
-                    ok = false;
-                    break;
-                }
-            }
-            if (ok)
-                issue_pv(nkv - 1);
-            tc_commit(drain_bar);
-            volatile int no_abort = 0;
-            mbar_wait_bounded(drain_bar, 0u, &no_abort, p.timeout_ns);
-        }
-    } else {
-        // ------------------------------------------------------------ softmax (warps 2..)
-        // TPR threads per query row: warps w, w + 4, ... share the TMEM lane quarter w % 4 and
-        // take key columns (and O columns) [COLS part, COLS part + COLS). They combine their
-        // row maxima and sums through shared memory and a named barrier of the row's warps
-        // (ids 1..4, 32 TPR threads).
-        constexpr int TPR = C::TPR, COLS = 128 / TPR, NCH = COLS / 32;
-        const uint32_t quad = warp & 3u;
-        const uint32_t part = (warp - 2u) >> 2;
-        const uint32_t row_bar = 1u + quad;
-        const int32_t r = static_cast<int32_t>(quad * 32u + lane);   // query row in the block
-        const bool row_ok = q0 + r < p.Lq;
-        const float sqr = row_ok ? p.sq[static_cast<int64_t>(bh) * p.lq_pad + q0 + r] : 0.0f;
-        // logit * log2(e) = acc * (s_q * scale * log2 e) * s_k: the row factor folded once
-        const float row_f = sqr * p.scale * 1.4426950408889634f;
-        const uint32_t t_lane = tmem_base + ((quad * 32u) << 16);
-        const uint32_t col0 = part * COLS;    // this thread's first key / O column
-        float *xch = reinterpret_cast<float *>(smem + C::XCH_OFF);   // [3][128][TPR]
-        float m_used = -INFINITY;  // base-2 maximum the exponentials are taken against
-        float l_sum = 0.0f;        // this thread's share of the row sum
-        bool ok = true;
-        for (int j = 0; ok && j < nkv; ++j) {
-            const int s = j % C::SBUF;           // S buffer
-            const int ss = j % NSK;              // key-scale stage
-            bool got = mbar_wait_bounded(s_full(s), static_cast<uint32_t>(j / C::SBUF) & 1u, abort,
-                                         p.timeout_ns) &&
-                       mbar_wait_bounded(sk_full(ss), static_cast<uint32_t>(j / NSK) & 1u, abort,
-                                         p.timeout_ns);
-            if (!__all_sync(0xffffffffu, got)) {
-                ok = false;
-                break;
-            }
-            tc_fence_after_sync();
-            // fp32(acc) without the conversion pipe: |acc| <= 127 * 127 * 128 < 2^22, so the
-            // bits of acc + 0x4B400000 are the float 1.5 * 2^23 + acc, and subtracting
-            // 1.5 * 2^23 (below, exact) leaves acc
-            float y[COLS];
-            {
-                uint32_t a[NCH][32];
-#pragma unroll
-                for (int c = 0; c < NCH; ++c)
-                    tmem_ld_32x32b_x32(t_lane + s * 128 + col0 + c * 32, a[c]);
-                tmem_ld_wait();
-#pragma unroll
-                for (int c = 0; c < NCH; ++c)
-#pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        y[c * 32 + i] = __uint_as_float(a[c][i] + 0x4B400000u);
-            }
-            tc_fence_before_sync();
-            __syncwarp();
-            if (lane == 0)
-                mbar_arrive(s_empty(s));
-            const int32_t j0 = j * kAttnBlock + static_cast<int32_t>(col0);
-            const float4 *skb = reinterpret_cast<const float4 *>(sk_smem + ss * kAttnBlock + col0);
-#pragma unroll
-            for (int c4 = 0; c4 < COLS / 4; ++c4) {
-                const float4 k4 = skb[c4];   // same address across the warp: a broadcast
-                float r0, r1, r2, r3, f0, f1, f2, f3;
-                mul2(r0, r1, row_f, row_f, k4.x, k4.y);
-                mul2(r2, r3, row_f, row_f, k4.z, k4.w);
-                sub2(f0, f1, y[4 * c4], y[4 * c4 + 1], 12582912.0f, 12582912.0f);
-                sub2(f2, f3, y[4 * c4 + 2], y[4 * c4 + 3], 12582912.0f, 12582912.0f);
-                mul2(y[4 * c4], y[4 * c4 + 1], f0, f1, r0, r1);
-                mul2(y[4 * c4 + 2], y[4 * c4 + 3], f2, f3, r2, r3);
-            }
-            __syncwarp();
-            if (lane == 0)
-                mbar_arrive(sk_empty(ss));   // the stage's key scales are read
-            if (j0 + COLS > p.Lk) {          // the ragged last block (warp-uniform)
-#pragma unroll
-                for (int c = 0; c < COLS; ++c)
-                    if (j0 + c >= p.Lk)
-                        y[c] = -INFINITY;
-            }
-            // 4 independent chains, chain i over the columns i + 4k (k = 0 .. COLS/4 - 1)
-            constexpr int KN = COLS / 4;
-            float mx[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                mx[i] = y[i];
-#pragma unroll
-                for (int k = 1; k + 1 < KN; k += 2)
-                    mx[i] = max3f(mx[i], y[i + 4 * k], y[i + 4 * k + 4]);
-                if ((KN - 1) % 2 == 1)
-                    mx[i] = fmaxf(mx[i], y[i + 4 * (KN - 1)]);
-            }
-            float mb = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
-            xch[((j & 1) * 128 + r) * TPR + part] = mb;
-            asm volatile("bar.sync %0, %1;" ::"r"(row_bar), "r"(32 * TPR) : "memory");
-#pragma unroll
-            for (int t = 0; t < TPR; ++t)
-                mb = fmaxf(mb, xch[((j & 1) * 128 + r) * TPR + t]);
-            // P tile j % PBUF is free once PV_{j - PBUF}, its last reader, is done
-            if (j >= C::PBUF) {
-                got = mbar_wait_bounded(pv_done(j % C::PBUF),
-                                        static_cast<uint32_t>((j - C::PBUF) / C::PBUF) & 1u, abort,
-                                        p.timeout_ns);
-                if (!__all_sync(0xffffffffu, got)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after_sync();
-            }
-            // rescale O and l only when the maximum grows by more than 8 (p stays <= 256);
-            // all threads of a row see the same maximum and decide alike
-            const bool grow = mb > m_used + 8.0f;
-            if (__any_sync(0xffffffffu, grow)) {
-                const float m_new = grow ? mb : m_used;
-                const float alpha = grow && m_used != -INFINITY ? ex2_approx(m_used - m_new)
-                                                                : (grow ? 0.0f : 1.0f);
-                if (j >= 1 && C::PBUF > 1) {
-                    // O is stable once PV_{j-1} is done (PV_j waits for this block's P)
-                    got = mbar_wait_bounded(pv_done((j - 1) % C::PBUF),
-                                            static_cast<uint32_t>((j - 1) / C::PBUF) & 1u, abort,
-                                            p.timeout_ns);
-                    if (!__all_sync(0xffffffffu, got)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after_sync();
-                }
-                if (j >= 1) {
-#pragma unroll 1
-                    for (int c = 0; c < NCH; ++c) {
-                        uint32_t a[32];
-                        tmem_ld_32x32b_x32(t_lane + C::O_COL + col0 + c * 32, a);
-                        tmem_ld_wait();
-#pragma unroll
-                        for (int i = 0; i < 32; ++i)
-                            a[i] = __float_as_uint(__uint_as_float(a[i]) * alpha);
-                        tmem_st_32x32b_x32(t_lane + C::O_COL + col0 + c * 32, a);
-                    }
-                    tmem_st_wait();
-                }
-                l_sum *= alpha;
-                m_used = m_new;
-            }
-            // P = 2^(y - m), bf16, into the swizzled K-major tile: 64-column atoms, row r of
-            // an atom = 8 chunks of 16 bytes, chunk index XOR r mod 8
-            const uint32_t prow = base + C::P_OFF + (j % C::PBUF) * 32768u + (col0 >> 6) * 16384u +
-                                  static_cast<uint32_t>(r) * 128u;
-            const uint32_t cfirst = (col0 & 63u) >> 3;
-            float ls[8] = {0, 0, 0, 0, 0, 0, 0, 0};  // 8 independent partial sums
-#pragma unroll
-            for (int ch = 0; ch < COLS / 8; ++ch) {
-                uint32_t w[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    float d0, d1;
-                    sub2(d0, d1, y[ch * 8 + 2 * e], y[ch * 8 + 2 * e + 1], m_used, m_used);
-                    const float p0 = ex2_approx(d0);
-                    const float p1 = ex2_approx(d1);
-                    add2(ls[2 * e], ls[2 * e + 1], ls[2 * e], ls[2 * e + 1], p0, p1);
-                    const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
-                    w[e] = *reinterpret_cast<const uint32_t *>(&h2);
-                }
-                const uint32_t c16 = (cfirst + static_cast<uint32_t>(ch)) ^ (static_cast<uint32_t>(r) & 7u);
-                sts_v4(prow + (c16 << 4), w[0], w[1], w[2], w[3]);
-            }
-            l_sum += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
-            fence_proxy_async_smem();
-            tc_fence_before_sync();
-            __syncwarp();
-            if (lane == 0)
-                mbar_arrive(p_full(j % C::PBUF));
-        }
-        // O / l as bf16: the row's TPR partial sums combined, each thread its COLS O columns
-        bool fin = ok && mbar_wait_bounded(pv_done((nkv - 1) % C::PBUF),
-                                           static_cast<uint32_t>((nkv - 1) / C::PBUF) & 1u, abort,
-                                           p.timeout_ns);
-        xch[(2 * 128 + r) * TPR + part] = l_sum;
-        asm volatile("bar.sync %0, %1;" ::"r"(row_bar), "r"(32 * TPR) : "memory");
-        float l_tot = 0.0f;
-#pragma unroll
-        for (int t = 0; t < TPR; ++t)
-            l_tot += xch[(2 * 128 + r) * TPR + t];
-        if (__all_sync(0xffffffffu, fin)) {
-            tc_fence_after_sync();
-            const float inv = 1.0f / l_tot;
-            uint16_t *orow = p.o + ((static_cast<int64_t>(b) * p.Lq + q0 + r) * p.H + h) * kAttnD +
-                             col0;
-#pragma unroll 1
-            for (int c = 0; c < NCH; ++c) {
-                uint32_t a[32];
-                tmem_ld_32x32b_x32(t_lane + C::O_COL + col0 + c * 32, a);
-                tmem_ld_wait();
-                uint32_t w[16];
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(a[2 * i]) * inv,
-                                                                    __uint_as_float(a[2 * i + 1]) * inv);
-                    w[i] = *reinterpret_cast<const uint32_t *>(&h2);
-                }
-                if (row_ok) {
-#pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        st_v4(orow + c * 32 + q * 8, w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
-                }
-            }
-        }
-    }
-
-    tc_fence_before_sync();
-    __syncthreads();
-    if (warp == 1) {
-        tc_fence_after_sync();
-        tmem_dealloc(tmem_base, C::TMEM_COLS);
-    }
-}
-
-// ---------------------------------------------------------------- two-tile (ping-pong) kernel
+// ---------------------------------------------------------------- the attention kernel
 //
 // One CTA per (b, h, 256 queries) = two 128-query tiles sharing every K / V block. Warps 2..5
 // run the softmax of tile 0 and warps 6..9 that of tile 1, one thread per query row (all 128
@@ -638,7 +203,7 @@ __global__ void __launch_bounds__(AttnConfig::THREADS, AttnConfig::CTAS_PER_SM)
 // softmax covers the other's waits on S and PV. TMEM: S_0, S_1, O_0, O_1 (128 columns each).
 // The MMA warp issues S_t(j+1) as soon as tile t has read S_t(j), and PV_t(j) once tile t
 // has written P_t(j); a tile overwrites its P tile once PV_t(j-1) is done.
-struct AttnPPConfig {
+struct AttnConfig {
     static constexpr int THREADS = 320;                   // loader, MMA, 2 x 4 softmax warps
     static constexpr int NK = 3, NV = 2, NSK = 2;         // K, V, key-scale stages
     static constexpr int Q_OFF = 0;                       // 2 x int8 [128 x 128]
@@ -655,11 +220,11 @@ struct AttnPPConfig {
     static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 };
 
-__global__ void __launch_bounds__(AttnPPConfig::THREADS, 1)
-    attn_pp_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+__global__ void __launch_bounds__(AttnConfig::THREADS, 1)
+    attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const AttnParams p)
 {
-    using C = AttnPPConfig;
+    using C = AttnConfig;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_addr = smem_u32(smem_raw);
     const uint32_t base = (raw_addr + 1023u) & ~1023u;
@@ -861,8 +426,11 @@ __global__ void __launch_bounds__(AttnPPConfig::THREADS, 1)
         const int32_t qrow = q0 + static_cast<int32_t>(tile) * kAttnBlock + r;
         const bool row_ok = qrow < p.Lq;
         const float sqr = row_ok ? p.sq[static_cast<int64_t>(bh) * p.lq_pad + qrow] : 0.0f;
-        // logit * log2(e) = acc * (s_q * scale * log2 e) * s_k: the row factor folded once
-        const float row_f = sqr * p.scale * 1.4426950408889634f;
+        // logit * log2(e) = (acc * s_k) * row_f with row_f = s_q * scale * log2 e >= 0, applied
+        // in the exponent's fused multiply-add; rounding is monotone, so the row maximum of
+        // the logits is row_f times that of acc * s_k. The floor keeps a zero row (or scale)
+        // finite against the padded keys' -inf (its logits stay 0 to within 2^-100).
+        const float row_f = fmaxf(sqr * p.scale * 1.4426950408889634f, 0x1p-126f);
         const uint32_t t_lane = tmem_base + ((quad * 32u) << 16);
         const uint32_t s_col = tile * 128u, o_col = 256u + tile * 128u;
         float m_used = -INFINITY;  // base-2 maximum the exponentials are taken against
@@ -903,13 +471,11 @@ __global__ void __launch_bounds__(AttnPPConfig::THREADS, 1)
 #pragma unroll
             for (int c4 = 0; c4 < 32; ++c4) {
                 const float4 k4 = skb[c4];   // same address across the warp: a broadcast
-                float r0, r1, r2, r3, f0, f1, f2, f3;
-                mul2(r0, r1, row_f, row_f, k4.x, k4.y);
-                mul2(r2, r3, row_f, row_f, k4.z, k4.w);
+                float f0, f1, f2, f3;
                 sub2(f0, f1, y[4 * c4], y[4 * c4 + 1], 12582912.0f, 12582912.0f);
                 sub2(f2, f3, y[4 * c4 + 2], y[4 * c4 + 3], 12582912.0f, 12582912.0f);
-                mul2(y[4 * c4], y[4 * c4 + 1], f0, f1, r0, r1);
-                mul2(y[4 * c4 + 2], y[4 * c4 + 3], f2, f3, r2, r3);
+                mul2(y[4 * c4], y[4 * c4 + 1], f0, f1, k4.x, k4.y);          // acc * s_k
+                mul2(y[4 * c4 + 2], y[4 * c4 + 3], f2, f3, k4.z, k4.w);
             }
             __syncwarp();
             if (lane == 0)
@@ -931,7 +497,7 @@ __global__ void __launch_bounds__(AttnPPConfig::THREADS, 1)
                     mx[i] = max3f(mx[i], y[i + 4 * k], y[i + 4 * k + 4]);
                 mx[i] = fmaxf(mx[i], y[i + 124]);
             }
-            const float mb = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+            const float mb = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * row_f;
             // P_t(j-1) has left the P tile, and O_t is stable, once PV_t(j-1) is done
             if (j >= 1) {
                 got = mbar_wait_bounded(pv_done(tile), ph ^ 1u, abort, p.timeout_ns);
@@ -963,14 +529,15 @@ __global__ void __launch_bounds__(AttnPPConfig::THREADS, 1)
             // P = 2^(y - m), bf16, into the tile's swizzled K-major P: two 64-column atoms,
             // row r of an atom = 8 chunks of 16 bytes, chunk index XOR r mod 8
             const uint32_t prow = base + C::P_OFF + tile * 32768u + static_cast<uint32_t>(r) * 128u;
+            const float neg_m = -m_used;
             float ls[8] = {0, 0, 0, 0, 0, 0, 0, 0};  // 8 independent partial sums
 #pragma unroll
             for (int ch = 0; ch < 16; ++ch) {
                 uint32_t w[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    float d0, d1;
-                    sub2(d0, d1, y[ch * 8 + 2 * e], y[ch * 8 + 2 * e + 1], m_used, m_used);
+                    float d0, d1;   // (acc * s_k) * row_f - m in one rounding
+                    fma2(d0, d1, y[ch * 8 + 2 * e], y[ch * 8 + 2 * e + 1], row_f, row_f, neg_m, neg_m);
                     const float p0 = ex2_approx(d0);
                     const float p1 = ex2_approx(d1);
                     add2(ls[2 * e], ls[2 * e + 1], ls[2 * e], ls[2 * e + 1], p0, p1);

@@ -1,6 +1,7 @@
 // libsdnq.so: the C ABI declared in include/sdnq.h. Host side: argument validation, TMA
 // tensor-map encoding, launch configuration and the device error word. All arithmetic of the
 // layer runs in the kernels included below.
+#include <cfloat>
 #include <cmath>
 #include <cstdint>
 #include <cstdlib>
@@ -769,10 +770,7 @@ sdnq_status launch_attention_core(const uint16_t *v, int64_t B, int64_t Lq, int6
         return SDNQ_ERR_CUDA;
     static std::once_flag once;
     static bool smem_ok = false;
-    std::call_once(once, [] {
-        smem_ok = kAttnPingPong ? set_smem(attn_pp_kernel, AttnPPConfig::SMEM_BYTES)
-                                : set_smem(attn_kernel, AttnConfig::SMEM_BYTES);
-    });
+    std::call_once(once, [] { smem_ok = set_smem(attn_kernel, AttnConfig::SMEM_BYTES); });
     if (!smem_ok)
         return SDNQ_ERR_CUDA;
     AttnParams p = {};
@@ -783,20 +781,14 @@ sdnq_status launch_attention_core(const uint16_t *v, int64_t B, int64_t Lq, int6
     p.Lq = static_cast<int32_t>(Lq);
     p.Lk = static_cast<int32_t>(Lk);
     p.H = static_cast<int32_t>(H);
-    p.q_blocks = static_cast<int32_t>((Lq + 127) / 128);
-    p.lq_pad = p.q_blocks * 128;   // the workspace's query-scale row stride
+    p.q_blocks = static_cast<int32_t>((Lq + 255) / 256);   // pairs of query tiles
+    p.lq_pad = static_cast<int32_t>((Lq + 127) / 128 * 128);   // query-scale row stride
     p.lk_pad = static_cast<int32_t>((Lk + 127) / 128 * 128);
     p.scale = scale;
     p.timeout_ns = kDefaultTimeoutNs;
     cudaGetLastError();
-    if (kAttnPingPong) {
-        p.q_blocks = static_cast<int32_t>((Lq + 255) / 256);   // pairs of query tiles
-        attn_pp_kernel<<<static_cast<unsigned>(B * H * p.q_blocks), AttnPPConfig::THREADS,
-                         AttnPPConfig::SMEM_BYTES, cs>>>(tmQ, tmK, tmV, p);
-    } else {
-        attn_kernel<<<static_cast<unsigned>(B * H * p.q_blocks), AttnConfig::THREADS,
-                      AttnConfig::SMEM_BYTES, cs>>>(tmQ, tmK, tmV, p);
-    }
+    attn_kernel<<<static_cast<unsigned>(B * H * p.q_blocks), AttnConfig::THREADS,
+                  AttnConfig::SMEM_BYTES, cs>>>(tmQ, tmK, tmV, p);
     return launch_status();
 }
 
@@ -811,6 +803,8 @@ sdnq_status run_attention(const uint16_t *q, const uint16_t *k, const uint16_t *
     sdnq_status st = validate_attention(q, k, v, o, B, Lq, Lk, H, D, group, ws, ws_bytes, off);
     if (st != SDNQ_OK)
         return st;
+    if ((which & 2) && !(scale >= 0.0f && scale <= FLT_MAX))   // the softmax scale: finite, >= 0
+        return SDNQ_ERR_UNSUPPORTED;
     DeviceInfo dev;
     if ((st = current_device(&dev)) != SDNQ_OK)
         return st;

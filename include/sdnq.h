@@ -274,7 +274,8 @@ sdnq_status sdnq_fp8_linear(const uint8_t *qx, const float *sx, const uint8_t *q
  *   quantized per row exactly as sdnq_rotquant_act does; logits are
  *   fp32(fp32(fp32(acc) * fp32(s_q * s_k)) * scale), acc the int32 dot product of the codes;
  *   o = softmax(logits) v, with the probabilities rounded to bf16 for the PV product (fp32
- *   accumulation) and o rounded to bf16. A usual scale is fp32(1/sqrt(D)).
+ *   accumulation) and o rounded to bf16. scale: finite and >= 0 (else SDNQ_ERR_UNSUPPORTED);
+ *   a usual scale is fp32(1/sqrt(D)).
  *   group: power of two, SDNQ_MIN_GROUP..SDNQ_MAX_GROUP (groups above D act as D).
  *   ws: caller workspace of sdnq_attention_workspace(...) bytes, 256-byte aligned. Afterwards
  *   it holds, at the offsets that function reports: [0] Q codes int8 [B, Lq, H, D], [1] K codes,

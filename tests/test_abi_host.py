@@ -174,6 +174,36 @@ def test_gelu_and_selftest_validation(lib):
     assert lib.sdnq_selftest_wait_timeout(10, S) == _native.SDNQ_ERR_SHAPE
 
 
+W256 = 0x100000    # 256-byte aligned fake workspace address
+
+
+def attn(lib, q=A16, k=A16, v=A16, B=1, Lq=64, Lk=96, H=2, D=128, g=256, scale=0.088,
+         smooth=1, ws=W256, ws_bytes=None, o=A16):
+    if ws_bytes is None:
+        ws_bytes = lib.sdnq_attention_workspace(B, Lq, Lk, H, 128, None)
+    return lib.sdnq_attention_int8qk(q, k, v, B, Lq, Lk, H, D, g, scale, smooth, ws, ws_bytes,
+                                     o, S)
+
+
+def test_attention_validation(lib):
+    assert attn(lib, q=0) == _native.SDNQ_ERR_NULL
+    assert attn(lib, ws=0) == _native.SDNQ_ERR_NULL
+    assert attn(lib, D=64) == _native.SDNQ_ERR_UNSUPPORTED
+    assert attn(lib, g=96) == _native.SDNQ_ERR_UNSUPPORTED
+    assert attn(lib, Lk=0) == _native.SDNQ_ERR_SHAPE
+    assert attn(lib, ws_bytes=1024) == _native.SDNQ_ERR_SHAPE
+    assert attn(lib, ws=W256 + 16) == _native.SDNQ_ERR_ALIGN
+    assert attn(lib, v=MIS) == _native.SDNQ_ERR_ALIGN
+    # the softmax scale must be finite and >= 0 (the kernel takes the row maximum of
+    # acc * s_k and scales it afterwards, which needs a nonnegative factor)
+    for bad in (-0.5, float("nan"), float("inf")):
+        assert attn(lib, scale=bad) == _native.SDNQ_ERR_UNSUPPORTED
+    ws_bytes = lib.sdnq_attention_workspace(1, 64, 96, 2, 128, None)
+    assert lib.sdnq_attention_core(A16, 1, 64, 96, 2, 128, -1.0, W256, ws_bytes, A16, S) == \
+        _native.SDNQ_ERR_UNSUPPORTED
+    assert lib.sdnq_attention_workspace(1, 0, 96, 2, 128, None) < 0
+
+
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU path only")
 def test_valid_arguments_without_a_b200_are_refused(lib):
     # no silent CPU path: a well-formed call on a machine without an sm_100 GPU is refused
@@ -184,6 +214,8 @@ def test_valid_arguments_without_a_b200_are_refused(lib):
     assert lib.sdnq_gelu_bf16(A16, 4, 8, 8, A16, 8, S) == _native.SDNQ_ERR_UNSUPPORTED
     assert grad(lib) == _native.SDNQ_ERR_UNSUPPORTED
     assert fused(lib) == _native.SDNQ_ERR_UNSUPPORTED
+    assert attn(lib) == _native.SDNQ_ERR_UNSUPPORTED
+    assert attn(lib, scale=0.0) == _native.SDNQ_ERR_UNSUPPORTED
 
 
 def test_binding_refuses_cpu_tensors(lib):

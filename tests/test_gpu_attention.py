@@ -2,8 +2,8 @@
 
 Bit-exact: the smooth_k key means, the int8 codes and fp32 scales of Q and K (same fp32
 arithmetic on both sides). Outputs: the oracle takes the softmax and PV in fp64 from its fp32
-logits; the GPU forms base-2 logits acc * (s_q * scale * log2 e) * s_k (within a few fp32 ulps
-of the oracle's, which moves a probability by about |logit| 2^-22), takes ex2.approx
+logits; the GPU forms base-2 logits (acc * s_k) * (s_q * scale * log2 e) (within a few fp32
+ulps of the oracle's, which moves a probability by about |logit| 2^-22), takes ex2.approx
 (2^-22), rounds P to bf16 for the PV product and accumulates in fp32. So per element
 |o - o_ref| <= 2^-8 |o_ref| + (2^-8 + 2 Lk 2^-24 + 2^-16) S, with
 S = sum_j p_ij |v_j| / sum_j p_ij (one bf16 rounding of P and of o, the fp32 sums over Lk
@@ -107,3 +107,26 @@ def test_split_calls_equal_the_composed_call():
     o = sd.sdnq_attention_int8qk(qg, kg, vg, 128)
     torch.cuda.synchronize()
     assert_equal(bits_of(o_split), bits_of(o), "split against composed")
+
+
+def wide_qkv(seed, sign):
+    """Keys whose norms alternate 1x / 8x inside every block, queries (anti-)aligned with a
+    shared key direction: logits of several hundred in base 2 and a key-scale range of about
+    8x per block."""
+    gen = torch.Generator().manual_seed(seed)
+    B, Lq, Lk, H = 1, 96, 520, 2
+    amp = torch.where(torch.arange(Lk) % 2 == 0, 1.0, 8.0).reshape(1, Lk, 1, 1)
+    base = torch.randn(1, 1, H, 128, generator=gen)
+    k = (0.5 * base + torch.randn(B, Lk, H, 128, generator=gen)) * amp
+    q = sign * 6.0 * base + torch.randn(B, Lq, H, 128, generator=gen)
+    v = torch.randn(B, Lk, H, 128, generator=gen)
+    return q.to(torch.bfloat16), k.to(torch.bfloat16), v.to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("sign,smooth", [(1.0, True), (1.0, False), (-1.0, False)])
+def test_attention_wide_logits(sign, smooth):
+    """Logits of several hundred (base 2), positive and negative row maxima, a ragged last key
+    block, workspace left uninitialised: outputs within the same bound."""
+    q, k, v = wide_qkv(31 + int(sign), sign)
+    check(q, k, v, 256, smooth)
+
