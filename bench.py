@@ -55,6 +55,7 @@ def measured_peaks():
 KERNEL_SOURCES = {
     "gemm_s8": ("device.cuh", "gemm.cuh"),
     "rotquant": ("device.cuh", "rotquant.cuh"),
+    "attn_kernel": ("device.cuh", "rotquant.cuh", "attention.cuh"),
 }
 
 
@@ -599,7 +600,8 @@ def main():
         "roofline": {
             "kernel": gemm_kernel, "bound": "tensor", "achieved": gemm_tops,
             "peak": int8_peak, "unit": "TFLOP/s", "frac": gemm_tops / int8_peak,
-            "traffic": profiled_traffic("gemm_s8", args.workload),
+            "traffic": profiled_traffic("attn_kernel" if case.extra.get("attn") else "gemm_s8",
+                                        args.workload),
             "ops_per_launch": ops / len(step.gemm_stages), "ms_per_launch": gemm_launch_ms,
             "peak_source": f"{peak_src} bf16 burst x {NOMINAL_INT8_OVER_BF16} (int8/bf16 nominal)",
             "frac_of_int8_spec": gemm_tops / INT8_SPEC_TOPS,

@@ -45,14 +45,24 @@ __global__ void __launch_bounds__(256) attn_ksum_kernel(const uint16_t *k, int32
     const int32_t lane_row = threadIdx.x >> 4;   // 16 keys per pass
     const int32_t per = (Lk + kAttnSumSplits - 1) / kAttnSumSplits;
     const int32_t j0 = split * per, j1 = j0 + per < Lk ? j0 + per : Lk;
+    // three keys in flight per thread (the fp64 sums of bf16 values are exact, so the order
+    // of the additions does not matter)
     double acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    for (int32_t j = j0 + lane_row; j < j1; j += 16) {
-        const uint4 r = ld_nc_v4(k + ((static_cast<int64_t>(b) * Lk + j) * H + h) * kAttnD + d8);
-        const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+    for (int32_t j = j0 + lane_row; j < j1; j += 48) {
+        uint4 r[3];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            acc[2 * i] += static_cast<double>(__uint_as_float(w[i] << 16));
-            acc[2 * i + 1] += static_cast<double>(__uint_as_float(w[i] & 0xffff0000u));
+        for (int u = 0; u < 3; ++u)
+            r[u] = j + 16 * u < j1
+                       ? ld_nc_v4(k + ((static_cast<int64_t>(b) * Lk + j + 16 * u) * H + h) * kAttnD + d8)
+                       : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+        for (int u = 0; u < 3; ++u) {
+            const uint32_t w[4] = {r[u].x, r[u].y, r[u].z, r[u].w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                acc[2 * i] += static_cast<double>(__uint_as_float(w[i] << 16));
+                acc[2 * i + 1] += static_cast<double>(__uint_as_float(w[i] & 0xffff0000u));
+            }
         }
     }
     __shared__ double red[16][kAttnD];
@@ -73,9 +83,14 @@ __global__ void __launch_bounds__(256) attn_ksum_kernel(const uint16_t *k, int32
 __global__ void attn_kmean_kernel(const double *partial, int32_t Lk, float *mu)
 {
     const int32_t bh = blockIdx.x, d = threadIdx.x;
-    double s = 0.0;
+    double part[kAttnSumSplits];   // all loads in flight, then the sum
+#pragma unroll
     for (int i = 0; i < kAttnSumSplits; ++i)
-        s += partial[(static_cast<int64_t>(bh) * kAttnSumSplits + i) * kAttnD + d];
+        part[i] = partial[(static_cast<int64_t>(bh) * kAttnSumSplits + i) * kAttnD + d];
+    double s = 0.0;
+#pragma unroll
+    for (int i = 0; i < kAttnSumSplits; ++i)
+        s += part[i];
     mu[static_cast<int64_t>(bh) * kAttnD + d] = static_cast<float>(s / static_cast<double>(Lk));
 }
 
@@ -86,7 +101,7 @@ struct AttnQuantParams {
     const float *mu;       // [B][H][D] or nullptr (queries)
     int8_t *q;             // [B][L][H][D]
     float *s;              // [B][H][ls]
-    int64_t rows;          // B * L * H
+    int64_t rows;          // B * L * H (below 2^31)
     int32_t L, H;
     int32_t ls;            // scale row stride: L rounded up to a multiple of 128
     float c_g;
@@ -96,7 +111,7 @@ struct AttnQuantParams {
 // groups of G <= 128 never crosses a row. Lane (hi2, lo3) holds rows 2 hi2 (t = 0, 1) and
 // 2 hi2 + 1 (t = 2, 3) of the chunk; a row's maximum combines its 8 lanes by shuffles.
 template <int G>
-__global__ void __launch_bounds__(256) attn_rowquant_kernel(const AttnQuantParams p)
+__global__ void __launch_bounds__(256, 4) attn_rowquant_kernel(const AttnQuantParams p)
 {
     const uint32_t lane = lane_id();
     const int64_t nchunks = (p.rows + 7) / 8;
@@ -106,6 +121,21 @@ __global__ void __launch_bounds__(256) attn_rowquant_kernel(const AttnQuantParam
         const int64_t row0 = c * 8 + 2 * static_cast<int64_t>(lane >> 3);
         const int64_t base = c * 1024 + static_cast<int64_t>(lane >> 3) * 256 +
                              static_cast<int64_t>(lane & 7u) * 8;
+        // (b, l, h) of the lane's two rows, in 32-bit arithmetic (rows < 2^31), once
+        const uint32_t H = static_cast<uint32_t>(p.H), L = static_cast<uint32_t>(p.L);
+        uint32_t hr[2], lr[2], br[2];
+        {
+            const uint32_t r0 = static_cast<uint32_t>(row0), t0 = r0 / H;
+            hr[0] = r0 - t0 * H;
+            br[0] = t0 / L;
+            lr[0] = t0 - br[0] * L;
+            hr[1] = hr[0] + 1u, lr[1] = lr[0], br[1] = br[0];
+            if (hr[1] == H) {
+                hr[1] = 0u;
+                if (++lr[1] == L)
+                    lr[1] = 0u, ++br[1];
+            }
+        }
         float v[4][8];
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
@@ -115,10 +145,9 @@ __global__ void __launch_bounds__(256) attn_rowquant_kernel(const AttnQuantParam
                 r = ld_nc_v4(p.x + base + t * 64);
             bf16x8_to_f32(r, v[t]);
             if (p.mu != nullptr && row < p.rows) {
-                const int64_t b = row / (static_cast<int64_t>(p.L) * p.H);
-                const int64_t h = row % p.H;
+                const int64_t bh = static_cast<int64_t>(br[t >> 1]) * H + hr[t >> 1];
                 const int32_t d = (t & 1) * 64 + static_cast<int32_t>(lane & 7u) * 8;
-                const float *m = p.mu + (b * p.H + h) * kAttnD + d;
+                const float *m = p.mu + bh * kAttnD + d;
                 const uint4 a = ld_nc_v4(m), bb = ld_nc_v4(m + 4);
                 const uint32_t w[8] = {a.x, a.y, a.z, a.w, bb.x, bb.y, bb.z, bb.w};
 #pragma unroll
@@ -156,10 +185,8 @@ __global__ void __launch_bounds__(256) attn_rowquant_kernel(const AttnQuantParam
                     st_v2(p.q + base + t * 64, w.x, w.y);
             }
             if (row < p.rows && (lane & 7u) == 0u) {
-                const int64_t h = row % p.H;
-                const int64_t l = (row / p.H) % p.L;
-                const int64_t b = row / (static_cast<int64_t>(p.L) * p.H);
-                p.s[(b * p.H + h) * p.ls + l] = zero ? 0.0f : __fmul_rn(s_z, p.c_g);
+                const int64_t bh = static_cast<int64_t>(br[rr]) * H + hr[rr];
+                p.s[bh * p.ls + lr[rr]] = zero ? 0.0f : __fmul_rn(s_z, p.c_g);
             }
         }
     }

@@ -698,7 +698,8 @@ sdnq_status validate_attention(const void *q, const void *k, const void *v, cons
     if (!q || !k || !v || !o || !ws)
         return SDNQ_ERR_NULL;
     if (B <= 0 || Lq <= 0 || Lk <= 0 || H <= 0 || B * H > INT32_MAX || Lq > INT32_MAX ||
-        Lk > INT32_MAX || (B * H) * ((Lq + 127) / 128) > INT32_MAX)
+        Lk > INT32_MAX || (B * H) * ((Lq + 127) / 128) > INT32_MAX || B * H * Lq > INT32_MAX ||
+        B * H * Lk > INT32_MAX)
         return SDNQ_ERR_SHAPE;
     if (D != kAttnD || !is_pow2(group) || group < SDNQ_MIN_GROUP || group > SDNQ_MAX_GROUP)
         return SDNQ_ERR_UNSUPPORTED;
