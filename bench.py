@@ -494,28 +494,41 @@ def main():
     torch.cuda.synchronize()
     assert sd.sdnq_device_status() == 0
 
-    # timed region: K steps, L2 flushed before each, per-stage CUDA events on the stream
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]
-           for _ in range(args.steps)]
+    # timed region: K steps, L2 flushed before each, one CUDA event pair around each step on
+    # the stream (nothing between the step's launches, so a kernel launched programmatically
+    # may overlap the tail of the one before it, as in use)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     with ClockSampler(local) as clocks:
         for i in range(args.steps):
             flush.zero_()
-            e = evs[i]
-            e[0].record()
-            for j, (_, fn) in enumerate(step.stages):
+            evs[i][0].record()
+            for _, fn in step.stages:
                 fn()
-                e[j + 1].record()
+            evs[i][1].record()
         torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
+    step_ms_total = sum(e[0].elapsed_time(e[1]) for e in evs)
+
+    # per-kernel times for the rooflines: the same K steps again with an event between the
+    # stages (which serialises them)
+    sevs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]
+            for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.zero_()
+        e = sevs[i]
+        e[0].record()
+        for j, (_, fn) in enumerate(step.stages):
+            fn()
+            e[j + 1].record()
+    torch.cuda.synchronize()
     stage_ms = {n: 0.0 for n in names}
-    for e in evs:
+    for e in sevs:
         for j, n in enumerate(names):
             stage_ms[n] += e[j].elapsed_time(e[j + 1])
-    step_ms_total = sum(stage_ms.values())
     t = reduce_max_over_ranks([step_ms_total] + [stage_ms[n] for n in names], dist, world)
     step_ms_total = t[0]
     stage_ms = {n: t[1 + j] for j, n in enumerate(names)}
@@ -615,6 +628,7 @@ def main():
             "peak_source": f"{peak_src} copy bandwidth", "timing": rq_note,
         },
         "stage_ms_per_step": {n: stage_ms[n] / args.steps for n in names},
+        "stage_timing": "a second pass of the same steps with an event between the stages",
         "clocks": clocks.summary(),
         "gpu_launches": step.launches * args.steps,
         "e2e": e2e,

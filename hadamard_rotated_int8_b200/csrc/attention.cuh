@@ -113,6 +113,7 @@ struct AttnQuantParams {
 template <int G>
 __global__ void __launch_bounds__(256, 4) attn_rowquant_kernel(const AttnQuantParams p)
 {
+    grid_dependents_launch();
     const uint32_t lane = lane_id();
     const int64_t nchunks = (p.rows + 7) / 8;
     const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
@@ -322,6 +323,9 @@ __global__ void __launch_bounds__(AttnConfig::THREADS, 1)
     __syncthreads();
     tc_fence_after_sync();
     const uint32_t tmem_base = *tmem_holder;
+    // the prologue may overlap the preparation (programmatic launch); its codes and scales
+    // are read from here on
+    grid_dependency_wait();
 
     if (warp == 0) {
         // ------------------------------------------------------------ loads

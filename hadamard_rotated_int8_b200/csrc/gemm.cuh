@@ -347,6 +347,9 @@ __global__ void __launch_bounds__(GemmConfig<BN, LORA, GELU, (FUSE_G > 0)>::THRE
     __syncthreads();
     tc_fence_after_sync();
     const uint32_t tmem_base = *tmem_holder;
+    // the prologue above may overlap the previous kernel (programmatic launch); from here on
+    // the codes, scales and LoRA terms it wrote are read
+    grid_dependency_wait();
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer

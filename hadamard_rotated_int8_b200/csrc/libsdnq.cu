@@ -302,7 +302,22 @@ sdnq_status launch_gemm(const DeviceInfo &dev, const int8_t *qx, const int8_t *q
             return SDNQ_ERR_CUDA;
         }
     } else {
-        kernel<<<grid, C::THREADS, C::SMEM_BYTES, cs>>>(tmA, tmB, tmU, tmL, tmO, p);
+        // programmatic launch: the prologue overlaps the tail of the kernel before it (the
+        // quantizer), whose results the kernel reads only after griddepcontrol.wait
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>(grid));
+        cfg.blockDim = dim3(C::THREADS);
+        cfg.dynamicSmemBytes = C::SMEM_BYTES;
+        cfg.stream = cs;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (cudaLaunchKernelEx(&cfg, kernel, tmA, tmB, tmU, tmL, tmO, p) != cudaSuccess) {
+            cudaGetLastError();
+            return SDNQ_ERR_CUDA;
+        }
     }
     return launch_status();
 }
@@ -788,8 +803,21 @@ sdnq_status launch_attention_core(const uint16_t *v, int64_t B, int64_t Lq, int6
     p.scale = scale;
     p.timeout_ns = kDefaultTimeoutNs;
     cudaGetLastError();
-    attn_kernel<<<static_cast<unsigned>(B * H * p.q_blocks), AttnConfig::THREADS,
-                  AttnConfig::SMEM_BYTES, cs>>>(tmQ, tmK, tmV, p);
+    // programmatic launch: the prologue overlaps the end of the preparation
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(B * H * p.q_blocks));
+    cfg.blockDim = dim3(AttnConfig::THREADS);
+    cfg.dynamicSmemBytes = AttnConfig::SMEM_BYTES;
+    cfg.stream = cs;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, attn_kernel, tmQ, tmK, tmV, p) != cudaSuccess) {
+        cudaGetLastError();
+        return SDNQ_ERR_CUDA;
+    }
     return launch_status();
 }
 

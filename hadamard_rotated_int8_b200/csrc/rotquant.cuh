@@ -406,6 +406,7 @@ __device__ __forceinline__ void rotquant_worker_rows(const RotquantParams &p, in
 template <int G, bool COLSCALE, bool FP8 = false>
 __global__ void __launch_bounds__(512) rotquant_persistent_kernel(const RotquantParams p)
 {
+    grid_dependents_launch();
     __shared__ float s_amax[2][32];
     const uint32_t lane = lane_id();
     const int32_t warp = static_cast<int32_t>(threadIdx.x >> 5);
@@ -463,6 +464,7 @@ __global__ void __launch_bounds__(512) rotquant_persistent_kernel(const Rotquant
 template <int G, bool COLSCALE, bool FP8 = false>
 __global__ void __launch_bounds__(512) rotquant_kernel(const RotquantParams p)
 {
+    grid_dependents_launch();
     __shared__ float s_amax[32];
     const uint32_t lane = lane_id();
     const int32_t warp = static_cast<int32_t>(threadIdx.x >> 5);
