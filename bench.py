@@ -114,10 +114,12 @@ def rotquant_bytes(M, K):
 
 def fused_one_launch(case, torch):
     """The library's automatic choice for sdnq_int8_linear_fused: one launch when the GEMM has
-    at least three waves of 128 x 256 tiles and the rows fit the in-kernel quantizer."""
+    at least three waves of 128 x 256 tiles, the quantizer is a small share of the work
+    (N >= 3584 or K >= 6144) and the rows fit the in-kernel quantizer."""
     sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
     tiles = ((case.M + 127) // 128) * ((case.N + 255) // 256)
-    return (case.K + 1023) // 1024 <= 8 and tiles >= 3 * sms
+    return ((case.K + 1023) // 1024 <= 8 and tiles >= 3 * sms
+            and (case.N >= 3584 or case.K >= 6144))
 
 
 class Step:

@@ -442,13 +442,16 @@ sdnq_status run_linear_fused(const uint16_t *x, int64_t ldx, int32_t group, cons
         return SDNQ_OK;
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     const int32_t nchunks = static_cast<int32_t>((K + 1023) / 1024);
-    // The one-launch kernel overlaps the quantizer with the GEMM; it pays off once the GEMM
-    // has at least three waves of tiles (with fewer, its first wave needs most rows before
-    // it can start). Rows longer than the quantizer warps can hold take the two launches.
+    // The one-launch kernel overlaps the quantizer with the GEMM. It pays off once the GEMM
+    // has at least three waves of tiles (with fewer, its first wave needs most rows before it
+    // can start) and the quantizer is a small share of the work (N >= 3584, or K >= 6144);
+    // otherwise the two launches, the GEMM's prologue overlapping the quantizer's tail, are
+    // faster (measured on 14 shapes from 4096 x 3072 x 3072 to 16384 x 6144 x 8192). Rows
+    // longer than the quantizer warps can hold take the two launches.
     const int64_t tiles = ((M + 127) / 128) * ((N + 255) / 256);
+    const bool auto_one = tiles >= 3ll * dev.sm_count && (N >= 3584 || K >= 6144);
     const bool fuse = nchunks <= kFusedMaxChunks &&
-                      (policy == SDNQ_FUSE_ALWAYS ||
-                       (policy == SDNQ_FUSE_AUTO && tiles >= 3ll * dev.sm_count));
+                      (policy == SDNQ_FUSE_ALWAYS || (policy == SDNQ_FUSE_AUTO && auto_one));
     if (!fuse) {
         // the two launches (same results)
         if ((st = launch_rowquant(x, M, K, ldx, group, nullptr, qx_ws, sx_ws, dev, cs)) != SDNQ_OK)

@@ -118,7 +118,8 @@ sdnq_status sdnq_int8_linear(const int8_t *qx, const float *sx, const int8_t *qW
  * for bit those of the two calls, which is also what the call runs when `policy` asks for it
  * or when the one launch does not pay off:
  *   policy SDNQ_FUSE_AUTO: one launch when the GEMM has at least three waves of 128 x 256
- *          tiles (ceil(M/128) * ceil(N/256) >= 3 * SM count) and K <= 8192, else two;
+ *          tiles (ceil(M/128) * ceil(N/256) >= 3 * SM count), N >= 3584 or K >= 6144, and
+ *          K <= 8192, else two;
  *   policy SDNQ_FUSE_ALWAYS: one launch whenever K <= 8192;  SDNQ_FUSE_NEVER: two launches.
  *   x [M, K] bf16, row stride ldx; group as in sdnq_rotquant_act.
  *   qW, sW, bias, out, ldo, acc_out as in sdnq_int8_linear.
