@@ -39,6 +39,8 @@ constexpr int kAttnSumSplits = 32;     // key splits of the channel sums
 __global__ void __launch_bounds__(256) attn_ksum_kernel(const uint16_t *k, int32_t Lk, int32_t H,
                                                         double *partial)
 {
+    grid_dependents_launch();
+    grid_dependency_wait();   // launched programmatically: nothing is read or written before
     const int32_t bh = blockIdx.x, split = blockIdx.y;
     const int32_t b = bh / H, h = bh % H;
     const int32_t d8 = (threadIdx.x & 15) * 8;   // 16 threads cover the 128 channels
@@ -82,6 +84,8 @@ __global__ void __launch_bounds__(256) attn_ksum_kernel(const uint16_t *k, int32
 // channel spans less than 2^45 in magnitude, so the split order does not matter.
 __global__ void attn_kmean_kernel(const double *partial, int32_t Lk, float *mu)
 {
+    grid_dependents_launch();
+    grid_dependency_wait();
     const int32_t bh = blockIdx.x, d = threadIdx.x;
     double part[kAttnSumSplits];   // all loads in flight, then the sum
 #pragma unroll
@@ -114,6 +118,7 @@ template <int G>
 __global__ void __launch_bounds__(256, 4) attn_rowquant_kernel(const AttnQuantParams p)
 {
     grid_dependents_launch();
+    grid_dependency_wait();
     const uint32_t lane = lane_id();
     const int64_t nchunks = (p.rows + 7) / 8;
     const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);

@@ -126,6 +126,25 @@ bool set_smem(Kernel k, int bytes)
     return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess;
 }
 
+// Programmatic launch (the kernel may start while the previous one in the stream drains; it
+// waits with griddepcontrol.wait before touching memory). Errors are left for launch_status.
+template <typename... KArgs, typename... Args>
+void launch_programmatic(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                         cudaStream_t cs, Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = cs;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 // ---------------------------------------------------------------- rotate + quantize
 
 sdnq_status validate_rotquant(const void *x, int64_t rows, int64_t K, int64_t ld, int32_t group,
@@ -706,7 +725,8 @@ void launch_attn_rowquant(const AttnQuantParams &p, int sm_count, cudaStream_t c
     const int64_t cap = static_cast<int64_t>(sm_count) * 8;
     if (blocks > cap)
         blocks = cap;
-    attn_rowquant_kernel<G><<<static_cast<unsigned>(blocks), 256, 0, cs>>>(p);
+    launch_programmatic(attn_rowquant_kernel<G>, dim3(static_cast<unsigned>(blocks)), dim3(256), 0,
+                        cs, p);
 }
 
 sdnq_status validate_attention(const void *q, const void *k, const void *v, const void *o,
@@ -744,9 +764,10 @@ sdnq_status launch_attention_prep(const uint16_t *q, const uint16_t *k, int64_t 
     cudaGetLastError();
     const int32_t bh = static_cast<int32_t>(B * H);
     if (smooth_k) {
-        attn_ksum_kernel<<<dim3(bh, kAttnSumSplits), 256, 0, cs>>>(k, static_cast<int32_t>(Lk),
-                                                                   static_cast<int32_t>(H), partial);
-        attn_kmean_kernel<<<bh, kAttnD, 0, cs>>>(partial, static_cast<int32_t>(Lk), mu);
+        launch_programmatic(attn_ksum_kernel, dim3(bh, kAttnSumSplits), dim3(256), 0, cs, k,
+                            static_cast<int32_t>(Lk), static_cast<int32_t>(H), partial);
+        launch_programmatic(attn_kmean_kernel, dim3(bh), dim3(kAttnD), 0, cs,
+                            static_cast<const double *>(partial), static_cast<int32_t>(Lk), mu);
     } else {
         cudaMemsetAsync(mu, 0, 4 * B * H * D, cs);
     }
