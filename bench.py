@@ -585,7 +585,7 @@ def main():
     gemm_tops = ops / (gemm_ms * 1e-3) / 1e12
     if "rotquant" in stage_ms:
         rq_ms = stage_ms["rotquant"] / args.steps
-        rq_note = "the rotate+quantize stage of the timed step"
+        rq_note = "the rotate+quantize stage, from the per-stage pass of the same steps"
     else:
         # the step's quantizer runs inside the fused kernel: time the standalone kernel on
         # the same input (L2 flushed before each launch) for its own roofline
