@@ -43,6 +43,11 @@
  *    device error word; sdnq_device_status() reads and clears it (SDNQ_ERR_TIMEOUT).
  *  - Only sm_100 devices are supported (SDNQ_ERR_UNSUPPORTED otherwise). There is no CPU
  *    and no other-architecture path.
+ *  - The int8 GEMMs, the attention kernel and the attention preparation are launched with
+ *    programmatic stream serialization. Such a kernel may start its prologue (barriers,
+ *    tensor memory, descriptor prefetch) while the previous kernel in the stream drains. It
+ *    reads or writes no global memory before that kernel has completed, so stream order
+ *    holds for the caller's own kernels as well.
  */
 #ifndef SDNQ_H
 #define SDNQ_H
