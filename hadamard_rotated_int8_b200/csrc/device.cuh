@@ -186,27 +186,6 @@ __device__ __forceinline__ void bulk_load_1d(uint32_t dst, const void *src, uint
                  : "memory");
 }
 
-// Per-thread asynchronous 16-byte copy global -> shared, bypassing L1; with `valid` false
-// nothing is read and the 16 bytes are zero-filled.
-__device__ __forceinline__ void cp_async_16(uint32_t dst, const void *src, bool valid)
-{
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
-                 "r"(valid ? 16u : 0u)
-                 : "memory");
-}
-
-__device__ __forceinline__ void cp_async_commit()
-{
-    asm volatile("cp.async.commit_group;" ::: "memory");
-}
-
-// Wait until at most N of this thread's committed groups are still pending.
-template <int N>
-__device__ __forceinline__ void cp_async_wait()
-{
-    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-
 // Named barrier over `count` threads that also ORs a predicate across them.
 __device__ __forceinline__ bool bar_sync_or(uint32_t id, uint32_t count, bool pred)
 {
@@ -217,33 +196,6 @@ __device__ __forceinline__ bool bar_sync_or(uint32_t id, uint32_t count, bool pr
                  : "r"(pred ? 1u : 0u), "r"(id), "r"(count)
                  : "memory");
     return r != 0u;
-}
-
-__device__ __forceinline__ void sts_u8(uint32_t addr, uint32_t v)
-{
-    asm volatile("st.shared.u8 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
-}
-
-__device__ __forceinline__ void sts_b64(uint32_t addr, unsigned long long v)
-{
-    asm volatile("st.shared.b64 [%0], %1;" ::"r"(addr), "l"(v) : "memory");
-}
-
-__device__ __forceinline__ unsigned long long lds_b64(uint32_t addr)
-{
-    unsigned long long v;
-    asm volatile("ld.shared.b64 %0, [%1];" : "=l"(v) : "r"(addr) : "memory");
-    return v;
-}
-
-__device__ __forceinline__ uint4 lds_v4u(uint32_t addr)
-{
-    uint4 v;
-    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "r"(addr)
-                 : "memory");
-    return v;
 }
 
 // TMA: 2-D tiled bulk tensor copy shared -> global (elements outside the tensor are not

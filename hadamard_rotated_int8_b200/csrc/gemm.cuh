@@ -98,11 +98,6 @@ struct GemmConfig {
 
 __device__ __forceinline__ float bf16_bits_to_float(uint32_t b) { return __uint_as_float(b << 16); }
 
-__device__ __forceinline__ uint32_t float_to_bf16_bits(float f)
-{
-    return static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(f)));
-}
-
 // One output block: 16 packed bf16 pairs (32 columns) of this thread's row go through the
 // warp's 64-byte-swizzled staging buffer to a TMA store of the warp's 32 x 32 block at
 // (column nc, row mrow0); rows >= M and columns >= N fall outside the tensor and are dropped.
