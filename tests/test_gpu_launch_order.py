@@ -134,3 +134,28 @@ def test_attention_back_to_back():
     torch.cuda.synchronize()
     for i, (a, b) in enumerate(zip(alone, outs)):
         assert_equal(bits_of(b), bits_of(a), f"round {i}")
+
+
+def test_weights_quantized_right_before_the_gemm():
+    """The weight quantizer triggers its dependents at entry; the GEMM launched right after it
+    must still read the finished codes and scales (a new weight every round, same buffers)."""
+    M, N, K = 1024, 1536, 2048
+    x = inputs(M, K, 500)[0]
+    Ws = [synthetic.make_case(M=8, N=N, K=K, g=256, seed=600 + i).W.cuda() for i in range(ROUNDS)]
+    qx, sx = sd.sdnq_rotquant_act(x, 256)
+    torch.cuda.synchronize()
+    alone = []
+    for W in Ws:
+        qW, sW = sd.sdnq_rotate_quant_weight(W, 256)
+        torch.cuda.synchronize()
+        alone.append(sd.sdnq_int8_linear(qx, sx, qW, sW))
+        torch.cuda.synchronize()
+    qW = torch.empty((N, K), dtype=torch.int8, device="cuda")
+    sW = torch.empty((N,), dtype=torch.float32, device="cuda")
+    outs = []
+    for W in Ws:   # quantize the weight, then the GEMM at once, no synchronisation
+        sd.sdnq_rotate_quant_weight(W, 256, qW, sW)
+        outs.append(sd.sdnq_int8_linear(qx, sx, qW, sW))
+    torch.cuda.synchronize()
+    for i, (a, b) in enumerate(zip(alone, outs)):
+        assert_equal(bits_of(b), bits_of(a), f"round {i}")
