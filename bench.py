@@ -450,7 +450,7 @@ def config_of(case, args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="sdnq", choices=["sdnq", "reference"])
     ap.add_argument("--workload", default="dit_attn_4096x3072x3072")
