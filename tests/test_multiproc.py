@@ -73,3 +73,13 @@ def test_reference_arm_prints_on_rank_zero_only():
     line = json.loads(r0.stdout.strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["unit"] == "TOPS" and line["value"] > 0
     assert line["e2e"]["h2d_bytes_per_step"] == 0
+    # the JSON line's contract: every key present, the baseline described
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+                "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["steps"] == 1 and line["warmup"] >= 3 and line["higher_is_better"] is True
+    assert line["config"]["workload"] == "tiny_256"
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["sample"] and cb["value"] == line["value"]
+    assert line["e2e"]["value"] == line["value"] and line["e2e"]["unit"] == line["unit"]
