@@ -30,7 +30,7 @@
 namespace sdnq {
 
 constexpr int kAttnD = 128;
-constexpr int kAttnBlock = 128;        // queries per CTA and keys per step
+constexpr int kAttnBlock = 128;        // queries per tile (two tiles per CTA) and keys per step
 constexpr int kAttnSumSplits = 32;     // key splits of the channel sums
 
 // ---------------------------------------------------------------- smooth_k channel means
