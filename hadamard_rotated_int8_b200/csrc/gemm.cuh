@@ -19,6 +19,11 @@
 // Two accumulator buffers in TMEM let the epilogue of tile i overlap the MMAs of tile i+1
 // (one buffer when a tile's accumulators fill all 512 columns, as with LoRA at N = 256).
 // Operand tiles use the 128-byte swizzle written by TMA and read by the MMA descriptors.
+// Further modes: the input gradient (N-major B, an inverse-butterfly epilogue), FP8 operands
+// (kind::f8f6f4, fp32 accumulators) and the activation quantizer inside the kernel (extra
+// warps that quantize x into the A operand and publish rows to the producers).
+// Launched programmatically: the prologue may overlap the kernel before it in the stream,
+// and every thread waits (griddepcontrol.wait) before it touches global memory.
 //
 // Every wait is bounded (mbar_wait_bounded): on timeout the CTA raises its abort flag and
 // the device error word, each role leaves its loop, in-flight copies and MMAs are drained

@@ -2,7 +2,9 @@
 // Walsh-Hadamard butterfly over groups of G columns, the full-row absmax, the fp32 scale and
 // round-half-to-even int8 codes, in one pass over HBM. With G = 1 and a column multiplier
 // (COLSCALE) the same kernels quantize dy * sW per token for the input gradient of the frozen
-// base (no rotation on that operand).
+// base (no rotation on that operand); with FP8 they write e4m3 codes on the +-448 grid.
+// The kernels let the next kernel in the stream launch at once (griddepcontrol), which waits
+// for their completion before it reads their codes and scales.
 //
 // Sources: "SDNQ: SD.Next Quantization Engine" README (Hadamard rotations on both the
 // quantized weights and the quantized matmul; row-wise scales, FP32 de-quant); "ConvRot /
