@@ -5,8 +5,10 @@ quantize the activations (per-token scales) and run the tensor-core int8 matmul 
 fused fp32 de-quant epilogue (plus the LoRA term, or the MLP chain, for those workloads).
 Weights are rotated and quantized once before timing (offline, as on the pages).
 
-Default workload: the DiT attention projection, x [4096, 3072] bf16 with 1% outlier
-channels x30, W [3072, 3072], bias, Hadamard group 256.
+Default workload: the DiT MLP pair, x [4608, 3840] bf16 Student-t(4) activations through the
+up-projection W_up [10240, 3840] with GELU in its epilogue, per-token requantisation of the
+hidden layer and the down-projection W_down [3840, 10240], Hadamard group 256 (725 GOP of int8
+matmul per step).
 
 Output: one JSON line on rank 0. ``value`` is int8 TOPS of the whole step (2*M*N*K per
 GEMM over the device time of every kernel of the step), summed over ranks (replicas:
@@ -54,7 +56,8 @@ def measured_peaks():
 # The sources each profiled kernel is compiled from (its own header and the shared PTX
 # helpers): an ncu summary stays valid until one of these changes.
 KERNEL_SOURCES = {
-    "gemm_s8": ("device.cuh", "gemm.cuh"),
+    "gemm_s8": ("device.cuh", "gemm.cuh", "gelu.cuh", "rotquant.cuh"),
+    "lora_down": ("device.cuh", "lora_down.cuh"),
     "rotquant": ("device.cuh", "rotquant.cuh"),
     "attn_kernel": ("device.cuh", "rotquant.cuh", "attention.cuh"),
 }
@@ -77,10 +80,11 @@ def kernel_source_hash(kernel: str) -> str:
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(kernel: str, workload: str):
-    """DRAM bytes per launch of `kernel` from the committed ncu summary for this workload,
-    if it was taken on the current kernel sources; else None."""
-    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
+def profiled_traffic(profile: str, kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary `profiles/<profile>_<workload>.md`
+    of a kernel of family `kernel`, if it was taken on the current kernel sources; else
+    None."""
+    path = os.path.join(ROOT, "profiles", f"{profile}_{workload}.md")
     try:
         text = open(path).read()
     except OSError:
@@ -119,16 +123,6 @@ def workload_ops(case, name):
 
 def rotquant_bytes(M, K):
     return M * K * 2 + M * K + M * 4   # read bf16, write int8 codes, write fp32 scale
-
-
-def fused_one_launch(case, torch):
-    """The library's automatic choice for sdnq_int8_linear_fused: one launch when the GEMM has
-    at least three waves of 128 x 256 tiles, the quantizer is a small share of the work
-    (N >= 3584 or K >= 6144) and the rows fit the in-kernel quantizer."""
-    sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
-    tiles = ((case.M + 127) // 128) * ((case.N + 255) // 256)
-    return ((case.K + 1023) // 1024 <= 8 and tiles >= 3 * sms
-            and (case.N >= 3584 or case.K >= 6144))
 
 
 class Step:
@@ -210,7 +204,8 @@ class Step:
             ]
             self.gemm_stages = ["gemm_lora"]
             self.launches = 3  # rotquant, LoRA down-projection, fused GEMM
-        elif fused_one_launch(case, torch):
+        elif sd.sdnq_int8_linear_fused_plan(case.M, case.N, case.K):
+            # the library's own choice for sdnq_int8_linear_fused (one launch here)
             # one launch: the activation quantizer runs inside the GEMM kernel
             self.sync = torch.zeros(4 * ((case.M + 127) // 128) + 64, dtype=torch.int32,
                                     device=dev)
@@ -462,7 +457,7 @@ def main():
     ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="sdnq", choices=["sdnq", "reference"])
-    ap.add_argument("--workload", default="dit_attn_4096x3072x3072")
+    ap.add_argument("--workload", default="dit_mlp_4608x3840x10240")
     ap.add_argument("--group", type=int, default=None)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -619,39 +614,77 @@ def main():
                "streams": "copy in / compute / copy out, two buffer sets"}
 
     peaks, peak_src = measured_peaks()
-    # the burst GEMM peak for a kernel that ran at full clock; the sustained one (a seconds-long
-    # loop under the power cap) when the timed region itself reached the power cap
+    # GEMM rooflines against the published dense INT8 peak of the B200 (the denominator the
+    # targets are stated against); the measured cuBLAS bf16 peak x 2 (the nominal int8/bf16
+    # ratio) is given beside it: the burst figure for a kernel that ran at full clock, the
+    # sustained one when the timed region itself reached the power cap
     capped = "sw_power_cap" in clocks.summary()["reasons"] and "bf16_tflops_sustained" in peaks
     bf16_peak = peaks["bf16_tflops_sustained"] if capped else peaks["bf16_tflops"]
     bf16_kind = "sustained (the timed region reached the power cap)" if capped else "burst"
-    int8_peak = bf16_peak * NOMINAL_INT8_OVER_BF16
+    measured_int8 = bf16_peak * NOMINAL_INT8_OVER_BF16
+    spec_peak = INT8_SPEC_TOPS
     if case.extra.get("attn"):
         # half the ops run int8 (QK), half bf16 (PV): the ceiling of that mix
-        int8_peak = 2.0 / (1.0 / int8_peak + 1.0 / bf16_peak)
-    gemm_ms = sum(stage_ms[n] for n in step.gemm_stages) / args.steps
-    gemm_launch_ms = gemm_ms / len(step.gemm_stages)
-    gemm_tops = ops / (gemm_ms * 1e-3) / 1e12
-    if "rotquant" in stage_ms:
-        rq_ms = stage_ms["rotquant"] / args.steps
-        rq_note = "the rotate+quantize stage, from the per-stage pass of the same steps"
-    else:
-        # the step's quantizer runs inside the fused kernel: time the standalone kernel on
-        # the same input (L2 flushed before each launch) for its own roofline
-        rq_ms = standalone_rotquant_ms(step, flush, torch, sd, max(args.steps // 4, 10))
-        rq_note = "standalone rotquant kernel on the step's input (the step itself runs it fused)"
+        measured_int8 = 2.0 / (1.0 / measured_int8 + 1.0 / bf16_peak)
+        spec_peak = 2.0 / (1.0 / INT8_SPEC_TOPS + 1.0 / (INT8_SPEC_TOPS / 2))
     grad = args.workload.startswith("grad_")
-    rq_rows_k = case.N if grad else case.K        # row length of the quantized operand
-    rq_bytes = rotquant_bytes(case.M, rq_rows_k)
-    if case.extra.get("attn"):
-        # q and k rows of D (read bf16, write int8 + scale) and k read once more for the means
-        n_el = case.extra["B"] * case.M * case.N * case.K
-        rq_bytes = 2 * (3 * n_el + 4 * n_el // case.K) + 2 * n_el
-    rq_gbs = rq_bytes / (rq_ms * 1e-3) / 1e9
     gemm_kernel = ("attn_kernel" if case.extra.get("attn") else
                    "gemm_s8_kernel_e4m3" if args.workload.startswith("fp8_") else
                    "gemm_s8_kernel_grad_input" if grad else
                    "gemm_s8_kernel_fused_quantizer" if "fused" in stage_ms else
                    "gemm_s8_kernel" if case.A is None else "gemm_s8_kernel_lora")
+    kernel_of = {"gemm_up": "gemm_s8_kernel_gelu_epilogue", "gemm_down": "gemm_s8_kernel"}
+    ops_per_gemm = ops / len(step.gemm_stages)
+    gemm_lines = {}
+    for n in step.gemm_stages:
+        ms = stage_ms[n] / args.steps
+        tops = ops_per_gemm / (ms * 1e-3) / 1e12
+        gemm_lines[n] = {
+            "kernel": kernel_of.get(n, gemm_kernel), "bound": "tensor", "achieved": tops,
+            "peak": spec_peak, "unit": "TFLOP/s", "frac": tops / spec_peak,
+            "traffic": profiled_traffic(n, "attn_kernel" if case.extra.get("attn") else "gemm_s8",
+                                        args.workload),
+            "ops_per_launch": ops_per_gemm, "ms_per_launch": ms,
+            "peak_source": ("NVIDIA B200 dense INT8 spec, 4500 TOPS"
+                            + (" (int8 QK / bf16 PV mix)" if case.extra.get("attn") else "")),
+            "measured_peak": measured_int8,
+            "frac_of_measured": tops / measured_int8,
+            "measured_peak_source": f"{peak_src} cuBLAS bf16 {bf16_kind} x "
+                                    f"{NOMINAL_INT8_OVER_BF16} (int8/bf16 nominal)",
+        }
+    dominant = max(step.gemm_stages, key=lambda n: stage_ms[n])
+    gemm_tops = ops / (sum(stage_ms[n] for n in step.gemm_stages) / args.steps * 1e-3) / 1e12
+
+    rq_rows_k = case.N if grad else case.K        # row length of the quantized operand
+    rq_lines = {}
+    rq_stages = [n for n in names if n.startswith("rotquant")]
+    if not rq_stages:
+        # the step's quantizer runs inside the fused kernel: time the standalone kernel on
+        # the same input (L2 flushed before each launch) for its own roofline
+        rq_ms = standalone_rotquant_ms(step, flush, torch, sd, max(args.steps // 4, 10))
+        rq_timed = {"rotquant": (rq_ms, rq_rows_k, "standalone rotquant kernel on the step's "
+                                 "input (the step itself runs it fused)")}
+    else:
+        rq_timed = {n: (stage_ms[n] / args.steps,
+                        case.N if n == "rotquant_h" else rq_rows_k,
+                        "the stage's time in the per-stage pass of the same steps")
+                    for n in rq_stages}
+    for n, (ms, rows_k, note) in rq_timed.items():
+        nbytes = rotquant_bytes(case.M, rows_k)
+        if case.extra.get("attn"):
+            # q and k rows of D (read bf16, write int8 + scale) and k read once more for the
+            # means
+            n_el = case.extra["B"] * case.M * case.N * case.K
+            nbytes = 2 * (3 * n_el + 4 * n_el // case.K) + 2 * n_el
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        rq_lines[n] = {
+            "kernel": "rotquant_persistent_kernel" if rows_k <= 16384 else "rotquant_kernel",
+            "bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": gbs / peaks["hbm_gbs"],
+            "traffic": profiled_traffic(n, "rotquant", args.workload),
+            "bytes_per_launch": nbytes, "row_length": rows_k, "ms_per_launch": ms,
+            "peak_source": f"{peak_src} copy bandwidth", "timing": note,
+        }
     line = {
         "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
@@ -660,24 +693,8 @@ def main():
         "data": "synthetic (seeded DiT-shaped bf16 activations with outlier channels, "
                 "random-init weights)",
         "config": config_of(case, args),
-        "roofline": {
-            "kernel": gemm_kernel, "bound": "tensor", "achieved": gemm_tops,
-            "peak": int8_peak, "unit": "TFLOP/s", "frac": gemm_tops / int8_peak,
-            "traffic": profiled_traffic("attn_kernel" if case.extra.get("attn") else "gemm_s8",
-                                        args.workload),
-            "ops_per_launch": ops / len(step.gemm_stages), "ms_per_launch": gemm_launch_ms,
-            "peak_source": f"{peak_src} bf16 {bf16_kind} x {NOMINAL_INT8_OVER_BF16} "
-                           "(int8/bf16 nominal)",
-            "frac_of_int8_spec": gemm_tops / INT8_SPEC_TOPS,
-        },
-        "roofline_rotquant": {
-            "kernel": ("rotquant_persistent_kernel" if rq_rows_k <= 16384 else "rotquant_kernel"),
-            "bound": "hbm", "achieved": rq_gbs,
-            "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": rq_gbs / peaks["hbm_gbs"],
-            "traffic": profiled_traffic("rotquant", args.workload),
-            "bytes_per_launch": rq_bytes, "ms_per_launch": rq_ms,
-            "peak_source": f"{peak_src} copy bandwidth", "timing": rq_note,
-        },
+        "roofline": gemm_lines[dominant],
+        "gemm_tops": gemm_tops,
         "stage_ms_per_step": {n: stage_ms[n] / args.steps for n in names},
         "stage_timing": "a second pass of the same steps with an event between the stages",
         "clocks": clocks.summary(),
@@ -685,6 +702,11 @@ def main():
         "e2e": e2e,
     }
     line["config"]["stages"] = names
+    for n in step.gemm_stages:
+        if len(step.gemm_stages) > 1:
+            line[f"roofline_{n}"] = gemm_lines[n]
+    for n, r in rq_lines.items():
+        line[f"roofline_{n}"] = r
     if lora_flops:
         line["tops_with_lora_flops"] = whole_job_tops(ops + lora_flops, world, ms_per_step)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

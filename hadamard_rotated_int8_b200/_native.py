@@ -44,6 +44,7 @@ SIGNATURES = {
     "sdnq_int8_linear_gelu": [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _I64, _P, _P],
     "sdnq_int8_linear_fused": [_P, _I64, _I32, _P, _P, _P, _I64, _I64, _I64, _P, _P, _P, _P, _I64,
                                _P, _I32, _P],
+    "sdnq_int8_linear_fused_plan": [_I64, _I64, _I64, _I32, _P],
     "sdnq_int8_linear_grad_input": [_P, _I64, _P, _P, _I64, _I64, _I64, _I32, _P, _P, _P, _I64,
                                     _P, _P],
     "sdnq_quant_grad_output": [_P, _I64, _P, _I64, _I64, _P, _P, _P],
@@ -125,17 +126,53 @@ def _ptr(t: torch.Tensor | None):
     return _P(t.data_ptr()) if t is not None else _P(0)
 
 
+def _on_current_device(t: torch.Tensor, name: str):
+    """The library launches on the current CUDA device; a tensor elsewhere would be read
+    through a peer mapping or fault, so it is refused here."""
+    if t.device.type != "cuda":
+        raise ValueError(f"{name}: must be a CUDA tensor (no CPU path)")
+    if t.device.index != torch.cuda.current_device():
+        raise ValueError(f"{name}: on {t.device}, but the current device is "
+                         f"cuda:{torch.cuda.current_device()}")
+
+
 def _req(t: torch.Tensor, dtype, name: str, ndim: int):
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name}: expected a torch.Tensor")
     if t.dtype != dtype:
         raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
-    if t.device.type != "cuda":
-        raise ValueError(f"{name}: must be a CUDA tensor (no CPU path)")
+    _on_current_device(t, name)
     if t.dim() != ndim:
         raise ValueError(f"{name}: expected {ndim} dims, got {t.dim()}")
     if t.stride(-1) != 1:
         raise ValueError(f"{name}: last dimension must be contiguous")
+
+
+def _vec(t, dtype, n: int, name: str, optional: bool = False):
+    """A dense 1-D tensor of at least n elements (a scale or bias vector the kernels index
+    up to n - 1); None is accepted only where the argument is optional."""
+    if t is None:
+        if optional:
+            return
+        raise ValueError(f"{name}: required")
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name}: expected a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    _on_current_device(t, name)
+    if t.dim() != 1 or not t.is_contiguous():
+        raise ValueError(f"{name}: expected a contiguous 1-D tensor")
+    if t.numel() < n:
+        raise ValueError(f"{name}: has {t.numel()} elements, needs {n}")
+
+
+def _mat(t, dtype, rows: int, cols: int, name: str, dense: bool = False):
+    """A 2-D tensor of exactly [rows, cols] with unit column stride (dense if asked)."""
+    _req(t, dtype, name, 2)
+    if tuple(t.shape) != (rows, cols):
+        raise ValueError(f"{name}: expected shape {(rows, cols)}, got {tuple(t.shape)}")
+    if dense:
+        _dense(t, name)
 
 
 def _dense(t: torch.Tensor, name: str):
@@ -159,6 +196,8 @@ def sdnq_rotate_quant_weight(W: torch.Tensor, group: int = 256, qW=None, sW=None
     N, K = W.shape
     qW = torch.empty((N, K), dtype=torch.int8, device=W.device) if qW is None else qW
     sW = torch.empty((N,), dtype=torch.float32, device=W.device) if sW is None else sW
+    _mat(qW, torch.int8, N, K, "qW", dense=True)
+    _vec(sW, torch.float32, N, "sW")
     _check(lib().sdnq_rotate_quant_weight(_ptr(W), N, K, W.stride(0), group, _ptr(qW), _ptr(sW),
                                           _stream(stream)), "sdnq_rotate_quant_weight")
     return qW, sW
@@ -170,21 +209,36 @@ def sdnq_rotquant_act(x: torch.Tensor, group: int = 256, qx=None, sx=None, strea
     M, K = x.shape
     qx = torch.empty((M, K), dtype=torch.int8, device=x.device) if qx is None else qx
     sx = torch.empty((M,), dtype=torch.float32, device=x.device) if sx is None else sx
+    _mat(qx, torch.int8, M, K, "qx", dense=True)
+    _vec(sx, torch.float32, M, "sx")
     _check(lib().sdnq_rotquant_act(_ptr(x), M, K, x.stride(0), group, _ptr(qx), _ptr(sx),
                                    _stream(stream)), "sdnq_rotquant_act")
     return qx, sx
 
 
-def _linear_call(name, qx, sx, qW, sW, bias, out, acc_out, stream):
-    _req(qx, torch.int8, "qx", 2)
-    _req(qW, torch.int8, "qW", 2)
+def _linear_operands(qx, sx, qW, sW, bias, out, acc_out, code_dtype=torch.int8,
+                     acc_dtype=torch.int32):
+    """Checks the operands of a linear call; returns (M, N, K, out)."""
+    _req(qx, code_dtype, "qx", 2)
+    _req(qW, code_dtype, "qW", 2)
     _dense(qx, "qx")
     _dense(qW, "qW")
     M, K = qx.shape
     N = qW.shape[0]
     if qW.shape[1] != K:
         raise ValueError("qx and qW disagree on K")
+    _vec(sx, torch.float32, M, "sx")
+    _vec(sW, torch.float32, N, "sW")
+    _vec(bias, torch.bfloat16, N, "bias", optional=True)
     out = _rows_out(M, N, torch.bfloat16, qx.device) if out is None else out
+    _mat(out, torch.bfloat16, M, N, "out")
+    if acc_out is not None:
+        _mat(acc_out, acc_dtype, M, N, "acc_out", dense=True)
+    return M, N, K, out
+
+
+def _linear_call(name, qx, sx, qW, sW, bias, out, acc_out, stream):
+    M, N, K, out = _linear_operands(qx, sx, qW, sW, bias, out, acc_out)
     _check(getattr(lib(), name)(_ptr(qx), _ptr(sx), _ptr(qW), _ptr(sW), _ptr(bias), M, N, K,
                                 _ptr(out), out.stride(0), _ptr(acc_out), _stream(stream)), name)
     return out
@@ -201,6 +255,8 @@ def sdnq_rotquant_fp8(x, group: int, q=None, s=None, stream=None):
     M, K = x.shape
     q = torch.empty((M, K), dtype=torch.uint8, device=x.device) if q is None else q
     s = torch.empty((M,), dtype=torch.float32, device=x.device) if s is None else s
+    _mat(q, torch.uint8, M, K, "q", dense=True)
+    _vec(s, torch.float32, M, "s")
     _check(lib().sdnq_rotquant_fp8(_ptr(x), M, K, x.stride(0), group, _ptr(q), _ptr(s),
                                    _stream(stream)), "sdnq_rotquant_fp8")
     return q, s
@@ -208,15 +264,8 @@ def sdnq_rotquant_fp8(x, group: int, q=None, s=None, stream=None):
 
 def sdnq_fp8_linear(qx, sx, qW, sW, bias=None, out=None, acc_out=None, stream=None):
     """out [M, N] bf16 from e4m3 codes qx [M, K], qW [N, K] (uint8) and their scales."""
-    _req(qx, torch.uint8, "qx", 2)
-    _req(qW, torch.uint8, "qW", 2)
-    _dense(qx, "qx")
-    _dense(qW, "qW")
-    M, K = qx.shape
-    N = qW.shape[0]
-    if qW.shape[1] != K:
-        raise ValueError("qx and qW disagree on K")
-    out = _rows_out(M, N, torch.bfloat16, qx.device) if out is None else out
+    M, N, K, out = _linear_operands(qx, sx, qW, sW, bias, out, acc_out, torch.uint8,
+                                    torch.float32)
     _check(lib().sdnq_fp8_linear(_ptr(qx), _ptr(sx), _ptr(qW), _ptr(sW), _ptr(bias), M, N, K,
                                  _ptr(out), out.stride(0), _ptr(acc_out), _stream(stream)),
            "sdnq_fp8_linear")
@@ -245,7 +294,12 @@ def sdnq_attention_int8qk(q, k, v, group: int = 256, scale: float | None = None,
         raise ValueError("q, k, v shapes disagree")
     total, _ = attention_workspace(B, Lq, Lk, H, D)
     ws = torch.empty(total, dtype=torch.uint8, device=q.device) if ws is None else ws
+    _vec(ws, torch.uint8, total, "ws")
     out = torch.empty_like(q) if out is None else out
+    _req(out, torch.bfloat16, "out", 4)
+    _dense(out, "out")
+    if out.shape != q.shape:
+        raise ValueError("out must have q's shape")
     scale = float(1.0 / math.sqrt(D)) if scale is None else float(scale)
     _check(lib().sdnq_attention_int8qk(_ptr(q), _ptr(k), _ptr(v), B, Lq, Lk, H, D, group, scale,
                                        1 if smooth_k else 0, _ptr(ws), ws.numel(), _ptr(out),
@@ -260,8 +314,11 @@ def sdnq_attention_prep(q, k, group: int = 256, smooth_k: bool = True, ws=None, 
         _dense(t, n)
     B, Lq, H, D = q.shape
     Lk = k.shape[1]
+    if k.shape[0] != B or k.shape[2:] != q.shape[2:]:
+        raise ValueError("q and k shapes disagree")
     total, _ = attention_workspace(B, Lq, Lk, H, D)
     ws = torch.empty(total, dtype=torch.uint8, device=q.device) if ws is None else ws
+    _vec(ws, torch.uint8, total, "ws")
     _check(lib().sdnq_attention_prep(_ptr(q), _ptr(k), B, Lq, Lk, H, D, group,
                                      1 if smooth_k else 0, _ptr(ws), ws.numel(), _stream(stream)),
            "sdnq_attention_prep")
@@ -273,7 +330,13 @@ def sdnq_attention_core(v, Lq: int, ws, scale: float | None = None, out=None, st
     _req(v, torch.bfloat16, "v", 4)
     _dense(v, "v")
     B, Lk, H, D = v.shape
+    total, _ = attention_workspace(B, Lq, Lk, H, D)
+    _vec(ws, torch.uint8, total, "ws")
     out = torch.empty((B, Lq, H, D), dtype=torch.bfloat16, device=v.device) if out is None else out
+    _req(out, torch.bfloat16, "out", 4)
+    _dense(out, "out")
+    if tuple(out.shape) != (B, Lq, H, D):
+        raise ValueError(f"out: expected shape {(B, Lq, H, D)}")
     scale = float(1.0 / math.sqrt(D)) if scale is None else float(scale)
     _check(lib().sdnq_attention_core(_ptr(v), B, Lq, Lk, H, D, scale, _ptr(ws), ws.numel(),
                                      _ptr(out), _stream(stream)), "sdnq_attention_core")
@@ -318,15 +381,26 @@ def sdnq_int8_linear_fused(x, group: int, qW, sW, bias=None, qx_ws=None, sx_ws=N
     dev = x.device
     qx_ws = torch.empty((M, K), dtype=torch.int8, device=dev) if qx_ws is None else qx_ws
     sx_ws = torch.empty((M,), dtype=torch.float32, device=dev) if sx_ws is None else sx_ws
+    _, _, _, out = _linear_operands(qx_ws, sx_ws, qW, sW, bias, out, acc_out)
+    if sync_ws is not None:
+        _vec(sync_ws, torch.int32, fused_sync_words(M), "sync_ws")
     st = _stream(stream)
     if sync_ws is None:
         sync_ws = _sync_buffer(dev, st.value or 0, M)
-    out = _rows_out(M, N, torch.bfloat16, dev) if out is None else out
     _check(lib().sdnq_int8_linear_fused(_ptr(x), x.stride(0), group, _ptr(qW), _ptr(sW),
                                         _ptr(bias), M, N, K, _ptr(qx_ws), _ptr(sx_ws),
                                         _ptr(sync_ws), _ptr(out), out.stride(0), _ptr(acc_out),
                                         int(policy), st), "sdnq_int8_linear_fused")
     return out
+
+
+def sdnq_int8_linear_fused_plan(M: int, N: int, K: int, policy: int = FUSE_AUTO) -> bool:
+    """True if sdnq_int8_linear_fused takes one launch for these sizes on the current
+    device, False for the two launches (the library's own rule; nothing is launched)."""
+    one = ctypes.c_int32(0)
+    _check(lib().sdnq_int8_linear_fused_plan(M, N, K, int(policy), ctypes.byref(one)),
+           "sdnq_int8_linear_fused_plan")
+    return bool(one.value)
 
 
 def sdnq_int8_linear_gelu(qx, sx, qW, sW, bias=None, out=None, acc_out=None, stream=None):
@@ -346,9 +420,15 @@ def sdnq_int8_linear_grad_input(dy, qW, sW, group: int, qg_ws=None, sg_ws=None, 
         raise ValueError("dy and qW disagree on N")
     K = qW.shape[1]
     dev = dy.device
+    _vec(sW, torch.float32, N, "sW")
     qg_ws = torch.empty((M, N), dtype=torch.int8, device=dev) if qg_ws is None else qg_ws
     sg_ws = torch.empty((M,), dtype=torch.float32, device=dev) if sg_ws is None else sg_ws
+    _mat(qg_ws, torch.int8, M, N, "qg_ws", dense=True)
+    _vec(sg_ws, torch.float32, M, "sg_ws")
     out = _rows_out(M, K, torch.bfloat16, dev) if out is None else out
+    _mat(out, torch.bfloat16, M, K, "out")
+    if acc_out is not None:
+        _mat(acc_out, torch.int32, M, K, "acc_out", dense=True)
     _check(lib().sdnq_int8_linear_grad_input(_ptr(dy), dy.stride(0), _ptr(qW), _ptr(sW), M, N, K,
                                              group, _ptr(qg_ws), _ptr(sg_ws), _ptr(out),
                                              out.stride(0), _ptr(acc_out), _stream(stream)),
@@ -360,8 +440,11 @@ def sdnq_quant_grad_output(dy, sW, qg=None, sg=None, stream=None):
     """(qg [M, N] int8, sg [M] fp32): per-token int8 of fp32(dy) * sW."""
     _req(dy, torch.bfloat16, "dy", 2)
     M, N = dy.shape
+    _vec(sW, torch.float32, N, "sW")
     qg = torch.empty((M, N), dtype=torch.int8, device=dy.device) if qg is None else qg
     sg = torch.empty((M,), dtype=torch.float32, device=dy.device) if sg is None else sg
+    _mat(qg, torch.int8, M, N, "qg", dense=True)
+    _vec(sg, torch.float32, M, "sg")
     _check(lib().sdnq_quant_grad_output(_ptr(dy), dy.stride(0), _ptr(sW), M, N, _ptr(qg),
                                         _ptr(sg), _stream(stream)), "sdnq_quant_grad_output")
     return qg, sg
@@ -377,28 +460,39 @@ def sdnq_int8_grad_input_gemm(qg, sg, qW, group: int, out=None, acc_out=None, st
     if qW.shape[0] != N:
         raise ValueError("qg and qW disagree on N")
     K = qW.shape[1]
+    _vec(sg, torch.float32, M, "sg")
     out = _rows_out(M, K, torch.bfloat16, qg.device) if out is None else out
+    _mat(out, torch.bfloat16, M, K, "out")
+    if acc_out is not None:
+        _mat(acc_out, torch.int32, M, K, "acc_out", dense=True)
     _check(lib().sdnq_int8_grad_input_gemm(_ptr(qg), _ptr(sg), _ptr(qW), M, N, K, group,
                                            _ptr(out), out.stride(0), _ptr(acc_out),
                                            _stream(stream)), "sdnq_int8_grad_input_gemm")
     return out
 
 
+def _lora_operands(qx, sx, qW, sW, bias, x, A, B, out, acc_out):
+    """Checks the operands of a LoRA linear call; returns (M, N, K, rank, out)."""
+    M, N, K, out = _linear_operands(qx, sx, qW, sW, bias, out, acc_out)
+    _req(x, torch.bfloat16, "x", 2)
+    if tuple(x.shape) != (M, K):
+        raise ValueError(f"x: expected shape {(M, K)}, got {tuple(x.shape)}")
+    _req(A, torch.bfloat16, "A", 2)
+    _req(B, torch.bfloat16, "B", 2)
+    _dense(A, "A")
+    _dense(B, "B")
+    rank = A.shape[1]
+    if A.shape[0] != K or tuple(B.shape) != (rank, N):
+        raise ValueError("LoRA shapes disagree: A must be [K, rank] and B [rank, N]")
+    return M, N, K, rank, out
+
+
 def sdnq_int8_linear_lora(qx, sx, qW, sW, bias, x, A, B, lora_scale: float = 1.0, u_ws=None,
                           out=None, acc_out=None, stream=None):
     """As sdnq_int8_linear plus lora_scale * bf16(x A) B; u_ws [M, rank] receives bf16(x A)."""
-    _req(qx, torch.int8, "qx", 2)
-    _req(qW, torch.int8, "qW", 2)
-    _req(x, torch.bfloat16, "x", 2)
-    _dense(A, "A")
-    _dense(B, "B")
-    M, K = qx.shape
-    N = qW.shape[0]
-    rank = A.shape[1]
-    if A.shape[0] != K or B.shape != (rank, N) or x.shape != (M, K):
-        raise ValueError("LoRA shapes disagree")
+    M, N, K, rank, out = _lora_operands(qx, sx, qW, sW, bias, x, A, B, out, acc_out)
     u_ws = torch.empty((M, rank), dtype=torch.bfloat16, device=qx.device) if u_ws is None else u_ws
-    out = _rows_out(M, N, torch.bfloat16, qx.device) if out is None else out
+    _mat(u_ws, torch.bfloat16, M, rank, "u_ws", dense=True)
     _check(lib().sdnq_int8_linear_lora(_ptr(qx), _ptr(sx), _ptr(qW), _ptr(sW), _ptr(bias),
                                        _ptr(x), x.stride(0), _ptr(A), _ptr(B), rank,
                                        float(lora_scale), _ptr(u_ws), M, N, K, _ptr(out),
@@ -415,20 +509,10 @@ def sdnq_int8_linear_lora_noalloc(qx, sx, qW, sW, bias, x, A, B, lora_scale: flo
     """sdnq_int8_linear_lora for callers that cannot provide device memory for the u
     workspace: u lives in a fixed 8 MiB array inside the library (M * rank must not exceed
     NOALLOC_MAX_U_ELEMS). Calls that overlap on the GPU share that array and race."""
-    _req(qx, torch.int8, "qx", 2)
-    _req(qW, torch.int8, "qW", 2)
-    _req(x, torch.bfloat16, "x", 2)
-    _dense(A, "A")
-    _dense(B, "B")
-    M, K = qx.shape
-    N = qW.shape[0]
-    rank = A.shape[1]
-    if A.shape[0] != K or B.shape != (rank, N) or x.shape != (M, K):
-        raise ValueError("LoRA shapes disagree")
+    M, N, K, rank, out = _lora_operands(qx, sx, qW, sW, bias, x, A, B, out, acc_out)
     if M * rank > NOALLOC_MAX_U_ELEMS:
         raise ValueError(f"M * rank = {M * rank} exceeds the library's fixed scratch of "
                          f"{NOALLOC_MAX_U_ELEMS} values; use sdnq_int8_linear_lora with u_ws")
-    out = _rows_out(M, N, torch.bfloat16, qx.device) if out is None else out
     _check(lib().sdnq_int8_linear_lora_noalloc(_ptr(qx), _ptr(sx), _ptr(qW), _ptr(sW),
                                                _ptr(bias), _ptr(x), x.stride(0), _ptr(A),
                                                _ptr(B), rank, float(lora_scale), M, N, K,
@@ -443,6 +527,7 @@ def sdnq_gelu_bf16(x: torch.Tensor, out=None, stream=None):
     _req(x, torch.bfloat16, "x", 2)
     M, N = x.shape
     out = _rows_out(M, N, torch.bfloat16, x.device) if out is None else out
+    _mat(out, torch.bfloat16, M, N, "out")
     _check(lib().sdnq_gelu_bf16(_ptr(x), M, N, x.stride(0), _ptr(out), out.stride(0),
                                 _stream(stream)), "sdnq_gelu_bf16")
     return out

@@ -10,6 +10,7 @@
 
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include "sdnq.h"
 
@@ -21,6 +22,17 @@
 #include "rotquant.cuh"
 
 #define SDNQ_API extern "C" __attribute__((visibility("default")))
+
+// Every entry point that validates and launches work opens an NVTX range named after itself,
+// so that a profiler's timeline attributes kernels to the call that launched them. Without a
+// profiler attached the push and pop do nothing.
+struct NvtxRange {
+    explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange &) = delete;
+    NvtxRange &operator=(const NvtxRange &) = delete;
+};
+#define SDNQ_NVTX_RANGE() NvtxRange sdnq_nvtx_range_(__func__)
 
 namespace sdnq {
 namespace {
@@ -39,6 +51,7 @@ struct DeviceInfo {
     int checked = 0;
     int supported = 0;
     int sm_count = 0;
+    int index = 0;    // CUDA device ordinal
 };
 DeviceInfo g_dev[64];
 std::mutex g_dev_mutex;
@@ -62,6 +75,7 @@ sdnq_status current_device(DeviceInfo *out)
         }
         d.supported = (major == 10 && minor == 0) ? 1 : 0;
         d.sm_count = sms;
+        d.index = dev;
         d.checked = 1;
     }
     *out = d;
@@ -114,16 +128,39 @@ bool make_tmap_2d(CUtensorMap *map, CUtensorMapDataType dtype, const void *ptr, 
 inline bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 inline bool is_pow2(int64_t v) { return v > 0 && (v & (v - 1)) == 0; }
 
+// A value computed once per (device, key) and cached: kernel attributes and occupancy are
+// properties of a kernel on one device, so each device gets its own entry. Lookups and the
+// first computation hold a lock (host threads may call the library concurrently).
+template <int NKEYS>
+struct PerDeviceCache {
+    int value[64][NKEYS] = {};   // 0 = not computed yet
+    std::mutex mutex;
+    template <typename F>
+    int get(int dev, int key, F compute)
+    {
+        std::lock_guard<std::mutex> lock(mutex);
+        int &v = value[dev][key];
+        if (v == 0)
+            v = compute();
+        return v;
+    }
+};
+
+// Sets a kernel's dynamic shared-memory limit on the given (current) device, once per
+// device. Returns false if the runtime refused it.
+template <typename Kernel>
+bool smem_attr_once(PerDeviceCache<1> &cache, int dev, Kernel k, int bytes)
+{
+    return cache.get(dev, 0, [&] {
+               return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           bytes) == cudaSuccess ? 1 : -1;
+           }) == 1;
+}
+
 sdnq_status launch_status()
 {
     const cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? SDNQ_OK : SDNQ_ERR_CUDA;
-}
-
-template <typename Kernel>
-bool set_smem(Kernel k, int bytes)
-{
-    return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess;
 }
 
 // Programmatic launch (the kernel may start while the previous one in the stream drains; it
@@ -166,22 +203,25 @@ sdnq_status validate_rotquant(const void *x, int64_t rows, int64_t K, int64_t ld
 // Rows of at most 16 chunks go to the persistent, prefetching kernel (grid = resident
 // CTAs); longer rows to the two-pass kernel with one CTA per row.
 template <int G, bool COLSCALE = false, bool FP8 = false>
-void launch_rotquant_g(const RotquantParams &p, dim3 grid, dim3 block, int sm_count,
+void launch_rotquant_g(const RotquantParams &p, dim3 grid, dim3 block, const DeviceInfo &dev,
                        cudaStream_t st)
 {
     if (p.nchunks <= 16) {
-        static int per_sm[33] = {0};  // resident CTAs per SM, by warps per CTA
+        // resident CTAs per SM, by device and warps per CTA
+        static PerDeviceCache<33> per_sm;
         const int warps = static_cast<int>(block.x / 32);
-        if (per_sm[warps] == 0) {
+        const int n_sm = per_sm.get(dev.index, warps, [&] {
             int n = 0;
             if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(
                     &n, rotquant_persistent_kernel<G, COLSCALE, FP8>, block.x, 0) != cudaSuccess ||
-                n < 1)
+                n < 1) {
+                cudaGetLastError();
                 n = 1;
-            per_sm[warps] = n;
-        }
+            }
+            return n;
+        });
         const int64_t groups = grid.x;
-        const int64_t resident = static_cast<int64_t>(per_sm[warps]) * sm_count;
+        const int64_t resident = static_cast<int64_t>(n_sm) * dev.sm_count;
         const dim3 pgrid(static_cast<unsigned>(groups < resident ? groups : resident));
         rotquant_persistent_kernel<G, COLSCALE, FP8><<<pgrid, block, 0, st>>>(p);
     } else {
@@ -212,23 +252,23 @@ sdnq_status launch_rowquant(const uint16_t *x, int64_t rows, int64_t K, int64_t 
     cudaGetLastError();
     if (fp8) {
         switch (group) {
-        case 8: launch_rotquant_g<8, false, true>(p, grid, block, dev.sm_count, cs); break;
-        case 16: launch_rotquant_g<16, false, true>(p, grid, block, dev.sm_count, cs); break;
-        case 32: launch_rotquant_g<32, false, true>(p, grid, block, dev.sm_count, cs); break;
-        case 64: launch_rotquant_g<64, false, true>(p, grid, block, dev.sm_count, cs); break;
-        case 128: launch_rotquant_g<128, false, true>(p, grid, block, dev.sm_count, cs); break;
-        default: launch_rotquant_g<256, false, true>(p, grid, block, dev.sm_count, cs); break;
+        case 8: launch_rotquant_g<8, false, true>(p, grid, block, dev, cs); break;
+        case 16: launch_rotquant_g<16, false, true>(p, grid, block, dev, cs); break;
+        case 32: launch_rotquant_g<32, false, true>(p, grid, block, dev, cs); break;
+        case 64: launch_rotquant_g<64, false, true>(p, grid, block, dev, cs); break;
+        case 128: launch_rotquant_g<128, false, true>(p, grid, block, dev, cs); break;
+        default: launch_rotquant_g<256, false, true>(p, grid, block, dev, cs); break;
         }
         return launch_status();
     }
     switch (group) {
-    case 1: launch_rotquant_g<1, true>(p, grid, block, dev.sm_count, cs); break;
-    case 8: launch_rotquant_g<8>(p, grid, block, dev.sm_count, cs); break;
-    case 16: launch_rotquant_g<16>(p, grid, block, dev.sm_count, cs); break;
-    case 32: launch_rotquant_g<32>(p, grid, block, dev.sm_count, cs); break;
-    case 64: launch_rotquant_g<64>(p, grid, block, dev.sm_count, cs); break;
-    case 128: launch_rotquant_g<128>(p, grid, block, dev.sm_count, cs); break;
-    default: launch_rotquant_g<256>(p, grid, block, dev.sm_count, cs); break;
+    case 1: launch_rotquant_g<1, true>(p, grid, block, dev, cs); break;
+    case 8: launch_rotquant_g<8>(p, grid, block, dev, cs); break;
+    case 16: launch_rotquant_g<16>(p, grid, block, dev, cs); break;
+    case 32: launch_rotquant_g<32>(p, grid, block, dev, cs); break;
+    case 64: launch_rotquant_g<64>(p, grid, block, dev, cs); break;
+    case 128: launch_rotquant_g<128>(p, grid, block, dev, cs); break;
+    default: launch_rotquant_g<256>(p, grid, block, dev, cs); break;
     }
     return launch_status();
 }
@@ -294,10 +334,8 @@ sdnq_status launch_gemm(const DeviceInfo &dev, const int8_t *qx, const int8_t *q
         tmU = tmA;
         tmL = tmA;
     }
-    static std::once_flag once;
-    static bool smem_ok = false;
-    std::call_once(once, [] { smem_ok = set_smem(kernel, C::SMEM_BYTES); });
-    if (!smem_ok)
+    static PerDeviceCache<1> smem_attr;
+    if (!smem_attr_once(smem_attr, dev.index, kernel, C::SMEM_BYTES))
         return SDNQ_ERR_CUDA;
     p.num_kb = (p.K + C::BK - 1) / C::BK;
     p.num_m_blocks = (p.M + C::BM - 1) / C::BM;
@@ -342,18 +380,17 @@ sdnq_status launch_gemm(const DeviceInfo &dev, const int8_t *qx, const int8_t *q
 }
 
 template <int RANK_PAD>
-sdnq_status launch_lora_down(const uint16_t *x, int64_t ldx, const uint16_t *A, int32_t rank,
-                             uint16_t *u, int32_t M, int32_t K, cudaStream_t cs)
+sdnq_status launch_lora_down(const DeviceInfo &dev, const uint16_t *x, int64_t ldx,
+                             const uint16_t *A, int32_t rank, uint16_t *u, int32_t M, int32_t K,
+                             cudaStream_t cs)
 {
     using C = LoraDownConfig<RANK_PAD>;
     CUtensorMap tmX, tmA;
     if (!make_tmap_2d(&tmX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, K, M, 2ull * ldx, 64, 128) ||
         !make_tmap_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, A, rank, K, 2ull * rank, 64, 64))
         return SDNQ_ERR_CUDA;
-    static std::once_flag once;
-    static bool smem_ok = false;
-    std::call_once(once, [] { smem_ok = set_smem(lora_down_kernel<RANK_PAD>, C::SMEM_BYTES); });
-    if (!smem_ok)
+    static PerDeviceCache<1> smem_attr;
+    if (!smem_attr_once(smem_attr, dev.index, lora_down_kernel<RANK_PAD>, C::SMEM_BYTES))
         return SDNQ_ERR_CUDA;
     LoraDownParams p;
     p.u = u;
@@ -414,11 +451,11 @@ sdnq_status run_linear(const int8_t *qx, const float *sx, const int8_t *qW, cons
                     : launch_gemm<256, false>(dev, qx, qW, nullptr, nullptr, 0, p, cs);
     const int32_t Mi = static_cast<int32_t>(M), Ki = static_cast<int32_t>(K);
     if (rank <= 64)
-        st = launch_lora_down<64>(x, ldx, A, rank, u_ws, Mi, Ki, cs);
+        st = launch_lora_down<64>(dev, x, ldx, A, rank, u_ws, Mi, Ki, cs);
     else if (rank <= 128)
-        st = launch_lora_down<128>(x, ldx, A, rank, u_ws, Mi, Ki, cs);
+        st = launch_lora_down<128>(dev, x, ldx, A, rank, u_ws, Mi, Ki, cs);
     else
-        st = launch_lora_down<256>(x, ldx, A, rank, u_ws, Mi, Ki, cs);
+        st = launch_lora_down<256>(dev, x, ldx, A, rank, u_ws, Mi, Ki, cs);
     if (st != SDNQ_OK)
         return st;
     p.lora_chunks = (rank + 63) / 64;
@@ -429,6 +466,22 @@ sdnq_status run_linear(const int8_t *qx, const float *sx, const int8_t *qW, cons
 
 // the quantizer warps hold at most this many 1024-element chunks of a row
 constexpr int kFusedMaxChunks = SDNQ_FUSED_QUANT_WARPS;
+
+// Whether sdnq_int8_linear_fused takes one launch. The one-launch kernel overlaps the
+// quantizer with the GEMM. It pays off once the GEMM has at least three waves of tiles (with
+// fewer, its first wave needs most rows before it can start) and the quantizer is a small
+// share of the work (N >= 3584, or K >= 6144); otherwise the two launches, the GEMM's
+// prologue overlapping the quantizer's tail, are faster (measured on 14 shapes from
+// 4096 x 3072 x 3072 to 16384 x 6144 x 8192). Rows longer than the quantizer warps can hold
+// take the two launches.
+bool fused_one_launch(const DeviceInfo &dev, int64_t M, int64_t N, int64_t K, int32_t policy)
+{
+    const int64_t nchunks = (K + 1023) / 1024;
+    const int64_t tiles = ((M + 127) / 128) * ((N + 255) / 256);
+    const bool auto_one = tiles >= 3ll * dev.sm_count && (N >= 3584 || K >= 6144);
+    return nchunks <= kFusedMaxChunks &&
+           (policy == SDNQ_FUSE_ALWAYS || (policy == SDNQ_FUSE_AUTO && auto_one));
+}
 
 template <int G>
 sdnq_status launch_linear_fused_g(const DeviceInfo &dev, GemmParams p, const int8_t *qW,
@@ -461,16 +514,7 @@ sdnq_status run_linear_fused(const uint16_t *x, int64_t ldx, int32_t group, cons
         return SDNQ_OK;
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     const int32_t nchunks = static_cast<int32_t>((K + 1023) / 1024);
-    // The one-launch kernel overlaps the quantizer with the GEMM. It pays off once the GEMM
-    // has at least three waves of tiles (with fewer, its first wave needs most rows before it
-    // can start) and the quantizer is a small share of the work (N >= 3584, or K >= 6144);
-    // otherwise the two launches, the GEMM's prologue overlapping the quantizer's tail, are
-    // faster (measured on 14 shapes from 4096 x 3072 x 3072 to 16384 x 6144 x 8192). Rows
-    // longer than the quantizer warps can hold take the two launches.
-    const int64_t tiles = ((M + 127) / 128) * ((N + 255) / 256);
-    const bool auto_one = tiles >= 3ll * dev.sm_count && (N >= 3584 || K >= 6144);
-    const bool fuse = nchunks <= kFusedMaxChunks &&
-                      (policy == SDNQ_FUSE_ALWAYS || (policy == SDNQ_FUSE_AUTO && auto_one));
+    const bool fuse = fused_one_launch(dev, M, N, K, policy);
     if (!fuse) {
         // the two launches (same results)
         if ((st = launch_rowquant(x, M, K, ldx, group, nullptr, qx_ws, sx_ws, dev, cs)) != SDNQ_OK)
@@ -795,9 +839,9 @@ sdnq_status launch_attention_prep(const uint16_t *q, const uint16_t *k, int64_t 
 }
 
 // the attention kernel on prepared codes
-sdnq_status launch_attention_core(const uint16_t *v, int64_t B, int64_t Lq, int64_t Lk, int64_t H,
-                                  int64_t D, float scale, uint8_t *w, const int64_t *off,
-                                  uint16_t *o, cudaStream_t cs)
+sdnq_status launch_attention_core(const DeviceInfo &dev, const uint16_t *v, int64_t B, int64_t Lq,
+                                  int64_t Lk, int64_t H, int64_t D, float scale, uint8_t *w,
+                                  const int64_t *off, uint16_t *o, cudaStream_t cs)
 {
     CUtensorMap tmQ, tmK, tmV;
     const uint64_t row = static_cast<uint64_t>(H * D);
@@ -808,10 +852,8 @@ sdnq_status launch_attention_core(const uint16_t *v, int64_t B, int64_t Lq, int6
         !make_tmap_3d(&tmV, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, v, row, Lk, B, 2 * row, 2 * row * Lk,
                       64, 128))
         return SDNQ_ERR_CUDA;
-    static std::once_flag once;
-    static bool smem_ok = false;
-    std::call_once(once, [] { smem_ok = set_smem(attn_kernel, AttnConfig::SMEM_BYTES); });
-    if (!smem_ok)
+    static PerDeviceCache<1> smem_attr;
+    if (!smem_attr_once(smem_attr, dev.index, attn_kernel, AttnConfig::SMEM_BYTES))
         return SDNQ_ERR_CUDA;
     AttnParams p = {};
     p.sq = reinterpret_cast<const float *>(w + off[2]);
@@ -867,7 +909,7 @@ sdnq_status run_attention(const uint16_t *q, const uint16_t *k, const uint16_t *
         (st = launch_attention_prep(q, k, B, Lq, Lk, H, D, group, smooth_k, w, off, dev, cs)) != SDNQ_OK)
         return st;
     if (which & 2)
-        return launch_attention_core(v, B, Lq, Lk, H, D, scale, w, off, o, cs);
+        return launch_attention_core(dev, v, B, Lq, Lk, H, D, scale, w, off, o, cs);
     return SDNQ_OK;
 }
 
@@ -895,12 +937,14 @@ using namespace sdnq;
 SDNQ_API sdnq_status sdnq_rotate_quant_weight(const uint16_t *W, int64_t N, int64_t K, int64_t ldw,
                                               int32_t group, int8_t *qW, float *sW, void *stream)
 {
+    SDNQ_NVTX_RANGE();
     return run_rotquant(W, N, K, ldw, group, qW, sW, stream);
 }
 
 SDNQ_API sdnq_status sdnq_rotquant_act(const uint16_t *x, int64_t M, int64_t K, int64_t ldx,
                                        int32_t group, int8_t *qx, float *sx, void *stream)
 {
+    SDNQ_NVTX_RANGE();
     return run_rotquant(x, M, K, ldx, group, qx, sx, stream);
 }
 
@@ -909,6 +953,7 @@ SDNQ_API sdnq_status sdnq_int8_linear(const int8_t *qx, const float *sx, const i
                                       int64_t K, uint16_t *out, int64_t ldo, int32_t *acc_out,
                                       void *stream)
 {
+    SDNQ_NVTX_RANGE();
     return run_linear(qx, sx, qW, sW, bias, nullptr, 0, nullptr, nullptr, 0, 0.0f, nullptr, M, N, K,
                       out, ldo, acc_out, stream, false);
 }
@@ -920,6 +965,7 @@ SDNQ_API sdnq_status sdnq_int8_linear_fused(const uint16_t *x, int64_t ldx, int3
                                             uint16_t *out, int64_t ldo, int32_t *acc_out,
                                             int32_t policy, void *stream)
 {
+    SDNQ_NVTX_RANGE();
     return run_linear_fused(x, ldx, group, qW, sW, bias, M, N, K, qx_ws, sx_ws, sync_ws, out, ldo,
                             acc_out, policy, stream);
 }
@@ -927,6 +973,7 @@ SDNQ_API sdnq_status sdnq_int8_linear_fused(const uint16_t *x, int64_t ldx, int3
 SDNQ_API sdnq_status sdnq_rotquant_fp8(const uint16_t *x, int64_t M, int64_t K, int64_t ldx,
                                        int32_t group, uint8_t *q, float *s, void *stream)
 {
+    SDNQ_NVTX_RANGE();
     return run_rotquant_fp8(x, M, K, ldx, group, q, s, stream);
 }
 
@@ -935,6 +982,7 @@ SDNQ_API sdnq_status sdnq_fp8_linear(const uint8_t *qx, const float *sx, const u
                                      int64_t K, uint16_t *out, int64_t ldo, float *acc_out,
                                      void *stream)
 {
+    SDNQ_NVTX_RANGE();
     return run_fp8_linear(qx, sx, qW, sW, bias, M, N, K, out, ldo, acc_out, stream);
 }
 
@@ -951,6 +999,7 @@ SDNQ_API sdnq_status sdnq_attention_int8qk(const uint16_t *q, const uint16_t *k,
                                            int32_t group, float scale, int32_t smooth_k, void *ws,
                                            int64_t ws_bytes, uint16_t *o, void *stream)
 {
+    SDNQ_NVTX_RANGE();
     return run_attention(q, k, v, B, Lq, Lk, H, D, group, scale, smooth_k, ws, ws_bytes, o, stream, 3);
 }
 
@@ -959,6 +1008,7 @@ SDNQ_API sdnq_status sdnq_attention_prep(const uint16_t *q, const uint16_t *k, i
                                          int32_t group, int32_t smooth_k, void *ws,
                                          int64_t ws_bytes, void *stream)
 {
+    SDNQ_NVTX_RANGE();
     // v and o are not touched by the preparation: the workspace stands in for them
     return run_attention(q, k, static_cast<const uint16_t *>(ws), B, Lq, Lk, H, D, group, 1.0f,
                          smooth_k, ws, ws_bytes, static_cast<uint16_t *>(ws), stream, 1);
@@ -968,6 +1018,7 @@ SDNQ_API sdnq_status sdnq_attention_core(const uint16_t *v, int64_t B, int64_t L
                                          int64_t H, int64_t D, float scale, void *ws,
                                          int64_t ws_bytes, uint16_t *o, void *stream)
 {
+    SDNQ_NVTX_RANGE();
     // q and k are not read by the attention kernel (their codes are in ws)
     return run_attention(static_cast<const uint16_t *>(ws), static_cast<const uint16_t *>(ws), v,
                          B, Lq, Lk, H, D, SDNQ_MAX_GROUP, scale, 0, ws, ws_bytes, o, stream, 2);
@@ -978,6 +1029,7 @@ SDNQ_API sdnq_status sdnq_int8_linear_gelu(const int8_t *qx, const float *sx, co
                                            int64_t N, int64_t K, uint16_t *out, int64_t ldo,
                                            int32_t *acc_out, void *stream)
 {
+    SDNQ_NVTX_RANGE();
     return run_linear(qx, sx, qW, sW, bias, nullptr, 0, nullptr, nullptr, 0, 0.0f, nullptr, M, N, K,
                       out, ldo, acc_out, stream, false, true);
 }
@@ -988,6 +1040,7 @@ SDNQ_API sdnq_status sdnq_int8_linear_grad_input(const uint16_t *dy, int64_t ldd
                                                  int8_t *qg_ws, float *sg_ws, uint16_t *dx,
                                                  int64_t lddx, int32_t *acc_out, void *stream)
 {
+    SDNQ_NVTX_RANGE();
     return run_grad_input(dy, lddy, qW, sW, M, N, K, group, qg_ws, sg_ws, dx, lddx, acc_out,
                           stream);
 }
@@ -996,6 +1049,7 @@ SDNQ_API sdnq_status sdnq_quant_grad_output(const uint16_t *dy, int64_t lddy, co
                                             int64_t M, int64_t N, int8_t *qg, float *sg,
                                             void *stream)
 {
+    SDNQ_NVTX_RANGE();
     return run_grad_quant(dy, lddy, sW, M, N, qg, sg, stream);
 }
 
@@ -1004,6 +1058,7 @@ SDNQ_API sdnq_status sdnq_int8_grad_input_gemm(const int8_t *qg, const float *sg
                                                uint16_t *dx, int64_t lddx, int32_t *acc_out,
                                                void *stream)
 {
+    SDNQ_NVTX_RANGE();
     return run_grad_gemm(qg, sg, qW, M, N, K, group, dx, lddx, acc_out, stream);
 }
 
@@ -1014,6 +1069,7 @@ SDNQ_API sdnq_status sdnq_int8_linear_lora(const int8_t *qx, const float *sx, co
                                            int64_t M, int64_t N, int64_t K, uint16_t *out,
                                            int64_t ldo, int32_t *acc_out, void *stream)
 {
+    SDNQ_NVTX_RANGE();
     return run_linear(qx, sx, qW, sW, bias, x, ldx, A, B, rank, lora_scale, u_ws, M, N, K, out, ldo,
                       acc_out, stream, true);
 }
@@ -1021,6 +1077,7 @@ SDNQ_API sdnq_status sdnq_int8_linear_lora(const int8_t *qx, const float *sx, co
 SDNQ_API sdnq_status sdnq_gelu_bf16(const uint16_t *in, int64_t M, int64_t N, int64_t ld_in,
                                     uint16_t *out, int64_t ld_out, void *stream)
 {
+    SDNQ_NVTX_RANGE();
     if (M != 0 && (!in || !out))
         return SDNQ_ERR_NULL;
     if (M < 0 || N <= 0 || ld_in < N || ld_out < N)
@@ -1055,6 +1112,7 @@ SDNQ_API sdnq_status sdnq_gelu_bf16(const uint16_t *in, int64_t M, int64_t N, in
 
 SDNQ_API sdnq_status sdnq_device_status(void *stream)
 {
+    SDNQ_NVTX_RANGE();
     if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) {
         cudaGetLastError();
         return SDNQ_ERR_CUDA;
@@ -1073,6 +1131,7 @@ SDNQ_API sdnq_status sdnq_device_status(void *stream)
 
 SDNQ_API sdnq_status sdnq_selftest_wait_timeout(int64_t limit_ns, void *stream)
 {
+    SDNQ_NVTX_RANGE();
     if (limit_ns < 1000 || limit_ns > 10000000000ll)
         return SDNQ_ERR_SHAPE;
     DeviceInfo dev;
@@ -1083,6 +1142,23 @@ SDNQ_API sdnq_status sdnq_selftest_wait_timeout(int64_t limit_ns, void *stream)
     wait_timeout_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
         static_cast<uint64_t>(limit_ns));
     return launch_status();
+}
+
+SDNQ_API sdnq_status sdnq_int8_linear_fused_plan(int64_t M, int64_t N, int64_t K,
+                                                 int32_t policy, int32_t *one_launch)
+{
+    if (!one_launch)
+        return SDNQ_ERR_NULL;
+    if (M < 0 || N < 1 || N > INT32_MAX || K < 16 || K % 16 != 0 || K > SDNQ_MAX_K)
+        return SDNQ_ERR_SHAPE;
+    if (policy < SDNQ_FUSE_AUTO || policy > SDNQ_FUSE_NEVER)
+        return SDNQ_ERR_UNSUPPORTED;
+    DeviceInfo dev;
+    const sdnq_status st = current_device(&dev);
+    if (st != SDNQ_OK)
+        return st;
+    *one_launch = fused_one_launch(dev, M, N, K, policy) ? 1 : 0;
+    return SDNQ_OK;
 }
 
 SDNQ_API const char *sdnq_status_string(sdnq_status s)

@@ -58,10 +58,13 @@ SDNQ_API sdnq_status sdnq_int8_linear_lora_noalloc(const int8_t *qx, const float
                                                    int64_t K, uint16_t *out, int64_t ldo,
                                                    int32_t *acc_out, void *stream)
 {
+    SDNQ_NVTX_RANGE();
     if (M < 0 || rank < 0)
         return SDNQ_ERR_SHAPE;
-    if (M * static_cast<int64_t>(rank) > SDNQ_NOALLOC_MAX_U_ELEMS)
-        return SDNQ_ERR_SHAPE;  // u would not fit the library's fixed scratch array
+    // u would not fit the library's fixed scratch array (the division keeps the check free
+    // of overflow for any M)
+    if (rank > 0 && M > SDNQ_NOALLOC_MAX_U_ELEMS / rank)
+        return SDNQ_ERR_SHAPE;
     DeviceInfo dev;
     sdnq_status st = current_device(&dev);
     if (st != SDNQ_OK)

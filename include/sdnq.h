@@ -147,6 +147,17 @@ sdnq_status sdnq_int8_linear_fused(const uint16_t *x, int64_t ldx, int32_t group
                                    int32_t *acc_out, int32_t policy, void *stream);
 
 /*
+ * The path sdnq_int8_linear_fused takes for these sizes and this policy on the current
+ * device: *one_launch = 1 for the single kernel, 0 for the two launches (same results either
+ * way). Nothing is launched and no pointer but one_launch is read, so a caller can label or
+ * plan the path without restating the rule above.
+ *   Errors: SDNQ_ERR_NULL (one_launch NULL), SDNQ_ERR_SHAPE (M < 0, N < 1, K < 16, K % 16,
+ *   K > SDNQ_MAX_K), SDNQ_ERR_UNSUPPORTED (unknown policy or not an sm_100 device).
+ */
+sdnq_status sdnq_int8_linear_fused_plan(int64_t M, int64_t N, int64_t K, int32_t policy,
+                                        int32_t *one_launch);
+
+/*
  * sdnq_int8_linear with GELU fused into its epilogue, for the up-projection of a DiT MLP
  * whose output feeds the down-projection's rotate + quantize:
  *   out = gelu(bf16(float(acc) * (sx * sw) [+ bias])), GELU(y) = y * Phi(y) in the exact

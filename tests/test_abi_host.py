@@ -166,6 +166,22 @@ def test_fused_validation(lib):
     assert fused(lib, policy=3) == _native.SDNQ_ERR_UNSUPPORTED
 
 
+def test_fused_plan_validation(lib):
+    import ctypes
+    one = ctypes.c_int32(7)
+    ref = ctypes.byref(one)
+    assert lib.sdnq_int8_linear_fused_plan(4096, 3072, 3072, 0, None) == _native.SDNQ_ERR_NULL
+    assert lib.sdnq_int8_linear_fused_plan(-1, 3072, 3072, 0, ref) == _native.SDNQ_ERR_SHAPE
+    assert lib.sdnq_int8_linear_fused_plan(4096, 0, 3072, 0, ref) == _native.SDNQ_ERR_SHAPE
+    assert lib.sdnq_int8_linear_fused_plan(4096, 3072, 3000, 0, ref) == _native.SDNQ_ERR_SHAPE
+    assert lib.sdnq_int8_linear_fused_plan(4096, 3072, 3072, 5, ref) == \
+        _native.SDNQ_ERR_UNSUPPORTED
+    assert one.value == 7   # nothing written on an error
+    if not torch.cuda.is_available():
+        assert lib.sdnq_int8_linear_fused_plan(4096, 3072, 3072, 0, ref) == \
+            _native.SDNQ_ERR_UNSUPPORTED
+
+
 def test_gelu_and_selftest_validation(lib):
     assert lib.sdnq_gelu_bf16(0, 4, 8, 8, A16, 8, S) == _native.SDNQ_ERR_NULL
     assert lib.sdnq_gelu_bf16(A16, 4, 0, 8, A16, 8, S) == _native.SDNQ_ERR_SHAPE

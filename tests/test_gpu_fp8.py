@@ -88,11 +88,3 @@ def test_fp8_zero_and_extreme_rows():
     got = run_fp8(case)
     assert got["sx"][4] == 0 and np.all(got["qx"][4] == 0)
     check_against_oracle(case, got)
-
-
-def test_fp8_full_size_sampled_rows():
-    case = synthetic.workload("dit_attn_4096x3072x3072")
-    got = run_fp8(case)
-    rng = np.random.default_rng(8)
-    rows = np.unique(np.concatenate([[0, case.M - 1], rng.choice(case.M, 14, replace=False)]))
-    check_against_oracle(case, got, rows)

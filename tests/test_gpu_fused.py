@@ -2,8 +2,9 @@
 quantize runs on warps inside the int8 GEMM kernel) against the oracle: bit-exact activation
 codes, scales, int32 accumulators and bf16 outputs on ragged shapes, every group size, with
 and without bias, rows longer than the fused limit (two launches), repeated calls on one
-counter buffer, and the full-size workloads in the launch configuration the benchmark times
-(sampled rows). Every input is seeded; every expected value comes from the oracle."""
+counter buffer. The full-size workloads are compared on every element in
+tests/test_gpu_fullsize.py. Every input is seeded; every expected value comes from the
+oracle."""
 import numpy as np
 import pytest
 import torch
@@ -113,18 +114,3 @@ def test_fused_equals_two_launches_on_zero_and_huge_rows():
     assert got["sx"][7] == 0
     assert_equal(got["qx"], qx.cpu().numpy(), "codes against the two-launch path")
     assert_equal(got["out"], bits_of(two), "outputs against the two-launch path")
-
-
-@pytest.mark.parametrize("name", ["dit_attn_4096x3072x3072", "quarot_16384x4096x4096",
-                                  "peft_lora_8192x12288x3072_r64"])
-def test_fused_full_size_sampled_rows(name):
-    case = synthetic.workload(name)
-    case.A = case.B = None  # the base layer (the adapter path is not fused)
-    got = run_fused(case)
-    rng = np.random.default_rng(len(name))
-    rows = np.unique(np.concatenate([[0, case.M - 1], rng.choice(case.M, 14, replace=False)]))
-    ref = oracle_ref(case, rows)
-    assert_equal(got["qx"][rows], ref["qx"], "codes (sampled rows)")
-    assert_equal(got["sx"][rows].view(np.uint32), ref["sx"].view(np.uint32), "scales")
-    assert_equal(got["acc"][rows], ref["acc"], "accumulators (sampled rows)")
-    assert_equal(got["out"][rows], ref["out"], "outputs (sampled rows)")

@@ -2,8 +2,9 @@
 (sdnq_int8_linear_grad_input) against the oracle's three steps: bit-exact int8 codes of
 dy * sW, fp32 scales, int32 accumulators and bf16 dx, on ragged shapes (M, the contraction N
 and the output width K not multiples of the tiles), every group size, strided dy, zero rows,
-and at the full size of the attention and PEFT layers on sampled rows. Every input is seeded;
-every expected value comes from the oracle."""
+and the split calls against the composed one (the full-size attention and PEFT layers are
+compared on every element in tests/test_gpu_fullsize.py). Every input is seeded; every
+expected value comes from the oracle."""
 import numpy as np
 import pytest
 import torch
@@ -89,24 +90,6 @@ def test_grad_input_empty_batch_is_a_noop():
     dx = sd.sdnq_int8_linear_grad_input(torch.zeros(0, 64, dtype=torch.bfloat16, device="cuda"),
                                         qW, sW, 256)
     assert dx.shape == (0, 256)
-
-
-@pytest.mark.parametrize("name", sorted(synthetic.GRAD_WORKLOADS))
-def test_grad_input_full_size_sampled_rows(name):
-    """The attention projection and the PEFT feed-forward layer at full size, in the launch
-    configuration of a real call: codes, scales, accumulators and dx on sampled rows (every
-    column)."""
-    case = synthetic.workload(name)
-    M, N, g = case.M, case.N, case.g
-    dy, W = case.x, case.W
-    got = run_gpu(dy, W, g, N)
-    rng = np.random.default_rng(M + N)
-    rows = np.unique(np.concatenate([[0, M - 1], rng.choice(M, 14, replace=False)]))
-    ref = oracle_ref(dy, W, g, N, rows=rows)
-    assert_equal(got["qg"][rows], ref["qg"], "codes (sampled rows)")
-    assert_equal(got["sg"][rows].view(np.uint32), ref["sg"].view(np.uint32), "scales")
-    assert_equal(got["acc"][rows], ref["acc"], "accumulators (sampled rows)")
-    assert_equal(got["dx"][rows], ref["dx"], "dx (sampled rows)")
 
 
 def test_split_calls_equal_the_composed_call():

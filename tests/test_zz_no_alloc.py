@@ -1,12 +1,13 @@
-"""The no-allocation LoRA entry point, checked against the regular one.
+"""The no-allocation LoRA entry point, checked against the regular one and the oracle.
 
 Some callers cannot hand the library a workspace: their framework owns all device memory
 (a caching allocator or a fixed memory plan) and does not permit allocations from outside
 it, or a cudaMalloc, with its possible device synchronisation and unpredictable latency, is
 not acceptable where they run. sdnq_int8_linear_lora_noalloc serves them by keeping the
 LoRA intermediate u in a fixed array inside the library. Here it is called through the C ABI
-twice in a row, on two different problems, and each result is compared with
-sdnq_int8_linear_lora given a caller-allocated u_ws.
+twice in a row, on two different problems, and each result must be bit for bit that of
+sdnq_int8_linear_lora given a caller-allocated u_ws (both run the same kernels on the same
+inputs), and within one bf16 ulp of the CPU oracle. The Python wrapper is exercised too.
 
 This file is collected last so that a run stopping at its first failure has run every
 other test; it also passes on its own in a fresh process.
@@ -17,6 +18,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 import hadamard_rotated_int8_b200 as sd
 from hadamard_rotated_int8_b200 import _build, _native, synthetic
 
@@ -43,8 +45,9 @@ def _prepared(M, N, K, rank, seed):
     x = case.x.cuda()
     qW, sW = sd.sdnq_rotate_quant_weight(case.W.cuda(), 256)
     qx, sx = sd.sdnq_rotquant_act(x, 256)
-    return dict(x=x, qx=qx, sx=sx, qW=qW, sW=sW, bias=case.bias.cuda(), A=case.A.cuda(),
-                B=case.B.cuda(), scale=case.lora_scale, M=M, N=N, K=K, rank=rank)
+    return dict(case=case, x=x, qx=qx, sx=sx, qW=qW, sW=sW, bias=case.bias.cuda(),
+                A=case.A.cuda(), B=case.B.cuda(), scale=case.lora_scale, M=M, N=N, K=K,
+                rank=rank)
 
 
 def _noalloc_via_cabi(p):
@@ -66,20 +69,47 @@ def _with_workspace(p):
                                     p["A"], p["B"], p["scale"], u_ws=u)
 
 
+def _oracle_out(p):
+    c = p["case"]
+    ref = oracle.linear(synthetic.bits(c.x), *oracle.rotate_quantize(synthetic.bits(c.W), 256),
+                        256, bias_bits=synthetic.bits(c.bias), A_bits=synthetic.bits(c.A),
+                        B_bits=synthetic.bits(c.B), lora_scale=c.lora_scale)
+    return ref["out"]
+
+
 def test_noalloc_matches_workspace_entry_point_twice():
     _build.build()
+    oracle.build()
     first = _prepared(M=300, N=264, K=512, rank=64, seed=31)
     second = _prepared(M=1024, N=520, K=1024, rank=32, seed=32)
-    # two calls in a row on the shared scratch array, then the reference calls
+    # two calls in a row on the shared scratch array, then the workspace calls
     got1 = _noalloc_via_cabi(first)
     got2 = _noalloc_via_cabi(second)
     want1 = _with_workspace(first)
     want2 = _with_workspace(second)
     torch.cuda.synchronize()
     assert sd.sdnq_device_status() == 0
-    for got, want in ((got1, want1), (got2, want2)):
-        d = _ulp_diff(_bits(got), _bits(want))
-        assert d.max() <= 1, f"no-alloc output differs by {d.max()} ulp"
+    for p, got, want in ((first, got1, want1), (second, got2, want2)):
+        g, w = _bits(got), _bits(want)
+        assert np.array_equal(g, w), \
+            f"no-alloc output differs from the workspace call in {np.count_nonzero(g != w)} places"
+        assert _ulp_diff(g, _oracle_out(p)).max() <= 1, "no-alloc output vs the oracle"
+
+
+def test_noalloc_python_wrapper_after_a_larger_call():
+    """The wrapper on a small problem right after a larger one left the shared array full of
+    other rows: its rows of u are rewritten before they are read."""
+    _build.build()
+    big = _prepared(M=2048, N=256, K=512, rank=128, seed=33)
+    small = _prepared(M=130, N=136, K=256, rank=16, seed=34)
+    _noalloc_via_cabi(big)
+    got = sd._native.sdnq_int8_linear_lora_noalloc(small["qx"], small["sx"], small["qW"],
+                                                   small["sW"], small["bias"], small["x"],
+                                                   small["A"], small["B"], small["scale"])
+    want = _with_workspace(small)
+    torch.cuda.synchronize()
+    assert sd.sdnq_device_status() == 0
+    assert np.array_equal(_bits(got), _bits(want))
 
 
 def test_noalloc_rejects_problems_larger_than_its_scratch():
@@ -88,5 +118,10 @@ def test_noalloc_rejects_problems_larger_than_its_scratch():
     M = _native.NOALLOC_MAX_U_ELEMS // rank + 1
     st = _native.lib().sdnq_int8_linear_lora_noalloc(
         P(0), P(0), P(0), P(0), P(0), P(0), 256, P(0), P(0), rank, 1.0, M, 256, 256, P(0),
+        256, P(0), P(0))
+    assert st == _native.SDNQ_ERR_SHAPE
+    # a row count whose product with the rank overflows 64 bits is refused the same way
+    st = _native.lib().sdnq_int8_linear_lora_noalloc(
+        P(0), P(0), P(0), P(0), P(0), P(0), 256, P(0), P(0), rank, 1.0, 2 ** 62, 256, 256, P(0),
         256, P(0), P(0))
     assert st == _native.SDNQ_ERR_SHAPE
