@@ -56,7 +56,7 @@ def measured_peaks():
 # The sources each profiled kernel is compiled from (its own header and the shared PTX
 # helpers): an ncu summary stays valid until one of these changes.
 KERNEL_SOURCES = {
-    "gemm_s8": ("device.cuh", "gemm.cuh", "gelu.cuh", "rotquant.cuh"),
+    "gemm_s8": ("device.cuh", "gemm.cuh", "gemm_pair.cuh", "gelu.cuh", "rotquant.cuh"),
     "lora_down": ("device.cuh", "lora_down.cuh"),
     "rotquant": ("device.cuh", "rotquant.cuh"),
     "attn_kernel": ("device.cuh", "rotquant.cuh", "attention.cuh"),

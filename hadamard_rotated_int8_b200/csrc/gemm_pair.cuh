@@ -1,0 +1,358 @@
+// The int8 (or e4m3) linear on CTA pairs: one tcgen05 MMA spans the tensor cores of two SMs
+// (cta_group::2). A pair computes a 256 x 256 output tile: each CTA loads its own 128 rows
+// of the activation codes and its own 128 rows of the weight codes (the tile's columns are
+// split between the CTAs), so every SM streams 32 KB of operands per 128-byte K step where a
+// single-SM 128 x 256 tile streams 48 KB, for the same tensor-core work per SM. Each CTA's
+// tensor memory receives its 128 rows of the int32 (fp32 for e4m3) accumulators, and its own
+// epilogue warps apply the same fp32 de-quant epilogue (and the GELU table) as the single-SM
+// kernel, so outputs are bit for bit the same.
+//
+// Sources: as the single-SM kernel ("SDNQ: SD.Next Quantization Engine" README, INT8
+// quantized matmul and dequantize_fp32; "ConvRot / Hadamard SDNQ").
+//
+// Roles (320 threads per CTA):
+//   warp 0      TMA producer of this CTA's halves; its loads complete on this CTA's own
+//               full barrier, so a CTA can always wait for its own copies in flight.
+//   warp 1      rank 0: allocates tensor memory (both CTAs allocate the same columns) and
+//               issues the pair's MMAs once its own stage and the peer's are full.
+//               rank 1: forwards each of its completed stages to rank 0 (a remote arrive
+//               on rank 0's peer-full barrier).
+//   warps 2..9  epilogue of this CTA's 128 rows; they release the accumulator buffer with a
+//               remote arrive on rank 0's tensor-empty barrier (16 arrivals per use).
+// The MMA completion (tcgen05.commit, multicast to both CTAs) frees each stage in both CTAs
+// and announces each finished accumulator buffer to both epilogues. Every wait is bounded.
+#pragma once
+
+#include "gemm.cuh"
+
+namespace sdnq {
+
+template <bool GELU>
+struct PairConfig {
+    static constexpr int BM = 128;                       // rows per CTA (256 per pair)
+    static constexpr int BN = 256;                       // columns per pair tile
+    static constexpr int BK = 128;                       // bytes of K per stage
+    static constexpr int A_BYTES = BM * BK;              // 16 KB
+    static constexpr int B_BYTES = (BN / 2) * BK;        // this CTA's 128 columns: 16 KB
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    static constexpr int ACC_COLS = BN;                  // int32 / fp32 columns per buffer
+    static constexpr int NBUF = 2;
+    static constexpr int TMEM_COLS = NBUF * ACC_COLS;    // 512
+    static constexpr int THREADS = 320;
+    static constexpr int EPI_WARPS = 8;
+    static constexpr int EPI_COLS = BN / 2;
+    static constexpr int STAGE_OUT_BYTES = 32 * 64;
+    static constexpr int LUT_BYTES = GELU ? kGeluLutBytes : 0;
+    static constexpr int SCALE_BYTES = EPI_COLS * 8;
+    static constexpr int FIXED = EPI_WARPS * (STAGE_OUT_BYTES + SCALE_BYTES) + LUT_BYTES;
+    static constexpr int STAGES = (232448 - 1024 - 512 - FIXED) / STAGE_BYTES > 6
+                                      ? 6 : (232448 - 1024 - 512 - FIXED) / STAGE_BYTES;
+    static constexpr int OUT_OFF = STAGES * STAGE_BYTES;
+    static constexpr int SCALE_OFF = OUT_OFF + EPI_WARPS * STAGE_OUT_BYTES;
+    static constexpr int LUT_OFF = SCALE_OFF + EPI_WARPS * SCALE_BYTES;
+    static constexpr int BAR_OFF = LUT_OFF + LUT_BYTES;
+    // full[S], empty[S], pfull[S], tfull[2], tempty[2], drain; then tmem base + abort flag
+    static constexpr int BAR_BYTES = (3 * STAGES + 5) * 8;
+    static constexpr int SMEM_BYTES = 1024 + BAR_OFF + BAR_BYTES + 16;
+    static_assert(STAGES >= 3, "pipeline depth");
+    static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
+};
+
+template <bool GELU, bool FP8>
+__global__ void __launch_bounds__(320, 1)
+    gemm_s8_pair_kernel(const __grid_constant__ CUtensorMap tmA,
+                        const __grid_constant__ CUtensorMap tmB,
+                        const __grid_constant__ CUtensorMap tmO, const GemmParams p)
+{
+    using C = PairConfig<GELU>;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_addr = smem_u32(smem_raw);
+    const uint32_t base = (raw_addr + 1023u) & ~1023u;
+    uint8_t *smem = smem_raw + (base - raw_addr);
+    const uint32_t bar0 = base + C::BAR_OFF;
+    auto full_bar = [&](int s) { return bar0 + 8u * s; };
+    auto empty_bar = [&](int s) { return bar0 + 8u * (C::STAGES + s); };
+    auto pfull_bar = [&](int s) { return bar0 + 8u * (2 * C::STAGES + s); };
+    auto tfull_bar = [&](int b) { return bar0 + 8u * (3 * C::STAGES + b); };
+    auto tempty_bar = [&](int b) { return bar0 + 8u * (3 * C::STAGES + 2 + b); };
+    const uint32_t drain_bar = bar0 + 8u * (3 * C::STAGES + 4);
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C::BAR_OFF + C::BAR_BYTES);
+    volatile int *abort = reinterpret_cast<volatile int *>(tmem_holder + 1);
+
+    const uint32_t warp = threadIdx.x >> 5;
+    const uint32_t lane = lane_id();
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = rank == 0u;
+    const int pair = static_cast<int>(cluster_id_x());
+    const int npairs = static_cast<int>(nclusters_x());
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::STAGES; ++s) {
+            mbar_init(full_bar(s), 1);
+            mbar_init(empty_bar(s), 1);
+            mbar_init(pfull_bar(s), 1);
+        }
+        for (int b = 0; b < C::NBUF; ++b) {
+            mbar_init(tfull_bar(b), 1);
+            mbar_init(tempty_bar(b), 2 * C::EPI_WARPS);
+        }
+        mbar_init(drain_bar, 1);
+        *abort = 0;
+        fence_mbar_init();
+        prefetch_tensormap(&tmA);
+        prefetch_tensormap(&tmB);
+        prefetch_tensormap(&tmO);
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(smem_u32(tmem_holder), C::TMEM_COLS);
+        tmem_relinquish_pair();
+    }
+    // both CTAs' barriers are initialised and their tensor memory allocated before any
+    // remote arrive or multicast commit reaches them
+    tc_fence_before_sync();
+    cluster_sync_all();
+    tc_fence_after_sync();
+    const uint32_t tmem_base = *tmem_holder;
+    grid_dependency_wait();
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int issued = 0;
+            bool ok = true;
+            for (int tile = pair; ok && tile < p.num_tiles; tile += npairs) {
+                const int m0 = (tile % p.num_m_blocks) * 2 * C::BM + static_cast<int>(rank) * C::BM;
+                const int nr0 = (tile / p.num_m_blocks) * C::BN + static_cast<int>(rank) * (C::BN / 2);
+                for (int kb = 0; kb < p.num_kb; ++kb) {
+                    if (!mbar_wait_bounded(empty_bar(stage), phase ^ 1u, abort, p.timeout_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t sa = base + stage * C::STAGE_BYTES;
+                    mbar_arrive_expect_tx(full_bar(stage), C::STAGE_BYTES);
+                    tma_load_2d(sa, &tmA, full_bar(stage), kb * C::BK, m0);
+                    tma_load_2d(sa + C::A_BYTES, &tmB, full_bar(stage), kb * C::BK, nr0);
+                    ++issued;
+                    if (++stage == C::STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (!ok) {
+                // drain: wait (bounded) for this CTA's copies of the last stages issued
+                const int n = issued < C::STAGES ? issued : C::STAGES;
+                int s = stage;
+                uint32_t ph = phase;
+                for (int i = 0; i < n; ++i) {
+                    if (--s < 0) {
+                        s = C::STAGES - 1;
+                        ph ^= 1u;
+                    }
+                    volatile int no_abort = 0;
+                    mbar_wait_bounded(full_bar(s), ph, &no_abort, p.timeout_ns);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && leader) {
+            // -------------------------------------------------------- MMA issuer (rank 0)
+            constexpr uint32_t IDESC = FP8 ? idesc_e4m3_f32(256, C::BN) : idesc_s8_s32(256, C::BN);
+            int stage = 0;
+            uint32_t phase = 0;
+            int local = 0;
+            bool ok = true;
+            for (int tile = pair; ok && tile < p.num_tiles; tile += npairs, ++local) {
+                const int buf = local % C::NBUF;
+                const uint32_t use = static_cast<uint32_t>(local / C::NBUF);
+                if (!mbar_wait_bounded_cluster(tempty_bar(buf), (use & 1u) ^ 1u, abort, p.timeout_ns)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after_sync();
+                const uint32_t d_acc = tmem_base + buf * C::ACC_COLS;
+                for (int kb = 0; kb < p.num_kb; ++kb) {
+                    if (!mbar_wait_bounded(full_bar(stage), phase, abort, p.timeout_ns) ||
+                        !mbar_wait_bounded_cluster(pfull_bar(stage), phase, abort, p.timeout_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after_sync();
+                    const uint32_t sa = base + stage * C::STAGE_BYTES;
+                    const uint32_t sb = sa + C::A_BYTES;
+#pragma unroll
+                    for (int k = 0; k < C::BK / 32; ++k) {
+                        if constexpr (FP8)
+                            mma_f8_pair(d_acc, kmajor_desc(sa + 32 * k), kmajor_desc(sb + 32 * k), IDESC,
+                                        (kb | k) != 0 ? 1u : 0u);
+                        else
+                            mma_s8_pair(d_acc, kmajor_desc(sa + 32 * k), kmajor_desc(sb + 32 * k), IDESC,
+                                        (kb | k) != 0 ? 1u : 0u);
+                    }
+                    tc_commit_pair(empty_bar(stage), 0x3);
+                    if (++stage == C::STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok)
+                    break;
+                tc_commit_pair(tfull_bar(buf), 0x3);
+            }
+            // drain: every MMA issued has completed before either CTA frees its tensor memory
+            tc_commit_pair(drain_bar, 0x1);
+            volatile int no_abort = 0;
+            mbar_wait_bounded(drain_bar, 0u, &no_abort, p.timeout_ns);
+        } else if (lane == 0) {
+            // -------------------------------------------------------- stage forwarder (rank 1)
+            const uint32_t peer_pfull0 = mapa_shared(pfull_bar(0), 0u);
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int tile = pair; ok && tile < p.num_tiles; tile += npairs) {
+                for (int kb = 0; kb < p.num_kb; ++kb) {
+                    if (!mbar_wait_bounded(full_bar(stage), phase, abort, p.timeout_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_remote(peer_pfull0 + 8u * stage);
+                    if (++stage == C::STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue (warps 2..9)
+        const uint32_t quad = warp & 3u;
+        const uint32_t ew = warp - 2u;
+        const int col_base = static_cast<int>(ew >> 2) * C::EPI_COLS;
+        const int row_in_tile = static_cast<int>(quad * 32u + lane);
+        const uint32_t s_out = base + C::OUT_OFF + ew * C::STAGE_OUT_BYTES;
+        const uint32_t s_sw = base + C::SCALE_OFF + ew * C::SCALE_BYTES;
+        const uint32_t s_bias = s_sw + C::EPI_COLS * 4;
+        const bool has_bias = p.bias != nullptr;
+        const uint32_t leader_tempty0 = mapa_shared(tempty_bar(0), 0u);
+        uint16_t *lut = reinterpret_cast<uint16_t *>(smem + C::LUT_OFF);
+        if constexpr (GELU) {
+            for (int i = static_cast<int>(ew * 32u + lane); i < kGeluLutEntries; i += 32 * C::EPI_WARPS)
+                lut[i] = static_cast<uint16_t>(gelu_bf16_bits(gelu_lut_input(i)));
+            bar_sync_or(1, 32 * C::EPI_WARPS, false);
+        }
+        int local = 0;
+        for (int tile = pair; tile < p.num_tiles; tile += npairs, ++local) {
+            const int buf = local % C::NBUF;
+            const uint32_t use = static_cast<uint32_t>(local / C::NBUF);
+            const int m0 = (tile % p.num_m_blocks) * 2 * C::BM + static_cast<int>(rank) * C::BM;
+            const int n0 = (tile / p.num_m_blocks) * C::BN;
+            const int nw = n0 + col_base;
+#pragma unroll
+            for (int j = static_cast<int>(lane) * 4; j < C::EPI_COLS; j += 128) {
+                float w4[4], b4[4];
+                if (nw + j + 4 <= p.N) {
+                    const float4 f = __ldg(reinterpret_cast<const float4 *>(p.sw + nw + j));
+                    w4[0] = f.x; w4[1] = f.y; w4[2] = f.z; w4[3] = f.w;
+                    if (has_bias) {
+                        const uint2 bb = __ldg(reinterpret_cast<const uint2 *>(p.bias + nw + j));
+                        b4[0] = bf16_bits_to_float(bb.x & 0xffffu);
+                        b4[1] = bf16_bits_to_float(bb.x >> 16);
+                        b4[2] = bf16_bits_to_float(bb.y & 0xffffu);
+                        b4[3] = bf16_bits_to_float(bb.y >> 16);
+                    }
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const bool ok = nw + j + e < p.N;
+                        w4[e] = ok ? __ldg(p.sw + nw + j + e) : 0.0f;
+                        b4[e] = (ok && has_bias) ? bf16_bits_to_float(__ldg(p.bias + nw + j + e)) : 0.0f;
+                    }
+                }
+                if (!has_bias)
+                    b4[0] = b4[1] = b4[2] = b4[3] = 0.0f;
+                sts_v4(s_sw + 4 * j, __float_as_uint(w4[0]), __float_as_uint(w4[1]),
+                       __float_as_uint(w4[2]), __float_as_uint(w4[3]));
+                sts_v4(s_bias + 4 * j, __float_as_uint(b4[0]), __float_as_uint(b4[1]),
+                       __float_as_uint(b4[2]), __float_as_uint(b4[3]));
+            }
+            __syncwarp();
+            const bool ready = mbar_wait_bounded(tfull_bar(buf), use & 1u, abort, p.timeout_ns);
+            if (!__all_sync(0xffffffffu, ready))
+                break;
+            tc_fence_after_sync();
+            const int m = m0 + row_in_tile;
+            const bool row_ok = m < p.M;
+            const float sxm = row_ok ? p.sx[m] : 0.0f;
+            const uint32_t t_row = tmem_base + ((quad * 32u) << 16) + buf * C::ACC_COLS;
+#pragma unroll 1
+            for (int c = 0; c < C::EPI_COLS; c += 32) {
+                const int cc = col_base + c;
+                const int nc = n0 + cc;
+                if (nc >= p.N)
+                    break;  // warp-uniform
+                uint32_t acc[32];
+                tmem_ld_32x32b_x32(t_row + cc, acc);
+                tmem_ld_wait();
+                uint32_t ob[16];
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const float4 w = lds_v4(s_sw + 4 * (c + 4 * q));
+                    const float4 b = lds_v4(s_bias + 4 * (c + 4 * q));
+                    const float wv[4] = {w.x, w.y, w.z, w.w};
+                    const float bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const int j = 4 * q + 2 * h;
+                        // the same fp32 steps as the single-SM epilogue: t in f32x2, the
+                        // products that feed an add as scalar intrinsics
+                        float t0, t1;
+                        mul2(t0, t1, sxm, sxm, wv[2 * h], wv[2 * h + 1]);
+                        const float a0 = FP8 ? __uint_as_float(acc[j]) : __int2float_rn(static_cast<int>(acc[j]));
+                        const float a1 = FP8 ? __uint_as_float(acc[j + 1])
+                                             : __int2float_rn(static_cast<int>(acc[j + 1]));
+                        float v0 = __fmul_rn(a0, t0);
+                        float v1 = __fmul_rn(a1, t1);
+                        if (has_bias) {
+                            v0 = __fadd_rn(v0, bv[2 * h]);
+                            v1 = __fadd_rn(v1, bv[2 * h + 1]);
+                        }
+                        const __nv_bfloat162 h2 = __floats2bfloat162_rn(v0, v1);
+                        ob[j >> 1] = *reinterpret_cast<const uint32_t *>(&h2);
+                    }
+                }
+                if constexpr (GELU) {
+                    gelu_bf16x16_lut(ob, lut);
+                    gelu_bf16x16_lut(ob + 8, lut);
+                }
+                store_block(ob, s_out, lane, &tmO, nc, m0 + static_cast<int>(quad * 32u));
+                if (p.acc_out != nullptr && row_ok) {
+                    int32_t *arow = p.acc_out + static_cast<int64_t>(m) * p.N;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        if (nc + j < p.N)
+                            arow[nc + j] = static_cast<int32_t>(acc[j]);
+                }
+            }
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive_remote(leader_tempty0 + 8u * buf);
+        }
+        if (lane == 0)
+            bulk_wait_all();
+    }
+
+    // neither CTA frees its tensor memory or shared memory while the pair's MMAs may still
+    // use them: rank 0's MMA warp has drained every MMA before it arrives here
+    tc_fence_before_sync();
+    __syncthreads();
+    cluster_sync_all();
+    if (warp == 1) {
+        tc_fence_after_sync();
+        tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+    }
+}
+
+} // namespace sdnq

@@ -17,6 +17,7 @@
 #include "device.cuh"
 #include "gelu.cuh"
 #include "gemm.cuh"
+#include "gemm_pair.cuh"
 #include "attention.cuh"
 #include "lora_down.cuh"
 #include "rotquant.cuh"
@@ -202,10 +203,92 @@ sdnq_status validate_rotquant(const void *x, int64_t rows, int64_t K, int64_t ld
 
 // Rows of at most 16 chunks go to the persistent, prefetching kernel (grid = resident
 // CTAs); longer rows to the two-pass kernel with one CTA per row.
+// Block shape of the run-per-lane kernel: `warps` warps hold `rows` = floor(32 warps / rpr)
+// rows of rpr runs of 64 elements; the warp count in 4..16 that leaves the fewest lanes idle
+// (the smallest such count). rows == 0 means the row is too long for it (rpr > 512).
+struct RunShape {
+    int warps = 0;
+    int rows = 0;
+};
+
+RunShape run_shape(int64_t rpr)
+{
+    RunShape best;
+    double best_used = -1.0;
+    for (int w = 4; w <= 16; ++w) {
+        const int64_t rows = 32 * w / rpr;
+        if (rows < 1)
+            continue;
+        const double used = static_cast<double>(rows * rpr) / (32.0 * w);
+        if (used > best_used + 1e-9) {
+            best.warps = w;
+            best.rows = static_cast<int>(rows);
+            best_used = used;
+        }
+    }
+    return best;
+}
+
+constexpr int kRunTransposeBytesPerWarp = 32 * 272;   // 32 owners x 17 units of 16 bytes
+
+template <int G, bool FP8, bool V8>
+void launch_rotquant_run(const RotquantParams &rp, const RunShape &shape, const DeviceInfo &dev,
+                         cudaStream_t st)
+{
+    constexpr auto kernel = rotquant_run_kernel<G, FP8, V8>;
+    const int threads = 32 * shape.warps;
+    auto smem_for = [](int warps, int rows) {
+        return (G >= 128 ? warps * kRunTransposeBytesPerWarp : 0) + 3 * rows * 4;
+    };
+    static PerDeviceCache<1> smem_attr;
+    static PerDeviceCache<17> per_sm;   // resident blocks per SM, by warps per block
+    if (!smem_attr_once(smem_attr, dev.index, kernel, smem_for(16, 512)))
+        return;   // the launch below is then skipped; launch_status reports the error
+    const int n_sm = per_sm.get(dev.index, shape.warps, [&] {
+        int n = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, threads,
+                                                          smem_for(shape.warps, 32 * shape.warps)) !=
+                cudaSuccess ||
+            n < 1) {
+            cudaGetLastError();
+            n = 1;
+        }
+        return n;
+    });
+    RotquantRunParams p;
+    p.x = rp.x;
+    p.ldx = rp.ldx;
+    p.q = rp.q;
+    p.s = rp.s;
+    p.M = rp.M;
+    p.K = rp.K;
+    p.rpr = (rp.K + 63) / 64;
+    p.rows = shape.rows;
+    p.c_g = rp.c_g;
+    const int64_t blocks = (rp.M + shape.rows - 1) / shape.rows;
+    const int64_t resident = static_cast<int64_t>(n_sm) * dev.sm_count;
+    const unsigned grid = static_cast<unsigned>(blocks < resident ? blocks : resident);
+    kernel<<<grid, threads, smem_for(shape.warps, shape.rows), st>>>(p);
+}
+
+// Rows of up to 512 runs (K <= 32768) go to the run-per-lane kernel; the column-multiplier
+// mode (the input gradient's quantizer) to the chunk-per-warp persistent kernel for rows of
+// at most 16 chunks; longer rows to the two-pass kernel with one block per row.
 template <int G, bool COLSCALE = false, bool FP8 = false>
 void launch_rotquant_g(const RotquantParams &p, dim3 grid, dim3 block, const DeviceInfo &dev,
                        cudaStream_t st)
 {
+    if constexpr (!COLSCALE) {
+        const RunShape shape = run_shape((p.K + 63) / 64);
+        if (shape.rows > 0) {
+            const bool v8 = (reinterpret_cast<uintptr_t>(p.x) % 32) == 0 && (p.ldx % 16) == 0;
+            if (v8)
+                launch_rotquant_run<G, FP8, true>(p, shape, dev, st);
+            else
+                launch_rotquant_run<G, FP8, false>(p, shape, dev, st);
+            return;
+        }
+    }
     if (p.nchunks <= 16) {
         // resident CTAs per SM, by device and warps per CTA
         static PerDeviceCache<33> per_sm;
@@ -379,6 +462,69 @@ sdnq_status launch_gemm(const DeviceInfo &dev, const int8_t *qx, const int8_t *q
     return launch_status();
 }
 
+// The CTA-pair kernel (cta_group::2, 256 x 256 tiles) for the plain, GELU and e4m3 linears.
+// A cluster of two CTAs per pair, launched programmatically like the single-SM kernel; the
+// grid holds as many pairs as the device can keep resident at once (or fewer, one per
+// tile), each walking the tiles persistently.
+template <bool GELU, bool FP8>
+sdnq_status launch_gemm_pair(const DeviceInfo &dev, const int8_t *qx, const int8_t *qW,
+                             GemmParams p, cudaStream_t cs)
+{
+    using C = PairConfig<GELU>;
+    constexpr auto kernel = gemm_s8_pair_kernel<GELU, FP8>;
+    CUtensorMap tmA, tmB, tmO;
+    if (!make_tmap_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, qx, p.K, p.M, p.K, 128, 128) ||
+        !make_tmap_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, qW, p.K, p.N, p.K, 128, C::BN / 2) ||
+        !make_tmap_2d(&tmO, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.out, p.N, p.M, 2ull * p.ldo, 32, 32,
+                      CU_TENSOR_MAP_SWIZZLE_64B))
+        return SDNQ_ERR_CUDA;
+    static PerDeviceCache<1> smem_attr;
+    if (!smem_attr_once(smem_attr, dev.index, kernel, C::SMEM_BYTES))
+        return SDNQ_ERR_CUDA;
+    p.num_kb = (p.K + C::BK - 1) / C::BK;
+    p.num_m_blocks = (p.M + 2 * C::BM - 1) / (2 * C::BM);
+    p.num_n_blocks = (p.N + C::BN - 1) / C::BN;
+    p.num_tiles = p.num_m_blocks * p.num_n_blocks;
+
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(C::THREADS);
+    cfg.dynamicSmemBytes = C::SMEM_BYTES;
+    cfg.stream = cs;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    static PerDeviceCache<1> max_pairs;
+    const int resident_pairs = max_pairs.get(dev.index, 0, [&] {
+        cudaLaunchConfig_t q = cfg;
+        q.gridDim = dim3(static_cast<unsigned>(dev.sm_count / 2 * 2));
+        q.numAttrs = 1;   // the cluster shape alone
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, kernel, &q) != cudaSuccess || n < 1) {
+            cudaGetLastError();
+            n = dev.sm_count / 2;
+        }
+        return n;
+    });
+    const int pairs = p.num_tiles < resident_pairs ? p.num_tiles : resident_pairs;
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
+    cudaGetLastError();
+    if (cudaLaunchKernelEx(&cfg, kernel, tmA, tmB, tmO, p) != cudaSuccess) {
+        cudaGetLastError();
+        return SDNQ_ERR_CUDA;
+    }
+    return launch_status();
+}
+
+// Rows per call at which the CTA-pair kernel takes over from the single-SM one (below it,
+// half of every 256-row pair tile would be padding).
+constexpr int64_t kPairMinRows = 129;
+
 template <int RANK_PAD>
 sdnq_status launch_lora_down(const DeviceInfo &dev, const uint16_t *x, int64_t ldx,
                              const uint16_t *A, int32_t rank, uint16_t *u, int32_t M, int32_t K,
@@ -446,6 +592,9 @@ sdnq_status run_linear(const int8_t *qx, const float *sx, const int8_t *qW, cons
     p.lora_scale = lora_scale;
     p.c_g = 1.0f;
     p.timeout_ns = kDefaultTimeoutNs;
+    if (!lora && M >= kPairMinRows)
+        return gelu ? launch_gemm_pair<true, false>(dev, qx, qW, p, cs)
+                    : launch_gemm_pair<false, false>(dev, qx, qW, p, cs);
     if (!lora)
         return gelu ? launch_gemm<256, false, true>(dev, qx, qW, nullptr, nullptr, 0, p, cs)
                     : launch_gemm<256, false>(dev, qx, qW, nullptr, nullptr, 0, p, cs);
@@ -718,6 +867,10 @@ sdnq_status run_fp8_linear(const uint8_t *qx, const float *sx, const uint8_t *qW
     p.K = static_cast<int32_t>(K);
     p.c_g = 1.0f;
     p.timeout_ns = kDefaultTimeoutNs;
+    if (M >= kPairMinRows)
+        return launch_gemm_pair<false, true>(dev, reinterpret_cast<const int8_t *>(qx),
+                                             reinterpret_cast<const int8_t *>(qW), p,
+                                             static_cast<cudaStream_t>(stream));
     return launch_gemm<256, false, false, 0, 0, true>(
         dev, reinterpret_cast<const int8_t *>(qx), reinterpret_cast<const int8_t *>(qW), nullptr,
         nullptr, 0, p, static_cast<cudaStream_t>(stream));

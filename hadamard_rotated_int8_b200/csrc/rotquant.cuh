@@ -528,4 +528,245 @@ __global__ void __launch_bounds__(512) rotquant_kernel(const RotquantParams p)
     }
 }
 
+// ---------------------------------------------------------------------------------------
+// Run-per-lane rotate + quantize (rows up to 32768 elements).
+//
+// Each lane owns one run of 64 consecutive elements of a row, loaded as four 32-byte pieces
+// (one full sector each), so that the butterfly stages h = 1 .. 32 run in its registers.
+// For groups of 128 and 256 the remaining stages (h = 64, 128) cross the runs of a group,
+// which sit on the group's G / 64 neighbouring lanes: the lanes swap their values through a
+// padded shared-memory buffer (one store and one load of 16 bytes per 4 values) so that
+// each lane then holds, for every run of its group, one contiguous piece of 64 / (G / 64)
+// elements, and those stages run in registers too. The buffer keeps owner o's slot s (four
+// fp32 values) at 16-byte unit o * 17 + Pc * (s % spp) + s / spp, with Pc = G / 64 lanes per
+// group and spp = 16 / Pc slots per piece: both the stores (fixed s, consecutive owners) and
+// the loads (fixed run and slot, consecutive lanes) hit eight different bank groups per
+// quarter warp, and both are a lane base plus a compile-time offset.
+//
+// A block holds `rows` rows of runs per iteration (slot = row_local * rpr + run for its
+// threads), walks the row blocks persistently and loads the next block's runs into
+// registers while it rotates and quantizes the current one. The row maximum combines the
+// lanes of a row inside each warp (segmented shuffle), then across warps with one shared
+// atomic max per warp segment and one block barrier per iteration; the three row-maximum
+// buffers rotate so that resetting one never races with the iterations around it.
+struct RotquantRunParams {
+    const uint16_t *x;   // [M, K] bf16 patterns, row stride ldx
+    int64_t ldx;
+    int8_t *q;           // [M, K] dense
+    float *s;            // [M]
+    int64_t M;
+    int32_t K;
+    int32_t rpr;         // runs of 64 elements per row, ceil(K / 64)
+    int32_t rows;        // rows per block iteration
+    float c_g;           // fp32(1 / sqrt(G))
+};
+
+__device__ __forceinline__ void ld_nc_v8(const void *ptr, uint32_t *r)
+{
+    asm volatile("ld.global.nc.L1::no_allocate.v8.u32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                   "=r"(r[6]), "=r"(r[7])
+                 : "l"(ptr));
+}
+
+__device__ __forceinline__ void ld_nc_v4_l1(const void *ptr, uint32_t *r)
+{
+    asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "l"(ptr));
+}
+
+// The lane's run of 64 elements (4 pieces of 16; a piece past the row end reads zeros).
+// V8: one 32-byte load per piece (row start 32-byte aligned); otherwise two 16-byte loads
+// through L1, so that the second half of each sector is served from there.
+template <bool V8>
+__device__ __forceinline__ void load_run(const uint16_t *xr, int32_t e0, int32_t K, bool ok,
+                                         uint32_t (&raw)[32])
+{
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+        const int32_t e = e0 + 16 * t;
+        if (ok && e < K) {
+            if constexpr (V8) {
+                ld_nc_v8(xr + e, raw + 8 * t);
+            } else {
+                ld_nc_v4_l1(xr + e, raw + 8 * t);
+                ld_nc_v4_l1(xr + e + 8, raw + 8 * t + 4);
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                raw[8 * t + i] = 0u;
+        }
+    }
+}
+
+// fmax of m and the magnitudes of a and b, one three-input maximum
+__device__ __forceinline__ float max3_abs(float m, float a, float b)
+{
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(m), "f"(fabsf(a)), "f"(fabsf(b)));
+    return d;
+}
+
+// Butterfly stages h = 1 .. min(G, 64) / 2 over the run's 64 consecutive values. Stage 1
+// pairs the two halves of each register pair (scalar); the later stages pair registers
+// pairwise (f32x2, two lanes of IEEE fp32 per instruction).
+template <int G>
+__device__ __forceinline__ void run_butterfly(float (&v)[64])
+{
+    if (G > 1) {
+#pragma unroll
+        for (int i = 0; i < 64; i += 2) {
+            const float a = v[i], b = v[i + 1];
+            v[i] = __fadd_rn(a, b);
+            v[i + 1] = __fsub_rn(a, b);
+        }
+    }
+#pragma unroll
+    for (int h = 2; h < 64 && h < G; h <<= 1) {
+#pragma unroll
+        for (int i = 0; i < 64; i += 2)
+            if ((i & h) == 0)
+                bfly2(v[i], v[i + 1], v[i + h], v[i + h + 1]);
+    }
+}
+
+template <int G, bool FP8, bool V8>
+__global__ void __launch_bounds__(512) rotquant_run_kernel(const RotquantRunParams p)
+{
+    grid_dependents_launch();
+    constexpr int PC = G >= 128 ? G / 64 : 1;   // lanes (runs) per group in the transposed stages
+    constexpr int PIECE = 64 / PC;              // elements of each run a lane holds afterwards
+    extern __shared__ __align__(16) uint8_t rq_smem[];
+    const int32_t nwarps = static_cast<int32_t>(blockDim.x >> 5);
+    uint32_t *s_max = reinterpret_cast<uint32_t *>(rq_smem + (G >= 128 ? nwarps * 32 * 272 : 0));
+    const uint32_t lane = lane_id();
+    const int32_t warp = static_cast<int32_t>(threadIdx.x >> 5);
+    const int32_t slot = static_cast<int32_t>(threadIdx.x);
+    const int32_t row_local = slot / p.rpr;
+    const int32_t run = slot - row_local * p.rpr;
+    const bool active = row_local < p.rows;
+    const int32_t e0 = run * 64;
+    const int64_t n_blocks = (p.M + p.rows - 1) / p.rows;
+
+    // segmented maximum over the lanes of this lane's row inside the warp: step d takes
+    // lane + d's value when that lane holds the same row
+    const int32_t row_end = (row_local + 1) * p.rpr;   // first slot of the next row
+    const bool seg_first = active && (lane == 0u || run == 0);
+    for (int32_t i = slot; i < 3 * p.rows; i += static_cast<int32_t>(blockDim.x))
+        s_max[i] = 0u;
+    __syncthreads();
+
+    // transposition buffer of this warp (groups of 128 and 256)
+    const uint32_t tbuf = smem_u32(rq_smem) + static_cast<uint32_t>(warp) * (32u * 272u);
+    const uint32_t t_wr = tbuf + lane * 272u;                          // owner = lane
+    const uint32_t t_rd = tbuf + ((lane / PC) * PC * 17u + lane % PC) * 16u;
+    const int32_t p_in_group = static_cast<int32_t>(lane % PC);
+    const int32_t group_run0 = run - p_in_group;                       // first run of the group
+
+    int64_t rb = blockIdx.x;
+    uint32_t raw[32];
+    {
+        const int64_t row = rb * p.rows + row_local;
+        const bool ok = rb < n_blocks && active && row < p.M;
+        load_run<V8>(p.x + (ok ? row : 0) * p.ldx, e0, p.K, ok, raw);
+    }
+    for (int it = 0; rb < n_blocks; rb += gridDim.x, ++it) {
+        const int64_t row = rb * p.rows + row_local;
+        const bool row_ok = active && row < p.M;
+        float v[64];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            v[2 * i] = __uint_as_float(raw[i] << 16);
+            v[2 * i + 1] = __uint_as_float(raw[i] & 0xffff0000u);
+        }
+        {   // the next row block's runs, while this one is computed
+            const int64_t nrb = rb + gridDim.x;
+            const int64_t nrow = nrb * p.rows + row_local;
+            const bool ok = nrb < n_blocks && active && nrow < p.M;
+            load_run<V8>(p.x + (ok ? nrow : 0) * p.ldx, e0, p.K, ok, raw);
+        }
+        run_butterfly<G>(v);
+        if constexpr (G >= 128) {
+            // to the transposed layout: owner `lane` stores its 16 slots of four values
+            constexpr int SPP = 16 / PC;
+#pragma unroll
+            for (int sl = 0; sl < 16; ++sl)
+                sts_v4(t_wr + static_cast<uint32_t>(PC * (sl % SPP) + sl / SPP) * 16u,
+                       __float_as_uint(v[4 * sl]), __float_as_uint(v[4 * sl + 1]),
+                       __float_as_uint(v[4 * sl + 2]), __float_as_uint(v[4 * sl + 3]));
+            __syncwarp();
+            // v[j * PIECE + i] = element p_in_group * PIECE + i of run j of the group
+#pragma unroll
+            for (int j = 0; j < PC; ++j)
+#pragma unroll
+                for (int k = 0; k < SPP; ++k) {
+                    const float4 f = lds_v4(t_rd + static_cast<uint32_t>(j * 17 + PC * k) * 16u);
+                    v[j * PIECE + 4 * k] = f.x;
+                    v[j * PIECE + 4 * k + 1] = f.y;
+                    v[j * PIECE + 4 * k + 2] = f.z;
+                    v[j * PIECE + 4 * k + 3] = f.w;
+                }
+            // stage h = 64 across runs j, j + 1; h = 128 across runs j, j + 2
+#pragma unroll
+            for (int d = 1; d < PC; d <<= 1)
+#pragma unroll
+                for (int j = 0; j < PC; ++j)
+                    if ((j & d) == 0)
+#pragma unroll
+                        for (int i = 0; i < PIECE; i += 2)
+                            bfly2(v[j * PIECE + i], v[j * PIECE + i + 1], v[(j + d) * PIECE + i],
+                                  v[(j + d) * PIECE + i + 1]);
+        }
+        float amax = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 64; i += 2)
+            amax = max3_abs(amax, v[i], v[i + 1]);
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const float o = __shfl_down_sync(0xffffffffu, amax, d);
+            if (static_cast<int32_t>(lane) + d < 32 && slot + d < row_end)
+                amax = fmaxf(amax, o);
+        }
+        uint32_t *mx = s_max + (it % 3) * p.rows;
+        if (seg_first)
+            atomicMax(mx + row_local, __float_as_uint(amax));   // amax >= 0: bits order as values
+        __syncthreads();
+        if (slot < p.rows)
+            s_max[((it + 2) % 3) * p.rows + slot] = 0u;          // the buffer of iteration it + 2
+        amax = active ? __uint_as_float(mx[row_local]) : 0.0f;
+        const float s_z = __fdiv_rn(amax, FP8 ? 448.0f : 127.0f);
+        const bool zero = !(amax > 0.0f);
+        if (row_ok && run == 0)
+            p.s[row] = zero ? 0.0f : __fmul_rn(s_z, p.c_g);
+        const bool fast = s_z >= 0x1p-126f;
+        const float rcp = __frcp_rn(s_z);
+        int8_t *qr = p.q + (row_ok ? row : 0) * static_cast<int64_t>(p.K);
+        // codes of 16 consecutive values -> one 16-byte store
+        auto store16 = [&](const float *z, int32_t e) {
+            uint2 a = make_uint2(0u, 0u), b = make_uint2(0u, 0u);
+            if (!zero) {
+                const float za[8] = {z[0], z[1], z[2], z[3], z[4], z[5], z[6], z[7]};
+                const float zb[8] = {z[8], z[9], z[10], z[11], z[12], z[13], z[14], z[15]};
+                a = FP8 ? quant8_e4m3(za, s_z, rcp, fast) : quant8(za, s_z, rcp, fast);
+                b = FP8 ? quant8_e4m3(zb, s_z, rcp, fast) : quant8(zb, s_z, rcp, fast);
+            }
+            if (row_ok && e < p.K)
+                st_v4(qr + e, a.x, a.y, b.x, b.y);
+        };
+        if constexpr (G >= 128) {
+#pragma unroll
+            for (int j = 0; j < PC; ++j)
+#pragma unroll
+                for (int i = 0; i < PIECE; i += 16)
+                    store16(v + j * PIECE + i, (group_run0 + j) * 64 + p_in_group * PIECE + i);
+        } else {
+#pragma unroll
+            for (int t = 0; t < 4; ++t)
+                store16(v + 16 * t, e0 + 16 * t);
+        }
+    }
+}
+
 } // namespace sdnq

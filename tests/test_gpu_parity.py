@@ -86,6 +86,30 @@ def test_rotquant_bit_exact(M, K, g):
     assert_equal(s.view(np.uint32), s_ref.view(np.uint32), f"scales M={M} K={K} g={g}")
 
 
+@pytest.mark.parametrize("M,K,g,offset,pad", [
+    (77, 3072, 256, 8, 0),      # rows 16 but not 32 bytes aligned: the 16-byte load path
+    (50, 4096, 128, 0, 8),      # row stride K + 8: every other row off the 32-byte grid
+    (33, 1040, 16, 8, 24),      # a partial last run (1040 = 16 runs + 16 elements)
+    (129, 10240, 256, 0, 16),   # 40 groups per row, stride padded by 32 bytes
+    (3, 32768, 256, 0, 0),      # the longest row of the run-per-lane kernel (512 runs)
+    (2, 32768 + 256, 256, 0, 0),  # one group more: the two-pass kernel
+])
+def test_rotquant_offsets_and_strides(M, K, g, offset, pad):
+    """Rows that start off the 32-byte grid (a view into a larger buffer), padded row
+    strides, a partial last run and the row lengths where the kernel choice changes:
+    codes and scales bit-exact."""
+    case = synthetic.make_case(M=M, N=8, K=K, g=g, seed=K + pad + offset, outlier_count=K // 200,
+                               outlier_factor=30.0)
+    buf = torch.zeros((M, offset + K + pad), dtype=torch.bfloat16, device="cuda")
+    buf[:, offset:offset + K] = case.x.cuda()
+    x = buf[:, offset:offset + K]
+    q, s = sd.sdnq_rotquant_act(x, g)
+    torch.cuda.synchronize()
+    q_ref, s_ref = oracle.rotate_quantize(synthetic.bits(case.x), g)
+    assert_equal(q.cpu().numpy(), q_ref, "codes")
+    assert_equal(s.cpu().numpy().view(np.uint32), s_ref.view(np.uint32), "scales")
+
+
 @pytest.mark.parametrize("g", [8, 64, 256])
 def test_rotquant_exact_ties_round_half_even(g):
     """Integer rows whose rotated absmax is 127 * 2^k make s_z a power of two, so many
