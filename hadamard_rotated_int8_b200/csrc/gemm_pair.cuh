@@ -5,7 +5,10 @@
 // single-SM 128 x 256 tile streams 48 KB, for the same tensor-core work per SM. Each CTA's
 // tensor memory receives its 128 rows of the int32 (fp32 for e4m3) accumulators, and its own
 // epilogue warps apply the same fp32 de-quant epilogue (and the GELU table) as the single-SM
-// kernel, so outputs are bit for bit the same.
+// kernel, so outputs are bit for bit the same. With LORA the pair also accumulates the
+// adapter term L = u B (bf16 operands, fp32, kind::f16) in a second 256-column accumulator
+// after the int8 K loop, as the single-SM kernel does; the int32 and fp32 accumulators then
+// fill the 512 columns, so there is one buffer.
 //
 // Sources: as the single-SM kernel ("SDNQ: SD.Next Quantization Engine" README, INT8
 // quantized matmul and dequantize_fp32; "ConvRot / Hadamard SDNQ").
@@ -27,7 +30,7 @@
 
 namespace sdnq {
 
-template <bool GELU>
+template <bool GELU, bool LORA = false>
 struct PairConfig {
     static constexpr int BM = 128;                       // rows per CTA (256 per pair)
     static constexpr int BN = 256;                       // columns per pair tile
@@ -35,8 +38,8 @@ struct PairConfig {
     static constexpr int A_BYTES = BM * BK;              // 16 KB
     static constexpr int B_BYTES = (BN / 2) * BK;        // this CTA's 128 columns: 16 KB
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-    static constexpr int ACC_COLS = BN;                  // int32 / fp32 columns per buffer
-    static constexpr int NBUF = 2;
+    static constexpr int ACC_COLS = LORA ? 2 * BN : BN;  // int32 (+ fp32 LoRA) columns per buffer
+    static constexpr int NBUF = LORA ? 1 : 2;
     static constexpr int TMEM_COLS = NBUF * ACC_COLS;    // 512
     static constexpr int THREADS = 320;
     static constexpr int EPI_WARPS = 8;
@@ -58,13 +61,16 @@ struct PairConfig {
     static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 };
 
-template <bool GELU, bool FP8>
+template <bool GELU, bool FP8, bool LORA>
 __global__ void __launch_bounds__(320, 1)
     gemm_s8_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB,
+                        const __grid_constant__ CUtensorMap tmU,
+                        const __grid_constant__ CUtensorMap tmL,
                         const __grid_constant__ CUtensorMap tmO, const GemmParams p)
 {
-    using C = PairConfig<GELU>;
+    using C = PairConfig<GELU, LORA>;
+    static_assert(!LORA || (!GELU && !FP8), "the adapter term rides on the plain int8 linear");
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_addr = smem_u32(smem_raw);
     const uint32_t base = (raw_addr + 1023u) & ~1023u;
@@ -102,6 +108,10 @@ __global__ void __launch_bounds__(320, 1)
         prefetch_tensormap(&tmA);
         prefetch_tensormap(&tmB);
         prefetch_tensormap(&tmO);
+        if (LORA) {
+            prefetch_tensormap(&tmU);
+            prefetch_tensormap(&tmL);
+        }
     }
     if (warp == 1) {
         tmem_alloc_pair(smem_u32(tmem_holder), C::TMEM_COLS);
@@ -125,15 +135,26 @@ __global__ void __launch_bounds__(320, 1)
             for (int tile = pair; ok && tile < p.num_tiles; tile += npairs) {
                 const int m0 = (tile % p.num_m_blocks) * 2 * C::BM + static_cast<int>(rank) * C::BM;
                 const int nr0 = (tile / p.num_m_blocks) * C::BN + static_cast<int>(rank) * (C::BN / 2);
-                for (int kb = 0; kb < p.num_kb; ++kb) {
+                const int steps = p.num_kb + (LORA ? p.lora_chunks : 0);
+                for (int kb = 0; kb < steps; ++kb) {
                     if (!mbar_wait_bounded(empty_bar(stage), phase ^ 1u, abort, p.timeout_ns)) {
                         ok = false;
                         break;
                     }
                     const uint32_t sa = base + stage * C::STAGE_BYTES;
                     mbar_arrive_expect_tx(full_bar(stage), C::STAGE_BYTES);
-                    tma_load_2d(sa, &tmA, full_bar(stage), kb * C::BK, m0);
-                    tma_load_2d(sa + C::A_BYTES, &tmB, full_bar(stage), kb * C::BK, nr0);
+                    if (!LORA || kb < p.num_kb) {
+                        tma_load_2d(sa, &tmA, full_bar(stage), kb * C::BK, m0);
+                        tma_load_2d(sa + C::A_BYTES, &tmB, full_bar(stage), kb * C::BK, nr0);
+                    } else {
+                        // LoRA chunk c: this CTA's U rows [128 x 64 rank] (K-major) into the A
+                        // slot, its 128 columns of B [64 rank x 128] (N-major) as two 64-column
+                        // boxes into the B slot
+                        const int c = kb - p.num_kb;
+                        tma_load_2d(sa, &tmU, full_bar(stage), c * 64, m0);
+                        tma_load_2d(sa + C::A_BYTES, &tmL, full_bar(stage), nr0, c * 64);
+                        tma_load_2d(sa + C::A_BYTES + 8192, &tmL, full_bar(stage), nr0 + 64, c * 64);
+                    }
                     ++issued;
                     if (++stage == C::STAGES) {
                         stage = 0;
@@ -197,6 +218,31 @@ __global__ void __launch_bounds__(320, 1)
                         phase ^= 1u;
                     }
                 }
+                if constexpr (LORA) {
+                    constexpr uint32_t IDESC_BF = idesc_bf16_f32(256, C::BN, true);
+                    const uint32_t d_lora = d_acc + C::BN;
+                    for (int c = 0; ok && c < p.lora_chunks; ++c) {
+                        if (!mbar_wait_bounded(full_bar(stage), phase, abort, p.timeout_ns) ||
+                            !mbar_wait_bounded_cluster(pfull_bar(stage), phase, abort, p.timeout_ns)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after_sync();
+                        const uint32_t sa = base + stage * C::STAGE_BYTES;
+                        const uint32_t sb = sa + C::A_BYTES;
+                        // 4 MMAs of K = 16 rank rows: A advances 32 bytes along its swizzled
+                        // rows, B (two 64-column atoms 8 KB apart) 16 rows = 2048 bytes
+#pragma unroll
+                        for (int k = 0; k < 4; ++k)
+                            mma_f16_pair(d_lora, kmajor_desc(sa + 32 * k), mnmajor_desc(sb + 2048 * k, 8192),
+                                         IDESC_BF, (c | k) != 0 ? 1u : 0u);
+                        tc_commit_pair(empty_bar(stage), 0x3);
+                        if (++stage == C::STAGES) {
+                            stage = 0;
+                            phase ^= 1u;
+                        }
+                    }
+                }
                 if (!ok)
                     break;
                 tc_commit_pair(tfull_bar(buf), 0x3);
@@ -211,8 +257,9 @@ __global__ void __launch_bounds__(320, 1)
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
+            const int steps = p.num_kb + (LORA ? p.lora_chunks : 0);
             for (int tile = pair; ok && tile < p.num_tiles; tile += npairs) {
-                for (int kb = 0; kb < p.num_kb; ++kb) {
+                for (int kb = 0; kb < steps; ++kb) {
                     if (!mbar_wait_bounded(full_bar(stage), phase, abort, p.timeout_ns)) {
                         ok = false;
                         break;
@@ -294,6 +341,9 @@ __global__ void __launch_bounds__(320, 1)
                     break;  // warp-uniform
                 uint32_t acc[32];
                 tmem_ld_32x32b_x32(t_row + cc, acc);
+                uint32_t lacc[LORA ? 32 : 1];
+                if constexpr (LORA)
+                    tmem_ld_32x32b_x32(t_row + C::BN + cc, lacc);
                 tmem_ld_wait();
                 uint32_t ob[16];
 #pragma unroll
@@ -317,6 +367,10 @@ __global__ void __launch_bounds__(320, 1)
                         if (has_bias) {
                             v0 = __fadd_rn(v0, bv[2 * h]);
                             v1 = __fadd_rn(v1, bv[2 * h + 1]);
+                        }
+                        if constexpr (LORA) {
+                            v0 = __fadd_rn(v0, __fmul_rn(p.lora_scale, __uint_as_float(lacc[j])));
+                            v1 = __fadd_rn(v1, __fmul_rn(p.lora_scale, __uint_as_float(lacc[j + 1])));
                         }
                         const __nv_bfloat162 h2 = __floats2bfloat162_rn(v0, v1);
                         ob[j >> 1] = *reinterpret_cast<const uint32_t *>(&h2);

@@ -466,18 +466,27 @@ sdnq_status launch_gemm(const DeviceInfo &dev, const int8_t *qx, const int8_t *q
 // A cluster of two CTAs per pair, launched programmatically like the single-SM kernel; the
 // grid holds as many pairs as the device can keep resident at once (or fewer, one per
 // tile), each walking the tiles persistently.
-template <bool GELU, bool FP8>
+template <bool GELU, bool FP8, bool LORA = false>
 sdnq_status launch_gemm_pair(const DeviceInfo &dev, const int8_t *qx, const int8_t *qW,
-                             GemmParams p, cudaStream_t cs)
+                             GemmParams p, cudaStream_t cs, const uint16_t *u = nullptr,
+                             const uint16_t *B = nullptr, int32_t rank = 0)
 {
-    using C = PairConfig<GELU>;
-    constexpr auto kernel = gemm_s8_pair_kernel<GELU, FP8>;
-    CUtensorMap tmA, tmB, tmO;
+    using C = PairConfig<GELU, LORA>;
+    constexpr auto kernel = gemm_s8_pair_kernel<GELU, FP8, LORA>;
+    CUtensorMap tmA, tmB, tmU, tmL, tmO;
     if (!make_tmap_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, qx, p.K, p.M, p.K, 128, 128) ||
         !make_tmap_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, qW, p.K, p.N, p.K, 128, C::BN / 2) ||
         !make_tmap_2d(&tmO, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.out, p.N, p.M, 2ull * p.ldo, 32, 32,
                       CU_TENSOR_MAP_SWIZZLE_64B))
         return SDNQ_ERR_CUDA;
+    if (LORA) {
+        if (!make_tmap_2d(&tmU, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, u, rank, p.M, 2ull * rank, 64, 128) ||
+            !make_tmap_2d(&tmL, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, B, p.N, rank, 2ull * p.N, 64, 64))
+            return SDNQ_ERR_CUDA;
+    } else {
+        tmU = tmA;
+        tmL = tmA;
+    }
     static PerDeviceCache<1> smem_attr;
     if (!smem_attr_once(smem_attr, dev.index, kernel, C::SMEM_BYTES))
         return SDNQ_ERR_CUDA;
@@ -514,7 +523,7 @@ sdnq_status launch_gemm_pair(const DeviceInfo &dev, const int8_t *qx, const int8
     const int pairs = p.num_tiles < resident_pairs ? p.num_tiles : resident_pairs;
     cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
     cudaGetLastError();
-    if (cudaLaunchKernelEx(&cfg, kernel, tmA, tmB, tmO, p) != cudaSuccess) {
+    if (cudaLaunchKernelEx(&cfg, kernel, tmA, tmB, tmU, tmL, tmO, p) != cudaSuccess) {
         cudaGetLastError();
         return SDNQ_ERR_CUDA;
     }
@@ -608,6 +617,8 @@ sdnq_status run_linear(const int8_t *qx, const float *sx, const int8_t *qW, cons
     if (st != SDNQ_OK)
         return st;
     p.lora_chunks = (rank + 63) / 64;
+    if (M >= kPairMinRows)
+        return launch_gemm_pair<false, false, true>(dev, qx, qW, p, cs, u_ws, B, rank);
     return launch_gemm<SDNQ_LORA_BN, true>(dev, qx, qW, u_ws, B, rank, p, cs);
 }
 
