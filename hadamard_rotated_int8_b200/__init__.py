@@ -7,6 +7,7 @@ The compute lives in ``libsdnq.so`` (hand-written CUDA behind the C ABI of
 * ``sdnq_rotquant_act``         online activation rotate + per-token int8 quantize
 * ``sdnq_int8_linear``          int8 x int8 -> int32 tensor-core matmul + fp32 de-quant epilogue
 * ``sdnq_int8_linear_fused``    rotate + quantize and the int8 linear in one launch
+* ``sdnq_int8_linear_fused_plan`` whether that call takes one launch or two for a shape
 * ``sdnq_int8_linear_gelu``     the same with GELU fused into the epilogue (MLP up-projection)
 * ``sdnq_int8_linear_lora``     the same plus the bf16 LoRA side term
 * ``sdnq_int8_linear_grad_input`` input gradient through the frozen rotated int8 base
@@ -20,7 +21,8 @@ The compute lives in ``libsdnq.so`` (hand-written CUDA behind the C ABI of
 from ._native import (SdnqError, lib, sdnq_attention_int8qk, sdnq_device_status,
                       sdnq_fp8_linear, sdnq_gelu_bf16,
                       sdnq_int8_linear, sdnq_rotquant_fp8,
-                      sdnq_int8_grad_input_gemm, sdnq_int8_linear_fused, sdnq_int8_linear_gelu,
+                      sdnq_int8_grad_input_gemm, sdnq_int8_linear_fused,
+                      sdnq_int8_linear_fused_plan, sdnq_int8_linear_gelu,
                       sdnq_int8_linear_grad_input, sdnq_int8_linear_lora,
                       sdnq_int8_linear_lora_noalloc, sdnq_rotate_quant_weight,
                       sdnq_quant_grad_output, sdnq_rotquant_act, sdnq_selftest_wait_timeout,
@@ -30,7 +32,8 @@ __all__ = [
     "SdnqError", "lib", "linear", "sdnq_attention_int8qk", "sdnq_device_status",
     "sdnq_fp8_linear", "sdnq_gelu_bf16",
     "sdnq_int8_linear", "sdnq_rotquant_fp8",
-    "sdnq_int8_grad_input_gemm", "sdnq_int8_linear_fused", "sdnq_int8_linear_gelu",
+    "sdnq_int8_grad_input_gemm", "sdnq_int8_linear_fused", "sdnq_int8_linear_fused_plan",
+    "sdnq_int8_linear_gelu",
     "sdnq_int8_linear_grad_input",
     "sdnq_int8_linear_lora", "sdnq_quant_grad_output",
     "sdnq_int8_linear_lora_noalloc",

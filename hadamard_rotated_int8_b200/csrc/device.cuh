@@ -474,6 +474,28 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank)
     return r;
 }
 
+// 2-D tiled TMA load into this CTA's shared memory whose completion (bytes) is counted on
+// an mbarrier of either CTA of the pair (`mbar_cluster`, a shared::cluster address). Same
+// alignment rules as tma_load_2d.
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap *map,
+                                                 uint32_t mbar_cluster, int32_t x, int32_t y)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(mbar_cluster), "r"(x), "r"(y)
+        : "memory");
+}
+
+// Sleeps for about `ns` nanoseconds of global time (bounded drain of copies whose
+// completion this thread cannot observe).
+__device__ __forceinline__ void sleep_ns_bounded(uint64_t ns)
+{
+    const uint64_t t0 = global_timer_ns();
+    while (global_timer_ns() - t0 < ns)
+        __nanosleep(1000);
+}
+
 // Every thread of both CTAs of the cluster arrives, then waits for all of them.
 __device__ __forceinline__ void cluster_sync_all()
 {

@@ -14,16 +14,19 @@
 // quantized matmul and dequantize_fp32; "ConvRot / Hadamard SDNQ").
 //
 // Roles (320 threads per CTA):
-//   warp 0      TMA producer of this CTA's halves; its loads complete on this CTA's own
-//               full barrier, so a CTA can always wait for its own copies in flight.
-//   warp 1      rank 0: allocates tensor memory (both CTAs allocate the same columns) and
-//               issues the pair's MMAs once its own stage and the peer's are full.
-//               rank 1: forwards each of its completed stages to rank 0 (a remote arrive
-//               on rank 0's peer-full barrier).
+//   warp 0      TMA producer of this CTA's halves. The loads of both CTAs complete on rank
+//               0's full barrier (the cta_group::2 form of the tensor copy), whose
+//               expected byte count rank 0 sets for both halves.
+//   warp 1      both CTAs allocate the same tensor-memory columns; rank 0 issues the
+//               pair's MMAs once a stage is full.
 //   warps 2..9  epilogue of this CTA's 128 rows; they release the accumulator buffer with a
 //               remote arrive on rank 0's tensor-empty barrier (16 arrivals per use).
 // The MMA completion (tcgen05.commit, multicast to both CTAs) frees each stage in both CTAs
 // and announces each finished accumulator buffer to both epilogues. Every wait is bounded.
+// A producer that gives up drains its own copies: rank 0 by waiting (bounded) on its full
+// barriers; rank 1, whose copies complete on rank 0's barriers, by a bounded sleep far
+// longer than a copy takes, before the final cluster barrier (until which rank 0's barriers
+// stay valid).
 #pragma once
 
 #include "gemm.cuh"
@@ -54,8 +57,8 @@ struct PairConfig {
     static constexpr int SCALE_OFF = OUT_OFF + EPI_WARPS * STAGE_OUT_BYTES;
     static constexpr int LUT_OFF = SCALE_OFF + EPI_WARPS * SCALE_BYTES;
     static constexpr int BAR_OFF = LUT_OFF + LUT_BYTES;
-    // full[S], empty[S], pfull[S], tfull[2], tempty[2], drain; then tmem base + abort flag
-    static constexpr int BAR_BYTES = (3 * STAGES + 5) * 8;
+    // full[S], empty[S], tfull[2], tempty[2], drain; then tmem base + abort flag
+    static constexpr int BAR_BYTES = (2 * STAGES + 5) * 8;
     static constexpr int SMEM_BYTES = 1024 + BAR_OFF + BAR_BYTES + 16;
     static_assert(STAGES >= 3, "pipeline depth");
     static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
@@ -78,10 +81,9 @@ __global__ void __launch_bounds__(320, 1)
     const uint32_t bar0 = base + C::BAR_OFF;
     auto full_bar = [&](int s) { return bar0 + 8u * s; };
     auto empty_bar = [&](int s) { return bar0 + 8u * (C::STAGES + s); };
-    auto pfull_bar = [&](int s) { return bar0 + 8u * (2 * C::STAGES + s); };
-    auto tfull_bar = [&](int b) { return bar0 + 8u * (3 * C::STAGES + b); };
-    auto tempty_bar = [&](int b) { return bar0 + 8u * (3 * C::STAGES + 2 + b); };
-    const uint32_t drain_bar = bar0 + 8u * (3 * C::STAGES + 4);
+    auto tfull_bar = [&](int b) { return bar0 + 8u * (2 * C::STAGES + b); };
+    auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * C::STAGES + 2 + b); };
+    const uint32_t drain_bar = bar0 + 8u * (2 * C::STAGES + 4);
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C::BAR_OFF + C::BAR_BYTES);
     volatile int *abort = reinterpret_cast<volatile int *>(tmem_holder + 1);
 
@@ -96,7 +98,6 @@ __global__ void __launch_bounds__(320, 1)
         for (int s = 0; s < C::STAGES; ++s) {
             mbar_init(full_bar(s), 1);
             mbar_init(empty_bar(s), 1);
-            mbar_init(pfull_bar(s), 1);
         }
         for (int b = 0; b < C::NBUF; ++b) {
             mbar_init(tfull_bar(b), 1);
@@ -132,6 +133,7 @@ __global__ void __launch_bounds__(320, 1)
             uint32_t phase = 0;
             int issued = 0;
             bool ok = true;
+            const uint32_t leader_full0 = mapa_shared(full_bar(0), 0u);
             for (int tile = pair; ok && tile < p.num_tiles; tile += npairs) {
                 const int m0 = (tile % p.num_m_blocks) * 2 * C::BM + static_cast<int>(rank) * C::BM;
                 const int nr0 = (tile / p.num_m_blocks) * C::BN + static_cast<int>(rank) * (C::BN / 2);
@@ -142,18 +144,21 @@ __global__ void __launch_bounds__(320, 1)
                         break;
                     }
                     const uint32_t sa = base + stage * C::STAGE_BYTES;
-                    mbar_arrive_expect_tx(full_bar(stage), C::STAGE_BYTES);
+                    const uint32_t sb = sa + C::A_BYTES;
+                    const uint32_t fb = leader_full0 + 8u * stage;   // rank 0's full barrier
+                    if (leader)
+                        mbar_arrive_expect_tx(full_bar(stage), 2 * C::STAGE_BYTES);
                     if (!LORA || kb < p.num_kb) {
-                        tma_load_2d(sa, &tmA, full_bar(stage), kb * C::BK, m0);
-                        tma_load_2d(sa + C::A_BYTES, &tmB, full_bar(stage), kb * C::BK, nr0);
+                        tma_load_2d_pair(sa, &tmA, fb, kb * C::BK, m0);
+                        tma_load_2d_pair(sb, &tmB, fb, kb * C::BK, nr0);
                     } else {
                         // LoRA chunk c: this CTA's U rows [128 x 64 rank] (K-major) into the A
                         // slot, its 128 columns of B [64 rank x 128] (N-major) as two 64-column
                         // boxes into the B slot
                         const int c = kb - p.num_kb;
-                        tma_load_2d(sa, &tmU, full_bar(stage), c * 64, m0);
-                        tma_load_2d(sa + C::A_BYTES, &tmL, full_bar(stage), nr0, c * 64);
-                        tma_load_2d(sa + C::A_BYTES + 8192, &tmL, full_bar(stage), nr0 + 64, c * 64);
+                        tma_load_2d_pair(sa, &tmU, fb, c * 64, m0);
+                        tma_load_2d_pair(sb, &tmL, fb, nr0, c * 64);
+                        tma_load_2d_pair(sb + 8192, &tmL, fb, nr0 + 64, c * 64);
                     }
                     ++issued;
                     if (++stage == C::STAGES) {
@@ -163,17 +168,21 @@ __global__ void __launch_bounds__(320, 1)
                 }
             }
             if (!ok) {
-                // drain: wait (bounded) for this CTA's copies of the last stages issued
-                const int n = issued < C::STAGES ? issued : C::STAGES;
-                int s = stage;
-                uint32_t ph = phase;
-                for (int i = 0; i < n; ++i) {
-                    if (--s < 0) {
-                        s = C::STAGES - 1;
-                        ph ^= 1u;
+                if (leader) {
+                    // drain: wait (bounded) for the copies of the last stages issued
+                    const int n = issued < C::STAGES ? issued : C::STAGES;
+                    int s = stage;
+                    uint32_t ph = phase;
+                    for (int i = 0; i < n; ++i) {
+                        if (--s < 0) {
+                            s = C::STAGES - 1;
+                            ph ^= 1u;
+                        }
+                        volatile int no_abort = 0;
+                        mbar_wait_bounded(full_bar(s), ph, &no_abort, p.timeout_ns);
                     }
-                    volatile int no_abort = 0;
-                    mbar_wait_bounded(full_bar(s), ph, &no_abort, p.timeout_ns);
+                } else {
+                    sleep_ns_bounded(1000000);   // 1 ms: this CTA's copies have landed
                 }
             }
         }
@@ -195,8 +204,7 @@ __global__ void __launch_bounds__(320, 1)
                 tc_fence_after_sync();
                 const uint32_t d_acc = tmem_base + buf * C::ACC_COLS;
                 for (int kb = 0; kb < p.num_kb; ++kb) {
-                    if (!mbar_wait_bounded(full_bar(stage), phase, abort, p.timeout_ns) ||
-                        !mbar_wait_bounded_cluster(pfull_bar(stage), phase, abort, p.timeout_ns)) {
+                    if (!mbar_wait_bounded(full_bar(stage), phase, abort, p.timeout_ns)) {
                         ok = false;
                         break;
                     }
@@ -222,8 +230,7 @@ __global__ void __launch_bounds__(320, 1)
                     constexpr uint32_t IDESC_BF = idesc_bf16_f32(256, C::BN, true);
                     const uint32_t d_lora = d_acc + C::BN;
                     for (int c = 0; ok && c < p.lora_chunks; ++c) {
-                        if (!mbar_wait_bounded(full_bar(stage), phase, abort, p.timeout_ns) ||
-                            !mbar_wait_bounded_cluster(pfull_bar(stage), phase, abort, p.timeout_ns)) {
+                        if (!mbar_wait_bounded(full_bar(stage), phase, abort, p.timeout_ns)) {
                             ok = false;
                             break;
                         }
@@ -251,26 +258,6 @@ __global__ void __launch_bounds__(320, 1)
             tc_commit_pair(drain_bar, 0x1);
             volatile int no_abort = 0;
             mbar_wait_bounded(drain_bar, 0u, &no_abort, p.timeout_ns);
-        } else if (lane == 0) {
-            // -------------------------------------------------------- stage forwarder (rank 1)
-            const uint32_t peer_pfull0 = mapa_shared(pfull_bar(0), 0u);
-            int stage = 0;
-            uint32_t phase = 0;
-            bool ok = true;
-            const int steps = p.num_kb + (LORA ? p.lora_chunks : 0);
-            for (int tile = pair; ok && tile < p.num_tiles; tile += npairs) {
-                for (int kb = 0; kb < steps; ++kb) {
-                    if (!mbar_wait_bounded(full_bar(stage), phase, abort, p.timeout_ns)) {
-                        ok = false;
-                        break;
-                    }
-                    mbar_arrive_remote(peer_pfull0 + 8u * stage);
-                    if (++stage == C::STAGES) {
-                        stage = 0;
-                        phase ^= 1u;
-                    }
-                }
-            }
         }
     } else {
         // ------------------------------------------------------------ epilogue (warps 2..9)

@@ -257,6 +257,24 @@ __device__ __forceinline__ uint2 quant8(const float (&z)[8], float s_z, float rc
                             __float_as_uint(f[7])));
 }
 
+// The row scale s_z = RN(amax / D) for the grid's largest code D (127 for int8, 448 for
+// e4m3), without a division: with y = RN(1 / D) and q0 = RN(amax * y), the residual
+// amax - q0 * D is exact in one fused multiply-add and RN(q0 + r * y) is the IEEE quotient
+// (Markstein's correction, as in quant8; checked on every fp32 input of two binades, which
+// covers all inputs whose intermediates stay normal). Tiny maxima take the IEEE division.
+template <int D>
+__device__ __forceinline__ float div_by_grid(float amax)
+{
+    static_assert(D == 127 || D == 448, "the int8 and e4m3 grids");
+    if (!(amax >= 0x1p-100f))
+        return __fdiv_rn(amax, static_cast<float>(D));
+    // RN(1 / D): 0x3c010204 for 127, 0x3b124925 for 448
+    const float y = __uint_as_float(D == 127 ? 0x3c010204u : 0x3b124925u);
+    const float q0 = __fmul_rn(amax, y);
+    const float r = __fmaf_rn(-q0, static_cast<float>(D), amax);
+    return __fmaf_rn(r, y, q0);
+}
+
 // e4m3 codes of two fp32 values (round to nearest even, saturating at +-448), low byte = lo
 __device__ __forceinline__ uint32_t e4m3x2(float lo, float hi)
 {
@@ -736,7 +754,7 @@ __global__ void __launch_bounds__(512) rotquant_run_kernel(const RotquantRunPara
         if (slot < p.rows)
             s_max[((it + 2) % 3) * p.rows + slot] = 0u;          // the buffer of iteration it + 2
         amax = active ? __uint_as_float(mx[row_local]) : 0.0f;
-        const float s_z = __fdiv_rn(amax, FP8 ? 448.0f : 127.0f);
+        const float s_z = div_by_grid<FP8 ? 448 : 127>(amax);
         const bool zero = !(amax > 0.0f);
         if (row_ok && run == 0)
             p.s[row] = zero ? 0.0f : __fmul_rn(s_z, p.c_g);
