@@ -204,8 +204,11 @@ sdnq_status validate_rotquant(const void *x, int64_t rows, int64_t K, int64_t ld
 // Rows of at most 16 chunks go to the persistent, prefetching kernel (grid = resident
 // CTAs); longer rows to the two-pass kernel with one CTA per row.
 // Block shape of the run-per-lane kernel: `warps` warps hold `rows` = floor(32 warps / rpr)
-// rows of rpr runs of 64 elements; the warp count in 4..16 that leaves the fewest lanes idle
-// (the smallest such count). rows == 0 means the row is too long for it (rpr > 512).
+// rows of rpr runs of 64 elements. Small blocks keep more of them resident per SM, so that
+// one block's row barrier overlaps the others' work (measured: 2-warp blocks beat 4- and
+// 8-warp ones on 16384 x 4096); the shape is the smallest warp count in 2..16 that leaves at
+// most a tenth of the lanes idle, else the one that leaves the fewest. rows == 0 means the
+// row is too long for the kernel (rpr > 512).
 struct RunShape {
     int warps = 0;
     int rows = 0;
@@ -215,11 +218,13 @@ RunShape run_shape(int64_t rpr)
 {
     RunShape best;
     double best_used = -1.0;
-    for (int w = 4; w <= 16; ++w) {
+    for (int w = 2; w <= 16; ++w) {
         const int64_t rows = 32 * w / rpr;
         if (rows < 1)
             continue;
         const double used = static_cast<double>(rows * rpr) / (32.0 * w);
+        if (used >= 0.9)
+            return RunShape{w, static_cast<int>(rows)};
         if (used > best_used + 1e-9) {
             best.warps = w;
             best.rows = static_cast<int>(rows);
