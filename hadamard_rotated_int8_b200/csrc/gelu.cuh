@@ -97,32 +97,36 @@ __device__ __forceinline__ uint32_t gelu_lut_input(int i)
 __device__ __noinline__ uint32_t gelu_bf16_bits_rare(uint32_t b) { return gelu_bf16_bits(b); }
 
 // Table-form GELU of the 16 bf16 patterns packed in w[8] (two per word), in place; `lut`
-// is the table in shared memory. Branch-free apart from the rare inputs (subnormal, NaN,
-// Inf), so that the table loads are independent and in flight together.
+// is the table in shared memory. The hot path is only the index, one table load and an
+// out-of-table flag per value, all independent so that the loads are in flight together;
+// the closed forms (tiny, |x| >= 16, zero) and the exact function (subnormal, NaN, Inf) run
+// only for a group of 16 that holds such a value.
 __device__ __forceinline__ void gelu_bf16x16_lut(uint32_t *w, const uint16_t *lut)
 {
+    constexpr uint32_t kLo = static_cast<uint32_t>(kGeluLutExpLo) << 7;   // first magnitude
     uint32_t r[16];
-    bool rare = false;
+    bool out = false;
 #pragma unroll
     for (int k = 0; k < 16; ++k) {
         const uint32_t b = (k & 1) ? (w[k >> 1] >> 16) : (w[k >> 1] & 0xffffu);
-        const uint32_t e = (b >> 7) & 0xffu;
-        const uint32_t sign = b >> 15;
-        const bool in_tab = e - kGeluLutExpLo <= static_cast<uint32_t>(kGeluLutExpHi - kGeluLutExpLo);
-        const uint32_t i = in_tab ? sign * kGeluLutHalf + ((e - kGeluLutExpLo) << 7) + (b & 127u) : 0u;
-        // outside the table: x >= 16 -> x, x <= -16 -> -0, tiny normal -> x/2, +-0 -> +-0
-        const uint32_t alt = e > kGeluLutExpHi ? (sign ? 0x8000u : b) : (e >= 2u ? b - 0x80u : b);
-        const uint32_t t = lut[i];
-        r[k] = in_tab ? t : alt;
-        rare |= e == 255u || (e < 2u && (b & 0x7fffu) != 0u);
+        const uint32_t d = (b & 0x7fffu) - kLo;            // offset inside the table's half
+        const bool in_tab = d < static_cast<uint32_t>(kGeluLutHalf);
+        const uint32_t i = d + (b >> 15) * static_cast<uint32_t>(kGeluLutHalf);
+        r[k] = lut[in_tab ? i : 0u];
+        out |= !in_tab;
     }
-    if (rare) {
+    if (out) {
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
             const uint32_t b = (k & 1) ? (w[k >> 1] >> 16) : (w[k >> 1] & 0xffffu);
             const uint32_t e = (b >> 7) & 0xffu;
+            const uint32_t sign = b >> 15;
+            if (e - kGeluLutExpLo <= static_cast<uint32_t>(kGeluLutExpHi - kGeluLutExpLo))
+                continue;   // in the table
             if (e == 255u || (e < 2u && (b & 0x7fffu) != 0u))
-                r[k] = gelu_bf16_bits_rare(b);
+                r[k] = gelu_bf16_bits_rare(b);     // subnormal, NaN, Inf: the exact function
+            else   // x >= 16 -> x, x <= -16 -> -0, tiny normal -> x/2, +-0 -> +-0
+                r[k] = e > kGeluLutExpHi ? (sign ? 0x8000u : b) : (e >= 2u ? b - 0x80u : b);
         }
     }
 #pragma unroll

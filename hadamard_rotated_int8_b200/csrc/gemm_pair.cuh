@@ -13,14 +13,15 @@
 // Sources: as the single-SM kernel ("SDNQ: SD.Next Quantization Engine" README, INT8
 // quantized matmul and dequantize_fp32; "ConvRot / Hadamard SDNQ").
 //
-// Roles (320 threads per CTA):
+// Roles (320 threads per CTA; 576 with GELU):
 //   warp 0      TMA producer of this CTA's halves. The loads of both CTAs complete on rank
 //               0's full barrier (the cta_group::2 form of the tensor copy), whose
 //               expected byte count rank 0 sets for both halves.
 //   warp 1      both CTAs allocate the same tensor-memory columns; rank 0 issues the
 //               pair's MMAs once a stage is full.
-//   warps 2..9  epilogue of this CTA's 128 rows; they release the accumulator buffer with a
-//               remote arrive on rank 0's tensor-empty barrier (16 arrivals per use).
+//   warps 2..   epilogue of this CTA's 128 rows (8 warps; 16 with the GELU table); they
+//               release the accumulator buffer with a remote arrive on rank 0's
+//               tensor-empty barrier (one arrival per epilogue warp of both CTAs).
 // The MMA completion (tcgen05.commit, multicast to both CTAs) frees each stage in both CTAs
 // and announces each finished accumulator buffer to both epilogues. Every wait is bounded.
 // A producer that gives up drains its own copies: rank 0 by waiting (bounded) on its full
@@ -30,6 +31,10 @@
 #pragma once
 
 #include "gemm.cuh"
+
+#ifndef SDNQ_GELU_EPI_WARPS
+#define SDNQ_GELU_EPI_WARPS 16
+#endif
 
 namespace sdnq {
 
@@ -44,9 +49,11 @@ struct PairConfig {
     static constexpr int ACC_COLS = LORA ? 2 * BN : BN;  // int32 (+ fp32 LoRA) columns per buffer
     static constexpr int NBUF = LORA ? 1 : 2;
     static constexpr int TMEM_COLS = NBUF * ACC_COLS;    // 512
-    static constexpr int THREADS = 320;
-    static constexpr int EPI_WARPS = 8;
-    static constexpr int EPI_COLS = BN / 2;
+    // the GELU epilogue (table lookups, integer-heavy) gets four warps per TMEM lane quarter,
+    // the others two
+    static constexpr int EPI_WARPS = GELU ? SDNQ_GELU_EPI_WARPS : 8;
+    static constexpr int THREADS = 64 + 32 * EPI_WARPS;
+    static constexpr int EPI_COLS = BN / (EPI_WARPS / 4);
     static constexpr int STAGE_OUT_BYTES = 32 * 64;
     static constexpr int LUT_BYTES = GELU ? kGeluLutBytes : 0;
     static constexpr int SCALE_BYTES = EPI_COLS * 8;
@@ -65,7 +72,7 @@ struct PairConfig {
 };
 
 template <bool GELU, bool FP8, bool LORA>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(PairConfig<GELU, LORA>::THREADS, 1)
     gemm_s8_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB,
                         const __grid_constant__ CUtensorMap tmU,

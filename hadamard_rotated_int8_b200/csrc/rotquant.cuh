@@ -668,14 +668,10 @@ __global__ void __launch_bounds__(512) rotquant_run_kernel(const RotquantRunPara
     const int32_t e0 = run * 64;
     const int64_t n_blocks = (p.M + p.rows - 1) / p.rows;
 
-    // the lanes of this lane's row inside the warp (a contiguous range): their maximum is
-    // one redux over that mask (non-negative fp32 values order like their bit patterns)
-    const int32_t warp_lo = warp * 32;
-    const int32_t seg_lo = max(row_local * p.rpr, warp_lo) - warp_lo;
-    const int32_t seg_hi = min((row_local + 1) * p.rpr, warp_lo + 32) - 1 - warp_lo;
-    const uint32_t seg_mask = (seg_hi >= 31 ? 0xffffffffu : ((1u << (seg_hi + 1)) - 1u)) &
-                              ~((1u << seg_lo) - 1u);
-    const bool seg_first = active && static_cast<int32_t>(lane) == seg_lo;
+    // segmented maximum over the lanes of this lane's row inside the warp: step d takes
+    // lane + d's value when that lane holds the same row
+    const int32_t row_end = (row_local + 1) * p.rpr;   // first slot of the next row
+    const bool seg_first = active && (lane == 0u || run == 0);
     for (int32_t i = slot; i < 3 * p.rows; i += static_cast<int32_t>(blockDim.x))
         s_max[i] = 0u;
     __syncthreads();
@@ -745,10 +741,15 @@ __global__ void __launch_bounds__(512) rotquant_run_kernel(const RotquantRunPara
 #pragma unroll
         for (int i = 0; i < 64; i += 2)
             amax = max3_abs(amax, v[i], v[i + 1]);
-        const uint32_t seg_max = __reduce_max_sync(seg_mask, __float_as_uint(amax));
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const float o = __shfl_down_sync(0xffffffffu, amax, d);
+            if (static_cast<int32_t>(lane) + d < 32 && slot + d < row_end)
+                amax = fmaxf(amax, o);
+        }
         uint32_t *mx = s_max + (it % 3) * p.rows;
         if (seg_first)
-            atomicMax(mx + row_local, seg_max);
+            atomicMax(mx + row_local, __float_as_uint(amax));   // amax >= 0: bits order as values
         __syncthreads();
         if (slot < p.rows)
             s_max[((it + 2) % 3) * p.rows + slot] = 0u;          // the buffer of iteration it + 2
