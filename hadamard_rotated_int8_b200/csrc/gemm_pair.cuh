@@ -13,13 +13,13 @@
 // Sources: as the single-SM kernel ("SDNQ: SD.Next Quantization Engine" README, INT8
 // quantized matmul and dequantize_fp32; "ConvRot / Hadamard SDNQ").
 //
-// Roles (320 threads per CTA; 576 with GELU):
+// Roles (320 threads per CTA; 576 with GELU or LoRA):
 //   warp 0      TMA producer of this CTA's halves. The loads of both CTAs complete on rank
 //               0's full barrier (the cta_group::2 form of the tensor copy), whose
 //               expected byte count rank 0 sets for both halves.
 //   warp 1      both CTAs allocate the same tensor-memory columns; rank 0 issues the
 //               pair's MMAs once a stage is full.
-//   warps 2..   epilogue of this CTA's 128 rows (8 warps; 16 with the GELU table); they
+//   warps 2..   epilogue of this CTA's 128 rows (8 warps; 16 with GELU or LoRA); they
 //               release the accumulator buffer with a remote arrive on rank 0's
 //               tensor-empty barrier (one arrival per epilogue warp of both CTAs).
 // The MMA completion (tcgen05.commit, multicast to both CTAs) frees each stage in both CTAs
@@ -32,8 +32,8 @@
 
 #include "gemm.cuh"
 
-#ifndef SDNQ_GELU_EPI_WARPS
-#define SDNQ_GELU_EPI_WARPS 16
+#ifndef SDNQ_WIDE_EPI_WARPS
+#define SDNQ_WIDE_EPI_WARPS 16
 #endif
 
 namespace sdnq {
@@ -49,9 +49,10 @@ struct PairConfig {
     static constexpr int ACC_COLS = LORA ? 2 * BN : BN;  // int32 (+ fp32 LoRA) columns per buffer
     static constexpr int NBUF = LORA ? 1 : 2;
     static constexpr int TMEM_COLS = NBUF * ACC_COLS;    // 512
-    // the GELU epilogue (table lookups, integer-heavy) gets four warps per TMEM lane quarter,
-    // the others two
-    static constexpr int EPI_WARPS = GELU ? SDNQ_GELU_EPI_WARPS : 8;
+    // four epilogue warps per TMEM lane quarter for the GELU table lookups (integer-heavy)
+    // and for LoRA (one accumulator buffer: the drain is not hidden under the next tile's
+    // MMAs, so a faster drain is time saved); two for the plain epilogue
+    static constexpr int EPI_WARPS = (GELU || LORA) ? SDNQ_WIDE_EPI_WARPS : 8;
     static constexpr int THREADS = 64 + 32 * EPI_WARPS;
     static constexpr int EPI_COLS = BN / (EPI_WARPS / 4);
     static constexpr int STAGE_OUT_BYTES = 32 * 64;

@@ -7,7 +7,8 @@ not acceptable where they run. sdnq_int8_linear_lora_noalloc serves them by keep
 LoRA intermediate u in a fixed array inside the library. Here it is called through the C ABI
 twice in a row, on two different problems, and each result must be bit for bit that of
 sdnq_int8_linear_lora given a caller-allocated u_ws (both run the same kernels on the same
-inputs), and within one bf16 ulp of the CPU oracle. The Python wrapper is exercised too.
+inputs), and within the LoRA bound of the CPU oracle that the parity tests use. The Python
+wrapper is exercised too.
 
 This file is collected last so that a run stopping at its first failure has run every
 other test; it also passes on its own in a fresh process.
@@ -21,6 +22,7 @@ import torch
 import oracle
 import hadamard_rotated_int8_b200 as sd
 from hadamard_rotated_int8_b200 import _build, _native, synthetic
+from tests.test_gpu_parity import check_lora_tolerance
 
 pytestmark = pytest.mark.gpu
 
@@ -69,12 +71,11 @@ def _with_workspace(p):
                                     p["A"], p["B"], p["scale"], u_ws=u)
 
 
-def _oracle_out(p):
+def _oracle(p):
     c = p["case"]
-    ref = oracle.linear(synthetic.bits(c.x), *oracle.rotate_quantize(synthetic.bits(c.W), 256),
-                        256, bias_bits=synthetic.bits(c.bias), A_bits=synthetic.bits(c.A),
-                        B_bits=synthetic.bits(c.B), lora_scale=c.lora_scale)
-    return ref["out"]
+    return oracle.linear(synthetic.bits(c.x), *oracle.rotate_quantize(synthetic.bits(c.W), 256),
+                         256, bias_bits=synthetic.bits(c.bias), A_bits=synthetic.bits(c.A),
+                         B_bits=synthetic.bits(c.B), lora_scale=c.lora_scale)
 
 
 def test_noalloc_matches_workspace_entry_point_twice():
@@ -93,7 +94,15 @@ def test_noalloc_matches_workspace_entry_point_twice():
         g, w = _bits(got), _bits(want)
         assert np.array_equal(g, w), \
             f"no-alloc output differs from the workspace call in {np.count_nonzero(g != w)} places"
-        assert _ulp_diff(g, _oracle_out(p)).max() <= 1, "no-alloc output vs the oracle"
+        # against the oracle: the LoRA bound of the parity tests (one bf16 ulp plus the fp32
+        # accumulation bound of the adapter terms; outputs where the sum cancels may sit more
+        # than one ulp away)
+        ref = _oracle(p)
+        u = torch.empty((p["M"], p["rank"]), dtype=torch.bfloat16, device="cuda")
+        sd.sdnq_int8_linear_lora(p["qx"], p["sx"], p["qW"], p["sW"], p["bias"], p["x"], p["A"],
+                                 p["B"], p["scale"], u_ws=u)
+        torch.cuda.synchronize()
+        check_lora_tolerance(p["case"], _bits(u), g, ref, p["scale"])
 
 
 def test_noalloc_python_wrapper_after_a_larger_call():
