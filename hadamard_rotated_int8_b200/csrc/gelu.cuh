@@ -78,8 +78,9 @@ __device__ __forceinline__ uint32_t gelu_bf16_bits(uint32_t xb)
 //     below half the smallest bf16 subnormal, the result is -0;
 //   * +-0: +-0.
 // The 3584 inputs in between (both signs, biased exponents 117..130, all 128 mantissas) go
-// through a table built with gelu_bf16_bits; subnormal, NaN and Inf inputs take
-// gelu_bf16_bits directly.
+// through a table built with gelu_bf16_bits. Below 2^-125 (subnormal and the smallest normal
+// binade) Phi(x) rounds to 0.5 even in fp64, so the result is x/2 rounded half to even on
+// the subnormal grid; +Inf gives +Inf, -Inf and NaN give NaN (0x7fc0).
 constexpr int kGeluLutExpLo = 117;                    // 2^-10
 constexpr int kGeluLutExpHi = 130;                    // [8, 16)
 constexpr int kGeluLutHalf = (kGeluLutExpHi - kGeluLutExpLo + 1) * 128;
@@ -94,13 +95,36 @@ __device__ __forceinline__ uint32_t gelu_lut_input(int i)
     return (sign << 15) | ((kGeluLutExpLo + (r >> 7)) << 7) | (r & 127u);
 }
 
-__device__ __noinline__ uint32_t gelu_bf16_bits_rare(uint32_t b) { return gelu_bf16_bits(b); }
+
+// The table, built once per device by gelu_lut_build_kernel (the library launches it, and
+// waits for it, on the first call that needs it), then copied into each GEMM CTA's shared
+// memory. Keeping the exact evaluation out of the GEMM kernels keeps their register
+// allocation to what the epilogue needs.
+__device__ __align__(16) uint16_t g_gelu_lut[kGeluLutEntries];
+
+__global__ void gelu_lut_build_kernel()
+{
+    const int i = static_cast<int>(blockIdx.x * blockDim.x + threadIdx.x);
+    if (i < kGeluLutEntries)
+        g_gelu_lut[i] = static_cast<uint16_t>(gelu_bf16_bits(gelu_lut_input(i)));
+}
+
+// Copies the table into shared memory with `nthreads` threads of index `t` (16 bytes each);
+// the caller synchronises those threads before the first lookup.
+__device__ __forceinline__ void gelu_lut_load(uint16_t *lut, int t, int nthreads)
+{
+    const uint4 *src = reinterpret_cast<const uint4 *>(g_gelu_lut);
+    uint4 *dst = reinterpret_cast<uint4 *>(lut);
+    for (int i = t; i < kGeluLutBytes / 16; i += nthreads)
+        dst[i] = src[i];
+}
+
 
 // Table-form GELU of the 16 bf16 patterns packed in w[8] (two per word), in place; `lut`
 // is the table in shared memory. The hot path is only the index, one table load and an
 // out-of-table flag per value, all independent so that the loads are in flight together;
-// the closed forms (tiny, |x| >= 16, zero) and the exact function (subnormal, NaN, Inf) run
-// only for a group of 16 that holds such a value.
+// the closed forms of the other inputs (tiny and subnormal: x/2 rounded half to even;
+// |x| >= 16: x or -0; zero; Inf, NaN) run only for a group of 16 that holds such a value.
 __device__ __forceinline__ void gelu_bf16x16_lut(uint32_t *w, const uint16_t *lut)
 {
     constexpr uint32_t kLo = static_cast<uint32_t>(kGeluLutExpLo) << 7;   // first magnitude
@@ -123,10 +147,16 @@ __device__ __forceinline__ void gelu_bf16x16_lut(uint32_t *w, const uint16_t *lu
             const uint32_t sign = b >> 15;
             if (e - kGeluLutExpLo <= static_cast<uint32_t>(kGeluLutExpHi - kGeluLutExpLo))
                 continue;   // in the table
-            if (e == 255u || (e < 2u && (b & 0x7fffu) != 0u))
-                r[k] = gelu_bf16_bits_rare(b);     // subnormal, NaN, Inf: the exact function
-            else   // x >= 16 -> x, x <= -16 -> -0, tiny normal -> x/2, +-0 -> +-0
-                r[k] = e > kGeluLutExpHi ? (sign ? 0x8000u : b) : (e >= 2u ? b - 0x80u : b);
+            if (e == 255u) {           // +Inf -> +Inf; -Inf (-inf * 0) and NaN -> NaN
+                r[k] = ((b & 127u) != 0u || sign) ? 0x7fc0u : 0x7f80u;
+            } else if (e < 2u) {
+                // |x| < 2^-125: Phi(x) is 0.5 to far below the precision, GELU(x) = x / 2
+                // rounded half to even on the subnormal grid (n * 2^-133, n = b & 0x7fff)
+                const uint32_t n = b & 0x7fffu, h = n >> 1;
+                r[k] = (b & 0x8000u) | (h + (n & h & 1u));
+            } else {   // x >= 16 -> x, x <= -16 -> -0, tiny normal -> x/2
+                r[k] = e > kGeluLutExpHi ? (sign ? 0x8000u : b) : b - 0x80u;
+            }
         }
     }
 #pragma unroll

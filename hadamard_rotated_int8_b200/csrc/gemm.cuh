@@ -558,9 +558,8 @@ __global__ void __launch_bounds__(GemmConfig<BN, LORA, GELU, (FUSE_G > 0)>::THRE
         const bool has_bias = p.bias != nullptr;
         uint16_t *lut = reinterpret_cast<uint16_t *>(smem + C::LUT_OFF);
         if constexpr (GELU) {
-            // the GELU table, while the first tile's operands load and multiply
-            for (int i = static_cast<int>(ew * 32u + lane); i < kGeluLutEntries; i += 32 * C::EPI_WARPS)
-                lut[i] = static_cast<uint16_t>(gelu_bf16_bits(gelu_lut_input(i)));
+            // the GELU table (built once per device), while the first tile's operands load
+            gelu_lut_load(lut, static_cast<int>(ew * 32u + lane), 32 * C::EPI_WARPS);
             bar_sync_or(1, 32 * C::EPI_WARPS, false);  // epilogue warps only
         }
         int local = 0;

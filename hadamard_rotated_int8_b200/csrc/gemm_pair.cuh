@@ -280,8 +280,7 @@ __global__ void __launch_bounds__(PairConfig<GELU, LORA>::THREADS, 1)
         const uint32_t leader_tempty0 = mapa_shared(tempty_bar(0), 0u);
         uint16_t *lut = reinterpret_cast<uint16_t *>(smem + C::LUT_OFF);
         if constexpr (GELU) {
-            for (int i = static_cast<int>(ew * 32u + lane); i < kGeluLutEntries; i += 32 * C::EPI_WARPS)
-                lut[i] = static_cast<uint16_t>(gelu_bf16_bits(gelu_lut_input(i)));
+            gelu_lut_load(lut, static_cast<int>(ew * 32u + lane), 32 * C::EPI_WARPS);
             bar_sync_or(1, 32 * C::EPI_WARPS, false);
         }
         int local = 0;

@@ -564,6 +564,24 @@ sdnq_status launch_lora_down(const DeviceInfo &dev, const uint16_t *x, int64_t l
     return launch_status();
 }
 
+// The GELU table in device memory (g_gelu_lut), built once per device: the first call that
+// needs it launches the build kernel on its stream and waits for it, so that later calls on
+// any stream find it complete. A failed build is retried by the next call.
+sdnq_status ensure_gelu_lut(const DeviceInfo &dev, cudaStream_t cs)
+{
+    static PerDeviceCache<1> built;
+    const int ok = built.get(dev.index, 0, [&] {
+        cudaGetLastError();
+        gelu_lut_build_kernel<<<(kGeluLutEntries + 255) / 256, 256, 0, cs>>>();
+        if (cudaGetLastError() != cudaSuccess || cudaStreamSynchronize(cs) != cudaSuccess) {
+            cudaGetLastError();
+            return 0;
+        }
+        return 1;
+    });
+    return ok == 1 ? SDNQ_OK : SDNQ_ERR_CUDA;
+}
+
 sdnq_status run_linear(const int8_t *qx, const float *sx, const int8_t *qW, const float *sW,
                        const uint16_t *bias, const uint16_t *x, int64_t ldx, const uint16_t *A,
                        const uint16_t *B, int32_t rank, float lora_scale, uint16_t *u_ws,
@@ -606,6 +624,8 @@ sdnq_status run_linear(const int8_t *qx, const float *sx, const int8_t *qW, cons
     p.lora_scale = lora_scale;
     p.c_g = 1.0f;
     p.timeout_ns = kDefaultTimeoutNs;
+    if (gelu && (st = ensure_gelu_lut(dev, cs)) != SDNQ_OK)
+        return st;
     if (!lora && M >= kPairMinRows)
         return gelu ? launch_gemm_pair<true, false>(dev, qx, qW, p, cs)
                     : launch_gemm_pair<false, false>(dev, qx, qW, p, cs);

@@ -165,6 +165,9 @@ sdnq_status sdnq_int8_linear_fused_plan(int64_t M, int64_t N, int64_t K, int32_t
  * i.e. bit for bit sdnq_int8_linear followed by sdnq_gelu_bf16 on its output, without the
  * second pass over [M, N] in HBM. Arguments, layouts, alignment and errors are those of
  * sdnq_int8_linear; acc_out (if set) receives the raw accumulators.
+ * The GELU values come from a 7 KB table that the library keeps in device memory: the first
+ * call on a device builds it with a small kernel on `stream` and waits for that kernel (so
+ * make the first call outside any stream capture); later calls only read it.
  */
 sdnq_status sdnq_int8_linear_gelu(const int8_t *qx, const float *sx, const int8_t *qW,
                                   const float *sW, const uint16_t *bias, int64_t M, int64_t N,

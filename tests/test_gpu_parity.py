@@ -309,20 +309,21 @@ def test_gelu_exhaustive_over_finite_bf16():
     assert_equal(bits_of(out).reshape(-1), oracle.gelu_bf16(pats), "gelu, every finite bf16 input")
 
 
-def test_linear_gelu_epilogue_exhaustive_over_finite_bf16():
+@pytest.mark.parametrize("M", [3, 130])
+def test_linear_gelu_epilogue_exhaustive_over_finite_bf16(M):
     """Zero codes make the pre-GELU value exactly the bias, so a bias holding every finite
     bf16 pattern drives the epilogue's GELU (its table and its closed-form ranges) through
-    all of them."""
+    all of them; 3 rows run the single-SM kernel, 130 the CTA-pair kernel."""
     pats = _finite_bf16_patterns()
     N, K = len(pats), 16
-    qx = torch.zeros((3, K), dtype=torch.int8, device="cuda")
+    qx = torch.zeros((M, K), dtype=torch.int8, device="cuda")
     qW = torch.zeros((N, K), dtype=torch.int8, device="cuda")
-    sx = torch.ones(3, dtype=torch.float32, device="cuda")
+    sx = torch.ones(M, dtype=torch.float32, device="cuda")
     sW = torch.ones(N, dtype=torch.float32, device="cuda")
     bias = torch.from_numpy(pats.view(np.int16)).view(torch.bfloat16).cuda()
     out = sd.sdnq_int8_linear_gelu(qx, sx, qW, sW, bias)
     torch.cuda.synchronize()
-    want = oracle.gelu_bf16(oracle.dequant_epilogue(np.zeros((3, N), np.int32), np.ones(3, np.float32),
+    want = oracle.gelu_bf16(oracle.dequant_epilogue(np.zeros((M, N), np.int32), np.ones(M, np.float32),
                                                     np.ones(N, np.float32), bias_bits=pats))
     assert_equal(bits_of(out), want, "fused GELU, every finite bf16 pre-activation")
 
