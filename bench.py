@@ -634,6 +634,8 @@ def main():
                "streams": "copy in / compute / copy out, two buffer sets"}
 
     peaks, peak_src = measured_peaks()
+    # committed ncu summaries are named <stage>_<workload>[_g<group>].md
+    profile_key = args.workload + (f"_g{args.group}" if args.group else "")
     # GEMM rooflines against the published dense INT8 peak of the B200 (the denominator the
     # targets are stated against); the measured cuBLAS bf16 peak x 2 (the nominal int8/bf16
     # ratio) is given beside it: the burst figure for a kernel that ran at full clock, the
@@ -663,7 +665,7 @@ def main():
             "kernel": kernel_of.get(n, gemm_kernel), "bound": "tensor", "achieved": tops,
             "peak": spec_peak, "unit": "TFLOP/s", "frac": tops / spec_peak,
             "traffic": profiled_traffic(n, "attn_kernel" if case.extra.get("attn") else "gemm_s8",
-                                        args.workload),
+                                        profile_key),
             "ops_per_launch": ops_per_gemm, "ms_per_launch": ms,
             "peak_source": ("NVIDIA B200 dense INT8 spec, 4500 TOPS"
                             + (" (int8 QK / bf16 PV mix)" if case.extra.get("attn") else "")),
@@ -701,7 +703,7 @@ def main():
             "kernel": "rotquant_persistent_kernel" if rows_k <= 16384 else "rotquant_kernel",
             "bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
             "frac": gbs / peaks["hbm_gbs"],
-            "traffic": profiled_traffic(n, "rotquant", args.workload),
+            "traffic": profiled_traffic(n, "rotquant", profile_key),
             "bytes_per_launch": nbytes, "row_length": rows_k, "ms_per_launch": ms,
             "peak_source": f"{peak_src} copy bandwidth", "timing": note,
         }
