@@ -125,6 +125,21 @@ def rotquant_bytes(M, K):
     return M * K * 2 + M * K + M * 4   # read bf16, write int8 codes, write fp32 scale
 
 
+def rotquant_kernel_name(case, rows_k, grad, fp8):
+    """The quantizer kernel the library launches for rows of `rows_k` elements (the run-per-lane
+    kernel up to 512 runs of 64; the input gradient's column-multiplier mode on the
+    chunk-per-warp kernels)."""
+    if case.extra.get("attn"):
+        return "attention quantizers (smooth_k means, q and k short-row quantizers)"
+    f = str(fp8).lower()
+    if grad:
+        kind = "rotquant_persistent_kernel" if (rows_k + 1023) // 1024 <= 16 else "rotquant_kernel"
+        return f"{kind}<{case.g},true,{f}>"
+    if rows_k <= 32768:
+        return f"rotquant_run_kernel<{case.g},{f},V8>"
+    return f"rotquant_kernel<{case.g},false,{f}>"
+
+
 class Step:
     """Device buffers and the stages of one step of a workload."""
 
@@ -650,12 +665,30 @@ def main():
         measured_int8 = 2.0 / (1.0 / measured_int8 + 1.0 / bf16_peak)
         spec_peak = 2.0 / (1.0 / INT8_SPEC_TOPS + 1.0 / (INT8_SPEC_TOPS / 2))
     grad = args.workload.startswith("grad_")
-    gemm_kernel = ("attn_kernel" if case.extra.get("attn") else
-                   "gemm_s8_kernel_e4m3" if args.workload.startswith("fp8_") else
-                   "gemm_s8_kernel_grad_input" if grad else
-                   "gemm_s8_kernel_fused_quantizer" if "fused" in stage_ms else
-                   "gemm_s8_kernel" if case.A is None else "gemm_s8_kernel_lora")
-    kernel_of = {"gemm_up": "gemm_s8_kernel_gelu_epilogue", "gemm_down": "gemm_s8_kernel"}
+    # the kernel each GEMM stage launches: the CTA-pair kernel above 128 rows (the int8
+    # input-gradient GEMM stays on one SM), template arguments as in the library
+    pair = case.M >= 129
+    fp8 = bool(case.extra.get("fp8"))
+    if case.extra.get("attn"):
+        gemm_kernel = "attn_kernel"
+    elif grad:
+        gemm_kernel = f"gemm_s8_kernel<256,false,false,{case.g}> (input gradient)"
+    elif "fused" in stage_ms:
+        gemm_kernel = (f"gemm_s8_pair_kernel<false,false,false,{case.g}>" if pair else
+                       f"gemm_s8_kernel<256,false,false,0,{case.g}>") \
+            + " (quantizer warps inside)"
+    elif args.workload.startswith("fp8_"):
+        gemm_kernel = ("gemm_s8_pair_kernel<false,true,false,0>" if pair else
+                       "gemm_s8_kernel<256,false,false,0,0,true>") + " (e4m3)"
+    elif case.A is not None:
+        gemm_kernel = ("gemm_s8_pair_kernel<false,false,true,0>" if pair else
+                       "gemm_s8_kernel<SDNQ_LORA_BN,true>") + " (LoRA second accumulator)"
+    else:
+        gemm_kernel = ("gemm_s8_pair_kernel<false,false,false,0>" if pair else
+                       "gemm_s8_kernel<256,false>")
+    kernel_of = {"gemm_up": ("gemm_s8_pair_kernel<true,false,false,0>" if pair else
+                             "gemm_s8_kernel<256,false,true>") + " (GELU epilogue)",
+                 "gemm_down": gemm_kernel}
     ops_per_gemm = ops / len(step.gemm_stages)
     gemm_lines = {}
     for n in step.gemm_stages:
@@ -700,7 +733,7 @@ def main():
             nbytes = 2 * (3 * n_el + 4 * n_el // case.K) + 2 * n_el
         gbs = nbytes / (ms * 1e-3) / 1e9
         rq_lines[n] = {
-            "kernel": "rotquant_persistent_kernel" if rows_k <= 16384 else "rotquant_kernel",
+            "kernel": rotquant_kernel_name(case, rows_k, grad, fp8),
             "bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
             "frac": gbs / peaks["hbm_gbs"],
             "traffic": profiled_traffic(n, "rotquant", profile_key),

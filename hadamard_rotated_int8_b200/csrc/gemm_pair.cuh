@@ -38,7 +38,7 @@
 
 namespace sdnq {
 
-template <bool GELU, bool LORA = false>
+template <bool GELU, bool LORA = false, bool FUSE = false>
 struct PairConfig {
     static constexpr int BM = 128;                       // rows per CTA (256 per pair)
     static constexpr int BN = 256;                       // columns per pair tile
@@ -53,35 +53,45 @@ struct PairConfig {
     // and for LoRA (one accumulator buffer: the drain is not hidden under the next tile's
     // MMAs, so a faster drain is time saved); two for the plain epilogue
     static constexpr int EPI_WARPS = (GELU || LORA) ? SDNQ_WIDE_EPI_WARPS : 8;
-    static constexpr int THREADS = 64 + 32 * EPI_WARPS;
+    // with the activation quantizer inside: 8 quantizer warps and one scale warp more
+    static constexpr int QUANT_WARPS = FUSE ? SDNQ_FUSED_QUANT_WARPS : 0;
+    static constexpr int THREADS = 64 + 32 * EPI_WARPS + (FUSE ? 32 * (QUANT_WARPS + 1) : 0);
     static constexpr int EPI_COLS = BN / (EPI_WARPS / 4);
     static constexpr int STAGE_OUT_BYTES = 32 * 64;
     static constexpr int LUT_BYTES = GELU ? kGeluLutBytes : 0;
     static constexpr int SCALE_BYTES = EPI_COLS * 8;
-    static constexpr int FIXED = EPI_WARPS * (STAGE_OUT_BYTES + SCALE_BYTES) + LUT_BYTES;
+    static constexpr int FIXED = EPI_WARPS * (STAGE_OUT_BYTES + SCALE_BYTES) + LUT_BYTES +
+                                 (FUSE ? 2 * 128 * 4 + 2 * SDNQ_FUSED_QUANT_WARPS * 4 + 32 : 0);
     static constexpr int STAGES = (232448 - 1024 - 512 - FIXED) / STAGE_BYTES > 6
                                       ? 6 : (232448 - 1024 - 512 - FIXED) / STAGE_BYTES;
     static constexpr int OUT_OFF = STAGES * STAGE_BYTES;
     static constexpr int SCALE_OFF = OUT_OFF + EPI_WARPS * STAGE_OUT_BYTES;
     static constexpr int LUT_OFF = SCALE_OFF + EPI_WARPS * SCALE_BYTES;
-    static constexpr int BAR_OFF = LUT_OFF + LUT_BYTES;
-    // full[S], empty[S], tfull[2], tempty[2], drain; then tmem base + abort flag
-    static constexpr int BAR_BYTES = (2 * STAGES + 5) * 8;
+    static constexpr int SX_OFF = LUT_OFF + LUT_BYTES;     // fused: row scales per buffer
+    static constexpr int SX_BYTES = FUSE ? 2 * 128 * 4 : 0;
+    static constexpr int AMAX_OFF = SX_OFF + SX_BYTES;     // fused: quantizer row maxima
+    static constexpr int AMAX_BYTES = FUSE ? 2 * QUANT_WARPS * 4 : 0;
+    static constexpr int BAR_OFF = AMAX_OFF + AMAX_BYTES;
+    // full[S], empty[S], tfull[2], tempty[2], drain, sxfull[2], sxempty[2]; then tmem base +
+    // abort flag
+    static constexpr int BAR_BYTES = (2 * STAGES + 9) * 8;
     static constexpr int SMEM_BYTES = 1024 + BAR_OFF + BAR_BYTES + 16;
     static_assert(STAGES >= 3, "pipeline depth");
     static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 };
 
-template <bool GELU, bool FP8, bool LORA>
-__global__ void __launch_bounds__(PairConfig<GELU, LORA>::THREADS, 1)
+template <bool GELU, bool FP8, bool LORA, int FUSE_G = 0>
+__global__ void __launch_bounds__(PairConfig<GELU, LORA, (FUSE_G > 0)>::THREADS, 1)
     gemm_s8_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB,
                         const __grid_constant__ CUtensorMap tmU,
                         const __grid_constant__ CUtensorMap tmL,
                         const __grid_constant__ CUtensorMap tmO, const GemmParams p)
 {
-    using C = PairConfig<GELU, LORA>;
+    using C = PairConfig<GELU, LORA, (FUSE_G > 0)>;
     static_assert(!LORA || (!GELU && !FP8), "the adapter term rides on the plain int8 linear");
+    static_assert(FUSE_G == 0 || (!LORA && !GELU && !FP8),
+                  "the activation quantizer inside: the plain int8 linear");
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_addr = smem_u32(smem_raw);
     const uint32_t base = (raw_addr + 1023u) & ~1023u;
@@ -92,6 +102,14 @@ __global__ void __launch_bounds__(PairConfig<GELU, LORA>::THREADS, 1)
     auto tfull_bar = [&](int b) { return bar0 + 8u * (2 * C::STAGES + b); };
     auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * C::STAGES + 2 + b); };
     const uint32_t drain_bar = bar0 + 8u * (2 * C::STAGES + 4);
+    auto sxfull_bar = [&](int b) { return bar0 + 8u * (2 * C::STAGES + 5 + b); };
+    auto sxempty_bar = [&](int b) { return bar0 + 8u * (2 * C::STAGES + 7 + b); };
+    float *sx_smem = reinterpret_cast<float *>(smem + C::SX_OFF);     // [2][128], fused only
+    float *amax_smem = reinterpret_cast<float *>(smem + C::AMAX_OFF); // fused only
+    // tile -> (pair-row block, column block): rows fastest; columns fastest with the
+    // quantizer inside, whose 128-row blocks become ready in order
+    auto tile_mb = [&](int tile) { return FUSE_G > 0 ? tile / p.num_n_blocks : tile % p.num_m_blocks; };
+    auto tile_nb = [&](int tile) { return FUSE_G > 0 ? tile % p.num_n_blocks : tile / p.num_m_blocks; };
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C::BAR_OFF + C::BAR_BYTES);
     volatile int *abort = reinterpret_cast<volatile int *>(tmem_holder + 1);
 
@@ -112,6 +130,11 @@ __global__ void __launch_bounds__(PairConfig<GELU, LORA>::THREADS, 1)
             mbar_init(tempty_bar(b), 2 * C::EPI_WARPS);
         }
         mbar_init(drain_bar, 1);
+        if (FUSE_G > 0)
+            for (int b = 0; b < C::NBUF; ++b) {
+                mbar_init(sxfull_bar(b), 1);
+                mbar_init(sxempty_bar(b), C::EPI_WARPS);
+            }
         *abort = 0;
         fence_mbar_init();
         prefetch_tensormap(&tmA);
@@ -142,9 +165,21 @@ __global__ void __launch_bounds__(PairConfig<GELU, LORA>::THREADS, 1)
             int issued = 0;
             bool ok = true;
             const uint32_t leader_full0 = mapa_shared(full_bar(0), 0u);
-            for (int tile = pair; ok && tile < p.num_tiles; tile += npairs) {
-                const int m0 = (tile % p.num_m_blocks) * 2 * C::BM + static_cast<int>(rank) * C::BM;
-                const int nr0 = (tile / p.num_m_blocks) * C::BN + static_cast<int>(rank) * (C::BN / 2);
+            int local = 0;
+            for (int tile = pair; ok && tile < p.num_tiles; tile += npairs, ++local) {
+                const int m0 = tile_mb(tile) * 2 * C::BM + static_cast<int>(rank) * C::BM;
+                const int nr0 = tile_nb(tile) * C::BN + static_cast<int>(rank) * (C::BN / 2);
+                if constexpr (FUSE_G > 0) {
+                    // the scale warp has seen this CTA's 128 activation rows published; order
+                    // that before the tensor copies read them
+                    const int buf = local % C::NBUF;
+                    const uint32_t use = static_cast<uint32_t>(local / C::NBUF);
+                    if (!mbar_wait_bounded(sxfull_bar(buf), use & 1u, abort, p.timeout_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    fence_proxy_async_global();
+                }
                 const int steps = p.num_kb + (LORA ? p.lora_chunks : 0);
                 for (int kb = 0; kb < steps; ++kb) {
                     if (!mbar_wait_bounded(empty_bar(stage), phase ^ 1u, abort, p.timeout_ns)) {
@@ -267,6 +302,56 @@ __global__ void __launch_bounds__(PairConfig<GELU, LORA>::THREADS, 1)
             volatile int no_abort = 0;
             mbar_wait_bounded(drain_bar, 0u, &no_abort, p.timeout_ns);
         }
+    } else if (FUSE_G > 0 && warp == 2 + C::EPI_WARPS + C::QUANT_WARPS) {
+        // ------------------------------------------------------------ scale warp (fused)
+        // Per tile of this CTA, ahead of the producer: wait (bounded, acquire) until this
+        // CTA's 128 activation rows are published, count this CTA as one of the block's
+        // readers (the last one clears the block's counters for the next launch), wait until
+        // this CTA's epilogue has finished with the buffer's scales, copy the rows' scales to
+        // shared memory and arrive on sxfull, which the producer and the epilogue wait for.
+        if constexpr (FUSE_G > 0) {
+            const int nb128 = (p.M + 127) / 128;
+            int local = 0;
+            for (int tile = pair; tile < p.num_tiles; tile += npairs, ++local) {
+                const int m0 = tile_mb(tile) * 2 * C::BM + static_cast<int>(rank) * C::BM;
+                const int b128 = m0 / 128;
+                const int buf = local % C::NBUF;
+                const uint32_t use = static_cast<uint32_t>(local / C::NBUF);
+                const int rows = p.M - m0 < 128 ? (p.M - m0 > 0 ? p.M - m0 : 0) : 128;
+                bool good = true;
+                if (lane == 0) {
+                    if (rows > 0) {
+                        good = wait_count_bounded(p.sync + b128,
+                                                  static_cast<uint32_t>(rows * p.rq.wpr), abort,
+                                                  p.timeout_ns);
+                        if (good) {
+                            const uint32_t seen = atomicAdd(p.sync + nb128 + b128, 1u);
+                            if (seen == static_cast<uint32_t>(p.num_n_blocks) - 1u) {
+                                p.sync[b128] = 0u;
+                                p.sync[nb128 + b128] = 0u;
+                            }
+                        }
+                    }
+                    if (good)
+                        good = mbar_wait_bounded(sxempty_bar(buf), (use & 1u) ^ 1u, abort,
+                                                 p.timeout_ns);
+                }
+                if (__shfl_sync(0xffffffffu, good ? 1 : 0, 0) == 0)
+                    break;
+                for (int i = static_cast<int>(lane); i < 128; i += 32)
+                    sx_smem[buf * 128 + i] = m0 + i < p.M ? p.rq.s[m0 + i] : 0.0f;
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(sxfull_bar(buf));
+            }
+        }
+    } else if (FUSE_G > 0 && warp >= 2 + C::EPI_WARPS) {
+        // ------------------------------------------------------------ activation quantizer
+        // rows of x -> rotated int8 codes (the A operand) and their scales, published per
+        // 128-row block for the scale warps of every CTA
+        if constexpr (FUSE_G > 0)
+            rotquant_worker_rows<FUSE_G>(p.rq, static_cast<int32_t>(warp) - 2 - C::EPI_WARPS,
+                                         C::QUANT_WARPS, 6u, amax_smem, p.sync);
     } else {
         // ------------------------------------------------------------ epilogue (warps 2..9)
         const uint32_t quad = warp & 3u;
@@ -287,8 +372,8 @@ __global__ void __launch_bounds__(PairConfig<GELU, LORA>::THREADS, 1)
         for (int tile = pair; tile < p.num_tiles; tile += npairs, ++local) {
             const int buf = local % C::NBUF;
             const uint32_t use = static_cast<uint32_t>(local / C::NBUF);
-            const int m0 = (tile % p.num_m_blocks) * 2 * C::BM + static_cast<int>(rank) * C::BM;
-            const int n0 = (tile / p.num_m_blocks) * C::BN;
+            const int m0 = tile_mb(tile) * 2 * C::BM + static_cast<int>(rank) * C::BM;
+            const int n0 = tile_nb(tile) * C::BN;
             const int nw = n0 + col_base;
 #pragma unroll
             for (int j = static_cast<int>(lane) * 4; j < C::EPI_COLS; j += 128) {
@@ -325,7 +410,16 @@ __global__ void __launch_bounds__(PairConfig<GELU, LORA>::THREADS, 1)
             tc_fence_after_sync();
             const int m = m0 + row_in_tile;
             const bool row_ok = m < p.M;
-            const float sxm = row_ok ? p.sx[m] : 0.0f;
+            float sxm;
+            if constexpr (FUSE_G > 0) {
+                // the row scales the scale warp copied once the rows were published
+                const bool got = mbar_wait_bounded(sxfull_bar(buf), use & 1u, abort, p.timeout_ns);
+                if (!__all_sync(0xffffffffu, got))
+                    break;
+                sxm = row_ok ? sx_smem[buf * 128 + row_in_tile] : 0.0f;
+            } else {
+                sxm = row_ok ? p.sx[m] : 0.0f;
+            }
             const uint32_t t_row = tmem_base + ((quad * 32u) << 16) + buf * C::ACC_COLS;
 #pragma unroll 1
             for (int c = 0; c < C::EPI_COLS; c += 32) {
@@ -385,8 +479,11 @@ __global__ void __launch_bounds__(PairConfig<GELU, LORA>::THREADS, 1)
             }
             tc_fence_before_sync();
             __syncwarp();
-            if (lane == 0)
+            if (lane == 0) {
                 mbar_arrive_remote(leader_tempty0 + 8u * buf);
+                if (FUSE_G > 0)
+                    mbar_arrive(sxempty_bar(buf));
+            }
         }
         if (lane == 0)
             bulk_wait_all();

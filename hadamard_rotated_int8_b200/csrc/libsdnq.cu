@@ -471,13 +471,13 @@ sdnq_status launch_gemm(const DeviceInfo &dev, const int8_t *qx, const int8_t *q
 // A cluster of two CTAs per pair, launched programmatically like the single-SM kernel; the
 // grid holds as many pairs as the device can keep resident at once (or fewer, one per
 // tile), each walking the tiles persistently.
-template <bool GELU, bool FP8, bool LORA = false>
+template <bool GELU, bool FP8, bool LORA = false, int FUSE_G = 0>
 sdnq_status launch_gemm_pair(const DeviceInfo &dev, const int8_t *qx, const int8_t *qW,
                              GemmParams p, cudaStream_t cs, const uint16_t *u = nullptr,
                              const uint16_t *B = nullptr, int32_t rank = 0)
 {
-    using C = PairConfig<GELU, LORA>;
-    constexpr auto kernel = gemm_s8_pair_kernel<GELU, FP8, LORA>;
+    using C = PairConfig<GELU, LORA, (FUSE_G > 0)>;
+    constexpr auto kernel = gemm_s8_pair_kernel<GELU, FP8, LORA, FUSE_G>;
     CUtensorMap tmA, tmB, tmU, tmL, tmO;
     if (!make_tmap_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, qx, p.K, p.M, p.K, 128, 128) ||
         !make_tmap_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, qW, p.K, p.N, p.K, 128, C::BN / 2) ||
@@ -509,8 +509,15 @@ sdnq_status launch_gemm_pair(const DeviceInfo &dev, const int8_t *qx, const int8
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
-    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    if constexpr (FUSE_G > 0) {
+        // the producers wait for rows that other CTAs' quantizer warps publish: every CTA
+        // must be resident at once
+        attr[1].id = cudaLaunchAttributeCooperative;
+        attr[1].val.cooperative = 1;
+    } else {
+        attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[1].val.programmaticStreamSerializationAllowed = 1;
+    }
     cfg.attrs = attr;
     cfg.numAttrs = 2;
     static PerDeviceCache<1> max_pairs;
@@ -653,25 +660,39 @@ sdnq_status run_linear(const int8_t *qx, const float *sx, const int8_t *qW, cons
 constexpr int kFusedMaxChunks = SDNQ_FUSED_QUANT_WARPS;
 
 // Whether sdnq_int8_linear_fused takes one launch. The one-launch kernel overlaps the
-// quantizer with the GEMM. It pays off once the GEMM has at least three waves of tiles (with
-// fewer, its first wave needs most rows before it can start) and the quantizer is a small
-// share of the work (N >= 3584, or K >= 6144); otherwise the two launches, the GEMM's
-// prologue overlapping the quantizer's tail, are faster (measured on 14 shapes from
-// 4096 x 3072 x 3072 to 16384 x 6144 x 8192). Rows longer than the quantizer warps can hold
-// take the two launches.
+// quantizer with the GEMM. It pays off once the GEMM has at least three waves of 128 x 256
+// tiles (with fewer, its first wave needs most rows before it can start), N >= 3584 (the
+// quantizer's share of the work shrinks with N) and K < 2 N (long rows delay the first
+// published row block); otherwise the two launches, the GEMM's prologue overlapping the
+// quantizer's tail, are as fast or faster (measured on 10 shapes from 4096 x 3072 x 3072 to
+// 8192 x 12288 x 3072, one-launch kernel on CTA pairs). Rows longer than the quantizer warps
+// can hold take the two launches.
 bool fused_one_launch(const DeviceInfo &dev, int64_t M, int64_t N, int64_t K, int32_t policy)
 {
     const int64_t nchunks = (K + 1023) / 1024;
     const int64_t tiles = ((M + 127) / 128) * ((N + 255) / 256);
-    const bool auto_one = tiles >= 3ll * dev.sm_count && (N >= 3584 || K >= 6144);
+    const bool auto_one = tiles >= 3ll * dev.sm_count && N >= 3584 && K < 2 * N;
     return nchunks <= kFusedMaxChunks &&
            (policy == SDNQ_FUSE_ALWAYS || (policy == SDNQ_FUSE_AUTO && auto_one));
 }
 
+// Above 128 rows the one-launch path runs on CTA pairs; if the device refuses that launch
+// (a cooperative launch of clusters), the single-SM one-launch kernel runs instead, and the
+// refusal is remembered for the device.
 template <int G>
 sdnq_status launch_linear_fused_g(const DeviceInfo &dev, GemmParams p, const int8_t *qW,
                                   cudaStream_t cs)
 {
+    static PerDeviceCache<1> pair_refused;
+    if (p.M >= kPairMinRows && pair_refused.get(dev.index, 0, [] { return 2; }) == 2) {
+        const sdnq_status st = launch_gemm_pair<false, false, false, G>(dev, p.rq.q, qW, p, cs);
+        if (st == SDNQ_OK)
+            return st;
+        {
+            std::lock_guard<std::mutex> lock(pair_refused.mutex);
+            pair_refused.value[dev.index][0] = 1;
+        }
+    }
     return launch_gemm<256, false, false, 0, G>(dev, p.rq.q, qW, nullptr, nullptr, 0, p, cs);
 }
 

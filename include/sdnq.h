@@ -123,9 +123,13 @@ sdnq_status sdnq_int8_linear(const int8_t *qx, const float *sx, const int8_t *qW
  * for bit those of the two calls, which is also what the call runs when `policy` asks for it
  * or when the one launch does not pay off:
  *   policy SDNQ_FUSE_AUTO: one launch when the GEMM has at least three waves of 128 x 256
- *          tiles (ceil(M/128) * ceil(N/256) >= 3 * SM count), N >= 3584 or K >= 6144, and
+ *          tiles (ceil(M/128) * ceil(N/256) >= 3 * SM count), N >= 3584, K < 2 N and
  *          K <= 8192, else two;
  *   policy SDNQ_FUSE_ALWAYS: one launch whenever K <= 8192;  SDNQ_FUSE_NEVER: two launches.
+ *   Above 128 rows the one launch runs on CTA pairs as a cooperative launch of two-CTA
+ *   clusters (every CTA resident at once, since tile loads wait on rows that other CTAs
+ *   quantize); if the device refuses that launch, the single-SM one-launch kernel runs
+ *   instead (same bits) and the refusal is remembered for the device.
  *   x [M, K] bf16, row stride ldx; group as in sdnq_rotquant_act.
  *   qW, sW, bias, out, ldo, acc_out as in sdnq_int8_linear.
  *   qx_ws [M, K] int8 dense, sx_ws [M] fp32: caller-provided workspace for the activation
