@@ -344,6 +344,23 @@ __device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)
                  : "r"(taddr));
 }
 
+// 32 columns into two 16-column halves (one load instruction).
+__device__ __forceinline__ void tmem_ld_32x32b_x32_halves(uint32_t taddr, uint32_t (&a)[16],
+                                                          uint32_t (&b)[16])
+{
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32"
+                 " {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15,"
+                 " %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31},"
+                 " [%32];"
+                 : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3]), "=r"(a[4]), "=r"(a[5]),
+                   "=r"(a[6]), "=r"(a[7]), "=r"(a[8]), "=r"(a[9]), "=r"(a[10]), "=r"(a[11]),
+                   "=r"(a[12]), "=r"(a[13]), "=r"(a[14]), "=r"(a[15]), "=r"(b[0]), "=r"(b[1]),
+                   "=r"(b[2]), "=r"(b[3]), "=r"(b[4]), "=r"(b[5]), "=r"(b[6]), "=r"(b[7]),
+                   "=r"(b[8]), "=r"(b[9]), "=r"(b[10]), "=r"(b[11]), "=r"(b[12]), "=r"(b[13]),
+                   "=r"(b[14]), "=r"(b[15])
+                 : "r"(taddr));
+}
+
 // Same, 4 columns.
 __device__ __forceinline__ void tmem_ld_32x32b_x4(uint32_t taddr, uint32_t (&r)[4])
 {
@@ -452,6 +469,13 @@ __device__ __forceinline__ uint32_t cluster_ctarank()
     return r;
 }
 
+__device__ __forceinline__ uint32_t cluster_nctarank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+    return r;
+}
+
 __device__ __forceinline__ uint32_t cluster_id_x()
 {
     uint32_t r;
@@ -503,47 +527,14 @@ __device__ __forceinline__ void cluster_sync_all()
                      : "memory");
 }
 
-// Arrive (release at cluster scope) on an mbarrier in another CTA of the cluster.
+// Arrive on an mbarrier in another CTA of the cluster, with the default semantics (release
+// at CTA scope). The pair kernels use it only to hand tensor-memory columns back to the MMA
+// issuer, an ordering the tcgen05 fences on both sides establish; no generic-memory data
+// passes through the barrier, so a cluster-scope release (a fence that waited about 0.6 us
+// behind the warp's earlier stores) is not needed.
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr)
 {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
-                 : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity)
-{
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    return ok != 0u;
-}
-
-// As mbar_wait_bounded, for a barrier that threads of the other CTA arrive on (acquire at
-// cluster scope).
-__device__ __forceinline__ bool mbar_wait_bounded_cluster(uint32_t bar, uint32_t parity,
-                                                          volatile int *abort, uint64_t limit_ns)
-{
-    if (mbar_try_wait_cluster(bar, parity))
-        return true;
-    const uint64_t t0 = global_timer_ns();
-    for (uint32_t it = 1;; ++it) {
-        if (mbar_try_wait_cluster(bar, parity))
-            return true;
-        if ((it & 63u) == 0u) {
-            if (*abort)
-                return false;
-            if (global_timer_ns() - t0 > limit_ns) {
-                *abort = 1;
-                atomicOr(&g_device_error, kDevTimeout);
-                return false;
-            }
-        }
-    }
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
 // Tensor memory for a CTA pair: one warp of each CTA (the same warp index) allocates the
@@ -638,6 +629,17 @@ __device__ __forceinline__ void sts_v4(uint32_t addr, uint32_t a, uint32_t b, ui
     asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
                  "r"(d)
                  : "memory");
+}
+
+// 16 bytes from the shared memory of a CTA of the cluster (a shared::cluster address).
+__device__ __forceinline__ float4 ld_cluster_v4(uint32_t cluster_addr)
+{
+    float4 v;
+    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "r"(cluster_addr)
+                 : "memory");
+    return v;
 }
 
 __device__ __forceinline__ float4 lds_v4(uint32_t addr)

@@ -8,20 +8,28 @@
 // kernel, so outputs are bit for bit the same. With LORA the pair also accumulates the
 // adapter term L = u B (bf16 operands, fp32, kind::f16) in a second 256-column accumulator
 // after the int8 K loop, as the single-SM kernel does; the int32 and fp32 accumulators then
-// fill the 512 columns, so there is one buffer.
+// fill the 512 columns, so there is one buffer. Its epilogue copies the int32 columns to
+// registers and hands them back at once (tempty[0]), so the next tile's int8 K loop runs
+// while the outputs of this one are formed; the adapter columns go back (tempty[1]) before
+// the next tile's adapter MMAs.
 //
 // Sources: as the single-SM kernel ("SDNQ: SD.Next Quantization Engine" README, INT8
 // quantized matmul and dequantize_fp32; "ConvRot / Hadamard SDNQ").
 //
-// Roles (320 threads per CTA; 576 with GELU or LoRA):
+// Roles (320 threads per CTA; 576 with GELU; 608 with the activation quantizer inside):
 //   warp 0      TMA producer of this CTA's halves. The loads of both CTAs complete on rank
 //               0's full barrier (the cta_group::2 form of the tensor copy), whose
 //               expected byte count rank 0 sets for both halves.
 //   warp 1      both CTAs allocate the same tensor-memory columns; rank 0 issues the
 //               pair's MMAs once a stage is full.
-//   warps 2..   epilogue of this CTA's 128 rows (8 warps; 16 with GELU or LoRA); they
+//   warps 2..   epilogue of this CTA's 128 rows (8 warps; 16 with GELU); they
 //               release the accumulator buffer with a remote arrive on rank 0's
 //               tensor-empty barrier (one arrival per epilogue warp of both CTAs).
+//   then, with the activation quantizer inside (plain linear only): 8 warps that rotate and
+//               quantize rows of x into the A operand, publishing 128-row blocks through
+//               global counters, and one scale warp that waits (bounded) for this CTA's
+//               block of each tile and copies its row scales to shared memory for the
+//               producer and the epilogue. Tiles then run columns-fastest.
 // The MMA completion (tcgen05.commit, multicast to both CTAs) frees each stage in both CTAs
 // and announces each finished accumulator buffer to both epilogues. Every wait is bounded.
 // A producer that gives up drains its own copies: rank 0 by waiting (bounded) on its full
@@ -34,6 +42,9 @@
 
 #ifndef SDNQ_WIDE_EPI_WARPS
 #define SDNQ_WIDE_EPI_WARPS 16
+#endif
+#ifndef SDNQ_LORA_EPI_WARPS
+#define SDNQ_LORA_EPI_WARPS 8
 #endif
 
 namespace sdnq {
@@ -49,10 +60,10 @@ struct PairConfig {
     static constexpr int ACC_COLS = LORA ? 2 * BN : BN;  // int32 (+ fp32 LoRA) columns per buffer
     static constexpr int NBUF = LORA ? 1 : 2;
     static constexpr int TMEM_COLS = NBUF * ACC_COLS;    // 512
-    // four epilogue warps per TMEM lane quarter for the GELU table lookups (integer-heavy)
-    // and for LoRA (one accumulator buffer: the drain is not hidden under the next tile's
-    // MMAs, so a faster drain is time saved); two for the plain epilogue
-    static constexpr int EPI_WARPS = (GELU || LORA) ? SDNQ_WIDE_EPI_WARPS : 8;
+    // four epilogue warps per TMEM lane quarter for the GELU table lookups (integer-heavy);
+    // two for the plain epilogue and for LoRA, whose warps hold a row's fp32 partials for
+    // their 128 columns in registers (168 per thread at 10 warps per CTA)
+    static constexpr int EPI_WARPS = GELU ? SDNQ_WIDE_EPI_WARPS : LORA ? SDNQ_LORA_EPI_WARPS : 8;
     // with the activation quantizer inside: 8 quantizer warps and one scale warp more
     static constexpr int QUANT_WARPS = FUSE ? SDNQ_FUSED_QUANT_WARPS : 0;
     static constexpr int THREADS = 64 + 32 * EPI_WARPS + (FUSE ? 32 * (QUANT_WARPS + 1) : 0);
@@ -79,6 +90,112 @@ struct PairConfig {
     static_assert(STAGES >= 3, "pipeline depth");
     static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 };
+
+// The first fp32 steps of the de-quant epilogue for two adjacent columns: t = sx * sw (f32x2),
+// v = fp32(acc) * t, then + bias; the products that feed an add as scalar intrinsics, the
+// same steps as the single-SM epilogue.
+template <bool FP8>
+__device__ __forceinline__ void dequant_pair(uint32_t acc0, uint32_t acc1, float sxm, float w0,
+                                             float w1, float b0, float b1, bool has_bias,
+                                             float &v0, float &v1)
+{
+    float t0, t1;
+    mul2(t0, t1, sxm, sxm, w0, w1);
+    const float a0 = FP8 ? __uint_as_float(acc0) : __int2float_rn(static_cast<int>(acc0));
+    const float a1 = FP8 ? __uint_as_float(acc1) : __int2float_rn(static_cast<int>(acc1));
+    v0 = __fmul_rn(a0, t0);
+    v1 = __fmul_rn(a1, t1);
+    if (has_bias) {
+        v0 = __fadd_rn(v0, b0);
+        v1 = __fadd_rn(v1, b1);
+    }
+}
+
+// LoRA epilogue of one warp (one TMEM lane quarter, EPI_COLS columns of the tile). The int32
+// columns are copied to registers with one wait and released at once through rank 0's
+// tempty[0]: the pair's next int8 K loop then runs while this warp de-quantizes, reads the
+// adapter columns, adds lora_scale * L and stores the bf16 outputs; tempty[1] releases the
+// adapter columns for the next tile's adapter MMAs. The arithmetic and its order are those
+// of the one-pass epilogue, so outputs are unchanged.
+template <class C>
+__device__ __forceinline__ void lora_epilogue(uint32_t t_row, int col_base, int n0, int m0,
+                                              uint32_t quad, uint32_t lane, float sxm,
+                                              bool row_ok, int m, uint32_t s_sw,
+                                              uint32_t s_bias, uint32_t s_out,
+                                              const CUtensorMap *tmO, const GemmParams &p,
+                                              uint32_t leader_tempty0)
+{
+    constexpr int NCH = C::EPI_COLS / 16;
+    const bool has_bias = p.bias != nullptr;
+    uint32_t acc[NCH][16];
+#pragma unroll
+    for (int k = 0; k < NCH; ++k)
+        if (n0 + col_base + 16 * k < p.N)   // warp-uniform
+            tmem_ld_32x32b_x16(t_row + col_base + 16 * k, acc[k]);
+    tmem_ld_wait();
+    tc_fence_before_sync();
+    __syncwarp();
+    if (lane == 0)
+        mbar_arrive_remote(leader_tempty0);
+    if (p.acc_out != nullptr && row_ok) {
+        int32_t *arow = p.acc_out + static_cast<int64_t>(m) * p.N;
+#pragma unroll
+        for (int k = 0; k < NCH; ++k)
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+                if (n0 + col_base + 16 * k + j < p.N)
+                    arow[n0 + col_base + 16 * k + j] = static_cast<int32_t>(acc[k][j]);
+    }
+    // fp32(acc) * t + bias, in place
+#pragma unroll
+    for (int k = 0; k < NCH; ++k) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const float4 w = lds_v4(s_sw + 4 * (16 * k + 4 * q));
+            const float4 b = lds_v4(s_bias + 4 * (16 * k + 4 * q));
+            const float wv[4] = {w.x, w.y, w.z, w.w};
+            const float bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int j = 4 * q + 2 * h;
+                float v0, v1;
+                dequant_pair<false>(acc[k][j], acc[k][j + 1], sxm, wv[2 * h], wv[2 * h + 1],
+                                    bv[2 * h], bv[2 * h + 1], has_bias, v0, v1);
+                acc[k][j] = __float_as_uint(v0);
+                acc[k][j + 1] = __float_as_uint(v1);
+            }
+        }
+    }
+#pragma unroll
+    for (int c = 0; c < C::EPI_COLS; c += 32) {
+        const int cc = col_base + c;
+        const int nc = n0 + cc;
+        if (nc < p.N) {   // warp-uniform
+            uint32_t ob[16];
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const int k = c / 16 + hh;
+                uint32_t l[16];
+                tmem_ld_32x32b_x16(t_row + C::BN + cc + 16 * hh, l);
+                tmem_ld_wait();
+#pragma unroll
+                for (int j = 0; j < 16; j += 2) {
+                    const float v0 = __fadd_rn(__uint_as_float(acc[k][j]),
+                                               __fmul_rn(p.lora_scale, __uint_as_float(l[j])));
+                    const float v1 = __fadd_rn(__uint_as_float(acc[k][j + 1]),
+                                               __fmul_rn(p.lora_scale, __uint_as_float(l[j + 1])));
+                    const __nv_bfloat162 h2 = __floats2bfloat162_rn(v0, v1);
+                    ob[(16 * hh + j) >> 1] = *reinterpret_cast<const uint32_t *>(&h2);
+                }
+            }
+            store_block(ob, s_out, lane, tmO, nc, m0 + static_cast<int>(quad * 32u));
+        }
+    }
+    tc_fence_before_sync();
+    __syncwarp();
+    if (lane == 0)
+        mbar_arrive_remote(leader_tempty0 + 8u);
+}
 
 template <bool GELU, bool FP8, bool LORA, int FUSE_G = 0>
 __global__ void __launch_bounds__(PairConfig<GELU, LORA, (FUSE_G > 0)>::THREADS, 1)
@@ -125,10 +242,11 @@ __global__ void __launch_bounds__(PairConfig<GELU, LORA, (FUSE_G > 0)>::THREADS,
             mbar_init(full_bar(s), 1);
             mbar_init(empty_bar(s), 1);
         }
-        for (int b = 0; b < C::NBUF; ++b) {
+        for (int b = 0; b < C::NBUF; ++b)
             mbar_init(tfull_bar(b), 1);
+        // with LoRA: tempty[0] releases the int32 columns, tempty[1] the adapter columns
+        for (int b = 0; b < (LORA ? 2 : C::NBUF); ++b)
             mbar_init(tempty_bar(b), 2 * C::EPI_WARPS);
-        }
         mbar_init(drain_bar, 1);
         if (FUSE_G > 0)
             for (int b = 0; b < C::NBUF; ++b) {
@@ -240,7 +358,7 @@ __global__ void __launch_bounds__(PairConfig<GELU, LORA, (FUSE_G > 0)>::THREADS,
             for (int tile = pair; ok && tile < p.num_tiles; tile += npairs, ++local) {
                 const int buf = local % C::NBUF;
                 const uint32_t use = static_cast<uint32_t>(local / C::NBUF);
-                if (!mbar_wait_bounded_cluster(tempty_bar(buf), (use & 1u) ^ 1u, abort, p.timeout_ns)) {
+                if (!mbar_wait_bounded(tempty_bar(buf), (use & 1u) ^ 1u, abort, p.timeout_ns)) {
                     ok = false;
                     break;
                 }
@@ -272,6 +390,12 @@ __global__ void __launch_bounds__(PairConfig<GELU, LORA, (FUSE_G > 0)>::THREADS,
                 if constexpr (LORA) {
                     constexpr uint32_t IDESC_BF = idesc_bf16_f32(256, C::BN, true);
                     const uint32_t d_lora = d_acc + C::BN;
+                    // the epilogues of both CTAs have read the previous tile's adapter columns
+                    if (!mbar_wait_bounded(tempty_bar(1), (use & 1u) ^ 1u, abort, p.timeout_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after_sync();
                     for (int c = 0; ok && c < p.lora_chunks; ++c) {
                         if (!mbar_wait_bounded(full_bar(stage), phase, abort, p.timeout_ns)) {
                             ok = false;
@@ -404,85 +528,83 @@ __global__ void __launch_bounds__(PairConfig<GELU, LORA, (FUSE_G > 0)>::THREADS,
                        __float_as_uint(b4[2]), __float_as_uint(b4[3]));
             }
             __syncwarp();
+            const int m = m0 + row_in_tile;
+            const bool row_ok = m < p.M;
+            // the row's scale is read before the accumulator wait (written by an earlier
+            // launch, visible since the dependency wait)
+            float sxm = (FUSE_G == 0 && row_ok) ? p.sx[m] : 0.0f;
             const bool ready = mbar_wait_bounded(tfull_bar(buf), use & 1u, abort, p.timeout_ns);
             if (!__all_sync(0xffffffffu, ready))
                 break;
             tc_fence_after_sync();
-            const int m = m0 + row_in_tile;
-            const bool row_ok = m < p.M;
-            float sxm;
             if constexpr (FUSE_G > 0) {
                 // the row scales the scale warp copied once the rows were published
                 const bool got = mbar_wait_bounded(sxfull_bar(buf), use & 1u, abort, p.timeout_ns);
                 if (!__all_sync(0xffffffffu, got))
                     break;
                 sxm = row_ok ? sx_smem[buf * 128 + row_in_tile] : 0.0f;
-            } else {
-                sxm = row_ok ? p.sx[m] : 0.0f;
             }
             const uint32_t t_row = tmem_base + ((quad * 32u) << 16) + buf * C::ACC_COLS;
+            if constexpr (LORA) {
+                lora_epilogue<C>(t_row, col_base, n0, m0, quad, lane, sxm, row_ok, m, s_sw, s_bias,
+                                 s_out, &tmO, p, leader_tempty0);
+            } else {
 #pragma unroll 1
-            for (int c = 0; c < C::EPI_COLS; c += 32) {
-                const int cc = col_base + c;
-                const int nc = n0 + cc;
-                if (nc >= p.N)
-                    break;  // warp-uniform
-                uint32_t acc[32];
-                tmem_ld_32x32b_x32(t_row + cc, acc);
-                uint32_t lacc[LORA ? 32 : 1];
-                if constexpr (LORA)
-                    tmem_ld_32x32b_x32(t_row + C::BN + cc, lacc);
-                tmem_ld_wait();
-                uint32_t ob[16];
+                for (int c = 0; c < C::EPI_COLS; c += 32) {
+                    const int cc = col_base + c;
+                    const int nc = n0 + cc;
+                    if (nc >= p.N)
+                        break;  // warp-uniform
+                    uint32_t acc[32];
+                    tmem_ld_32x32b_x32(t_row + cc, acc);
+                    tmem_ld_wait();
+                    uint32_t ob[16];
 #pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    const float4 w = lds_v4(s_sw + 4 * (c + 4 * q));
-                    const float4 b = lds_v4(s_bias + 4 * (c + 4 * q));
-                    const float wv[4] = {w.x, w.y, w.z, w.w};
-                    const float bv[4] = {b.x, b.y, b.z, b.w};
+                    for (int q = 0; q < 8; ++q) {
+                        const float4 w = lds_v4(s_sw + 4 * (c + 4 * q));
+                        const float4 b = lds_v4(s_bias + 4 * (c + 4 * q));
+                        const float wv[4] = {w.x, w.y, w.z, w.w};
+                        const float bv[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        const int j = 4 * q + 2 * h;
-                        // the same fp32 steps as the single-SM epilogue: t in f32x2, the
-                        // products that feed an add as scalar intrinsics
-                        float t0, t1;
-                        mul2(t0, t1, sxm, sxm, wv[2 * h], wv[2 * h + 1]);
-                        const float a0 = FP8 ? __uint_as_float(acc[j]) : __int2float_rn(static_cast<int>(acc[j]));
-                        const float a1 = FP8 ? __uint_as_float(acc[j + 1])
-                                             : __int2float_rn(static_cast<int>(acc[j + 1]));
-                        float v0 = __fmul_rn(a0, t0);
-                        float v1 = __fmul_rn(a1, t1);
-                        if (has_bias) {
-                            v0 = __fadd_rn(v0, bv[2 * h]);
-                            v1 = __fadd_rn(v1, bv[2 * h + 1]);
+                        for (int h = 0; h < 2; ++h) {
+                            const int j = 4 * q + 2 * h;
+                            // the same fp32 steps as the single-SM epilogue: t in f32x2, the
+                            // products that feed an add as scalar intrinsics
+                            float t0, t1;
+                            mul2(t0, t1, sxm, sxm, wv[2 * h], wv[2 * h + 1]);
+                            const float a0 = FP8 ? __uint_as_float(acc[j]) : __int2float_rn(static_cast<int>(acc[j]));
+                            const float a1 = FP8 ? __uint_as_float(acc[j + 1])
+                                                 : __int2float_rn(static_cast<int>(acc[j + 1]));
+                            float v0 = __fmul_rn(a0, t0);
+                            float v1 = __fmul_rn(a1, t1);
+                            if (has_bias) {
+                                v0 = __fadd_rn(v0, bv[2 * h]);
+                                v1 = __fadd_rn(v1, bv[2 * h + 1]);
+                            }
+                            const __nv_bfloat162 h2 = __floats2bfloat162_rn(v0, v1);
+                            ob[j >> 1] = *reinterpret_cast<const uint32_t *>(&h2);
                         }
-                        if constexpr (LORA) {
-                            v0 = __fadd_rn(v0, __fmul_rn(p.lora_scale, __uint_as_float(lacc[j])));
-                            v1 = __fadd_rn(v1, __fmul_rn(p.lora_scale, __uint_as_float(lacc[j + 1])));
-                        }
-                        const __nv_bfloat162 h2 = __floats2bfloat162_rn(v0, v1);
-                        ob[j >> 1] = *reinterpret_cast<const uint32_t *>(&h2);
+                    }
+                    if constexpr (GELU) {
+                        gelu_bf16x16_lut(ob, lut);
+                        gelu_bf16x16_lut(ob + 8, lut);
+                    }
+                    store_block(ob, s_out, lane, &tmO, nc, m0 + static_cast<int>(quad * 32u));
+                    if (p.acc_out != nullptr && row_ok) {
+                        int32_t *arow = p.acc_out + static_cast<int64_t>(m) * p.N;
+#pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            if (nc + j < p.N)
+                                arow[nc + j] = static_cast<int32_t>(acc[j]);
                     }
                 }
-                if constexpr (GELU) {
-                    gelu_bf16x16_lut(ob, lut);
-                    gelu_bf16x16_lut(ob + 8, lut);
+                tc_fence_before_sync();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive_remote(leader_tempty0 + 8u * buf);
+                    if (FUSE_G > 0)
+                        mbar_arrive(sxempty_bar(buf));
                 }
-                store_block(ob, s_out, lane, &tmO, nc, m0 + static_cast<int>(quad * 32u));
-                if (p.acc_out != nullptr && row_ok) {
-                    int32_t *arow = p.acc_out + static_cast<int64_t>(m) * p.N;
-#pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        if (nc + j < p.N)
-                            arow[nc + j] = static_cast<int32_t>(acc[j]);
-                }
-            }
-            tc_fence_before_sync();
-            __syncwarp();
-            if (lane == 0) {
-                mbar_arrive_remote(leader_tempty0 + 8u * buf);
-                if (FUSE_G > 0)
-                    mbar_arrive(sxempty_bar(buf));
             }
         }
         if (lane == 0)

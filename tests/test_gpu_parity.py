@@ -254,6 +254,31 @@ def test_lora_within_one_ulp(M, N, K, rank):
     check_lora_tolerance(case, got["u"], got["out"], ref, 0.75)
 
 
+@pytest.mark.parametrize("M,N,K,rank,g", [
+    (200, 64, 64, 16, 64),      # one k-block: a down-projection stage half used
+    (300, 64, 192, 32, 64),     # three k-blocks: a full stage, then a half one
+    (9000, 64, 512, 64, 256),   # 71 row blocks of the down-projection
+    (20000, 32, 256, 48, 256),  # 157 row blocks: more than one CTA per SM over the launch
+])
+def test_lora_few_k_blocks_and_many_row_blocks(M, N, K, rank, g):
+    """The down-projection u = x A streams two 64-column k-blocks of x per pipeline stage,
+    one 128-row block per CTA: an odd number of k-blocks and launches of more row blocks
+    than SMs stay within the fp32 accumulation bound of the oracle's u and output, and
+    repeating the call gives the same bits."""
+    case = synthetic.make_case(M=M, N=N, K=K, g=g, seed=M + K + rank, outlier_count=K // 64,
+                               outlier_factor=30.0, bias_std=None, lora_rank=rank,
+                               lora_scale=0.5)
+    got = run_linear_case(case, lora=True)
+    again = run_linear_case(case, lora=True)
+    assert_equal(again["u"], got["u"], "repeat: u")
+    assert_equal(again["out"], got["out"], "repeat: outputs")
+    ref = oracle.linear(synthetic.bits(case.x), *oracle.rotate_quantize(synthetic.bits(case.W), g),
+                        g, A_bits=synthetic.bits(case.A), B_bits=synthetic.bits(case.B),
+                        lora_scale=0.5)
+    assert_equal(got["acc"], ref["acc"], "int32 accumulators (LoRA kernel)")
+    check_lora_tolerance(case, got["u"], got["out"], ref, 0.5)
+
+
 def lora_tolerances(x_bits, A_bits, B_bits, u_ref_bits, out_ref_bits, scale, rows=None):
     """Tolerance derived from the arithmetic (the adapter path accumulates in fp32, the
     oracle in fp64): one bf16 ulp of the result plus the fp32 accumulation bound
