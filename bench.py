@@ -211,14 +211,17 @@ class Step:
         elif case.A is not None:
             self.A, self.B = case.A.to(dev), case.B.to(dev)
             self.u = torch.empty((case.M, case.A.shape[1]), dtype=torch.bfloat16, device=dev)
+            # sdnq_int8_linear_lora as its two calls (the same kernels and bits), so that the
+            # GEMM with the adapter term is timed on its own
             self.stages = [
                 ("rotquant", lambda: sd.sdnq_rotquant_act(self.x, g, self.qx, self.sx)),
-                ("gemm_lora", lambda: sd.sdnq_int8_linear_lora(
-                    self.qx, self.sx, self.qW, self.sW, self.bias, self.x, self.A, self.B,
-                    case.lora_scale, u_ws=self.u, out=self.out)),
+                ("lora_down", lambda: sd.sdnq_lora_down(self.x, self.A, u=self.u)),
+                ("gemm_lora", lambda: sd.sdnq_int8_linear_lora_up(
+                    self.qx, self.sx, self.qW, self.sW, self.bias, self.u, self.B,
+                    case.lora_scale, out=self.out)),
             ]
             self.gemm_stages = ["gemm_lora"]
-            self.launches = 3  # rotquant, LoRA down-projection, fused GEMM
+            self.launches = 3  # rotquant, LoRA down-projection, GEMM with the adapter term
         elif sd.sdnq_int8_linear_fused_plan(case.M, case.N, case.K):
             # the library's own choice for sdnq_int8_linear_fused (one launch here)
             # one launch: the activation quantizer runs inside the GEMM kernel
@@ -739,6 +742,21 @@ def main():
             "traffic": profiled_traffic(n, "rotquant", profile_key),
             "bytes_per_launch": nbytes, "row_length": rows_k, "ms_per_launch": ms,
             "peak_source": f"{peak_src} copy bandwidth", "timing": note,
+        }
+    if "lora_down" in stage_ms:
+        # u = bf16(x A): reads x and A, writes u
+        r = case.A.shape[1]
+        ms = stage_ms["lora_down"] / args.steps
+        nbytes = 2 * (case.M * case.K + case.K * r + case.M * r)
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        rq_lines["lora_down"] = {
+            "kernel": f"lora_down_kernel<{(r + 63) // 64 * 64}>", "bound": "hbm",
+            "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": gbs / peaks["hbm_gbs"],
+            "traffic": profiled_traffic("lora_down", "lora_down", profile_key),
+            "bytes_per_launch": nbytes, "ms_per_launch": ms,
+            "peak_source": f"{peak_src} copy bandwidth",
+            "timing": "the stage's time in the per-stage pass of the same steps",
         }
     line = {
         "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world,

@@ -10,6 +10,7 @@ The compute lives in ``libsdnq.so`` (hand-written CUDA behind the C ABI of
 * ``sdnq_int8_linear_fused_plan`` whether that call takes one launch or two for a shape
 * ``sdnq_int8_linear_gelu``     the same with GELU fused into the epilogue (MLP up-projection)
 * ``sdnq_int8_linear_lora``     the same plus the bf16 LoRA side term
+  (= ``sdnq_lora_down`` then ``sdnq_int8_linear_lora_up``)
 * ``sdnq_int8_linear_grad_input`` input gradient through the frozen rotated int8 base
   (= ``sdnq_quant_grad_output`` then ``sdnq_int8_grad_input_gemm``)
 * ``sdnq_gelu_bf16``            exact-erf GELU (MLP glue)
@@ -24,7 +25,8 @@ from ._native import (SdnqError, lib, sdnq_attention_int8qk, sdnq_device_status,
                       sdnq_int8_grad_input_gemm, sdnq_int8_linear_fused,
                       sdnq_int8_linear_fused_plan, sdnq_int8_linear_gelu,
                       sdnq_int8_linear_grad_input, sdnq_int8_linear_lora,
-                      sdnq_int8_linear_lora_noalloc, sdnq_rotate_quant_weight,
+                      sdnq_int8_linear_lora_noalloc, sdnq_int8_linear_lora_up,
+                      sdnq_lora_down, sdnq_rotate_quant_weight,
                       sdnq_quant_grad_output, sdnq_rotquant_act, sdnq_selftest_wait_timeout,
                       status_string, version)
 
@@ -36,7 +38,7 @@ __all__ = [
     "sdnq_int8_linear_gelu",
     "sdnq_int8_linear_grad_input",
     "sdnq_int8_linear_lora", "sdnq_quant_grad_output",
-    "sdnq_int8_linear_lora_noalloc",
+    "sdnq_int8_linear_lora_noalloc", "sdnq_int8_linear_lora_up", "sdnq_lora_down",
     "sdnq_rotate_quant_weight", "sdnq_rotquant_act", "sdnq_selftest_wait_timeout",
     "status_string", "version",
 ]

@@ -53,6 +53,9 @@ SIGNATURES = {
                               _I64, _P, _I64, _P, _P],
     "sdnq_int8_linear_lora_noalloc": [_P, _P, _P, _P, _P, _P, _I64, _P, _P, _I32, _F, _I64,
                                       _I64, _I64, _P, _I64, _P, _P],
+    "sdnq_lora_down": [_P, _I64, _P, _I32, _I64, _I64, _P, _P],
+    "sdnq_int8_linear_lora_up": [_P, _P, _P, _P, _P, _P, _P, _I32, _F, _I64, _I64, _I64, _P,
+                                 _I64, _P, _P],
     "sdnq_gelu_bf16": [_P, _I64, _I64, _I64, _P, _I64, _P],
     "sdnq_rotquant_fp8": [_P, _I64, _I64, _I64, _I32, _P, _P, _P],
     "sdnq_attention_workspace": [_I64, _I64, _I64, _I64, _I64, _P],
@@ -498,6 +501,41 @@ def sdnq_int8_linear_lora(qx, sx, qW, sW, bias, x, A, B, lora_scale: float = 1.0
                                        float(lora_scale), _ptr(u_ws), M, N, K, _ptr(out),
                                        out.stride(0), _ptr(acc_out), _stream(stream)),
            "sdnq_int8_linear_lora")
+    return out
+
+
+def sdnq_lora_down(x, A, u=None, stream=None):
+    """u [M, rank] = bf16(x A): the LoRA down-projection of sdnq_int8_linear_lora alone
+    (x the unrotated bf16 layer input [M, K], A [K, rank] bf16)."""
+    _req(x, torch.bfloat16, "x", 2)
+    _req(A, torch.bfloat16, "A", 2)
+    _dense(A, "A")
+    M, K = x.shape
+    if A.shape[0] != K:
+        raise ValueError(f"A: expected {K} rows, got {A.shape[0]}")
+    rank = A.shape[1]
+    u = torch.empty((M, rank), dtype=torch.bfloat16, device=x.device) if u is None else u
+    _mat(u, torch.bfloat16, M, rank, "u", dense=True)
+    _check(lib().sdnq_lora_down(_ptr(x), x.stride(0), _ptr(A), rank, M, K, _ptr(u),
+                                _stream(stream)), "sdnq_lora_down")
+    return u
+
+
+def sdnq_int8_linear_lora_up(qx, sx, qW, sW, bias, u, B, lora_scale: float = 1.0, out=None,
+                             acc_out=None, stream=None):
+    """sdnq_int8_linear plus lora_scale * u B from a given u [M, rank] (as written by
+    sdnq_lora_down); B [rank, N] bf16."""
+    M, N, K, out = _linear_operands(qx, sx, qW, sW, bias, out, acc_out)
+    _req(B, torch.bfloat16, "B", 2)
+    _dense(B, "B")
+    rank = B.shape[0]
+    if B.shape[1] != N:
+        raise ValueError(f"B: expected shape {(rank, N)}, got {tuple(B.shape)}")
+    _mat(u, torch.bfloat16, M, rank, "u", dense=True)
+    _check(lib().sdnq_int8_linear_lora_up(_ptr(qx), _ptr(sx), _ptr(qW), _ptr(sW), _ptr(bias),
+                                          _ptr(u), _ptr(B), rank, float(lora_scale), M, N, K,
+                                          _ptr(out), out.stride(0), _ptr(acc_out),
+                                          _stream(stream)), "sdnq_int8_linear_lora_up")
     return out
 
 

@@ -589,26 +589,55 @@ sdnq_status ensure_gelu_lut(const DeviceInfo &dev, cudaStream_t cs)
     return ok == 1 ? SDNQ_OK : SDNQ_ERR_CUDA;
 }
 
+// The adapter's part of a linear call: none, the down-projection u = bf16(x A) followed by
+// the GEMM with the term lora_scale * (u B), or that GEMM alone from a given u.
+enum LoraMode { kNoLora = 0, kLoraFull = 1, kLoraUp = 2 };
+
+// Arguments of the down-projection u [M, rank] = bf16(x [M, K] A [K, rank]).
+sdnq_status validate_lora_down(const uint16_t *x, int64_t ldx, const uint16_t *A, int32_t rank,
+                               int64_t M, int64_t K, const uint16_t *u)
+{
+    if (!A || (M != 0 && (!x || !u)))
+        return SDNQ_ERR_NULL;
+    if (M < 0 || M > INT32_MAX || K < 16 || K > SDNQ_MAX_K || K % 16 != 0 || ldx < K)
+        return SDNQ_ERR_SHAPE;
+    if (rank < 16 || rank > SDNQ_MAX_RANK || rank % 16 != 0)
+        return SDNQ_ERR_UNSUPPORTED;
+    if (ldx % 8 != 0 || !aligned(x, 16) || !aligned(A, 16) || !aligned(u, 16))
+        return SDNQ_ERR_ALIGN;
+    return SDNQ_OK;
+}
+
+sdnq_status run_lora_down(const DeviceInfo &dev, const uint16_t *x, int64_t ldx, const uint16_t *A,
+                          int32_t rank, uint16_t *u, int64_t M, int64_t K, cudaStream_t cs)
+{
+    const int32_t Mi = static_cast<int32_t>(M), Ki = static_cast<int32_t>(K);
+    if (rank <= 64)
+        return launch_lora_down<64>(dev, x, ldx, A, rank, u, Mi, Ki, cs);
+    if (rank <= 128)
+        return launch_lora_down<128>(dev, x, ldx, A, rank, u, Mi, Ki, cs);
+    return launch_lora_down<256>(dev, x, ldx, A, rank, u, Mi, Ki, cs);
+}
+
 sdnq_status run_linear(const int8_t *qx, const float *sx, const int8_t *qW, const float *sW,
                        const uint16_t *bias, const uint16_t *x, int64_t ldx, const uint16_t *A,
                        const uint16_t *B, int32_t rank, float lora_scale, uint16_t *u_ws,
                        int64_t M, int64_t N, int64_t K, uint16_t *out, int64_t ldo,
-                       int32_t *acc_out, void *stream, bool lora, bool gelu = false)
+                       int32_t *acc_out, void *stream, LoraMode lora, bool gelu = false)
 {
     sdnq_status st = validate_linear(qx, sx, qW, sW, bias, M, N, K, out, ldo, acc_out);
     if (st != SDNQ_OK)
         return st;
-    if (lora) {
-        if (!A || !B || (M != 0 && (!x || !u_ws)))
+    if (lora != kNoLora) {
+        if (!B || (M != 0 && !u_ws))
             return SDNQ_ERR_NULL;
-        if (ldx < K)
-            return SDNQ_ERR_SHAPE;
+        if (lora == kLoraFull && (st = validate_lora_down(x, ldx, A, rank, M, K, u_ws)) != SDNQ_OK)
+            return st;
         if (rank < 16 || rank > SDNQ_MAX_RANK || rank % 16 != 0)
             return SDNQ_ERR_UNSUPPORTED;
         if (N % 8 != 0)
             return SDNQ_ERR_SHAPE;
-        if (ldx % 8 != 0 || !aligned(x, 16) || !aligned(A, 16) || !aligned(B, 16) ||
-            !aligned(u_ws, 16))
+        if (!aligned(B, 16) || !aligned(u_ws, 16))
             return SDNQ_ERR_ALIGN;
     }
     DeviceInfo dev;
@@ -633,20 +662,13 @@ sdnq_status run_linear(const int8_t *qx, const float *sx, const int8_t *qW, cons
     p.timeout_ns = kDefaultTimeoutNs;
     if (gelu && (st = ensure_gelu_lut(dev, cs)) != SDNQ_OK)
         return st;
-    if (!lora && M >= kPairMinRows)
+    if (lora == kNoLora && M >= kPairMinRows)
         return gelu ? launch_gemm_pair<true, false>(dev, qx, qW, p, cs)
                     : launch_gemm_pair<false, false>(dev, qx, qW, p, cs);
-    if (!lora)
+    if (lora == kNoLora)
         return gelu ? launch_gemm<256, false, true>(dev, qx, qW, nullptr, nullptr, 0, p, cs)
                     : launch_gemm<256, false>(dev, qx, qW, nullptr, nullptr, 0, p, cs);
-    const int32_t Mi = static_cast<int32_t>(M), Ki = static_cast<int32_t>(K);
-    if (rank <= 64)
-        st = launch_lora_down<64>(dev, x, ldx, A, rank, u_ws, Mi, Ki, cs);
-    else if (rank <= 128)
-        st = launch_lora_down<128>(dev, x, ldx, A, rank, u_ws, Mi, Ki, cs);
-    else
-        st = launch_lora_down<256>(dev, x, ldx, A, rank, u_ws, Mi, Ki, cs);
-    if (st != SDNQ_OK)
+    if (lora == kLoraFull && (st = run_lora_down(dev, x, ldx, A, rank, u_ws, M, K, cs)) != SDNQ_OK)
         return st;
     p.lora_chunks = (rank + 63) / 64;
     if (M >= kPairMinRows)
@@ -726,7 +748,7 @@ sdnq_status run_linear_fused(const uint16_t *x, int64_t ldx, int32_t group, cons
         if ((st = launch_rowquant(x, M, K, ldx, group, nullptr, qx_ws, sx_ws, dev, cs)) != SDNQ_OK)
             return st;
         return run_linear(qx_ws, sx_ws, qW, sW, bias, nullptr, 0, nullptr, nullptr, 0, 0.0f,
-                          nullptr, M, N, K, out, ldo, acc_out, stream, false);
+                          nullptr, M, N, K, out, ldo, acc_out, stream, kNoLora);
     }
     GemmParams p = {};
     p.sx = sx_ws;
@@ -1165,7 +1187,7 @@ SDNQ_API sdnq_status sdnq_int8_linear(const int8_t *qx, const float *sx, const i
 {
     SDNQ_NVTX_RANGE();
     return run_linear(qx, sx, qW, sW, bias, nullptr, 0, nullptr, nullptr, 0, 0.0f, nullptr, M, N, K,
-                      out, ldo, acc_out, stream, false);
+                      out, ldo, acc_out, stream, kNoLora);
 }
 
 SDNQ_API sdnq_status sdnq_int8_linear_fused(const uint16_t *x, int64_t ldx, int32_t group,
@@ -1241,7 +1263,7 @@ SDNQ_API sdnq_status sdnq_int8_linear_gelu(const int8_t *qx, const float *sx, co
 {
     SDNQ_NVTX_RANGE();
     return run_linear(qx, sx, qW, sW, bias, nullptr, 0, nullptr, nullptr, 0, 0.0f, nullptr, M, N, K,
-                      out, ldo, acc_out, stream, false, true);
+                      out, ldo, acc_out, stream, kNoLora, true);
 }
 
 SDNQ_API sdnq_status sdnq_int8_linear_grad_input(const uint16_t *dy, int64_t lddy,
@@ -1281,7 +1303,34 @@ SDNQ_API sdnq_status sdnq_int8_linear_lora(const int8_t *qx, const float *sx, co
 {
     SDNQ_NVTX_RANGE();
     return run_linear(qx, sx, qW, sW, bias, x, ldx, A, B, rank, lora_scale, u_ws, M, N, K, out, ldo,
-                      acc_out, stream, true);
+                      acc_out, stream, kLoraFull);
+}
+
+SDNQ_API sdnq_status sdnq_lora_down(const uint16_t *x, int64_t ldx, const uint16_t *A,
+                                    int32_t rank, int64_t M, int64_t K, uint16_t *u, void *stream)
+{
+    SDNQ_NVTX_RANGE();
+    sdnq_status st = validate_lora_down(x, ldx, A, rank, M, K, u);
+    if (st != SDNQ_OK)
+        return st;
+    DeviceInfo dev;
+    if ((st = current_device(&dev)) != SDNQ_OK)
+        return st;
+    if (M == 0)
+        return SDNQ_OK;
+    return run_lora_down(dev, x, ldx, A, rank, u, M, K, static_cast<cudaStream_t>(stream));
+}
+
+SDNQ_API sdnq_status sdnq_int8_linear_lora_up(const int8_t *qx, const float *sx, const int8_t *qW,
+                                              const float *sW, const uint16_t *bias,
+                                              const uint16_t *u, const uint16_t *B, int32_t rank,
+                                              float lora_scale, int64_t M, int64_t N, int64_t K,
+                                              uint16_t *out, int64_t ldo, int32_t *acc_out,
+                                              void *stream)
+{
+    SDNQ_NVTX_RANGE();
+    return run_linear(qx, sx, qW, sW, bias, nullptr, 0, nullptr, B, rank, lora_scale,
+                      const_cast<uint16_t *>(u), M, N, K, out, ldo, acc_out, stream, kLoraUp);
 }
 
 SDNQ_API sdnq_status sdnq_gelu_bf16(const uint16_t *in, int64_t M, int64_t N, int64_t ld_in,

@@ -75,5 +75,5 @@ SDNQ_API sdnq_status sdnq_int8_linear_lora_noalloc(const int8_t *qx, const float
     // u is written in full (rows < M) by the down-projection before the main kernel reads
     // it, and rows >= M are never read, so nothing has to be cleared between calls.
     return run_linear(qx, sx, qW, sW, bias, x, ldx, A, B, rank, lora_scale,
-                      static_cast<uint16_t *>(u), M, N, K, out, ldo, acc_out, stream, true);
+                      static_cast<uint16_t *>(u), M, N, K, out, ldo, acc_out, stream, kLoraFull);
 }

@@ -238,6 +238,29 @@ sdnq_status sdnq_int8_linear_lora(const int8_t *qx, const float *sx, const int8_
                                   int32_t *acc_out, void *stream);
 
 /*
+ * The two halves of sdnq_int8_linear_lora as calls of their own (same kernels, same bits):
+ * the LoRA down-projection u = bf16(x A), and the int8 linear with the adapter term from a
+ * given u, out = bf16(v + lora_scale * (u B)). A caller that keeps u (the adapter's weight
+ * gradient dB = u^T dy reads it), or computes it on another stream, uses these.
+ *
+ * sdnq_lora_down: x [M, K] bf16, the UNROTATED layer input, row stride ldx (multiple of 8);
+ *   A [K, rank] bf16 dense; u [M, rank] bf16 dense (output). K % 16 == 0, 16 <= K <=
+ *   SDNQ_MAX_K; rank a multiple of 16, 16..SDNQ_MAX_RANK (else SDNQ_ERR_UNSUPPORTED);
+ *   x, A, u 16-byte aligned. M == 0 is a no-op. u is rounded once from fp32 tensor-core
+ *   sums (the order of the products is the tensor cores').
+ * sdnq_int8_linear_lora_up: qx, sx, qW, sW, bias, M, N, K, out, ldo, acc_out as in
+ *   sdnq_int8_linear; u [M, rank] bf16 dense as written by sdnq_lora_down (or any bf16
+ *   values); B [rank, N] bf16 dense, N % 8 == 0; rank and alignment as above.
+ */
+sdnq_status sdnq_lora_down(const uint16_t *x, int64_t ldx, const uint16_t *A, int32_t rank,
+                           int64_t M, int64_t K, uint16_t *u, void *stream);
+sdnq_status sdnq_int8_linear_lora_up(const int8_t *qx, const float *sx, const int8_t *qW,
+                                     const float *sW, const uint16_t *bias, const uint16_t *u,
+                                     const uint16_t *B, int32_t rank, float lora_scale,
+                                     int64_t M, int64_t N, int64_t K, uint16_t *out,
+                                     int64_t ldo, int32_t *acc_out, void *stream);
+
+/*
  * sdnq_int8_linear_lora without the caller-provided workspace. The pages have no
  * counterpart: this entry point is for callers that cannot allocate device memory for u_ws,
  * because their host framework owns all device memory (a caching allocator or a fixed

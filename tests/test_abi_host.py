@@ -126,6 +126,37 @@ def test_lora_validation(lib):
     assert lora(lib, A=MIS) == _native.SDNQ_ERR_ALIGN
 
 
+def lora_down(lib, x=A16, ldx=256, A=A16, rank=64, M=128, K=256, u=A16):
+    return lib.sdnq_lora_down(x, ldx, A, rank, M, K, u, S)
+
+
+def lora_up(lib, u=A16, B=A16, rank=64, N=256, M=128):
+    return lib.sdnq_int8_linear_lora_up(A16, A16, A16, A16, 0, u, B, rank, 1.0, M, N, 256, A16,
+                                        256, 0, S)
+
+
+def test_lora_halves_validation(lib):
+    """The down-projection and the up-projection GEMM as calls of their own refuse what the
+    whole LoRA call refuses, before any device work."""
+    assert lora_down(lib, x=0) == _native.SDNQ_ERR_NULL
+    assert lora_down(lib, A=0) == _native.SDNQ_ERR_NULL
+    assert lora_down(lib, u=0) == _native.SDNQ_ERR_NULL
+    assert lora_down(lib, M=-1) == _native.SDNQ_ERR_SHAPE
+    assert lora_down(lib, K=8) == _native.SDNQ_ERR_SHAPE
+    assert lora_down(lib, K=264) == _native.SDNQ_ERR_SHAPE      # K % 16
+    assert lora_down(lib, ldx=128) == _native.SDNQ_ERR_SHAPE
+    assert lora_down(lib, rank=24) == _native.SDNQ_ERR_UNSUPPORTED
+    assert lora_down(lib, rank=512) == _native.SDNQ_ERR_UNSUPPORTED
+    assert lora_down(lib, ldx=260) == _native.SDNQ_ERR_ALIGN     # rows not 16-byte strided
+    assert lora_down(lib, u=MIS) == _native.SDNQ_ERR_ALIGN
+    assert lora_up(lib, u=0) == _native.SDNQ_ERR_NULL
+    assert lora_up(lib, B=0) == _native.SDNQ_ERR_NULL
+    assert lora_up(lib, rank=8) == _native.SDNQ_ERR_UNSUPPORTED
+    assert lora_up(lib, N=252) == _native.SDNQ_ERR_SHAPE
+    assert lora_up(lib, B=MIS) == _native.SDNQ_ERR_ALIGN
+    assert lora_up(lib, u=MIS) == _native.SDNQ_ERR_ALIGN
+
+
 def grad(lib, dy=A16, lddy=256, qW=A16, sW=A16, M=128, N=256, K=512, g=256, qg=A16, sg=A16,
          dx=A16, lddx=512, acc=0):
     return lib.sdnq_int8_linear_grad_input(dy, lddy, qW, sW, M, N, K, g, qg, sg, dx, lddx, acc, S)

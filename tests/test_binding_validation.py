@@ -100,6 +100,22 @@ def test_lora_refuses_bad_operands(what):
                                                   a["bias"], a["x"], a["A"], a["B"], 1.0)
 
 
+def test_lora_halves_refuse_bad_operands():
+    with pytest.raises(ValueError):   # A rows != K
+        _native.sdnq_lora_down(bf(M, K), bf(K + 16, R))
+    with pytest.raises(ValueError):   # u of the wrong shape
+        _native.sdnq_lora_down(bf(M, K), bf(K, R), u=bf(M, R + 16))
+    with pytest.raises(TypeError):
+        _native.sdnq_lora_down(f32(M, K), bf(K, R))
+    a = dict(qx=t8(M, K), sx=f32(M), qW=t8(N, K), sW=f32(N), bias=bf(N), u=bf(M, R), B=bf(R, N))
+    for key, bad, err in (("u", bf(M - 1, R), ValueError), ("B", bf(R, N + 8), ValueError),
+                          ("u", f32(M, R), TypeError), ("sx", f32(M - 1), ValueError)):
+        b = dict(a, **{key: bad})
+        with pytest.raises(err):
+            _native.sdnq_int8_linear_lora_up(b["qx"], b["sx"], b["qW"], b["sW"], b["bias"],
+                                             b["u"], b["B"], 1.0)
+
+
 def test_noalloc_refuses_more_rows_than_its_scratch_holds():
     rows = _native.NOALLOC_MAX_U_ELEMS // R + 1
     with pytest.raises(ValueError, match="scratch"):

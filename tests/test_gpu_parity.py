@@ -279,6 +279,30 @@ def test_lora_few_k_blocks_and_many_row_blocks(M, N, K, rank, g):
     check_lora_tolerance(case, got["u"], got["out"], ref, 0.5)
 
 
+@pytest.mark.parametrize("M,N,K,rank", [(300, 264, 512, 16), (4608, 1024, 3072, 64)])
+def test_lora_halves_equal_the_whole_call(M, N, K, rank):
+    """sdnq_lora_down then sdnq_int8_linear_lora_up give the bits of sdnq_int8_linear_lora
+    (u and outputs), and u is within the fp32 accumulation bound of the oracle's."""
+    case = synthetic.make_case(M=M, N=N, K=K, g=256, seed=M + rank, outlier_count=K // 100,
+                               outlier_factor=30.0, bias_std=0.01, lora_rank=rank,
+                               lora_scale=0.75)
+    xg, A, B = case.x.cuda(), case.A.cuda(), case.B.cuda()
+    qW, sW = sd.sdnq_rotate_quant_weight(case.W.cuda(), 256)
+    qx, sx = sd.sdnq_rotquant_act(xg, 256)
+    bias = case.bias.cuda()
+    u_whole = torch.empty((M, rank), dtype=torch.bfloat16, device="cuda")
+    whole = sd.sdnq_int8_linear_lora(qx, sx, qW, sW, bias, xg, A, B, 0.75, u_ws=u_whole)
+    u = sd.sdnq_lora_down(xg, A)
+    halves = sd.sdnq_int8_linear_lora_up(qx, sx, qW, sW, bias, u, B, 0.75)
+    torch.cuda.synchronize()
+    assert_equal(bits_of(u), bits_of(u_whole), "u")
+    assert_equal(bits_of(halves), bits_of(whole), "outputs")
+    ref = oracle.linear(synthetic.bits(case.x), *oracle.rotate_quantize(synthetic.bits(case.W), 256),
+                        256, bias_bits=synthetic.bits(case.bias), A_bits=synthetic.bits(case.A),
+                        B_bits=synthetic.bits(case.B), lora_scale=0.75)
+    check_lora_tolerance(case, bits_of(u), bits_of(halves), ref, 0.75)
+
+
 def lora_tolerances(x_bits, A_bits, B_bits, u_ref_bits, out_ref_bits, scale, rows=None):
     """Tolerance derived from the arithmetic (the adapter path accumulates in fp32, the
     oracle in fp64): one bf16 ulp of the result plus the fp32 accumulation bound
