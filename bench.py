@@ -133,8 +133,10 @@ def rotquant_kernel_name(case, rows_k, grad, fp8):
         return "attention quantizers (smooth_k means, q and k short-row quantizers)"
     f = str(fp8).lower()
     if grad:
+        # the output gradient is quantized per token without a rotation (group 1), with the
+        # weight's row scales as column multipliers
         kind = "rotquant_persistent_kernel" if (rows_k + 1023) // 1024 <= 16 else "rotquant_kernel"
-        return f"{kind}<{case.g},true,{f}>"
+        return f"{kind}<1,true,{f}>"
     if rows_k <= 32768:
         return f"rotquant_run_kernel<{case.g},{f},V8>"
     return f"rotquant_kernel<{case.g},false,{f}>"
@@ -151,7 +153,7 @@ class Step:
         self.qx = torch.empty((case.M, case.K), dtype=torch.int8, device=dev)
         self.sx = torch.empty((case.M,), dtype=torch.float32, device=dev)
         self.bias = case.bias.to(dev) if case.bias is not None else None
-        if not case.extra.get("attn"):
+        if not case.extra.get("attn") and not name.startswith("fp8_"):
             self.qW, self.sW = sd.sdnq_rotate_quant_weight(case.W.to(dev), g)
         self.out = torch.empty((case.M, case.N), dtype=torch.bfloat16, device=dev)
         self.gemm_stages = []
@@ -739,7 +741,8 @@ def main():
             "kernel": rotquant_kernel_name(case, rows_k, grad, fp8),
             "bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
             "frac": gbs / peaks["hbm_gbs"],
-            "traffic": profiled_traffic(n, "rotquant", profile_key),
+            "traffic": profiled_traffic(n, "attn_kernel" if case.extra.get("attn") else "rotquant",
+                                        profile_key),
             "bytes_per_launch": nbytes, "row_length": rows_k, "ms_per_launch": ms,
             "peak_source": f"{peak_src} copy bandwidth", "timing": note,
         }
