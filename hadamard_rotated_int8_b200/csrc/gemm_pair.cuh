@@ -46,6 +46,9 @@
 #ifndef SDNQ_LORA_EPI_WARPS
 #define SDNQ_LORA_EPI_WARPS 8
 #endif
+#ifndef SDNQ_PAIR_KPS
+#define SDNQ_PAIR_KPS 2
+#endif
 
 namespace sdnq {
 
@@ -53,9 +56,15 @@ template <bool GELU, bool LORA = false, bool FUSE = false>
 struct PairConfig {
     static constexpr int BM = 128;                       // rows per CTA (256 per pair)
     static constexpr int BN = 256;                       // columns per pair tile
-    static constexpr int BK = 128;                       // bytes of K per stage
-    static constexpr int A_BYTES = BM * BK;              // 16 KB
-    static constexpr int B_BYTES = (BN / 2) * BK;        // this CTA's 128 columns: 16 KB
+    static constexpr int BK = 128;                       // bytes of K per k-block (one TMA box)
+    // k-blocks per pipeline stage: two halve the stage barriers and MMA commits per byte of
+    // K (each stage costs the tensor pipe a little; measured with the loads removed: 148 us
+    // against 163 us on 8192 x 12288 x 3072); one with GELU, whose epilogue needs the room
+    static constexpr int KPS = GELU ? 1 : SDNQ_PAIR_KPS;
+    static constexpr int A_KB = BM * BK;                 // 16 KB per k-block
+    static constexpr int B_KB = (BN / 2) * BK;           // this CTA's 128 columns: 16 KB
+    static constexpr int A_BYTES = KPS * A_KB;
+    static constexpr int B_BYTES = KPS * B_KB;
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
     static constexpr int ACC_COLS = LORA ? 2 * BN : BN;  // int32 (+ fp32 LoRA) columns per buffer
     static constexpr int NBUF = LORA ? 1 : 2;
@@ -298,8 +307,9 @@ __global__ void __launch_bounds__(PairConfig<GELU, LORA, (FUSE_G > 0)>::THREADS,
                     }
                     fence_proxy_async_global();
                 }
-                const int steps = p.num_kb + (LORA ? p.lora_chunks : 0);
-                for (int kb = 0; kb < steps; ++kb) {
+                const int kstages = (p.num_kb + C::KPS - 1) / C::KPS;
+                const int steps = kstages + (LORA ? p.lora_chunks : 0);
+                for (int st = 0; st < steps; ++st) {
                     if (!mbar_wait_bounded(empty_bar(stage), phase ^ 1u, abort, p.timeout_ns)) {
                         ok = false;
                         break;
@@ -307,16 +317,25 @@ __global__ void __launch_bounds__(PairConfig<GELU, LORA, (FUSE_G > 0)>::THREADS,
                     const uint32_t sa = base + stage * C::STAGE_BYTES;
                     const uint32_t sb = sa + C::A_BYTES;
                     const uint32_t fb = leader_full0 + 8u * stage;   // rank 0's full barrier
-                    if (leader)
-                        mbar_arrive_expect_tx(full_bar(stage), 2 * C::STAGE_BYTES);
-                    if (!LORA || kb < p.num_kb) {
-                        tma_load_2d_pair(sa, &tmA, fb, kb * C::BK, m0);
-                        tma_load_2d_pair(sb, &tmB, fb, kb * C::BK, nr0);
+                    if (!LORA || st < kstages) {
+                        // k-blocks kb0 .. kb0 + nkb - 1 of this CTA's A rows and B columns
+                        const int kb0 = st * C::KPS;
+                        const int nkb = p.num_kb - kb0 < C::KPS ? p.num_kb - kb0 : C::KPS;
+                        if (leader)
+                            mbar_arrive_expect_tx(full_bar(stage),
+                                                  static_cast<uint32_t>(2 * nkb * (C::A_KB + C::B_KB)));
+                        for (int i = 0; i < nkb; ++i) {
+                            tma_load_2d_pair(sa + i * C::A_KB, &tmA, fb, (kb0 + i) * C::BK, m0);
+                            tma_load_2d_pair(sb + i * C::B_KB, &tmB, fb, (kb0 + i) * C::BK, nr0);
+                        }
                     } else {
                         // LoRA chunk c: this CTA's U rows [128 x 64 rank] (K-major) into the A
                         // slot, its 128 columns of B [64 rank x 128] (N-major) as two 64-column
-                        // boxes into the B slot
-                        const int c = kb - p.num_kb;
+                        // boxes into the B slot (32 KB per CTA)
+                        if (leader)
+                            mbar_arrive_expect_tx(full_bar(stage),
+                                                  static_cast<uint32_t>(2 * (C::A_KB + C::B_KB)));
+                        const int c = st - kstages;
                         tma_load_2d_pair(sa, &tmU, fb, c * 64, m0);
                         tma_load_2d_pair(sb, &tmL, fb, nr0, c * 64);
                         tma_load_2d_pair(sb + 8192, &tmL, fb, nr0 + 64, c * 64);
@@ -364,7 +383,7 @@ __global__ void __launch_bounds__(PairConfig<GELU, LORA, (FUSE_G > 0)>::THREADS,
                 }
                 tc_fence_after_sync();
                 const uint32_t d_acc = tmem_base + buf * C::ACC_COLS;
-                for (int kb = 0; kb < p.num_kb; ++kb) {
+                for (int kb0 = 0; kb0 < p.num_kb; kb0 += C::KPS) {
                     if (!mbar_wait_bounded(full_bar(stage), phase, abort, p.timeout_ns)) {
                         ok = false;
                         break;
@@ -372,14 +391,21 @@ __global__ void __launch_bounds__(PairConfig<GELU, LORA, (FUSE_G > 0)>::THREADS,
                     tc_fence_after_sync();
                     const uint32_t sa = base + stage * C::STAGE_BYTES;
                     const uint32_t sb = sa + C::A_BYTES;
+                    const int nkb = p.num_kb - kb0 < C::KPS ? p.num_kb - kb0 : C::KPS;
 #pragma unroll
-                    for (int k = 0; k < C::BK / 32; ++k) {
-                        if constexpr (FP8)
-                            mma_f8_pair(d_acc, kmajor_desc(sa + 32 * k), kmajor_desc(sb + 32 * k), IDESC,
-                                        (kb | k) != 0 ? 1u : 0u);
-                        else
-                            mma_s8_pair(d_acc, kmajor_desc(sa + 32 * k), kmajor_desc(sb + 32 * k), IDESC,
-                                        (kb | k) != 0 ? 1u : 0u);
+                    for (int i = 0; i < C::KPS; ++i) {
+                        if (i < nkb) {
+#pragma unroll
+                            for (int k = 0; k < C::BK / 32; ++k) {
+                                const uint64_t da = kmajor_desc(sa + i * C::A_KB + 32 * k);
+                                const uint64_t db = kmajor_desc(sb + i * C::B_KB + 32 * k);
+                                const uint32_t accum = ((kb0 + i) | k) != 0 ? 1u : 0u;
+                                if constexpr (FP8)
+                                    mma_f8_pair(d_acc, da, db, IDESC, accum);
+                                else
+                                    mma_s8_pair(d_acc, da, db, IDESC, accum);
+                            }
+                        }
                     }
                     tc_commit_pair(empty_bar(stage), 0x3);
                     if (++stage == C::STAGES) {
