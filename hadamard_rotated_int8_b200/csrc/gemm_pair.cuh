@@ -59,8 +59,8 @@ struct PairConfig {
     static constexpr int BK = 128;                       // bytes of K per k-block (one TMA box)
     // k-blocks per pipeline stage: two halve the stage barriers and MMA commits per byte of
     // K (each stage costs the tensor pipe a little; measured with the loads removed: 148 us
-    // against 163 us on 8192 x 12288 x 3072); one with GELU, whose epilogue needs the room
-    static constexpr int KPS = GELU ? 1 : SDNQ_PAIR_KPS;
+    // against 163 us on 8192 x 12288 x 3072)
+    static constexpr int KPS = SDNQ_PAIR_KPS;
     static constexpr int A_KB = BM * BK;                 // 16 KB per k-block
     static constexpr int B_KB = (BN / 2) * BK;           // this CTA's 128 columns: 16 KB
     static constexpr int A_BYTES = KPS * A_KB;
@@ -77,7 +77,10 @@ struct PairConfig {
     static constexpr int QUANT_WARPS = FUSE ? SDNQ_FUSED_QUANT_WARPS : 0;
     static constexpr int THREADS = 64 + 32 * EPI_WARPS + (FUSE ? 32 * (QUANT_WARPS + 1) : 0);
     static constexpr int EPI_COLS = BN / (EPI_WARPS / 4);
-    static constexpr int STAGE_OUT_BYTES = 32 * 64;
+    // output staging per epilogue warp: a 32 x 32 bf16 block; with GELU (16 warps and the
+    // table) a 32 x 16 block, so that three stages of two k-blocks still fit
+    static constexpr int OUT_COLS = GELU ? 16 : 32;
+    static constexpr int STAGE_OUT_BYTES = 32 * OUT_COLS * 2;
     static constexpr int LUT_BYTES = GELU ? kGeluLutBytes : 0;
     static constexpr int SCALE_BYTES = EPI_COLS * 8;
     static constexpr int FIXED = EPI_WARPS * (STAGE_OUT_BYTES + SCALE_BYTES) + LUT_BYTES +
@@ -99,6 +102,26 @@ struct PairConfig {
     static_assert(STAGES >= 3, "pipeline depth");
     static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 };
+
+// One 16-column output block: 8 packed bf16 pairs of this thread's row go through the warp's
+// unswizzled 32 x 32-byte staging buffer to a TMA store of the warp's 32 x 16 block at
+// (column nc, row mrow0); rows >= M and columns >= N fall outside the tensor and are dropped.
+__device__ __forceinline__ void store_block16(const uint32_t *ob, uint32_t s_out, uint32_t lane,
+                                              const CUtensorMap *tmO, int nc, int mrow0)
+{
+    if (lane == 0)
+        bulk_wait_read_all();  // the previous block has left the staging buffer
+    __syncwarp();
+    const uint32_t row_addr = s_out + lane * 32u;
+    sts_v4(row_addr, ob[0], ob[1], ob[2], ob[3]);
+    sts_v4(row_addr + 16u, ob[4], ob[5], ob[6], ob[7]);
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+        tma_store_2d(tmO, s_out, nc, mrow0);
+        bulk_commit_group();
+    }
+}
 
 // The first fp32 steps of the de-quant epilogue for two adjacent columns: t = sx * sw (f32x2),
 // v = fp32(acc) * t, then + bias; the products that feed an add as scalar intrinsics, the
@@ -614,8 +637,11 @@ __global__ void __launch_bounds__(PairConfig<GELU, LORA, (FUSE_G > 0)>::THREADS,
                     if constexpr (GELU) {
                         gelu_bf16x16_lut(ob, lut);
                         gelu_bf16x16_lut(ob + 8, lut);
+                        store_block16(ob, s_out, lane, &tmO, nc, m0 + static_cast<int>(quad * 32u));
+                        store_block16(ob + 8, s_out, lane, &tmO, nc + 16, m0 + static_cast<int>(quad * 32u));
+                    } else {
+                        store_block(ob, s_out, lane, &tmO, nc, m0 + static_cast<int>(quad * 32u));
                     }
-                    store_block(ob, s_out, lane, &tmO, nc, m0 + static_cast<int>(quad * 32u));
                     if (p.acc_out != nullptr && row_ok) {
                         int32_t *arow = p.acc_out + static_cast<int64_t>(m) * p.N;
 #pragma unroll

@@ -481,8 +481,9 @@ sdnq_status launch_gemm_pair(const DeviceInfo &dev, const int8_t *qx, const int8
     CUtensorMap tmA, tmB, tmU, tmL, tmO;
     if (!make_tmap_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, qx, p.K, p.M, p.K, 128, 128) ||
         !make_tmap_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, qW, p.K, p.N, p.K, 128, C::BN / 2) ||
-        !make_tmap_2d(&tmO, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.out, p.N, p.M, 2ull * p.ldo, 32, 32,
-                      CU_TENSOR_MAP_SWIZZLE_64B))
+        !make_tmap_2d(&tmO, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.out, p.N, p.M, 2ull * p.ldo,
+                      C::OUT_COLS, 32,
+                      C::OUT_COLS == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_NONE))
         return SDNQ_ERR_CUDA;
     if (LORA) {
         if (!make_tmap_2d(&tmU, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, u, rank, p.M, 2ull * rank, 64, 128) ||
