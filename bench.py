@@ -670,14 +670,15 @@ def main():
         measured_int8 = 2.0 / (1.0 / measured_int8 + 1.0 / bf16_peak)
         spec_peak = 2.0 / (1.0 / INT8_SPEC_TOPS + 1.0 / (INT8_SPEC_TOPS / 2))
     grad = args.workload.startswith("grad_")
-    # the kernel each GEMM stage launches: the CTA-pair kernel above 128 rows (the int8
-    # input-gradient GEMM stays on one SM), template arguments as in the library
+    # the kernel each GEMM stage launches: the CTA-pair kernel above 128 rows, template
+    # arguments as in the library
     pair = case.M >= 129
     fp8 = bool(case.extra.get("fp8"))
     if case.extra.get("attn"):
         gemm_kernel = "attn_kernel"
     elif grad:
-        gemm_kernel = f"gemm_s8_kernel<256,false,false,{case.g}> (input gradient)"
+        gemm_kernel = (f"gemm_s8_pair_kernel<false,false,false,0,{case.g}>" if pair else
+                       f"gemm_s8_kernel<256,false,false,{case.g}>") + " (input gradient)"
     elif "fused" in stage_ms:
         gemm_kernel = (f"gemm_s8_pair_kernel<false,false,false,{case.g}>" if pair else
                        f"gemm_s8_kernel<256,false,false,0,{case.g}>") \

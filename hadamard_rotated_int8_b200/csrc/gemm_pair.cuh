@@ -229,7 +229,7 @@ __device__ __forceinline__ void lora_epilogue(uint32_t t_row, int col_base, int 
         mbar_arrive_remote(leader_tempty0 + 8u);
 }
 
-template <bool GELU, bool FP8, bool LORA, int FUSE_G = 0>
+template <bool GELU, bool FP8, bool LORA, int FUSE_G = 0, int GRAD_G = 0>
 __global__ void __launch_bounds__(PairConfig<GELU, LORA, (FUSE_G > 0)>::THREADS, 1)
     gemm_s8_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB,
@@ -241,6 +241,9 @@ __global__ void __launch_bounds__(PairConfig<GELU, LORA, (FUSE_G > 0)>::THREADS,
     static_assert(!LORA || (!GELU && !FP8), "the adapter term rides on the plain int8 linear");
     static_assert(FUSE_G == 0 || (!LORA && !GELU && !FP8),
                   "the activation quantizer inside: the plain int8 linear");
+    static_assert(GRAD_G == 0 || (!LORA && !GELU && !FP8 && FUSE_G == 0 &&
+                                  (GRAD_G & (GRAD_G - 1)) == 0 && GRAD_G <= 256),
+                  "the input gradient: the int8 product with the inverse-rotation epilogue");
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_addr = smem_u32(smem_raw);
     const uint32_t base = (raw_addr + 1023u) & ~1023u;
@@ -349,7 +352,10 @@ __global__ void __launch_bounds__(PairConfig<GELU, LORA, (FUSE_G > 0)>::THREADS,
                                                   static_cast<uint32_t>(2 * nkb * (C::A_KB + C::B_KB)));
                         for (int i = 0; i < nkb; ++i) {
                             tma_load_2d_pair(sa + i * C::A_KB, &tmA, fb, (kb0 + i) * C::BK, m0);
-                            tma_load_2d_pair(sb + i * C::B_KB, &tmB, fb, (kb0 + i) * C::BK, nr0);
+                            if constexpr (GRAD_G > 0)   // qW rows = contraction, N-major columns
+                                tma_load_2d_pair(sb + i * C::B_KB, &tmB, fb, nr0, (kb0 + i) * C::BK);
+                            else
+                                tma_load_2d_pair(sb + i * C::B_KB, &tmB, fb, (kb0 + i) * C::BK, nr0);
                         }
                     } else {
                         // LoRA chunk c: this CTA's U rows [128 x 64 rank] (K-major) into the A
@@ -392,7 +398,8 @@ __global__ void __launch_bounds__(PairConfig<GELU, LORA, (FUSE_G > 0)>::THREADS,
     } else if (warp == 1) {
         if (lane == 0 && leader) {
             // -------------------------------------------------------- MMA issuer (rank 0)
-            constexpr uint32_t IDESC = FP8 ? idesc_e4m3_f32(256, C::BN) : idesc_s8_s32(256, C::BN);
+            constexpr uint32_t IDESC =
+                FP8 ? idesc_e4m3_f32(256, C::BN) : idesc_s8_s32(256, C::BN, GRAD_G > 0);
             int stage = 0;
             uint32_t phase = 0;
             int local = 0;
@@ -421,7 +428,10 @@ __global__ void __launch_bounds__(PairConfig<GELU, LORA, (FUSE_G > 0)>::THREADS,
 #pragma unroll
                             for (int k = 0; k < C::BK / 32; ++k) {
                                 const uint64_t da = kmajor_desc(sa + i * C::A_KB + 32 * k);
-                                const uint64_t db = kmajor_desc(sb + i * C::B_KB + 32 * k);
+                                // the input gradient's N-major B: K = 32 rows of 128 bytes
+                                const uint64_t db = GRAD_G > 0
+                                                        ? mnmajor_desc(sb + i * C::B_KB + 4096 * k, 16384)
+                                                        : kmajor_desc(sb + i * C::B_KB + 32 * k);
                                 const uint32_t accum = ((kb0 + i) | k) != 0 ? 1u : 0u;
                                 if constexpr (FP8)
                                     mma_f8_pair(d_acc, da, db, IDESC, accum);
@@ -549,7 +559,7 @@ __global__ void __launch_bounds__(PairConfig<GELU, LORA, (FUSE_G > 0)>::THREADS,
             const int n0 = tile_nb(tile) * C::BN;
             const int nw = n0 + col_base;
 #pragma unroll
-            for (int j = static_cast<int>(lane) * 4; j < C::EPI_COLS; j += 128) {
+            for (int j = static_cast<int>(lane) * 4; GRAD_G == 0 && j < C::EPI_COLS; j += 128) {
                 float w4[4], b4[4];
                 if (nw + j + 4 <= p.N) {
                     const float4 f = __ldg(reinterpret_cast<const float4 *>(p.sw + nw + j));
@@ -583,8 +593,15 @@ __global__ void __launch_bounds__(PairConfig<GELU, LORA, (FUSE_G > 0)>::THREADS,
             // launch, visible since the dependency wait)
             float sxm = (FUSE_G == 0 && row_ok) ? p.sx[m] : 0.0f;
             const bool ready = mbar_wait_bounded(tfull_bar(buf), use & 1u, abort, p.timeout_ns);
-            if (!__all_sync(0xffffffffu, ready))
-                break;
+            if constexpr (GRAD_G > 0) {
+                // the two warps of a lane quarter leave together: they meet at named
+                // barriers inside the tile
+                if (bar_sync_or(2u + quad, 64, !__all_sync(0xffffffffu, ready)))
+                    break;
+            } else {
+                if (!__all_sync(0xffffffffu, ready))
+                    break;
+            }
             tc_fence_after_sync();
             if constexpr (FUSE_G > 0) {
                 // the row scales the scale warp copied once the rows were published
@@ -597,6 +614,17 @@ __global__ void __launch_bounds__(PairConfig<GELU, LORA, (FUSE_G > 0)>::THREADS,
             if constexpr (LORA) {
                 lora_epilogue<C>(t_row, col_base, n0, m0, quad, lane, sxm, row_ok, m, s_sw, s_bias,
                                  s_out, &tmO, p, leader_tempty0);
+            } else if constexpr (GRAD_G > 0) {
+                // the same per-CTA tile (128 rows x 256 columns) as the single-SM kernel
+                int32_t *acc_row = (p.acc_out != nullptr && row_ok)
+                                       ? p.acc_out + static_cast<int64_t>(m) * p.N : nullptr;
+                grad_epilogue_tile<GRAD_G>(t_row, static_cast<int>(ew >> 2), n0, p.N,
+                                           m0 + static_cast<int>(quad * 32u), sxm, p.c_g, lane,
+                                           2u + quad, s_out, &tmO, acc_row);
+                tc_fence_before_sync();
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive_remote(leader_tempty0 + 8u * buf);
             } else {
 #pragma unroll 1
                 for (int c = 0; c < C::EPI_COLS; c += 32) {

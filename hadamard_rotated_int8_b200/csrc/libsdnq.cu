@@ -471,16 +471,20 @@ sdnq_status launch_gemm(const DeviceInfo &dev, const int8_t *qx, const int8_t *q
 // A cluster of two CTAs per pair, launched programmatically like the single-SM kernel; the
 // grid holds as many pairs as the device can keep resident at once (or fewer, one per
 // tile), each walking the tiles persistently.
-template <bool GELU, bool FP8, bool LORA = false, int FUSE_G = 0>
+template <bool GELU, bool FP8, bool LORA = false, int FUSE_G = 0, int GRAD_G = 0>
 sdnq_status launch_gemm_pair(const DeviceInfo &dev, const int8_t *qx, const int8_t *qW,
                              GemmParams p, cudaStream_t cs, const uint16_t *u = nullptr,
                              const uint16_t *B = nullptr, int32_t rank = 0)
 {
     using C = PairConfig<GELU, LORA, (FUSE_G > 0)>;
-    constexpr auto kernel = gemm_s8_pair_kernel<GELU, FP8, LORA, FUSE_G>;
+    constexpr auto kernel = gemm_s8_pair_kernel<GELU, FP8, LORA, FUSE_G, GRAD_G>;
     CUtensorMap tmA, tmB, tmU, tmL, tmO;
     if (!make_tmap_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, qx, p.K, p.M, p.K, 128, 128) ||
-        !make_tmap_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, qW, p.K, p.N, p.K, 128, C::BN / 2) ||
+        !(GRAD_G > 0
+              // the input gradient reads qW [contraction rows, output columns] N-major: boxes
+              // of this CTA's 128 columns x 128 contraction rows
+              ? make_tmap_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, qW, p.N, p.K, p.N, C::BN / 2, 128)
+              : make_tmap_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, qW, p.K, p.N, p.K, 128, C::BN / 2)) ||
         !make_tmap_2d(&tmO, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.out, p.N, p.M, 2ull * p.ldo,
                       C::OUT_COLS, 32,
                       C::OUT_COLS == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_NONE))
@@ -845,6 +849,16 @@ sdnq_status launch_grad_gemm(const DeviceInfo &dev, const int8_t *qg, const floa
     p.lora_scale = 0.0f;
     p.c_g = static_cast<float>(1.0 / std::sqrt(static_cast<double>(group)));
     p.timeout_ns = kDefaultTimeoutNs;
+    if (M >= kPairMinRows) {
+        switch (group) {
+        case 8: return launch_gemm_pair<false, false, false, 0, 8>(dev, qg, qW, p, cs);
+        case 16: return launch_gemm_pair<false, false, false, 0, 16>(dev, qg, qW, p, cs);
+        case 32: return launch_gemm_pair<false, false, false, 0, 32>(dev, qg, qW, p, cs);
+        case 64: return launch_gemm_pair<false, false, false, 0, 64>(dev, qg, qW, p, cs);
+        case 128: return launch_gemm_pair<false, false, false, 0, 128>(dev, qg, qW, p, cs);
+        default: return launch_gemm_pair<false, false, false, 0, 256>(dev, qg, qW, p, cs);
+        }
+    }
     switch (group) {
     case 8: return launch_gemm<256, false, false, 8>(dev, qg, qW, nullptr, nullptr, 0, p, cs);
     case 16: return launch_gemm<256, false, false, 16>(dev, qg, qW, nullptr, nullptr, 0, p, cs);
