@@ -11,7 +11,9 @@
 // fill the 512 columns, so there is one buffer. Its epilogue copies the int32 columns to
 // registers and hands them back at once (tempty[0]), so the next tile's int8 K loop runs
 // while the outputs of this one are formed; the adapter columns go back (tempty[1]) before
-// the next tile's adapter MMAs.
+// the next tile's adapter MMAs. With GRAD_G the pair computes the input gradient: the weight
+// codes are read N-major (each CTA one 128 x 128 box of its columns per k-block) and each
+// CTA runs the single-SM kernel's inverse-rotation epilogue on its 128 x 256 tile.
 //
 // Sources: as the single-SM kernel ("SDNQ: SD.Next Quantization Engine" README, INT8
 // quantized matmul and dequantize_fp32; "ConvRot / Hadamard SDNQ").
