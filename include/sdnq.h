@@ -139,8 +139,9 @@ sdnq_status sdnq_int8_linear(const int8_t *qx, const float *sx, const int8_t *qW
  *   zeroed buffer serves every later call on the same stream. Calls whose kernels overlap on
  *   the GPU need separate buffers. After a device timeout (sdnq_device_status) re-zero it.
  *   The two launches leave sync_ws untouched.
- *   The kernel is a cooperative launch (one CTA per SM, all resident at once); if the device
- *   cannot run it, the call returns SDNQ_ERR_CUDA.
+ *   The kernel is a cooperative launch (one CTA per SM, or one two-CTA cluster per two SMs,
+ *   all resident at once); if the device can run neither form, the call returns
+ *   SDNQ_ERR_CUDA.
  */
 #define SDNQ_FUSED_SYNC_WORDS(M) (2 * (((M) + 127) / 128))
 enum { SDNQ_FUSE_AUTO = 0, SDNQ_FUSE_ALWAYS = 1, SDNQ_FUSE_NEVER = 2 };
