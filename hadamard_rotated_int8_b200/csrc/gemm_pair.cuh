@@ -99,7 +99,9 @@ struct PairConfig {
     static constexpr int BAR_OFF = AMAX_OFF + AMAX_BYTES;
     // full[S], empty[S], tfull[2], tempty[2], drain, sxfull[2], sxempty[2]; then tmem base +
     // abort flag
-    static constexpr int BAR_BYTES = (2 * STAGES + 9) * 8;
+    // then one full barrier per further k-block of a stage (the MMAs of a k-block start as
+    // soon as its own copies have landed)
+    static constexpr int BAR_BYTES = (2 * STAGES + 9 + (KPS - 1) * STAGES) * 8;
     static constexpr int SMEM_BYTES = 1024 + BAR_OFF + BAR_BYTES + 16;
     static_assert(STAGES >= 3, "pipeline depth");
     static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
@@ -258,6 +260,10 @@ __global__ void __launch_bounds__(PairConfig<GELU, LORA, (FUSE_G > 0)>::THREADS,
     const uint32_t drain_bar = bar0 + 8u * (2 * C::STAGES + 4);
     auto sxfull_bar = [&](int b) { return bar0 + 8u * (2 * C::STAGES + 5 + b); };
     auto sxempty_bar = [&](int b) { return bar0 + 8u * (2 * C::STAGES + 7 + b); };
+    // full barrier of k-block i of stage s (i = 0 is full_bar(s))
+    auto kfull_bar = [&](int s, int i) {
+        return i == 0 ? full_bar(s) : bar0 + 8u * (2 * C::STAGES + 9 + (i - 1) * C::STAGES + s);
+    };
     float *sx_smem = reinterpret_cast<float *>(smem + C::SX_OFF);     // [2][128], fused only
     float *amax_smem = reinterpret_cast<float *>(smem + C::AMAX_OFF); // fused only
     // tile -> (pair-row block, column block): rows fastest; columns fastest with the
@@ -276,7 +282,8 @@ __global__ void __launch_bounds__(PairConfig<GELU, LORA, (FUSE_G > 0)>::THREADS,
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::STAGES; ++s) {
-            mbar_init(full_bar(s), 1);
+            for (int i = 0; i < C::KPS; ++i)
+                mbar_init(kfull_bar(s, i), 1);
             mbar_init(empty_bar(s), 1);
         }
         for (int b = 0; b < C::NBUF; ++b)
@@ -319,7 +326,7 @@ __global__ void __launch_bounds__(PairConfig<GELU, LORA, (FUSE_G > 0)>::THREADS,
             uint32_t phase = 0;
             int issued = 0;
             bool ok = true;
-            const uint32_t leader_full0 = mapa_shared(full_bar(0), 0u);
+            const uint32_t leader_bar0 = mapa_shared(bar0, 0u);   // rank 0's barriers
             int local = 0;
             for (int tile = pair; ok && tile < p.num_tiles; tile += npairs, ++local) {
                 const int m0 = tile_mb(tile) * 2 * C::BM + static_cast<int>(rank) * C::BM;
@@ -344,28 +351,39 @@ __global__ void __launch_bounds__(PairConfig<GELU, LORA, (FUSE_G > 0)>::THREADS,
                     }
                     const uint32_t sa = base + stage * C::STAGE_BYTES;
                     const uint32_t sb = sa + C::A_BYTES;
-                    const uint32_t fb = leader_full0 + 8u * stage;   // rank 0's full barrier
+                    // rank 0's full barrier of k-block i of this stage
+                    auto kfb = [&](int i) { return leader_bar0 + (kfull_bar(stage, i) - bar0); };
+                    const uint32_t fb = kfb(0);
                     if (!LORA || st < kstages) {
-                        // k-blocks kb0 .. kb0 + nkb - 1 of this CTA's A rows and B columns
+                        // k-blocks kb0 .. kb0 + nkb - 1 of this CTA's A rows and B columns,
+                        // each completing on its own barrier; a k-block past the end of K
+                        // completes its barrier without copies (rank 0's plain arrive)
                         const int kb0 = st * C::KPS;
                         const int nkb = p.num_kb - kb0 < C::KPS ? p.num_kb - kb0 : C::KPS;
-                        if (leader)
-                            mbar_arrive_expect_tx(full_bar(stage),
-                                                  static_cast<uint32_t>(2 * nkb * (C::A_KB + C::B_KB)));
-                        for (int i = 0; i < nkb; ++i) {
-                            tma_load_2d_pair(sa + i * C::A_KB, &tmA, fb, (kb0 + i) * C::BK, m0);
-                            if constexpr (GRAD_G > 0)   // qW rows = contraction, N-major columns
-                                tma_load_2d_pair(sb + i * C::B_KB, &tmB, fb, nr0, (kb0 + i) * C::BK);
-                            else
-                                tma_load_2d_pair(sb + i * C::B_KB, &tmB, fb, (kb0 + i) * C::BK, nr0);
+                        for (int i = 0; i < C::KPS; ++i) {
+                            if (i < nkb) {
+                                if (leader)
+                                    mbar_arrive_expect_tx(kfull_bar(stage, i),
+                                                          static_cast<uint32_t>(2 * (C::A_KB + C::B_KB)));
+                                tma_load_2d_pair(sa + i * C::A_KB, &tmA, kfb(i), (kb0 + i) * C::BK, m0);
+                                if constexpr (GRAD_G > 0)   // qW rows = contraction, N-major columns
+                                    tma_load_2d_pair(sb + i * C::B_KB, &tmB, kfb(i), nr0, (kb0 + i) * C::BK);
+                                else
+                                    tma_load_2d_pair(sb + i * C::B_KB, &tmB, kfb(i), (kb0 + i) * C::BK, nr0);
+                            } else if (leader) {
+                                mbar_arrive(kfull_bar(stage, i));
+                            }
                         }
                     } else {
                         // LoRA chunk c: this CTA's U rows [128 x 64 rank] (K-major) into the A
                         // slot, its 128 columns of B [64 rank x 128] (N-major) as two 64-column
-                        // boxes into the B slot (32 KB per CTA)
-                        if (leader)
+                        // boxes into the B slot (32 KB per CTA), on the stage's first barrier
+                        if (leader) {
                             mbar_arrive_expect_tx(full_bar(stage),
                                                   static_cast<uint32_t>(2 * (C::A_KB + C::B_KB)));
+                            for (int i = 1; i < C::KPS; ++i)
+                                mbar_arrive(kfull_bar(stage, i));
+                        }
                         const int c = st - kstages;
                         tma_load_2d_pair(sa, &tmU, fb, c * 64, m0);
                         tma_load_2d_pair(sb, &tmL, fb, nr0, c * 64);
@@ -389,8 +407,10 @@ __global__ void __launch_bounds__(PairConfig<GELU, LORA, (FUSE_G > 0)>::THREADS,
                             s = C::STAGES - 1;
                             ph ^= 1u;
                         }
-                        volatile int no_abort = 0;
-                        mbar_wait_bounded(full_bar(s), ph, &no_abort, p.timeout_ns);
+                        for (int k = 0; k < C::KPS; ++k) {
+                            volatile int no_abort = 0;
+                            mbar_wait_bounded(kfull_bar(s, k), ph, &no_abort, p.timeout_ns);
+                        }
                     }
                 } else {
                     sleep_ns_bounded(1000000);   // 1 ms: this CTA's copies have landed
@@ -415,17 +435,19 @@ __global__ void __launch_bounds__(PairConfig<GELU, LORA, (FUSE_G > 0)>::THREADS,
                 }
                 tc_fence_after_sync();
                 const uint32_t d_acc = tmem_base + buf * C::ACC_COLS;
-                for (int kb0 = 0; kb0 < p.num_kb; kb0 += C::KPS) {
-                    if (!mbar_wait_bounded(full_bar(stage), phase, abort, p.timeout_ns)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after_sync();
+                for (int kb0 = 0; ok && kb0 < p.num_kb; kb0 += C::KPS) {
                     const uint32_t sa = base + stage * C::STAGE_BYTES;
                     const uint32_t sb = sa + C::A_BYTES;
                     const int nkb = p.num_kb - kb0 < C::KPS ? p.num_kb - kb0 : C::KPS;
 #pragma unroll
                     for (int i = 0; i < C::KPS; ++i) {
+                        // each k-block's MMAs as soon as its own copies have landed (a block
+                        // past the end of K has its barrier completed without copies)
+                        if (!mbar_wait_bounded(kfull_bar(stage, i), phase, abort, p.timeout_ns)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after_sync();
                         if (i < nkb) {
 #pragma unroll
                             for (int k = 0; k < C::BK / 32; ++k) {
