@@ -37,6 +37,16 @@ METRIC = "int8 rotated-linear TOPS and % of dense INT8 peak; rotate+quant HBM GB
 INT8_SPEC_TOPS = 4500.0        # B200 dense INT8, NVIDIA public spec
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 NOMINAL_INT8_OVER_BF16 = 2.0   # 4.5 / 2.25 PFLOP/s dense
+HBM_SPEC_GBS = 8000.0          # B200 HBM3e, NVIDIA public spec (8 TB/s)
+
+
+def clock_scaled_peak(peak, clocks):
+    """The peak scaled by the run's median SM clock under load over the GPU's maximum SM
+    clock (the tensor cores' rate is proportional to the SM clock); None without samples."""
+    mhz, max_mhz = clocks.get("sm_mhz"), clocks.get("sm_max_mhz")
+    if not mhz or not max_mhz:
+        return None
+    return peak * min(1.0, float(mhz) / float(max_mhz))
 
 
 def log(*a):
@@ -696,6 +706,7 @@ def main():
                              "gemm_s8_kernel<256,false,true>") + " (GELU epilogue)",
                  "gemm_down": gemm_kernel}
     ops_per_gemm = ops / len(step.gemm_stages)
+    scaled_peak = clock_scaled_peak(spec_peak, clocks.summary())
     gemm_lines = {}
     for n in step.gemm_stages:
         ms = stage_ms[n] / args.steps
@@ -712,6 +723,8 @@ def main():
             "frac_of_measured": tops / measured_int8,
             "measured_peak_source": f"{peak_src} cuBLAS bf16 {bf16_kind} x "
                                     f"{NOMINAL_INT8_OVER_BF16} (int8/bf16 nominal)",
+            "clock_scaled_peak": scaled_peak,
+            "frac_of_clock_scaled": tops / scaled_peak if scaled_peak else None,
         }
     dominant = max(step.gemm_stages, key=lambda n: stage_ms[n])
     gemm_tops = ops / (sum(stage_ms[n] for n in step.gemm_stages) / args.steps * 1e-3) / 1e12
@@ -746,6 +759,7 @@ def main():
                                         profile_key),
             "bytes_per_launch": nbytes, "row_length": rows_k, "ms_per_launch": ms,
             "peak_source": f"{peak_src} copy bandwidth", "timing": note,
+            "frac_of_spec": gbs / HBM_SPEC_GBS,
         }
     if "lora_down" in stage_ms:
         # u = bf16(x A): reads x and A, writes u
