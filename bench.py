@@ -567,7 +567,8 @@ def main():
         torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    step_ms_total = sum(e[0].elapsed_time(e[1]) for e in evs)
+    step_ms_each = [e[0].elapsed_time(e[1]) for e in evs]
+    step_ms_total = sum(step_ms_each)
 
     # per-kernel times for the rooflines: the same K steps again with an event between the
     # stages (which serialises them)
@@ -585,9 +586,10 @@ def main():
     for e in sevs:
         for j, n in enumerate(names):
             stage_ms[n] += e[j].elapsed_time(e[j + 1])
-    t = reduce_max_over_ranks([step_ms_total] + [stage_ms[n] for n in names], dist, world)
-    step_ms_total = t[0]
-    stage_ms = {n: t[1 + j] for j, n in enumerate(names)}
+    t = reduce_max_over_ranks([step_ms_total, statistics.median(step_ms_each), min(step_ms_each)]
+                              + [stage_ms[n] for n in names], dist, world)
+    step_ms_total, step_ms_median, step_ms_best = t[0], t[1], t[2]
+    stage_ms = {n: t[3 + j] for j, n in enumerate(names)}
     assert sd.sdnq_device_status() == 0
 
     ops, lora_flops = workload_ops(case, args.workload)
@@ -786,6 +788,11 @@ def main():
         "config": config_of(case, args),
         "roofline": gemm_lines[dominant],
         "gemm_tops": gemm_tops,
+        "step_stats": {"median_ms": step_ms_median, "best_ms": step_ms_best,
+                       "median_value": whole_job_tops(ops, world, step_ms_median),
+                       "best_value": whole_job_tops(ops, world, step_ms_best),
+                       "note": "per-step event times (each step alone between its L2 flush "
+                               "and the next); value is the mean over the timed steps"},
         "stage_ms_per_step": {n: stage_ms[n] / args.steps for n in names},
         "stage_timing": "a second pass of the same steps with an event between the stages",
         "clocks": clocks.summary(),
