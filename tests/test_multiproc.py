@@ -84,14 +84,3 @@ def test_reference_arm_prints_on_rank_zero_only():
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["sample"] and cb["value"] == line["value"]
     assert line["e2e"]["value"] == line["value"] and line["e2e"]["unit"] == line["unit"]
 
-
-def test_clock_scaled_peak():
-    sys.path.insert(0, ROOT)
-    import bench
-    # at the maximum clock the ceiling is the spec; under the power cap it scales with the clock
-    assert bench.clock_scaled_peak(4500.0, {"sm_mhz": 1965, "sm_max_mhz": 1965}) == 4500.0
-    assert bench.clock_scaled_peak(4500.0, {"sm_mhz": 1837, "sm_max_mhz": 1965}) == \
-        pytest.approx(4500.0 * 1837 / 1965)
-    # never above the spec, and no figure without clock samples
-    assert bench.clock_scaled_peak(4500.0, {"sm_mhz": 2000, "sm_max_mhz": 1965}) == 4500.0
-    assert bench.clock_scaled_peak(4500.0, {"sm_mhz": None, "sm_max_mhz": 1965}) is None
